@@ -1,0 +1,221 @@
+/*
+ * oracle.c -- plain, slow, fp64 CPU oracle for paged decode attention and the
+ * slot-mapped KV-cache append.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path links, loads or calls
+ * this file; only the tests, the smoke check and the benchmark's CPU baseline
+ * do.  It shares no code, header or constant with the CUDA library.
+ *
+ * What it computes (restated from the pages on PagedAttention):
+ *   - "vLLM Fundamentals: Paged Attention and Batching", section "Paged
+ *     Attention": the KV cache is split into blocks that are not contiguous;
+ *     each sequence has a block table, and the paged kernel follows that table
+ *     to gather the blocks.  Paging changes where keys and values live, not
+ *     what attention computes.
+ *   - "Deep Dive into vLLM", section 2.1: logical block -> physical block
+ *     through the block table.
+ *   - runbyai.xyz post 449 (an essay on vLLM and PagedAttention), section 1,
+ *     Decoding: each decode step uses the keys and values of all previous
+ *     tokens.
+ * So the oracle is the plain definition of single-query softmax attention,
+ * evaluated by walking the block table token by token in logical order:
+ *
+ *   for sequence s, query head j, kv head h = floor(j / (Hq / Hkv)):
+ *     k_t = K[table[s][t / bs]][t % bs][h][:]   (likewise v_t), t = 0 .. L_s-1
+ *     x_t = scale * sum_d q[s][j][d] * k_t[d]
+ *     mu  = max_t x_t,  w_t = exp(x_t - mu)
+ *     out[s][j][:] = sum_t w_t v_t / sum_t w_t         (0 when L_s == 0)
+ *
+ * All arithmetic is fp64; bf16 inputs are widened exactly.  The pages give no
+ * formula, scale, head grouping or layout: the readings used here are the
+ * plain softmax(scale * q K^T) V, q head j served by kv head floor(j / G), and
+ * the pool layout [num_blocks][block_size][num_kv_heads][head_dim].
+ *
+ * The append follows the same pages: each decode step computes and caches the
+ * new token's key and value (runbyai.xyz post 449, sections 1 and 2).
+ * Token i goes to slot slot_mapping[i] = physical_block * bs + offset; a
+ * negative slot means "no write".
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* bf16 bit pattern -> double, exactly (bf16 is the top half of an fp32). */
+static double bf16_bits_to_double(uint16_t bits)
+{
+    uint32_t u = (uint32_t)bits << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* Element offset of (physical block p, offset off, kv head h, dim 0) in the pool. */
+static int64_t pool_row(int64_t p, int off, int h, int block_size, int num_kv_heads, int head_dim)
+{
+    return ((p * block_size + off) * num_kv_heads + h) * (int64_t)head_dim;
+}
+
+/*
+ * One output row: out[0..head_dim) for sequence s, query head j.
+ * x is scratch of at least context_len doubles.
+ * Returns 0, or -2 when a table entry it needs is outside [0, num_blocks).
+ */
+static int decode_one(double *out, double *x,
+                      const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                      const int32_t *block_tables, int context_len,
+                      int s, int j, int num_q_heads, int num_kv_heads, int head_dim,
+                      int block_size, int max_blocks_per_seq, int64_t num_blocks, double scale)
+{
+    const int group = num_q_heads / num_kv_heads;
+    const int h = j / group;
+    const uint16_t *qrow = q + ((int64_t)s * num_q_heads + j) * head_dim;
+    const int32_t *table = block_tables + (int64_t)s * max_blocks_per_seq;
+
+    for (int d = 0; d < head_dim; ++d)
+        out[d] = 0.0;
+    if (context_len == 0)
+        return 0;
+
+    /* logits, walking the block table in logical token order */
+    for (int t = 0; t < context_len; ++t) {
+        int64_t p = table[t / block_size];
+        if (p < 0 || p >= num_blocks)
+            return -2;
+        const uint16_t *krow = k_cache + pool_row(p, t % block_size, h, block_size, num_kv_heads, head_dim);
+        double dot = 0.0;
+        for (int d = 0; d < head_dim; ++d)
+            dot += bf16_bits_to_double(qrow[d]) * bf16_bits_to_double(krow[d]);
+        x[t] = scale * dot;
+    }
+
+    double mu = x[0];
+    for (int t = 1; t < context_len; ++t)
+        if (x[t] > mu)
+            mu = x[t];
+
+    double z = 0.0;
+    for (int t = 0; t < context_len; ++t) {
+        double w = exp(x[t] - mu);
+        int64_t p = table[t / block_size];
+        const uint16_t *vrow = v_cache + pool_row(p, t % block_size, h, block_size, num_kv_heads, head_dim);
+        for (int d = 0; d < head_dim; ++d)
+            out[d] += w * bf16_bits_to_double(vrow[d]);
+        z += w;
+    }
+    for (int d = 0; d < head_dim; ++d)
+        out[d] /= z;
+    return 0;
+}
+
+/*
+ * Paged decode attention, fp64.
+ *
+ * out           [num_pairs][head_dim] doubles; row k is the output of pair k.
+ * q             bf16 bits [num_seqs][num_q_heads][head_dim]
+ * k_cache/v_cache bf16 bits [num_blocks][block_size][num_kv_heads][head_dim]
+ * block_tables  [num_seqs][max_blocks_per_seq]
+ * context_lens  [num_seqs]
+ * pairs         flat indices s * num_q_heads + j of the rows wanted, or NULL
+ *               for all rows in order (num_pairs must then be num_seqs * num_q_heads)
+ * num_threads   OpenMP threads (<= 0: the runtime's default)
+ *
+ * Returns 0; -1 for a bad argument; -2 for a table entry outside the pool;
+ * -3 for a context length outside [0, max_blocks_per_seq * block_size].
+ */
+int oracle_paged_decode(double *out, const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                        const int32_t *block_tables, const int32_t *context_lens,
+                        int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                        int max_blocks_per_seq, int64_t num_blocks, double scale,
+                        const int64_t *pairs, int64_t num_pairs, int num_threads)
+{
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
+        return -1;
+    if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
+        max_blocks_per_seq < 0 || num_blocks < 0 || num_q_heads % num_kv_heads != 0)
+        return -1;
+    if (!pairs && num_pairs != (int64_t)num_seqs * num_q_heads)
+        return -1;
+
+    int max_len = 0;
+    for (int s = 0; s < num_seqs; ++s) {
+        if (context_lens[s] < 0 || (int64_t)context_lens[s] > (int64_t)max_blocks_per_seq * block_size)
+            return -3;
+        if (context_lens[s] > max_len)
+            max_len = context_lens[s];
+    }
+    for (int64_t k = 0; pairs && k < num_pairs; ++k)
+        if (pairs[k] < 0 || pairs[k] >= (int64_t)num_seqs * num_q_heads)
+            return -1;
+
+    int status = 0;
+#ifdef _OPENMP
+    if (num_threads <= 0)
+        num_threads = omp_get_max_threads();
+#pragma omp parallel num_threads(num_threads)
+#endif
+    {
+        double *x = (double *)malloc(sizeof(double) * (size_t)(max_len > 0 ? max_len : 1));
+        int mine = x ? 0 : -1;
+#ifdef _OPENMP
+#pragma omp for schedule(dynamic, 1)
+#endif
+        for (int64_t k = 0; k < num_pairs; ++k) {
+            int64_t flat = pairs ? pairs[k] : k;
+            int s = (int)(flat / num_q_heads);
+            int j = (int)(flat % num_q_heads);
+            if (mine == 0)
+                mine = decode_one(out + k * head_dim, x, q, k_cache, v_cache, block_tables,
+                                  context_lens[s], s, j, num_q_heads, num_kv_heads, head_dim,
+                                  block_size, max_blocks_per_seq, num_blocks, scale);
+        }
+        free(x);
+#ifdef _OPENMP
+#pragma omp critical
+#endif
+        if (mine != 0 && status == 0)
+            status = mine;
+    }
+    return status;
+}
+
+/*
+ * Slot-mapped append: for every token i with slot_mapping[i] >= 0, copy
+ * k[i][h][:] and v[i][h][:] into block slot / bs, offset slot % bs, for every
+ * kv head h.  Later tokens win when two share a slot.
+ *
+ * Returns 0; -1 for a bad argument; -2 when a slot is at or past
+ * num_blocks * block_size (nothing is written in that case).
+ */
+int oracle_kv_append(uint16_t *k_cache, uint16_t *v_cache, const uint16_t *k, const uint16_t *v,
+                     const int64_t *slot_mapping, int64_t num_tokens, int num_kv_heads, int head_dim,
+                     int block_size, int64_t num_blocks)
+{
+    if (!k_cache || !v_cache || !k || !v || (!slot_mapping && num_tokens > 0))
+        return -1;
+    if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks < 0)
+        return -1;
+    for (int64_t i = 0; i < num_tokens; ++i)
+        if (slot_mapping[i] >= num_blocks * block_size)
+            return -2;
+
+    for (int64_t i = 0; i < num_tokens; ++i) {
+        int64_t slot = slot_mapping[i];
+        if (slot < 0)
+            continue;
+        int64_t p = slot / block_size;
+        int off = (int)(slot % block_size);
+        for (int h = 0; h < num_kv_heads; ++h) {
+            int64_t dst = pool_row(p, off, h, block_size, num_kv_heads, head_dim);
+            int64_t src = (i * num_kv_heads + h) * (int64_t)head_dim;
+            for (int d = 0; d < head_dim; ++d) {
+                k_cache[dst + d] = k[src + d];
+                v_cache[dst + d] = v[src + d];
+            }
+        }
+    }
+    return 0;
+}

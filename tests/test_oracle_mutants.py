@@ -1,0 +1,46 @@
+"""Plant mistakes in copies of oracle.c and check that the pins catch every one.
+
+Each mutant is a plausible slip (a dropped term, a wrong sign, index or
+operand).  All mutants keep every memory access inside its buffer, so running
+them on the CPU is safe.
+"""
+import pytest
+
+import oracle
+from oracle_pins import ALL_PINS
+
+MUTANTS = [
+    ("exponent sign", "exp(x[t] - mu)", "exp(mu - x[t])"),
+    ("no max subtraction", "exp(x[t] - mu)", "exp(x[t])"),
+    ("min instead of max", "if (x[t] > mu)", "if (x[t] < mu)"),
+    ("no normalisation", "out[d] /= z;", "out[d] /= 1.0;"),
+    ("normalise by count", "z += w;", "z += 1.0;"),
+    ("scale dropped", "x[t] = scale * dot;", "x[t] = dot;"),
+    ("head grouping j mod Hkv", "const int h = j / group;", "const int h = j % num_kv_heads;"),
+    ("q row of the kv head", "((int64_t)s * num_q_heads + j) * head_dim", "((int64_t)s * num_q_heads + h) * head_dim"),
+    ("values read from K", "v_cache + pool_row", "k_cache + pool_row"),
+    ("block table ignored", "table[t / block_size]", "(t / block_size)"),
+    ("offset off by one", "pool_row(p, t % block_size", "pool_row(p, (t + 1) % block_size"),
+    ("last token dropped from PV", "for (int t = 0; t < context_len; ++t) {\n        double w",
+     "for (int t = 0; t + 1 < context_len; ++t) {\n        double w"),
+    ("pool layout transposed", "((p * block_size + off) * num_kv_heads + h)", "((p * num_kv_heads + h) * block_size + off)"),
+    ("append ignores head", "int64_t src = (i * num_kv_heads + h) * (int64_t)head_dim;",
+     "int64_t src = (i * num_kv_heads) * (int64_t)head_dim;"),
+    ("append crosses k and v", "k_cache[dst + d] = k[src + d];", "k_cache[dst + d] = v[src + d];"),
+    ("append offset 0", "int off = (int)(slot % block_size);", "int off = 0;"),
+]
+
+
+@pytest.mark.parametrize("label,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_mutant(label, old, new, tmp_path):
+    src = oracle.source()
+    assert old in src, f"mutation site for '{label}' not found"
+    lib = oracle.build_variant(src.replace(old, new), str(tmp_path))
+    caught = []
+    for pin in ALL_PINS:
+        try:
+            pin(lib=lib)
+        except (AssertionError, oracle.OracleError) as e:
+            caught.append(pin.__name__)
+            break
+    assert caught, f"no pin caught the mutant '{label}'"
