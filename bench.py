@@ -1,0 +1,502 @@
+#!/usr/bin/env python
+"""Benchmark: one paged decode step (slot-mapped append + paged decode attention).
+
+A step is the whole hot path over one synthetic batch: kv_cache_append of the
+step's new keys/values, then paged_attn_decode (persistent decode kernel, plus
+the log-sum-exp merge kernel when contexts are split). The default workload is
+the Llama-3-8B-shaped GQA batch (256 sequences, 32 q / 8 kv heads, head_dim 128,
+block_size 16, context lengths U[128, 4096], pool 1.2x the needed blocks,
+shuffled) -- 2.25 GB of K/V read per step, far larger than L2; L2 is also
+flushed (memset of 2x its size) between timed steps, outside the step's events.
+
+Prints one JSON line (rank 0). `value` is KV GB/s (algorithmic K+V bytes of
+the step / device time); see the design doc for the metric's definition.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Under torchrun each rank runs its own independent batch (weak scaling, no
+data-path collective); the timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "paged decode KV GB/s & % of B200 HBM peak; seq·tokens/s per decode step"
+FALLBACK_HBM_GBS = 6650.0
+PROFILES = os.path.join(ROOT, "profiles")
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="llama3_8b", choices=workloads.CONFIG_ORDER)
+    p.add_argument("--partition-tokens", type=int, default=0)
+    p.add_argument("--num-stages", type=int, default=0)
+    p.add_argument("--ctas-per-sm", type=int, default=0)
+    p.add_argument("--math", type=int, default=0)
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args(argv)
+
+
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Each rank decodes its own batch; rank 0 uses the workload's canonical seed."""
+    return base_seed + 7919 * rank
+
+
+def aggregate(sum_values, max_values):
+    """Sum `sum_values` and max `max_values` over ranks (identity without a process group)."""
+    import torch.distributed as dist
+    s = torch.tensor(sum_values, dtype=torch.float64)
+    m = torch.tensor(max_values, dtype=torch.float64)
+    if dist.is_available() and dist.is_initialized():
+        dev = torch.device("cuda", torch.cuda.current_device()) if dist.get_backend() == "nccl" else torch.device("cpu")
+        s, m = s.to(dev), m.to(dev)
+        dist.all_reduce(s, op=dist.ReduceOp.SUM)
+        dist.all_reduce(m, op=dist.ReduceOp.MAX)
+    return s.cpu().tolist(), m.cpu().tolist()
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def decode_sources_sha():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "paged_kv_cache_377_b200", "csrc")
+    for name in ("decode.cu", "decode_common.cuh", "device_utils.cuh"):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per decode launch from a committed ncu capture, if it was taken
+    on the current decode sources (else None)."""
+    path = os.path.join(PROFILES, "decode_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(workload)
+    if not e or e.get("decode_sources_sha") != decode_sources_sha():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Polls SM clock, power and clock-event reasons through NVML while running."""
+
+    NAMES = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples = []
+        self.max_mhz = None
+        self.error = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = self._handle(pynvml, device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report the clocks as unknown
+            self.error = repr(e)
+            self._nvml = None
+        self.period = period_s
+
+    @staticmethod
+    def _handle(pynvml, device_index):
+        props = torch.cuda.get_device_properties(device_index)
+        try:
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            return pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + str(props.uuid)).encode())
+
+    def _run(self):
+        nv = self._nvml
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                pw = nv.nvmlDeviceGetPowerUsage(self._h) / 1000.0
+                self.samples.append((time.time(), mhz, rs, pw))
+            except Exception as e:
+                self.error = repr(e)
+            self._stop.wait(self.period)
+
+    def __enter__(self):
+        if self._nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "note": self.error or "no samples"}
+        reasons = set()
+        for _, _, rs, _ in self.samples:
+            for bit, name in self.NAMES.items():
+                if rs & bit:
+                    reasons.add(name)
+        return {
+            "sm_mhz": statistics.median(s[1] for s in self.samples),
+            "sm_max_mhz": self.max_mhz,
+            "reasons": sorted(reasons),
+            "samples": len(self.samples),
+            "power_w_max": max(s[3] for s in self.samples),
+            "source": "NVML, polled every 10 ms during the timed region",
+        }
+
+
+# ----------------------------------------------------------------------------- our arm
+
+class Step:
+    """Device buffers of one decode step and the two library calls that make it."""
+
+    def __init__(self, batch, args, device):
+        import paged_kv_cache_377_b200 as pkv
+        self.pkv = pkv
+        b = batch
+        self.b = b
+        self.kc = b.k_cache.to(device)
+        self.vc = b.v_cache.to(device)
+        self.q = b.q.to(device)
+        self.k_new = b.k_new.to(device)
+        self.v_new = b.v_new.to(device)
+        self.bt = b.block_tables.to(device)
+        self.cl = b.context_lens.to(device)
+        self.slots = b.slot_mapping.to(device)
+        self.out = torch.empty_like(self.q)
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+        self.opts = dict(partition_tokens=args.partition_tokens, num_stages=args.num_stages,
+                         ctas_per_sm=args.ctas_per_sm, math=args.math)
+        self.ws = pkv.allocate_workspace(b.num_seqs, b.num_q_heads, b.head_dim, b.max_blocks_per_seq,
+                                         b.block_size, args.partition_tokens, device=device)
+
+    def append(self, stream=None):
+        self.pkv.kv_cache_append(self.k_new, self.v_new, self.kc, self.vc, self.slots, self.status, stream=stream)
+
+    def decode(self, stream=None):
+        self.pkv.paged_attn_decode(self.out, self.q, self.kc, self.vc, self.bt, self.cl, self.b.scale, self.ws,
+                                   stream=stream, **self.opts)
+
+    def decode_launches(self):
+        """Kernels one paged_attn_decode call launches (decode, plus merge when split)."""
+        P = self.opts["partition_tokens"] or 512
+        n_split = -(-self.b.max_blocks_per_seq * self.b.block_size // P)
+        chunks = -(-self.b.num_seqs // 8192)
+        return chunks * (2 if n_split > 1 else 1)
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch.distributed as dist
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    cfg = workloads.CONFIGS[args.workload]
+    batch = workloads.make_batch(args.workload, seed=rank_seed(cfg.seed, rank), device=device, poison=False)
+    step = Step(batch, args, device)
+    kv = workloads.kv_bytes(batch)
+    ctx_tokens = int(batch.context_lens.sum())
+    S = batch.num_seqs
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    flush = torch.empty(2 * l2, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step.append()
+        step.decode()
+    torch.cuda.synchronize()
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    sampler = ClockSampler(local_rank)
+    barrier()
+    torch.cuda.synchronize()
+    with sampler:
+        for i in range(K):
+            flush.zero_()                      # L2 flush, outside the step's events
+            ev[i][0].record(stream)
+            step.append()
+            ev[i][1].record(stream)
+            step.decode()
+            ev[i][2].record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    step_ms = [e[0].elapsed_time(e[2]) for e in ev]
+    decode_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    append_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    total_ms = sum(step_ms)
+    status = step.pkv.read_status(step.status) | step.pkv.read_status(step.ws)
+    if status:
+        raise RuntimeError(f"device status {status} after the timed steps")
+
+    (sum_kv, sum_seq, sum_tok), (max_ms,) = aggregate([kv * K, S * K, ctx_tokens * K], [total_ms])
+    seconds = max_ms / 1e3
+    value = sum_kv / seconds / 1e9
+    hbm, hbm_kind = measured_peaks()
+    mean_decode_ms = statistics.fmean(decode_ms)
+    achieved = kv / (mean_decode_ms / 1e3) / 1e9
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(step, args, flush, stream, kv, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(batch, kv, S, ctx_tokens)
+
+    traffic = profiled_traffic(args.workload)
+    result = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(max_ms / K, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic",
+        "config": config_block(args, batch, world),
+        "pct_of_hbm_peak": round(100.0 * value / (hbm * world), 2),
+        "seq_per_s": round(sum_seq / seconds, 1),
+        "ctx_tokens_per_s": round(sum_tok / seconds, 1),
+        "append_us_mean": round(1e3 * statistics.fmean(append_ms), 3),
+        "decode_us_mean": round(1e3 * mean_decode_ms, 3),
+        "decode_us_median": round(1e3 * statistics.median(decode_ms), 3),
+        "roofline": {
+            "kernel": "paged_attn_decode (paged_decode_kernel + lse_merge_kernel)",
+            "bound": "hbm",
+            "achieved": round(achieved, 2),
+            "peak": hbm,
+            "peak_kind": f"{hbm_kind} hbm_gbs (copy)",
+            "unit": "GB/s",
+            "frac": round(achieved / hbm, 4),
+            "algorithmic_bytes_per_launch": kv,
+            "traffic": traffic,
+        },
+        "clocks": sampler.summary(),
+        "gpu_launches": K * (1 + step.decode_launches()),
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+    }
+    return result
+
+
+def run_e2e(step, args, flush, stream, kv, world):
+    """The same step through the public API with HOST inputs: every step copies its
+    inputs (q, new k/v, tables, lengths, slots) from pinned memory and reads `out`
+    back; the KV pool stays resident on the device (it is the cache)."""
+    host = {n: getattr(step, n).cpu().pin_memory() for n in ("q", "k_new", "v_new", "bt", "cl", "slots")}
+    out_host = torch.empty(step.out.shape, dtype=step.out.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+    K = args.steps
+
+    def one():
+        for n, t in host.items():
+            getattr(step, n).copy_(t, non_blocking=True)
+        step.append()
+        step.decode()
+        out_host.copy_(step.out, non_blocking=True)
+
+    for _ in range(max(args.warmup, 3)):
+        one()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for i in range(K):
+        flush.zero_()
+        ev[i][0].record(stream)
+        one()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    total_ms = sum(a.elapsed_time(b) for a, b in ev)
+    (sum_kv,), (max_ms,) = aggregate([kv * K], [total_ms])
+    return {"value": round(sum_kv / (max_ms / 1e3) / 1e9, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": round(max_ms / K, 5)}
+
+
+def config_block(args, batch, world):
+    cfg = workloads.CONFIGS[args.workload]
+    c = {
+        "workload": args.workload,
+        "description": cfg.description,
+        "num_seqs": batch.num_seqs,
+        "num_q_heads": batch.num_q_heads,
+        "num_kv_heads": batch.num_kv_heads,
+        "head_dim": batch.head_dim,
+        "block_size": batch.block_size,
+        "pool_blocks": batch.num_blocks,
+        "context_tokens": int(batch.context_lens.sum()),
+        "kv_bytes_per_step": workloads.kv_bytes(batch),
+        "unique_kv_bytes_per_step": workloads.unique_kv_bytes(batch),
+        "kv_dtype": "bf16",
+        "l2": "inputs larger than L2, and L2 flushed (memset 2x L2) between timed steps",
+        "parallelism": "replicas: one independent batch per GPU" if world > 1 else "single GPU",
+    }
+    for k in ("partition_tokens", "num_stages", "ctas_per_sm", "math"):
+        if getattr(args, k):
+            c[k] = getattr(args, k)
+    return c
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def cpu_baseline(batch, kv, S, ctx_tokens, min_seconds=10.0, max_runs=5):
+    """The fp64 oracle as it stands (append + decode), timed on the host cores on
+    the same batch: runs of the whole step until ~10 s of CPU work are done."""
+    import oracle
+    host = batch.to("cpu")
+    times = []
+    t_all = time.perf_counter()
+    while len(times) < max_runs and (time.perf_counter() - t_all) < min_seconds:
+        t0 = time.perf_counter()
+        oracle.decode_step(host)
+        times.append(time.perf_counter() - t0)
+    t = statistics.median(times)
+    return {
+        "value": round(kv / t / 1e9, 3),
+        "unit": "GB/s",
+        "cores": os.cpu_count(),
+        "kind": "oracle",
+        "sample": f"whole batch ({S} seqs, {ctx_tokens} context tokens), append + decode, "
+                  f"median of {len(times)} runs; {statistics.median(times):.2f} s per step",
+        "seq_per_s": round(S / t, 2),
+    }
+
+
+def run_reference(args):
+    """The oracle as it stands, on bounded samples of the workload: step i decodes
+    a slice of the batch's sequences (append + decode), sized so the whole run
+    stays within a few minutes."""
+    import oracle
+    cfg = workloads.CONFIGS[args.workload]
+    batch = workloads.make_batch(args.workload, device="cpu", poison=False)
+    S = batch.num_seqs
+    order = np.random.default_rng(0).permutation(S)
+
+    def sub(idx):
+        idx = np.sort(idx)
+        return workloads.DecodeBatch(**{
+            **batch.__dict__, "num_seqs": len(idx),
+            "context_lens": batch.context_lens[idx], "block_tables": batch.block_tables[idx],
+            "slot_mapping": batch.slot_mapping[idx], "q": batch.q[idx],
+            "k_new": batch.k_new[idx], "v_new": batch.v_new[idx]})
+
+    # size the slice from one probe step: aim at ~150 s for warmup + steps
+    probe = sub(order[:8])
+    t0 = time.perf_counter()
+    oracle.decode_step(probe)
+    t_probe = time.perf_counter() - t0
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    n = int(max(1, min(S, 8 * budget / max(t_probe, 1e-3))))
+    slices = [sub(order[(i * n) % S:(i * n) % S + n]) for i in range(args.steps + args.warmup)]
+    for sl in slices[:args.warmup]:
+        oracle.decode_step(sl)
+    kv_total = 0
+    seqs = 0
+    t0 = time.perf_counter()
+    for sl in slices[args.warmup:]:
+        oracle.decode_step(sl)
+        kv_total += workloads.kv_bytes(sl)
+        seqs += sl.num_seqs
+    seconds = time.perf_counter() - t0
+    value = kv_total / seconds / 1e9
+    sample = (f"{n} of {S} sequences per step (all heads), append + decode; "
+              f"{args.steps} timed steps, {args.warmup} warm-up")
+    return {
+        "metric": METRIC,
+        "value": round(value, 4),
+        "unit": "GB/s",
+        "n_gpus": args.gpus,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(1e3 * seconds / max(1, args.steps), 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic",
+        "config": config_block(args, batch, 1),
+        "impl": "reference",
+        "seq_per_s": round(seqs / seconds, 3),
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": os.cpu_count(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ----------------------------------------------------------------------------- main
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args)), flush=True)
+        return 0
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        result = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(result), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,188 @@
+/*
+ * pagedkv.h -- C ABI of the paged KV-cache decode library (libpagedkv.so).
+ *
+ * The operation: single-query attention for a batch of decoding sequences
+ * whose keys and values live in fixed-size blocks scattered through one
+ * preallocated pool, reached through a per-sequence block table.
+ *   - "vLLM Fundamentals: Paged Attention and Batching", section "Paged
+ *     Attention": the KV cache is split into blocks that are not contiguous,
+ *     each sequence gets a block table, and the paged kernel follows the table
+ *     to gather the blocks; section "Just a python process": the pool is one
+ *     large tensor allocated once, and the engine packs the block tables into
+ *     tensors and sends them to the GPU at every step.
+ *   - "Deep Dive into vLLM: PagedAttention & High-Performance Inference",
+ *     section 2.1: logical blocks map to physical blocks through the table.
+ *   - runbyai.xyz post 449, section 1: a decode step reads the keys and values
+ *     of all previous tokens, and is limited by memory bandwidth.
+ *
+ * Conventions for every call:
+ *   - Pointers named d_* or documented as "device" are device pointers owned by
+ *     the caller; the library never allocates, frees or keeps any memory.
+ *   - Tensors are dense, row-major, in the layouts given below. bf16 tensors
+ *     (k, v, q, out, caches) must be 16-byte aligned.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream). Calls only enqueue work; nothing is synchronised unless stated.
+ *   - Return value: PKV_OK (0) or a negative PKV_ERR_* code; pkv_last_error()
+ *     then gives a message (thread-local, valid until the next call on that
+ *     thread). Argument checks run before any CUDA call, so a rejected call
+ *     enqueues nothing.
+ *   - Problems that only the device can see (a table entry outside the pool, a
+ *     context length past the table, a slot past the pool, a bounded wait that
+ *     ran out) never trap: the kernels skip the bad access and OR a
+ *     PKV_STATUS_* bit into a device status word the caller can read.
+ *
+ * Readings where the pages are silent: the attention is softmax(scale*q.K^T).V
+ * over all context_lens[s] tokens of sequence s (no mask inside the context);
+ * query head j reads kv head floor(j / (num_q_heads / num_kv_heads)); the pool
+ * layout is [num_blocks][block_size][num_kv_heads][head_dim]; the slot of a
+ * token is physical_block * block_size + offset_in_block.
+ */
+#ifndef PAGEDKV_H
+#define PAGEDKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define PKV_OK 0
+#define PKV_ERR_INVALID_ARGUMENT (-1) /* null pointer, bad size, misaligned pointer, small workspace */
+#define PKV_ERR_UNSUPPORTED (-2)      /* head_dim, block_size or head grouping not compiled in */
+#define PKV_ERR_CUDA (-3)             /* a CUDA runtime call or a launch failed */
+
+/* Bits of the device status word (sticky: kernels only OR bits in). */
+#define PKV_STATUS_BAD_BLOCK_ID 1     /* a needed table entry is outside [0, num_blocks); that block is skipped */
+#define PKV_STATUS_BAD_CONTEXT_LEN 2  /* context_lens[s] < 0 or > max_blocks_per_seq * block_size; clamped */
+#define PKV_STATUS_WAIT_TIMEOUT 4     /* a bounded wait inside a kernel gave up; outputs are not valid */
+#define PKV_STATUS_BAD_SLOT 8         /* an append slot is >= num_blocks * block_size; that token is skipped */
+
+/* Supported shapes of the decode kernels. */
+#define PKV_MAX_GROUP 8               /* num_q_heads / num_kv_heads <= 8 */
+
+/*
+ * Tuning knobs of paged_attn_decode_ex. Zero in any field means "default".
+ *   partition_tokens  tokens of one context split (a multiple of block_size);
+ *                     default 512. Sequences longer than this are split and
+ *                     their partial results merged with a log-sum-exp
+ *                     reduction kernel.
+ *   num_stages        depth of the shared-memory ring of KV blocks in flight per
+ *                     CTA (2..16); default chosen from the block bytes.
+ *   ctas_per_sm       resident CTAs per SM of the persistent grid; default: the
+ *                     occupancy limit.
+ *   math              0 = default, 1 = fp32 CUDA cores, 2 = bf16 tensor cores
+ *                     (mma.sync m16n8k16, fp32 accumulate).
+ */
+typedef struct pkv_decode_options {
+    int partition_tokens;
+    int num_stages;
+    int ctas_per_sm;
+    int math;
+} pkv_decode_options;
+
+/*
+ * Bytes of device workspace paged_attn_decode needs for this shape.
+ * Layout: [0, 256) header whose first int32 is the device status word; then
+ * fp32 partial outputs [num_seqs][num_q_heads][n_split][head_dim] and fp32
+ * log2-sum-exp values [num_seqs][num_q_heads][n_split], n_split =
+ * ceil(max_blocks_per_seq * block_size / partition_tokens). Only splits that
+ * hold tokens are written.
+ * partition_tokens = 0 means the default. Host-only; returns PKV_OK and sets *bytes.
+ */
+int pkv_decode_workspace_bytes(int num_seqs, int num_q_heads, int head_dim, int max_blocks_per_seq,
+                               int block_size, int partition_tokens, size_t *bytes);
+
+/*
+ * Paged decode attention (one query token per sequence).
+ *
+ * out           device bf16 [num_seqs][num_q_heads][head_dim]   (written)
+ * q             device bf16 [num_seqs][num_q_heads][head_dim]
+ * k_cache       device bf16 [num_blocks][block_size][num_kv_heads][head_dim]
+ * v_cache       device bf16, same layout as k_cache
+ * block_tables  device int32 [num_seqs][max_blocks_per_seq]; entry b of row s is
+ *               the physical block of logical block b of sequence s. Only
+ *               entries b < ceil(context_lens[s] / block_size) are read.
+ * context_lens  device int32 [num_seqs]; 0 gives an all-zero output row.
+ * scale         multiplies q.k before the softmax (e.g. 1/sqrt(head_dim)).
+ * workspace     device, at least pkv_decode_workspace_bytes() bytes, 256-byte
+ *               aligned; its status word is ORed, never cleared, by this call.
+ *
+ * Supported: head_dim in {64, 128}; block_size in {16, 32}; num_q_heads a
+ * multiple of num_kv_heads with a ratio <= PKV_MAX_GROUP; num_blocks *
+ * block_size < 2^31. Any num_seqs >= 0 (0 is a no-op).
+ * Per call: one persistent decode kernel, plus one reduction kernel when a
+ * context can be longer than partition_tokens. Results are bitwise
+ * reproducible and depend only on the logical order of tokens, not on where
+ * their blocks sit in the pool.
+ */
+int paged_attn_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
+                      const int32_t *block_tables, const int32_t *context_lens,
+                      int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                      int block_size, float scale, int max_blocks_per_seq, int num_blocks,
+                      void *workspace, size_t workspace_bytes, void *stream);
+
+/* paged_attn_decode with tuning knobs (opts may be NULL = all defaults). */
+int paged_attn_decode_ex(void *out, const void *q, const void *k_cache, const void *v_cache,
+                         const int32_t *block_tables, const int32_t *context_lens,
+                         int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                         int block_size, float scale, int max_blocks_per_seq, int num_blocks,
+                         void *workspace, size_t workspace_bytes, const pkv_decode_options *opts,
+                         void *stream);
+
+/*
+ * Slot-mapped cache append: for every token i with slot_mapping[i] >= 0 and
+ * every kv head h, copies k[i][h][:] to k_cache[slot / block_size]
+ * [slot % block_size][h][:] and v[i][h][:] likewise (runbyai.xyz post 449,
+ * sections 1-2: each step computes and caches the new token's key and value).
+ *
+ * k, v          device bf16 [num_tokens][num_kv_heads][head_dim]
+ * k_cache/v_cache device bf16 [num_blocks][block_size][num_kv_heads][head_dim] (updated in place)
+ * slot_mapping  device int64 [num_tokens]; < 0 means "no write" (padding)
+ * d_status      device int32 status word, or NULL; gets PKV_STATUS_BAD_SLOT for
+ *               a slot >= num_blocks * block_size (that token is skipped)
+ *
+ * head_dim must be a multiple of 8. Bit-exact copy. Two tokens with the same
+ * slot race (either may win); the caller keeps slots distinct within a call.
+ */
+int kv_cache_append(const void *k, const void *v, void *k_cache, void *v_cache,
+                    const int64_t *slot_mapping, int num_tokens, int num_kv_heads, int head_dim,
+                    int block_size, int num_blocks, int32_t *d_status, void *stream);
+
+/*
+ * Device check of a batch's tables: ORs PKV_STATUS_BAD_CONTEXT_LEN for any
+ * context length outside [0, max_blocks_per_seq * block_size] and
+ * PKV_STATUS_BAD_BLOCK_ID for any needed entry outside [0, num_blocks) into
+ * *d_status. Never traps; enqueues one small kernel.
+ */
+int pkv_validate(const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
+                 int max_blocks_per_seq, int block_size, int num_blocks, int32_t *d_status,
+                 void *stream);
+
+/*
+ * Copies the device status word to *status (host) after synchronising `stream`,
+ * and zeroes it when clear != 0. For paged_attn_decode the word is the first
+ * int32 of the workspace.
+ */
+int pkv_read_status(int32_t *d_status, int32_t *status, int clear, void *stream);
+
+/*
+ * Self-test of the kernels' failure path: enqueues one kernel that waits on an
+ * mbarrier nothing ever arrives at. The bounded wait gives up after about one
+ * second and ORs PKV_STATUS_WAIT_TIMEOUT into *d_status (device int32); the
+ * kernel then returns normally and the context stays usable. Bit 0x40000000
+ * is set instead if the wait wrongly succeeded.
+ */
+int pkv_selftest_bounded_wait(int32_t *d_status, void *stream);
+
+/* Message of the last failed call on this thread ("" if none). */
+const char *pkv_last_error(void);
+
+/* Library version string. */
+const char *pkv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDKV_H */

@@ -1,0 +1,38 @@
+"""Paged KV-cache decode attention for B200 (sm_100a).
+
+A thin binding over the C ABI of ``libpagedkv.so`` (see include/pagedkv.h):
+argument marshalling only -- every step of the decode path runs in the CUDA
+kernels of the library. Tensors are torch tensors on the GPU; torch supplies
+device memory and streams. If the library cannot be loaded (or built with
+nvcc), every call raises: there is no CPU fallback.
+"""
+from __future__ import annotations
+
+from ._binding import (  # noqa: F401
+    PKV_STATUS_BAD_BLOCK_ID,
+    PKV_STATUS_BAD_CONTEXT_LEN,
+    PKV_STATUS_BAD_SLOT,
+    PKV_STATUS_WAIT_TIMEOUT,
+    PagedKVError,
+    allocate_workspace,
+    kv_cache_append,
+    library,
+    library_path,
+    paged_attn_decode,
+    read_status,
+    selftest_bounded_wait,
+    validate,
+    workspace_bytes,
+)
+
+__all__ = [
+    "PagedKVError",
+    "allocate_workspace",
+    "kv_cache_append",
+    "library",
+    "library_path",
+    "paged_attn_decode",
+    "read_status",
+    "validate",
+    "workspace_bytes",
+]

@@ -1,0 +1,208 @@
+"""ctypes binding of libpagedkv.so: same names as the C ABI, torch tensors in."""
+from __future__ import annotations
+
+import ctypes
+import fcntl
+import os
+import threading
+from typing import Optional
+
+import torch
+
+from . import build as _build
+
+PKV_OK = 0
+PKV_STATUS_BAD_BLOCK_ID = 1
+PKV_STATUS_BAD_CONTEXT_LEN = 2
+PKV_STATUS_WAIT_TIMEOUT = 4
+PKV_STATUS_BAD_SLOT = 8
+
+_lock = threading.Lock()
+_lib: Optional[ctypes.CDLL] = None
+
+
+class PagedKVError(RuntimeError):
+    """A library call returned an error code (message from pkv_last_error)."""
+
+    def __init__(self, fn: str, code: int, msg: str):
+        super().__init__(f"{fn} failed with code {code}: {msg}")
+        self.code = code
+
+
+class _Options(ctypes.Structure):
+    _fields_ = [("partition_tokens", ctypes.c_int), ("num_stages", ctypes.c_int),
+                ("ctas_per_sm", ctypes.c_int), ("math", ctypes.c_int)]
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def _ensure_built() -> str:
+    """Builds the library with nvcc when it is missing or older than its sources."""
+    if not _build.is_stale():
+        return _build.LIB
+    os.makedirs(_build.BUILD, exist_ok=True)
+    with open(os.path.join(_build.BUILD, ".lock"), "w") as lk:
+        fcntl.flock(lk, fcntl.LOCK_EX)
+        try:
+            return _build.build()
+        finally:
+            fcntl.flock(lk, fcntl.LOCK_UN)
+
+
+def library() -> ctypes.CDLL:
+    """The loaded libpagedkv.so (built first if needed). Raises if unavailable."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            path = _ensure_built()
+            lib = ctypes.CDLL(path)
+            P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+            lib.pkv_last_error.restype = ctypes.c_char_p
+            lib.pkv_last_error.argtypes = []
+            lib.pkv_version.restype = ctypes.c_char_p
+            lib.pkv_decode_workspace_bytes.restype = I
+            lib.pkv_decode_workspace_bytes.argtypes = [I, I, I, I, I, I, ctypes.POINTER(Z)]
+            lib.paged_attn_decode.restype = I
+            lib.paged_attn_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, I, I, P, Z, P]
+            lib.paged_attn_decode_ex.restype = I
+            lib.paged_attn_decode_ex.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, I, I, P, Z,
+                                                 ctypes.POINTER(_Options), P]
+            lib.kv_cache_append.restype = I
+            lib.kv_cache_append.argtypes = [P, P, P, P, P, I, I, I, I, I, P, P]
+            lib.pkv_validate.restype = I
+            lib.pkv_validate.argtypes = [P, P, I, I, I, I, P, P]
+            lib.pkv_selftest_bounded_wait.restype = I
+            lib.pkv_selftest_bounded_wait.argtypes = [P, P]
+            lib.pkv_read_status.restype = I
+            lib.pkv_read_status.argtypes = [P, ctypes.POINTER(ctypes.c_int32), I, P]
+            _lib = lib
+        return _lib
+
+
+def _check(fn: str, rc: int) -> None:
+    if rc != PKV_OK:
+        raise PagedKVError(fn, rc, library().pkv_last_error().decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        stream = stream.cuda_stream
+    return ctypes.c_void_p(int(stream))
+
+
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be on a CUDA device (got {t.device})")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype} (got {t.dtype})")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions (got shape {tuple(t.shape)})")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def workspace_bytes(num_seqs: int, num_q_heads: int, head_dim: int, max_blocks_per_seq: int, block_size: int,
+                    partition_tokens: int = 0) -> int:
+    n = ctypes.c_size_t(0)
+    _check("pkv_decode_workspace_bytes", library().pkv_decode_workspace_bytes(
+        num_seqs, num_q_heads, head_dim, max_blocks_per_seq, block_size, partition_tokens, ctypes.byref(n)))
+    return int(n.value)
+
+
+def allocate_workspace(num_seqs: int, num_q_heads: int, head_dim: int, max_blocks_per_seq: int, block_size: int,
+                       partition_tokens: int = 0, device=None) -> torch.Tensor:
+    """A zeroed uint8 workspace of the required size (its first int32 is the status word)."""
+    n = workspace_bytes(num_seqs, num_q_heads, head_dim, max_blocks_per_seq, block_size, partition_tokens)
+    return torch.zeros(n, dtype=torch.uint8, device=device if device is not None else "cuda")
+
+
+def paged_attn_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                      block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float,
+                      workspace: torch.Tensor, partition_tokens: int = 0, num_stages: int = 0,
+                      ctas_per_sm: int = 0, math: int = 0, stream=None) -> torch.Tensor:
+    """out[s, j] = softmax_t(scale * q[s, j] . K_t) . V_t over the sequence's paged tokens.
+
+    q, out: bf16 [S, Hq, D]; k_cache, v_cache: bf16 [NB, bs, Hkv, D];
+    block_tables: int32 [S, MB]; context_lens: int32 [S]; workspace: uint8 from
+    allocate_workspace(). Enqueued on ``stream`` (default: torch's current stream).
+    """
+    _need(q, "q", torch.bfloat16, 3)
+    _need(out, "out", torch.bfloat16, 3)
+    _need(k_cache, "k_cache", torch.bfloat16, 4)
+    _need(v_cache, "v_cache", torch.bfloat16, 4)
+    _need(block_tables, "block_tables", torch.int32, 2)
+    _need(context_lens, "context_lens", torch.int32, 1)
+    _need(workspace, "workspace", torch.uint8, 1)
+    S, Hq, D = q.shape
+    NB, bs, Hkv, D2 = k_cache.shape
+    if out.shape != q.shape or v_cache.shape != k_cache.shape or D2 != D:
+        raise ValueError("shape mismatch between q/out or k_cache/v_cache")
+    if block_tables.shape[0] != S or context_lens.shape[0] != S:
+        raise ValueError("block_tables and context_lens must have num_seqs rows")
+    opts = _Options(partition_tokens, num_stages, ctas_per_sm, math)
+    _check("paged_attn_decode", library().paged_attn_decode_ex(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
+        S, Hq, Hkv, D, bs, float(scale), block_tables.shape[1], NB, _ptr(workspace), workspace.numel(),
+        ctypes.byref(opts), _stream(stream)))
+    return out
+
+
+def kv_cache_append(k: torch.Tensor, v: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                    slot_mapping: torch.Tensor, status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """k_cache[slot // bs, slot % bs] = k[i] (and v) for every token i with slot >= 0.
+
+    k, v: bf16 [T, Hkv, D]; caches bf16 [NB, bs, Hkv, D]; slot_mapping int64 [T];
+    status: optional int32 device tensor (status word, PKV_STATUS_BAD_SLOT).
+    """
+    _need(k, "k", torch.bfloat16, 3)
+    _need(v, "v", torch.bfloat16, 3)
+    _need(k_cache, "k_cache", torch.bfloat16, 4)
+    _need(v_cache, "v_cache", torch.bfloat16, 4)
+    _need(slot_mapping, "slot_mapping", torch.int64, 1)
+    if status is not None:
+        _need(status, "status", torch.int32, 1)
+    T, Hkv, D = k.shape
+    NB, bs, Hkv2, D2 = k_cache.shape
+    if v.shape != k.shape or v_cache.shape != k_cache.shape or (Hkv2, D2) != (Hkv, D) or slot_mapping.shape[0] != T:
+        raise ValueError("shape mismatch between k/v, caches and slot_mapping")
+    _check("kv_cache_append", library().kv_cache_append(
+        _ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache), _ptr(slot_mapping), T, Hkv, D, bs, NB,
+        _ptr(status), _stream(stream)))
+
+
+def validate(block_tables: torch.Tensor, context_lens: torch.Tensor, num_blocks: int, block_size: int,
+             status: torch.Tensor, stream=None) -> None:
+    """Enqueues the device check of tables and lengths; bits go into ``status``."""
+    _need(block_tables, "block_tables", torch.int32, 2)
+    _need(context_lens, "context_lens", torch.int32, 1)
+    _need(status, "status", torch.int32, 1)
+    _check("pkv_validate", library().pkv_validate(
+        _ptr(block_tables), _ptr(context_lens), block_tables.shape[0], block_tables.shape[1], block_size,
+        num_blocks, _ptr(status), _stream(stream)))
+
+
+def read_status(status: torch.Tensor, clear: bool = False, stream=None) -> int:
+    """Synchronises the stream and returns the status word (a workspace's first int32, or an int32 tensor)."""
+    if status.dtype == torch.uint8:
+        status = status[:4].view(torch.int32)
+    _need(status, "status", torch.int32, 1)
+    out = ctypes.c_int32(0)
+    _check("pkv_read_status", library().pkv_read_status(_ptr(status), ctypes.byref(out), int(clear),
+                                                        _stream(stream)))
+    return int(out.value)
+
+
+def selftest_bounded_wait(status: torch.Tensor, stream=None) -> None:
+    """Enqueues the kernel whose bounded wait must give up (about one second)."""
+    _need(status, "status", torch.int32, 1)
+    _check("pkv_selftest_bounded_wait", library().pkv_selftest_bounded_wait(_ptr(status), _stream(stream)))

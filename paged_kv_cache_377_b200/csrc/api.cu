@@ -1,0 +1,298 @@
+// api.cu -- the C ABI of libpagedkv.so (declared in include/pagedkv.h).
+//
+// Every entry point checks its arguments on the host before any CUDA call,
+// then enqueues kernels on the caller's stream. The library allocates nothing
+// and keeps no per-call state: the KV pool, the tables and the workspace are
+// the caller's ("vLLM Fundamentals: Paged Attention and Batching", section
+// "Just a python process": one large pool tensor allocated once by the engine;
+// the engine sends the packed block tables to the GPU at every step).
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "launch.h"
+#include "pagedkv.h"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+int fail(int code, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof g_err, fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+int ok() {
+    g_err[0] = '\0';
+    return PKV_OK;
+}
+
+int cuda_fail(cudaError_t e, const char *what) {
+    return fail(PKV_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int group_pad(int g) { return g <= 1 ? 1 : g <= 2 ? 2 : g <= 4 ? 4 : 8; }
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// Tensor map over a pool [num_blocks][bs][Hkv][D] bf16 seen as 4D
+// (64, D/64, Hkv, num_blocks*bs), innermost first; one box = all bs rows of one
+// kv head of one block: (64, D/64, 1, bs), 128-byte swizzled in shared memory.
+int make_pool_map(CUtensorMap *map, const void *pool, int num_blocks, int bs, int hkv, int d) {
+    auto fn = encode_fn();
+    if (!fn) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(d / 64), static_cast<cuuint64_t>(hkv),
+                          static_cast<cuuint64_t>(num_blocks) * bs};
+    cuuint64_t strides[3] = {64 * 2, static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(hkv) * d * 2};
+    cuuint32_t box[4] = {64, static_cast<cuuint32_t>(d / 64), 1, static_cast<cuuint32_t>(bs)};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(pool), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return PKV_OK;
+}
+
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    static std::mutex mu;
+    static std::vector<int> cache;
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev >= static_cast<int>(cache.size())) cache.resize(dev + 1, 0);
+    if (cache[dev] == 0 && cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
+        cache[dev] = n;
+    return cache[dev];
+}
+
+int resolve_partition(int partition_tokens, int block_size) {
+    return partition_tokens > 0 ? partition_tokens : pkv::kDefaultPartitionTokens;
+}
+
+int64_t n_split_of(int max_blocks_per_seq, int block_size, int partition_tokens) {
+    const int64_t cap = static_cast<int64_t>(max_blocks_per_seq) * block_size;
+    return (cap + partition_tokens - 1) / partition_tokens;
+}
+
+int default_stages(int head_dim, int block_size) {
+    const int stage_bytes = 2 * block_size * head_dim * 2;
+    int ns = (48 * 1024) / stage_bytes;
+    return ns < 4 ? 4 : ns > 12 ? 12 : ns;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *pkv_last_error(void) { return g_err; }
+
+const char *pkv_version(void) { return "pagedkv 0.1 (sm_100a)"; }
+
+int pkv_decode_workspace_bytes(int num_seqs, int num_q_heads, int head_dim, int max_blocks_per_seq, int block_size,
+                               int partition_tokens, size_t *bytes) {
+    if (!bytes) return fail(PKV_ERR_INVALID_ARGUMENT, "bytes is NULL");
+    if (num_seqs < 0 || num_q_heads <= 0 || head_dim <= 0 || max_blocks_per_seq <= 0 || block_size <= 0 ||
+        partition_tokens < 0)
+        return fail(PKV_ERR_INVALID_ARGUMENT, "sizes must be positive (num_seqs >= 0, partition_tokens >= 0)");
+    const int P = resolve_partition(partition_tokens, block_size);
+    if (P % block_size != 0)
+        return fail(PKV_ERR_INVALID_ARGUMENT, "partition_tokens %d is not a multiple of block_size %d", P, block_size);
+    const int64_t ns = n_split_of(max_blocks_per_seq, block_size, P);
+    const int64_t rows = static_cast<int64_t>(num_seqs) * num_q_heads;
+    int64_t total = pkv::kWorkspaceHeaderBytes;
+    if (ns > 1) {
+        total += rows * ns * head_dim * 4;  // fp32 partial outputs
+        total += (rows * ns * 4 + 255) / 256 * 256;  // fp32 log2-sum-exp
+    }
+    *bytes = static_cast<size_t>(total);
+    return ok();
+}
+
+int paged_attn_decode_ex(void *out, const void *q, const void *k_cache, const void *v_cache,
+                         const int32_t *block_tables, const int32_t *context_lens, int num_seqs, int num_q_heads,
+                         int num_kv_heads, int head_dim, int block_size, float scale, int max_blocks_per_seq,
+                         int num_blocks, void *workspace, size_t workspace_bytes, const pkv_decode_options *opts,
+                         void *stream) {
+    if (num_seqs < 0) return fail(PKV_ERR_INVALID_ARGUMENT, "num_seqs < 0");
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !workspace)
+        return fail(PKV_ERR_INVALID_ARGUMENT, "a required pointer is NULL");
+    if (num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || max_blocks_per_seq <= 0 ||
+        num_blocks <= 0)
+        return fail(PKV_ERR_INVALID_ARGUMENT, "head counts, head_dim, block_size, max_blocks_per_seq and "
+                                              "num_blocks must be positive");
+    if (num_q_heads % num_kv_heads != 0)
+        return fail(PKV_ERR_INVALID_ARGUMENT, "num_q_heads %d is not a multiple of num_kv_heads %d", num_q_heads,
+                    num_kv_heads);
+    if (!std::isfinite(scale)) return fail(PKV_ERR_INVALID_ARGUMENT, "scale is not finite");
+    const int group = num_q_heads / num_kv_heads;
+    if (head_dim != 64 && head_dim != 128)
+        return fail(PKV_ERR_UNSUPPORTED, "head_dim %d not supported (64 or 128)", head_dim);
+    if (block_size != 16 && block_size != 32)
+        return fail(PKV_ERR_UNSUPPORTED, "block_size %d not supported (16 or 32)", block_size);
+    if (group > PKV_MAX_GROUP)
+        return fail(PKV_ERR_UNSUPPORTED, "num_q_heads / num_kv_heads = %d exceeds %d", group, PKV_MAX_GROUP);
+    if (static_cast<int64_t>(num_blocks) * block_size > 0x7fffffff ||
+        static_cast<int64_t>(max_blocks_per_seq) * block_size > 0x7fffffff)
+        return fail(PKV_ERR_INVALID_ARGUMENT, "pool or table too large: blocks * block_size must be < 2^31");
+    if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(workspace, 256))
+        return fail(PKV_ERR_INVALID_ARGUMENT,
+                    "out, q, k_cache and v_cache must be 16-byte aligned and workspace 256-byte aligned");
+    pkv_decode_options o = {0, 0, 0, 0};
+    if (opts) o = *opts;
+    if (o.partition_tokens < 0 || o.num_stages < 0 || o.ctas_per_sm < 0 || o.math < 0 || o.math > 2)
+        return fail(PKV_ERR_INVALID_ARGUMENT, "negative or unknown option");
+    const int P = resolve_partition(o.partition_tokens, block_size);
+    if (P % block_size != 0)
+        return fail(PKV_ERR_INVALID_ARGUMENT, "partition_tokens %d is not a multiple of block_size %d", P, block_size);
+    const int ns = o.num_stages ? o.num_stages : default_stages(head_dim, block_size);
+    if (ns < 2 || ns > pkv::kMaxStages)
+        return fail(PKV_ERR_INVALID_ARGUMENT, "num_stages %d outside [2, %d]", ns, pkv::kMaxStages);
+    const int math = o.math ? o.math : pkv::kMathCudaCore;
+    const int gp = group_pad(group);
+    if (!pkv::decode_variant_exists(head_dim, block_size, gp, math))
+        return fail(PKV_ERR_UNSUPPORTED, "no kernel for head_dim %d, block_size %d, group %d, math %d", head_dim,
+                    block_size, group, math);
+    size_t need = 0;
+    int rc = pkv_decode_workspace_bytes(num_seqs, num_q_heads, head_dim, max_blocks_per_seq, block_size, P, &need);
+    if (rc != PKV_OK) return rc;
+    if (workspace_bytes < need)
+        return fail(PKV_ERR_INVALID_ARGUMENT, "workspace_bytes %zu < required %zu", workspace_bytes, need);
+    if (num_seqs == 0) return ok();
+
+    CUtensorMap tm_k, tm_v;
+    if ((rc = make_pool_map(&tm_k, k_cache, num_blocks, block_size, num_kv_heads, head_dim)) != PKV_OK) return rc;
+    if ((rc = make_pool_map(&tm_v, v_cache, num_blocks, block_size, num_kv_heads, head_dim)) != PKV_OK) return rc;
+
+    const int64_t n_split = n_split_of(max_blocks_per_seq, block_size, P);
+    const int64_t rows = static_cast<int64_t>(num_seqs) * num_q_heads;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    float *o_part = reinterpret_cast<float *>(ws + pkv::kWorkspaceHeaderBytes);
+    float *lse_part = o_part + rows * n_split * head_dim;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int sms = sm_count();
+    if (sms <= 0) return fail(PKV_ERR_CUDA, "no CUDA device");
+
+    // Sequences go in launches of at most kMaxSeqsPerLaunch (their prefix sums
+    // live in shared memory); the workspace rows follow the sequences.
+    for (int s0 = 0; s0 < num_seqs; s0 += pkv::kMaxSeqsPerLaunch) {
+        const int sc = num_seqs - s0 < pkv::kMaxSeqsPerLaunch ? num_seqs - s0 : pkv::kMaxSeqsPerLaunch;
+        const size_t smem = pkv::decode_smem_bytes(head_dim, block_size, gp, math, ns, sc);
+        int per_sm = 0;
+        cudaError_t e = pkv::decode_prepare(head_dim, block_size, gp, math, smem, &per_sm);
+        if (e != cudaSuccess) return cuda_fail(e, "decode kernel setup");
+        if (per_sm <= 0) return fail(PKV_ERR_INVALID_ARGUMENT, "shared memory %zu bytes per CTA does not fit", smem);
+        if (o.ctas_per_sm > 0 && o.ctas_per_sm < per_sm) per_sm = o.ctas_per_sm;
+        pkv::DecodeArgs a;
+        a.out = static_cast<__nv_bfloat16 *>(out) + static_cast<size_t>(s0) * num_q_heads * head_dim;
+        a.q = static_cast<const __nv_bfloat16 *>(q) + static_cast<size_t>(s0) * num_q_heads * head_dim;
+        a.block_tables = block_tables + static_cast<size_t>(s0) * max_blocks_per_seq;
+        a.context_lens = context_lens + s0;
+        a.o_part = o_part + static_cast<size_t>(s0) * num_q_heads * n_split * head_dim;
+        a.lse_part = lse_part + static_cast<size_t>(s0) * num_q_heads * n_split;
+        a.status = reinterpret_cast<int32_t *>(ws);
+        a.num_seqs = sc;
+        a.num_q_heads = num_q_heads;
+        a.num_kv_heads = num_kv_heads;
+        a.group = group;
+        a.max_blocks_per_seq = max_blocks_per_seq;
+        a.num_blocks = num_blocks;
+        a.partition_blocks = P / block_size;
+        a.n_split = static_cast<int>(n_split);
+        a.num_stages = ns;
+        a.scale_log2 = scale * 1.4426950408889634f;
+        const int64_t items = static_cast<int64_t>(sc) * n_split * num_kv_heads;
+        const int64_t cap = static_cast<int64_t>(sms) * per_sm;
+        const int grid = static_cast<int>(items < cap ? items : cap);
+        e = pkv::decode_launch(head_dim, block_size, gp, math, tm_k, tm_v, a, grid, smem, st);
+        if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
+        if (n_split > 1) {
+            e = pkv::lse_merge_launch(head_dim, block_size, a, st);
+            if (e != cudaSuccess) return cuda_fail(e, "lse merge launch");
+        }
+    }
+    return ok();
+}
+
+int paged_attn_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
+                      const int32_t *block_tables, const int32_t *context_lens, int num_seqs, int num_q_heads,
+                      int num_kv_heads, int head_dim, int block_size, float scale, int max_blocks_per_seq,
+                      int num_blocks, void *workspace, size_t workspace_bytes, void *stream) {
+    return paged_attn_decode_ex(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs, num_q_heads,
+                                num_kv_heads, head_dim, block_size, scale, max_blocks_per_seq, num_blocks, workspace,
+                                workspace_bytes, nullptr, stream);
+}
+
+int kv_cache_append(const void *k, const void *v, void *k_cache, void *v_cache, const int64_t *slot_mapping,
+                    int num_tokens, int num_kv_heads, int head_dim, int block_size, int num_blocks, int32_t *d_status,
+                    void *stream) {
+    if (num_tokens < 0) return fail(PKV_ERR_INVALID_ARGUMENT, "num_tokens < 0");
+    if (!k || !v || !k_cache || !v_cache || !slot_mapping)
+        return fail(PKV_ERR_INVALID_ARGUMENT, "a required pointer is NULL");
+    if (num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0)
+        return fail(PKV_ERR_INVALID_ARGUMENT, "num_kv_heads, head_dim, block_size and num_blocks must be positive");
+    if (head_dim % 8 != 0) return fail(PKV_ERR_UNSUPPORTED, "head_dim %d is not a multiple of 8", head_dim);
+    if (!aligned(k, 16) || !aligned(v, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16))
+        return fail(PKV_ERR_INVALID_ARGUMENT, "k, v, k_cache and v_cache must be 16-byte aligned");
+    if (d_status && !aligned(d_status, 4)) return fail(PKV_ERR_INVALID_ARGUMENT, "d_status misaligned");
+    if (num_tokens == 0) return ok();
+    cudaError_t e = pkv::append_launch(k, v, k_cache, v_cache, slot_mapping, num_tokens, num_kv_heads, head_dim,
+                                       block_size, num_blocks, d_status, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "append launch");
+    return ok();
+}
+
+int pkv_validate(const int32_t *block_tables, const int32_t *context_lens, int num_seqs, int max_blocks_per_seq,
+                 int block_size, int num_blocks, int32_t *d_status, void *stream) {
+    if (num_seqs < 0) return fail(PKV_ERR_INVALID_ARGUMENT, "num_seqs < 0");
+    if (!block_tables || !context_lens || !d_status) return fail(PKV_ERR_INVALID_ARGUMENT, "a pointer is NULL");
+    if (max_blocks_per_seq <= 0 || block_size <= 0 || num_blocks <= 0)
+        return fail(PKV_ERR_INVALID_ARGUMENT, "sizes must be positive");
+    if (num_seqs == 0) return ok();
+    cudaError_t e = pkv::validate_launch(block_tables, context_lens, num_seqs, max_blocks_per_seq, block_size,
+                                         num_blocks, d_status, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "validate launch");
+    return ok();
+}
+
+int pkv_read_status(int32_t *d_status, int32_t *status, int clear, void *stream) {
+    if (!d_status || !status) return fail(PKV_ERR_INVALID_ARGUMENT, "a pointer is NULL");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(status, d_status, sizeof(int32_t), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess && clear) e = cudaMemsetAsync(d_status, 0, sizeof(int32_t), st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "status read");
+    return ok();
+}
+
+int pkv_selftest_bounded_wait(int32_t *d_status, void *stream) {
+    if (!d_status) return fail(PKV_ERR_INVALID_ARGUMENT, "d_status is NULL");
+    cudaError_t e = pkv::selftest_bounded_wait_launch(d_status, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
+    return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,72 @@
+// decode_common.cuh -- launch-shape constants and the shared-memory layout of the
+// paged decode kernel, used by both the kernel and its host launcher.
+#pragma once
+
+#include <stdint.h>
+
+namespace pkv {
+
+constexpr int kConsumerWarps = 4;                     // warps doing the attention math
+constexpr int kDecodeThreads = 32 * (kConsumerWarps + 1);  // + one TMA producer warp
+constexpr int kMaxStages = 16;                        // depth limit of the KV-block ring
+constexpr int kMaxSeqsPerLaunch = 8192;               // prefix-sum table kept in shared memory
+constexpr int kDefaultPartitionTokens = 512;
+constexpr int kWorkspaceHeaderBytes = 256;
+
+struct DecodeArgs {
+    void *out;                   // bf16 [S][Hq][D]
+    const void *q;               // bf16 [S][Hq][D]
+    const int32_t *block_tables; // [S][MB]
+    const int32_t *context_lens; // [S]
+    float *o_part;               // fp32 [S][Hq][n_split][D]
+    float *lse_part;             // fp32 [S][Hq][n_split], log2 domain
+    int32_t *status;             // device status word
+    int num_seqs;
+    int num_q_heads;
+    int num_kv_heads;
+    int group;                   // Hq / Hkv
+    int max_blocks_per_seq;
+    int num_blocks;
+    int partition_blocks;        // partition_tokens / block_size
+    int n_split;                 // ceil(MB * bs / partition_tokens)
+    int num_stages;
+    float scale_log2;            // scale * log2(e): logits are kept in base 2
+};
+
+struct DecodeLayout {
+    uint32_t stages, qbuf, pscr, merge_acc, merge_m, merge_l, bars, flags, prefix, total;
+};
+
+__host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
+
+// Byte offsets from a 1024-byte aligned base. `total` includes 1024 bytes of
+// slack for aligning the dynamic shared-memory base.
+__host__ __device__ inline DecodeLayout decode_layout(int D, int BS, int GP, int num_stages, int num_seqs) {
+    DecodeLayout L;
+    uint32_t off = 0;
+    const uint32_t tile = static_cast<uint32_t>(BS * D * 2);
+    L.stages = off;
+    off += static_cast<uint32_t>(num_stages) * 2u * tile;          // [stage][K tile, V tile]
+    L.qbuf = off;
+    off += 2u * GP * D * 2;                                         // two query slots [GP][D] bf16
+    off = align_up(off, 16);
+    L.pscr = off;
+    off += kConsumerWarps * BS * GP * 8;                            // per warp float2 [BS][GP]
+    L.merge_acc = off;
+    off += kConsumerWarps * GP * D * 4;                             // per warp fp32 [GP][D]
+    L.merge_m = off;
+    off += kConsumerWarps * GP * 4;
+    L.merge_l = off;
+    off += kConsumerWarps * GP * 4;
+    off = align_up(off, 8);
+    L.bars = off;
+    off += (2 * kMaxStages + 4) * 8;                                // full, empty, qfull[2], qempty[2]
+    L.flags = off;
+    off += (kMaxStages + 8) * 4;                                    // stage_bad, abort, scan scratch
+    L.prefix = off;
+    off += static_cast<uint32_t>(num_seqs + 1) * 4;
+    L.total = align_up(off, 16) + 1024;
+    return L;
+}
+
+}  // namespace pkv

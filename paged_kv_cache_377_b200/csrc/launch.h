@@ -1,0 +1,44 @@
+// launch.h -- host-side entry points of the kernels (internal to libpagedkv.so).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "decode_common.cuh"
+
+namespace pkv {
+
+enum DecodeMath { kMathCudaCore = 1, kMathTensorCore = 2 };
+
+// True when the (head_dim, block_size, padded group, math) combination is compiled in.
+bool decode_variant_exists(int head_dim, int block_size, int group_pad, int math);
+
+// Shared-memory bytes per CTA of a decode variant.
+size_t decode_smem_bytes(int head_dim, int block_size, int group_pad, int math, int num_stages, int num_seqs);
+
+// Sets the variant's dynamic shared-memory limit (once per device) and returns
+// how many CTAs of it fit on one SM.
+cudaError_t decode_prepare(int head_dim, int block_size, int group_pad, int math, size_t smem_bytes,
+                           int *ctas_per_sm);
+
+cudaError_t decode_launch(int head_dim, int block_size, int group_pad, int math, const CUtensorMap &tm_k,
+                          const CUtensorMap &tm_v, const DecodeArgs &args, int grid, size_t smem_bytes,
+                          cudaStream_t stream);
+
+// Cross-partition log-sum-exp merge of the split partial results into `out`.
+cudaError_t lse_merge_launch(int head_dim, int block_size, const DecodeArgs &args, cudaStream_t stream);
+
+cudaError_t append_launch(const void *k, const void *v, void *k_cache, void *v_cache, const int64_t *slot_mapping,
+                          int num_tokens, int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                          int32_t *status, cudaStream_t stream);
+
+cudaError_t validate_launch(const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
+                            int max_blocks_per_seq, int block_size, int num_blocks, int32_t *status,
+                            cudaStream_t stream);
+
+// Launches a kernel whose bounded wait must give up (see selftest.cu).
+cudaError_t selftest_bounded_wait_launch(int32_t *status, cudaStream_t stream);
+
+}  // namespace pkv

@@ -1,0 +1,121 @@
+"""The C-ABI library on a host without a GPU: it loads, exports every symbol the
+header declares, and rejects bad arguments before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import paged_kv_cache_377_b200 as pkv
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "pagedkv.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(\w+)\s*\(", text, flags=re.M)) - {"defined"})
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    lib = pkv.library()
+    names = declared_functions()
+    assert {"paged_attn_decode", "kv_cache_append", "pkv_decode_workspace_bytes"} <= set(names)
+    for name in names:
+        assert hasattr(lib, name), f"{name} declared in pagedkv.h but not exported"
+    assert lib.pkv_version().startswith(b"pagedkv")
+
+
+def _ws(S, Hq, D, MB, bs, P=0):
+    return pkv.workspace_bytes(S, Hq, D, MB, bs, P)
+
+
+def test_workspace_size():
+    assert _ws(4, 2, 64, 3, 16) == 256                        # one split: header only
+    n_split = 8                                                # 256 blocks * 16 / 512
+    rows = 256 * 32
+    assert _ws(256, 32, 128, 256, 16) == 256 + rows * n_split * 128 * 4 + rows * n_split * 4
+    assert _ws(256, 32, 128, 256, 16, P=256) > _ws(256, 32, 128, 256, 16)
+    with pytest.raises(pkv.PagedKVError, match="multiple of block_size"):
+        _ws(4, 2, 64, 3, 16, P=24)
+
+
+P = ctypes.c_void_p(4096)  # a non-null, aligned address: argument checks never dereference it
+
+
+def _decode(**kw):
+    args = dict(out=P, q=P, k=P, v=P, bt=P, cl=P, S=4, Hq=2, Hkv=1, D=64, bs=16, scale=0.125, MB=3, NB=16,
+                ws=P, wsb=1 << 20)
+    args.update(kw)
+    lib = pkv.library()
+    rc = lib.paged_attn_decode(args["out"], args["q"], args["k"], args["v"], args["bt"], args["cl"], args["S"],
+                               args["Hq"], args["Hkv"], args["D"], args["bs"], args["scale"], args["MB"],
+                               args["NB"], args["ws"], args["wsb"], None)
+    return rc, lib.pkv_last_error().decode()
+
+
+@pytest.mark.parametrize("kw,code,msg", [
+    (dict(q=None), -1, "NULL"),
+    (dict(ws=None), -1, "NULL"),
+    (dict(S=-1), -1, "num_seqs"),
+    (dict(Hq=3, Hkv=2), -1, "multiple"),
+    (dict(D=96), -2, "head_dim"),
+    (dict(bs=8), -2, "block_size"),
+    (dict(Hq=16, Hkv=1), -2, "exceeds"),
+    (dict(scale=float("inf")), -1, "scale"),
+    (dict(q=ctypes.c_void_p(4098)), -1, "aligned"),
+    (dict(wsb=16), -1, "workspace_bytes"),
+    (dict(NB=1 << 28), -1, "2^31"),
+])
+def test_decode_rejects_bad_arguments_without_touching_the_gpu(kw, code, msg):
+    rc, err = _decode(**kw)
+    assert rc == code and msg in err, (rc, err)
+
+
+def test_decode_of_empty_batch_is_a_no_op():
+    rc, err = _decode(S=0)
+    assert rc == 0, err
+
+
+def test_append_rejects_bad_arguments():
+    lib = pkv.library()
+    rc = lib.kv_cache_append(P, P, P, P, P, 4, 1, 60, 16, 16, None, None)
+    assert rc == -2 and "multiple of 8" in lib.pkv_last_error().decode()
+    rc = lib.kv_cache_append(P, None, P, P, P, 4, 1, 64, 16, 16, None, None)
+    assert rc == -1
+    rc = lib.kv_cache_append(P, P, P, P, P, 0, 1, 64, 16, 16, None, None)
+    assert rc == 0
+
+
+def test_options_are_checked():
+    lib = pkv.library()
+    opts = pkv._binding._Options(24, 0, 0, 0)
+    rc = lib.paged_attn_decode_ex(P, P, P, P, P, P, 4, 2, 1, 64, 16, 0.125, 3, 16, P, 1 << 20,
+                                  ctypes.byref(opts), None)
+    assert rc == -1 and "partition_tokens" in lib.pkv_last_error().decode()
+    opts = pkv._binding._Options(0, 40, 0, 0)
+    rc = lib.paged_attn_decode_ex(P, P, P, P, P, P, 4, 2, 1, 64, 16, 0.125, 3, 16, P, 1 << 20,
+                                  ctypes.byref(opts), None)
+    assert rc == -1 and "num_stages" in lib.pkv_last_error().decode()
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    q = torch.zeros(1, 2, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        pkv.paged_attn_decode(q, q, q[None], q[None], torch.zeros(1, 1, dtype=torch.int32),
+                              torch.zeros(1, dtype=torch.int32), 0.1, torch.zeros(256, dtype=torch.uint8))
+
+
+def test_missing_library_fails_loudly(monkeypatch):
+    """No CPU fallback: when the library can be neither found nor built, calls raise."""
+    from paged_kv_cache_377_b200 import _binding
+
+    def no_build(*a, **k):
+        raise RuntimeError("nvcc not found")
+
+    monkeypatch.setattr(_binding, "_lib", None)
+    monkeypatch.setattr(_binding._build, "is_stale", lambda: True)
+    monkeypatch.setattr(_binding._build, "build", no_build)
+    with pytest.raises(RuntimeError, match="nvcc"):
+        pkv.workspace_bytes(1, 1, 64, 1, 16)
