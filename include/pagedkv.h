@@ -67,8 +67,9 @@ extern "C" {
  *                     default 512. Sequences longer than this are split and
  *                     their partial results merged with a log-sum-exp
  *                     reduction kernel.
- *   num_stages        depth of the shared-memory ring of KV blocks in flight per
- *                     CTA (2..16); default chosen from the block bytes.
+ *   num_stages        shared-memory stages (one KV block each) per consumer warp
+ *                     (1..4; a CTA has 4 consumer warps); default: about 64 KB
+ *                     of KV blocks in flight per CTA.
  *   ctas_per_sm       resident CTAs per SM of the persistent grid; default: the
  *                     occupancy limit.
  *   math              0 = default, 1 = fp32 CUDA cores, 2 = bf16 tensor cores

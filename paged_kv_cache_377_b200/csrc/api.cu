@@ -97,10 +97,11 @@ int64_t n_split_of(int max_blocks_per_seq, int block_size, int partition_tokens)
     return (cap + partition_tokens - 1) / partition_tokens;
 }
 
+// Stages per consumer warp: about 64 KB of KV blocks in flight per CTA.
 int default_stages(int head_dim, int block_size) {
     const int stage_bytes = 2 * block_size * head_dim * 2;
-    int ns = (48 * 1024) / stage_bytes;
-    return ns < 4 ? 4 : ns > 12 ? 12 : ns;
+    int r = (64 * 1024) / (pkv::kConsumerWarps * stage_bytes);
+    return r < 1 ? 1 : r > pkv::kMaxStagesPerWarp ? pkv::kMaxStagesPerWarp : r;
 }
 
 }  // namespace
@@ -169,8 +170,8 @@ int paged_attn_decode_ex(void *out, const void *q, const void *k_cache, const vo
     if (P % block_size != 0)
         return fail(PKV_ERR_INVALID_ARGUMENT, "partition_tokens %d is not a multiple of block_size %d", P, block_size);
     const int ns = o.num_stages ? o.num_stages : default_stages(head_dim, block_size);
-    if (ns < 2 || ns > pkv::kMaxStages)
-        return fail(PKV_ERR_INVALID_ARGUMENT, "num_stages %d outside [2, %d]", ns, pkv::kMaxStages);
+    if (ns < 1 || ns > pkv::kMaxStagesPerWarp)
+        return fail(PKV_ERR_INVALID_ARGUMENT, "num_stages %d outside [1, %d]", ns, pkv::kMaxStagesPerWarp);
     const int math = o.math ? o.math : pkv::kMathCudaCore;
     const int gp = group_pad(group);
     if (!pkv::decode_variant_exists(head_dim, block_size, gp, math))

@@ -17,8 +17,11 @@
 //     128-byte swizzle), completing on mbarriers. Block-table entries are read
 //     32 at a time by the warp's lanes. The producer runs ahead across item
 //     boundaries, so HBM stays busy while consumers merge.
-//   * Four consumer warps take the item's blocks round-robin; each keeps its
-//     own online-softmax state (running max m, running sum l, fp32 accumulator)
+//   * Four consumer warps take the blocks round-robin (block g of the CTA's
+//     stream goes to warp g % 4) and each warp owns its own ring of R stages,
+//     so every waiter sees every phase of its barriers in order (a parity wait
+//     can never alias a phase two steps ahead). Each warp keeps its own
+//     online-softmax state (running max m, running sum l, fp32 accumulator)
 //     for all G query heads of the GQA group (Milakov & Gimelshein 2018,
 //     "Online normalizer calculation for softmax"). Logits are kept in base 2
 //     (scale * log2 e folded into q).
@@ -213,11 +216,11 @@ template <int D, int BS, int GP>
 __device__ __forceinline__ void producer_warp(const CUtensorMap *tm_k, const CUtensorMap *tm_v, const DecodeArgs &a,
                                               const Smem &sm, const DecodeLayout &ly, int total_items, int lane) {
     constexpr uint32_t kTile = BS * D * 2;
-    const int NS = a.num_stages;
+    const int R = a.num_stages;  // stages per consumer warp
     const int P = a.partition_blocks * BS, cap = a.max_blocks_per_seq * BS;
     const uint32_t qbytes = static_cast<uint32_t>(a.group * D * 2);
-    int stage = 0, qslot = 0;
-    uint32_t phase = 0, qphase = 0;
+    int qslot = 0, gb = 0;
+    uint32_t qphase = 0;
     uint32_t issued = 0, issued_par = 0, q_issued = 0, q_issued_par = 0;  // copies possibly in flight
 
     for (int u = blockIdx.x; u < total_items; u += gridDim.x) {
@@ -242,9 +245,13 @@ __device__ __forceinline__ void producer_warp(const CUtensorMap *tm_k, const CUt
             const int b = bb + lane;
             const int p = (b < it.b1) ? __ldg(row + b) : 0;
             const int n = min(32, it.b1 - bb);
-            for (int i = 0; i < n; ++i) {
+            for (int i = 0; i < n; ++i, ++gb) {
                 const int pi = __shfl_sync(0xffffffffu, p, i);
                 if (lane == 0) {
+                    // block gb belongs to consumer warp gb % 4, slot (gb / 4) % R of its ring
+                    const int k = gb >> 2;
+                    const int stage = (gb & 3) + kConsumerWarps * (k % R);
+                    const uint32_t phase = static_cast<uint32_t>(k / R) & 1u;
                     if (mbar_wait_bounded(&sm.empty[stage], phase ^ 1u, sm.abort_flag, a.status) &&
                         !*sm.abort_flag) {
                         // every earlier copy into this stage has been consumed, hence landed
@@ -264,16 +271,12 @@ __device__ __forceinline__ void producer_warp(const CUtensorMap *tm_k, const CUt
                         }
                     }
                 }
-                if (++stage == NS) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
             }
         }
     }
     // Leave no copy in flight into shared memory when the CTA exits.
     if (lane == 0) {
-        for (int st = 0; st < NS; ++st)
+        for (int st = 0; st < kConsumerWarps * R; ++st)
             if ((issued >> st) & 1u) mbar_wait_drain(&sm.full[st], (issued_par >> st) & 1u, a.status);
         for (int qs = 0; qs < 2; ++qs)
             if ((q_issued >> qs) & 1u) mbar_wait_drain(&sm.qfull[qs], (q_issued_par >> qs) & 1u, a.status);
@@ -285,7 +288,7 @@ __device__ __forceinline__ void consumer_warps(const DecodeArgs &a, const Smem &
                                                int total_items, int warp, int lane) {
     constexpr int LPT = D / 8;
     constexpr uint32_t kTile = BS * D * 2;
-    const int NS = a.num_stages;
+    const int R = a.num_stages;  // this warp's ring: stages warp, warp + 4, ..., warp + 4 (R - 1)
     const int P = a.partition_blocks * BS, cap = a.max_blocks_per_seq * BS;
     const int tg = lane / LPT, ch = lane % LPT;
     const int g_own = g_own_of<GP, LPT>(lane);
@@ -296,8 +299,8 @@ __device__ __forceinline__ void consumer_warps(const DecodeArgs &a, const Smem &
     float *merge_m = reinterpret_cast<float *>(sm.base + ly.merge_m);
     float *merge_l = reinterpret_cast<float *>(sm.base + ly.merge_l);
     const int ctid = warp * 32 + lane;
-    int qslot = 0, gb_base = 0;
-    uint32_t qphase = 0;
+    int qslot = 0, gb_base = 0, ring = 0;
+    uint32_t qphase = 0, rphase = 0;
 
     for (int u = blockIdx.x; u < total_items; u += gridDim.x) {
         const Item it = decode_item<BS>(u, sm.prefix, a, P, cap);
@@ -340,10 +343,15 @@ __device__ __forceinline__ void consumer_warps(const DecodeArgs &a, const Smem &
             for (int k = 0; k < 4; ++k) acc[g][k] = make_float2(0.f, 0.f);
         }
 
-        for (int i = warp; i < nblk; i += kConsumerWarps) {
-            const int gb = gb_base + i;
-            const int stage = gb % NS;
-            const uint32_t par = static_cast<uint32_t>(gb / NS) & 1u;
+        // this warp's blocks of the item: item-local i with (gb_base + i) % 4 == warp
+        for (int i = (warp - gb_base % kConsumerWarps + kConsumerWarps) % kConsumerWarps; i < nblk;
+             i += kConsumerWarps) {
+            const int stage = warp + kConsumerWarps * ring;
+            const uint32_t par = rphase;
+            if (++ring == R) {
+                ring = 0;
+                rphase ^= 1u;
+            }
             mbar_wait_bounded(&sm.full[stage], par, sm.abort_flag, a.status);
             if (!sm.stage_bad[stage] && !*sm.abort_flag) {
                 const int valid = min(BS, it.tok1 - (it.b0 + i) * BS);
@@ -424,7 +432,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
     static_assert(BS == 16 || BS == 32, "block_size");
     static_assert(GP == 1 || GP == 2 || GP == 4 || GP == 8, "group");
     extern __shared__ uint8_t smem_raw[];
-    const DecodeLayout ly = decode_layout(D, BS, GP, a.num_stages, a.num_seqs);
+    const DecodeLayout ly = decode_layout(D, BS, GP, kConsumerWarps * a.num_stages, a.num_seqs);
     Smem sm;
     sm.base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     sm.full = reinterpret_cast<uint64_t *>(sm.base + ly.bars);
@@ -438,7 +446,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     if (tid == 0) {
-        for (int i = 0; i < a.num_stages; ++i) {
+        for (int i = 0; i < kConsumerWarps * a.num_stages; ++i) {
             mbar_init(&sm.full[i], 1);
             mbar_init(&sm.empty[i], 1);
             sm.stage_bad[i] = 0;
@@ -557,7 +565,7 @@ bool decode_variant_exists(int head_dim, int block_size, int group_pad, int math
 
 size_t decode_smem_bytes(int head_dim, int block_size, int group_pad, int math, int num_stages, int num_seqs) {
     (void)math;
-    return decode_layout(head_dim, block_size, group_pad, num_stages, num_seqs).total;
+    return decode_layout(head_dim, block_size, group_pad, kConsumerWarps * num_stages, num_seqs).total;
 }
 
 cudaError_t decode_prepare(int head_dim, int block_size, int group_pad, int math, size_t smem_bytes,

@@ -8,7 +8,8 @@ namespace pkv {
 
 constexpr int kConsumerWarps = 4;                     // warps doing the attention math
 constexpr int kDecodeThreads = 32 * (kConsumerWarps + 1);  // + one TMA producer warp
-constexpr int kMaxStages = 16;                        // depth limit of the KV-block ring
+constexpr int kMaxStages = 16;                        // KV-block stages per CTA (4 warps x up to 4 each)
+constexpr int kMaxStagesPerWarp = kMaxStages / kConsumerWarps;
 constexpr int kMaxSeqsPerLaunch = 8192;               // prefix-sum table kept in shared memory
 constexpr int kDefaultPartitionTokens = 512;
 constexpr int kWorkspaceHeaderBytes = 256;
@@ -29,7 +30,7 @@ struct DecodeArgs {
     int num_blocks;
     int partition_blocks;        // partition_tokens / block_size
     int n_split;                 // ceil(MB * bs / partition_tokens)
-    int num_stages;
+    int num_stages;              // ring stages per consumer warp (R); the CTA holds 4R
     float scale_log2;            // scale * log2(e): logits are kept in base 2
 };
 

@@ -15,7 +15,7 @@ enum DecodeMath { kMathCudaCore = 1, kMathTensorCore = 2 };
 // True when the (head_dim, block_size, padded group, math) combination is compiled in.
 bool decode_variant_exists(int head_dim, int block_size, int group_pad, int math);
 
-// Shared-memory bytes per CTA of a decode variant.
+// Shared-memory bytes per CTA of a decode variant (num_stages = stages per consumer warp).
 size_t decode_smem_bytes(int head_dim, int block_size, int group_pad, int math, int num_stages, int num_seqs);
 
 // Sets the variant's dynamic shared-memory limit (once per device) and returns

@@ -93,7 +93,7 @@ def test_options_are_checked():
     rc = lib.paged_attn_decode_ex(P, P, P, P, P, P, 4, 2, 1, 64, 16, 0.125, 3, 16, P, 1 << 20,
                                   ctypes.byref(opts), None)
     assert rc == -1 and "partition_tokens" in lib.pkv_last_error().decode()
-    opts = pkv._binding._Options(0, 40, 0, 0)
+    opts = pkv._binding._Options(0, 5, 0, 0)
     rc = lib.paged_attn_decode_ex(P, P, P, P, P, P, 4, 2, 1, 64, 16, 0.125, 3, 16, P, 1 << 20,
                                   ctypes.byref(opts), None)
     assert rc == -1 and "num_stages" in lib.pkv_last_error().decode()

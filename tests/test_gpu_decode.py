@@ -67,7 +67,7 @@ def test_forced_split_sizes(name, partition_tokens):
     assert_close_to_oracle(out.double().numpy(), ref, what=f"{name} P={partition_tokens}")
 
 
-@pytest.mark.parametrize("opts", [dict(num_stages=2), dict(num_stages=16), dict(ctas_per_sm=1),
+@pytest.mark.parametrize("opts", [dict(num_stages=1), dict(num_stages=2), dict(num_stages=4), dict(ctas_per_sm=1),
                                   dict(num_stages=3, ctas_per_sm=2, partition_tokens=128)])
 def test_launch_options(opts):
     b, ref, _, _ = config_case("opt125m")
