@@ -54,6 +54,8 @@ def parse_args(argv=None):
     p.add_argument("--num-stages", type=int, default=0)
     p.add_argument("--ctas-per-sm", type=int, default=0)
     p.add_argument("--math", type=int, default=0)
+    p.add_argument("--seqs", type=int, default=0,
+                   help="keep only the first N sequences of the workload (small cases for ncu captures)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args(argv)
@@ -232,6 +234,8 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(device)
     cfg = workloads.CONFIGS[args.workload]
     batch = workloads.make_batch(args.workload, seed=rank_seed(cfg.seed, rank), device=device, poison=False)
+    if args.seqs:
+        batch = first_sequences(batch, args.seqs)
     step = Step(batch, args, device)
     kv = workloads.kv_bytes(batch)
     ctx_tokens = int(batch.context_lens.sum())
@@ -360,6 +364,14 @@ def run_e2e(step, args, flush, stream, kv, world):
             "d2h_bytes_per_step": d2h, "ms_per_step": round(max_ms / K, 5)}
 
 
+def first_sequences(batch, n):
+    """The batch cut to its first n sequences (the pool is kept as it is)."""
+    return workloads.DecodeBatch(**{
+        **batch.__dict__, "num_seqs": n, "context_lens": batch.context_lens[:n],
+        "block_tables": batch.block_tables[:n], "slot_mapping": batch.slot_mapping[:n], "q": batch.q[:n],
+        "k_new": batch.k_new[:n], "v_new": batch.v_new[:n]})
+
+
 def config_block(args, batch, world):
     cfg = workloads.CONFIGS[args.workload]
     c = {
@@ -378,6 +390,8 @@ def config_block(args, batch, world):
         "l2": "inputs larger than L2, and L2 flushed (memset 2x L2) between timed steps",
         "parallelism": "replicas: one independent batch per GPU" if world > 1 else "single GPU",
     }
+    if args.seqs:
+        c["seqs_kept"] = args.seqs
     for k in ("partition_tokens", "num_stages", "ctas_per_sm", "math"):
         if getattr(args, k):
             c[k] = getattr(args, k)
