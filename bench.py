@@ -55,7 +55,7 @@ def parse_args(argv=None):
     p.add_argument("--ctas-per-sm", type=int, default=0)
     p.add_argument("--math", type=int, default=0)
     p.add_argument("--seqs", type=int, default=0,
-                   help="keep only the first N sequences of the workload (small cases for ncu captures)")
+                   help="build the workload with only its first N context lengths (small cases for ncu)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args(argv)
@@ -233,9 +233,11 @@ def run_ours(args, rank, world, local_rank):
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
     cfg = workloads.CONFIGS[args.workload]
-    batch = workloads.make_batch(args.workload, seed=rank_seed(cfg.seed, rank), device=device, poison=False)
-    if args.seqs:
-        batch = first_sequences(batch, args.seqs)
+    lens = None
+    if args.seqs:  # the workload's recipe cut to its first N lengths (pool sized for those)
+        lens = cfg.lengths(np.random.default_rng(rank_seed(cfg.seed, rank)))[:args.seqs].tolist()
+    batch = workloads.make_batch(args.workload, seed=rank_seed(cfg.seed, rank), device=device, poison=False,
+                                 lens_override=lens)
     step = Step(batch, args, device)
     kv = workloads.kv_bytes(batch)
     ctx_tokens = int(batch.context_lens.sum())
@@ -362,14 +364,6 @@ def run_e2e(step, args, flush, stream, kv, world):
     (sum_kv,), (max_ms,) = aggregate([kv * K], [total_ms])
     return {"value": round(sum_kv / (max_ms / 1e3) / 1e9, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": round(max_ms / K, 5)}
-
-
-def first_sequences(batch, n):
-    """The batch cut to its first n sequences (the pool is kept as it is)."""
-    return workloads.DecodeBatch(**{
-        **batch.__dict__, "num_seqs": n, "context_lens": batch.context_lens[:n],
-        "block_tables": batch.block_tables[:n], "slot_mapping": batch.slot_mapping[:n], "q": batch.q[:n],
-        "k_new": batch.k_new[:n], "v_new": batch.v_new[:n]})
 
 
 def config_block(args, batch, world):
