@@ -132,6 +132,41 @@ int paged_attn_decode_ex(void *out, const void *q, const void *k_cache, const vo
                          void *stream);
 
 /*
+ * paged_attn_decode for callers that cannot allocate device memory. The pages
+ * have no counterpart to this call.
+ *
+ * Who needs it: a caller that owns no device allocator of its own -- for
+ * example an engine that, as the pages describe for vLLM, handed all GPU
+ * memory left after the weights to one preallocated KV pool, or a plugin host
+ * that exposes no allocation hook -- cannot provide the workspace that
+ * paged_attn_decode asks for. This call takes the same inputs and output but
+ * no workspace: its scratch is a static device array of
+ * PKV_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads the
+ * library holds until the process exits. It calls no cudaMalloc, cudaFree or
+ * other allocating routine.
+ *
+ * Limits and rules:
+ *   - Batches whose workspace (pkv_decode_workspace_bytes with the default
+ *     partition) exceeds PKV_NOALLOC_SCRATCH_BYTES are rejected with
+ *     PKV_ERR_INVALID_ARGUMENT and a message giving both sizes.
+ *   - The first call on a device looks up the scratch's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture begins.
+ *   - All calls share the one scratch, which keeps the last call's contents.
+ *     Calls that overlap on the GPU (different streams, no ordering between
+ *     them) race on it and give wrong results: order them.
+ *   - d_status: device int32 or NULL. If given, it is overwritten (not ORed)
+ *     with this call's PKV_STATUS_* bits once the call's kernels finish.
+ * Results are identical to paged_attn_decode with the default options.
+ */
+#define PKV_NOALLOC_SCRATCH_BYTES (64u << 20)
+int paged_attn_decode_noalloc(void *out, const void *q, const void *k_cache, const void *v_cache,
+                              const int32_t *block_tables, const int32_t *context_lens,
+                              int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                              int block_size, float scale, int max_blocks_per_seq, int num_blocks,
+                              int32_t *d_status, void *stream);
+
+/*
  * Slot-mapped cache append: for every token i with slot_mapping[i] >= 0 and
  * every kv head h, copies k[i][h][:] to k_cache[slot / block_size]
  * [slot % block_size][h][:] and v[i][h][:] likewise (runbyai.xyz post 449,

@@ -206,3 +206,38 @@ def selftest_bounded_wait(status: torch.Tensor, stream=None) -> None:
     """Enqueues the kernel whose bounded wait must give up (about one second)."""
     _need(status, "status", torch.int32, 1)
     _check("pkv_selftest_bounded_wait", library().pkv_selftest_bounded_wait(_ptr(status), _stream(stream)))
+
+
+_noalloc_ready = False
+
+
+def paged_attn_decode_noalloc(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                              block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float,
+                              status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """paged_attn_decode without a workspace, for callers that cannot allocate device memory.
+
+    The library's static device scratch (64 MiB per GPU) stands in for the
+    workspace; calls that overlap on the GPU race on it. ``status``: optional
+    int32 device tensor overwritten with the call's status bits.
+    """
+    global _noalloc_ready
+    lib = library()
+    if not _noalloc_ready:
+        P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+        lib.paged_attn_decode_noalloc.restype = I
+        lib.paged_attn_decode_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, I, I, P, P]
+        _noalloc_ready = True
+    _need(q, "q", torch.bfloat16, 3)
+    _need(out, "out", torch.bfloat16, 3)
+    _need(k_cache, "k_cache", torch.bfloat16, 4)
+    _need(v_cache, "v_cache", torch.bfloat16, 4)
+    _need(block_tables, "block_tables", torch.int32, 2)
+    _need(context_lens, "context_lens", torch.int32, 1)
+    if status is not None:
+        _need(status, "status", torch.int32, 1)
+    S, Hq, D = q.shape
+    NB, bs, Hkv, _ = k_cache.shape
+    _check("paged_attn_decode_noalloc", lib.paged_attn_decode_noalloc(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
+        S, Hq, Hkv, D, bs, float(scale), block_tables.shape[1], NB, _ptr(status), _stream(stream)))
+    return out

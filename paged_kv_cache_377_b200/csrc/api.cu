@@ -297,3 +297,70 @@ int pkv_selftest_bounded_wait(int32_t *d_status, void *stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// paged_attn_decode_noalloc: decode for callers that cannot allocate device
+// memory. Its scratch (status word + split partials, the layout of the decode
+// workspace) is this file-scope device array, sized PKV_NOALLOC_SCRATCH_BYTES;
+// every GPU that loads the library holds it until the process exits.
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[PKV_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mu;
+std::vector<void *> g_noalloc_ptr;  // device address of g_noalloc_scratch, per device
+
+// In host code g_noalloc_scratch names a host-side stand-in, not device memory:
+// the kernels get the address cudaGetSymbolAddress returns for the current
+// device, looked up on the first call on that device and cached.
+int noalloc_scratch(void **ptr) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (dev >= static_cast<int>(g_noalloc_ptr.size())) g_noalloc_ptr.resize(dev + 1, nullptr);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the static decode scratch");
+        g_noalloc_ptr[dev] = p;
+    }
+    *ptr = g_noalloc_ptr[dev];
+    return PKV_OK;
+}
+
+}  // namespace
+
+extern "C" int paged_attn_decode_noalloc(void *out, const void *q, const void *k_cache, const void *v_cache,
+                                         const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
+                                         int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                                         float scale, int max_blocks_per_seq, int num_blocks, int32_t *d_status,
+                                         void *stream) {
+    size_t need = 0;
+    int rc = pkv_decode_workspace_bytes(num_seqs, num_q_heads, head_dim, max_blocks_per_seq, block_size, 0, &need);
+    if (rc != PKV_OK) return rc;
+    if (need > PKV_NOALLOC_SCRATCH_BYTES)
+        return fail(PKV_ERR_INVALID_ARGUMENT,
+                    "this batch needs %zu bytes of decode scratch but the static scratch of "
+                    "paged_attn_decode_noalloc holds %u; decode it in smaller batches or use paged_attn_decode "
+                    "with a caller-allocated workspace",
+                    need, static_cast<unsigned>(PKV_NOALLOC_SCRATCH_BYTES));
+    if (d_status && !aligned(d_status, 4)) return fail(PKV_ERR_INVALID_ARGUMENT, "d_status misaligned");
+    void *scratch = nullptr;
+    if ((rc = noalloc_scratch(&scratch)) != PKV_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // The scratch keeps the previous call's contents: zero its status word so
+    // this call reports only its own problems. The partials need no clearing
+    // (every one that is read was written earlier in the same call).
+    cudaError_t e = cudaMemsetAsync(scratch, 0, pkv::kWorkspaceHeaderBytes, st);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the static scratch's status word");
+    rc = paged_attn_decode_ex(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs, num_q_heads,
+                              num_kv_heads, head_dim, block_size, scale, max_blocks_per_seq, num_blocks, scratch,
+                              PKV_NOALLOC_SCRATCH_BYTES, nullptr, stream);
+    if (rc != PKV_OK) return rc;
+    if (d_status) {
+        e = cudaMemcpyAsync(d_status, scratch, sizeof(int32_t), cudaMemcpyDeviceToDevice, st);
+        if (e != cudaSuccess) return cuda_fail(e, "copying the status word");
+    }
+    return ok();
+}

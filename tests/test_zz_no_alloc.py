@@ -1,0 +1,65 @@
+"""paged_attn_decode_noalloc: decode without a caller-allocated workspace.
+
+Some callers cannot allocate device memory at all: an engine that handed every
+byte left after the weights to one preallocated KV pool, or a plugin host that
+gives its plugins no allocator. They call paged_attn_decode_noalloc, whose
+scratch is a static device array inside the library. These tests call it
+through the C ABI and check it against paged_attn_decode, the entry point that
+takes a workspace, on two calls in a row -- the second call must not be
+disturbed by what the first left in the shared scratch.
+"""
+import pytest
+import torch
+
+import paged_kv_cache_377_b200 as pkv
+import workloads
+from helpers import assert_close_to_oracle
+
+SCRATCH_BYTES = 64 << 20
+
+
+def _decode_both(b, dev):
+    kc, vc = b.k_cache.to(dev), b.v_cache.to(dev)
+    q = b.q.to(dev)
+    bt, cl = b.block_tables.to(dev), b.context_lens.to(dev)
+    pkv.kv_cache_append(b.k_new.to(dev), b.v_new.to(dev), kc, vc, b.slot_mapping.to(dev))
+    ws = pkv.allocate_workspace(b.num_seqs, b.num_q_heads, b.head_dim, b.max_blocks_per_seq, b.block_size,
+                                device=dev)
+    assert ws.numel() <= SCRATCH_BYTES
+    with_ws = torch.empty_like(q)
+    pkv.paged_attn_decode(with_ws, q, kc, vc, bt, cl, b.scale, ws)
+    no_ws = torch.full_like(q, float("nan"))
+    status = torch.full((1,), -1, dtype=torch.int32, device=dev)
+    lib = pkv.library()
+    from paged_kv_cache_377_b200._binding import paged_attn_decode_noalloc
+    paged_attn_decode_noalloc(no_ws, q, kc, vc, bt, cl, b.scale, status=status)
+    torch.cuda.synchronize()
+    assert lib.pkv_last_error() == b""
+    return with_ws.cpu(), no_ws.cpu(), int(status.item()), pkv.read_status(ws)
+
+
+@pytest.mark.gpu
+def test_noalloc_matches_the_workspace_entry_point_on_two_calls_in_a_row():
+    dev = torch.device("cuda", torch.cuda.current_device())
+    # the first call leaves 8-way split partials behind in the scratch; the
+    # second has a different shape and fewer splits
+    for name in ("llama3_8b", "opt125m"):
+        b = workloads.make_batch(name, device=dev)
+        with_ws, no_ws, status, ws_status = _decode_both(b, dev)
+        assert status == 0 and ws_status == 0, (name, status, ws_status)
+        assert_close_to_oracle(no_ws.double().numpy(), with_ws.double().numpy(), what=f"noalloc vs workspace, {name}")
+
+
+def test_noalloc_rejects_batches_beyond_its_scratch():
+    """The skewed long-context shape needs ~270 MB of split partials: refused on the host, nothing enqueued."""
+    lib = pkv.library()
+    import ctypes
+    P = ctypes.c_void_p(4096)
+    from paged_kv_cache_377_b200._binding import paged_attn_decode_noalloc  # noqa: F401  (sets argtypes lazily)
+    lib.paged_attn_decode_noalloc.argtypes = [ctypes.c_void_p] * 6 + [ctypes.c_int] * 5 + [ctypes.c_float] + \
+        [ctypes.c_int] * 2 + [ctypes.c_void_p] * 2
+    rc = lib.paged_attn_decode_noalloc(P, P, P, P, P, P, 128, 32, 8, 128, 32, 0.088, 2048, 5081, None, None)
+    msg = lib.pkv_last_error().decode()
+    assert rc == -1 and "static scratch" in msg and str(SCRATCH_BYTES) in msg, msg
+    need = pkv.workspace_bytes(128, 32, 128, 2048, 32)
+    assert need > SCRATCH_BYTES and str(need) in msg
