@@ -59,15 +59,16 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // Tensor map over a pool [num_blocks][bs][Hkv][D] bf16 seen as 4D
-// (64, D/64, Hkv, num_blocks*bs), innermost first; one box = all bs rows of one
-// kv head of one block: (64, D/64, 1, bs), 128-byte swizzled in shared memory.
+// (64, D/64, Hkv, num_blocks*bs), innermost first; one box = one 64-column half
+// of all bs rows of one kv head of one block: (64, 1, 1, bs), 128-byte
+// swizzled in shared memory (a tile is D/64 such [bs][128 B] halves).
 int make_pool_map(CUtensorMap *map, const void *pool, int num_blocks, int bs, int hkv, int d) {
     auto fn = encode_fn();
     if (!fn) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
     cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(d / 64), static_cast<cuuint64_t>(hkv),
                           static_cast<cuuint64_t>(num_blocks) * bs};
     cuuint64_t strides[3] = {64 * 2, static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(hkv) * d * 2};
-    cuuint32_t box[4] = {64, static_cast<cuuint32_t>(d / 64), 1, static_cast<cuuint32_t>(bs)};
+    cuuint32_t box[4] = {64, 1, 1, static_cast<cuuint32_t>(bs)};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(pool), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,

@@ -12,11 +12,11 @@
 //     grid of (SMs x resident CTAs) walks the items with a fixed stride; every
 //     CTA rebuilds the prefix sum of split counts in shared memory, so no
 //     planning kernel and no host/device synchronisation are needed.
-//   * One producer warp streams whole KV blocks of the item's kv head into a
-//     ring of shared-memory stages with TMA (one 4D tile copy per K or V block,
-//     128-byte swizzle), completing on mbarriers. Block-table entries are read
-//     32 at a time by the warp's lanes. The producer runs ahead across item
-//     boundaries, so HBM stays busy while consumers merge.
+//   * One producer warp streams whole KV blocks of the item's kv head into
+//     shared memory with TMA (4D tile copies of 64 columns, 128-byte swizzle),
+//     completing on mbarriers. Block-table entries are read 32 at a time by the
+//     warp's lanes. The producer runs ahead across item boundaries, so HBM
+//     stays busy while consumers merge.
 //   * Four consumer warps take the blocks round-robin (block g of the CTA's
 //     stream goes to warp g % 4) and each warp owns its own ring of R stages,
 //     so every waiter sees every phase of its barriers in order (a parity wait
@@ -24,7 +24,11 @@
 //     online-softmax state (running max m, running sum l, fp32 accumulator)
 //     for all G query heads of the GQA group (Milakov & Gimelshein 2018,
 //     "Online normalizer calculation for softmax"). Logits are kept in base 2
-//     (scale * log2 e folded into q).
+//     (scale * log2 e folded in).
+//   * Two interchangeable math paths per block: CoreMath (fp32 FMA on CUDA
+//     cores, packed f32x2) and MmaMath (bf16 tensor cores, mma.sync m16n8k16
+//     with fp32 accumulation: S^T = K.Q^T with the block's tokens as M and the
+//     G <= 8 query heads as N, then O^T += V^T.P^T).
 //   * At the end of an item the four warp states are merged in shared memory
 //     with the log-sum-exp identity. Unsplit sequences write bf16 output
 //     directly; split ones write fp32 partials + log2-sum-exp, merged by
@@ -70,6 +74,19 @@ __device__ __forceinline__ Item decode_item(int u, const int *prefix, const Deco
     return it;
 }
 
+// Shared address of 16-byte chunk c (0 <= c < D/8) of row t of a K or V tile.
+// A tile holds D/64 column halves of [BS rows][128 bytes], each loaded by one
+// TMA box with SWIZZLE_128B: the chunk index inside a 128-byte row is XORed
+// with the row index mod 8, so 8 consecutive rows at one chunk hit 8 distinct
+// bank groups.
+template <int BS>
+__device__ __forceinline__ uint32_t tile_addr(uint32_t tile, int t, int c) {
+    return tile + static_cast<uint32_t>((c >> 3) * (BS * 128) + t * 128) +
+           (static_cast<uint32_t>((c & 7) ^ (t & 7)) << 4);
+}
+
+// ------------------------------------------------------------------ CUDA-core math
+
 // Reduce N partial sums across the LPT lanes of a token group (xor masks
 // LPT/2 .. 1), halving the values a lane carries at each step: afterwards
 // v[0] holds the full sum for query head g_own (see g_own_of()).
@@ -103,105 +120,370 @@ __device__ __forceinline__ int g_own_of(int lane) {
     return g;
 }
 
-// Shared address of 16-byte chunk `ch` of row t of a TMA tile loaded with
-// SWIZZLE_128B: a row of D bf16 is D/64 lines of 128 bytes, and the chunk
-// index inside a line is XORed with the line index mod 8.
-template <int D>
-__device__ __forceinline__ uint32_t tile_chunk_addr(uint32_t tile, int t, int ch) {
-    const uint32_t line = static_cast<uint32_t>(t * (D / 64) + (ch >> 3));
-    return tile + line * 128u + ((static_cast<uint32_t>(ch & 7) ^ (line & 7u)) << 4);
-}
+// fp32 math on CUDA cores. A token group of LPT = D/8 lanes covers one row
+// (8 dims per lane, one 16-byte chunk); a warp handles 32/LPT tokens per pass.
+template <int D, int BS, int GP_>
+struct CoreMath {
+    static constexpr int GP = GP_;
+    static constexpr int LPT = D / 8, TPP = 32 / LPT, NPASS = BS / TPP, LPG = 32 / GP;
 
-// One KV block on CUDA cores: logits, block-wise online-softmax update, P.V.
-template <int D, int BS, int GP>
-__device__ __forceinline__ void block_cuda_core(uint32_t ktile, uint32_t vtile, int valid, const float2 (&q2)[GP][4],
-                                                float (&m_run)[GP], float &l_run, float2 (&acc)[GP][4],
-                                                float2 *pscr, int tg, int ch, int lane, int g_own, bool writer) {
-    constexpr int LPT = D / 8, TPP = 32 / LPT, NPASS = BS / TPP, LPG = 32 / GP;
+    int lane, tg, ch, g_own;
+    bool writer;
+    float2 *pscr;  // this warp's float2 [BS][GP]: logits, then (p, p)
+    float2 q2[GP][4];
+    float m_run[GP];
+    float l_run;
+    float2 acc[GP][4];
 
-    // logits: the LPT lanes of a token group each hold 8 dims of the row
-#pragma unroll
-    for (int pass = 0; pass < NPASS; ++pass) {
-        const int t = pass * TPP + tg;
-        const uint4 kr = lds128(tile_chunk_addr<D>(ktile, t, ch));
-        const float2 k0 = bf16x2_to_float2(kr.x), k1 = bf16x2_to_float2(kr.y);
-        const float2 k2 = bf16x2_to_float2(kr.z), k3 = bf16x2_to_float2(kr.w);
-        float part[GP];
+    __device__ __forceinline__ void init(int warp, int lane_, uint8_t *base, const DecodeLayout &ly) {
+        lane = lane_;
+        tg = lane / LPT;
+        ch = lane % LPT;
+        g_own = g_own_of<GP, LPT>(lane);
+        writer = (lane % (LPT / GP)) == 0;
+        pscr = reinterpret_cast<float2 *>(base + ly.pscr) + warp * BS * GP;
+    }
+
+    // query rows of the GQA group, pre-scaled into base-2 logits
+    __device__ __forceinline__ void load_q(uint32_t qslot, int group, float scale_log2) {
+        const uint32_t qa = qslot + ch * 16;
+        const float2 sc = make_float2(scale_log2, scale_log2);
 #pragma unroll
         for (int g = 0; g < GP; ++g) {
-            float2 s2 = fmul2(q2[g][0], k0);
-            s2 = ffma2(q2[g][1], k1, s2);
-            s2 = ffma2(q2[g][2], k2, s2);
-            s2 = ffma2(q2[g][3], k3, s2);
-            part[g] = s2.x + s2.y;
-        }
-        transpose_reduce<GP, LPT>(part, lane);
-        // a token past the context is selected away (its row may hold anything)
-        if (writer) pscr[t * GP + g_own].x = (t < valid) ? part[0] : -INFINITY;
-    }
-    __syncwarp();
-
-    // block max per head, new running max, probabilities, running sum
-    const int gs = lane % GP, ts = lane / GP;
-    float mx = -INFINITY;
+            if (g < group) {
+                const uint4 r = lds128(qa + g * D * 2);
+                q2[g][0] = fmul2(bf16x2_to_float2(r.x), sc);
+                q2[g][1] = fmul2(bf16x2_to_float2(r.y), sc);
+                q2[g][2] = fmul2(bf16x2_to_float2(r.z), sc);
+                q2[g][3] = fmul2(bf16x2_to_float2(r.w), sc);
+            } else {
 #pragma unroll
-    for (int t = ts; t < BS; t += LPG) mx = fmaxf(mx, pscr[t * GP + gs].x);
-#pragma unroll
-    for (int o = GP; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    float m_new[GP];
-    bool grew = false;
-    float m_own_old = m_run[0], m_own_new = 0.f;
-#pragma unroll
-    for (int g = 0; g < GP; ++g) {
-        m_new[g] = fmaxf(m_run[g], __shfl_sync(0xffffffffu, mx, g));
-        grew |= (m_new[g] != m_run[g]);
-        if (g == gs) {
-            m_own_old = m_run[g];
-            m_own_new = m_new[g];
-        }
-    }
-    float psum = 0.f;
-#pragma unroll
-    for (int t = ts; t < BS; t += LPG) {
-        const float p = fast_exp2(pscr[t * GP + gs].x - m_own_new);
-        pscr[t * GP + gs] = make_float2(p, p);
-        psum += p;
-    }
-#pragma unroll
-    for (int o = GP; o < 32; o <<= 1) psum += __shfl_xor_sync(0xffffffffu, psum, o);
-    l_run = l_run * fast_exp2(m_own_old - m_own_new) + psum;
-    if (grew) {  // warp-uniform: m_run is replicated in every lane
-#pragma unroll
-        for (int g = 0; g < GP; ++g) {
-            const float al = fast_exp2(m_run[g] - m_new[g]);
-            const float2 a2 = make_float2(al, al);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) acc[g][k] = fmul2(acc[g][k], a2);
-            m_run[g] = m_new[g];
-        }
-    }
-    __syncwarp();
-
-    // P.V: tokens past the context are skipped, never multiplied by p = 0
-#pragma unroll
-    for (int pass = 0; pass < NPASS; ++pass) {
-        const int t = pass * TPP + tg;
-        const uint4 vr = lds128(tile_chunk_addr<D>(vtile, t, ch));
-        if (t < valid) {
-            const float2 v0 = bf16x2_to_float2(vr.x), v1 = bf16x2_to_float2(vr.y);
-            const float2 v2 = bf16x2_to_float2(vr.z), v3 = bf16x2_to_float2(vr.w);
-#pragma unroll
-            for (int g = 0; g < GP; ++g) {
-                const float2 p = pscr[t * GP + g];
-                acc[g][0] = ffma2(p, v0, acc[g][0]);
-                acc[g][1] = ffma2(p, v1, acc[g][1]);
-                acc[g][2] = ffma2(p, v2, acc[g][2]);
-                acc[g][3] = ffma2(p, v3, acc[g][3]);
+                for (int k = 0; k < 4; ++k) q2[g][k] = make_float2(0.f, 0.f);
             }
         }
     }
-    __syncwarp();
+
+    __device__ __forceinline__ void reset() {
+        l_run = 0.f;
+#pragma unroll
+        for (int g = 0; g < GP; ++g) {
+            m_run[g] = -INFINITY;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) acc[g][k] = make_float2(0.f, 0.f);
+        }
+    }
+
+    // One KV block: logits, block-wise online-softmax update, P.V.
+    __device__ __forceinline__ void block(uint32_t ktile, uint32_t vtile, int valid) {
+#pragma unroll
+        for (int pass = 0; pass < NPASS; ++pass) {
+            const int t = pass * TPP + tg;
+            const uint4 kr = lds128(tile_addr<BS>(ktile, t, ch));
+            const float2 k0 = bf16x2_to_float2(kr.x), k1 = bf16x2_to_float2(kr.y);
+            const float2 k2 = bf16x2_to_float2(kr.z), k3 = bf16x2_to_float2(kr.w);
+            float part[GP];
+#pragma unroll
+            for (int g = 0; g < GP; ++g) {
+                float2 s2 = fmul2(q2[g][0], k0);
+                s2 = ffma2(q2[g][1], k1, s2);
+                s2 = ffma2(q2[g][2], k2, s2);
+                s2 = ffma2(q2[g][3], k3, s2);
+                part[g] = s2.x + s2.y;
+            }
+            transpose_reduce<GP, LPT>(part, lane);
+            // a token past the context is selected away (its row may hold anything)
+            if (writer) pscr[t * GP + g_own].x = (t < valid) ? part[0] : -INFINITY;
+        }
+        __syncwarp();
+
+        // block max per head, new running max, probabilities, running sum
+        const int gs = lane % GP, ts = lane / GP;
+        float mx = -INFINITY;
+#pragma unroll
+        for (int t = ts; t < BS; t += LPG) mx = fmaxf(mx, pscr[t * GP + gs].x);
+#pragma unroll
+        for (int o = GP; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        float m_new[GP];
+        bool grew = false;
+        float m_own_old = m_run[0], m_own_new = 0.f;
+#pragma unroll
+        for (int g = 0; g < GP; ++g) {
+            m_new[g] = fmaxf(m_run[g], __shfl_sync(0xffffffffu, mx, g));
+            grew |= (m_new[g] != m_run[g]);
+            if (g == gs) {
+                m_own_old = m_run[g];
+                m_own_new = m_new[g];
+            }
+        }
+        float psum = 0.f;
+#pragma unroll
+        for (int t = ts; t < BS; t += LPG) {
+            const float p = fast_exp2(pscr[t * GP + gs].x - m_own_new);
+            pscr[t * GP + gs] = make_float2(p, p);
+            psum += p;
+        }
+#pragma unroll
+        for (int o = GP; o < 32; o <<= 1) psum += __shfl_xor_sync(0xffffffffu, psum, o);
+        l_run = l_run * fast_exp2(m_own_old - m_own_new) + psum;
+        if (grew) {  // warp-uniform: m_run is replicated in every lane
+#pragma unroll
+            for (int g = 0; g < GP; ++g) {
+                const float al = fast_exp2(m_run[g] - m_new[g]);
+                const float2 a2 = make_float2(al, al);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) acc[g][k] = fmul2(acc[g][k], a2);
+                m_run[g] = m_new[g];
+            }
+        }
+        __syncwarp();
+
+        // P.V: tokens past the context are skipped, never multiplied by p = 0
+#pragma unroll
+        for (int pass = 0; pass < NPASS; ++pass) {
+            const int t = pass * TPP + tg;
+            const uint4 vr = lds128(tile_addr<BS>(vtile, t, ch));
+            if (t < valid) {
+                const float2 v0 = bf16x2_to_float2(vr.x), v1 = bf16x2_to_float2(vr.y);
+                const float2 v2 = bf16x2_to_float2(vr.z), v3 = bf16x2_to_float2(vr.w);
+#pragma unroll
+                for (int g = 0; g < GP; ++g) {
+                    const float2 p = pscr[t * GP + g];
+                    acc[g][0] = ffma2(p, v0, acc[g][0]);
+                    acc[g][1] = ffma2(p, v1, acc[g][1]);
+                    acc[g][2] = ffma2(p, v2, acc[g][2]);
+                    acc[g][3] = ffma2(p, v3, acc[g][3]);
+                }
+            }
+        }
+        __syncwarp();
+    }
+
+    // This warp's (m, l, acc) into the merge area ([warp][GP][D] etc).
+    __device__ __forceinline__ void export_state(float *merge_acc, float *merge_m, float *merge_l, int warp) {
+        // token groups of a warp share m_run: their accumulators just add
+#pragma unroll
+        for (int o = LPT; o < 32; o <<= 1)
+#pragma unroll
+            for (int g = 0; g < GP; ++g)
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    acc[g][k].x += __shfl_xor_sync(0xffffffffu, acc[g][k].x, o);
+                    acc[g][k].y += __shfl_xor_sync(0xffffffffu, acc[g][k].y, o);
+                }
+        if (tg == 0) {
+#pragma unroll
+            for (int g = 0; g < GP; ++g) {
+                float4 *dst = reinterpret_cast<float4 *>(merge_acc + (warp * GP + g) * D + ch * 8);
+                dst[0] = make_float4(acc[g][0].x, acc[g][0].y, acc[g][1].x, acc[g][1].y);
+                dst[1] = make_float4(acc[g][2].x, acc[g][2].y, acc[g][3].x, acc[g][3].y);
+            }
+        }
+        if (lane == 0) {
+#pragma unroll
+            for (int g = 0; g < GP; ++g) merge_m[warp * GP + g] = m_run[g];
+        }
+        if (lane < GP) merge_l[warp * GP + lane] = l_run;
+    }
+};
+
+// ------------------------------------------------------------------ tensor-core math
+
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
 }
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+// d += a (16x16 bf16, row) * b (16x8 bf16, col), fp32 accumulate.
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ void sts16(uint32_t addr, uint16_t v) {
+    asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
+}
+
+// bf16 tensor-core math (mma.sync m16n8k16, fp32 accumulate). Per block:
+//   S^T[t][g] = K[t][:] . q[g][:]   tokens t as M (16 per tile), heads g as N = 8
+//   O^T[d][g] += V[t][d] . P[g][t]  dims d as M (16 per tile), tokens as K
+// Lane l holds S^T/O^T elements of rows l/4 and l/4 + 8 and of heads
+// g0 = 2 (l % 4), g1 = g0 + 1, so the online-softmax state of a lane is the
+// running max and (partial) sum of its two heads.
+template <int D, int BS>
+struct MmaMath {
+    static constexpr int GP = 8;
+    static constexpr int KST = D / 16;  // k-steps of q.K
+    static constexpr int TT = BS / 16;  // token tiles per block
+    static constexpr int DT = D / 16;   // dim tiles of P.V
+
+    int lane;
+    uint32_t pscr;  // this warp's bf16 P[GP][BS] (shared address)
+    float scale_log2;
+    uint32_t qb[KST][2];  // B fragments of q
+    float acc[DT][4];     // O^T fragments
+    float m0, m1, l0, l1;
+
+    __device__ __forceinline__ void init(int warp, int lane_, uint8_t *base, const DecodeLayout &ly) {
+        lane = lane_;
+        pscr = smem_u32(base + ly.pscr) + warp * (GP * BS * 2);
+    }
+
+    // B fragment (k = dim, n = head): two consecutive dims of q[l/4]; heads past the group are 0.
+    __device__ __forceinline__ void load_q(uint32_t qslot, int group, float sl2) {
+        scale_log2 = sl2;
+        const int g = lane >> 2, k2 = (lane & 3) * 2;
+#pragma unroll
+        for (int kk = 0; kk < KST; ++kk) {
+            qb[kk][0] = g < group ? lds32(qslot + (g * D + 16 * kk + k2) * 2) : 0u;
+            qb[kk][1] = g < group ? lds32(qslot + (g * D + 16 * kk + 8 + k2) * 2) : 0u;
+        }
+    }
+
+    __device__ __forceinline__ void reset() {
+        m0 = m1 = -INFINITY;
+        l0 = l1 = 0.f;
+#pragma unroll
+        for (int dt = 0; dt < DT; ++dt)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) acc[dt][k] = 0.f;
+    }
+
+    __device__ __forceinline__ void block(uint32_t ktile, uint32_t vtile, int valid) {
+        const int mi = lane >> 3, r = lane & 7;
+        const int tr = lane >> 2;  // fragment row of this lane
+        // S^T = K . Q^T; ldmatrix x4 gives the A fragment (rows t, cols d) of one k-step
+        float s[TT][4];
+#pragma unroll
+        for (int mt = 0; mt < TT; ++mt) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) s[mt][k] = 0.f;
+#pragma unroll
+            for (int kk = 0; kk < KST; ++kk) {
+                uint32_t a[4];
+                ldsm_x4(a, tile_addr<BS>(ktile, 16 * mt + r + 8 * (mi & 1), 2 * kk + (mi >> 1)));
+                mma_16816(s[mt], a, qb[kk][0], qb[kk][1]);
+            }
+        }
+        // base-2 logits; tokens past the context are selected away (their rows may hold anything)
+        float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+        for (int mt = 0; mt < TT; ++mt) {
+            const int t0 = 16 * mt + tr, t1 = t0 + 8;
+            s[mt][0] = t0 < valid ? s[mt][0] * scale_log2 : -INFINITY;
+            s[mt][1] = t0 < valid ? s[mt][1] * scale_log2 : -INFINITY;
+            s[mt][2] = t1 < valid ? s[mt][2] * scale_log2 : -INFINITY;
+            s[mt][3] = t1 < valid ? s[mt][3] * scale_log2 : -INFINITY;
+            mx0 = fmaxf(mx0, fmaxf(s[mt][0], s[mt][2]));
+            mx1 = fmaxf(mx1, fmaxf(s[mt][1], s[mt][3]));
+        }
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+        }
+        const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+        const float a0 = fast_exp2(m0 - n0), a1 = fast_exp2(m1 - n1);
+        // probabilities, rounded to bf16 for the P.V product; the sums take the
+        // rounded values so numerator and denominator see the same weights
+        const int g0 = 2 * (lane & 3);
+        float ps0 = 0.f, ps1 = 0.f;
+#pragma unroll
+        for (int mt = 0; mt < TT; ++mt) {
+            const int t0 = 16 * mt + tr;
+            const __nv_bfloat16 p0 = __float2bfloat16_rn(fast_exp2(s[mt][0] - n0));
+            const __nv_bfloat16 p1 = __float2bfloat16_rn(fast_exp2(s[mt][1] - n1));
+            const __nv_bfloat16 p2 = __float2bfloat16_rn(fast_exp2(s[mt][2] - n0));
+            const __nv_bfloat16 p3 = __float2bfloat16_rn(fast_exp2(s[mt][3] - n1));
+            ps0 += __bfloat162float(p0) + __bfloat162float(p2);
+            ps1 += __bfloat162float(p1) + __bfloat162float(p3);
+            sts16(pscr + (g0 * BS + t0) * 2, __bfloat16_as_ushort(p0));
+            sts16(pscr + ((g0 + 1) * BS + t0) * 2, __bfloat16_as_ushort(p1));
+            sts16(pscr + (g0 * BS + t0 + 8) * 2, __bfloat16_as_ushort(p2));
+            sts16(pscr + ((g0 + 1) * BS + t0 + 8) * 2, __bfloat16_as_ushort(p3));
+        }
+        l0 = l0 * a0 + ps0;
+        l1 = l1 * a1 + ps1;
+        if (__any_sync(0xffffffffu, n0 != m0 || n1 != m1)) {
+#pragma unroll
+            for (int dt = 0; dt < DT; ++dt) {
+                acc[dt][0] *= a0;
+                acc[dt][1] *= a1;
+                acc[dt][2] *= a0;
+                acc[dt][3] *= a1;
+            }
+        }
+        m0 = n0;
+        m1 = n1;
+        __syncwarp();
+
+        // O^T += V^T . P^T; ldmatrix x4 .trans gives the A fragment (rows d, cols t)
+#pragma unroll
+        for (int ks = 0; ks < TT; ++ks) {
+            const uint32_t pb = pscr + ((lane >> 2) * BS + 16 * ks + 2 * (lane & 3)) * 2;
+            const uint32_t b0 = lds32(pb), b1 = lds32(pb + 16);
+            // V rows past the context may hold NaN: zero them in the fragments
+            uint32_t keep_lo = 0xffffffffu, keep_hi = 0xffffffffu;
+            if (valid < BS) {
+                const int t = 16 * ks + 2 * (lane & 3);
+                keep_lo = (t < valid ? 0x0000ffffu : 0u) | (t + 1 < valid ? 0xffff0000u : 0u);
+                keep_hi = (t + 8 < valid ? 0x0000ffffu : 0u) | (t + 9 < valid ? 0xffff0000u : 0u);
+            }
+#pragma unroll
+            for (int dt = 0; dt < DT; ++dt) {
+                uint32_t a[4];
+                ldsm_x4_trans(a, tile_addr<BS>(vtile, 16 * ks + r + 8 * (mi >> 1), 2 * dt + (mi & 1)));
+                a[0] &= keep_lo;
+                a[1] &= keep_lo;
+                a[2] &= keep_hi;
+                a[3] &= keep_hi;
+                mma_16816(acc[dt], a, b0, b1);
+            }
+        }
+        __syncwarp();  // P scratch is rewritten by the next block
+    }
+
+    __device__ __forceinline__ void export_state(float *merge_acc, float *merge_m, float *merge_l, int warp) {
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+            l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+            l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+        }
+        const int g0 = 2 * (lane & 3), dr = lane >> 2;
+        if (lane < 4) {
+            merge_m[warp * GP + g0] = m0;
+            merge_m[warp * GP + g0 + 1] = m1;
+            merge_l[warp * GP + g0] = l0;
+            merge_l[warp * GP + g0 + 1] = l1;
+        }
+        float *r0 = merge_acc + (warp * GP + g0) * D;
+        float *r1 = r0 + D;
+#pragma unroll
+        for (int dt = 0; dt < DT; ++dt) {
+            r0[16 * dt + dr] = acc[dt][0];
+            r1[16 * dt + dr] = acc[dt][1];
+            r0[16 * dt + dr + 8] = acc[dt][2];
+            r1[16 * dt + dr + 8] = acc[dt][3];
+        }
+    }
+};
+
+// ------------------------------------------------------------------ pipeline
 
 struct Smem {
     uint8_t *base;
@@ -216,6 +498,7 @@ template <int D, int BS, int GP>
 __device__ __forceinline__ void producer_warp(const CUtensorMap *tm_k, const CUtensorMap *tm_v, const DecodeArgs &a,
                                               const Smem &sm, const DecodeLayout &ly, int total_items, int lane) {
     constexpr uint32_t kTile = BS * D * 2;
+    constexpr uint32_t kHalf = BS * 128;
     const int R = a.num_stages;  // stages per consumer warp
     const int P = a.partition_blocks * BS, cap = a.max_blocks_per_seq * BS;
     const uint32_t qbytes = static_cast<uint32_t>(a.group * D * 2);
@@ -264,8 +547,12 @@ __device__ __forceinline__ void producer_warp(const CUtensorMap *tm_k, const CUt
                         } else {
                             uint8_t *dst = sm.base + ly.stages + static_cast<uint32_t>(stage) * 2u * kTile;
                             mbar_arrive_expect_tx(&sm.full[stage], 2u * kTile);
-                            tma_load_4d(dst, tm_k, &sm.full[stage], 0, 0, it.h, pi * BS);
-                            tma_load_4d(dst + kTile, tm_v, &sm.full[stage], 0, 0, it.h, pi * BS);
+#pragma unroll
+                            for (int half = 0; half < D / 64; ++half) {
+                                tma_load_4d(dst + half * kHalf, tm_k, &sm.full[stage], 0, half, it.h, pi * BS);
+                                tma_load_4d(dst + kTile + half * kHalf, tm_v, &sm.full[stage], 0, half, it.h,
+                                            pi * BS);
+                            }
                             issued |= 1u << stage;
                             issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
                         }
@@ -283,65 +570,36 @@ __device__ __forceinline__ void producer_warp(const CUtensorMap *tm_k, const CUt
     }
 }
 
-template <int D, int BS, int GP>
+template <int D, int BS, class Math>
 __device__ __forceinline__ void consumer_warps(const DecodeArgs &a, const Smem &sm, const DecodeLayout &ly,
                                                int total_items, int warp, int lane) {
-    constexpr int LPT = D / 8;
+    constexpr int GP = Math::GP;
     constexpr uint32_t kTile = BS * D * 2;
     const int R = a.num_stages;  // this warp's ring: stages warp, warp + 4, ..., warp + 4 (R - 1)
     const int P = a.partition_blocks * BS, cap = a.max_blocks_per_seq * BS;
-    const int tg = lane / LPT, ch = lane % LPT;
-    const int g_own = g_own_of<GP, LPT>(lane);
-    const bool writer = (lane % (LPT / GP)) == 0;
     const uint32_t sbase = smem_u32(sm.base);
-    float2 *pscr = reinterpret_cast<float2 *>(sm.base + ly.pscr) + warp * BS * GP;
     float *merge_acc = reinterpret_cast<float *>(sm.base + ly.merge_acc);
     float *merge_m = reinterpret_cast<float *>(sm.base + ly.merge_m);
     float *merge_l = reinterpret_cast<float *>(sm.base + ly.merge_l);
     const int ctid = warp * 32 + lane;
     int qslot = 0, gb_base = 0, ring = 0;
     uint32_t qphase = 0, rphase = 0;
+    Math math;
+    math.init(warp, lane, sm.base, ly);
 
     for (int u = blockIdx.x; u < total_items; u += gridDim.x) {
         const Item it = decode_item<BS>(u, sm.prefix, a, P, cap);
         const int nblk = it.b1 - it.b0;
 
-        // query rows of the GQA group, pre-scaled into base-2 logits
-        float2 q2[GP][4];
         mbar_wait_bounded(&sm.qfull[qslot], qphase, sm.abort_flag, a.status);
-        {
-            const uint32_t qa = sbase + ly.qbuf + qslot * (GP * D * 2) + ch * 16;
-            const float2 sc = make_float2(a.scale_log2, a.scale_log2);
-#pragma unroll
-            for (int g = 0; g < GP; ++g) {
-                if (g < a.group) {
-                    const uint4 r = lds128(qa + g * D * 2);
-                    q2[g][0] = fmul2(bf16x2_to_float2(r.x), sc);
-                    q2[g][1] = fmul2(bf16x2_to_float2(r.y), sc);
-                    q2[g][2] = fmul2(bf16x2_to_float2(r.z), sc);
-                    q2[g][3] = fmul2(bf16x2_to_float2(r.w), sc);
-                } else {
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) q2[g][k] = make_float2(0.f, 0.f);
-                }
-            }
-        }
+        math.load_q(sbase + ly.qbuf + qslot * (GP * D * 2), a.group, a.scale_log2);
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.qempty[qslot]);
         if (++qslot == 2) {
             qslot = 0;
             qphase ^= 1u;
         }
-
-        float m_run[GP];
-        float l_run = 0.f;
-        float2 acc[GP][4];
-#pragma unroll
-        for (int g = 0; g < GP; ++g) {
-            m_run[g] = -INFINITY;
-#pragma unroll
-            for (int k = 0; k < 4; ++k) acc[g][k] = make_float2(0.f, 0.f);
-        }
+        math.reset();
 
         // this warp's blocks of the item: item-local i with (gb_base + i) % 4 == warp
         for (int i = (warp - gb_base % kConsumerWarps + kConsumerWarps) % kConsumerWarps; i < nblk;
@@ -356,37 +614,14 @@ __device__ __forceinline__ void consumer_warps(const DecodeArgs &a, const Smem &
             if (!sm.stage_bad[stage] && !*sm.abort_flag) {
                 const int valid = min(BS, it.tok1 - (it.b0 + i) * BS);
                 const uint32_t ktile = sbase + ly.stages + static_cast<uint32_t>(stage) * 2u * kTile;
-                block_cuda_core<D, BS, GP>(ktile, ktile + kTile, valid, q2, m_run, l_run, acc, pscr, tg, ch, lane,
-                                           g_own, writer);
+                math.block(ktile, ktile + kTile, valid);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.empty[stage]);
         }
         gb_base += nblk;
 
-        // token groups of a warp share m_run: their accumulators just add
-#pragma unroll
-        for (int o = LPT; o < 32; o <<= 1)
-#pragma unroll
-            for (int g = 0; g < GP; ++g)
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    acc[g][k].x += __shfl_xor_sync(0xffffffffu, acc[g][k].x, o);
-                    acc[g][k].y += __shfl_xor_sync(0xffffffffu, acc[g][k].y, o);
-                }
-        if (tg == 0) {
-#pragma unroll
-            for (int g = 0; g < GP; ++g) {
-                float4 *dst = reinterpret_cast<float4 *>(merge_acc + (warp * GP + g) * D + ch * 8);
-                dst[0] = make_float4(acc[g][0].x, acc[g][0].y, acc[g][1].x, acc[g][1].y);
-                dst[1] = make_float4(acc[g][2].x, acc[g][2].y, acc[g][3].x, acc[g][3].y);
-            }
-        }
-        if (lane == 0) {
-#pragma unroll
-            for (int g = 0; g < GP; ++g) merge_m[warp * GP + g] = m_run[g];
-        }
-        if (lane < GP) merge_l[warp * GP + lane] = l_run;
+        math.export_state(merge_acc, merge_m, merge_l, warp);
         named_barrier_sync(1, kConsumerWarps * 32);
 
         // merge the warps' states (log-sum-exp identity) and store
@@ -424,13 +659,14 @@ __device__ __forceinline__ void consumer_warps(const DecodeArgs &a, const Smem &
     }
 }
 
-template <int D, int BS, int GP>
+template <int D, int BS, int GP, int MATH>
 __global__ void __launch_bounds__(kDecodeThreads)
     paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                         const DecodeArgs a) {
     static_assert(D == 64 || D == 128, "head_dim");
     static_assert(BS == 16 || BS == 32, "block_size");
     static_assert(GP == 1 || GP == 2 || GP == 4 || GP == 8, "group");
+    static_assert(MATH == kMathCudaCore || GP == 8, "the tensor-core path pads the group to 8");
     extern __shared__ uint8_t smem_raw[];
     const DecodeLayout ly = decode_layout(D, BS, GP, kConsumerWarps * a.num_stages, a.num_seqs);
     Smem sm;
@@ -502,8 +738,10 @@ __global__ void __launch_bounds__(kDecodeThreads)
 
     if (warp == kConsumerWarps) {
         producer_warp<D, BS, GP>(&tm_k, &tm_v, a, sm, ly, total_items, lane);
+    } else if constexpr (MATH == kMathCudaCore) {
+        consumer_warps<D, BS, CoreMath<D, BS, GP>>(a, sm, ly, total_items, warp, lane);
     } else {
-        consumer_warps<D, BS, GP>(a, sm, ly, total_items, warp, lane);
+        consumer_warps<D, BS, MmaMath<D, BS>>(a, sm, ly, total_items, warp, lane);
     }
 }
 
@@ -546,11 +784,15 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(const DecodeArgs a, int 
 
 using KernelFn = void (*)(const CUtensorMap, const CUtensorMap, const DecodeArgs);
 
+// The tensor-core path always pads the group to 8 (one n8 tile).
+int effective_group_pad(int group_pad, int math) { return math == kMathTensorCore ? 8 : group_pad; }
+
 KernelFn pick(int D, int BS, int GP, int math) {
-    if (math != kMathCudaCore) return nullptr;
-#define PKV_CASE(d, bs, gp) \
-    if (D == d && BS == bs && GP == gp) return paged_decode_kernel<d, bs, gp>;
-#define PKV_GP(d, bs) PKV_CASE(d, bs, 1) PKV_CASE(d, bs, 2) PKV_CASE(d, bs, 4) PKV_CASE(d, bs, 8)
+#define PKV_CASE(d, bs, gp, m) \
+    if (D == d && BS == bs && GP == gp && math == m) return paged_decode_kernel<d, bs, gp, m>;
+#define PKV_GP(d, bs)                                                                                \
+    PKV_CASE(d, bs, 1, kMathCudaCore) PKV_CASE(d, bs, 2, kMathCudaCore) PKV_CASE(d, bs, 4, kMathCudaCore) \
+    PKV_CASE(d, bs, 8, kMathCudaCore) PKV_CASE(d, bs, 8, kMathTensorCore)
     PKV_GP(64, 16) PKV_GP(64, 32) PKV_GP(128, 16) PKV_GP(128, 32)
 #undef PKV_GP
 #undef PKV_CASE
@@ -560,17 +802,18 @@ KernelFn pick(int D, int BS, int GP, int math) {
 }  // namespace
 
 bool decode_variant_exists(int head_dim, int block_size, int group_pad, int math) {
-    return pick(head_dim, block_size, group_pad, math) != nullptr;
+    return pick(head_dim, block_size, effective_group_pad(group_pad, math), math) != nullptr;
 }
 
 size_t decode_smem_bytes(int head_dim, int block_size, int group_pad, int math, int num_stages, int num_seqs) {
-    (void)math;
-    return decode_layout(head_dim, block_size, group_pad, kConsumerWarps * num_stages, num_seqs).total;
+    return decode_layout(head_dim, block_size, effective_group_pad(group_pad, math), kConsumerWarps * num_stages,
+                         num_seqs)
+        .total;
 }
 
 cudaError_t decode_prepare(int head_dim, int block_size, int group_pad, int math, size_t smem_bytes,
                            int *ctas_per_sm) {
-    KernelFn fn = pick(head_dim, block_size, group_pad, math);
+    KernelFn fn = pick(head_dim, block_size, effective_group_pad(group_pad, math), math);
     if (!fn) return cudaErrorInvalidValue;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -591,7 +834,7 @@ cudaError_t decode_prepare(int head_dim, int block_size, int group_pad, int math
 cudaError_t decode_launch(int head_dim, int block_size, int group_pad, int math, const CUtensorMap &tm_k,
                           const CUtensorMap &tm_v, const DecodeArgs &args, int grid, size_t smem_bytes,
                           cudaStream_t stream) {
-    KernelFn fn = pick(head_dim, block_size, group_pad, math);
+    KernelFn fn = pick(head_dim, block_size, effective_group_pad(group_pad, math), math);
     if (!fn) return cudaErrorInvalidValue;
     fn<<<grid, kDecodeThreads, smem_bytes, stream>>>(tm_k, tm_v, args);
     return cudaGetLastError();

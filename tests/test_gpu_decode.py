@@ -48,27 +48,33 @@ def config_case(name):
     return b, ref, kc_ref, vc_ref
 
 
+MATHS = [1, 2]  # 1 = fp32 CUDA cores, 2 = bf16 tensor cores (mma.sync)
+
+
+@pytest.mark.parametrize("math", MATHS)
 @pytest.mark.parametrize("name", workloads.CONFIG_ORDER)
-def test_config_parity(name):
+def test_config_parity(name, math):
     b, ref, kc_ref, vc_ref = config_case(name)
-    out, kc, vc, st = run_step(b)
+    out, kc, vc, st = run_step(b, math=math)
     assert st == 0, f"status {st}"
     assert np.array_equal(bf16_bits(kc), kc_ref), "append: K pool differs from the oracle's"
     assert np.array_equal(bf16_bits(vc), vc_ref), "append: V pool differs from the oracle's"
     assert_close_to_oracle(out.double().numpy(), ref, what=name)
 
 
+@pytest.mark.parametrize("math", MATHS)
 @pytest.mark.parametrize("name", ["tiny", "opt125m", "qwen25_7b_prefix", "skewed_long"])
 @pytest.mark.parametrize("partition_tokens", [32, 64, 1 << 20])
-def test_forced_split_sizes(name, partition_tokens):
+def test_forced_split_sizes(name, partition_tokens, math):
     b, ref, _, _ = config_case(name)
-    out, _, _, st = run_step(b, partition_tokens=partition_tokens)
+    out, _, _, st = run_step(b, partition_tokens=partition_tokens, math=math)
     assert st == 0
     assert_close_to_oracle(out.double().numpy(), ref, what=f"{name} P={partition_tokens}")
 
 
 @pytest.mark.parametrize("opts", [dict(num_stages=1), dict(num_stages=2), dict(num_stages=4), dict(ctas_per_sm=1),
-                                  dict(num_stages=3, ctas_per_sm=2, partition_tokens=128)])
+                                  dict(num_stages=3, ctas_per_sm=2, partition_tokens=128),
+                                  dict(math=2, num_stages=1), dict(math=2, num_stages=4, ctas_per_sm=1)])
 def test_launch_options(opts):
     b, ref, _, _ = config_case("opt125m")
     out, _, _, st = run_step(b, **opts)
@@ -76,10 +82,11 @@ def test_launch_options(opts):
     assert_close_to_oracle(out.double().numpy(), ref, what=str(opts))
 
 
+@pytest.mark.parametrize("math", MATHS)
 @pytest.mark.parametrize("name", golden_names())
-def test_golden_fixture(name):
+def test_golden_fixture(name, math):
     b, expected = load_golden(name)
-    out, _, _, st = run_step(b, append=False)
+    out, _, _, st = run_step(b, append=False, math=math)
     assert st == 0
     for (s, j), row in expected.items():
         assert_close_to_oracle(out[s, j].double().numpy(), row, what=f"golden {name} ({s},{j})")
@@ -91,58 +98,65 @@ def test_every_group_size_and_shape(G, D, bs):
     lens = [1, bs - 1, bs, bs + 1, 3 * bs + 5, 700, 0, 1029]
     b = workloads.make_custom(1000 + G * 7 + D + bs, lens, 2 * G, 2, D, bs)
     ref, _, _ = oracle.decode_step(b)
-    for P in (0, 2 * bs):
-        out, _, _, st = run_step(b, partition_tokens=P)
-        assert st == 0
-        assert_close_to_oracle(out.double().numpy(), ref, what=f"G={G} D={D} bs={bs} P={P}")
+    for math in MATHS:
+        for P in (0, 2 * bs):
+            out, _, _, st = run_step(b, partition_tokens=P, math=math)
+            assert st == 0
+            assert_close_to_oracle(out.double().numpy(), ref, what=f"G={G} D={D} bs={bs} P={P} math={math}")
 
 
-def test_block_permutation_is_bitwise_invariant():
+@pytest.mark.parametrize("math", MATHS)
+def test_block_permutation_is_bitwise_invariant(math):
     b, _, _, _ = config_case("opt125m")
-    out1, _, _, _ = run_step(b)
-    out2, _, _, _ = run_step(workloads.permute_pool(b, seed=123))
+    out1, _, _, _ = run_step(b, math=math)
+    out2, _, _, _ = run_step(workloads.permute_pool(b, seed=123), math=math)
     assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
 
 
-def test_shared_prefix_equals_private_copies_bitwise():
+@pytest.mark.parametrize("math", MATHS)
+def test_shared_prefix_equals_private_copies_bitwise(math):
     b, _, _, _ = config_case("qwen25_7b_prefix")
-    out1, _, _, _ = run_step(b)
-    out2, _, _, _ = run_step(workloads.unshare_prefix(b))
+    out1, _, _, _ = run_step(b, math=math)
+    out2, _, _, _ = run_step(workloads.unshare_prefix(b), math=math)
     assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
 
 
-def test_runs_are_bitwise_reproducible():
+@pytest.mark.parametrize("math", MATHS)
+def test_runs_are_bitwise_reproducible(math):
     b, _, _, _ = config_case("skewed_long")
-    out1, _, _, _ = run_step(b)
-    out2, _, _, _ = run_step(b)
+    out1, _, _, _ = run_step(b, math=math)
+    out2, _, _, _ = run_step(b, math=math)
     assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
 
 
-def test_context_len_one_returns_the_appended_value_exactly():
+@pytest.mark.parametrize("math", MATHS)
+def test_context_len_one_returns_the_appended_value_exactly(math):
     b = workloads.make_custom(77, [1] * 40, 32, 8, 128, 16)
-    out, _, _, st = run_step(b)
+    out, _, _, st = run_step(b, math=math)
     assert st == 0
     G = 4
     expect = b.v_new.repeat_interleave(G, dim=1)
     assert torch.equal(out.view(torch.int16), expect.view(torch.int16))
 
 
-def test_identical_keys_give_the_mean_of_values():
+@pytest.mark.parametrize("math", MATHS)
+def test_identical_keys_give_the_mean_of_values(math):
     b = workloads.make_custom(78, [37, 300, 1], 8, 2, 128, 16, with_append=False)
     bs = b.block_size
     for s in range(b.num_seqs):
         p0 = int(b.block_tables[s, 0])
         for t in range(int(b.context_lens[s])):
             b.k_cache[int(b.block_tables[s, t // bs]), t % bs] = b.k_cache[p0, 0]
-    out, _, _, _ = run_step(b, append=False)
+    out, _, _, _ = run_step(b, append=False, math=math)
     ref = oracle.paged_decode(b.q, b.k_cache, b.v_cache, b.block_tables.numpy(), b.context_lens.numpy(),
                               2, bs, b.scale)
     assert_close_to_oracle(out.double().numpy(), ref, what="identical keys")
 
 
-def test_empty_contexts_give_zero_rows():
+@pytest.mark.parametrize("math", MATHS)
+def test_empty_contexts_give_zero_rows(math):
     b = workloads.make_custom(79, [0, 50, 0, 0, 17], 8, 2, 64, 16, with_append=False)
-    out, _, _, st = run_step(b, append=False)
+    out, _, _, st = run_step(b, append=False, math=math)
     assert st == 0
     for s in (0, 2, 3):
         assert torch.equal(out[s], torch.zeros_like(out[s]))
@@ -160,12 +174,13 @@ def test_more_sequences_than_one_launch_holds():
     assert_close_to_oracle(out.double().numpy(), ref, what="8300 sequences")
 
 
-def test_bad_block_id_is_flagged_not_faulted():
+@pytest.mark.parametrize("math", MATHS)
+def test_bad_block_id_is_flagged_not_faulted(math):
     b = workloads.make_custom(81, [40, 40], 4, 2, 64, 16, with_append=False, poison=False)
     bt = b.block_tables.clone()
     bt[1, 1] = b.num_blocks + 5
     b2 = workloads.DecodeBatch(**{**b.__dict__, "block_tables": bt})
-    out, _, _, st = run_step(b2, append=False)
+    out, _, _, st = run_step(b2, append=False, math=math)
     assert st & pkv.PKV_STATUS_BAD_BLOCK_ID
     ref = oracle.paged_decode(b.q, b.k_cache, b.v_cache, b.block_tables.numpy(), b.context_lens.numpy(),
                               2, 16, b.scale)
