@@ -50,7 +50,7 @@ def parse_args(argv=None):
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default="llama3_8b", choices=workloads.CONFIG_ORDER)
-    p.add_argument("--partition-tokens", type=int, default=0)
+    p.add_argument("--num-ctas", type=int, default=0)
     p.add_argument("--num-stages", type=int, default=0)
     p.add_argument("--ctas-per-sm", type=int, default=0)
     p.add_argument("--math", type=int, default=0)
@@ -208,10 +208,9 @@ class Step:
         self.slots = b.slot_mapping.to(device)
         self.out = torch.empty_like(self.q)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
-        self.opts = dict(partition_tokens=args.partition_tokens, num_stages=args.num_stages,
+        self.opts = dict(num_ctas=args.num_ctas, num_stages=args.num_stages,
                          ctas_per_sm=args.ctas_per_sm, math=args.math)
-        self.ws = pkv.allocate_workspace(b.num_seqs, b.num_q_heads, b.head_dim, b.max_blocks_per_seq,
-                                         b.block_size, args.partition_tokens, device=device)
+        self.ws = pkv.allocate_workspace(b.num_seqs, b.num_q_heads, b.head_dim, device=device)
 
     def append(self, stream=None):
         self.pkv.kv_cache_append(self.k_new, self.v_new, self.kc, self.vc, self.slots, self.status, stream=stream)
@@ -221,11 +220,8 @@ class Step:
                                    stream=stream, **self.opts)
 
     def decode_launches(self):
-        """Kernels one paged_attn_decode call launches (decode, plus merge when split)."""
-        P = self.opts["partition_tokens"] or 512
-        n_split = -(-self.b.max_blocks_per_seq * self.b.block_size // P)
-        chunks = -(-self.b.num_seqs // 8192)
-        return chunks * (2 if n_split > 1 else 1)
+        """Kernels one paged_attn_decode call launches: decode + merge per 2048 sequences."""
+        return 2 * -(-self.b.num_seqs // 2048)
 
 
 def run_ours(args, rank, world, local_rank):
@@ -386,7 +382,7 @@ def config_block(args, batch, world):
     }
     if args.seqs:
         c["seqs_kept"] = args.seqs
-    for k in ("partition_tokens", "num_stages", "ctas_per_sm", "math"):
+    for k in ("num_ctas", "num_stages", "ctas_per_sm", "math"):
         if getattr(args, k):
             c[k] = getattr(args, k)
     return c

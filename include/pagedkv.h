@@ -63,36 +63,35 @@ extern "C" {
 
 /*
  * Tuning knobs of paged_attn_decode_ex. Zero in any field means "default".
- *   partition_tokens  tokens of one context split (a multiple of block_size);
- *                     default 512. Sequences longer than this are split and
- *                     their partial results merged with a log-sum-exp
- *                     reduction kernel.
+ *   num_ctas          CTAs of the persistent decode grid (1..1024); default:
+ *                     every CTA that fits on the device at once. The KV blocks
+ *                     of a launch are split evenly over the CTAs, so this also
+ *                     sets how finely long contexts are split.
  *   num_stages        shared-memory stages (one KV block each) per consumer warp
  *                     (1..4; a CTA has 4 consumer warps); default: about 64 KB
  *                     of KV blocks in flight per CTA.
- *   ctas_per_sm       resident CTAs per SM of the persistent grid; default: the
+ *   ctas_per_sm       resident CTAs per SM of the default grid; default: the
  *                     occupancy limit.
  *   math              0 = default, 1 = fp32 CUDA cores, 2 = bf16 tensor cores
  *                     (mma.sync m16n8k16, fp32 accumulate).
  */
 typedef struct pkv_decode_options {
-    int partition_tokens;
+    int num_ctas;
     int num_stages;
     int ctas_per_sm;
     int math;
 } pkv_decode_options;
 
 /*
- * Bytes of device workspace paged_attn_decode needs for this shape.
- * Layout: [0, 256) header whose first int32 is the device status word; then
- * fp32 partial outputs [num_seqs][num_q_heads][n_split][head_dim] and fp32
- * log2-sum-exp values [num_seqs][num_q_heads][n_split], n_split =
- * ceil(max_blocks_per_seq * block_size / partition_tokens). Only splits that
- * hold tokens are written.
- * partition_tokens = 0 means the default. Host-only; returns PKV_OK and sets *bytes.
+ * Bytes of device workspace paged_attn_decode needs for this shape
+ * (host-only; returns PKV_OK and sets *bytes).
+ * Layout: [0, 256) header whose first int32 is the device status word; the
+ * per-sequence block prefix sums of one launch; fp32 partial outputs and
+ * log2-sum-exp values of the context pieces that CTA boundaries cut. At most
+ * 2048 sequences go in one launch; longer batches reuse the workspace launch
+ * after launch.
  */
-int pkv_decode_workspace_bytes(int num_seqs, int num_q_heads, int head_dim, int max_blocks_per_seq,
-                               int block_size, int partition_tokens, size_t *bytes);
+int pkv_decode_workspace_bytes(int num_seqs, int num_q_heads, int head_dim, size_t *bytes);
 
 /*
  * Paged decode attention (one query token per sequence).
@@ -112,10 +111,11 @@ int pkv_decode_workspace_bytes(int num_seqs, int num_q_heads, int head_dim, int 
  * Supported: head_dim in {64, 128}; block_size in {16, 32}; num_q_heads a
  * multiple of num_kv_heads with a ratio <= PKV_MAX_GROUP; num_blocks *
  * block_size < 2^31. Any num_seqs >= 0 (0 is a no-op).
- * Per call: one persistent decode kernel, plus one reduction kernel when a
- * context can be longer than partition_tokens. Results are bitwise
- * reproducible and depend only on the logical order of tokens, not on where
- * their blocks sit in the pool.
+ * Per call (and per 2048 sequences): one persistent decode kernel whose CTAs
+ * each take an equal share of the batch's KV blocks, then one log-sum-exp
+ * merge kernel for the contexts that were split between CTAs. For a given
+ * device and options, results are bitwise reproducible and depend only on the
+ * logical order of tokens, not on where their blocks sit in the pool.
  */
 int paged_attn_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
                       const int32_t *block_tables, const int32_t *context_lens,
@@ -146,8 +146,8 @@ int paged_attn_decode_ex(void *out, const void *q, const void *k_cache, const vo
  * other allocating routine.
  *
  * Limits and rules:
- *   - Batches whose workspace (pkv_decode_workspace_bytes with the default
- *     partition) exceeds PKV_NOALLOC_SCRATCH_BYTES are rejected with
+ *   - Batches whose workspace (pkv_decode_workspace_bytes) exceeds
+ *     PKV_NOALLOC_SCRATCH_BYTES are rejected with
  *     PKV_ERR_INVALID_ARGUMENT and a message giving both sizes.
  *   - The first call on a device looks up the scratch's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call

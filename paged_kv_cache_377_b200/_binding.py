@@ -30,7 +30,7 @@ class PagedKVError(RuntimeError):
 
 
 class _Options(ctypes.Structure):
-    _fields_ = [("partition_tokens", ctypes.c_int), ("num_stages", ctypes.c_int),
+    _fields_ = [("num_ctas", ctypes.c_int), ("num_stages", ctypes.c_int),
                 ("ctas_per_sm", ctypes.c_int), ("math", ctypes.c_int)]
 
 
@@ -63,7 +63,7 @@ def library() -> ctypes.CDLL:
             lib.pkv_last_error.argtypes = []
             lib.pkv_version.restype = ctypes.c_char_p
             lib.pkv_decode_workspace_bytes.restype = I
-            lib.pkv_decode_workspace_bytes.argtypes = [I, I, I, I, I, I, ctypes.POINTER(Z)]
+            lib.pkv_decode_workspace_bytes.argtypes = [I, I, I, ctypes.POINTER(Z)]
             lib.paged_attn_decode.restype = I
             lib.paged_attn_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, I, I, P, Z, P]
             lib.paged_attn_decode_ex.restype = I
@@ -111,24 +111,22 @@ def _need(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int) -> None:
         raise ValueError(f"{name} must be contiguous")
 
 
-def workspace_bytes(num_seqs: int, num_q_heads: int, head_dim: int, max_blocks_per_seq: int, block_size: int,
-                    partition_tokens: int = 0) -> int:
+def workspace_bytes(num_seqs: int, num_q_heads: int, head_dim: int) -> int:
     n = ctypes.c_size_t(0)
     _check("pkv_decode_workspace_bytes", library().pkv_decode_workspace_bytes(
-        num_seqs, num_q_heads, head_dim, max_blocks_per_seq, block_size, partition_tokens, ctypes.byref(n)))
+        num_seqs, num_q_heads, head_dim, ctypes.byref(n)))
     return int(n.value)
 
 
-def allocate_workspace(num_seqs: int, num_q_heads: int, head_dim: int, max_blocks_per_seq: int, block_size: int,
-                       partition_tokens: int = 0, device=None) -> torch.Tensor:
+def allocate_workspace(num_seqs: int, num_q_heads: int, head_dim: int, device=None) -> torch.Tensor:
     """A zeroed uint8 workspace of the required size (its first int32 is the status word)."""
-    n = workspace_bytes(num_seqs, num_q_heads, head_dim, max_blocks_per_seq, block_size, partition_tokens)
+    n = workspace_bytes(num_seqs, num_q_heads, head_dim)
     return torch.zeros(n, dtype=torch.uint8, device=device if device is not None else "cuda")
 
 
 def paged_attn_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
                       block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float,
-                      workspace: torch.Tensor, partition_tokens: int = 0, num_stages: int = 0,
+                      workspace: torch.Tensor, num_ctas: int = 0, num_stages: int = 0,
                       ctas_per_sm: int = 0, math: int = 0, stream=None) -> torch.Tensor:
     """out[s, j] = softmax_t(scale * q[s, j] . K_t) . V_t over the sequence's paged tokens.
 
@@ -149,7 +147,7 @@ def paged_attn_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
         raise ValueError("shape mismatch between q/out or k_cache/v_cache")
     if block_tables.shape[0] != S or context_lens.shape[0] != S:
         raise ValueError("block_tables and context_lens must have num_seqs rows")
-    opts = _Options(partition_tokens, num_stages, ctas_per_sm, math)
+    opts = _Options(num_ctas, num_stages, ctas_per_sm, math)
     _check("paged_attn_decode", library().paged_attn_decode_ex(
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
         S, Hq, Hkv, D, bs, float(scale), block_tables.shape[1], NB, _ptr(workspace), workspace.numel(),

@@ -89,13 +89,23 @@ int sm_count() {
     return cache[dev];
 }
 
-int resolve_partition(int partition_tokens, int block_size) {
-    return partition_tokens > 0 ? partition_tokens : pkv::kDefaultPartitionTokens;
-}
+// Workspace layout: [0, 256) header (status word) | block prefix sums
+// [S_chunk + 1] int32 | fp32 partial outputs [rows][D] | fp32 log2-sum-exp [rows],
+// rows = (S_chunk + kMaxCtas) * Hq bounds the pieces' rows of one launch
+// (pieces <= S_chunk * Hkv + C, each with G <= Hq rows).
+struct WorkspaceLayout {
+    size_t seq_blocks, o_part, lse_part, total;
+};
 
-int64_t n_split_of(int max_blocks_per_seq, int block_size, int partition_tokens) {
-    const int64_t cap = static_cast<int64_t>(max_blocks_per_seq) * block_size;
-    return (cap + partition_tokens - 1) / partition_tokens;
+WorkspaceLayout workspace_layout(int num_seqs, int num_q_heads, int head_dim) {
+    const int64_t sc = num_seqs < pkv::kMaxSeqsPerLaunch ? num_seqs : pkv::kMaxSeqsPerLaunch;
+    const int64_t rows = (sc + pkv::kMaxCtas) * num_q_heads;
+    WorkspaceLayout w;
+    w.seq_blocks = pkv::kWorkspaceHeaderBytes;
+    w.o_part = w.seq_blocks + ((sc + 1) * 4 + 255) / 256 * 256;
+    w.lse_part = w.o_part + rows * head_dim * 4;
+    w.total = w.lse_part + (rows * 4 + 255) / 256 * 256;
+    return w;
 }
 
 // Stages per consumer warp: about 64 KB of KV blocks in flight per CTA.
@@ -113,23 +123,11 @@ const char *pkv_last_error(void) { return g_err; }
 
 const char *pkv_version(void) { return "pagedkv 0.1 (sm_100a)"; }
 
-int pkv_decode_workspace_bytes(int num_seqs, int num_q_heads, int head_dim, int max_blocks_per_seq, int block_size,
-                               int partition_tokens, size_t *bytes) {
+int pkv_decode_workspace_bytes(int num_seqs, int num_q_heads, int head_dim, size_t *bytes) {
     if (!bytes) return fail(PKV_ERR_INVALID_ARGUMENT, "bytes is NULL");
-    if (num_seqs < 0 || num_q_heads <= 0 || head_dim <= 0 || max_blocks_per_seq <= 0 || block_size <= 0 ||
-        partition_tokens < 0)
-        return fail(PKV_ERR_INVALID_ARGUMENT, "sizes must be positive (num_seqs >= 0, partition_tokens >= 0)");
-    const int P = resolve_partition(partition_tokens, block_size);
-    if (P % block_size != 0)
-        return fail(PKV_ERR_INVALID_ARGUMENT, "partition_tokens %d is not a multiple of block_size %d", P, block_size);
-    const int64_t ns = n_split_of(max_blocks_per_seq, block_size, P);
-    const int64_t rows = static_cast<int64_t>(num_seqs) * num_q_heads;
-    int64_t total = pkv::kWorkspaceHeaderBytes;
-    if (ns > 1) {
-        total += rows * ns * head_dim * 4;  // fp32 partial outputs
-        total += (rows * ns * 4 + 255) / 256 * 256;  // fp32 log2-sum-exp
-    }
-    *bytes = static_cast<size_t>(total);
+    if (num_seqs < 0 || num_q_heads <= 0 || head_dim <= 0)
+        return fail(PKV_ERR_INVALID_ARGUMENT, "num_seqs must be >= 0, num_q_heads and head_dim > 0");
+    *bytes = workspace_layout(num_seqs, num_q_heads, head_dim).total;
     return ok();
 }
 
@@ -165,11 +163,12 @@ int paged_attn_decode_ex(void *out, const void *q, const void *k_cache, const vo
                     "out, q, k_cache and v_cache must be 16-byte aligned and workspace 256-byte aligned");
     pkv_decode_options o = {0, 0, 0, 0};
     if (opts) o = *opts;
-    if (o.partition_tokens < 0 || o.num_stages < 0 || o.ctas_per_sm < 0 || o.math < 0 || o.math > 2)
+    if (o.num_ctas < 0 || o.num_stages < 0 || o.ctas_per_sm < 0 || o.math < 0 || o.math > 2)
         return fail(PKV_ERR_INVALID_ARGUMENT, "negative or unknown option");
-    const int P = resolve_partition(o.partition_tokens, block_size);
-    if (P % block_size != 0)
-        return fail(PKV_ERR_INVALID_ARGUMENT, "partition_tokens %d is not a multiple of block_size %d", P, block_size);
+    if (o.num_ctas > pkv::kMaxCtas)
+        return fail(PKV_ERR_INVALID_ARGUMENT, "num_ctas %d exceeds %d", o.num_ctas, pkv::kMaxCtas);
+    if (static_cast<int64_t>(num_kv_heads) * max_blocks_per_seq * pkv::kMaxSeqsPerLaunch > 0x7fffffff)
+        return fail(PKV_ERR_INVALID_ARGUMENT, "num_kv_heads * max_blocks_per_seq too large");
     const int ns = o.num_stages ? o.num_stages : default_stages(head_dim, block_size);
     if (ns < 1 || ns > pkv::kMaxStagesPerWarp)
         return fail(PKV_ERR_INVALID_ARGUMENT, "num_stages %d outside [1, %d]", ns, pkv::kMaxStagesPerWarp);
@@ -178,9 +177,9 @@ int paged_attn_decode_ex(void *out, const void *q, const void *k_cache, const vo
     if (!pkv::decode_variant_exists(head_dim, block_size, gp, math))
         return fail(PKV_ERR_UNSUPPORTED, "no kernel for head_dim %d, block_size %d, group %d, math %d", head_dim,
                     block_size, group, math);
-    size_t need = 0;
-    int rc = pkv_decode_workspace_bytes(num_seqs, num_q_heads, head_dim, max_blocks_per_seq, block_size, P, &need);
-    if (rc != PKV_OK) return rc;
+    const WorkspaceLayout wl = workspace_layout(num_seqs, num_q_heads, head_dim);
+    const size_t need = wl.total;
+    int rc = PKV_OK;
     if (workspace_bytes < need)
         return fail(PKV_ERR_INVALID_ARGUMENT, "workspace_bytes %zu < required %zu", workspace_bytes, need);
     if (num_seqs == 0) return ok();
@@ -189,17 +188,13 @@ int paged_attn_decode_ex(void *out, const void *q, const void *k_cache, const vo
     if ((rc = make_pool_map(&tm_k, k_cache, num_blocks, block_size, num_kv_heads, head_dim)) != PKV_OK) return rc;
     if ((rc = make_pool_map(&tm_v, v_cache, num_blocks, block_size, num_kv_heads, head_dim)) != PKV_OK) return rc;
 
-    const int64_t n_split = n_split_of(max_blocks_per_seq, block_size, P);
-    const int64_t rows = static_cast<int64_t>(num_seqs) * num_q_heads;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
-    float *o_part = reinterpret_cast<float *>(ws + pkv::kWorkspaceHeaderBytes);
-    float *lse_part = o_part + rows * n_split * head_dim;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int sms = sm_count();
     if (sms <= 0) return fail(PKV_ERR_CUDA, "no CUDA device");
 
-    // Sequences go in launches of at most kMaxSeqsPerLaunch (their prefix sums
-    // live in shared memory); the workspace rows follow the sequences.
+    // Sequences go in launches of at most kMaxSeqsPerLaunch (their tables live
+    // in shared memory); launches run in stream order and reuse the workspace.
     for (int s0 = 0; s0 < num_seqs; s0 += pkv::kMaxSeqsPerLaunch) {
         const int sc = num_seqs - s0 < pkv::kMaxSeqsPerLaunch ? num_seqs - s0 : pkv::kMaxSeqsPerLaunch;
         const size_t smem = pkv::decode_smem_bytes(head_dim, block_size, gp, math, ns, sc);
@@ -208,13 +203,16 @@ int paged_attn_decode_ex(void *out, const void *q, const void *k_cache, const vo
         if (e != cudaSuccess) return cuda_fail(e, "decode kernel setup");
         if (per_sm <= 0) return fail(PKV_ERR_INVALID_ARGUMENT, "shared memory %zu bytes per CTA does not fit", smem);
         if (o.ctas_per_sm > 0 && o.ctas_per_sm < per_sm) per_sm = o.ctas_per_sm;
+        int grid = o.num_ctas > 0 ? o.num_ctas : sms * per_sm;
+        if (grid > pkv::kMaxCtas) grid = pkv::kMaxCtas;
         pkv::DecodeArgs a;
         a.out = static_cast<__nv_bfloat16 *>(out) + static_cast<size_t>(s0) * num_q_heads * head_dim;
         a.q = static_cast<const __nv_bfloat16 *>(q) + static_cast<size_t>(s0) * num_q_heads * head_dim;
         a.block_tables = block_tables + static_cast<size_t>(s0) * max_blocks_per_seq;
         a.context_lens = context_lens + s0;
-        a.o_part = o_part + static_cast<size_t>(s0) * num_q_heads * n_split * head_dim;
-        a.lse_part = lse_part + static_cast<size_t>(s0) * num_q_heads * n_split;
+        a.o_part = reinterpret_cast<float *>(ws + wl.o_part);
+        a.lse_part = reinterpret_cast<float *>(ws + wl.lse_part);
+        a.seq_blocks = reinterpret_cast<int32_t *>(ws + wl.seq_blocks);
         a.status = reinterpret_cast<int32_t *>(ws);
         a.num_seqs = sc;
         a.num_q_heads = num_q_heads;
@@ -222,19 +220,12 @@ int paged_attn_decode_ex(void *out, const void *q, const void *k_cache, const vo
         a.group = group;
         a.max_blocks_per_seq = max_blocks_per_seq;
         a.num_blocks = num_blocks;
-        a.partition_blocks = P / block_size;
-        a.n_split = static_cast<int>(n_split);
         a.num_stages = ns;
         a.scale_log2 = scale * 1.4426950408889634f;
-        const int64_t items = static_cast<int64_t>(sc) * n_split * num_kv_heads;
-        const int64_t cap = static_cast<int64_t>(sms) * per_sm;
-        const int grid = static_cast<int>(items < cap ? items : cap);
         e = pkv::decode_launch(head_dim, block_size, gp, math, tm_k, tm_v, a, grid, smem, st);
         if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
-        if (n_split > 1) {
-            e = pkv::lse_merge_launch(head_dim, block_size, a, st);
-            if (e != cudaSuccess) return cuda_fail(e, "lse merge launch");
-        }
+        e = pkv::lse_merge_launch(head_dim, a, grid, st);
+        if (e != cudaSuccess) return cuda_fail(e, "lse merge launch");
     }
     return ok();
 }
@@ -338,7 +329,7 @@ extern "C" int paged_attn_decode_noalloc(void *out, const void *q, const void *k
                                          float scale, int max_blocks_per_seq, int num_blocks, int32_t *d_status,
                                          void *stream) {
     size_t need = 0;
-    int rc = pkv_decode_workspace_bytes(num_seqs, num_q_heads, head_dim, max_blocks_per_seq, block_size, 0, &need);
+    int rc = pkv_decode_workspace_bytes(num_seqs, num_q_heads, head_dim, &need);
     if (rc != PKV_OK) return rc;
     if (need > PKV_NOALLOC_SCRATCH_BYTES)
         return fail(PKV_ERR_INVALID_ARGUMENT,

@@ -8,15 +8,20 @@
 // blocks; "Deep Dive into vLLM", section 2.1: logical -> physical blocks).
 //
 // How (design for B200; the pages describe no kernel):
-//   * Work item = (sequence, kv head, context split of P tokens). A persistent
-//     grid of (SMs x resident CTAs) walks the items with a fixed stride; every
-//     CTA rebuilds the prefix sum of split counts in shared memory, so no
-//     planning kernel and no host/device synchronisation are needed.
+//   * Work decomposition: the unit is one KV block of one (sequence, kv head)
+//     "segment"; segments are ordered (sequence, head) and CTA c of C takes
+//     the contiguous range [c B / C, (c + 1) B / C) of the B blocks of the
+//     launch, so every CTA gets the same number of blocks (+-1) whatever the
+//     length skew. A CTA's range crosses a few segments; each crossing is a
+//     "piece". Every CTA rebuilds the per-sequence block prefix sums in shared
+//     memory, so no planning kernel and no host/device synchronisation are
+//     needed.
 //   * One producer warp streams whole KV blocks of the item's kv head into
 //     shared memory with TMA (4D tile copies of 64 columns, 128-byte swizzle),
 //     completing on mbarriers. Block-table entries are read 32 at a time by the
-//     warp's lanes. The producer runs ahead across item boundaries, so HBM
-//     stays busy while consumers merge.
+//     warp's lanes, one 32-block chunk ahead of the chunk being issued. The
+//     producer runs ahead across piece boundaries, so HBM stays busy while
+//     consumers merge.
 //   * Four consumer warps take the blocks round-robin (block g of the CTA's
 //     stream goes to warp g % 4) and each warp owns its own ring of R stages,
 //     so every waiter sees every phase of its barriers in order (a parity wait
@@ -29,10 +34,11 @@
 //     cores, packed f32x2) and MmaMath (bf16 tensor cores, mma.sync m16n8k16
 //     with fp32 accumulation: S^T = K.Q^T with the block's tokens as M and the
 //     G <= 8 query heads as N, then O^T += V^T.P^T).
-//   * At the end of an item the four warp states are merged in shared memory
-//     with the log-sum-exp identity. Unsplit sequences write bf16 output
-//     directly; split ones write fp32 partials + log2-sum-exp, merged by
-//     lse_merge_kernel in a fixed split order.
+//   * At the end of a piece the four warp states are merged in shared memory
+//     with the log-sum-exp identity. A piece that is a whole segment writes
+//     bf16 output directly; the pieces of a segment cut by CTA boundaries
+//     write fp32 partials + log2-sum-exp, merged by lse_merge_kernel in CTA
+//     order.
 // Every reduction order depends only on logical token positions, so results
 // are bitwise reproducible and independent of where blocks sit in the pool.
 #include <cstdio>
@@ -46,32 +52,48 @@
 namespace pkv {
 namespace {
 
-struct Item {
-    int s, split, h, tok0, tok1, b0, b1, n_split;
+// A piece: blocks [b0, b1) of segment (s, h), processed by one CTA.
+struct Piece {
+    int s, h, b0, b1, L;
+    bool whole;  // the piece is the entire segment (no merge needed)
 };
 
-// Item u -> (sequence, split, kv head) through the shared-memory prefix sums.
-template <int BS>
-__device__ __forceinline__ Item decode_item(int u, const int *prefix, const DecodeArgs &a, int P, int cap) {
-    Item it;
-    const int v = u / a.num_kv_heads;
-    it.h = u - v * a.num_kv_heads;
-    int lo = 0, hi = a.num_seqs - 1;
-    while (lo < hi) {  // largest s with prefix[s] <= v
-        const int mid = (lo + hi + 1) >> 1;
-        if (prefix[mid] <= v) lo = mid;
-        else hi = mid - 1;
+// Walks the pieces of this CTA's block range [x, x1) in order. pre[s] holds
+// the blocks of sequences < s; sequence s contributes Hkv segments of
+// pre[s + 1] - pre[s] blocks each.
+struct PieceIter {
+    long long x, x1;
+    const int *pre;
+    const int *lens;
+    int S, Hkv;
+
+    __device__ __forceinline__ bool next(Piece &pc) {
+        if (x >= x1) return false;
+        int lo = 0, hi = S - 1;
+        while (lo < hi) {  // the sequence holding global block x
+            const int mid = (lo + hi + 1) >> 1;
+            if (static_cast<long long>(Hkv) * pre[mid] <= x) lo = mid;
+            else hi = mid - 1;
+        }
+        const int n = pre[lo + 1] - pre[lo];
+        const long long base = static_cast<long long>(Hkv) * pre[lo];
+        const int r = static_cast<int>(x - base);
+        const int h = r / n;
+        const long long seg_end = base + static_cast<long long>(h + 1) * n;
+        const long long end = x1 < seg_end ? x1 : seg_end;
+        pc.s = lo;
+        pc.h = h;
+        pc.b0 = r - h * n;
+        pc.b1 = pc.b0 + static_cast<int>(end - x);
+        pc.L = lens[lo];
+        pc.whole = pc.b0 == 0 && end == seg_end;
+        x = end;
+        return true;
     }
-    it.s = lo;
-    it.split = v - prefix[lo];
-    it.n_split = prefix[lo + 1] - prefix[lo];
-    int L = __ldg(a.context_lens + lo);
-    L = min(max(L, 0), cap);
-    it.tok0 = it.split * P;
-    it.tok1 = min(L, it.tok0 + P);
-    it.b0 = it.tok0 / BS;
-    it.b1 = (it.tok1 > it.tok0) ? (it.tok1 + BS - 1) / BS : it.b0;
-    return it;
+};
+
+__device__ __forceinline__ long long range_begin(int c, long long B, int C) {
+    return static_cast<long long>(c) * B / C;
 }
 
 // Shared address of 16-byte chunk c (0 <= c < D/8) of row t of a K or V tile.
@@ -492,74 +514,93 @@ struct Smem {
     volatile int *abort_flag;
     int *scan;
     int *prefix;
+    int *lens;
 };
 
 template <int D, int BS, int GP>
 __device__ __forceinline__ void producer_warp(const CUtensorMap *tm_k, const CUtensorMap *tm_v, const DecodeArgs &a,
-                                              const Smem &sm, const DecodeLayout &ly, int total_items, int lane) {
+                                              const Smem &sm, const DecodeLayout &ly, PieceIter pieces, int lane) {
     constexpr uint32_t kTile = BS * D * 2;
     constexpr uint32_t kHalf = BS * 128;
     const int R = a.num_stages;  // stages per consumer warp
-    const int P = a.partition_blocks * BS, cap = a.max_blocks_per_seq * BS;
     const uint32_t qbytes = static_cast<uint32_t>(a.group * D * 2);
     int qslot = 0, gb = 0;
     uint32_t qphase = 0;
     uint32_t issued = 0, issued_par = 0, q_issued = 0, q_issued_par = 0;  // copies possibly in flight
 
-    for (int u = blockIdx.x; u < total_items; u += gridDim.x) {
-        const Item it = decode_item<BS>(u, sm.prefix, a, P, cap);
-        if (lane == 0) {
+    // Table entries come in chunks of up to 32 blocks of one piece; the next
+    // chunk's entries are loaded while the current chunk is issued.
+    Piece cur, nxt;
+    bool have_cur = pieces.next(cur), have_nxt = false;
+    int cur_b = have_cur ? cur.b0 : 0;          // first block of the current chunk
+    int p_cur = -1, p_nxt = -1;
+    auto load = [&](const Piece &pc, int b) {
+        const int idx = b + lane;
+        return idx < pc.b1 ? __ldg(a.block_tables + static_cast<size_t>(pc.s) * a.max_blocks_per_seq + idx) : 0;
+    };
+    if (have_cur) p_cur = load(cur, cur_b);
+    while (have_cur) {
+        // the chunk after this one: same piece, or the first chunk of the next piece
+        int nxt_b;
+        if (cur_b + 32 < cur.b1) {
+            nxt = cur;
+            nxt_b = cur_b + 32;
+            have_nxt = true;
+        } else {
+            have_nxt = pieces.next(nxt);
+            nxt_b = have_nxt ? nxt.b0 : 0;
+        }
+        if (have_nxt) p_nxt = load(nxt, nxt_b);
+
+        if (cur_b == cur.b0 && lane == 0) {  // first chunk of a piece: its query rows
             if (mbar_wait_bounded(&sm.qempty[qslot], qphase ^ 1u, sm.abort_flag, a.status) && !*sm.abort_flag) {
                 const __nv_bfloat16 *src = static_cast<const __nv_bfloat16 *>(a.q) +
-                                           (static_cast<size_t>(it.s) * a.num_q_heads +
-                                            static_cast<size_t>(it.h) * a.group) * D;
+                                           (static_cast<size_t>(cur.s) * a.num_q_heads +
+                                            static_cast<size_t>(cur.h) * a.group) * D;
                 mbar_arrive_expect_tx(&sm.qfull[qslot], qbytes);
                 bulk_load(sm.base + ly.qbuf + qslot * (GP * D * 2), src, qbytes, &sm.qfull[qslot]);
                 q_issued |= 1u << qslot;
                 q_issued_par = (q_issued_par & ~(1u << qslot)) | (qphase << qslot);
             }
         }
-        if (++qslot == 2) {
+        if (cur_b == cur.b0 && ++qslot == 2) {
             qslot = 0;
             qphase ^= 1u;
         }
-        const int32_t *row = a.block_tables + static_cast<size_t>(it.s) * a.max_blocks_per_seq;
-        for (int bb = it.b0; bb < it.b1; bb += 32) {
-            const int b = bb + lane;
-            const int p = (b < it.b1) ? __ldg(row + b) : 0;
-            const int n = min(32, it.b1 - bb);
-            for (int i = 0; i < n; ++i, ++gb) {
-                const int pi = __shfl_sync(0xffffffffu, p, i);
-                if (lane == 0) {
-                    // block gb belongs to consumer warp gb % 4, slot (gb / 4) % R of its ring
-                    const int k = gb >> 2;
-                    const int stage = (gb & 3) + kConsumerWarps * (k % R);
-                    const uint32_t phase = static_cast<uint32_t>(k / R) & 1u;
-                    if (mbar_wait_bounded(&sm.empty[stage], phase ^ 1u, sm.abort_flag, a.status) &&
-                        !*sm.abort_flag) {
-                        // every earlier copy into this stage has been consumed, hence landed
-                        issued &= ~(1u << stage);
-                        const bool bad = pi < 0 || pi >= a.num_blocks;
-                        sm.stage_bad[stage] = bad ? 1 : 0;
-                        if (bad) {
-                            atomicOr(a.status, PKV_STATUS_BAD_BLOCK_ID);
-                            mbar_arrive(&sm.full[stage]);
-                        } else {
-                            uint8_t *dst = sm.base + ly.stages + static_cast<uint32_t>(stage) * 2u * kTile;
-                            mbar_arrive_expect_tx(&sm.full[stage], 2u * kTile);
+        const int n = min(32, cur.b1 - cur_b);
+        for (int i = 0; i < n; ++i, ++gb) {
+            const int pi = __shfl_sync(0xffffffffu, p_cur, i);
+            if (lane == 0) {
+                // block gb belongs to consumer warp gb % 4, slot (gb / 4) % R of its ring
+                const int k = gb >> 2;
+                const int stage = (gb & 3) + kConsumerWarps * (k % R);
+                const uint32_t phase = static_cast<uint32_t>(k / R) & 1u;
+                if (mbar_wait_bounded(&sm.empty[stage], phase ^ 1u, sm.abort_flag, a.status) && !*sm.abort_flag) {
+                    // every earlier copy into this stage has been consumed, hence landed
+                    issued &= ~(1u << stage);
+                    const bool bad = pi < 0 || pi >= a.num_blocks;
+                    sm.stage_bad[stage] = bad ? 1 : 0;
+                    if (bad) {
+                        atomicOr(a.status, PKV_STATUS_BAD_BLOCK_ID);
+                        mbar_arrive(&sm.full[stage]);
+                    } else {
+                        uint8_t *dst = sm.base + ly.stages + static_cast<uint32_t>(stage) * 2u * kTile;
+                        mbar_arrive_expect_tx(&sm.full[stage], 2u * kTile);
 #pragma unroll
-                            for (int half = 0; half < D / 64; ++half) {
-                                tma_load_4d(dst + half * kHalf, tm_k, &sm.full[stage], 0, half, it.h, pi * BS);
-                                tma_load_4d(dst + kTile + half * kHalf, tm_v, &sm.full[stage], 0, half, it.h,
-                                            pi * BS);
-                            }
-                            issued |= 1u << stage;
-                            issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+                        for (int half = 0; half < D / 64; ++half) {
+                            tma_load_4d(dst + half * kHalf, tm_k, &sm.full[stage], 0, half, cur.h, pi * BS);
+                            tma_load_4d(dst + kTile + half * kHalf, tm_v, &sm.full[stage], 0, half, cur.h, pi * BS);
                         }
+                        issued |= 1u << stage;
+                        issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
                     }
                 }
             }
         }
+        cur = nxt;
+        cur_b = nxt_b;
+        p_cur = p_nxt;
+        have_cur = have_nxt;
     }
     // Leave no copy in flight into shared memory when the CTA exits.
     if (lane == 0) {
@@ -572,11 +613,10 @@ __device__ __forceinline__ void producer_warp(const CUtensorMap *tm_k, const CUt
 
 template <int D, int BS, class Math>
 __device__ __forceinline__ void consumer_warps(const DecodeArgs &a, const Smem &sm, const DecodeLayout &ly,
-                                               int total_items, int warp, int lane) {
+                                               PieceIter pieces, int warp, int lane) {
     constexpr int GP = Math::GP;
     constexpr uint32_t kTile = BS * D * 2;
     const int R = a.num_stages;  // this warp's ring: stages warp, warp + 4, ..., warp + 4 (R - 1)
-    const int P = a.partition_blocks * BS, cap = a.max_blocks_per_seq * BS;
     const uint32_t sbase = smem_u32(sm.base);
     float *merge_acc = reinterpret_cast<float *>(sm.base + ly.merge_acc);
     float *merge_m = reinterpret_cast<float *>(sm.base + ly.merge_m);
@@ -587,10 +627,9 @@ __device__ __forceinline__ void consumer_warps(const DecodeArgs &a, const Smem &
     Math math;
     math.init(warp, lane, sm.base, ly);
 
-    for (int u = blockIdx.x; u < total_items; u += gridDim.x) {
-        const Item it = decode_item<BS>(u, sm.prefix, a, P, cap);
-        const int nblk = it.b1 - it.b0;
-
+    Piece pc;
+    while (pieces.next(pc)) {
+        const int nblk = pc.b1 - pc.b0;
         mbar_wait_bounded(&sm.qfull[qslot], qphase, sm.abort_flag, a.status);
         math.load_q(sbase + ly.qbuf + qslot * (GP * D * 2), a.group, a.scale_log2);
         __syncwarp();
@@ -601,7 +640,7 @@ __device__ __forceinline__ void consumer_warps(const DecodeArgs &a, const Smem &
         }
         math.reset();
 
-        // this warp's blocks of the item: item-local i with (gb_base + i) % 4 == warp
+        // this warp's blocks of the piece: piece-local i with (gb_base + i) % 4 == warp
         for (int i = (warp - gb_base % kConsumerWarps + kConsumerWarps) % kConsumerWarps; i < nblk;
              i += kConsumerWarps) {
             const int stage = warp + kConsumerWarps * ring;
@@ -612,7 +651,7 @@ __device__ __forceinline__ void consumer_warps(const DecodeArgs &a, const Smem &
             }
             mbar_wait_bounded(&sm.full[stage], par, sm.abort_flag, a.status);
             if (!sm.stage_bad[stage] && !*sm.abort_flag) {
-                const int valid = min(BS, it.tok1 - (it.b0 + i) * BS);
+                const int valid = min(BS, pc.L - (pc.b0 + i) * BS);
                 const uint32_t ktile = sbase + ly.stages + static_cast<uint32_t>(stage) * 2u * kTile;
                 math.block(ktile, ktile + kTile, valid);
             }
@@ -626,7 +665,7 @@ __device__ __forceinline__ void consumer_warps(const DecodeArgs &a, const Smem &
 
         // merge the warps' states (log-sum-exp identity) and store
         const int G = a.group;
-        const bool split_mode = it.n_split > 1;
+        const size_t seg = static_cast<size_t>(pc.s) * a.num_kv_heads + pc.h;
         for (int e = ctid; e < G * D / 2; e += kConsumerWarps * 32) {
             const int g = e / (D / 2), d = (e % (D / 2)) * 2;
             float M = -INFINITY;
@@ -645,12 +684,12 @@ __device__ __forceinline__ void consumer_warps(const DecodeArgs &a, const Smem &
             }
             const float o0 = ls > 0.f ? a0 / ls : 0.f;
             const float o1 = ls > 0.f ? a1 / ls : 0.f;
-            const size_t row = static_cast<size_t>(it.s) * a.num_q_heads + static_cast<size_t>(it.h) * G + g;
-            if (!split_mode) {
+            if (pc.whole) {
+                const size_t row = static_cast<size_t>(pc.s) * a.num_q_heads + static_cast<size_t>(pc.h) * G + g;
                 *reinterpret_cast<__nv_bfloat162 *>(static_cast<__nv_bfloat16 *>(a.out) + row * D + d) =
                     __floats2bfloat162_rn(o0, o1);
             } else {
-                const size_t pr = row * a.n_split + it.split;
+                const size_t pr = (seg + blockIdx.x) * G + g;  // piece (segment + CTA), row g
                 *reinterpret_cast<float2 *>(a.o_part + pr * D + d) = make_float2(o0, o1);
                 if (d == 0) a.lse_part[pr] = ls > 0.f ? M + __log2f(ls) : -INFINITY;
             }
@@ -679,6 +718,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
     sm.abort_flag = sm.stage_bad + kMaxStages;
     sm.scan = reinterpret_cast<int *>(sm.base + ly.flags) + kMaxStages + 1;
     sm.prefix = reinterpret_cast<int *>(sm.base + ly.prefix);
+    sm.lens = reinterpret_cast<int *>(sm.base + ly.lens);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     if (tid == 0) {
@@ -699,9 +739,9 @@ __global__ void __launch_bounds__(kDecodeThreads)
         tma_prefetch_desc(&tm_v);
     }
 
-    // prefix[s] = number of (split) items of sequences < s; every sequence has >= 1
+    // prefix[s] = blocks of sequences < s (clamped lengths); lens[s] = clamped length
     const int S = a.num_seqs;
-    const int P = a.partition_blocks * BS, cap = a.max_blocks_per_seq * BS;
+    const int cap = a.max_blocks_per_seq * BS;
     const int per = (S + kDecodeThreads - 1) / kDecodeThreads;
     const int lo = min(S, tid * per), hi = min(S, lo + per);
     int mine = 0;
@@ -711,7 +751,8 @@ __global__ void __launch_bounds__(kDecodeThreads)
             if (blockIdx.x == 0) atomicOr(a.status, PKV_STATUS_BAD_CONTEXT_LEN);
             L = min(max(L, 0), cap);
         }
-        mine += L > 0 ? (L + P - 1) / P : 1;
+        sm.lens[s] = L;
+        mine += (L + BS - 1) / BS;
     }
     int incl = mine;
 #pragma unroll
@@ -725,8 +766,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
     for (int w = 0; w < warp; ++w) run += sm.scan[w];
     for (int s = lo; s < hi; ++s) {
         sm.prefix[s] = run;
-        int L = min(max(__ldg(a.context_lens + s), 0), cap);
-        run += L > 0 ? (L + P - 1) / P : 1;
+        run += (sm.lens[s] + BS - 1) / BS;
     }
     if (tid == 0) {
         int total = 0;
@@ -734,49 +774,77 @@ __global__ void __launch_bounds__(kDecodeThreads)
         sm.prefix[S] = total;
     }
     __syncthreads();
-    const int total_items = sm.prefix[S] * a.num_kv_heads;
+    if (blockIdx.x == 0)  // the merge kernel locates split segments from the same prefix sums
+        for (int s = tid; s <= S; s += kDecodeThreads) a.seq_blocks[s] = sm.prefix[s];
+
+    const long long B = static_cast<long long>(a.num_kv_heads) * sm.prefix[S];
+    PieceIter pieces;
+    pieces.x = range_begin(blockIdx.x, B, gridDim.x);
+    pieces.x1 = range_begin(blockIdx.x + 1, B, gridDim.x);
+    pieces.pre = sm.prefix;
+    pieces.lens = sm.lens;
+    pieces.S = S;
+    pieces.Hkv = a.num_kv_heads;
 
     if (warp == kConsumerWarps) {
-        producer_warp<D, BS, GP>(&tm_k, &tm_v, a, sm, ly, total_items, lane);
+        producer_warp<D, BS, GP>(&tm_k, &tm_v, a, sm, ly, pieces, lane);
     } else if constexpr (MATH == kMathCudaCore) {
-        consumer_warps<D, BS, CoreMath<D, BS, GP>>(a, sm, ly, total_items, warp, lane);
+        consumer_warps<D, BS, CoreMath<D, BS, GP>>(a, sm, ly, pieces, warp, lane);
     } else {
-        consumer_warps<D, BS, MmaMath<D, BS>>(a, sm, ly, total_items, warp, lane);
+        consumer_warps<D, BS, MmaMath<D, BS>>(a, sm, ly, pieces, warp, lane);
     }
 }
 
-// Merge of split partial results: out = sum_p 2^(lse_p - M) o_p / sum_p 2^(lse_p - M),
-// p = 0 .. n_split(s) - 1 in order. One warp per (sequence, query head).
+// Merge of the pieces of segments that CTA boundaries cut:
+//   out = sum_c 2^(lse_c - M) o_c / sum_c 2^(lse_c - M), c = the CTAs holding
+// pieces of the segment, in order. One warp per (sequence, query head); rows
+// of empty sequences (context length 0) get zeros here.
 template <int D>
-__global__ void __launch_bounds__(256) lse_merge_kernel(const DecodeArgs a, int BS) {
+__global__ void __launch_bounds__(256) lse_merge_kernel(const DecodeArgs a, int num_ctas) {
     constexpr int PER = D / 32;
     const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= a.num_seqs * a.num_q_heads) return;
-    const int s = row / a.num_q_heads;
-    const int P = a.partition_blocks * BS, cap = a.max_blocks_per_seq * BS;
-    const int L = min(max(__ldg(a.context_lens + s), 0), cap);
-    const int n = (L + P - 1) / P;
-    if (n <= 1) return;  // written directly by the decode kernel
-    const float *lse = a.lse_part + static_cast<size_t>(row) * a.n_split;
+    const int s = row / a.num_q_heads, j = row - s * a.num_q_heads;
+    const int G = a.group, h = j / G, g = j - h * G;
+    const int pre_s = a.seq_blocks[s];
+    const int n = a.seq_blocks[s + 1] - pre_s;
+    __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(a.out) + static_cast<size_t>(row) * D + lane * PER;
+    if (n == 0) {
+#pragma unroll
+        for (int i = 0; i < PER; i += 2) *reinterpret_cast<__nv_bfloat162 *>(out + i) = __floats2bfloat162_rn(0.f, 0.f);
+        return;
+    }
+    const long long B = static_cast<long long>(a.num_kv_heads) * a.seq_blocks[a.num_seqs];
+    const long long first_block = static_cast<long long>(a.num_kv_heads) * pre_s + static_cast<long long>(h) * n;
+    // CTA c covers [c B / C, (c + 1) B / C): the CTA of block x is ((x + 1) C - 1) / B
+    const int c0 = static_cast<int>(((first_block + 1) * num_ctas - 1) / B);
+    const int c1 = static_cast<int>(((first_block + n) * num_ctas - 1) / B);
+    if (c0 == c1) return;  // one piece: written directly by the decode kernel
+    // with more CTAs than blocks some CTA ranges are empty: they hold no piece
+    auto holds = [&](int c) { return range_begin(c + 1, B, num_ctas) > range_begin(c, B, num_ctas); };
+    const size_t seg = static_cast<size_t>(s) * a.num_kv_heads + h;
     float M = -INFINITY;
-    for (int p = lane; p < n; p += 32) M = fmaxf(M, lse[p]);
+    for (int c = c0 + lane; c <= c1; c += 32)
+        if (holds(c)) M = fmaxf(M, a.lse_part[(seg + c) * G + g]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float den = 0.f;
-    for (int p = lane; p < n; p += 32) den += fast_exp2(lse[p] - M);
+    for (int c = c0 + lane; c <= c1; c += 32)
+        if (holds(c)) den += fast_exp2(a.lse_part[(seg + c) * G + g] - M);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
     float acc[PER];
 #pragma unroll
     for (int i = 0; i < PER; ++i) acc[i] = 0.f;
-    const float *op = a.o_part + static_cast<size_t>(row) * a.n_split * D + lane * PER;
-    for (int p = 0; p < n; ++p) {
-        const float w = fast_exp2(lse[p] - M);
+    for (int c = c0; c <= c1; ++c) {
+        if (!holds(c)) continue;
+        const size_t pr = (seg + c) * G + g;
+        const float w = fast_exp2(a.lse_part[pr] - M);
+        const float *op = a.o_part + pr * D + lane * PER;
 #pragma unroll
-        for (int i = 0; i < PER; ++i) acc[i] += w * op[static_cast<size_t>(p) * D + i];
+        for (int i = 0; i < PER; ++i) acc[i] += w * op[i];
     }
-    __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(a.out) + static_cast<size_t>(row) * D + lane * PER;
 #pragma unroll
     for (int i = 0; i < PER; i += 2)
         *reinterpret_cast<__nv_bfloat162 *>(out + i) = __floats2bfloat162_rn(acc[i] / den, acc[i + 1] / den);
@@ -840,12 +908,12 @@ cudaError_t decode_launch(int head_dim, int block_size, int group_pad, int math,
     return cudaGetLastError();
 }
 
-cudaError_t lse_merge_launch(int head_dim, int block_size, const DecodeArgs &args, cudaStream_t stream) {
+cudaError_t lse_merge_launch(int head_dim, const DecodeArgs &args, int num_ctas, cudaStream_t stream) {
     const int rows = args.num_seqs * args.num_q_heads;
     const int grid = (rows + 7) / 8;
     if (grid == 0) return cudaSuccess;
-    if (head_dim == 64) lse_merge_kernel<64><<<grid, 256, 0, stream>>>(args, block_size);
-    else lse_merge_kernel<128><<<grid, 256, 0, stream>>>(args, block_size);
+    if (head_dim == 64) lse_merge_kernel<64><<<grid, 256, 0, stream>>>(args, num_ctas);
+    else lse_merge_kernel<128><<<grid, 256, 0, stream>>>(args, num_ctas);
     return cudaGetLastError();
 }
 

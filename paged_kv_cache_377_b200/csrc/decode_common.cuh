@@ -10,8 +10,8 @@ constexpr int kConsumerWarps = 4;                     // warps doing the attenti
 constexpr int kDecodeThreads = 32 * (kConsumerWarps + 1);  // + one TMA producer warp
 constexpr int kMaxStages = 16;                        // KV-block stages per CTA (4 warps x up to 4 each)
 constexpr int kMaxStagesPerWarp = kMaxStages / kConsumerWarps;
-constexpr int kMaxSeqsPerLaunch = 8192;               // prefix-sum table kept in shared memory
-constexpr int kDefaultPartitionTokens = 512;
+constexpr int kMaxSeqsPerLaunch = 2048;               // per-sequence tables kept in shared memory
+constexpr int kMaxCtas = 1024;                        // grid limit; bounds the pieces of a launch
 constexpr int kWorkspaceHeaderBytes = 256;
 
 struct DecodeArgs {
@@ -19,8 +19,9 @@ struct DecodeArgs {
     const void *q;               // bf16 [S][Hq][D]
     const int32_t *block_tables; // [S][MB]
     const int32_t *context_lens; // [S]
-    float *o_part;               // fp32 [S][Hq][n_split][D]
-    float *lse_part;             // fp32 [S][Hq][n_split], log2 domain
+    float *o_part;               // fp32 [piece][G][D], piece = s * Hkv + h + cta
+    float *lse_part;             // fp32 [piece][G], log2 domain
+    int32_t *seq_blocks;         // [S + 1] prefix sums of blocks per sequence, for the merge kernel
     int32_t *status;             // device status word
     int num_seqs;
     int num_q_heads;
@@ -28,14 +29,12 @@ struct DecodeArgs {
     int group;                   // Hq / Hkv
     int max_blocks_per_seq;
     int num_blocks;
-    int partition_blocks;        // partition_tokens / block_size
-    int n_split;                 // ceil(MB * bs / partition_tokens)
     int num_stages;              // ring stages per consumer warp (R); the CTA holds 4R
     float scale_log2;            // scale * log2(e): logits are kept in base 2
 };
 
 struct DecodeLayout {
-    uint32_t stages, qbuf, pscr, merge_acc, merge_m, merge_l, bars, flags, prefix, total;
+    uint32_t stages, qbuf, pscr, merge_acc, merge_m, merge_l, bars, flags, prefix, lens, total;
 };
 
 __host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
@@ -65,7 +64,9 @@ __host__ __device__ inline DecodeLayout decode_layout(int D, int BS, int GP, int
     L.flags = off;
     off += (kMaxStages + 8) * 4;                                    // stage_bad, abort, scan scratch
     L.prefix = off;
-    off += static_cast<uint32_t>(num_seqs + 1) * 4;
+    off += static_cast<uint32_t>(num_seqs + 1) * 4;                 // blocks before each sequence
+    L.lens = off;
+    off += static_cast<uint32_t>(num_seqs) * 4;                     // clamped context lengths
     L.total = align_up(off, 16) + 1024;
     return L;
 }

@@ -26,18 +26,17 @@ def test_library_loads_and_exports_every_declared_symbol():
     assert lib.pkv_version().startswith(b"pagedkv")
 
 
-def _ws(S, Hq, D, MB, bs, P=0):
-    return pkv.workspace_bytes(S, Hq, D, MB, bs, P)
-
-
 def test_workspace_size():
-    assert _ws(4, 2, 64, 3, 16) == 256                        # one split: header only
-    n_split = 8                                                # 256 blocks * 16 / 512
-    rows = 256 * 32
-    assert _ws(256, 32, 128, 256, 16) == 256 + rows * n_split * 128 * 4 + rows * n_split * 4
-    assert _ws(256, 32, 128, 256, 16, P=256) > _ws(256, 32, 128, 256, 16)
-    with pytest.raises(pkv.PagedKVError, match="multiple of block_size"):
-        _ws(4, 2, 64, 3, 16, P=24)
+    # header | prefix sums of one launch (<= 2048 seqs) | fp32 [rows][D] | fp32 [rows], rows = (S + 1024) * Hq
+    def expect(S, Hq, D):
+        sc = min(S, 2048)
+        rows = (sc + 1024) * Hq
+        return 256 + -(-(sc + 1) * 4 // 256) * 256 + rows * D * 4 + -(-rows * 4 // 256) * 256
+    for S, Hq, D in [(4, 2, 64), (256, 32, 128), (3000, 12, 64), (0, 8, 128)]:
+        assert pkv.workspace_bytes(S, Hq, D) == expect(S, Hq, D)
+    assert pkv.workspace_bytes(5000, 8, 128) == pkv.workspace_bytes(2048, 8, 128)
+    with pytest.raises(pkv.PagedKVError, match="num_q_heads"):
+        pkv.workspace_bytes(4, 0, 64)
 
 
 P = ctypes.c_void_p(4096)  # a non-null, aligned address: argument checks never dereference it
@@ -65,6 +64,7 @@ def _decode(**kw):
     (dict(scale=float("inf")), -1, "scale"),
     (dict(q=ctypes.c_void_p(4098)), -1, "aligned"),
     (dict(wsb=16), -1, "workspace_bytes"),
+    (dict(Hkv=2, Hq=2, MB=1 << 20), -1, "too large"),
     (dict(NB=1 << 28), -1, "2^31"),
 ])
 def test_decode_rejects_bad_arguments_without_touching_the_gpu(kw, code, msg):
@@ -89,10 +89,10 @@ def test_append_rejects_bad_arguments():
 
 def test_options_are_checked():
     lib = pkv.library()
-    opts = pkv._binding._Options(24, 0, 0, 0)
+    opts = pkv._binding._Options(2000, 0, 0, 0)
     rc = lib.paged_attn_decode_ex(P, P, P, P, P, P, 4, 2, 1, 64, 16, 0.125, 3, 16, P, 1 << 20,
                                   ctypes.byref(opts), None)
-    assert rc == -1 and "partition_tokens" in lib.pkv_last_error().decode()
+    assert rc == -1 and "num_ctas" in lib.pkv_last_error().decode()
     opts = pkv._binding._Options(0, 5, 0, 0)
     rc = lib.paged_attn_decode_ex(P, P, P, P, P, P, 4, 2, 1, 64, 16, 0.125, 3, 16, P, 1 << 20,
                                   ctypes.byref(opts), None)
@@ -118,4 +118,4 @@ def test_missing_library_fails_loudly(monkeypatch):
     monkeypatch.setattr(_binding._build, "is_stale", lambda: True)
     monkeypatch.setattr(_binding._build, "build", no_build)
     with pytest.raises(RuntimeError, match="nvcc"):
-        pkv.workspace_bytes(1, 1, 64, 1, 16)
+        pkv.workspace_bytes(1, 1, 64)

@@ -31,8 +31,7 @@ def run_step(b, append=True, **opts):
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
     if append:
         pkv.kv_cache_append(b.k_new.to(DEV), b.v_new.to(DEV), kc, vc, b.slot_mapping.to(DEV), status)
-    ws = pkv.allocate_workspace(b.num_seqs, b.num_q_heads, b.head_dim, b.max_blocks_per_seq, b.block_size,
-                                opts.get("partition_tokens", 0))
+    ws = pkv.allocate_workspace(b.num_seqs, b.num_q_heads, b.head_dim)
     out = torch.full_like(q, float("nan"))
     pkv.paged_attn_decode(out, q, kc, vc, bt, cl, b.scale, ws, **opts)
     torch.cuda.synchronize()
@@ -64,16 +63,18 @@ def test_config_parity(name, math):
 
 @pytest.mark.parametrize("math", MATHS)
 @pytest.mark.parametrize("name", ["tiny", "opt125m", "qwen25_7b_prefix", "skewed_long"])
-@pytest.mark.parametrize("partition_tokens", [32, 64, 1 << 20])
-def test_forced_split_sizes(name, partition_tokens, math):
+@pytest.mark.parametrize("num_ctas", [1, 7, 300, 1024])
+def test_grid_sizes_split_contexts_differently(name, num_ctas, math):
+    """num_ctas sets how the batch's blocks are cut between CTAs: 1 CTA splits
+    nothing; 1024 CTAs cut most contexts into several merged pieces."""
     b, ref, _, _ = config_case(name)
-    out, _, _, st = run_step(b, partition_tokens=partition_tokens, math=math)
+    out, _, _, st = run_step(b, num_ctas=num_ctas, math=math)
     assert st == 0
-    assert_close_to_oracle(out.double().numpy(), ref, what=f"{name} P={partition_tokens}")
+    assert_close_to_oracle(out.double().numpy(), ref, what=f"{name} num_ctas={num_ctas}")
 
 
 @pytest.mark.parametrize("opts", [dict(num_stages=1), dict(num_stages=2), dict(num_stages=4), dict(ctas_per_sm=1),
-                                  dict(num_stages=3, ctas_per_sm=2, partition_tokens=128),
+                                  dict(num_stages=3, ctas_per_sm=2, num_ctas=100),
                                   dict(math=2, num_stages=1), dict(math=2, num_stages=4, ctas_per_sm=1)])
 def test_launch_options(opts):
     b, ref, _, _ = config_case("opt125m")
@@ -99,10 +100,10 @@ def test_every_group_size_and_shape(G, D, bs):
     b = workloads.make_custom(1000 + G * 7 + D + bs, lens, 2 * G, 2, D, bs)
     ref, _, _ = oracle.decode_step(b)
     for math in MATHS:
-        for P in (0, 2 * bs):
-            out, _, _, st = run_step(b, partition_tokens=P, math=math)
+        for num_ctas in (0, 37):
+            out, _, _, st = run_step(b, num_ctas=num_ctas, math=math)
             assert st == 0
-            assert_close_to_oracle(out.double().numpy(), ref, what=f"G={G} D={D} bs={bs} P={P} math={math}")
+            assert_close_to_oracle(out.double().numpy(), ref, what=f"G={G} D={D} bs={bs} C={num_ctas} math={math}")
 
 
 @pytest.mark.parametrize("math", MATHS)

@@ -23,8 +23,7 @@ def _decode_both(b, dev):
     q = b.q.to(dev)
     bt, cl = b.block_tables.to(dev), b.context_lens.to(dev)
     pkv.kv_cache_append(b.k_new.to(dev), b.v_new.to(dev), kc, vc, b.slot_mapping.to(dev))
-    ws = pkv.allocate_workspace(b.num_seqs, b.num_q_heads, b.head_dim, b.max_blocks_per_seq, b.block_size,
-                                device=dev)
+    ws = pkv.allocate_workspace(b.num_seqs, b.num_q_heads, b.head_dim, device=dev)
     assert ws.numel() <= SCRATCH_BYTES
     with_ws = torch.empty_like(q)
     pkv.paged_attn_decode(with_ws, q, kc, vc, bt, cl, b.scale, ws)
@@ -41,8 +40,8 @@ def _decode_both(b, dev):
 @pytest.mark.gpu
 def test_noalloc_matches_the_workspace_entry_point_on_two_calls_in_a_row():
     dev = torch.device("cuda", torch.cuda.current_device())
-    # the first call leaves 8-way split partials behind in the scratch; the
-    # second has a different shape and fewer splits
+    # the first call leaves split partials behind in the scratch; the second
+    # has a different shape and cuts its contexts differently
     for name in ("llama3_8b", "opt125m"):
         b = workloads.make_batch(name, device=dev)
         with_ws, no_ws, status, ws_status = _decode_both(b, dev)
@@ -51,15 +50,15 @@ def test_noalloc_matches_the_workspace_entry_point_on_two_calls_in_a_row():
 
 
 def test_noalloc_rejects_batches_beyond_its_scratch():
-    """The skewed long-context shape needs ~270 MB of split partials: refused on the host, nothing enqueued."""
+    """2048 sequences of 64 query heads need ~100 MB of workspace: refused on the host, nothing enqueued."""
     lib = pkv.library()
     import ctypes
     P = ctypes.c_void_p(4096)
     from paged_kv_cache_377_b200._binding import paged_attn_decode_noalloc  # noqa: F401  (sets argtypes lazily)
     lib.paged_attn_decode_noalloc.argtypes = [ctypes.c_void_p] * 6 + [ctypes.c_int] * 5 + [ctypes.c_float] + \
         [ctypes.c_int] * 2 + [ctypes.c_void_p] * 2
-    rc = lib.paged_attn_decode_noalloc(P, P, P, P, P, P, 128, 32, 8, 128, 32, 0.088, 2048, 5081, None, None)
+    rc = lib.paged_attn_decode_noalloc(P, P, P, P, P, P, 2048, 64, 8, 128, 16, 0.088, 256, 50000, None, None)
     msg = lib.pkv_last_error().decode()
     assert rc == -1 and "static scratch" in msg and str(SCRATCH_BYTES) in msg, msg
-    need = pkv.workspace_bytes(128, 32, 128, 2048, 32)
+    need = pkv.workspace_bytes(2048, 64, 128)
     assert need > SCRATCH_BYTES and str(need) in msg
