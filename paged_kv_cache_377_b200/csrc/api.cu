@@ -197,7 +197,7 @@ int paged_attn_decode_ex(void *out, const void *q, const void *k_cache, const vo
     // in shared memory); launches run in stream order and reuse the workspace.
     for (int s0 = 0; s0 < num_seqs; s0 += pkv::kMaxSeqsPerLaunch) {
         const int sc = num_seqs - s0 < pkv::kMaxSeqsPerLaunch ? num_seqs - s0 : pkv::kMaxSeqsPerLaunch;
-        const size_t smem = pkv::decode_smem_bytes(head_dim, block_size, gp, math, ns, sc);
+        const size_t smem = pkv::decode_smem_bytes(head_dim, block_size, gp, group, math, ns, sc);
         int per_sm = 0;
         cudaError_t e = pkv::decode_prepare(head_dim, block_size, gp, math, smem, &per_sm);
         if (e != cudaSuccess) return cuda_fail(e, "decode kernel setup");

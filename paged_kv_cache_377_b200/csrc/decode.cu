@@ -16,17 +16,14 @@
 //     "piece". Every CTA rebuilds the per-sequence block prefix sums in shared
 //     memory, so no planning kernel and no host/device synchronisation are
 //     needed.
-//   * One producer warp streams whole KV blocks of the item's kv head into
-//     shared memory with TMA (4D tile copies of 64 columns, 128-byte swizzle),
-//     completing on mbarriers. Block-table entries are read 32 at a time by the
-//     warp's lanes, one 32-block chunk ahead of the chunk being issued. The
-//     producer runs ahead across piece boundaries, so HBM stays busy while
-//     consumers merge.
-//   * Four consumer warps take the blocks round-robin (block g of the CTA's
-//     stream goes to warp g % 4) and each warp owns its own ring of R stages,
-//     so every waiter sees every phase of its barriers in order (a parity wait
-//     can never alias a phase two steps ahead). Each warp keeps its own
-//     online-softmax state (running max m, running sum l, fp32 accumulator)
+//   * Four warps per CTA take the blocks round-robin (block g of the CTA's
+//     range goes to warp g % 4). Each warp owns a ring of R shared-memory
+//     stages and streams its own blocks into it with TMA (4D tile copies of 64
+//     columns, 128-byte swizzle), R blocks ahead of the one it computes and
+//     across piece boundaries, completing on mbarriers; block-table entries
+//     are looked up 32 blocks at a time, one batch ahead. No warp waits for
+//     another to refill its stages, and each waiter sees every phase of its
+//     barriers in order. Each warp keeps its own online-softmax state (running max m, running sum l, fp32 accumulator)
 //     for all G query heads of the GQA group (Milakov & Gimelshein 2018,
 //     "Online normalizer calculation for softmax"). Logits are kept in base 2
 //     (scale * log2 e folded in).
@@ -280,8 +277,8 @@ struct CoreMath {
         __syncwarp();
     }
 
-    // This warp's (m, l, acc) into the merge area ([warp][GP][D] etc).
-    __device__ __forceinline__ void export_state(float *merge_acc, float *merge_m, float *merge_l, int warp) {
+    // This warp's (m, l, acc) into the merge area ([warp][G][D], [warp][G]).
+    __device__ __forceinline__ void export_state(float *merge_acc, float *merge_m, float *merge_l, int warp, int G) {
         // token groups of a warp share m_run: their accumulators just add
 #pragma unroll
         for (int o = LPT; o < 32; o <<= 1)
@@ -295,16 +292,19 @@ struct CoreMath {
         if (tg == 0) {
 #pragma unroll
             for (int g = 0; g < GP; ++g) {
-                float4 *dst = reinterpret_cast<float4 *>(merge_acc + (warp * GP + g) * D + ch * 8);
-                dst[0] = make_float4(acc[g][0].x, acc[g][0].y, acc[g][1].x, acc[g][1].y);
-                dst[1] = make_float4(acc[g][2].x, acc[g][2].y, acc[g][3].x, acc[g][3].y);
+                if (g < G) {
+                    float4 *dst = reinterpret_cast<float4 *>(merge_acc + (warp * G + g) * D + ch * 8);
+                    dst[0] = make_float4(acc[g][0].x, acc[g][0].y, acc[g][1].x, acc[g][1].y);
+                    dst[1] = make_float4(acc[g][2].x, acc[g][2].y, acc[g][3].x, acc[g][3].y);
+                }
             }
         }
         if (lane == 0) {
 #pragma unroll
-            for (int g = 0; g < GP; ++g) merge_m[warp * GP + g] = m_run[g];
+            for (int g = 0; g < GP; ++g)
+                if (g < G) merge_m[warp * G + g] = m_run[g];
         }
-        if (lane < GP) merge_l[warp * GP + lane] = l_run;
+        if (lane < G) merge_l[warp * G + lane] = l_run;
     }
 };
 
@@ -480,7 +480,7 @@ struct MmaMath {
         __syncwarp();  // P scratch is rewritten by the next block
     }
 
-    __device__ __forceinline__ void export_state(float *merge_acc, float *merge_m, float *merge_l, int warp) {
+    __device__ __forceinline__ void export_state(float *merge_acc, float *merge_m, float *merge_l, int warp, int G) {
 #pragma unroll
         for (int o = 4; o < 32; o <<= 1) {
             l0 += __shfl_xor_sync(0xffffffffu, l0, o);
@@ -488,19 +488,27 @@ struct MmaMath {
         }
         const int g0 = 2 * (lane & 3), dr = lane >> 2;
         if (lane < 4) {
-            merge_m[warp * GP + g0] = m0;
-            merge_m[warp * GP + g0 + 1] = m1;
-            merge_l[warp * GP + g0] = l0;
-            merge_l[warp * GP + g0 + 1] = l1;
+            if (g0 < G) {
+                merge_m[warp * G + g0] = m0;
+                merge_l[warp * G + g0] = l0;
+            }
+            if (g0 + 1 < G) {
+                merge_m[warp * G + g0 + 1] = m1;
+                merge_l[warp * G + g0 + 1] = l1;
+            }
         }
-        float *r0 = merge_acc + (warp * GP + g0) * D;
+        float *r0 = merge_acc + (warp * G + g0) * D;
         float *r1 = r0 + D;
 #pragma unroll
         for (int dt = 0; dt < DT; ++dt) {
-            r0[16 * dt + dr] = acc[dt][0];
-            r1[16 * dt + dr] = acc[dt][1];
-            r0[16 * dt + dr + 8] = acc[dt][2];
-            r1[16 * dt + dr + 8] = acc[dt][3];
+            if (g0 < G) {
+                r0[16 * dt + dr] = acc[dt][0];
+                r0[16 * dt + dr + 8] = acc[dt][2];
+            }
+            if (g0 + 1 < G) {
+                r1[16 * dt + dr] = acc[dt][1];
+                r1[16 * dt + dr + 8] = acc[dt][3];
+            }
         }
     }
 };
@@ -509,7 +517,7 @@ struct MmaMath {
 
 struct Smem {
     uint8_t *base;
-    uint64_t *full, *empty, *qfull, *qempty;
+    uint64_t *full, *qfull;
     volatile int *stage_bad;
     volatile int *abort_flag;
     int *scan;
@@ -517,167 +525,153 @@ struct Smem {
     int *lens;
 };
 
-template <int D, int BS, int GP>
-__device__ __forceinline__ void producer_warp(const CUtensorMap *tm_k, const CUtensorMap *tm_v, const DecodeArgs &a,
-                                              const Smem &sm, const DecodeLayout &ly, PieceIter pieces, int lane) {
+// One decode warp. Warp w owns the blocks x0 + w + 4k (k = 0, 1, ...) of the
+// CTA's range and a ring of R shared-memory stages (stage w + 4 (k % R)). It
+// issues the TMA copies of its own blocks R ahead of the one it computes --
+// block k + R goes into the stage block k just freed -- so it waits on no other
+// warp to refill its ring. Block-table entries of its next 32 blocks are looked
+// up one batch ahead. Warp 0 also bulk-copies the query rows of the piece after
+// next. All four warps meet at the end of every piece to merge their states.
+template <int D, int BS, class Math>
+__device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUtensorMap *tm_v, const DecodeArgs &a,
+                                            const Smem &sm, const DecodeLayout &ly, PieceIter pieces, long long x0,
+                                            long long x1, int warp, int lane) {
     constexpr uint32_t kTile = BS * D * 2;
     constexpr uint32_t kHalf = BS * 128;
-    const int R = a.num_stages;  // stages per consumer warp
-    const uint32_t qbytes = static_cast<uint32_t>(a.group * D * 2);
-    int qslot = 0, gb = 0;
-    uint32_t qphase = 0;
-    uint32_t issued = 0, issued_par = 0, q_issued = 0, q_issued_par = 0;  // copies possibly in flight
-
-    // Table entries come in chunks of up to 32 blocks of one piece; the next
-    // chunk's entries are loaded while the current chunk is issued.
-    Piece cur, nxt;
-    bool have_cur = pieces.next(cur), have_nxt = false;
-    int cur_b = have_cur ? cur.b0 : 0;          // first block of the current chunk
-    int p_cur = -1, p_nxt = -1;
-    auto load = [&](const Piece &pc, int b) {
-        const int idx = b + lane;
-        return idx < pc.b1 ? __ldg(a.block_tables + static_cast<size_t>(pc.s) * a.max_blocks_per_seq + idx) : 0;
-    };
-    if (have_cur) p_cur = load(cur, cur_b);
-    while (have_cur) {
-        // the chunk after this one: same piece, or the first chunk of the next piece
-        int nxt_b;
-        if (cur_b + 32 < cur.b1) {
-            nxt = cur;
-            nxt_b = cur_b + 32;
-            have_nxt = true;
-        } else {
-            have_nxt = pieces.next(nxt);
-            nxt_b = have_nxt ? nxt.b0 : 0;
-        }
-        if (have_nxt) p_nxt = load(nxt, nxt_b);
-
-        if (cur_b == cur.b0 && lane == 0) {  // first chunk of a piece: its query rows
-            if (mbar_wait_bounded(&sm.qempty[qslot], qphase ^ 1u, sm.abort_flag, a.status) && !*sm.abort_flag) {
-                const __nv_bfloat16 *src = static_cast<const __nv_bfloat16 *>(a.q) +
-                                           (static_cast<size_t>(cur.s) * a.num_q_heads +
-                                            static_cast<size_t>(cur.h) * a.group) * D;
-                mbar_arrive_expect_tx(&sm.qfull[qslot], qbytes);
-                bulk_load(sm.base + ly.qbuf + qslot * (GP * D * 2), src, qbytes, &sm.qfull[qslot]);
-                q_issued |= 1u << qslot;
-                q_issued_par = (q_issued_par & ~(1u << qslot)) | (qphase << qslot);
-            }
-        }
-        if (cur_b == cur.b0 && ++qslot == 2) {
-            qslot = 0;
-            qphase ^= 1u;
-        }
-        const int n = min(32, cur.b1 - cur_b);
-        for (int i = 0; i < n; ++i, ++gb) {
-            const int pi = __shfl_sync(0xffffffffu, p_cur, i);
-            if (lane == 0) {
-                // block gb belongs to consumer warp gb % 4, slot (gb / 4) % R of its ring
-                const int k = gb >> 2;
-                const int stage = (gb & 3) + kConsumerWarps * (k % R);
-                const uint32_t phase = static_cast<uint32_t>(k / R) & 1u;
-                if (mbar_wait_bounded(&sm.empty[stage], phase ^ 1u, sm.abort_flag, a.status) && !*sm.abort_flag) {
-                    // every earlier copy into this stage has been consumed, hence landed
-                    issued &= ~(1u << stage);
-                    const bool bad = pi < 0 || pi >= a.num_blocks;
-                    sm.stage_bad[stage] = bad ? 1 : 0;
-                    if (bad) {
-                        atomicOr(a.status, PKV_STATUS_BAD_BLOCK_ID);
-                        mbar_arrive(&sm.full[stage]);
-                    } else {
-                        uint8_t *dst = sm.base + ly.stages + static_cast<uint32_t>(stage) * 2u * kTile;
-                        mbar_arrive_expect_tx(&sm.full[stage], 2u * kTile);
-#pragma unroll
-                        for (int half = 0; half < D / 64; ++half) {
-                            tma_load_4d(dst + half * kHalf, tm_k, &sm.full[stage], 0, half, cur.h, pi * BS);
-                            tma_load_4d(dst + kTile + half * kHalf, tm_v, &sm.full[stage], 0, half, cur.h, pi * BS);
-                        }
-                        issued |= 1u << stage;
-                        issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
-                    }
-                }
-            }
-        }
-        cur = nxt;
-        cur_b = nxt_b;
-        p_cur = p_nxt;
-        have_cur = have_nxt;
-    }
-    // Leave no copy in flight into shared memory when the CTA exits.
-    if (lane == 0) {
-        for (int st = 0; st < kConsumerWarps * R; ++st)
-            if ((issued >> st) & 1u) mbar_wait_drain(&sm.full[st], (issued_par >> st) & 1u, a.status);
-        for (int qs = 0; qs < 2; ++qs)
-            if ((q_issued >> qs) & 1u) mbar_wait_drain(&sm.qfull[qs], (q_issued_par >> qs) & 1u, a.status);
-    }
-}
-
-template <int D, int BS, class Math>
-__device__ __forceinline__ void consumer_warps(const DecodeArgs &a, const Smem &sm, const DecodeLayout &ly,
-                                               PieceIter pieces, int warp, int lane) {
-    constexpr int GP = Math::GP;
-    constexpr uint32_t kTile = BS * D * 2;
-    const int R = a.num_stages;  // this warp's ring: stages warp, warp + 4, ..., warp + 4 (R - 1)
+    const int R = a.num_stages;
+    const int G = a.group;
+    const uint32_t qbytes = static_cast<uint32_t>(G * D * 2);
     const uint32_t sbase = smem_u32(sm.base);
     float *merge_acc = reinterpret_cast<float *>(sm.base + ly.merge_acc);
     float *merge_m = reinterpret_cast<float *>(sm.base + ly.merge_m);
     float *merge_l = reinterpret_cast<float *>(sm.base + ly.merge_l);
     const int ctid = warp * 32 + lane;
-    int qslot = 0, gb_base = 0, ring = 0;
-    uint32_t qphase = 0, rphase = 0;
+
+    // ---- issue side: this warp's blocks k = 0 .. nk-1 are global blocks x0 + warp + 4k
+    const long long span = x1 - x0;
+    const int nk = span > warp ? static_cast<int>((span - warp + kConsumerWarps - 1) / kConsumerWarps) : 0;
+    auto lookup = [&](int kb, int &p, int &h) {  // lane j: block kb + j -> (physical block, kv head)
+        p = 0;
+        h = 0;
+        const int k = kb + lane;
+        if (k < nk) {
+            const long long x = x0 + warp + static_cast<long long>(kConsumerWarps) * k;
+            int lo = 0, hi = a.num_seqs - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (static_cast<long long>(a.num_kv_heads) * sm.prefix[mid] <= x) lo = mid;
+                else hi = mid - 1;
+            }
+            const int n = sm.prefix[lo + 1] - sm.prefix[lo];
+            const int r = static_cast<int>(x - static_cast<long long>(a.num_kv_heads) * sm.prefix[lo]);
+            h = r / n;
+            p = __ldg(a.block_tables + static_cast<size_t>(lo) * a.max_blocks_per_seq + (r - h * n));
+        }
+    };
+    int bat_k = 0, bat_p, bat_h, nxt_p, nxt_h;
+    lookup(0, bat_p, bat_h);
+    lookup(32, nxt_p, nxt_h);
+    uint32_t inflight = 0, inflight_par = 0;  // stages whose copy this warp issued and has not yet seen land
+    auto issue = [&](int k) {                 // warp-uniform; k increases call after call
+        if (k >= nk) return;
+        if (k - bat_k >= 32) {
+            bat_k += 32;
+            bat_p = nxt_p;
+            bat_h = nxt_h;
+            lookup(bat_k + 32, nxt_p, nxt_h);
+        }
+        const int p = __shfl_sync(0xffffffffu, bat_p, k - bat_k);
+        const int h = __shfl_sync(0xffffffffu, bat_h, k - bat_k);
+        const int stage = warp + kConsumerWarps * (k % R);
+        const uint32_t par = static_cast<uint32_t>(k / R) & 1u;
+        if (lane == 0 && !*sm.abort_flag) {
+            const bool bad = p < 0 || p >= a.num_blocks;
+            sm.stage_bad[stage] = bad ? 1 : 0;
+            if (bad) {
+                atomicOr(a.status, PKV_STATUS_BAD_BLOCK_ID);
+                mbar_arrive(&sm.full[stage]);
+            } else {
+                uint8_t *dst = sm.base + ly.stages + static_cast<uint32_t>(stage) * 2u * kTile;
+                fence_proxy_async_shared();  // this warp's reads of the stage come before the copy
+                mbar_arrive_expect_tx(&sm.full[stage], 2u * kTile);
+#pragma unroll
+                for (int half = 0; half < D / 64; ++half) {
+                    tma_load_4d(dst + half * kHalf, tm_k, &sm.full[stage], 0, half, h, p * BS);
+                    tma_load_4d(dst + kTile + half * kHalf, tm_v, &sm.full[stage], 0, half, h, p * BS);
+                }
+                inflight |= 1u << stage;
+                inflight_par = (inflight_par & ~(1u << stage)) | (par << stage);
+            }
+        }
+    };
+    for (int k = 0; k < R; ++k) issue(k);
+
+    // ---- query rows: warp 0 copies piece n + 1's rows while piece n is computed
+    uint32_t q_issued = 0, q_issued_par = 0;
+    PieceIter ahead = pieces;
+    Piece pa{};
+    auto issue_q = [&](int n) {  // piece n's rows into slot n % 2 (ahead has just returned piece n)
+        if (warp == 0 && lane == 0 && !*sm.abort_flag) {
+            const int slot = n & 1;
+            const __nv_bfloat16 *src = static_cast<const __nv_bfloat16 *>(a.q) +
+                                       (static_cast<size_t>(pa.s) * a.num_q_heads + static_cast<size_t>(pa.h) * G) * D;
+            fence_proxy_async_shared();
+            mbar_arrive_expect_tx(&sm.qfull[slot], qbytes);
+            bulk_load(sm.base + ly.qbuf + slot * qbytes, src, qbytes, &sm.qfull[slot]);
+            q_issued |= 1u << slot;
+            q_issued_par = (q_issued_par & ~(1u << slot)) | ((static_cast<uint32_t>(n >> 1) & 1u) << slot);
+        }
+    };
+    int n_ahead = 0;
+    if (ahead.next(pa)) issue_q(n_ahead++);
+    if (ahead.next(pa)) issue_q(n_ahead++);
+
+    // ---- compute side
     Math math;
     math.init(warp, lane, sm.base, ly);
-
+    int k = 0, gb_base = 0, npiece = 0;
     Piece pc;
     while (pieces.next(pc)) {
-        const int nblk = pc.b1 - pc.b0;
-        mbar_wait_bounded(&sm.qfull[qslot], qphase, sm.abort_flag, a.status);
-        math.load_q(sbase + ly.qbuf + qslot * (GP * D * 2), a.group, a.scale_log2);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.qempty[qslot]);
-        if (++qslot == 2) {
-            qslot = 0;
-            qphase ^= 1u;
-        }
+        const int slot = npiece & 1;
+        if (npiece >= 1 && ahead.next(pa)) issue_q(n_ahead++);  // every warp has read slot (npiece + 1) % 2
+        mbar_wait_bounded(&sm.qfull[slot], static_cast<uint32_t>(npiece >> 1) & 1u, sm.abort_flag, a.status);
+        math.load_q(sbase + ly.qbuf + slot * qbytes, G, a.scale_log2);
         math.reset();
+        ++npiece;
 
-        // this warp's blocks of the piece: piece-local i with (gb_base + i) % 4 == warp
+        const int nblk = pc.b1 - pc.b0;
         for (int i = (warp - gb_base % kConsumerWarps + kConsumerWarps) % kConsumerWarps; i < nblk;
-             i += kConsumerWarps) {
-            const int stage = warp + kConsumerWarps * ring;
-            const uint32_t par = rphase;
-            if (++ring == R) {
-                ring = 0;
-                rphase ^= 1u;
-            }
-            mbar_wait_bounded(&sm.full[stage], par, sm.abort_flag, a.status);
+             i += kConsumerWarps, ++k) {
+            const int stage = warp + kConsumerWarps * (k % R);
+            const uint32_t par = static_cast<uint32_t>(k / R) & 1u;
+            if (mbar_wait_bounded(&sm.full[stage], par, sm.abort_flag, a.status)) inflight &= ~(1u << stage);
             if (!sm.stage_bad[stage] && !*sm.abort_flag) {
                 const int valid = min(BS, pc.L - (pc.b0 + i) * BS);
                 const uint32_t ktile = sbase + ly.stages + static_cast<uint32_t>(stage) * 2u * kTile;
                 math.block(ktile, ktile + kTile, valid);
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.empty[stage]);
+            issue(k + R);  // the stage just freed takes this warp's block k + R
         }
         gb_base += nblk;
 
-        math.export_state(merge_acc, merge_m, merge_l, warp);
+        math.export_state(merge_acc, merge_m, merge_l, warp, G);
         named_barrier_sync(1, kConsumerWarps * 32);
 
         // merge the warps' states (log-sum-exp identity) and store
-        const int G = a.group;
         const size_t seg = static_cast<size_t>(pc.s) * a.num_kv_heads + pc.h;
         for (int e = ctid; e < G * D / 2; e += kConsumerWarps * 32) {
             const int g = e / (D / 2), d = (e % (D / 2)) * 2;
             float M = -INFINITY;
 #pragma unroll
-            for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, merge_m[w * GP + g]);
+            for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, merge_m[w * G + g]);
             float ls = 0.f, a0 = 0.f, a1 = 0.f;
             if (M != -INFINITY) {
 #pragma unroll
                 for (int w = 0; w < kConsumerWarps; ++w) {
-                    const float f = fast_exp2(merge_m[w * GP + g] - M);
-                    const float2 av = *reinterpret_cast<const float2 *>(merge_acc + (w * GP + g) * D + d);
-                    ls += merge_l[w * GP + g] * f;
+                    const float f = fast_exp2(merge_m[w * G + g] - M);
+                    const float2 av = *reinterpret_cast<const float2 *>(merge_acc + (w * G + g) * D + d);
+                    ls += merge_l[w * G + g] * f;
                     a0 += av.x * f;
                     a1 += av.y * f;
                 }
@@ -696,6 +690,16 @@ __device__ __forceinline__ void consumer_warps(const DecodeArgs &a, const Smem &
         }
         named_barrier_sync(1, kConsumerWarps * 32);
     }
+    // Leave no copy in flight into shared memory when the CTA exits (only
+    // possible after a wait gave up).
+    if (lane == 0) {
+        for (int st = 0; st < kMaxStages; ++st)
+            if ((inflight >> st) & 1u) mbar_wait_drain(&sm.full[st], (inflight_par >> st) & 1u, a.status);
+        // the last copy into each query slot: landed already unless a wait gave up
+        if (warp == 0)
+            for (int slot = 0; slot < 2; ++slot)
+                if ((q_issued >> slot) & 1u) mbar_wait_drain(&sm.qfull[slot], (q_issued_par >> slot) & 1u, a.status);
+    }
 }
 
 template <int D, int BS, int GP, int MATH>
@@ -707,13 +711,12 @@ __global__ void __launch_bounds__(kDecodeThreads)
     static_assert(GP == 1 || GP == 2 || GP == 4 || GP == 8, "group");
     static_assert(MATH == kMathCudaCore || GP == 8, "the tensor-core path pads the group to 8");
     extern __shared__ uint8_t smem_raw[];
-    const DecodeLayout ly = decode_layout(D, BS, GP, kConsumerWarps * a.num_stages, a.num_seqs);
+    const DecodeLayout ly = decode_layout(D, BS, GP, a.group, MATH == kMathTensorCore, kConsumerWarps * a.num_stages,
+                                          a.num_seqs);
     Smem sm;
     sm.base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     sm.full = reinterpret_cast<uint64_t *>(sm.base + ly.bars);
-    sm.empty = sm.full + kMaxStages;
-    sm.qfull = sm.empty + kMaxStages;
-    sm.qempty = sm.qfull + 2;
+    sm.qfull = sm.full + kMaxStages;
     sm.stage_bad = reinterpret_cast<volatile int *>(sm.base + ly.flags);
     sm.abort_flag = sm.stage_bad + kMaxStages;
     sm.scan = reinterpret_cast<int *>(sm.base + ly.flags) + kMaxStages + 1;
@@ -724,17 +727,13 @@ __global__ void __launch_bounds__(kDecodeThreads)
     if (tid == 0) {
         for (int i = 0; i < kConsumerWarps * a.num_stages; ++i) {
             mbar_init(&sm.full[i], 1);
-            mbar_init(&sm.empty[i], 1);
             sm.stage_bad[i] = 0;
         }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&sm.qfull[i], 1);
-            mbar_init(&sm.qempty[i], kConsumerWarps);
-        }
+        for (int i = 0; i < 2; ++i) mbar_init(&sm.qfull[i], 1);
         *sm.abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == kConsumerWarps && lane == 0) {
+    if (tid == 32) {
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
     }
@@ -778,20 +777,19 @@ __global__ void __launch_bounds__(kDecodeThreads)
         for (int s = tid; s <= S; s += kDecodeThreads) a.seq_blocks[s] = sm.prefix[s];
 
     const long long B = static_cast<long long>(a.num_kv_heads) * sm.prefix[S];
+    const long long x0 = range_begin(blockIdx.x, B, gridDim.x), x1 = range_begin(blockIdx.x + 1, B, gridDim.x);
     PieceIter pieces;
-    pieces.x = range_begin(blockIdx.x, B, gridDim.x);
-    pieces.x1 = range_begin(blockIdx.x + 1, B, gridDim.x);
+    pieces.x = x0;
+    pieces.x1 = x1;
     pieces.pre = sm.prefix;
     pieces.lens = sm.lens;
     pieces.S = S;
     pieces.Hkv = a.num_kv_heads;
 
-    if (warp == kConsumerWarps) {
-        producer_warp<D, BS, GP>(&tm_k, &tm_v, a, sm, ly, pieces, lane);
-    } else if constexpr (MATH == kMathCudaCore) {
-        consumer_warps<D, BS, CoreMath<D, BS, GP>>(a, sm, ly, pieces, warp, lane);
+    if constexpr (MATH == kMathCudaCore) {
+        decode_warp<D, BS, CoreMath<D, BS, GP>>(&tm_k, &tm_v, a, sm, ly, pieces, x0, x1, warp, lane);
     } else {
-        consumer_warps<D, BS, MmaMath<D, BS>>(a, sm, ly, pieces, warp, lane);
+        decode_warp<D, BS, MmaMath<D, BS>>(&tm_k, &tm_v, a, sm, ly, pieces, x0, x1, warp, lane);
     }
 }
 
@@ -873,9 +871,10 @@ bool decode_variant_exists(int head_dim, int block_size, int group_pad, int math
     return pick(head_dim, block_size, effective_group_pad(group_pad, math), math) != nullptr;
 }
 
-size_t decode_smem_bytes(int head_dim, int block_size, int group_pad, int math, int num_stages, int num_seqs) {
-    return decode_layout(head_dim, block_size, effective_group_pad(group_pad, math), kConsumerWarps * num_stages,
-                         num_seqs)
+size_t decode_smem_bytes(int head_dim, int block_size, int group_pad, int group, int math, int num_stages,
+                         int num_seqs) {
+    return decode_layout(head_dim, block_size, effective_group_pad(group_pad, math), group, math == kMathTensorCore,
+                         kConsumerWarps * num_stages, num_seqs)
         .total;
 }
 

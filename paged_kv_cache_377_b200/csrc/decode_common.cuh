@@ -6,8 +6,8 @@
 
 namespace pkv {
 
-constexpr int kConsumerWarps = 4;                     // warps doing the attention math
-constexpr int kDecodeThreads = 32 * (kConsumerWarps + 1);  // + one TMA producer warp
+constexpr int kConsumerWarps = 4;                     // warps of a decode CTA (each loads and computes)
+constexpr int kDecodeThreads = 32 * kConsumerWarps;
 constexpr int kMaxStages = 16;                        // KV-block stages per CTA (4 warps x up to 4 each)
 constexpr int kMaxStagesPerWarp = kMaxStages / kConsumerWarps;
 constexpr int kMaxSeqsPerLaunch = 2048;               // per-sequence tables kept in shared memory
@@ -40,27 +40,30 @@ struct DecodeLayout {
 __host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
 // Byte offsets from a 1024-byte aligned base. `total` includes 1024 bytes of
-// slack for aligning the dynamic shared-memory base.
-__host__ __device__ inline DecodeLayout decode_layout(int D, int BS, int GP, int num_stages, int num_seqs) {
+// slack for aligning the dynamic shared-memory base. GP = compile-time padded
+// group, G = the actual group (query heads per kv head), tensor_core = the
+// mma.sync math path (its probability scratch is bf16 [8][BS] per warp).
+__host__ __device__ inline DecodeLayout decode_layout(int D, int BS, int GP, int G, bool tensor_core, int num_stages,
+                                                      int num_seqs) {
     DecodeLayout L;
     uint32_t off = 0;
     const uint32_t tile = static_cast<uint32_t>(BS * D * 2);
     L.stages = off;
     off += static_cast<uint32_t>(num_stages) * 2u * tile;          // [stage][K tile, V tile]
     L.qbuf = off;
-    off += 2u * GP * D * 2;                                         // two query slots [GP][D] bf16
+    off += 2u * G * D * 2;                                          // two query slots [G][D] bf16
     off = align_up(off, 16);
     L.pscr = off;
-    off += kConsumerWarps * BS * GP * 8;                            // per warp float2 [BS][GP]
+    off += kConsumerWarps * (tensor_core ? BS * 16 : BS * GP * 8);  // per warp probabilities
     L.merge_acc = off;
-    off += kConsumerWarps * GP * D * 4;                             // per warp fp32 [GP][D]
+    off += kConsumerWarps * G * D * 4;                              // per warp fp32 [G][D]
     L.merge_m = off;
-    off += kConsumerWarps * GP * 4;
+    off += kConsumerWarps * G * 4;
     L.merge_l = off;
-    off += kConsumerWarps * GP * 4;
+    off += kConsumerWarps * G * 4;
     off = align_up(off, 8);
     L.bars = off;
-    off += (2 * kMaxStages + 4) * 8;                                // full, empty, qfull[2], qempty[2]
+    off += (kMaxStages + 2) * 8;                                    // full[stage], qfull[2]
     L.flags = off;
     off += (kMaxStages + 8) * 4;                                    // stage_bad, abort, scan scratch
     L.prefix = off;

@@ -90,6 +90,12 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity, 
 
 // ---------------------------------------------------------------- TMA / bulk copies
 
+// Orders this thread's earlier generic-proxy shared-memory accesses before its
+// later async-proxy (TMA / bulk copy) accesses.
+__device__ __forceinline__ void fence_proxy_async_shared() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // 4D tiled tensor load into shared memory, completing on `bar` (no multicast).
 __device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1,
                                             int c2, int c3) {
