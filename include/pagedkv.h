@@ -67,13 +67,14 @@ extern "C" {
  *                     every CTA that fits on the device at once. The KV blocks
  *                     of a launch are split evenly over the CTAs, so this also
  *                     sets how finely long contexts are split.
- *   num_stages        shared-memory stages (one KV block each) per consumer warp
- *                     (1..4; a CTA has 4 consumer warps); default: about 64 KB
- *                     of KV blocks in flight per CTA.
+ *   num_stages        shared-memory stages (one KV block each) per warp (1..4; a
+ *                     CTA has 4 warps); default: 1 on tensor cores, about 64 KB
+ *                     of KV blocks per CTA on CUDA cores.
  *   ctas_per_sm       resident CTAs per SM of the default grid; default: the
  *                     occupancy limit.
- *   math              0 = default, 1 = fp32 CUDA cores, 2 = bf16 tensor cores
- *                     (mma.sync m16n8k16, fp32 accumulate).
+ *   math              0 = default (2), 1 = fp32 CUDA cores, 2 = bf16 tensor cores
+ *                     (mma.sync m16n8k16, fp32 accumulate; probabilities rounded
+ *                     to bf16 for the P.V product).
  */
 typedef struct pkv_decode_options {
     int num_ctas;

@@ -108,8 +108,11 @@ WorkspaceLayout workspace_layout(int num_seqs, int num_q_heads, int head_dim) {
     return w;
 }
 
-// Stages per consumer warp: about 64 KB of KV blocks in flight per CTA.
-int default_stages(int head_dim, int block_size) {
+// Stages per warp: one for the tensor-core path (more resident CTAs beat a
+// deeper ring: 4 CTAs of 4 warps per SM with 8 KB blocks); about 64 KB of
+// blocks in flight per CTA for the CUDA-core path, which fits fewer CTAs.
+int default_stages(int head_dim, int block_size, int math) {
+    if (math == pkv::kMathTensorCore) return 1;
     const int stage_bytes = 2 * block_size * head_dim * 2;
     int r = (64 * 1024) / (pkv::kConsumerWarps * stage_bytes);
     return r < 1 ? 1 : r > pkv::kMaxStagesPerWarp ? pkv::kMaxStagesPerWarp : r;
@@ -169,10 +172,10 @@ int paged_attn_decode_ex(void *out, const void *q, const void *k_cache, const vo
         return fail(PKV_ERR_INVALID_ARGUMENT, "num_ctas %d exceeds %d", o.num_ctas, pkv::kMaxCtas);
     if (static_cast<int64_t>(num_kv_heads) * max_blocks_per_seq * pkv::kMaxSeqsPerLaunch > 0x7fffffff)
         return fail(PKV_ERR_INVALID_ARGUMENT, "num_kv_heads * max_blocks_per_seq too large");
-    const int ns = o.num_stages ? o.num_stages : default_stages(head_dim, block_size);
+    const int math = o.math ? o.math : pkv::kMathTensorCore;
+    const int ns = o.num_stages ? o.num_stages : default_stages(head_dim, block_size, math);
     if (ns < 1 || ns > pkv::kMaxStagesPerWarp)
         return fail(PKV_ERR_INVALID_ARGUMENT, "num_stages %d outside [1, %d]", ns, pkv::kMaxStagesPerWarp);
-    const int math = o.math ? o.math : pkv::kMathCudaCore;
     const int gp = group_pad(group);
     if (!pkv::decode_variant_exists(head_dim, block_size, gp, math))
         return fail(PKV_ERR_UNSUPPORTED, "no kernel for head_dim %d, block_size %d, group %d, math %d", head_dim,

@@ -390,17 +390,20 @@ struct MmaMath {
         const int mi = lane >> 3, r = lane & 7;
         const int tr = lane >> 2;  // fragment row of this lane
         // S^T = K . Q^T; ldmatrix x4 gives the A fragment (rows t, cols d) of one k-step
-        float s[TT][4];
+        // two accumulators per tile (even / odd k-steps) halve the dependent mma chain
+        float s[TT][4], s2[TT][4];
 #pragma unroll
         for (int mt = 0; mt < TT; ++mt) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) s[mt][k] = 0.f;
+            for (int k = 0; k < 4; ++k) s[mt][k] = s2[mt][k] = 0.f;
 #pragma unroll
             for (int kk = 0; kk < KST; ++kk) {
                 uint32_t a[4];
                 ldsm_x4(a, tile_addr<BS>(ktile, 16 * mt + r + 8 * (mi & 1), 2 * kk + (mi >> 1)));
-                mma_16816(s[mt], a, qb[kk][0], qb[kk][1]);
+                mma_16816((kk & 1) ? s2[mt] : s[mt], a, qb[kk][0], qb[kk][1]);
             }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) s[mt][k] += s2[mt][k];
         }
         // base-2 logits; tokens past the context are selected away (their rows may hold anything)
         float mx0 = -INFINITY, mx1 = -INFINITY;
@@ -572,7 +575,9 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
     lookup(0, bat_p, bat_h);
     lookup(32, nxt_p, nxt_h);
     uint32_t inflight = 0, inflight_par = 0;  // stages whose copy this warp issued and has not yet seen land
-    auto issue = [&](int k) {                 // warp-uniform; k increases call after call
+    // Block k goes to stage warp + 4 (k % R) with phase parity (k / R) & 1, so
+    // block k + R reuses block k's stage with the other parity.
+    auto issue = [&](int k, int stage, uint32_t par) {  // warp-uniform; k increases call after call
         if (k >= nk) return;
         if (k - bat_k >= 32) {
             bat_k += 32;
@@ -582,8 +587,6 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
         }
         const int p = __shfl_sync(0xffffffffu, bat_p, k - bat_k);
         const int h = __shfl_sync(0xffffffffu, bat_h, k - bat_k);
-        const int stage = warp + kConsumerWarps * (k % R);
-        const uint32_t par = static_cast<uint32_t>(k / R) & 1u;
         if (lane == 0 && !*sm.abort_flag) {
             const bool bad = p < 0 || p >= a.num_blocks;
             sm.stage_bad[stage] = bad ? 1 : 0;
@@ -604,7 +607,7 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
             }
         }
     };
-    for (int k = 0; k < R; ++k) issue(k);
+    for (int k = 0; k < R; ++k) issue(k, warp + kConsumerWarps * k, 0u);
 
     // ---- query rows: warp 0 copies piece n + 1's rows while piece n is computed
     uint32_t q_issued = 0, q_issued_par = 0;
@@ -629,7 +632,8 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
     // ---- compute side
     Math math;
     math.init(warp, lane, sm.base, ly);
-    int k = 0, gb_base = 0, npiece = 0;
+    int k = 0, gb_base = 0, npiece = 0, ring = 0;
+    uint32_t rphase = 0;
     Piece pc;
     while (pieces.next(pc)) {
         const int slot = npiece & 1;
@@ -642,8 +646,12 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
         const int nblk = pc.b1 - pc.b0;
         for (int i = (warp - gb_base % kConsumerWarps + kConsumerWarps) % kConsumerWarps; i < nblk;
              i += kConsumerWarps, ++k) {
-            const int stage = warp + kConsumerWarps * (k % R);
-            const uint32_t par = static_cast<uint32_t>(k / R) & 1u;
+            const int stage = warp + kConsumerWarps * ring;
+            const uint32_t par = rphase;
+            if (++ring == R) {
+                ring = 0;
+                rphase ^= 1u;
+            }
             if (mbar_wait_bounded(&sm.full[stage], par, sm.abort_flag, a.status)) inflight &= ~(1u << stage);
             if (!sm.stage_bad[stage] && !*sm.abort_flag) {
                 const int valid = min(BS, pc.L - (pc.b0 + i) * BS);
@@ -651,7 +659,7 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
                 math.block(ktile, ktile + kTile, valid);
             }
             __syncwarp();
-            issue(k + R);  // the stage just freed takes this warp's block k + R
+            issue(k + R, stage, par ^ 1u);  // the stage just freed takes this warp's block k + R
         }
         gb_base += nblk;
 
@@ -702,8 +710,10 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
     }
 }
 
+// The tensor-core path fits 128 registers per thread, so 4 CTAs (16 warps)
+// share an SM; the CUDA-core path keeps its larger per-thread state.
 template <int D, int BS, int GP, int MATH>
-__global__ void __launch_bounds__(kDecodeThreads)
+__global__ void __launch_bounds__(kDecodeThreads, MATH == kMathTensorCore ? 4 : 1)
     paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                         const DecodeArgs a) {
     static_assert(D == 64 || D == 128, "head_dim");
