@@ -75,12 +75,15 @@ extern "C" {
  *   math              0 = default (2), 1 = fp32 CUDA cores, 2 = bf16 tensor cores
  *                     (mma.sync m16n8k16, fp32 accumulate; probabilities rounded
  *                     to bf16 for the P.V product).
+ *   l2_prefetch       KV blocks each warp prefetches into L2 ahead of the ones
+ *                     it loads into shared memory (1..32); -1 = none; default 2.
  */
 typedef struct pkv_decode_options {
     int num_ctas;
     int num_stages;
     int ctas_per_sm;
     int math;
+    int l2_prefetch;
 } pkv_decode_options;
 
 /*

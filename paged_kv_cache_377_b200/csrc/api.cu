@@ -111,6 +111,8 @@ WorkspaceLayout workspace_layout(int num_seqs, int num_q_heads, int head_dim) {
 // Stages per warp: one for the tensor-core path (more resident CTAs beat a
 // deeper ring: 4 CTAs of 4 warps per SM with 8 KB blocks); about 64 KB of
 // blocks in flight per CTA for the CUDA-core path, which fits fewer CTAs.
+constexpr int kDefaultL2Prefetch = 2;
+
 int default_stages(int head_dim, int block_size, int math) {
     if (math == pkv::kMathTensorCore) return 1;
     const int stage_bytes = 2 * block_size * head_dim * 2;
@@ -164,9 +166,10 @@ int paged_attn_decode_ex(void *out, const void *q, const void *k_cache, const vo
         !aligned(workspace, 256))
         return fail(PKV_ERR_INVALID_ARGUMENT,
                     "out, q, k_cache and v_cache must be 16-byte aligned and workspace 256-byte aligned");
-    pkv_decode_options o = {0, 0, 0, 0};
+    pkv_decode_options o = {0, 0, 0, 0, 0};
     if (opts) o = *opts;
-    if (o.num_ctas < 0 || o.num_stages < 0 || o.ctas_per_sm < 0 || o.math < 0 || o.math > 2)
+    if (o.num_ctas < 0 || o.num_stages < 0 || o.ctas_per_sm < 0 || o.math < 0 || o.math > 2 ||
+        o.l2_prefetch < -1 || o.l2_prefetch > 32)
         return fail(PKV_ERR_INVALID_ARGUMENT, "negative or unknown option");
     if (o.num_ctas > pkv::kMaxCtas)
         return fail(PKV_ERR_INVALID_ARGUMENT, "num_ctas %d exceeds %d", o.num_ctas, pkv::kMaxCtas);
@@ -224,6 +227,7 @@ int paged_attn_decode_ex(void *out, const void *q, const void *k_cache, const vo
         a.max_blocks_per_seq = max_blocks_per_seq;
         a.num_blocks = num_blocks;
         a.num_stages = ns;
+        a.prefetch = o.l2_prefetch < 0 ? 0 : o.l2_prefetch == 0 ? kDefaultL2Prefetch : o.l2_prefetch;
         a.scale_log2 = scale * 1.4426950408889634f;
         e = pkv::decode_launch(head_dim, block_size, gp, math, tm_k, tm_v, a, grid, smem, st);
         if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");

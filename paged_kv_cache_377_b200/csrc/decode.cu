@@ -532,8 +532,10 @@ struct Smem {
 // CTA's range and a ring of R shared-memory stages (stage w + 4 (k % R)). It
 // issues the TMA copies of its own blocks R ahead of the one it computes --
 // block k + R goes into the stage block k just freed -- so it waits on no other
-// warp to refill its ring. Block-table entries of its next 32 blocks are looked
-// up one batch ahead. Warp 0 also bulk-copies the query rows of the piece after
+// warp to refill its ring -- and prefetches its blocks a further `prefetch`
+// ahead into L2, so that those copies are served from L2 and more HBM reads are
+// in flight than the ring can hold. Block-table entries of its next 32 blocks
+// are looked up one batch ahead. Warp 0 also bulk-copies the query rows of the piece after
 // next. All four warps meet at the end of every piece to merge their states.
 template <int D, int BS, class Math>
 __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUtensorMap *tm_v, const DecodeArgs &a,
@@ -587,6 +589,20 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
         }
         const int p = __shfl_sync(0xffffffffu, bat_p, k - bat_k);
         const int h = __shfl_sync(0xffffffffu, bat_h, k - bat_k);
+        // this warp's block k + prefetch, from the current or the next batch (prefetch <= 32)
+        const int kp = k + a.prefetch, jp = kp - bat_k;
+        const int pp_a = __shfl_sync(0xffffffffu, bat_p, jp & 31), pp_b = __shfl_sync(0xffffffffu, nxt_p, jp & 31);
+        const int hp_a = __shfl_sync(0xffffffffu, bat_h, jp & 31), hp_b = __shfl_sync(0xffffffffu, nxt_h, jp & 31);
+        if (lane == 0 && a.prefetch > 0 && kp < nk && !*sm.abort_flag) {
+            const int pp = jp < 32 ? pp_a : pp_b, hp = jp < 32 ? hp_a : hp_b;
+            if (pp >= 0 && pp < a.num_blocks) {
+#pragma unroll
+                for (int half = 0; half < D / 64; ++half) {
+                    tma_prefetch_l2_4d(tm_k, 0, half, hp, pp * BS);
+                    tma_prefetch_l2_4d(tm_v, 0, half, hp, pp * BS);
+                }
+            }
+        }
         if (lane == 0 && !*sm.abort_flag) {
             const bool bad = p < 0 || p >= a.num_blocks;
             sm.stage_bad[stage] = bad ? 1 : 0;

@@ -29,7 +29,8 @@ struct DecodeArgs {
     int group;                   // Hq / Hkv
     int max_blocks_per_seq;
     int num_blocks;
-    int num_stages;              // ring stages per consumer warp (R); the CTA holds 4R
+    int num_stages;              // ring stages per warp (R); the CTA holds 4R
+    int prefetch;                // blocks a warp prefetches into L2 beyond the one it loads (0 = none)
     float scale_log2;            // scale * log2(e): logits are kept in base 2
 };
 

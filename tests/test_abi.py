@@ -89,11 +89,11 @@ def test_append_rejects_bad_arguments():
 
 def test_options_are_checked():
     lib = pkv.library()
-    opts = pkv._binding._Options(2000, 0, 0, 0)
+    opts = pkv._binding._Options(2000, 0, 0, 0, 0)
     rc = lib.paged_attn_decode_ex(P, P, P, P, P, P, 4, 2, 1, 64, 16, 0.125, 3, 16, P, 1 << 20,
                                   ctypes.byref(opts), None)
     assert rc == -1 and "num_ctas" in lib.pkv_last_error().decode()
-    opts = pkv._binding._Options(0, 5, 0, 0)
+    opts = pkv._binding._Options(0, 5, 0, 0, 0)
     rc = lib.paged_attn_decode_ex(P, P, P, P, P, P, 4, 2, 1, 64, 16, 0.125, 3, 16, P, 1 << 20,
                                   ctypes.byref(opts), None)
     assert rc == -1 and "num_stages" in lib.pkv_last_error().decode()
