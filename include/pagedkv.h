@@ -76,8 +76,7 @@ extern "C" {
  *                     (mma.sync m16n8k16, fp32 accumulate; probabilities rounded
  *                     to bf16 for the P.V product).
  *   l2_prefetch       KV blocks each warp prefetches into L2 ahead of the ones
- *                     it loads into shared memory (1..32); -1 or 0 (default) =
- *                     none (on B200 every distance measured slower).
+ *                     it loads into shared memory (1..32); -1 = none; default 2.
  */
 typedef struct pkv_decode_options {
     int num_ctas;

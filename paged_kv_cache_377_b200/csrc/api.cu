@@ -111,7 +111,7 @@ WorkspaceLayout workspace_layout(int num_seqs, int num_q_heads, int head_dim) {
 // Stages per warp: one for the tensor-core path (more resident CTAs beat a
 // deeper ring: 4 CTAs of 4 warps per SM with 8 KB blocks); about 64 KB of
 // blocks in flight per CTA for the CUDA-core path, which fits fewer CTAs.
-constexpr int kDefaultL2Prefetch = 0;  // measured on the Llama-shaped batch: any prefetch distance was slower
+constexpr int kDefaultL2Prefetch = 2;
 
 int default_stages(int head_dim, int block_size, int math) {
     if (math == pkv::kMathTensorCore) return 1;
@@ -227,7 +227,7 @@ int paged_attn_decode_ex(void *out, const void *q, const void *k_cache, const vo
         a.max_blocks_per_seq = max_blocks_per_seq;
         a.num_blocks = num_blocks;
         a.num_stages = ns;
-        a.prefetch = o.l2_prefetch <= 0 ? kDefaultL2Prefetch * (o.l2_prefetch == 0) : o.l2_prefetch;
+        a.prefetch = o.l2_prefetch < 0 ? 0 : o.l2_prefetch == 0 ? kDefaultL2Prefetch : o.l2_prefetch;
         a.scale_log2 = scale * 1.4426950408889634f;
         e = pkv::decode_launch(head_dim, block_size, gp, math, tm_k, tm_v, a, grid, smem, st);
         if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");

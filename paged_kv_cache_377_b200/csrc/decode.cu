@@ -520,11 +520,10 @@ struct MmaMath {
 
 struct Smem {
     uint8_t *base;
-    uint64_t *full, *qfull, *qempty, *mfree;
+    uint64_t *full, *qfull;
     volatile int *stage_bad;
     volatile int *abort_flag;
     int *scan;
-    int *mcount;
     int *prefix;
     int *lens;
 };
@@ -533,15 +532,11 @@ struct Smem {
 // CTA's range and a ring of R shared-memory stages (stage w + 4 (k % R)). It
 // issues the TMA copies of its own blocks R ahead of the one it computes --
 // block k + R goes into the stage block k just freed -- so it waits on no other
-// warp to refill its ring -- and can also prefetch its blocks further ahead into
-// L2. Block-table entries of its next 32 blocks are looked up one batch ahead.
-//
-// Warps do not wait for one another at piece boundaries: each writes its
-// softmax state for the piece into the merge slot and moves on; the last of the
-// four to arrive (shared-memory counter) merges the slot and stores the
-// piece's result, then frees the slot. Warp 0 copies the query rows of the
-// pieces ahead into a ring of kQSlots slots, each freed when all four warps
-// have read it.
+// warp to refill its ring -- and prefetches its blocks a further `prefetch`
+// ahead into L2, so that those copies are served from L2 and more HBM reads are
+// in flight than the ring can hold. Block-table entries of its next 32 blocks
+// are looked up one batch ahead. Warp 0 also bulk-copies the query rows of the piece after
+// next. All four warps meet at the end of every piece to merge their states.
 template <int D, int BS, class Math>
 __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUtensorMap *tm_v, const DecodeArgs &a,
                                             const Smem &sm, const DecodeLayout &ly, PieceIter pieces, long long x0,
@@ -552,6 +547,10 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
     const int G = a.group;
     const uint32_t qbytes = static_cast<uint32_t>(G * D * 2);
     const uint32_t sbase = smem_u32(sm.base);
+    float *merge_acc = reinterpret_cast<float *>(sm.base + ly.merge_acc);
+    float *merge_m = reinterpret_cast<float *>(sm.base + ly.merge_m);
+    float *merge_l = reinterpret_cast<float *>(sm.base + ly.merge_l);
+    const int ctid = warp * 32 + lane;
 
     // ---- issue side: this warp's blocks k = 0 .. nk-1 are global blocks x0 + warp + 4k
     const long long span = x1 - x0;
@@ -626,60 +625,43 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
     };
     for (int k = 0; k < R; ++k) issue(k, warp + kConsumerWarps * k, 0u);
 
-    // ---- query rows: warp 0 keeps up to kQSlots pieces' rows staged ahead
+    // ---- query rows: warp 0 copies piece n + 1's rows while piece n is computed
     uint32_t q_issued = 0, q_issued_par = 0;
     PieceIter ahead = pieces;
     Piece pa{};
-    int q_next = 0;            // next piece whose rows warp 0 will copy
-    bool ahead_more = true;
-    auto top_up_q = [&](int npiece) {  // warp 0: copy rows of pieces up to npiece + kQSlots - 1
-        while (ahead_more && q_next < npiece + kQSlots) {
-            const int slot = q_next % kQSlots;
-            const uint32_t use = static_cast<uint32_t>(q_next / kQSlots);
-            // the slot's previous piece must have been read by all four warps
-            if (use > 0) mbar_wait_bounded(&sm.qempty[slot], (use - 1) & 1u, sm.abort_flag, a.status);
-            if (!ahead.next(pa)) {
-                ahead_more = false;
-                break;
-            }
-            if (lane == 0 && !*sm.abort_flag) {
-                const __nv_bfloat16 *src = static_cast<const __nv_bfloat16 *>(a.q) +
-                                           (static_cast<size_t>(pa.s) * a.num_q_heads + static_cast<size_t>(pa.h) * G) *
-                                               D;
-                fence_proxy_async_shared();
-                mbar_arrive_expect_tx(&sm.qfull[slot], qbytes);
-                bulk_load(sm.base + ly.qbuf + slot * qbytes, src, qbytes, &sm.qfull[slot]);
-                q_issued |= 1u << slot;
-                q_issued_par = (q_issued_par & ~(1u << slot)) | ((use & 1u) << slot);
-            }
-            ++q_next;
+    auto issue_q = [&](int n) {  // piece n's rows into slot n % 2 (ahead has just returned piece n)
+        if (warp == 0 && lane == 0 && !*sm.abort_flag) {
+            const int slot = n & 1;
+            const __nv_bfloat16 *src = static_cast<const __nv_bfloat16 *>(a.q) +
+                                       (static_cast<size_t>(pa.s) * a.num_q_heads + static_cast<size_t>(pa.h) * G) * D;
+            fence_proxy_async_shared();
+            mbar_arrive_expect_tx(&sm.qfull[slot], qbytes);
+            bulk_load(sm.base + ly.qbuf + slot * qbytes, src, qbytes, &sm.qfull[slot]);
+            q_issued |= 1u << slot;
+            q_issued_par = (q_issued_par & ~(1u << slot)) | ((static_cast<uint32_t>(n >> 1) & 1u) << slot);
         }
     };
-    if (warp == 0) top_up_q(0);
+    int n_ahead = 0;
+    if (ahead.next(pa)) issue_q(n_ahead++);
+    if (ahead.next(pa)) issue_q(n_ahead++);
 
     // ---- compute side
     Math math;
     math.init(warp, lane, sm.base, ly);
-    float *const mg_acc = reinterpret_cast<float *>(sm.base + ly.merge_acc);
-    float *const mg_m = reinterpret_cast<float *>(sm.base + ly.merge_m);
-    float *const mg_l = reinterpret_cast<float *>(sm.base + ly.merge_l);
     int k = 0, gb_base = 0, npiece = 0, ring = 0;
     uint32_t rphase = 0;
     Piece pc;
     while (pieces.next(pc)) {
-        const int n = npiece++;
-        if (warp == 0) top_up_q(n);
-        const int qs = n % kQSlots;
-        mbar_wait_bounded(&sm.qfull[qs], static_cast<uint32_t>(n / kQSlots) & 1u, sm.abort_flag, a.status);
-        math.load_q(sbase + ly.qbuf + qs * qbytes, G, a.scale_log2);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.qempty[qs]);
+        const int slot = npiece & 1;
+        if (npiece >= 1 && ahead.next(pa)) issue_q(n_ahead++);  // every warp has read slot (npiece + 1) % 2
+        mbar_wait_bounded(&sm.qfull[slot], static_cast<uint32_t>(npiece >> 1) & 1u, sm.abort_flag, a.status);
+        math.load_q(sbase + ly.qbuf + slot * qbytes, G, a.scale_log2);
         math.reset();
+        ++npiece;
 
         const int nblk = pc.b1 - pc.b0;
-        int mine = 0;
         for (int i = (warp - gb_base % kConsumerWarps + kConsumerWarps) % kConsumerWarps; i < nblk;
-             i += kConsumerWarps, ++k, ++mine) {
+             i += kConsumerWarps, ++k) {
             const int stage = warp + kConsumerWarps * ring;
             const uint32_t par = rphase;
             if (++ring == R) {
@@ -697,45 +679,23 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
         }
         gb_base += nblk;
 
-        // ---- hand this warp's state for the piece to the merge slot
-        const int ms = n % kMergeSlots;
-        const uint32_t muse = static_cast<uint32_t>(n / kMergeSlots);
-        if (muse > 0) mbar_wait_bounded(&sm.mfree[ms], (muse - 1) & 1u, sm.abort_flag, a.status);
-        float *s_acc = mg_acc + ms * (kConsumerWarps * G * D);
-        float *s_m = mg_m + ms * (kConsumerWarps * G);
-        float *s_l = mg_l + ms * (kConsumerWarps * G);
-        if (mine > 0) {
-            math.export_state(s_acc, s_m, s_l, warp, G);
-        } else if (lane < G) {  // no blocks here: an empty state (its acc row is never read)
-            s_m[warp * G + lane] = -INFINITY;
-            s_l[warp * G + lane] = 0.f;
-        }
-        __syncwarp();
-        int arrived = 0;
-        if (lane == 0) {
-            __threadfence_block();
-            arrived = atomicAdd(&sm.mcount[ms], 1);
-        }
-        arrived = __shfl_sync(0xffffffffu, arrived, 0);
-        if (arrived != kConsumerWarps - 1) continue;
+        math.export_state(merge_acc, merge_m, merge_l, warp, G);
+        named_barrier_sync(1, kConsumerWarps * 32);
 
-        // ---- last warp of the piece: merge the four states (log-sum-exp identity) and store
-        __threadfence_block();
+        // merge the warps' states (log-sum-exp identity) and store
         const size_t seg = static_cast<size_t>(pc.s) * a.num_kv_heads + pc.h;
-        for (int e = lane; e < G * D / 2; e += 32) {
+        for (int e = ctid; e < G * D / 2; e += kConsumerWarps * 32) {
             const int g = e / (D / 2), d = (e % (D / 2)) * 2;
             float M = -INFINITY;
 #pragma unroll
-            for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, s_m[w * G + g]);
+            for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, merge_m[w * G + g]);
             float ls = 0.f, a0 = 0.f, a1 = 0.f;
             if (M != -INFINITY) {
 #pragma unroll
                 for (int w = 0; w < kConsumerWarps; ++w) {
-                    const float mw = s_m[w * G + g];
-                    if (mw == -INFINITY) continue;  // a warp with no blocks in this piece
-                    const float f = fast_exp2(mw - M);
-                    const float2 av = *reinterpret_cast<const float2 *>(s_acc + (w * G + g) * D + d);
-                    ls += s_l[w * G + g] * f;
+                    const float f = fast_exp2(merge_m[w * G + g] - M);
+                    const float2 av = *reinterpret_cast<const float2 *>(merge_acc + (w * G + g) * D + d);
+                    ls += merge_l[w * G + g] * f;
                     a0 += av.x * f;
                     a1 += av.y * f;
                 }
@@ -752,11 +712,7 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
                 if (d == 0) a.lse_part[pr] = ls > 0.f ? M + __log2f(ls) : -INFINITY;
             }
         }
-        __syncwarp();
-        if (lane == 0) {
-            sm.mcount[ms] = 0;
-            mbar_arrive(&sm.mfree[ms]);  // release: the slot may take the next piece's states
-        }
+        named_barrier_sync(1, kConsumerWarps * 32);
     }
     // Leave no copy in flight into shared memory when the CTA exits (only
     // possible after a wait gave up).
@@ -765,7 +721,7 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
             if ((inflight >> st) & 1u) mbar_wait_drain(&sm.full[st], (inflight_par >> st) & 1u, a.status);
         // the last copy into each query slot: landed already unless a wait gave up
         if (warp == 0)
-            for (int slot = 0; slot < kQSlots; ++slot)
+            for (int slot = 0; slot < 2; ++slot)
                 if ((q_issued >> slot) & 1u) mbar_wait_drain(&sm.qfull[slot], (q_issued_par >> slot) & 1u, a.status);
     }
 }
@@ -787,12 +743,9 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathTensorCore ? 4 : 
     sm.base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     sm.full = reinterpret_cast<uint64_t *>(sm.base + ly.bars);
     sm.qfull = sm.full + kMaxStages;
-    sm.qempty = sm.qfull + kQSlots;
-    sm.mfree = sm.qempty + kQSlots;
     sm.stage_bad = reinterpret_cast<volatile int *>(sm.base + ly.flags);
     sm.abort_flag = sm.stage_bad + kMaxStages;
     sm.scan = reinterpret_cast<int *>(sm.base + ly.flags) + kMaxStages + 1;
-    sm.mcount = sm.scan + kDecodeThreads / 32;  // after the scan's per-warp totals
     sm.prefix = reinterpret_cast<int *>(sm.base + ly.prefix);
     sm.lens = reinterpret_cast<int *>(sm.base + ly.lens);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -802,14 +755,7 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathTensorCore ? 4 : 
             mbar_init(&sm.full[i], 1);
             sm.stage_bad[i] = 0;
         }
-        for (int i = 0; i < kQSlots; ++i) {
-            mbar_init(&sm.qfull[i], 1);
-            mbar_init(&sm.qempty[i], kConsumerWarps);
-        }
-        for (int i = 0; i < kMergeSlots; ++i) {
-            mbar_init(&sm.mfree[i], 1);
-            sm.mcount[i] = 0;
-        }
+        for (int i = 0; i < 2; ++i) mbar_init(&sm.qfull[i], 1);
         *sm.abort_flag = 0;
         fence_mbar_init();
     }

@@ -13,8 +13,6 @@ constexpr int kMaxStagesPerWarp = kMaxStages / kConsumerWarps;
 constexpr int kMaxSeqsPerLaunch = 2048;               // per-sequence tables kept in shared memory
 constexpr int kMaxCtas = 1024;                        // grid limit; bounds the pieces of a launch
 constexpr int kWorkspaceHeaderBytes = 256;
-constexpr int kQSlots = 4;                            // query-row slots (pieces whose rows are staged)
-constexpr int kMergeSlots = 1;                        // pieces whose warp states can wait to be merged
 
 struct DecodeArgs {
     void *out;                   // bf16 [S][Hq][D]
@@ -54,21 +52,21 @@ __host__ __device__ inline DecodeLayout decode_layout(int D, int BS, int GP, int
     L.stages = off;
     off += static_cast<uint32_t>(num_stages) * 2u * tile;          // [stage][K tile, V tile]
     L.qbuf = off;
-    off += kQSlots * G * D * 2;                                     // query slots [G][D] bf16
+    off += 2u * G * D * 2;                                          // two query slots [G][D] bf16
     off = align_up(off, 16);
     L.pscr = off;
     off += kConsumerWarps * (tensor_core ? BS * 16 : BS * GP * 8);  // per warp probabilities
     L.merge_acc = off;
-    off += kMergeSlots * kConsumerWarps * G * D * 4;                // [slot][warp][G][D] fp32
+    off += kConsumerWarps * G * D * 4;                              // per warp fp32 [G][D]
     L.merge_m = off;
-    off += kMergeSlots * kConsumerWarps * G * 4;
+    off += kConsumerWarps * G * 4;
     L.merge_l = off;
-    off += kMergeSlots * kConsumerWarps * G * 4;
+    off += kConsumerWarps * G * 4;
     off = align_up(off, 8);
     L.bars = off;
-    off += (kMaxStages + 2 * kQSlots + kMergeSlots) * 8;            // full, qfull, qempty, mfree
+    off += (kMaxStages + 2) * 8;                                    // full[stage], qfull[2]
     L.flags = off;
-    off += (kMaxStages + 1 + kConsumerWarps + kMergeSlots + 2) * 4;  // stage_bad, abort, scan, merge counters
+    off += (kMaxStages + 8) * 4;                                    // stage_bad, abort, scan scratch
     L.prefix = off;
     off += static_cast<uint32_t>(num_seqs + 1) * 4;                 // blocks before each sequence
     L.lens = off;
