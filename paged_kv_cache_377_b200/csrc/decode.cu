@@ -589,13 +589,12 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
         }
         const int p = __shfl_sync(0xffffffffu, bat_p, k - bat_k);
         const int h = __shfl_sync(0xffffffffu, bat_h, k - bat_k);
-        // this warp's block k + prefetch, from the current or the next batch (prefetch <= 32)
-        const int kp = k + a.prefetch, jp = kp - bat_k;
-        const int pp_a = __shfl_sync(0xffffffffu, bat_p, jp & 31), pp_b = __shfl_sync(0xffffffffu, nxt_p, jp & 31);
-        const int hp_a = __shfl_sync(0xffffffffu, bat_h, jp & 31), hp_b = __shfl_sync(0xffffffffu, nxt_h, jp & 31);
-        if (lane == 0 && a.prefetch > 0 && kp < nk && !*sm.abort_flag) {
+        if (a.prefetch > 0) {  // this warp's block k + prefetch, from the current or the next batch (<= 32 ahead)
+            const int kp = k + a.prefetch, jp = kp - bat_k;
+            const int pp_a = __shfl_sync(0xffffffffu, bat_p, jp & 31), pp_b = __shfl_sync(0xffffffffu, nxt_p, jp & 31);
+            const int hp_a = __shfl_sync(0xffffffffu, bat_h, jp & 31), hp_b = __shfl_sync(0xffffffffu, nxt_h, jp & 31);
             const int pp = jp < 32 ? pp_a : pp_b, hp = jp < 32 ? hp_a : hp_b;
-            if (pp >= 0 && pp < a.num_blocks) {
+            if (lane == 0 && kp < nk && pp >= 0 && pp < a.num_blocks && !*sm.abort_flag) {
 #pragma unroll
                 for (int half = 0; half < D / 64; ++half) {
                     tma_prefetch_l2_4d(tm_k, 0, half, hp, pp * BS);
@@ -610,8 +609,9 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
                 atomicOr(a.status, PKV_STATUS_BAD_BLOCK_ID);
                 mbar_arrive(&sm.full[stage]);
             } else {
+                // The stage's previous contents were read with ldmatrix / ld.shared whose
+                // results this warp has already consumed, so the copy cannot overtake them.
                 uint8_t *dst = sm.base + ly.stages + static_cast<uint32_t>(stage) * 2u * kTile;
-                fence_proxy_async_shared();  // this warp's reads of the stage come before the copy
                 mbar_arrive_expect_tx(&sm.full[stage], 2u * kTile);
 #pragma unroll
                 for (int half = 0; half < D / 64; ++half) {
@@ -634,7 +634,6 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
             const int slot = n & 1;
             const __nv_bfloat16 *src = static_cast<const __nv_bfloat16 *>(a.q) +
                                        (static_cast<size_t>(pa.s) * a.num_q_heads + static_cast<size_t>(pa.h) * G) * D;
-            fence_proxy_async_shared();
             mbar_arrive_expect_tx(&sm.qfull[slot], qbytes);
             bulk_load(sm.base + ly.qbuf + slot * qbytes, src, qbytes, &sm.qfull[slot]);
             q_issued |= 1u << slot;
