@@ -55,6 +55,7 @@ def parse_args(argv=None):
     p.add_argument("--ctas-per-sm", type=int, default=0)
     p.add_argument("--math", type=int, default=0)
     p.add_argument("--l2-prefetch", type=int, default=0)
+    p.add_argument("--piece-cost", type=int, default=0)
     p.add_argument("--seqs", type=int, default=0,
                    help="build the workload with only its first N context lengths (small cases for ncu)")
     p.add_argument("--no-e2e", action="store_true")
@@ -210,7 +211,8 @@ class Step:
         self.out = torch.empty_like(self.q)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
         self.opts = dict(num_ctas=args.num_ctas, num_stages=args.num_stages,
-                         ctas_per_sm=args.ctas_per_sm, math=args.math, l2_prefetch=args.l2_prefetch)
+                         ctas_per_sm=args.ctas_per_sm, math=args.math, l2_prefetch=args.l2_prefetch,
+                         piece_cost=args.piece_cost)
         self.ws = pkv.allocate_workspace(b.num_seqs, b.num_q_heads, b.head_dim, device=device)
 
     def append(self, stream=None):
@@ -383,7 +385,7 @@ def config_block(args, batch, world):
     }
     if args.seqs:
         c["seqs_kept"] = args.seqs
-    for k in ("num_ctas", "num_stages", "ctas_per_sm", "math", "l2_prefetch"):
+    for k in ("num_ctas", "num_stages", "ctas_per_sm", "math", "l2_prefetch", "piece_cost"):
         if getattr(args, k):
             c[k] = getattr(args, k)
     return c

@@ -76,7 +76,13 @@ extern "C" {
  *                     (mma.sync m16n8k16, fp32 accumulate; probabilities rounded
  *                     to bf16 for the P.V product).
  *   l2_prefetch       KV blocks each warp prefetches into L2 ahead of the ones
- *                     it loads into shared memory (1..32); -1 = none; default 2.
+ *                     it loads into shared memory (1..32); -1 or 0 (default) =
+ *                     none (on B200 every distance measured slower).
+ *   piece_cost        extra weight, in KV blocks, that every non-empty (sequence,
+ *                     kv head) segment adds when the batch is split between CTAs,
+ *                     standing for a piece's fixed cost (1..64); -1 = none;
+ *                     default 2. Keeps CTAs that get many short contexts from
+ *                     finishing last.
  */
 typedef struct pkv_decode_options {
     int num_ctas;
@@ -84,13 +90,14 @@ typedef struct pkv_decode_options {
     int ctas_per_sm;
     int math;
     int l2_prefetch;
+    int piece_cost;
 } pkv_decode_options;
 
 /*
  * Bytes of device workspace paged_attn_decode needs for this shape
  * (host-only; returns PKV_OK and sets *bytes).
  * Layout: [0, 256) header whose first int32 is the device status word; the
- * per-sequence block prefix sums of one launch; fp32 partial outputs and
+ * per-sequence block and weight prefix sums of one launch; fp32 partial outputs and
  * log2-sum-exp values of the context pieces that CTA boundaries cut. At most
  * 2048 sequences go in one launch; longer batches reuse the workspace launch
  * after launch.

@@ -89,8 +89,8 @@ int sm_count() {
     return cache[dev];
 }
 
-// Workspace layout: [0, 256) header (status word) | block prefix sums
-// [S_chunk + 1] int32 | fp32 partial outputs [rows][D] | fp32 log2-sum-exp [rows],
+// Workspace layout: [0, 256) header (status word) | block and weight prefix
+// sums [2][S_chunk + 1] int32 | fp32 partial outputs [rows][D] | fp32 log2-sum-exp [rows],
 // rows = (S_chunk + kMaxCtas) * Hq bounds the pieces' rows of one launch
 // (pieces <= S_chunk * Hkv + C, each with G <= Hq rows).
 struct WorkspaceLayout {
@@ -102,7 +102,7 @@ WorkspaceLayout workspace_layout(int num_seqs, int num_q_heads, int head_dim) {
     const int64_t rows = (sc + pkv::kMaxCtas) * num_q_heads;
     WorkspaceLayout w;
     w.seq_blocks = pkv::kWorkspaceHeaderBytes;
-    w.o_part = w.seq_blocks + ((sc + 1) * 4 + 255) / 256 * 256;
+    w.o_part = w.seq_blocks + (2 * (sc + 1) * 4 + 255) / 256 * 256;
     w.lse_part = w.o_part + rows * head_dim * 4;
     w.total = w.lse_part + (rows * 4 + 255) / 256 * 256;
     return w;
@@ -111,7 +111,8 @@ WorkspaceLayout workspace_layout(int num_seqs, int num_q_heads, int head_dim) {
 // Stages per warp: one for the tensor-core path (more resident CTAs beat a
 // deeper ring: 4 CTAs of 4 warps per SM with 8 KB blocks); about 64 KB of
 // blocks in flight per CTA for the CUDA-core path, which fits fewer CTAs.
-constexpr int kDefaultL2Prefetch = 2;
+constexpr int kDefaultL2Prefetch = 0;  // measured on the Llama-shaped batch: any prefetch distance was slower
+constexpr int kDefaultPieceCost = 2;   // weight of a piece's fixed cost, in KV blocks
 
 int default_stages(int head_dim, int block_size, int math) {
     if (math == pkv::kMathTensorCore) return 1;
@@ -166,14 +167,14 @@ int paged_attn_decode_ex(void *out, const void *q, const void *k_cache, const vo
         !aligned(workspace, 256))
         return fail(PKV_ERR_INVALID_ARGUMENT,
                     "out, q, k_cache and v_cache must be 16-byte aligned and workspace 256-byte aligned");
-    pkv_decode_options o = {0, 0, 0, 0, 0};
+    pkv_decode_options o = {0, 0, 0, 0, 0, 0};
     if (opts) o = *opts;
     if (o.num_ctas < 0 || o.num_stages < 0 || o.ctas_per_sm < 0 || o.math < 0 || o.math > 2 ||
-        o.l2_prefetch < -1 || o.l2_prefetch > 32)
+        o.l2_prefetch < -1 || o.l2_prefetch > 32 || o.piece_cost < -1 || o.piece_cost > 64)
         return fail(PKV_ERR_INVALID_ARGUMENT, "negative or unknown option");
     if (o.num_ctas > pkv::kMaxCtas)
         return fail(PKV_ERR_INVALID_ARGUMENT, "num_ctas %d exceeds %d", o.num_ctas, pkv::kMaxCtas);
-    if (static_cast<int64_t>(num_kv_heads) * max_blocks_per_seq * pkv::kMaxSeqsPerLaunch > 0x7fffffff)
+    if (static_cast<int64_t>(num_kv_heads) * (max_blocks_per_seq + 64) * pkv::kMaxSeqsPerLaunch > 0x7fffffff)
         return fail(PKV_ERR_INVALID_ARGUMENT, "num_kv_heads * max_blocks_per_seq too large");
     const int math = o.math ? o.math : pkv::kMathTensorCore;
     const int ns = o.num_stages ? o.num_stages : default_stages(head_dim, block_size, math);
@@ -211,7 +212,7 @@ int paged_attn_decode_ex(void *out, const void *q, const void *k_cache, const vo
         if (o.ctas_per_sm > 0 && o.ctas_per_sm < per_sm) per_sm = o.ctas_per_sm;
         int grid = o.num_ctas > 0 ? o.num_ctas : sms * per_sm;
         if (grid > pkv::kMaxCtas) grid = pkv::kMaxCtas;
-        pkv::DecodeArgs a;
+        pkv::DecodeArgs a{};
         a.out = static_cast<__nv_bfloat16 *>(out) + static_cast<size_t>(s0) * num_q_heads * head_dim;
         a.q = static_cast<const __nv_bfloat16 *>(q) + static_cast<size_t>(s0) * num_q_heads * head_dim;
         a.block_tables = block_tables + static_cast<size_t>(s0) * max_blocks_per_seq;
@@ -227,7 +228,8 @@ int paged_attn_decode_ex(void *out, const void *q, const void *k_cache, const vo
         a.max_blocks_per_seq = max_blocks_per_seq;
         a.num_blocks = num_blocks;
         a.num_stages = ns;
-        a.prefetch = o.l2_prefetch < 0 ? 0 : o.l2_prefetch == 0 ? kDefaultL2Prefetch : o.l2_prefetch;
+        a.prefetch = o.l2_prefetch > 0 ? o.l2_prefetch : o.l2_prefetch == 0 ? kDefaultL2Prefetch : 0;
+        a.piece_cost = o.piece_cost > 0 ? o.piece_cost : o.piece_cost == 0 ? kDefaultPieceCost : 0;
         a.scale_log2 = scale * 1.4426950408889634f;
         e = pkv::decode_launch(head_dim, block_size, gp, math, tm_k, tm_v, a, grid, smem, st);
         if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");

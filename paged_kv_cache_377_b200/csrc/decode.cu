@@ -89,9 +89,29 @@ struct PieceIter {
     }
 };
 
-__device__ __forceinline__ long long range_begin(int c, long long B, int C) {
-    return static_cast<long long>(c) * B / C;
+// Work is split between CTAs by weight: a non-empty segment of n blocks weighs
+// n + piece_cost, its first piece_cost units standing for the fixed cost of a
+// piece (query load, merge of the warps' states). CTA c takes the weight range
+// [c W / C, (c + 1) W / C); its blocks are the real blocks whose weight
+// position falls in that range -- a contiguous range of the launch's blocks.
+// pre[s] / wpre[s] = blocks / weight of the sequences before s (per head).
+// Returns the number of real blocks whose weight position is below v.
+__device__ __forceinline__ long long blocks_below(long long v, const int *pre, const int *wpre, int S, int Hkv,
+                                                  int piece_cost) {
+    if (v >= static_cast<long long>(Hkv) * wpre[S]) return static_cast<long long>(Hkv) * pre[S];
+    int lo = 0, hi = S - 1;
+    while (lo < hi) {  // the sequence holding weight position v
+        const int mid = (lo + hi + 1) >> 1;
+        if (static_cast<long long>(Hkv) * wpre[mid] <= v) lo = mid;
+        else hi = mid - 1;
+    }
+    const int w = wpre[lo + 1] - wpre[lo], n = pre[lo + 1] - pre[lo];
+    const long long r = v - static_cast<long long>(Hkv) * wpre[lo];
+    const int h = static_cast<int>(r / w), o = static_cast<int>(r - static_cast<long long>(h) * w);
+    return static_cast<long long>(Hkv) * pre[lo] + static_cast<long long>(h) * n + max(0, o - piece_cost);
 }
+
+__device__ __forceinline__ long long weight_begin(int c, long long W, int C) { return static_cast<long long>(c) * W / C; }
 
 // Shared address of 16-byte chunk c (0 <= c < D/8) of row t of a K or V tile.
 // A tile holds D/64 column halves of [BS rows][128 bytes], each loaded by one
@@ -525,6 +545,7 @@ struct Smem {
     volatile int *abort_flag;
     int *scan;
     int *prefix;
+    int *wprefix;
     int *lens;
 };
 
@@ -746,6 +767,7 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathTensorCore ? 4 : 
     sm.abort_flag = sm.stage_bad + kMaxStages;
     sm.scan = reinterpret_cast<int *>(sm.base + ly.flags) + kMaxStages + 1;
     sm.prefix = reinterpret_cast<int *>(sm.base + ly.prefix);
+    sm.wprefix = reinterpret_cast<int *>(sm.base + ly.wprefix);
     sm.lens = reinterpret_cast<int *>(sm.base + ly.lens);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -763,12 +785,14 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathTensorCore ? 4 : 
         tma_prefetch_desc(&tm_v);
     }
 
-    // prefix[s] = blocks of sequences < s (clamped lengths); lens[s] = clamped length
+    // prefix[s] = blocks of sequences < s (clamped lengths), wprefix[s] = their
+    // weight (blocks + piece_cost per non-empty sequence); lens[s] = clamped length
     const int S = a.num_seqs;
     const int cap = a.max_blocks_per_seq * BS;
+    const int pcost = min(max(a.piece_cost, 0), 64);  // validated on the host; a bad value moves no index
     const int per = (S + kDecodeThreads - 1) / kDecodeThreads;
     const int lo = min(S, tid * per), hi = min(S, lo + per);
-    int mine = 0;
+    int mine = 0, mine_w = 0;
     for (int s = lo; s < hi; ++s) {
         int L = __ldg(a.context_lens + s);
         if (L < 0 || L > cap) {
@@ -776,33 +800,58 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathTensorCore ? 4 : 
             L = min(max(L, 0), cap);
         }
         sm.lens[s] = L;
-        mine += (L + BS - 1) / BS;
+        const int n = (L + BS - 1) / BS;
+        mine += n;
+        mine_w += n > 0 ? n + pcost : 0;
     }
-    int incl = mine;
+    int incl = mine, incl_w = mine_w;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
+        const int yw = __shfl_up_sync(0xffffffffu, incl_w, o);
+        if (lane >= o) {
+            incl += y;
+            incl_w += yw;
+        }
     }
-    if (lane == 31) sm.scan[warp] = incl;
+    if (lane == 31) {
+        sm.scan[warp] = incl;
+        sm.scan[4 + warp] = incl_w;
+    }
     __syncthreads();
-    int run = incl - mine;
-    for (int w = 0; w < warp; ++w) run += sm.scan[w];
+    int run = incl - mine, run_w = incl_w - mine_w;
+    for (int w = 0; w < warp; ++w) {
+        run += sm.scan[w];
+        run_w += sm.scan[4 + w];
+    }
     for (int s = lo; s < hi; ++s) {
         sm.prefix[s] = run;
-        run += (sm.lens[s] + BS - 1) / BS;
+        sm.wprefix[s] = run_w;
+        const int n = (sm.lens[s] + BS - 1) / BS;
+        run += n;
+        run_w += n > 0 ? n + pcost : 0;
     }
     if (tid == 0) {
-        int total = 0;
-        for (int w = 0; w < kDecodeThreads / 32; ++w) total += sm.scan[w];
+        int total = 0, total_w = 0;
+        for (int w = 0; w < kDecodeThreads / 32; ++w) {
+            total += sm.scan[w];
+            total_w += sm.scan[4 + w];
+        }
         sm.prefix[S] = total;
+        sm.wprefix[S] = total_w;
     }
     __syncthreads();
     if (blockIdx.x == 0)  // the merge kernel locates split segments from the same prefix sums
-        for (int s = tid; s <= S; s += kDecodeThreads) a.seq_blocks[s] = sm.prefix[s];
+        for (int s = tid; s <= S; s += kDecodeThreads) {
+            a.seq_blocks[s] = sm.prefix[s];
+            a.seq_blocks[S + 1 + s] = sm.wprefix[s];
+        }
 
-    const long long B = static_cast<long long>(a.num_kv_heads) * sm.prefix[S];
-    const long long x0 = range_begin(blockIdx.x, B, gridDim.x), x1 = range_begin(blockIdx.x + 1, B, gridDim.x);
+    const long long W = static_cast<long long>(a.num_kv_heads) * sm.wprefix[S];
+    const long long x0 = blocks_below(weight_begin(blockIdx.x, W, gridDim.x), sm.prefix, sm.wprefix, S,
+                                      a.num_kv_heads, pcost);
+    const long long x1 = blocks_below(weight_begin(blockIdx.x + 1, W, gridDim.x), sm.prefix, sm.wprefix, S,
+                                      a.num_kv_heads, pcost);
     PieceIter pieces;
     pieces.x = x0;
     pieces.x1 = x1;
@@ -830,6 +879,7 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(const DecodeArgs a, int 
     if (row >= a.num_seqs * a.num_q_heads) return;
     const int s = row / a.num_q_heads, j = row - s * a.num_q_heads;
     const int G = a.group, h = j / G, g = j - h * G;
+    const int *wpre = a.seq_blocks + a.num_seqs + 1;
     const int pre_s = a.seq_blocks[s];
     const int n = a.seq_blocks[s + 1] - pre_s;
     __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(a.out) + static_cast<size_t>(row) * D + lane * PER;
@@ -838,14 +888,17 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(const DecodeArgs a, int 
         for (int i = 0; i < PER; i += 2) *reinterpret_cast<__nv_bfloat162 *>(out + i) = __floats2bfloat162_rn(0.f, 0.f);
         return;
     }
-    const long long B = static_cast<long long>(a.num_kv_heads) * a.seq_blocks[a.num_seqs];
-    const long long first_block = static_cast<long long>(a.num_kv_heads) * pre_s + static_cast<long long>(h) * n;
-    // CTA c covers [c B / C, (c + 1) B / C): the CTA of block x is ((x + 1) C - 1) / B
-    const int c0 = static_cast<int>(((first_block + 1) * num_ctas - 1) / B);
-    const int c1 = static_cast<int>(((first_block + n) * num_ctas - 1) / B);
+    // weight positions of the segment's first and last blocks (see blocks_below)
+    const long long W = static_cast<long long>(a.num_kv_heads) * wpre[a.num_seqs];
+    const int pcost = min(max(a.piece_cost, 0), 64);
+    const long long v_first =
+        static_cast<long long>(a.num_kv_heads) * wpre[s] + static_cast<long long>(h) * (n + pcost) + pcost;
+    // CTA c covers weight positions [c W / C, (c + 1) W / C): position v is in CTA ((v + 1) C - 1) / W
+    const int c0 = static_cast<int>(((v_first + 1) * num_ctas - 1) / W);
+    const int c1 = static_cast<int>(((v_first + n) * num_ctas - 1) / W);
     if (c0 == c1) return;  // one piece: written directly by the decode kernel
-    // with more CTAs than blocks some CTA ranges are empty: they hold no piece
-    auto holds = [&](int c) { return range_begin(c + 1, B, num_ctas) > range_begin(c, B, num_ctas); };
+    // CTAs strictly between c0 and c1 lie inside the segment's blocks; empty ones hold no piece
+    auto holds = [&](int c) { return weight_begin(c + 1, W, num_ctas) > weight_begin(c, W, num_ctas); };
     const size_t seg = static_cast<size_t>(s) * a.num_kv_heads + h;
     float M = -INFINITY;
     for (int c = c0 + lane; c <= c1; c += 32)

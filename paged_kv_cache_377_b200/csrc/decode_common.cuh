@@ -21,7 +21,7 @@ struct DecodeArgs {
     const int32_t *context_lens; // [S]
     float *o_part;               // fp32 [piece][G][D], piece = s * Hkv + h + cta
     float *lse_part;             // fp32 [piece][G], log2 domain
-    int32_t *seq_blocks;         // [S + 1] prefix sums of blocks per sequence, for the merge kernel
+    int32_t *seq_blocks;         // [2][S + 1] block and weighted-block prefix sums, for the merge kernel
     int32_t *status;             // device status word
     int num_seqs;
     int num_q_heads;
@@ -31,11 +31,12 @@ struct DecodeArgs {
     int num_blocks;
     int num_stages;              // ring stages per warp (R); the CTA holds 4R
     int prefetch;                // blocks a warp prefetches into L2 beyond the one it loads (0 = none)
+    int piece_cost;              // extra weight, in blocks, of every non-empty segment when splitting work
     float scale_log2;            // scale * log2(e): logits are kept in base 2
 };
 
 struct DecodeLayout {
-    uint32_t stages, qbuf, pscr, merge_acc, merge_m, merge_l, bars, flags, prefix, lens, total;
+    uint32_t stages, qbuf, pscr, merge_acc, merge_m, merge_l, bars, flags, prefix, wprefix, lens, total;
 };
 
 __host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
@@ -66,9 +67,11 @@ __host__ __device__ inline DecodeLayout decode_layout(int D, int BS, int GP, int
     L.bars = off;
     off += (kMaxStages + 2) * 8;                                    // full[stage], qfull[2]
     L.flags = off;
-    off += (kMaxStages + 8) * 4;                                    // stage_bad, abort, scan scratch
+    off += (kMaxStages + 1 + 2 * kConsumerWarps + 3) * 4;           // stage_bad, abort, scan scratch
     L.prefix = off;
     off += static_cast<uint32_t>(num_seqs + 1) * 4;                 // blocks before each sequence
+    L.wprefix = off;
+    off += static_cast<uint32_t>(num_seqs + 1) * 4;                 // weighted blocks before each sequence
     L.lens = off;
     off += static_cast<uint32_t>(num_seqs) * 4;                     // clamped context lengths
     L.total = align_up(off, 16) + 1024;

@@ -27,11 +27,12 @@ def test_library_loads_and_exports_every_declared_symbol():
 
 
 def test_workspace_size():
-    # header | prefix sums of one launch (<= 2048 seqs) | fp32 [rows][D] | fp32 [rows], rows = (S + 1024) * Hq
+    # header | block + weight prefix sums of one launch (<= 2048 seqs) | fp32 [rows][D] | fp32 [rows],
+    # rows = (S + 1024) * Hq
     def expect(S, Hq, D):
         sc = min(S, 2048)
         rows = (sc + 1024) * Hq
-        return 256 + -(-(sc + 1) * 4 // 256) * 256 + rows * D * 4 + -(-rows * 4 // 256) * 256
+        return 256 + -(-2 * (sc + 1) * 4 // 256) * 256 + rows * D * 4 + -(-rows * 4 // 256) * 256
     for S, Hq, D in [(4, 2, 64), (256, 32, 128), (3000, 12, 64), (0, 8, 128)]:
         assert pkv.workspace_bytes(S, Hq, D) == expect(S, Hq, D)
     assert pkv.workspace_bytes(5000, 8, 128) == pkv.workspace_bytes(2048, 8, 128)
@@ -89,11 +90,11 @@ def test_append_rejects_bad_arguments():
 
 def test_options_are_checked():
     lib = pkv.library()
-    opts = pkv._binding._Options(2000, 0, 0, 0, 0)
+    opts = pkv._binding._Options(2000, 0, 0, 0, 0, 0)
     rc = lib.paged_attn_decode_ex(P, P, P, P, P, P, 4, 2, 1, 64, 16, 0.125, 3, 16, P, 1 << 20,
                                   ctypes.byref(opts), None)
     assert rc == -1 and "num_ctas" in lib.pkv_last_error().decode()
-    opts = pkv._binding._Options(0, 5, 0, 0, 0)
+    opts = pkv._binding._Options(0, 5, 0, 0, 0, 0)
     rc = lib.paged_attn_decode_ex(P, P, P, P, P, P, 4, 2, 1, 64, 16, 0.125, 3, 16, P, 1 << 20,
                                   ctypes.byref(opts), None)
     assert rc == -1 and "num_stages" in lib.pkv_last_error().decode()

@@ -76,7 +76,8 @@ def test_grid_sizes_split_contexts_differently(name, num_ctas, math):
 @pytest.mark.parametrize("opts", [dict(num_stages=1), dict(num_stages=2), dict(num_stages=4), dict(ctas_per_sm=1),
                                   dict(num_stages=3, ctas_per_sm=2, num_ctas=100),
                                   dict(math=2, num_stages=1), dict(math=2, num_stages=4, ctas_per_sm=1),
-                                  dict(l2_prefetch=-1), dict(l2_prefetch=32), dict(math=1, l2_prefetch=5)])
+                                  dict(l2_prefetch=-1), dict(l2_prefetch=32), dict(math=1, l2_prefetch=5),
+                                  dict(piece_cost=-1), dict(piece_cost=64), dict(piece_cost=7, num_ctas=333)])
 def test_launch_options(opts):
     b, ref, _, _ = config_case("opt125m")
     out, _, _, st = run_step(b, **opts)
