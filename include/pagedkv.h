@@ -81,7 +81,7 @@ extern "C" {
  *   piece_cost        extra weight, in KV blocks, that every non-empty (sequence,
  *                     kv head) segment adds when the batch is split between CTAs,
  *                     standing for a piece's fixed cost (1..64); -1 = none;
- *                     default 2. Keeps CTAs that get many short contexts from
+ *                     default 4. Keeps CTAs that get many short contexts from
  *                     finishing last.
  */
 typedef struct pkv_decode_options {
