@@ -96,8 +96,9 @@ typedef struct pkv_decode_options {
 /*
  * Bytes of device workspace paged_attn_decode needs for this shape
  * (host-only; returns PKV_OK and sets *bytes).
- * Layout: [0, 256) header whose first int32 is the device status word; the
- * per-sequence block and weight prefix sums of one launch; fp32 partial outputs and
+ * Layout: [0, 256) header whose first int32 is the device status word; one
+ * counter per (sequence, kv head) of a launch, tagged with the launch's epoch
+ * so the workspace never needs clearing; fp32 partial outputs and
  * log2-sum-exp values of the context pieces that CTA boundaries cut. At most
  * 2048 sequences go in one launch; longer batches reuse the workspace launch
  * after launch.
@@ -123,10 +124,11 @@ int pkv_decode_workspace_bytes(int num_seqs, int num_q_heads, int head_dim, size
  * multiple of num_kv_heads with a ratio <= PKV_MAX_GROUP; num_blocks *
  * block_size < 2^31. Any num_seqs >= 0 (0 is a no-op).
  * Per call (and per 2048 sequences): one persistent decode kernel whose CTAs
- * each take an equal share of the batch's KV blocks, then one log-sum-exp
- * merge kernel for the contexts that were split between CTAs. For a given
- * device and options, results are bitwise reproducible and depend only on the
- * logical order of tokens, not on where their blocks sit in the pool.
+ * each take an equal share of the batch's KV blocks (weighted per context
+ * piece); a context split between CTAs is merged (log-sum-exp) by the CTA that
+ * stores its last piece. For a given device and options, results are bitwise
+ * reproducible and depend only on the logical order of tokens, not on where
+ * their blocks sit in the pool.
  */
 int paged_attn_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
                       const int32_t *block_tables, const int32_t *context_lens,

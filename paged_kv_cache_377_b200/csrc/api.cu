@@ -9,6 +9,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -77,6 +78,13 @@ int make_pool_map(CUtensorMap *map, const void *pool, int num_blocks, int bs, in
     return PKV_OK;
 }
 
+// Launch epochs tag the per-segment piece counters, so a workspace never needs
+// clearing between calls (a counter from an older launch restarts at 1).
+unsigned long long next_epoch() {
+    static std::atomic<unsigned long long> epoch{0};
+    return (epoch.fetch_add(1, std::memory_order_relaxed) + 1) & ((1ull << 48) - 1);
+}
+
 int sm_count() {
     int dev = 0, n = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 0;
@@ -89,20 +97,20 @@ int sm_count() {
     return cache[dev];
 }
 
-// Workspace layout: [0, 256) header (status word) | block and weight prefix
-// sums [2][S_chunk + 1] int32 | fp32 partial outputs [rows][D] | fp32 log2-sum-exp [rows],
+// Workspace layout: [0, 256) header (status word) | per-segment piece
+// counters [S_chunk * Hkv <= S_chunk * Hq] uint64 | fp32 partial outputs [rows][D] | fp32 log2-sum-exp [rows],
 // rows = (S_chunk + kMaxCtas) * Hq bounds the pieces' rows of one launch
 // (pieces <= S_chunk * Hkv + C, each with G <= Hq rows).
 struct WorkspaceLayout {
-    size_t seq_blocks, o_part, lse_part, total;
+    size_t seg_count, o_part, lse_part, total;
 };
 
 WorkspaceLayout workspace_layout(int num_seqs, int num_q_heads, int head_dim) {
     const int64_t sc = num_seqs < pkv::kMaxSeqsPerLaunch ? num_seqs : pkv::kMaxSeqsPerLaunch;
     const int64_t rows = (sc + pkv::kMaxCtas) * num_q_heads;
     WorkspaceLayout w;
-    w.seq_blocks = pkv::kWorkspaceHeaderBytes;
-    w.o_part = w.seq_blocks + (2 * (sc + 1) * 4 + 255) / 256 * 256;
+    w.seg_count = pkv::kWorkspaceHeaderBytes;
+    w.o_part = w.seg_count + (sc * num_q_heads * 8 + 255) / 256 * 256;
     w.lse_part = w.o_part + rows * head_dim * 4;
     w.total = w.lse_part + (rows * 4 + 255) / 256 * 256;
     return w;
@@ -221,7 +229,8 @@ int paged_attn_decode_ex(void *out, const void *q, const void *k_cache, const vo
         a.context_lens = context_lens + s0;
         a.o_part = reinterpret_cast<float *>(ws + wl.o_part);
         a.lse_part = reinterpret_cast<float *>(ws + wl.lse_part);
-        a.seq_blocks = reinterpret_cast<int32_t *>(ws + wl.seq_blocks);
+        a.seg_count = reinterpret_cast<unsigned long long *>(ws + wl.seg_count);
+        a.epoch = next_epoch();
         a.status = reinterpret_cast<int32_t *>(ws);
         a.num_seqs = sc;
         a.num_q_heads = num_q_heads;
@@ -235,8 +244,6 @@ int paged_attn_decode_ex(void *out, const void *q, const void *k_cache, const vo
         a.scale_log2 = scale * 1.4426950408889634f;
         e = pkv::decode_launch(head_dim, block_size, gp, math, tm_k, tm_v, a, grid, smem, st);
         if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
-        e = pkv::lse_merge_launch(head_dim, a, grid, st);
-        if (e != cudaSuccess) return cuda_fail(e, "lse merge launch");
     }
     return ok();
 }

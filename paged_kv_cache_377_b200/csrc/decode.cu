@@ -34,8 +34,9 @@
 //   * At the end of a piece the four warp states are merged in shared memory
 //     with the log-sum-exp identity. A piece that is a whole segment writes
 //     bf16 output directly; the pieces of a segment cut by CTA boundaries
-//     write fp32 partials + log2-sum-exp, merged by lse_merge_kernel in CTA
-//     order.
+//     write fp32 partials + log2-sum-exp, and the CTA that stores a segment's
+//     last piece (a per-segment counter tagged with the launch's epoch, so it
+//     never needs clearing) merges them in CTA order.
 // Every reduction order depends only on logical token positions, so results
 // are bitwise reproducible and independent of where blocks sit in the pool.
 #include <cstdio>
@@ -543,11 +544,53 @@ struct Smem {
     uint64_t *full, *qfull;
     volatile int *stage_bad;
     volatile int *abort_flag;
+    volatile int *merge_flag;  // [3]: this CTA completes the segment's pieces, first CTA, last CTA
     int *scan;
     int *prefix;
     int *wprefix;
     int *lens;
 };
+
+// The CTAs holding pieces of segment (s, h): c0 .. c1, skipping CTAs whose
+// weight range is empty; npieces = how many hold one. CTA c covers weight
+// positions [c W / C, (c + 1) W / C), so position v lies in CTA ((v + 1) C - 1) / W.
+__device__ __forceinline__ void segment_ctas(int s, int h, const Smem &sm, int Hkv, long long W, int C, int pcost,
+                                             int &c0, int &c1, int &npieces) {
+    const int n = sm.prefix[s + 1] - sm.prefix[s];
+    const long long v_first = static_cast<long long>(Hkv) * sm.wprefix[s] + static_cast<long long>(h) * (n + pcost) + pcost;
+    c0 = static_cast<int>(((v_first + 1) * C - 1) / W);
+    c1 = static_cast<int>(((v_first + n) * C - 1) / W);
+    npieces = 0;
+    for (int c = c0; c <= c1; ++c) npieces += weight_begin(c + 1, W, C) > weight_begin(c, W, C);
+}
+
+// Merge of the pieces of segment (s, h) stored by CTAs c0 .. c1 (log-sum-exp
+// identity, pieces in CTA order): out = sum_c 2^(lse_c - M) o_c / sum_c 2^(lse_c - M).
+// Partials written by other SMs are read past L1.
+template <int D>
+__device__ __forceinline__ void merge_pieces(const DecodeArgs &a, size_t seg, int s, int h, int c0, int c1,
+                                             long long W, int C, int ctid) {
+    const int G = a.group;
+    for (int e = ctid; e < G * D / 2; e += kConsumerWarps * 32) {
+        const int g = e / (D / 2), d = (e % (D / 2)) * 2;
+        float M = -INFINITY;
+        for (int c = c0; c <= c1; ++c)
+            if (weight_begin(c + 1, W, C) > weight_begin(c, W, C)) M = fmaxf(M, __ldcg(a.lse_part + (seg + c) * G + g));
+        float den = 0.f, a0 = 0.f, a1 = 0.f;
+        for (int c = c0; c <= c1; ++c) {
+            if (weight_begin(c + 1, W, C) <= weight_begin(c, W, C)) continue;
+            const size_t pr = (seg + c) * G + g;
+            const float w = fast_exp2(__ldcg(a.lse_part + pr) - M);
+            const float2 o = __ldcg(reinterpret_cast<const float2 *>(a.o_part + pr * D + d));
+            den += w;
+            a0 += w * o.x;
+            a1 += w * o.y;
+        }
+        const size_t row = static_cast<size_t>(s) * a.num_q_heads + static_cast<size_t>(h) * G + g;
+        *reinterpret_cast<__nv_bfloat162 *>(static_cast<__nv_bfloat16 *>(a.out) + row * D + d) =
+            __floats2bfloat162_rn(a0 / den, a1 / den);
+    }
+}
 
 // One decode warp. Warp w owns the blocks x0 + w + 4k (k = 0, 1, ...) of the
 // CTA's range and a ring of R shared-memory stages (stage w + 4 (k % R)). It
@@ -561,7 +604,7 @@ struct Smem {
 template <int D, int BS, class Math>
 __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUtensorMap *tm_v, const DecodeArgs &a,
                                             const Smem &sm, const DecodeLayout &ly, PieceIter pieces, long long x0,
-                                            long long x1, int warp, int lane) {
+                                            long long x1, long long W, int C, int pcost, int warp, int lane) {
     constexpr uint32_t kTile = BS * D * 2;
     constexpr uint32_t kHalf = BS * 128;
     const int R = a.num_stages;
@@ -732,6 +775,32 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
                 if (d == 0) a.lse_part[pr] = ls > 0.f ? M + __log2f(ls) : -INFINITY;
             }
         }
+        if (!pc.whole) {
+            // A segment cut between CTAs: count this CTA's piece in; the CTA that
+            // stores the segment's last piece merges them all.
+            __threadfence();
+            named_barrier_sync(1, kConsumerWarps * 32);
+            if (ctid == 0) {
+                int c0, c1, npieces;
+                segment_ctas(pc.s, pc.h, sm, a.num_kv_heads, W, C, pcost, c0, c1, npieces);
+                unsigned long long *cnt = a.seg_count + seg;
+                unsigned long long old = atomicAdd(cnt, 0ull), now;
+                for (;;) {  // count = 1 for the first piece of this launch (stale epochs restart)
+                    now = (old >> 16) == a.epoch ? old + 1 : (a.epoch << 16) | 1ull;
+                    const unsigned long long prev = atomicCAS(cnt, old, now);
+                    if (prev == old) break;
+                    old = prev;
+                }
+                sm.merge_flag[0] = static_cast<int>(now & 0xffffull) == npieces;
+                sm.merge_flag[1] = c0;
+                sm.merge_flag[2] = c1;
+            }
+            named_barrier_sync(1, kConsumerWarps * 32);
+            if (sm.merge_flag[0]) {
+                __threadfence();
+                merge_pieces<D>(a, seg, pc.s, pc.h, sm.merge_flag[1], sm.merge_flag[2], W, C, ctid);
+            }
+        }
         named_barrier_sync(1, kConsumerWarps * 32);
     }
     // Leave no copy in flight into shared memory when the CTA exits (only
@@ -766,6 +835,7 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathTensorCore ? 4 : 
     sm.stage_bad = reinterpret_cast<volatile int *>(sm.base + ly.flags);
     sm.abort_flag = sm.stage_bad + kMaxStages;
     sm.scan = reinterpret_cast<int *>(sm.base + ly.flags) + kMaxStages + 1;
+    sm.merge_flag = reinterpret_cast<volatile int *>(sm.scan + 2 * kConsumerWarps);
     sm.prefix = reinterpret_cast<int *>(sm.base + ly.prefix);
     sm.wprefix = reinterpret_cast<int *>(sm.base + ly.wprefix);
     sm.lens = reinterpret_cast<int *>(sm.base + ly.lens);
@@ -841,11 +911,13 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathTensorCore ? 4 : 
         sm.wprefix[S] = total_w;
     }
     __syncthreads();
-    if (blockIdx.x == 0)  // the merge kernel locates split segments from the same prefix sums
-        for (int s = tid; s <= S; s += kDecodeThreads) {
-            a.seq_blocks[s] = sm.prefix[s];
-            a.seq_blocks[S + 1 + s] = sm.wprefix[s];
-        }
+    if (blockIdx.x == 0)  // sequences with no context get all-zero rows (no piece covers them)
+        for (int s = 0; s < S; ++s)
+            if (sm.lens[s] == 0)
+                for (int e = tid; e < a.num_q_heads * D / 2; e += kDecodeThreads)
+                    reinterpret_cast<__nv_bfloat162 *>(static_cast<__nv_bfloat16 *>(a.out) +
+                                                       static_cast<size_t>(s) * a.num_q_heads * D)[e] =
+                        __floats2bfloat162_rn(0.f, 0.f);
 
     const long long W = static_cast<long long>(a.num_kv_heads) * sm.wprefix[S];
     const long long x0 = blocks_below(weight_begin(blockIdx.x, W, gridDim.x), sm.prefix, sm.wprefix, S,
@@ -861,69 +933,11 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathTensorCore ? 4 : 
     pieces.Hkv = a.num_kv_heads;
 
     if constexpr (MATH == kMathCudaCore) {
-        decode_warp<D, BS, CoreMath<D, BS, GP>>(&tm_k, &tm_v, a, sm, ly, pieces, x0, x1, warp, lane);
+        decode_warp<D, BS, CoreMath<D, BS, GP>>(&tm_k, &tm_v, a, sm, ly, pieces, x0, x1, W, gridDim.x, pcost, warp,
+                                                lane);
     } else {
-        decode_warp<D, BS, MmaMath<D, BS>>(&tm_k, &tm_v, a, sm, ly, pieces, x0, x1, warp, lane);
+        decode_warp<D, BS, MmaMath<D, BS>>(&tm_k, &tm_v, a, sm, ly, pieces, x0, x1, W, gridDim.x, pcost, warp, lane);
     }
-}
-
-// Merge of the pieces of segments that CTA boundaries cut:
-//   out = sum_c 2^(lse_c - M) o_c / sum_c 2^(lse_c - M), c = the CTAs holding
-// pieces of the segment, in order. One warp per (sequence, query head); rows
-// of empty sequences (context length 0) get zeros here.
-template <int D>
-__global__ void __launch_bounds__(256) lse_merge_kernel(const DecodeArgs a, int num_ctas) {
-    constexpr int PER = D / 32;
-    const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (row >= a.num_seqs * a.num_q_heads) return;
-    const int s = row / a.num_q_heads, j = row - s * a.num_q_heads;
-    const int G = a.group, h = j / G, g = j - h * G;
-    const int *wpre = a.seq_blocks + a.num_seqs + 1;
-    const int pre_s = a.seq_blocks[s];
-    const int n = a.seq_blocks[s + 1] - pre_s;
-    __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(a.out) + static_cast<size_t>(row) * D + lane * PER;
-    if (n == 0) {
-#pragma unroll
-        for (int i = 0; i < PER; i += 2) *reinterpret_cast<__nv_bfloat162 *>(out + i) = __floats2bfloat162_rn(0.f, 0.f);
-        return;
-    }
-    // weight positions of the segment's first and last blocks (see blocks_below)
-    const long long W = static_cast<long long>(a.num_kv_heads) * wpre[a.num_seqs];
-    const int pcost = min(max(a.piece_cost, 0), 64);
-    const long long v_first =
-        static_cast<long long>(a.num_kv_heads) * wpre[s] + static_cast<long long>(h) * (n + pcost) + pcost;
-    // CTA c covers weight positions [c W / C, (c + 1) W / C): position v is in CTA ((v + 1) C - 1) / W
-    const int c0 = static_cast<int>(((v_first + 1) * num_ctas - 1) / W);
-    const int c1 = static_cast<int>(((v_first + n) * num_ctas - 1) / W);
-    if (c0 == c1) return;  // one piece: written directly by the decode kernel
-    // CTAs strictly between c0 and c1 lie inside the segment's blocks; empty ones hold no piece
-    auto holds = [&](int c) { return weight_begin(c + 1, W, num_ctas) > weight_begin(c, W, num_ctas); };
-    const size_t seg = static_cast<size_t>(s) * a.num_kv_heads + h;
-    float M = -INFINITY;
-    for (int c = c0 + lane; c <= c1; c += 32)
-        if (holds(c)) M = fmaxf(M, a.lse_part[(seg + c) * G + g]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float den = 0.f;
-    for (int c = c0 + lane; c <= c1; c += 32)
-        if (holds(c)) den += fast_exp2(a.lse_part[(seg + c) * G + g] - M);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-    float acc[PER];
-#pragma unroll
-    for (int i = 0; i < PER; ++i) acc[i] = 0.f;
-    for (int c = c0; c <= c1; ++c) {
-        if (!holds(c)) continue;
-        const size_t pr = (seg + c) * G + g;
-        const float w = fast_exp2(a.lse_part[pr] - M);
-        const float *op = a.o_part + pr * D + lane * PER;
-#pragma unroll
-        for (int i = 0; i < PER; ++i) acc[i] += w * op[i];
-    }
-#pragma unroll
-    for (int i = 0; i < PER; i += 2)
-        *reinterpret_cast<__nv_bfloat162 *>(out + i) = __floats2bfloat162_rn(acc[i] / den, acc[i + 1] / den);
 }
 
 using KernelFn = void (*)(const CUtensorMap, const CUtensorMap, const DecodeArgs);
@@ -985,13 +999,5 @@ cudaError_t decode_launch(int head_dim, int block_size, int group_pad, int math,
     return cudaGetLastError();
 }
 
-cudaError_t lse_merge_launch(int head_dim, const DecodeArgs &args, int num_ctas, cudaStream_t stream) {
-    const int rows = args.num_seqs * args.num_q_heads;
-    const int grid = (rows + 7) / 8;
-    if (grid == 0) return cudaSuccess;
-    if (head_dim == 64) lse_merge_kernel<64><<<grid, 256, 0, stream>>>(args, num_ctas);
-    else lse_merge_kernel<128><<<grid, 256, 0, stream>>>(args, num_ctas);
-    return cudaGetLastError();
-}
 
 }  // namespace pkv

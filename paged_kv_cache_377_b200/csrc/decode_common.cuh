@@ -21,7 +21,8 @@ struct DecodeArgs {
     const int32_t *context_lens; // [S]
     float *o_part;               // fp32 [piece][G][D], piece = s * Hkv + h + cta
     float *lse_part;             // fp32 [piece][G], log2 domain
-    int32_t *seq_blocks;         // [2][S + 1] block and weighted-block prefix sums, for the merge kernel
+    unsigned long long *seg_count;  // [S * Hkv] (call epoch << 16 | pieces stored), per segment
+    unsigned long long epoch;    // this launch's epoch (< 2^48), unique in the process
     int32_t *status;             // device status word
     int num_seqs;
     int num_q_heads;

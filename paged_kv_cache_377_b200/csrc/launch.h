@@ -28,9 +28,6 @@ cudaError_t decode_launch(int head_dim, int block_size, int group_pad, int math,
                           const CUtensorMap &tm_v, const DecodeArgs &args, int grid, size_t smem_bytes,
                           cudaStream_t stream);
 
-// Log-sum-exp merge of the pieces of segments split across CTAs into `out`
-// (and zero rows for empty sequences). num_ctas = the decode launch's grid.
-cudaError_t lse_merge_launch(int head_dim, const DecodeArgs &args, int num_ctas, cudaStream_t stream);
 
 cudaError_t append_launch(const void *k, const void *v, void *k_cache, void *v_cache, const int64_t *slot_mapping,
                           int num_tokens, int num_kv_heads, int head_dim, int block_size, int num_blocks,

@@ -27,12 +27,12 @@ def test_library_loads_and_exports_every_declared_symbol():
 
 
 def test_workspace_size():
-    # header | block + weight prefix sums of one launch (<= 2048 seqs) | fp32 [rows][D] | fp32 [rows],
-    # rows = (S + 1024) * Hq
+    # header | per-segment piece counters (<= S * Hq uint64, one launch of <= 2048 seqs)
+    # | fp32 partials [rows][D] | fp32 log2-sum-exp [rows], rows = (S + 1024) * Hq
     def expect(S, Hq, D):
         sc = min(S, 2048)
         rows = (sc + 1024) * Hq
-        return 256 + -(-2 * (sc + 1) * 4 // 256) * 256 + rows * D * 4 + -(-rows * 4 // 256) * 256
+        return 256 + -(-sc * Hq * 8 // 256) * 256 + rows * D * 4 + -(-rows * 4 // 256) * 256
     for S, Hq, D in [(4, 2, 64), (256, 32, 128), (3000, 12, 64), (0, 8, 128)]:
         assert pkv.workspace_bytes(S, Hq, D) == expect(S, Hq, D)
     assert pkv.workspace_bytes(5000, 8, 128) == pkv.workspace_bytes(2048, 8, 128)
