@@ -81,6 +81,17 @@ def aggregate(sum_values, max_values):
     return s.cpu().tolist(), m.cpu().tolist()
 
 
+def job_totals(kv_bytes, seqs, ctx_tokens, steps, total_ms):
+    """Whole-job figures over all ranks: each rank processed its own batch
+    `steps` times in `total_ms` of device time; the job takes as long as its
+    slowest rank (weak scaling: per-rank work is fixed as ranks are added)."""
+    (sum_kv, sum_seq, sum_tok), (max_ms,) = aggregate(
+        [kv_bytes * steps, seqs * steps, ctx_tokens * steps], [total_ms])
+    seconds = max_ms / 1e3
+    return {"value": sum_kv / seconds / 1e9, "seq_per_s": sum_seq / seconds,
+            "ctx_tokens_per_s": sum_tok / seconds, "max_ms": max_ms}
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -277,9 +288,8 @@ def run_ours(args, rank, world, local_rank):
     if status:
         raise RuntimeError(f"device status {status} after the timed steps")
 
-    (sum_kv, sum_seq, sum_tok), (max_ms,) = aggregate([kv * K, S * K, ctx_tokens * K], [total_ms])
-    seconds = max_ms / 1e3
-    value = sum_kv / seconds / 1e9
+    job = job_totals(kv, S, ctx_tokens, K, total_ms)
+    value, max_ms = job["value"], job["max_ms"]
     hbm, hbm_kind = measured_peaks()
     mean_decode_ms = statistics.fmean(decode_ms)
     achieved = kv / (mean_decode_ms / 1e3) / 1e9
@@ -308,8 +318,8 @@ def run_ours(args, rank, world, local_rank):
         "data": "synthetic",
         "config": config_block(args, batch, world),
         "pct_of_hbm_peak": round(100.0 * value / (hbm * world), 2),
-        "seq_per_s": round(sum_seq / seconds, 1),
-        "ctx_tokens_per_s": round(sum_tok / seconds, 1),
+        "seq_per_s": round(job["seq_per_s"], 1),
+        "ctx_tokens_per_s": round(job["ctx_tokens_per_s"], 1),
         "append_us_mean": round(1e3 * statistics.fmean(append_ms), 3),
         "decode_us_mean": round(1e3 * mean_decode_ms, 3),
         "decode_us_median": round(1e3 * statistics.median(decode_ms), 3),
@@ -492,7 +502,7 @@ def main(argv=None):
     if world > 1:
         import torch.distributed as dist
         torch.cuda.set_device(local_rank)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
         result = run_ours(args, rank, world, local_rank)
