@@ -544,7 +544,8 @@ struct Smem {
     uint64_t *full, *qfull;
     volatile int *stage_bad;
     volatile int *abort_flag;
-    volatile int *merge_flag;  // [3]: this CTA completes the segment's pieces, first CTA, last CTA
+    volatile int *merge_flag;  // [1 + 4 * 2]: how many segments this CTA completed (<= 2), then
+                               // for each (s, h, first CTA, last CTA)
     int *scan;
     int *prefix;
     int *wprefix;
@@ -560,35 +561,64 @@ __device__ __forceinline__ void segment_ctas(int s, int h, const Smem &sm, int H
     const long long v_first = static_cast<long long>(Hkv) * sm.wprefix[s] + static_cast<long long>(h) * (n + pcost) + pcost;
     c0 = static_cast<int>(((v_first + 1) * C - 1) / W);
     c1 = static_cast<int>(((v_first + n) * C - 1) / W);
+    if (W >= C) {  // no CTA range is empty
+        npieces = c1 - c0 + 1;
+        return;
+    }
     npieces = 0;
     for (int c = c0; c <= c1; ++c) npieces += weight_begin(c + 1, W, C) > weight_begin(c, W, C);
 }
 
 // Merge of the pieces of segment (s, h) stored by CTAs c0 .. c1 (log-sum-exp
-// identity, pieces in CTA order): out = sum_c 2^(lse_c - M) o_c / sum_c 2^(lse_c - M).
-// Partials written by other SMs are read past L1.
+// identity, pieces in CTA order): out = sum_c 2^(lse_c - M) o_c / sum_c 2^(lse_c - M),
+// taken in one pass with a running maximum. A thread merges 4-dim elements of
+// the G x D output (at most two) and loads four pieces ahead, so that the merge
+// costs a few L2 round trips rather than one per piece. Partials written by
+// other SMs are read past L1.
 template <int D>
 __device__ __forceinline__ void merge_pieces(const DecodeArgs &a, size_t seg, int s, int h, int c0, int c1,
                                              long long W, int C, int ctid) {
+    constexpr int kAhead = 4;
     const int G = a.group;
-    for (int e = ctid; e < G * D / 2; e += kConsumerWarps * 32) {
-        const int g = e / (D / 2), d = (e % (D / 2)) * 2;
-        float M = -INFINITY;
-        for (int c = c0; c <= c1; ++c)
-            if (weight_begin(c + 1, W, C) > weight_begin(c, W, C)) M = fmaxf(M, __ldcg(a.lse_part + (seg + c) * G + g));
-        float den = 0.f, a0 = 0.f, a1 = 0.f;
-        for (int c = c0; c <= c1; ++c) {
-            if (weight_begin(c + 1, W, C) <= weight_begin(c, W, C)) continue;
-            const size_t pr = (seg + c) * G + g;
-            const float w = fast_exp2(__ldcg(a.lse_part + pr) - M);
-            const float2 o = __ldcg(reinterpret_cast<const float2 *>(a.o_part + pr * D + d));
-            den += w;
-            a0 += w * o.x;
-            a1 += w * o.y;
+    const bool dense = W >= C;  // then every CTA in [c0, c1] holds a piece (no divisions needed)
+    auto holds = [&](int c) { return dense || weight_begin(c + 1, W, C) > weight_begin(c, W, C); };
+#pragma unroll 1
+    for (int e = ctid; e < G * (D / 4); e += kConsumerWarps * 32) {
+        const int g = e / (D / 4);
+        float M = -INFINITY, den = 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int cb = c0; cb <= c1; cb += kAhead) {
+            float lse[kAhead];
+            float4 o[kAhead];
+#pragma unroll
+            for (int i = 0; i < kAhead; ++i) {
+                const int c = cb + i;
+                lse[i] = -INFINITY;
+                if (c <= c1 && holds(c)) {
+                    const size_t pr = (seg + c) * G + g;
+                    lse[i] = __ldcg(a.lse_part + pr);
+                    o[i] = __ldcg(reinterpret_cast<const float4 *>(a.o_part + pr * D) + e % (D / 4));
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < kAhead; ++i) {
+                if (!(lse[i] > -INFINITY)) continue;  // no piece here
+                const float Mn = fmaxf(M, lse[i]);
+                const float r = fast_exp2(M - Mn), w = fast_exp2(lse[i] - Mn);
+                den = den * r + w;
+                acc.x = acc.x * r + w * o[i].x;
+                acc.y = acc.y * r + w * o[i].y;
+                acc.z = acc.z * r + w * o[i].z;
+                acc.w = acc.w * r + w * o[i].w;
+                M = Mn;
+            }
         }
         const size_t row = static_cast<size_t>(s) * a.num_q_heads + static_cast<size_t>(h) * G + g;
-        *reinterpret_cast<__nv_bfloat162 *>(static_cast<__nv_bfloat16 *>(a.out) + row * D + d) =
-            __floats2bfloat162_rn(a0 / den, a1 / den);
+        const float inv = 1.f / den;
+        __nv_bfloat162 *dst =
+            reinterpret_cast<__nv_bfloat162 *>(static_cast<__nv_bfloat16 *>(a.out) + row * D + (e % (D / 4)) * 4);
+        dst[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+        dst[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
     }
 }
 
@@ -791,14 +821,15 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
                     if (prev == old) break;
                     old = prev;
                 }
-                sm.merge_flag[0] = static_cast<int>(now & 0xffffull) == npieces;
-                sm.merge_flag[1] = c0;
-                sm.merge_flag[2] = c1;
-            }
-            named_barrier_sync(1, kConsumerWarps * 32);
-            if (sm.merge_flag[0]) {
-                __threadfence();
-                merge_pieces<D>(a, seg, pc.s, pc.h, sm.merge_flag[1], sm.merge_flag[2], W, C, ctid);
+                const int pending = sm.merge_flag[0];
+                if (static_cast<int>(now & 0xffffull) == npieces && pending < 2) {  // never more than two (below)
+                    volatile int *m = sm.merge_flag + 1 + 4 * pending;
+                    m[0] = pc.s;
+                    m[1] = pc.h;
+                    m[2] = c0;
+                    m[3] = c1;
+                    sm.merge_flag[0] = pending + 1;
+                }
             }
         }
         named_barrier_sync(1, kConsumerWarps * 32);
@@ -812,6 +843,18 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
         if (warp == 0)
             for (int slot = 0; slot < 2; ++slot)
                 if ((q_issued >> slot) & 1u) mbar_wait_drain(&sm.qfull[slot], (q_issued_par >> slot) & 1u, a.status);
+    }
+    // The merges this CTA completes run after its last piece, when the loop's
+    // state is dead (a CTA's range cuts at most two segments: its first and
+    // its last piece; all pieces between are whole).
+    const int pending = sm.merge_flag[0];  // written by thread 0 before the loop's last barrier
+    for (int i = 0; i < pending; ++i) {
+        const volatile int *m = sm.merge_flag + 1 + 4 * i;
+        const int s = m[0], h = m[1], c0 = m[2], c1 = m[3];
+        __threadfence();
+        // the grid's total weight, reloaded rather than kept live across the loop
+        const long long Wt = static_cast<long long>(a.num_kv_heads) * sm.wprefix[a.num_seqs];
+        merge_pieces<D>(a, static_cast<size_t>(s) * a.num_kv_heads + h, s, h, c0, c1, Wt, gridDim.x, ctid);
     }
 }
 
@@ -848,6 +891,7 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathTensorCore ? 4 : 
         }
         for (int i = 0; i < 2; ++i) mbar_init(&sm.qfull[i], 1);
         *sm.abort_flag = 0;
+        sm.merge_flag[0] = 0;
         fence_mbar_init();
     }
     if (tid == 32) {

@@ -68,7 +68,7 @@ __host__ __device__ inline DecodeLayout decode_layout(int D, int BS, int GP, int
     L.bars = off;
     off += (kMaxStages + 2) * 8;                                    // full[stage], qfull[2]
     L.flags = off;
-    off += (kMaxStages + 1 + 2 * kConsumerWarps + 3) * 4;           // stage_bad, abort, scan scratch
+    off += (kMaxStages + 1 + 2 * kConsumerWarps + 1 + 4 * 2) * 4;   // stage_bad, abort, scan scratch, merges
     L.prefix = off;
     off += static_cast<uint32_t>(num_seqs + 1) * 4;                 // blocks before each sequence
     L.wprefix = off;
