@@ -56,6 +56,7 @@ def parse_args(argv=None):
     p.add_argument("--math", type=int, default=0)
     p.add_argument("--l2-prefetch", type=int, default=0)
     p.add_argument("--piece-cost", type=int, default=0)
+    p.add_argument("--head-pack", type=int, default=0)
     p.add_argument("--seqs", type=int, default=0,
                    help="build the workload with only its first N context lengths (small cases for ncu)")
     p.add_argument("--no-e2e", action="store_true")
@@ -223,7 +224,7 @@ class Step:
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
         self.opts = dict(num_ctas=args.num_ctas, num_stages=args.num_stages,
                          ctas_per_sm=args.ctas_per_sm, math=args.math, l2_prefetch=args.l2_prefetch,
-                         piece_cost=args.piece_cost)
+                         piece_cost=args.piece_cost, head_pack=args.head_pack)
         self.ws = pkv.allocate_workspace(b.num_seqs, b.num_q_heads, b.head_dim, device=device)
 
     def append(self, stream=None):
@@ -395,7 +396,7 @@ def config_block(args, batch, world):
     }
     if args.seqs:
         c["seqs_kept"] = args.seqs
-    for k in ("num_ctas", "num_stages", "ctas_per_sm", "math", "l2_prefetch", "piece_cost"):
+    for k in ("num_ctas", "num_stages", "ctas_per_sm", "math", "l2_prefetch", "piece_cost", "head_pack"):
         if getattr(args, k):
             c[k] = getattr(args, k)
     return c
@@ -415,6 +416,15 @@ def cpu_baseline(batch, kv, S, ctx_tokens, min_seconds=10.0, max_runs=5):
         oracle.decode_step(host)
         times.append(time.perf_counter() - t0)
     t = statistics.median(times)
+    # one thread, decode only, on the first sequences of the batch (about 2 s)
+    per_seq = t * host.context_lens.double() / max(1, ctx_tokens) * (os.cpu_count() or 1)
+    n1 = int(max(1, min(S, int((per_seq.cumsum(0) < 2.0).sum()) or 1)))
+    pairs = np.arange(n1 * host.num_q_heads, dtype=np.int64)
+    t0 = time.perf_counter()
+    oracle.paged_decode(host.q, host.k_cache, host.v_cache, host.block_tables.numpy(), host.context_lens.numpy(),
+                        host.num_kv_heads, host.block_size, host.scale, pairs=pairs, num_threads=1)
+    t1 = time.perf_counter() - t0
+    kv1 = int(host.context_lens[:n1].sum()) * host.num_kv_heads * host.head_dim * 2 * 2
     return {
         "value": round(kv / t / 1e9, 3),
         "unit": "GB/s",
@@ -423,6 +433,8 @@ def cpu_baseline(batch, kv, S, ctx_tokens, min_seconds=10.0, max_runs=5):
         "sample": f"whole batch ({S} seqs, {ctx_tokens} context tokens), append + decode, "
                   f"median of {len(times)} runs; {statistics.median(times):.2f} s per step",
         "seq_per_s": round(S / t, 2),
+        "single_thread": {"value": round(kv1 / t1 / 1e9, 4), "unit": "GB/s", "cores": 1,
+                          "sample": f"decode of the first {n1} sequences (all heads), {t1:.2f} s"},
     }
 
 

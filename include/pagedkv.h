@@ -83,6 +83,14 @@ extern "C" {
  *                     standing for a piece's fixed cost (1..64); -1 = none;
  *                     default 4. Keeps CTAs that get many short contexts from
  *                     finishing last.
+ *   head_pack         0 = default (2 where possible), 1 = off, 2 = read kv heads
+ *                     2h and 2h + 1 together as one head of twice the head_dim
+ *                     (the pool's [bs][Hkv][D] rows are the same bytes as
+ *                     [bs][Hkv/2][2D]), so that each token row of a read is
+ *                     256 contiguous bytes instead of 128. Possible on tensor
+ *                     cores with head_dim 64, an even num_kv_heads and a group
+ *                     of at most 4; asking for 2 elsewhere returns
+ *                     PKV_ERR_UNSUPPORTED.
  */
 typedef struct pkv_decode_options {
     int num_ctas;
@@ -91,6 +99,7 @@ typedef struct pkv_decode_options {
     int math;
     int l2_prefetch;
     int piece_cost;
+    int head_pack;
 } pkv_decode_options;
 
 /*

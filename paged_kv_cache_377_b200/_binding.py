@@ -32,7 +32,7 @@ class PagedKVError(RuntimeError):
 class _Options(ctypes.Structure):
     _fields_ = [("num_ctas", ctypes.c_int), ("num_stages", ctypes.c_int),
                 ("ctas_per_sm", ctypes.c_int), ("math", ctypes.c_int), ("l2_prefetch", ctypes.c_int),
-                ("piece_cost", ctypes.c_int)]
+                ("piece_cost", ctypes.c_int), ("head_pack", ctypes.c_int)]
 
 
 def library_path() -> str:
@@ -129,6 +129,7 @@ def paged_attn_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
                       block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float,
                       workspace: torch.Tensor, num_ctas: int = 0, num_stages: int = 0,
                       ctas_per_sm: int = 0, math: int = 0, l2_prefetch: int = 0, piece_cost: int = 0,
+                      head_pack: int = 0,
                       stream=None) -> torch.Tensor:
     """out[s, j] = softmax_t(scale * q[s, j] . K_t) . V_t over the sequence's paged tokens.
 
@@ -149,7 +150,7 @@ def paged_attn_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
         raise ValueError("shape mismatch between q/out or k_cache/v_cache")
     if block_tables.shape[0] != S or context_lens.shape[0] != S:
         raise ValueError("block_tables and context_lens must have num_seqs rows")
-    opts = _Options(num_ctas, num_stages, ctas_per_sm, math, l2_prefetch, piece_cost)
+    opts = _Options(num_ctas, num_stages, ctas_per_sm, math, l2_prefetch, piece_cost, head_pack)
     _check("paged_attn_decode", library().paged_attn_decode_ex(
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
         S, Hq, Hkv, D, bs, float(scale), block_tables.shape[1], NB, _ptr(workspace), workspace.numel(),

@@ -177,21 +177,32 @@ int paged_attn_decode_ex(void *out, const void *q, const void *k_cache, const vo
         !aligned(workspace, 256))
         return fail(PKV_ERR_INVALID_ARGUMENT,
                     "out, q, k_cache and v_cache must be 16-byte aligned and workspace 256-byte aligned");
-    pkv_decode_options o = {0, 0, 0, 0, 0, 0};
+    pkv_decode_options o = {0, 0, 0, 0, 0, 0, 0};
     if (opts) o = *opts;
     if (o.num_ctas < 0 || o.num_stages < 0 || o.ctas_per_sm < 0 || o.math < 0 || o.math > 2 ||
-        o.l2_prefetch < -1 || o.l2_prefetch > 32 || o.piece_cost < -1 || o.piece_cost > 64)
+        o.l2_prefetch < -1 || o.l2_prefetch > 32 || o.piece_cost < -1 || o.piece_cost > 64 || o.head_pack < 0 ||
+        o.head_pack > 2)
         return fail(PKV_ERR_INVALID_ARGUMENT, "negative or unknown option");
     if (o.num_ctas > pkv::kMaxCtas)
         return fail(PKV_ERR_INVALID_ARGUMENT, "num_ctas %d exceeds %d", o.num_ctas, pkv::kMaxCtas);
     if (static_cast<int64_t>(num_kv_heads) * (max_blocks_per_seq + 64) * pkv::kMaxSeqsPerLaunch > 0x7fffffff)
         return fail(PKV_ERR_INVALID_ARGUMENT, "num_kv_heads * max_blocks_per_seq too large");
     const int math = o.math ? o.math : pkv::kMathTensorCore;
-    const int ns = o.num_stages ? o.num_stages : default_stages(head_dim, block_size, math);
+    // Head packing: kv heads 2h, 2h + 1 of head_dim 64 read as one head of 128
+    // (256-byte rows instead of 128-byte ones); the kernel then sees half the
+    // kv heads, twice the head_dim and twice the group.
+    const bool can_pack = math == pkv::kMathTensorCore && head_dim == 64 && num_kv_heads % 2 == 0 &&
+                          2 * group <= PKV_MAX_GROUP;
+    if (o.head_pack == 2 && !can_pack)
+        return fail(PKV_ERR_UNSUPPORTED, "head_pack 2 needs tensor-core math, head_dim 64, an even num_kv_heads "
+                                         "and num_q_heads / num_kv_heads <= %d", PKV_MAX_GROUP / 2);
+    const int pack = o.head_pack == 1 ? 1 : can_pack ? 2 : 1;
+    const int kd = head_dim * pack, khkv = num_kv_heads / pack, kgroup = group * pack;  // as the kernel sees them
+    const int ns = o.num_stages ? o.num_stages : default_stages(kd, block_size, math);
     if (ns < 1 || ns > pkv::kMaxStagesPerWarp)
         return fail(PKV_ERR_INVALID_ARGUMENT, "num_stages %d outside [1, %d]", ns, pkv::kMaxStagesPerWarp);
-    const int gp = group_pad(group);
-    if (!pkv::decode_variant_exists(head_dim, block_size, gp, math))
+    const int gp = group_pad(kgroup);
+    if (!pkv::decode_variant_exists(kd, block_size, gp, math))
         return fail(PKV_ERR_UNSUPPORTED, "no kernel for head_dim %d, block_size %d, group %d, math %d", head_dim,
                     block_size, group, math);
     const WorkspaceLayout wl = workspace_layout(num_seqs, num_q_heads, head_dim);
@@ -202,8 +213,8 @@ int paged_attn_decode_ex(void *out, const void *q, const void *k_cache, const vo
     if (num_seqs == 0) return ok();
 
     CUtensorMap tm_k, tm_v;
-    if ((rc = make_pool_map(&tm_k, k_cache, num_blocks, block_size, num_kv_heads, head_dim)) != PKV_OK) return rc;
-    if ((rc = make_pool_map(&tm_v, v_cache, num_blocks, block_size, num_kv_heads, head_dim)) != PKV_OK) return rc;
+    if ((rc = make_pool_map(&tm_k, k_cache, num_blocks, block_size, khkv, kd)) != PKV_OK) return rc;
+    if ((rc = make_pool_map(&tm_v, v_cache, num_blocks, block_size, khkv, kd)) != PKV_OK) return rc;
 
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -214,9 +225,9 @@ int paged_attn_decode_ex(void *out, const void *q, const void *k_cache, const vo
     // in shared memory); launches run in stream order and reuse the workspace.
     for (int s0 = 0; s0 < num_seqs; s0 += pkv::kMaxSeqsPerLaunch) {
         const int sc = num_seqs - s0 < pkv::kMaxSeqsPerLaunch ? num_seqs - s0 : pkv::kMaxSeqsPerLaunch;
-        const size_t smem = pkv::decode_smem_bytes(head_dim, block_size, gp, group, math, ns, sc);
+        const size_t smem = pkv::decode_smem_bytes(kd, block_size, gp, kgroup, math, ns, sc);
         int per_sm = 0;
-        cudaError_t e = pkv::decode_prepare(head_dim, block_size, gp, math, smem, &per_sm);
+        cudaError_t e = pkv::decode_prepare(kd, block_size, gp, math, smem, &per_sm);
         if (e != cudaSuccess) return cuda_fail(e, "decode kernel setup");
         if (per_sm <= 0) return fail(PKV_ERR_INVALID_ARGUMENT, "shared memory %zu bytes per CTA does not fit", smem);
         if (o.ctas_per_sm > 0 && o.ctas_per_sm < per_sm) per_sm = o.ctas_per_sm;
@@ -234,15 +245,16 @@ int paged_attn_decode_ex(void *out, const void *q, const void *k_cache, const vo
         a.status = reinterpret_cast<int32_t *>(ws);
         a.num_seqs = sc;
         a.num_q_heads = num_q_heads;
-        a.num_kv_heads = num_kv_heads;
-        a.group = group;
+        a.num_kv_heads = khkv;
+        a.group = kgroup;
+        a.pack = pack;
         a.max_blocks_per_seq = max_blocks_per_seq;
         a.num_blocks = num_blocks;
         a.num_stages = ns;
         a.prefetch = o.l2_prefetch > 0 ? o.l2_prefetch : o.l2_prefetch == 0 ? kDefaultL2Prefetch : 0;
         a.piece_cost = o.piece_cost > 0 ? o.piece_cost : o.piece_cost == 0 ? kDefaultPieceCost : 0;
         a.scale_log2 = scale * 1.4426950408889634f;
-        e = pkv::decode_launch(head_dim, block_size, gp, math, tm_k, tm_v, a, grid, smem, st);
+        e = pkv::decode_launch(kd, block_size, gp, math, tm_k, tm_v, a, grid, smem, st);
         if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
     }
     return ok();

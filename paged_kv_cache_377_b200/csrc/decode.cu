@@ -185,7 +185,7 @@ struct CoreMath {
     }
 
     // query rows of the GQA group, pre-scaled into base-2 logits
-    __device__ __forceinline__ void load_q(uint32_t qslot, int group, float scale_log2) {
+    __device__ __forceinline__ void load_q(uint32_t qslot, int group, float scale_log2, int /*pack: always 1 here*/) {
         const uint32_t qa = qslot + ch * 16;
         const float2 sc = make_float2(scale_log2, scale_log2);
 #pragma unroll
@@ -388,13 +388,19 @@ struct MmaMath {
     }
 
     // B fragment (k = dim, n = head): two consecutive dims of q[l/4]; heads past the group are 0.
-    __device__ __forceinline__ void load_q(uint32_t qslot, int group, float sl2) {
+    // With pack = 2 the slot holds rows of D / 2 dims and query row g is
+    // placed in half g / (group / 2) of the virtual head, zeros in the other.
+    __device__ __forceinline__ void load_q(uint32_t qslot, int group, float sl2, int pack) {
         scale_log2 = sl2;
         const int g = lane >> 2, k2 = (lane & 3) * 2;
+        const int half = pack == 2 ? g / (group >> 1) : 0;
+        const int dr = D / pack;  // dims per stored row
 #pragma unroll
         for (int kk = 0; kk < KST; ++kk) {
-            qb[kk][0] = g < group ? lds32(qslot + (g * D + 16 * kk + k2) * 2) : 0u;
-            qb[kk][1] = g < group ? lds32(qslot + (g * D + 16 * kk + 8 + k2) * 2) : 0u;
+            const bool mine = g < group && (pack == 1 || kk / (KST / 2) == half);
+            const int col = 16 * kk - half * dr;
+            qb[kk][0] = mine ? lds32(qslot + (g * dr + col + k2) * 2) : 0u;
+            qb[kk][1] = mine ? lds32(qslot + (g * dr + col + 8 + k2) * 2) : 0u;
         }
     }
 
@@ -544,60 +550,69 @@ struct Smem {
     uint64_t *full, *qfull;
     volatile int *stage_bad;
     volatile int *abort_flag;
-    volatile int *merge_flag;  // [1 + 4 * 2]: how many segments this CTA completed (<= 2), then
-                               // for each (s, h, first CTA, last CTA)
+    volatile int *merge_flag;  // [1 + 2 * 2]: how many segments this CTA completed (<= 2), then
+                               // (s, h) of each
     int *scan;
     int *prefix;
     int *wprefix;
     int *lens;
 };
 
-// The CTAs holding pieces of segment (s, h): c0 .. c1, skipping CTAs whose
-// weight range is empty; npieces = how many hold one. CTA c covers weight
-// positions [c W / C, (c + 1) W / C), so position v lies in CTA ((v + 1) C - 1) / W.
-__device__ __forceinline__ void segment_ctas(int s, int h, const Smem &sm, int Hkv, long long W, int C, int pcost,
-                                             int &c0, int &c1, int &npieces) {
+// The CTAs holding pieces of segment (s, h). CTA c covers weight positions
+// [c W / C, (c + 1) W / C), so position v lies in CTA ((v + 1) C - 1) / W; the
+// segment's real blocks sit at positions v_first .. v_first + n - 1. With
+// W >= C no CTA range is empty and the pieces are held by CTAs c0 .. c0 +
+// npieces - 1; with W < C every range holds at most one position, so each of
+// the n blocks is a piece of its own, in CTA ((v_first + i + 1) C - 1) / W.
+struct SegmentSpan {
+    long long v_first;
+    int c0, npieces;
+};
+
+__device__ __forceinline__ SegmentSpan segment_span(int s, int h, const Smem &sm, int Hkv, long long W, int C,
+                                                    int pcost) {
+    SegmentSpan sp;
     const int n = sm.prefix[s + 1] - sm.prefix[s];
-    const long long v_first = static_cast<long long>(Hkv) * sm.wprefix[s] + static_cast<long long>(h) * (n + pcost) + pcost;
-    c0 = static_cast<int>(((v_first + 1) * C - 1) / W);
-    c1 = static_cast<int>(((v_first + n) * C - 1) / W);
-    if (W >= C) {  // no CTA range is empty
-        npieces = c1 - c0 + 1;
-        return;
-    }
-    npieces = 0;
-    for (int c = c0; c <= c1; ++c) npieces += weight_begin(c + 1, W, C) > weight_begin(c, W, C);
+    sp.v_first = static_cast<long long>(Hkv) * sm.wprefix[s] + static_cast<long long>(h) * (n + pcost) + pcost;
+    sp.c0 = static_cast<int>(((sp.v_first + 1) * C - 1) / W);
+    sp.npieces = W >= C ? static_cast<int>(((sp.v_first + n) * C - 1) / W) - sp.c0 + 1 : n;
+    return sp;
 }
 
-// Merge of the pieces of segment (s, h) stored by CTAs c0 .. c1 (log-sum-exp
-// identity, pieces in CTA order): out = sum_c 2^(lse_c - M) o_c / sum_c 2^(lse_c - M),
-// taken in one pass with a running maximum. A thread merges 4-dim elements of
-// the G x D output (at most two) and loads four pieces ahead, so that the merge
-// costs a few L2 round trips rather than one per piece. Partials written by
-// other SMs are read past L1.
+// The CTA holding piece i of a segment.
+__device__ __forceinline__ int piece_cta(const SegmentSpan &sp, int i, long long W, int C) {
+    return W >= C ? sp.c0 + i : static_cast<int>(((sp.v_first + i + 1) * C - 1) / W);
+}
+
+// Merge of the pieces of segment (s, h), held by CTAs piece_ctas[0 ..
+// npieces) (log-sum-exp identity, pieces in CTA order): out = sum_c 2^(lse_c - M) o_c / sum_c 2^(lse_c - M), taken in one
+// pass with a running maximum. A thread merges 4-dim elements of the G x D
+// output (at most two) and loads four pieces ahead, so that the merge costs a
+// few L2 round trips rather than one per piece. Partials written by other SMs
+// are read past L1.
 template <int D>
-__device__ __forceinline__ void merge_pieces(const DecodeArgs &a, size_t seg, int s, int h, int c0, int c1,
-                                             long long W, int C, int ctid) {
+__device__ __forceinline__ void merge_pieces(const DecodeArgs &a, const int *piece_ctas, int npieces, size_t seg,
+                                             int s, int h, int ctid) {
     constexpr int kAhead = 4;
     const int G = a.group;
-    const bool dense = W >= C;  // then every CTA in [c0, c1] holds a piece (no divisions needed)
-    auto holds = [&](int c) { return dense || weight_begin(c + 1, W, C) > weight_begin(c, W, C); };
+    const int DR = D / a.pack;
 #pragma unroll 1
     for (int e = ctid; e < G * (D / 4); e += kConsumerWarps * 32) {
         const int g = e / (D / 4);
+        const int col = (e % (D / 4)) * 4 - (a.pack == 2 ? g / (G >> 1) : 0) * DR;
+        if (col < 0 || col >= DR) continue;  // the other half of a packed virtual head
         float M = -INFINITY, den = 0.f;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int cb = c0; cb <= c1; cb += kAhead) {
+        for (int ib = 0; ib < npieces; ib += kAhead) {
             float lse[kAhead];
             float4 o[kAhead];
 #pragma unroll
             for (int i = 0; i < kAhead; ++i) {
-                const int c = cb + i;
                 lse[i] = -INFINITY;
-                if (c <= c1 && holds(c)) {
-                    const size_t pr = (seg + c) * G + g;
+                if (ib + i < npieces) {
+                    const size_t pr = (seg + piece_ctas[ib + i]) * G + g;
                     lse[i] = __ldcg(a.lse_part + pr);
-                    o[i] = __ldcg(reinterpret_cast<const float4 *>(a.o_part + pr * D) + e % (D / 4));
+                    o[i] = __ldcg(reinterpret_cast<const float4 *>(a.o_part + pr * DR + col));
                 }
             }
 #pragma unroll
@@ -616,7 +631,7 @@ __device__ __forceinline__ void merge_pieces(const DecodeArgs &a, size_t seg, in
         const size_t row = static_cast<size_t>(s) * a.num_q_heads + static_cast<size_t>(h) * G + g;
         const float inv = 1.f / den;
         __nv_bfloat162 *dst =
-            reinterpret_cast<__nv_bfloat162 *>(static_cast<__nv_bfloat16 *>(a.out) + row * D + (e % (D / 4)) * 4);
+            reinterpret_cast<__nv_bfloat162 *>(static_cast<__nv_bfloat16 *>(a.out) + row * DR + col);
         dst[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
         dst[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
     }
@@ -639,7 +654,8 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
     constexpr uint32_t kHalf = BS * 128;
     const int R = a.num_stages;
     const int G = a.group;
-    const uint32_t qbytes = static_cast<uint32_t>(G * D * 2);
+    const int DR = D / a.pack;  // dims per row of q, out and the partials
+    const uint32_t qbytes = static_cast<uint32_t>(G * DR * 2);
     const uint32_t sbase = smem_u32(sm.base);
     float *merge_acc = reinterpret_cast<float *>(sm.base + ly.merge_acc);
     float *merge_m = reinterpret_cast<float *>(sm.base + ly.merge_m);
@@ -727,7 +743,7 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
         if (warp == 0 && lane == 0 && !*sm.abort_flag) {
             const int slot = n & 1;
             const __nv_bfloat16 *src = static_cast<const __nv_bfloat16 *>(a.q) +
-                                       (static_cast<size_t>(pa.s) * a.num_q_heads + static_cast<size_t>(pa.h) * G) * D;
+                                       (static_cast<size_t>(pa.s) * a.num_q_heads + static_cast<size_t>(pa.h) * G) * DR;
             mbar_arrive_expect_tx(&sm.qfull[slot], qbytes);
             bulk_load(sm.base + ly.qbuf + slot * qbytes, src, qbytes, &sm.qfull[slot]);
             q_issued |= 1u << slot;
@@ -748,7 +764,7 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
         const int slot = npiece & 1;
         if (npiece >= 1 && ahead.next(pa)) issue_q(n_ahead++);  // every warp has read slot (npiece + 1) % 2
         mbar_wait_bounded(&sm.qfull[slot], static_cast<uint32_t>(npiece >> 1) & 1u, sm.abort_flag, a.status);
-        math.load_q(sbase + ly.qbuf + slot * qbytes, G, a.scale_log2);
+        math.load_q(sbase + ly.qbuf + slot * qbytes, G, a.scale_log2, a.pack);
         math.reset();
         ++npiece;
 
@@ -779,6 +795,8 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
         const size_t seg = static_cast<size_t>(pc.s) * a.num_kv_heads + pc.h;
         for (int e = ctid; e < G * D / 2; e += kConsumerWarps * 32) {
             const int g = e / (D / 2), d = (e % (D / 2)) * 2;
+            const int col = d - (a.pack == 2 ? g / (G >> 1) : 0) * DR;  // dim within the stored row
+            if (col < 0 || col >= DR) continue;  // the other half of a packed virtual head
             float M = -INFINITY;
 #pragma unroll
             for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, merge_m[w * G + g]);
@@ -797,12 +815,12 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
             const float o1 = ls > 0.f ? a1 / ls : 0.f;
             if (pc.whole) {
                 const size_t row = static_cast<size_t>(pc.s) * a.num_q_heads + static_cast<size_t>(pc.h) * G + g;
-                *reinterpret_cast<__nv_bfloat162 *>(static_cast<__nv_bfloat16 *>(a.out) + row * D + d) =
+                *reinterpret_cast<__nv_bfloat162 *>(static_cast<__nv_bfloat16 *>(a.out) + row * DR + col) =
                     __floats2bfloat162_rn(o0, o1);
             } else {
                 const size_t pr = (seg + blockIdx.x) * G + g;  // piece (segment + CTA), row g
-                *reinterpret_cast<float2 *>(a.o_part + pr * D + d) = make_float2(o0, o1);
-                if (d == 0) a.lse_part[pr] = ls > 0.f ? M + __log2f(ls) : -INFINITY;
+                *reinterpret_cast<float2 *>(a.o_part + pr * DR + col) = make_float2(o0, o1);
+                if (col == 0) a.lse_part[pr] = ls > 0.f ? M + __log2f(ls) : -INFINITY;
             }
         }
         if (!pc.whole) {
@@ -811,8 +829,7 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
             __threadfence();
             named_barrier_sync(1, kConsumerWarps * 32);
             if (ctid == 0) {
-                int c0, c1, npieces;
-                segment_ctas(pc.s, pc.h, sm, a.num_kv_heads, W, C, pcost, c0, c1, npieces);
+                const SegmentSpan sp = segment_span(pc.s, pc.h, sm, a.num_kv_heads, W, C, pcost);
                 unsigned long long *cnt = a.seg_count + seg;
                 unsigned long long old = atomicAdd(cnt, 0ull), now;
                 for (;;) {  // count = 1 for the first piece of this launch (stale epochs restart)
@@ -822,12 +839,10 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
                     old = prev;
                 }
                 const int pending = sm.merge_flag[0];
-                if (static_cast<int>(now & 0xffffull) == npieces && pending < 2) {  // never more than two (below)
-                    volatile int *m = sm.merge_flag + 1 + 4 * pending;
+                if (static_cast<int>(now & 0xffffull) == sp.npieces && pending < 2) {  // never more than two (below)
+                    volatile int *m = sm.merge_flag + 1 + 2 * pending;
                     m[0] = pc.s;
                     m[1] = pc.h;
-                    m[2] = c0;
-                    m[3] = c1;
                     sm.merge_flag[0] = pending + 1;
                 }
             }
@@ -847,14 +862,25 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
     // The merges this CTA completes run after its last piece, when the loop's
     // state is dead (a CTA's range cuts at most two segments: its first and
     // its last piece; all pieces between are whole).
-    const int pending = sm.merge_flag[0];  // written by thread 0 before the loop's last barrier
+    // (none after a wait gave up: a copy may still be landing in the stage buffers).
+    // The barrier makes every warp's drain complete and the flags final and
+    // the same for all threads.
+    named_barrier_sync(1, kConsumerWarps * 32);
+    const int pending = *sm.abort_flag ? 0 : sm.merge_flag[0];
     for (int i = 0; i < pending; ++i) {
-        const volatile int *m = sm.merge_flag + 1 + 4 * i;
-        const int s = m[0], h = m[1], c0 = m[2], c1 = m[3];
+        const volatile int *m = sm.merge_flag + 1 + 2 * i;
+        const int s = m[0], h = m[1];
         __threadfence();
         // the grid's total weight, reloaded rather than kept live across the loop
         const long long Wt = static_cast<long long>(a.num_kv_heads) * sm.wprefix[a.num_seqs];
-        merge_pieces<D>(a, static_cast<size_t>(s) * a.num_kv_heads + h, s, h, c0, c1, Wt, gridDim.x, ctid);
+        const SegmentSpan sp = segment_span(s, h, sm, a.num_kv_heads, Wt, gridDim.x, pcost);
+        // the CTA of each piece, listed in the (now idle) stage buffers: at least
+        // 16 KB, and a segment has at most kMaxCtas pieces
+        int *piece_ctas = reinterpret_cast<int *>(sm.base + ly.stages);
+        if (i > 0) named_barrier_sync(1, kConsumerWarps * 32);  // the previous merge is done with the list
+        for (int j = ctid; j < sp.npieces; j += kConsumerWarps * 32) piece_ctas[j] = piece_cta(sp, j, Wt, gridDim.x);
+        named_barrier_sync(1, kConsumerWarps * 32);
+        merge_pieces<D>(a, piece_ctas, sp.npieces, static_cast<size_t>(s) * a.num_kv_heads + h, s, h, ctid);
     }
 }
 
@@ -958,9 +984,9 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathTensorCore ? 4 : 
     if (blockIdx.x == 0)  // sequences with no context get all-zero rows (no piece covers them)
         for (int s = 0; s < S; ++s)
             if (sm.lens[s] == 0)
-                for (int e = tid; e < a.num_q_heads * D / 2; e += kDecodeThreads)
+                for (int e = tid; e < a.num_q_heads * (D / a.pack) / 2; e += kDecodeThreads)
                     reinterpret_cast<__nv_bfloat162 *>(static_cast<__nv_bfloat16 *>(a.out) +
-                                                       static_cast<size_t>(s) * a.num_q_heads * D)[e] =
+                                                       static_cast<size_t>(s) * a.num_q_heads * (D / a.pack))[e] =
                         __floats2bfloat162_rn(0.f, 0.f);
 
     const long long W = static_cast<long long>(a.num_kv_heads) * sm.wprefix[S];

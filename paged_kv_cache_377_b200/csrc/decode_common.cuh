@@ -14,12 +14,18 @@ constexpr int kMaxSeqsPerLaunch = 2048;               // per-sequence tables kep
 constexpr int kMaxCtas = 1024;                        // grid limit; bounds the pieces of a launch
 constexpr int kWorkspaceHeaderBytes = 256;
 
+// With pack = 2 the kernel runs on a view of the pool with half the kv heads
+// and twice the head_dim: kv heads 2h', 2h' + 1 of head_dim D / 2 are the two
+// halves of one 'virtual' head h' of head_dim D, and its 2G query rows are the
+// real query heads of both (query row p G + g sees only half p). num_kv_heads,
+// group and D below are then the virtual ones; q, out and the partials keep the
+// real head_dim D / pack per row.
 struct DecodeArgs {
-    void *out;                   // bf16 [S][Hq][D]
-    const void *q;               // bf16 [S][Hq][D]
+    void *out;                   // bf16 [S][Hq][D / pack]
+    const void *q;               // bf16 [S][Hq][D / pack]
     const int32_t *block_tables; // [S][MB]
     const int32_t *context_lens; // [S]
-    float *o_part;               // fp32 [piece][G][D], piece = s * Hkv + h + cta
+    float *o_part;               // fp32 [piece][G][D / pack], piece = s * Hkv + h + cta
     float *lse_part;             // fp32 [piece][G], log2 domain
     unsigned long long *seg_count;  // [S * Hkv] (call epoch << 16 | pieces stored), per segment
     unsigned long long epoch;    // this launch's epoch (< 2^48), unique in the process
@@ -33,6 +39,7 @@ struct DecodeArgs {
     int num_stages;              // ring stages per warp (R); the CTA holds 4R
     int prefetch;                // blocks a warp prefetches into L2 beyond the one it loads (0 = none)
     int piece_cost;              // extra weight, in blocks, of every non-empty segment when splitting work
+    int pack;                    // 1, or 2: two real kv heads per virtual head (see above)
     float scale_log2;            // scale * log2(e): logits are kept in base 2
 };
 

@@ -98,6 +98,18 @@ def test_options_are_checked():
     rc = lib.paged_attn_decode_ex(P, P, P, P, P, P, 4, 2, 1, 64, 16, 0.125, 3, 16, P, 1 << 20,
                                   ctypes.byref(opts), None)
     assert rc == -1 and "num_stages" in lib.pkv_last_error().decode()
+    opts = pkv._binding._Options(0, 0, 0, 0, 0, 0, 3)
+    rc = lib.paged_attn_decode_ex(P, P, P, P, P, P, 4, 2, 1, 64, 16, 0.125, 3, 16, P, 1 << 20,
+                                  ctypes.byref(opts), None)
+    assert rc == -1 and "unknown option" in lib.pkv_last_error().decode()
+    # packing two kv heads needs an even number of them (here 1) and head_dim 64
+    opts = pkv._binding._Options(0, 0, 0, 0, 0, 0, 2)
+    rc = lib.paged_attn_decode_ex(P, P, P, P, P, P, 4, 2, 1, 64, 16, 0.125, 3, 16, P, 1 << 20,
+                                  ctypes.byref(opts), None)
+    assert rc == -2 and "head_pack" in lib.pkv_last_error().decode()
+    rc = lib.paged_attn_decode_ex(P, P, P, P, P, P, 4, 8, 2, 128, 16, 0.125, 3, 16, P, 1 << 20,
+                                  ctypes.byref(opts), None)
+    assert rc == -2 and "head_pack" in lib.pkv_last_error().decode()
 
 
 def test_binding_refuses_cpu_tensors():

@@ -77,7 +77,9 @@ def test_grid_sizes_split_contexts_differently(name, num_ctas, math):
                                   dict(num_stages=3, ctas_per_sm=2, num_ctas=100),
                                   dict(math=2, num_stages=1), dict(math=2, num_stages=4, ctas_per_sm=1),
                                   dict(l2_prefetch=-1), dict(l2_prefetch=32), dict(math=1, l2_prefetch=5),
-                                  dict(piece_cost=-1), dict(piece_cost=64), dict(piece_cost=7, num_ctas=333)])
+                                  dict(piece_cost=-1), dict(piece_cost=64), dict(piece_cost=7, num_ctas=333),
+                                  dict(head_pack=1), dict(head_pack=2), dict(head_pack=2, num_ctas=1024),
+                                  dict(head_pack=2, num_ctas=5)])
 def test_launch_options(opts):
     b, ref, _, _ = config_case("opt125m")
     out, _, _, st = run_step(b, **opts)
@@ -101,11 +103,13 @@ def test_every_group_size_and_shape(G, D, bs):
     lens = [1, bs - 1, bs, bs + 1, 3 * bs + 5, 700, 0, 1029]
     b = workloads.make_custom(1000 + G * 7 + D + bs, lens, 2 * G, 2, D, bs)
     ref, _, _ = oracle.decode_step(b)
-    for math in MATHS:
+    # head_pack 0 packs kv-head pairs where it can (tensor cores, D 64, G <= 4); 1 never does
+    for math, pack in [(1, 0), (2, 0), (2, 1)]:
         for num_ctas in (0, 37):
-            out, _, _, st = run_step(b, num_ctas=num_ctas, math=math)
+            out, _, _, st = run_step(b, num_ctas=num_ctas, math=math, head_pack=pack)
             assert st == 0
-            assert_close_to_oracle(out.double().numpy(), ref, what=f"G={G} D={D} bs={bs} C={num_ctas} math={math}")
+            assert_close_to_oracle(out.double().numpy(), ref,
+                                   what=f"G={G} D={D} bs={bs} C={num_ctas} math={math} pack={pack}")
 
 
 @pytest.mark.parametrize("math", MATHS)
