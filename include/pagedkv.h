@@ -154,6 +154,39 @@ int paged_attn_decode_ex(void *out, const void *q, const void *k_cache, const vo
                          void *stream);
 
 /*
+ * One whole decode step in one launch: kv_cache_append of the step's token of
+ * every sequence, then paged_attn_decode over contexts that include it (the
+ * decode step of "Deep Dive into vLLM", section 2: each generated token's key
+ * and value are cached, and attention reads all cached tokens).
+ *
+ * Same arguments as paged_attn_decode_ex, plus
+ * k_new, v_new   device bf16 [num_seqs][num_kv_heads][head_dim]: the step's key
+ *                and value of each sequence (16-byte aligned).
+ * slot_mapping   device int64 [num_seqs]: slot of sequence s's new token, which
+ *                must be the slot of its last position L_s - 1, i.e.
+ *                block_tables[s][(L_s - 1) / block_size] * block_size +
+ *                (L_s - 1) % block_size; < 0 = no append for s (attention then
+ *                reads position L_s - 1 from the pool as it is).
+ * k_cache, v_cache are written (the appended rows).
+ *
+ * Results (out and the pools) are bit-identical to kv_cache_append followed
+ * by paged_attn_decode_ex with the same options. The warp that computes the
+ * block holding position L_s - 1 takes the new rows from k_new / v_new into
+ * its staged copy of the block and writes them to the pool, so the append
+ * costs no launch and no extra read. A slot that is >= 0 but not the last
+ * position (or, for L_s = 0, not inside the pool) is not written and sets
+ * PKV_STATUS_BAD_SLOT in the workspace status word. The caller guarantees,
+ * as with any append, that no other sequence of the batch reads a slot that
+ * is being written (copy-on-write of shared blocks is the caller's).
+ */
+int paged_attn_decode_append(void *out, const void *q, const void *k_new, const void *v_new,
+                             const int64_t *slot_mapping, void *k_cache, void *v_cache,
+                             const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
+                             int num_q_heads, int num_kv_heads, int head_dim, int block_size, float scale,
+                             int max_blocks_per_seq, int num_blocks, void *workspace, size_t workspace_bytes,
+                             const pkv_decode_options *opts, void *stream);
+
+/*
  * paged_attn_decode for callers that cannot allocate device memory. The pages
  * have no counterpart to this call.
  *

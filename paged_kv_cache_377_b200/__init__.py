@@ -19,6 +19,7 @@ from ._binding import (  # noqa: F401
     library,
     library_path,
     paged_attn_decode,
+    paged_attn_decode_append,
     read_status,
     selftest_bounded_wait,
     validate,
@@ -32,6 +33,7 @@ __all__ = [
     "library",
     "library_path",
     "paged_attn_decode",
+    "paged_attn_decode_append",
     "read_status",
     "validate",
     "workspace_bytes",

@@ -70,6 +70,9 @@ def library() -> ctypes.CDLL:
             lib.paged_attn_decode_ex.restype = I
             lib.paged_attn_decode_ex.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, I, I, P, Z,
                                                  ctypes.POINTER(_Options), P]
+            lib.paged_attn_decode_append.restype = I
+            lib.paged_attn_decode_append.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, F, I, I, P, Z,
+                                                     ctypes.POINTER(_Options), P]
             lib.kv_cache_append.restype = I
             lib.kv_cache_append.argtypes = [P, P, P, P, P, I, I, I, I, I, P, P]
             lib.pkv_validate.restype = I
@@ -155,6 +158,43 @@ def paged_attn_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
         S, Hq, Hkv, D, bs, float(scale), block_tables.shape[1], NB, _ptr(workspace), workspace.numel(),
         ctypes.byref(opts), _stream(stream)))
+    return out
+
+
+def paged_attn_decode_append(out: torch.Tensor, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                             slot_mapping: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                             block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float,
+                             workspace: torch.Tensor, num_ctas: int = 0, num_stages: int = 0,
+                             ctas_per_sm: int = 0, math: int = 0, l2_prefetch: int = 0, piece_cost: int = 0,
+                             head_pack: int = 0, stream=None) -> torch.Tensor:
+    """One decode step in one launch: append k_new / v_new (bf16 [S, Hkv, D]) at
+    slot_mapping (int64 [S], the slot of each sequence's last position, < 0 =
+    none), then the same attention as paged_attn_decode over contexts that
+    include the new token. Bit-identical to kv_cache_append + paged_attn_decode.
+    """
+    _need(q, "q", torch.bfloat16, 3)
+    _need(out, "out", torch.bfloat16, 3)
+    _need(k_new, "k_new", torch.bfloat16, 3)
+    _need(v_new, "v_new", torch.bfloat16, 3)
+    _need(slot_mapping, "slot_mapping", torch.int64, 1)
+    _need(k_cache, "k_cache", torch.bfloat16, 4)
+    _need(v_cache, "v_cache", torch.bfloat16, 4)
+    _need(block_tables, "block_tables", torch.int32, 2)
+    _need(context_lens, "context_lens", torch.int32, 1)
+    _need(workspace, "workspace", torch.uint8, 1)
+    S, Hq, D = q.shape
+    NB, bs, Hkv, D2 = k_cache.shape
+    if out.shape != q.shape or v_cache.shape != k_cache.shape or D2 != D:
+        raise ValueError("shape mismatch between q/out or k_cache/v_cache")
+    if k_new.shape != (S, Hkv, D) or v_new.shape != k_new.shape or slot_mapping.shape[0] != S:
+        raise ValueError("k_new / v_new must be [num_seqs, num_kv_heads, head_dim] and slot_mapping [num_seqs]")
+    if block_tables.shape[0] != S or context_lens.shape[0] != S:
+        raise ValueError("block_tables and context_lens must have num_seqs rows")
+    opts = _Options(num_ctas, num_stages, ctas_per_sm, math, l2_prefetch, piece_cost, head_pack)
+    _check("paged_attn_decode_append", library().paged_attn_decode_append(
+        _ptr(out), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(slot_mapping), _ptr(k_cache), _ptr(v_cache),
+        _ptr(block_tables), _ptr(context_lens), S, Hq, Hkv, D, bs, float(scale), block_tables.shape[1], NB,
+        _ptr(workspace), workspace.numel(), ctypes.byref(opts), _stream(stream)))
     return out
 
 

@@ -147,12 +147,21 @@ int pkv_decode_workspace_bytes(int num_seqs, int num_q_heads, int head_dim, size
     return ok();
 }
 
-int paged_attn_decode_ex(void *out, const void *q, const void *k_cache, const void *v_cache,
-                         const int32_t *block_tables, const int32_t *context_lens, int num_seqs, int num_q_heads,
-                         int num_kv_heads, int head_dim, int block_size, float scale, int max_blocks_per_seq,
-                         int num_blocks, void *workspace, size_t workspace_bytes, const pkv_decode_options *opts,
-                         void *stream) {
+}  // extern "C"
+
+namespace {
+
+// Decode, optionally with the fused append (k_new, v_new, slots all non-NULL).
+int decode_impl(void *out, const void *q, const void *k_new, const void *v_new, const int64_t *slots,
+                const void *k_cache, const void *v_cache, const int32_t *block_tables, const int32_t *context_lens,
+                int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size, float scale,
+                int max_blocks_per_seq, int num_blocks, void *workspace, size_t workspace_bytes,
+                const pkv_decode_options *opts, void *stream) {
     if (num_seqs < 0) return fail(PKV_ERR_INVALID_ARGUMENT, "num_seqs < 0");
+    const bool fused = slots != nullptr;
+    if (fused && (!k_new || !v_new)) return fail(PKV_ERR_INVALID_ARGUMENT, "k_new and v_new must not be NULL");
+    if (fused && (!aligned(k_new, 16) || !aligned(v_new, 16)))
+        return fail(PKV_ERR_INVALID_ARGUMENT, "k_new and v_new must be 16-byte aligned");
     if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !workspace)
         return fail(PKV_ERR_INVALID_ARGUMENT, "a required pointer is NULL");
     if (num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || max_blocks_per_seq <= 0 ||
@@ -254,10 +263,44 @@ int paged_attn_decode_ex(void *out, const void *q, const void *k_cache, const vo
         a.prefetch = o.l2_prefetch > 0 ? o.l2_prefetch : o.l2_prefetch == 0 ? kDefaultL2Prefetch : 0;
         a.piece_cost = o.piece_cost > 0 ? o.piece_cost : o.piece_cost == 0 ? kDefaultPieceCost : 0;
         a.scale_log2 = scale * 1.4426950408889634f;
+        if (fused) {
+            const size_t row = static_cast<size_t>(num_kv_heads) * head_dim;  // elements per token
+            a.k_new = static_cast<const __nv_bfloat16 *>(k_new) + static_cast<size_t>(s0) * row;
+            a.v_new = static_cast<const __nv_bfloat16 *>(v_new) + static_cast<size_t>(s0) * row;
+            a.slots = slots + s0;
+            a.k_cache = const_cast<void *>(k_cache);
+            a.v_cache = const_cast<void *>(v_cache);
+        }
         e = pkv::decode_launch(kd, block_size, gp, math, tm_k, tm_v, a, grid, smem, st);
         if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
     }
     return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+int paged_attn_decode_ex(void *out, const void *q, const void *k_cache, const void *v_cache,
+                         const int32_t *block_tables, const int32_t *context_lens, int num_seqs, int num_q_heads,
+                         int num_kv_heads, int head_dim, int block_size, float scale, int max_blocks_per_seq,
+                         int num_blocks, void *workspace, size_t workspace_bytes, const pkv_decode_options *opts,
+                         void *stream) {
+    return decode_impl(out, q, nullptr, nullptr, nullptr, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                       num_q_heads, num_kv_heads, head_dim, block_size, scale, max_blocks_per_seq, num_blocks,
+                       workspace, workspace_bytes, opts, stream);
+}
+
+int paged_attn_decode_append(void *out, const void *q, const void *k_new, const void *v_new,
+                             const int64_t *slot_mapping, void *k_cache, void *v_cache,
+                             const int32_t *block_tables, const int32_t *context_lens, int num_seqs, int num_q_heads,
+                             int num_kv_heads, int head_dim, int block_size, float scale, int max_blocks_per_seq,
+                             int num_blocks, void *workspace, size_t workspace_bytes,
+                             const pkv_decode_options *opts, void *stream) {
+    if (!slot_mapping) return fail(PKV_ERR_INVALID_ARGUMENT, "slot_mapping must not be NULL");
+    return decode_impl(out, q, k_new, v_new, slot_mapping, k_cache, v_cache, block_tables, context_lens, num_seqs,
+                       num_q_heads, num_kv_heads, head_dim, block_size, scale, max_blocks_per_seq, num_blocks,
+                       workspace, workspace_bytes, opts, stream);
 }
 
 int paged_attn_decode(void *out, const void *q, const void *k_cache, const void *v_cache,

@@ -549,6 +549,7 @@ struct Smem {
     uint8_t *base;
     uint64_t *full, *qfull;
     volatile int *stage_bad;
+    int *stage_blk;  // [kMaxStages] physical block whose copy the stage holds
     volatile int *abort_flag;
     volatile int *merge_flag;  // [1 + 2 * 2]: how many segments this CTA completed (<= 2), then
                                // (s, h) of each
@@ -715,6 +716,7 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
         if (lane == 0 && !*sm.abort_flag) {
             const bool bad = p < 0 || p >= a.num_blocks;
             sm.stage_bad[stage] = bad ? 1 : 0;
+            sm.stage_blk[stage] = p;
             if (bad) {
                 atomicOr(a.status, PKV_STATUS_BAD_BLOCK_ID);
                 mbar_arrive(&sm.full[stage]);
@@ -777,10 +779,40 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
                 ring = 0;
                 rphase ^= 1u;
             }
+            // Fused append: the block holding position L - 1 takes the step's new
+            // row (fetched while the block's copy is in flight).
+            constexpr int kChunks = D / 8;  // 16-byte chunks of a row
+            const int bi = pc.b0 + i;      // block within the segment
+            const bool tail = a.slots != nullptr && (bi + 1) * BS >= pc.L;
+            long long slot = -1;
+            uint4 patch = make_uint4(0u, 0u, 0u, 0u);
+            if (tail) {
+                slot = __ldg(a.slots + pc.s);
+                if (slot >= 0 && lane < 2 * kChunks)
+                    patch = __ldg(reinterpret_cast<const uint4 *>(
+                        static_cast<const __nv_bfloat16 *>(lane < kChunks ? a.k_new : a.v_new) +
+                        (static_cast<size_t>(pc.s) * a.num_kv_heads + pc.h) * D + (lane % kChunks) * 8));
+            }
             if (mbar_wait_bounded(&sm.full[stage], par, sm.abort_flag, a.status)) inflight &= ~(1u << stage);
             if (!sm.stage_bad[stage] && !*sm.abort_flag) {
-                const int valid = min(BS, pc.L - (pc.b0 + i) * BS);
+                const int valid = min(BS, pc.L - bi * BS);
                 const uint32_t ktile = sbase + ly.stages + static_cast<uint32_t>(stage) * 2u * kTile;
+                if (tail && slot >= 0) {
+                    const int t = valid - 1;  // row of position L - 1 in this block
+                    const long long want = static_cast<long long>(sm.stage_blk[stage]) * BS + t;
+                    if (slot == want) {
+                        if (lane < 2 * kChunks) {
+                            const int c = lane % kChunks;
+                            sts128(tile_addr<BS>(lane < kChunks ? ktile : ktile + kTile, t, c), patch);
+                            *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(lane < kChunks ? a.k_cache : a.v_cache) +
+                                                       (static_cast<size_t>(want) * a.num_kv_heads + pc.h) * D + c * 8) = patch;
+                            fence_proxy_async_shared();  // before a later copy overwrites the stage
+                        }
+                        __syncwarp();
+                    } else if (lane == 0) {
+                        atomicOr(a.status, PKV_STATUS_BAD_SLOT);  // not the last position: not appended
+                    }
+                }
                 math.block(ktile, ktile + kTile, valid);
             }
             __syncwarp();
@@ -905,6 +937,7 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathTensorCore ? 4 : 
     sm.abort_flag = sm.stage_bad + kMaxStages;
     sm.scan = reinterpret_cast<int *>(sm.base + ly.flags) + kMaxStages + 1;
     sm.merge_flag = reinterpret_cast<volatile int *>(sm.scan + 2 * kConsumerWarps);
+    sm.stage_blk = const_cast<int *>(sm.merge_flag) + 1 + 4 * 2;
     sm.prefix = reinterpret_cast<int *>(sm.base + ly.prefix);
     sm.wprefix = reinterpret_cast<int *>(sm.base + ly.wprefix);
     sm.lens = reinterpret_cast<int *>(sm.base + ly.lens);
@@ -983,11 +1016,27 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathTensorCore ? 4 : 
     __syncthreads();
     if (blockIdx.x == 0)  // sequences with no context get all-zero rows (no piece covers them)
         for (int s = 0; s < S; ++s)
-            if (sm.lens[s] == 0)
+            if (sm.lens[s] == 0) {
                 for (int e = tid; e < a.num_q_heads * (D / a.pack) / 2; e += kDecodeThreads)
                     reinterpret_cast<__nv_bfloat162 *>(static_cast<__nv_bfloat16 *>(a.out) +
                                                        static_cast<size_t>(s) * a.num_q_heads * (D / a.pack))[e] =
                         __floats2bfloat162_rn(0.f, 0.f);
+                // fused append of a sequence with no context: no block computes it,
+                // so its rows go straight to the pool (if the slot is in it)
+                const long long slot = a.slots ? __ldg(a.slots + s) : -1;
+                if (slot >= static_cast<long long>(a.num_blocks) * BS) {
+                    if (tid == 0) atomicOr(a.status, PKV_STATUS_BAD_SLOT);
+                } else if (slot >= 0) {
+                    const size_t row = static_cast<size_t>(a.num_kv_heads) * D;  // elements of one token's row
+                    for (int e = tid; e < 2 * static_cast<int>(row / 8); e += kDecodeThreads) {
+                        const int kv = e / static_cast<int>(row / 8), c = e % static_cast<int>(row / 8);
+                        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(
+                            static_cast<const __nv_bfloat16 *>(kv ? a.v_new : a.k_new) + s * row + c * 8));
+                        *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(kv ? a.v_cache : a.k_cache) +
+                                                   static_cast<size_t>(slot) * row + c * 8) = v;
+                    }
+                }
+            }
 
     const long long W = static_cast<long long>(a.num_kv_heads) * sm.wprefix[S];
     const long long x0 = blocks_below(weight_begin(blockIdx.x, W, gridDim.x), sm.prefix, sm.wprefix, S,

@@ -40,6 +40,16 @@ struct DecodeArgs {
     int prefetch;                // blocks a warp prefetches into L2 beyond the one it loads (0 = none)
     int piece_cost;              // extra weight, in blocks, of every non-empty segment when splitting work
     int pack;                    // 1, or 2: two real kv heads per virtual head (see above)
+    // Fused append (slots != nullptr): the step's new token of sequence s, rows
+    // k_new[s][h] / v_new[s][h] ([S][Hkv][D] like a pool row), belongs at
+    // slots[s], which must be the slot of position L_s - 1. The warp that
+    // computes that block puts the rows into its staged tile (so attention
+    // sees them) and writes them to the pool.
+    const void *k_new;
+    const void *v_new;
+    const int64_t *slots;
+    void *k_cache;               // bf16 pool [NB][BS][Hkv][D], written by the fused append
+    void *v_cache;
     float scale_log2;            // scale * log2(e): logits are kept in base 2
 };
 
@@ -75,7 +85,7 @@ __host__ __device__ inline DecodeLayout decode_layout(int D, int BS, int GP, int
     L.bars = off;
     off += (kMaxStages + 2) * 8;                                    // full[stage], qfull[2]
     L.flags = off;
-    off += (kMaxStages + 1 + 2 * kConsumerWarps + 1 + 4 * 2) * 4;   // stage_bad, abort, scan scratch, merges
+    off += (2 * kMaxStages + 1 + 2 * kConsumerWarps + 1 + 4 * 2) * 4;  // stage_bad, abort, scan, merges, stage_blk
     L.prefix = off;
     off += static_cast<uint32_t>(num_seqs + 1) * 4;                 // blocks before each sequence
     L.wprefix = off;

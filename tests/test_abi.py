@@ -112,6 +112,20 @@ def test_options_are_checked():
     assert rc == -2 and "head_pack" in lib.pkv_last_error().decode()
 
 
+def test_fused_step_checks_its_extra_arguments():
+    lib = pkv.library()
+    args = [P, P, P, P, P, P, P, P, P, 4, 2, 1, 64, 16, 0.125, 3, 16, P, 1 << 20, None, None]
+    bad = list(args)
+    bad[4] = None  # slot_mapping
+    assert lib.paged_attn_decode_append(*bad) == -1 and "slot_mapping" in lib.pkv_last_error().decode()
+    bad = list(args)
+    bad[2] = None  # k_new
+    assert lib.paged_attn_decode_append(*bad) == -1 and "k_new" in lib.pkv_last_error().decode()
+    bad = list(args)
+    bad[3] = ctypes.c_void_p(4096 + 8)  # v_new misaligned
+    assert lib.paged_attn_decode_append(*bad) == -1 and "aligned" in lib.pkv_last_error().decode()
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     q = torch.zeros(1, 2, 64, dtype=torch.bfloat16)
