@@ -1,16 +1,19 @@
 #!/usr/bin/env python
 """Benchmark: one paged decode step (slot-mapped append + paged decode attention).
 
-A step is the whole hot path over one synthetic batch: kv_cache_append of the
-step's new keys/values, then paged_attn_decode (one persistent decode kernel
-that also merges the contexts it splits between CTAs). The default workload is
-the Llama-3-8B-shaped GQA batch (256 sequences, 32 q / 8 kv heads, head_dim 128,
+A step is the whole hot path over one synthetic batch: the append of each
+sequence's new key/value and the paged decode attention over contexts that
+include it, in one launch of paged_attn_decode_append (a persistent decode
+kernel that also merges the contexts it splits between CTAs); --two-launch
+runs kv_cache_append + paged_attn_decode instead. The default workload is the
+Llama-3-8B-shaped GQA batch (256 sequences, 32 q / 8 kv heads, head_dim 128,
 block_size 16, context lengths U[128, 4096], pool 1.2x the needed blocks,
 shuffled) -- 2.25 GB of K/V read per step, far larger than L2; L2 is also
 flushed (memset of 2x its size) between timed steps, outside the step's events.
 
-Prints one JSON line (rank 0). `value` is KV GB/s (algorithmic K+V bytes of
-the step / device time); see the design doc for the metric's definition.
+Prints one JSON line (rank 0). `value` is KV GB/s: the algorithmic bytes of
+the step, sum over sequences of context_len * num_kv_heads * head_dim * 2
+(K and V) * 2 (bf16), divided by the device time of the step.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 Under torchrun each rank runs its own independent batch (weak scaling, no
@@ -57,6 +60,8 @@ def parse_args(argv=None):
     p.add_argument("--l2-prefetch", type=int, default=0)
     p.add_argument("--piece-cost", type=int, default=0)
     p.add_argument("--head-pack", type=int, default=0)
+    p.add_argument("--two-launch", action="store_true",
+                   help="run the step as kv_cache_append + paged_attn_decode instead of the one-launch call")
     p.add_argument("--seqs", type=int, default=0,
                    help="build the workload with only its first N context lengths (small cases for ncu)")
     p.add_argument("--no-e2e", action="store_true")
@@ -205,9 +210,12 @@ class ClockSampler:
 # ----------------------------------------------------------------------------- our arm
 
 class Step:
-    """Device buffers of one decode step and the two library calls that make it."""
+    """Device buffers of one decode step and the library call(s) that make it:
+    paged_attn_decode_append (append + attention in one launch) by default, or
+    kv_cache_append followed by paged_attn_decode with --two-launch."""
 
     def __init__(self, batch, args, device):
+        self.fused = not args.two_launch
         import paged_kv_cache_377_b200 as pkv
         self.pkv = pkv
         b = batch
@@ -234,9 +242,30 @@ class Step:
         self.pkv.paged_attn_decode(self.out, self.q, self.kc, self.vc, self.bt, self.cl, self.b.scale, self.ws,
                                    stream=stream, **self.opts)
 
+    def fused_step(self, stream=None):
+        self.pkv.paged_attn_decode_append(self.out, self.q, self.k_new, self.v_new, self.slots, self.kc, self.vc,
+                                          self.bt, self.cl, self.b.scale, self.ws, stream=stream, **self.opts)
+
+    def run(self, stream=None, mid_event=None):
+        """One decode step; in two-launch mode `mid_event` is recorded between the calls."""
+        if self.fused:
+            self.fused_step(stream)
+            return
+        self.append(stream)
+        if mid_event is not None:
+            mid_event.record(stream if stream is not None else torch.cuda.current_stream())
+        self.decode(stream)
+
     def decode_launches(self):
-        """Kernels one paged_attn_decode call launches: one per 2048 sequences."""
+        """Decode kernels per call: one per 2048 sequences."""
         return -(-self.b.num_seqs // 2048)
+
+    def launches(self):
+        """Kernels of this library launched per step."""
+        return self.decode_launches() + (0 if self.fused else 1)
+
+    def status_word(self):
+        return self.pkv.read_status(self.status) | self.pkv.read_status(self.ws)
 
 
 def run_ours(args, rank, world, local_rank):
@@ -262,8 +291,7 @@ def run_ours(args, rank, world, local_rank):
             dist.barrier()
 
     for _ in range(args.warmup):
-        step.append()
-        step.decode()
+        step.run()
     torch.cuda.synchronize()
 
     K = args.steps
@@ -275,17 +303,16 @@ def run_ours(args, rank, world, local_rank):
         for i in range(K):
             flush.zero_()                      # L2 flush, outside the step's events
             ev[i][0].record(stream)
-            step.append()
-            ev[i][1].record(stream)
-            step.decode()
+            step.run(mid_event=ev[i][1])
             ev[i][2].record(stream)
         torch.cuda.synchronize()
     barrier()
     step_ms = [e[0].elapsed_time(e[2]) for e in ev]
-    decode_ms = [e[1].elapsed_time(e[2]) for e in ev]
-    append_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    # the decode kernel's time: the whole step when the append is fused into it
+    decode_ms = step_ms if step.fused else [e[1].elapsed_time(e[2]) for e in ev]
+    append_ms = None if step.fused else [e[0].elapsed_time(e[1]) for e in ev]
     total_ms = sum(step_ms)
-    status = step.pkv.read_status(step.status) | step.pkv.read_status(step.ws)
+    status = step.status_word()
     if status:
         raise RuntimeError(f"device status {status} after the timed steps")
 
@@ -321,11 +348,12 @@ def run_ours(args, rank, world, local_rank):
         "pct_of_hbm_peak": round(100.0 * value / (hbm * world), 2),
         "seq_per_s": round(job["seq_per_s"], 1),
         "ctx_tokens_per_s": round(job["ctx_tokens_per_s"], 1),
-        "append_us_mean": round(1e3 * statistics.fmean(append_ms), 3),
+        "append_us_mean": None if append_ms is None else round(1e3 * statistics.fmean(append_ms), 3),
         "decode_us_mean": round(1e3 * mean_decode_ms, 3),
         "decode_us_median": round(1e3 * statistics.median(decode_ms), 3),
         "roofline": {
-            "kernel": "paged_decode_kernel (one launch per paged_attn_decode call)",
+            "kernel": ("paged_decode_kernel (the step's one launch: append fused)" if step.fused else
+                       "paged_decode_kernel (one launch per paged_attn_decode call)"),
             "bound": "hbm",
             "achieved": round(achieved, 2),
             "peak": hbm,
@@ -336,7 +364,7 @@ def run_ours(args, rank, world, local_rank):
             "traffic": traffic,
         },
         "clocks": sampler.summary(),
-        "gpu_launches": K * (1 + step.decode_launches()),
+        "gpu_launches": K * step.launches(),
         "e2e": e2e,
         "cpu_baseline": cpu,
     }
@@ -356,8 +384,7 @@ def run_e2e(step, args, flush, stream, kv, world):
     def one():
         for n, t in host.items():
             getattr(step, n).copy_(t, non_blocking=True)
-        step.append()
-        step.decode()
+        step.run()
         out_host.copy_(step.out, non_blocking=True)
 
     for _ in range(max(args.warmup, 3)):
@@ -393,6 +420,8 @@ def config_block(args, batch, world):
         "kv_dtype": "bf16",
         "l2": "inputs larger than L2, and L2 flushed (memset 2x L2) between timed steps",
         "parallelism": "replicas: one independent batch per GPU" if world > 1 else "single GPU",
+        "step": ("kv_cache_append + paged_attn_decode (two launches)" if args.two_launch else
+                 "paged_attn_decode_append (append + attention, one launch)"),
     }
     if args.seqs:
         c["seqs_kept"] = args.seqs
