@@ -51,6 +51,7 @@ extern "C" {
 #define PKV_ERR_INVALID_ARGUMENT (-1) /* null pointer, bad size, misaligned pointer, small workspace */
 #define PKV_ERR_UNSUPPORTED (-2)      /* head_dim, block_size or head grouping not compiled in */
 #define PKV_ERR_CUDA (-3)             /* a CUDA runtime call or a launch failed */
+#define PKV_ERR_OUT_OF_BLOCKS (-4)    /* the block manager has too few free blocks; nothing changed */
 
 /* Bits of the device status word (sticky: kernels only OR bits in). */
 #define PKV_STATUS_BAD_BLOCK_ID 1     /* a needed table entry is outside [0, num_blocks); that block is skipped */
@@ -265,6 +266,105 @@ int pkv_read_status(int32_t *d_status, int32_t *status, int clear, void *stream)
  * is set instead if the wait wrongly succeeded.
  */
 int pkv_selftest_bounded_wait(int32_t *d_status, void *stream);
+
+/*
+ * Copy-on-write block copies: for c < num_copies, physical block dst[c] of
+ * both pools becomes a copy of block src[c] (block_size rows of num_kv_heads *
+ * head_dim bf16). src, dst: device int32 [num_copies] (from
+ * pkv_bm_take_copies). The copies must not chain (no dst is another copy's
+ * src); the block manager never produces such a list. An id outside
+ * [0, num_blocks) skips that copy and ORs PKV_STATUS_BAD_BLOCK_ID into
+ * *d_status (device int32, may be NULL). Runs on `stream`; issue it before any
+ * other write of the pools in the same step.
+ */
+int kv_block_copy(void *k_cache, void *v_cache, const int32_t *src, const int32_t *dst, int num_copies,
+                  int num_kv_heads, int head_dim, int block_size, int num_blocks, int32_t *d_status, void *stream);
+
+/*
+ * Host-side block manager of one KV pool (no CUDA calls; thread-safe).
+ *
+ * It follows the block-table scheme of "Deep Dive into vLLM" (section 2.1:
+ * logical blocks map to physical blocks through a per-sequence block table;
+ * section 2.2: blocks are allocated only when tokens are stored, and the
+ * sequences of parallel sampling or beam search share their prompt's blocks,
+ * copy-on-write like an OS) and runbyai post 449 (section 3: prompts that
+ * start alike share those blocks; section 4: a finished sequence's blocks are
+ * freed at once for new sequences). Each physical block has a reference
+ * count; a block is free exactly when the count is 0 (LIFO free list, block 0
+ * handed out first). Sequence ids are any int64 the caller chooses.
+ *
+ * A decode step with the manager: pkv_bm_append for every running sequence
+ * (each gives the slot of its new token, the slot of its last position),
+ * pkv_bm_take_copies, kv_block_copy of those copies, pkv_bm_pack of the running
+ * sequences' tables and lengths, then paged_attn_decode_append with the slots.
+ * Fork only between steps (after the step that wrote the parent's last token);
+ * pkv_bm_fork refuses while copies are pending.
+ *
+ * Errors: PKV_ERR_INVALID_ARGUMENT (unknown or reused id, bad sizes) and
+ * PKV_ERR_OUT_OF_BLOCKS leave the manager unchanged; pkv_bm_last_error()
+ * gives the message.
+ */
+typedef struct pkv_block_manager pkv_block_manager;
+
+/* A manager of num_blocks free blocks of block_size tokens; NULL if either is <= 0. */
+pkv_block_manager *pkv_bm_create(int num_blocks, int block_size);
+void pkv_bm_destroy(pkv_block_manager *bm);
+
+/* Free blocks, or a negative error code. */
+int pkv_bm_num_free(const pkv_block_manager *bm);
+
+/* References to `block` (sequences holding it + pending copies reading it). */
+int pkv_bm_refcount(const pkv_block_manager *bm, int block);
+
+/*
+ * A new sequence holding num_tokens tokens (its prompt). With prefix_seq >= 0,
+ * its first prefix_tokens tokens are those of sequence prefix_seq: the whole
+ * blocks among them (prefix_tokens / block_size blocks) are shared, not
+ * copied. slots (host int64 [num_tokens], may be NULL) receives each token's
+ * slot for writing the prompt with kv_cache_append, -1 for the shared tokens
+ * (already in the pool).
+ */
+int pkv_bm_add(pkv_block_manager *bm, int64_t seq_id, int64_t num_tokens, int64_t prefix_seq,
+               int64_t prefix_tokens, int64_t *slots);
+
+/* Sequence `child` shares every block of `parent` (same tokens). */
+int pkv_bm_fork(pkv_block_manager *bm, int64_t parent, int64_t child);
+
+/*
+ * Reserves the next position of the sequence for one new token; *slot = its
+ * slot. A full last block (or none) takes a fresh block; a last block that
+ * has room but is shared is first copied to a fresh block (copy-on-write: the
+ * copy is queued for pkv_bm_take_copies).
+ */
+int pkv_bm_append(pkv_block_manager *bm, int64_t seq_id, int64_t *slot);
+
+/* The sequence leaves: each of its blocks loses a reference. */
+int pkv_bm_free(pkv_block_manager *bm, int64_t seq_id);
+
+/* Copies queued since the last call (0 if none). */
+int pkv_bm_pending_copies(const pkv_block_manager *bm);
+
+/*
+ * Moves the queued copies, in queue order, into src / dst (host int32
+ * [capacity]) and returns how many; fails, taking none, if there are more
+ * than `capacity`. A queued copy holds a reference on its source block until
+ * it is taken, so the source cannot be reused before the copy is issued.
+ */
+int pkv_bm_take_copies(pkv_block_manager *bm, int32_t *src, int32_t *dst, int capacity);
+
+/* *len = the sequence's token count. */
+int pkv_bm_seq_len(const pkv_block_manager *bm, int64_t seq_id, int64_t *len);
+
+/*
+ * The step's inputs for sequences seq_ids[0 .. num_seqs): block_tables (host
+ * int32 [num_seqs][max_blocks_per_seq], padded with -1) and context_lens (host
+ * int32 [num_seqs]), as paged_attn_decode takes them.
+ */
+int pkv_bm_pack(const pkv_block_manager *bm, const int64_t *seq_ids, int num_seqs, int max_blocks_per_seq,
+                int32_t *block_tables, int32_t *context_lens);
+
+/* Message of the last failed block-manager call on this thread. */
+const char *pkv_bm_last_error(void);
 
 /* Message of the last failed call on this thread ("" if none). */
 const char *pkv_last_error(void);

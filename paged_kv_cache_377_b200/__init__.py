@@ -25,10 +25,14 @@ from ._binding import (  # noqa: F401
     validate,
     workspace_bytes,
 )
+from .block_manager import BlockManager, OutOfBlocks, kv_block_copy  # noqa: F401
 
 __all__ = [
+    "BlockManager",
+    "OutOfBlocks",
     "PagedKVError",
     "allocate_workspace",
+    "kv_block_copy",
     "kv_cache_append",
     "library",
     "library_path",

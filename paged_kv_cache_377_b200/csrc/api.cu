@@ -331,6 +331,24 @@ int kv_cache_append(const void *k, const void *v, void *k_cache, void *v_cache, 
     return ok();
 }
 
+int kv_block_copy(void *k_cache, void *v_cache, const int32_t *src, const int32_t *dst, int num_copies,
+                  int num_kv_heads, int head_dim, int block_size, int num_blocks, int32_t *d_status, void *stream) {
+    if (num_copies < 0) return fail(PKV_ERR_INVALID_ARGUMENT, "num_copies < 0");
+    if (!k_cache || !v_cache || (num_copies > 0 && (!src || !dst)))
+        return fail(PKV_ERR_INVALID_ARGUMENT, "a required pointer is NULL");
+    if (num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0)
+        return fail(PKV_ERR_INVALID_ARGUMENT, "num_kv_heads, head_dim, block_size and num_blocks must be positive");
+    if (head_dim % 8 != 0) return fail(PKV_ERR_UNSUPPORTED, "head_dim %d is not a multiple of 8", head_dim);
+    if (!aligned(k_cache, 16) || !aligned(v_cache, 16))
+        return fail(PKV_ERR_INVALID_ARGUMENT, "k_cache and v_cache must be 16-byte aligned");
+    if (d_status && !aligned(d_status, 4)) return fail(PKV_ERR_INVALID_ARGUMENT, "d_status misaligned");
+    if (num_copies == 0) return ok();
+    cudaError_t e = pkv::block_copy_launch(k_cache, v_cache, src, dst, num_copies, block_size, num_kv_heads,
+                                           head_dim, num_blocks, d_status, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "block copy launch");
+    return ok();
+}
+
 int pkv_validate(const int32_t *block_tables, const int32_t *context_lens, int num_seqs, int max_blocks_per_seq,
                  int block_size, int num_blocks, int32_t *d_status, void *stream) {
     if (num_seqs < 0) return fail(PKV_ERR_INVALID_ARGUMENT, "num_seqs < 0");

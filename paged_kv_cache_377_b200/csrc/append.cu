@@ -59,7 +59,43 @@ __global__ void __launch_bounds__(256)
     if (p < 0 || p >= num_blocks) atomicOr(status, PKV_STATUS_BAD_BLOCK_ID);
 }
 
+// Copy-on-write block copies: whole blocks (bs rows of Hkv * D bf16, K and V)
+// from src[c] to dst[c]; one grid-stride pass over 16-byte elements. A copy
+// with an id outside [0, num_blocks) is skipped and flagged.
+__global__ void block_copy_kernel(uint4 *__restrict__ k_cache, uint4 *__restrict__ v_cache,
+                                  const int32_t *__restrict__ src, const int32_t *__restrict__ dst, int num_copies,
+                                  int64_t per_block, int num_blocks, int32_t *status) {
+    const int64_t total = static_cast<int64_t>(num_copies) * 2 * per_block;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
+        const int64_t c = i / (2 * per_block), r = i % (2 * per_block);
+        const int kv = static_cast<int>(r / per_block);
+        const int64_t e = r % per_block;
+        const int32_t s = __ldg(src + c), d = __ldg(dst + c);
+        if (s < 0 || s >= num_blocks || d < 0 || d >= num_blocks) {
+            if (e == 0 && kv == 0 && status) atomicOr(status, PKV_STATUS_BAD_BLOCK_ID);
+            continue;
+        }
+        uint4 *pool = kv ? v_cache : k_cache;
+        pool[d * per_block + e] = pool[s * per_block + e];
+    }
+}
+
 }  // namespace
+
+cudaError_t block_copy_launch(void *k_cache, void *v_cache, const int32_t *src, const int32_t *dst,
+                              int num_copies, int block_size, int num_kv_heads, int head_dim, int num_blocks,
+                              int32_t *status, cudaStream_t stream) {
+    const int64_t per_block = static_cast<int64_t>(block_size) * num_kv_heads * head_dim / 8;  // 16-byte elements
+    const int64_t total = static_cast<int64_t>(num_copies) * 2 * per_block;
+    if (total == 0) return cudaSuccess;
+    int64_t grid = (total + 255) / 256;
+    if (grid > 148 * 16) grid = 148 * 16;
+    block_copy_kernel<<<static_cast<unsigned>(grid), 256, 0, stream>>>(
+        static_cast<uint4 *>(k_cache), static_cast<uint4 *>(v_cache), src, dst, num_copies, per_block, num_blocks,
+        status);
+    return cudaGetLastError();
+}
 
 cudaError_t append_launch(const void *k, const void *v, void *k_cache, void *v_cache, const int64_t *slot_mapping,
                           int num_tokens, int num_kv_heads, int head_dim, int block_size, int num_blocks,

@@ -33,6 +33,10 @@ cudaError_t append_launch(const void *k, const void *v, void *k_cache, void *v_c
                           int num_tokens, int num_kv_heads, int head_dim, int block_size, int num_blocks,
                           int32_t *status, cudaStream_t stream);
 
+cudaError_t block_copy_launch(void *k_cache, void *v_cache, const int32_t *src, const int32_t *dst,
+                              int num_copies, int block_size, int num_kv_heads, int head_dim, int num_blocks,
+                              int32_t *status, cudaStream_t stream);
+
 cudaError_t validate_launch(const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
                             int max_blocks_per_seq, int block_size, int num_blocks, int32_t *status,
                             cudaStream_t stream);
