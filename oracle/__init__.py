@@ -66,6 +66,21 @@ def _bind(path: str):
     lib.oracle_kv_append.argtypes = [
         P, P, P, P, P, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64,
     ]
+    lib.oracle_e4m3_to_double.restype = ctypes.c_double
+    lib.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
+    lib.oracle_e4m3_from_float.restype = ctypes.c_uint8
+    lib.oracle_e4m3_from_float.argtypes = [ctypes.c_float]
+    lib.oracle_paged_decode_fp8.restype = ctypes.c_int
+    lib.oracle_paged_decode_fp8.argtypes = [
+        P, P, P, P, P, P, P, P,
+        ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+        ctypes.c_int, ctypes.c_int64, ctypes.c_double,
+        P, ctypes.c_int64, ctypes.c_int,
+    ]
+    lib.oracle_kv_append_fp8.restype = ctypes.c_int
+    lib.oracle_kv_append_fp8.argtypes = [
+        P, P, P, P, P, P, P, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64,
+    ]
     return lib
 
 
@@ -102,6 +117,22 @@ def _bits(a) -> np.ndarray:
     import torch
     assert a.dtype == torch.bfloat16
     return a.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def _u8(a) -> np.ndarray:
+    """e4m3 codes (torch uint8 tensor or numpy uint8) -> contiguous uint8."""
+    if isinstance(a, np.ndarray):
+        assert a.dtype == np.uint8
+        return np.ascontiguousarray(a)
+    import torch
+    assert a.dtype == torch.uint8
+    return a.detach().cpu().contiguous().numpy()
+
+
+def _f32(a) -> np.ndarray:
+    if not isinstance(a, np.ndarray):
+        a = a.detach().cpu().numpy()
+    return np.ascontiguousarray(a, dtype=np.float32)
 
 
 def _i32(a) -> np.ndarray:
@@ -162,11 +193,81 @@ def kv_append(k_cache, v_cache, k, v, slot_mapping, block_size: int, lib=None):
 def decode_step(batch, pairs: Optional[Sequence[int]] = None, num_threads: int = 0, lib=None):
     """One whole decode step of a ``workloads.DecodeBatch``: append, then attend.
 
-    Returns (out fp64, k_cache' bits, v_cache' bits).
+    Returns (out fp64, k_cache' bits, v_cache' bits) -- codes for an e4m3 batch.
     """
+    if getattr(batch, "kv_dtype", "bf16") == "fp8":
+        return decode_step_fp8(batch, pairs=pairs, num_threads=num_threads, lib=lib)
     kc, vc = kv_append(batch.k_cache, batch.v_cache, batch.k_new, batch.v_new,
                        batch.slot_mapping.numpy(), batch.block_size, lib=lib)
     out = paged_decode(batch.q, kc, vc, batch.block_tables.numpy(), batch.context_lens.numpy(),
                        batch.num_kv_heads, batch.block_size, batch.scale, pairs=pairs,
                        num_threads=num_threads, lib=lib)
+    return out, kc, vc
+
+
+def e4m3_to_double(codes, lib=None) -> np.ndarray:
+    """Values of e4m3 codes (NaN for the two NaN codes), one C call per code."""
+    c = np.asarray(codes, dtype=np.uint8)
+    f = (lib or _load()).oracle_e4m3_to_double
+    return np.array([f(int(x)) for x in c.ravel()], dtype=np.float64).reshape(c.shape)
+
+
+def e4m3_from_float(x, lib=None) -> np.ndarray:
+    """Nearest e4m3 codes of fp32 values (ties to even, saturating at +-448)."""
+    a = np.asarray(x, dtype=np.float32)
+    f = (lib or _load()).oracle_e4m3_from_float
+    return np.array([f(float(v)) for v in a.ravel()], dtype=np.uint8).reshape(a.shape)
+
+
+def paged_decode_fp8(q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens, num_kv_heads: int,
+                     block_size: int, scale: float, pairs: Optional[Sequence[int]] = None,
+                     num_threads: int = 0, lib=None) -> np.ndarray:
+    """fp64 paged decode attention over an e4m3 cache (codes [NB][bs][Hkv][D], fp32 scales [Hkv])."""
+    qb, kb, vb = _bits(q), _u8(k_cache), _u8(v_cache)
+    ks, vs = _f32(k_scale), _f32(v_scale)
+    S, Hq, D = qb.shape
+    NB = kb.shape[0]
+    assert kb.shape == (NB, block_size, num_kv_heads, D) and vb.shape == kb.shape
+    assert ks.shape == (num_kv_heads,) and vs.shape == ks.shape
+    bt = _i32(block_tables)
+    cl = _i32(context_lens)
+    MB = bt.shape[1]
+    if pairs is None:
+        npairs, pp = S * Hq, None
+    else:
+        pp = np.ascontiguousarray(np.asarray(pairs), dtype=np.int64)
+        npairs = len(pp)
+    out = np.zeros((npairs, D), dtype=np.float64)
+    rc = (lib or _load()).oracle_paged_decode_fp8(
+        _ptr(out), _ptr(qb), _ptr(kb), _ptr(vb), _ptr(ks), _ptr(vs), _ptr(bt), _ptr(cl),
+        S, Hq, num_kv_heads, D, block_size, MB, NB, float(scale),
+        _ptr(pp) if pp is not None else None, npairs, int(num_threads))
+    if rc != 0:
+        raise OracleError(f"oracle_paged_decode_fp8 returned {rc}")
+    return out.reshape(S, Hq, D) if pairs is None else out
+
+
+def kv_append_fp8(k_cache, v_cache, k, v, k_scale, v_scale, slot_mapping, block_size: int, lib=None):
+    """Quantizing append on copies of e4m3 pools; returns (k_cache', v_cache') as uint8 codes."""
+    kc = _u8(k_cache).copy()
+    vc = _u8(v_cache).copy()
+    kb, vb = _bits(k), _bits(v)
+    ks, vs = _f32(k_scale), _f32(v_scale)
+    sm = np.ascontiguousarray(np.asarray(slot_mapping), dtype=np.int64)
+    NB, bs, Hkv, D = kc.shape
+    assert bs == block_size and kb.shape == (len(sm), Hkv, D) and vb.shape == kb.shape
+    rc = (lib or _load()).oracle_kv_append_fp8(_ptr(kc), _ptr(vc), _ptr(kb), _ptr(vb), _ptr(ks), _ptr(vs),
+                                               _ptr(sm), len(sm), Hkv, D, block_size, NB)
+    if rc != 0:
+        raise OracleError(f"oracle_kv_append_fp8 returned {rc}")
+    return kc, vc
+
+
+def decode_step_fp8(batch, pairs: Optional[Sequence[int]] = None, num_threads: int = 0, lib=None):
+    """decode_step over a batch whose pools are e4m3 codes (batch.k_scale / v_scale per kv head)."""
+    kc, vc = kv_append_fp8(batch.k_cache, batch.v_cache, batch.k_new, batch.v_new, batch.k_scale,
+                           batch.v_scale, batch.slot_mapping.numpy(), batch.block_size, lib=lib)
+    out = paged_decode_fp8(batch.q, kc, vc, batch.k_scale, batch.v_scale, batch.block_tables.numpy(),
+                           batch.context_lens.numpy(), batch.num_kv_heads, batch.block_size, batch.scale,
+                           pairs=pairs, num_threads=num_threads, lib=lib)
     return out, kc, vc

@@ -35,6 +35,16 @@
  * new token's key and value (runbyai.xyz post 449, sections 1 and 2).
  * Token i goes to slot slot_mapping[i] = physical_block * bs + offset; a
  * negative slot means "no write".
+ *
+ * FP8 cache (runbyai post 449, section 5, names quantization among the means
+ * for long contexts; the format is the task's reading): pools of e4m3 codes
+ * (1 sign, 4 exponent bits with bias 7, 3 mantissa bits; exponent 15 with
+ * mantissa 7 is NaN; exponent 0 is subnormal, m * 2^-9) and one fp32 scale
+ * per kv head for K and one for V. A stored code c of head h stands for
+ * e4m3(c) * scale[h]. The append quantizes x (bf16) as the e4m3 value nearest
+ * to the fp32 quotient x / scale[h] (ties to an even mantissa), saturating at
+ * +-448, the largest finite e4m3 value. The decode dequantizes exactly in
+ * fp64 and is otherwise the plain definition above.
  */
 #include <math.h>
 #include <stdint.h>
@@ -53,6 +63,54 @@ static double bf16_bits_to_double(uint16_t bits)
     return (double)f;
 }
 
+/* e4m3 code -> its value, from the format's definition. */
+double oracle_e4m3_to_double(uint8_t c)
+{
+    int e = (c >> 3) & 15, m = c & 7;
+    if (e == 15 && m == 7)
+        return NAN;
+    double v = e == 0 ? ldexp((double)m, -9) : ldexp((double)(8 + m), e - 10); /* (1 + m/8) 2^(e-7) */
+    return (c & 0x80) ? -v : v;
+}
+
+/* fp32 -> nearest e4m3 code, ties to an even mantissa, saturating at +-448. */
+uint8_t oracle_e4m3_from_float(float xf)
+{
+    if (isnan(xf))
+        return 0x7f;
+    uint8_t sign = signbit(xf) ? 0x80 : 0;
+    double a = fabs((double)xf);
+    if (a >= 448.0)
+        return sign | 0x7e;
+    if (a < ldexp(1.0, -6)) {                  /* subnormal range: multiples of 2^-9 */
+        double m = nearbyint(a * 512.0);       /* 8 is the smallest normal, code 0x08 */
+        return sign | (uint8_t)m;
+    }
+    int e;
+    frexp(a, &e);                              /* a = f 2^e, f in [0.5, 1) */
+    int E = e - 1;                             /* a = 2^E (1 + mantissa) */
+    double m = nearbyint((a / ldexp(1.0, E) - 1.0) * 8.0);
+    if (m == 8.0) {
+        m = 0.0;
+        E += 1;
+    }
+    return sign | (uint8_t)((E + 7) << 3) | (uint8_t)m;
+}
+
+/* A KV pool as the decode reads it: bf16 values, or e4m3 codes with a scale per kv head. */
+typedef struct {
+    const uint16_t *bf16;
+    const uint8_t *fp8;
+    const float *scale;
+} Pool;
+
+static double pool_value(const Pool *P, int64_t elem, int h)
+{
+    if (P->bf16)
+        return bf16_bits_to_double(P->bf16[elem]);
+    return oracle_e4m3_to_double(P->fp8[elem]) * (double)P->scale[h];
+}
+
 /* Element offset of (physical block p, offset off, kv head h, dim 0) in the pool. */
 static int64_t pool_row(int64_t p, int off, int h, int block_size, int num_kv_heads, int head_dim)
 {
@@ -65,7 +123,7 @@ static int64_t pool_row(int64_t p, int off, int h, int block_size, int num_kv_he
  * Returns 0, or -2 when a table entry it needs is outside [0, num_blocks).
  */
 static int decode_one(double *out, double *x,
-                      const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                      const uint16_t *q, const Pool *K, const Pool *V,
                       const int32_t *block_tables, int context_len,
                       int s, int j, int num_q_heads, int num_kv_heads, int head_dim,
                       int block_size, int max_blocks_per_seq, int64_t num_blocks, double scale)
@@ -85,10 +143,10 @@ static int decode_one(double *out, double *x,
         int64_t p = table[t / block_size];
         if (p < 0 || p >= num_blocks)
             return -2;
-        const uint16_t *krow = k_cache + pool_row(p, t % block_size, h, block_size, num_kv_heads, head_dim);
+        int64_t krow = pool_row(p, t % block_size, h, block_size, num_kv_heads, head_dim);
         double dot = 0.0;
         for (int d = 0; d < head_dim; ++d)
-            dot += bf16_bits_to_double(qrow[d]) * bf16_bits_to_double(krow[d]);
+            dot += bf16_bits_to_double(qrow[d]) * pool_value(K, krow + d, h);
         x[t] = scale * dot;
     }
 
@@ -101,9 +159,9 @@ static int decode_one(double *out, double *x,
     for (int t = 0; t < context_len; ++t) {
         double w = exp(x[t] - mu);
         int64_t p = table[t / block_size];
-        const uint16_t *vrow = v_cache + pool_row(p, t % block_size, h, block_size, num_kv_heads, head_dim);
+        int64_t vrow = pool_row(p, t % block_size, h, block_size, num_kv_heads, head_dim);
         for (int d = 0; d < head_dim; ++d)
-            out[d] += w * bf16_bits_to_double(vrow[d]);
+            out[d] += w * pool_value(V, vrow + d, h);
         z += w;
     }
     for (int d = 0; d < head_dim; ++d)
@@ -126,13 +184,13 @@ static int decode_one(double *out, double *x,
  * Returns 0; -1 for a bad argument; -2 for a table entry outside the pool;
  * -3 for a context length outside [0, max_blocks_per_seq * block_size].
  */
-int oracle_paged_decode(double *out, const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
-                        const int32_t *block_tables, const int32_t *context_lens,
-                        int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
-                        int max_blocks_per_seq, int64_t num_blocks, double scale,
-                        const int64_t *pairs, int64_t num_pairs, int num_threads)
+static int decode_pool(double *out, const uint16_t *q, const Pool *K, const Pool *V,
+                       const int32_t *block_tables, const int32_t *context_lens,
+                       int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                       int max_blocks_per_seq, int64_t num_blocks, double scale,
+                       const int64_t *pairs, int64_t num_pairs, int num_threads)
 {
-    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
+    if (!out || !q || !block_tables || !context_lens)
         return -1;
     if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 ||
         max_blocks_per_seq < 0 || num_blocks < 0 || num_q_heads % num_kv_heads != 0)
@@ -168,7 +226,7 @@ int oracle_paged_decode(double *out, const uint16_t *q, const uint16_t *k_cache,
             int s = (int)(flat / num_q_heads);
             int j = (int)(flat % num_q_heads);
             if (mine == 0)
-                mine = decode_one(out + k * head_dim, x, q, k_cache, v_cache, block_tables,
+                mine = decode_one(out + k * head_dim, x, q, K, V, block_tables,
                                   context_lens[s], s, j, num_q_heads, num_kv_heads, head_dim,
                                   block_size, max_blocks_per_seq, num_blocks, scale);
         }
@@ -180,6 +238,40 @@ int oracle_paged_decode(double *out, const uint16_t *q, const uint16_t *k_cache,
             status = mine;
     }
     return status;
+}
+
+int oracle_paged_decode(double *out, const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                        const int32_t *block_tables, const int32_t *context_lens,
+                        int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                        int max_blocks_per_seq, int64_t num_blocks, double scale,
+                        const int64_t *pairs, int64_t num_pairs, int num_threads)
+{
+    if (!k_cache || !v_cache)
+        return -1;
+    Pool K = {k_cache, NULL, NULL}, V = {v_cache, NULL, NULL};
+    return decode_pool(out, q, &K, &V, block_tables, context_lens, num_seqs, num_q_heads, num_kv_heads,
+                       head_dim, block_size, max_blocks_per_seq, num_blocks, scale, pairs, num_pairs,
+                       num_threads);
+}
+
+/*
+ * The same over an e4m3 cache: k_cache / v_cache hold codes
+ * [num_blocks][block_size][num_kv_heads][head_dim], k_scale / v_scale one fp32
+ * per kv head; element e of head h stands for e4m3(code) * scale[h].
+ */
+int oracle_paged_decode_fp8(double *out, const uint16_t *q, const uint8_t *k_cache, const uint8_t *v_cache,
+                            const float *k_scale, const float *v_scale,
+                            const int32_t *block_tables, const int32_t *context_lens,
+                            int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                            int max_blocks_per_seq, int64_t num_blocks, double scale,
+                            const int64_t *pairs, int64_t num_pairs, int num_threads)
+{
+    if (!k_cache || !v_cache || !k_scale || !v_scale)
+        return -1;
+    Pool K = {NULL, k_cache, k_scale}, V = {NULL, v_cache, v_scale};
+    return decode_pool(out, q, &K, &V, block_tables, context_lens, num_seqs, num_q_heads, num_kv_heads,
+                       head_dim, block_size, max_blocks_per_seq, num_blocks, scale, pairs, num_pairs,
+                       num_threads);
 }
 
 /*
@@ -214,6 +306,44 @@ int oracle_kv_append(uint16_t *k_cache, uint16_t *v_cache, const uint16_t *k, co
             for (int d = 0; d < head_dim; ++d) {
                 k_cache[dst + d] = k[src + d];
                 v_cache[dst + d] = v[src + d];
+            }
+        }
+    }
+    return 0;
+}
+
+/*
+ * The append into an e4m3 cache: element d of token i, kv head h becomes the
+ * code of (float) k[i][h][d] / k_scale[h] (and likewise for v), computed as one
+ * fp32 division and then oracle_e4m3_from_float.  Same slots and returns as
+ * oracle_kv_append.
+ */
+int oracle_kv_append_fp8(uint8_t *k_cache, uint8_t *v_cache, const uint16_t *k, const uint16_t *v,
+                         const float *k_scale, const float *v_scale, const int64_t *slot_mapping,
+                         int64_t num_tokens, int num_kv_heads, int head_dim, int block_size, int64_t num_blocks)
+{
+    if (!k_cache || !v_cache || !k || !v || !k_scale || !v_scale || (!slot_mapping && num_tokens > 0))
+        return -1;
+    if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks < 0)
+        return -1;
+    for (int64_t i = 0; i < num_tokens; ++i)
+        if (slot_mapping[i] >= num_blocks * block_size)
+            return -2;
+
+    for (int64_t i = 0; i < num_tokens; ++i) {
+        int64_t slot = slot_mapping[i];
+        if (slot < 0)
+            continue;
+        int64_t p = slot / block_size;
+        int off = (int)(slot % block_size);
+        for (int h = 0; h < num_kv_heads; ++h) {
+            int64_t dst = pool_row(p, off, h, block_size, num_kv_heads, head_dim);
+            int64_t src = (i * num_kv_heads + h) * (int64_t)head_dim;
+            for (int d = 0; d < head_dim; ++d) {
+                float kq = (float)bf16_bits_to_double(k[src + d]) / k_scale[h];
+                float vq = (float)bf16_bits_to_double(v[src + d]) / v_scale[h];
+                k_cache[dst + d] = oracle_e4m3_from_float(kq);
+                v_cache[dst + d] = oracle_e4m3_from_float(vq);
             }
         }
     }

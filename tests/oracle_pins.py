@@ -287,6 +287,118 @@ def pin_append_duplicate_slot_last_wins(lib=None):
     assert np.array_equal(kc[1, 1], bf16_bits(k[1])) and np.array_equal(vc[1, 1], bf16_bits(v[1]))
 
 
+# ---------------------------------------------------------------- fp8 (e4m3) cache
+
+_E4M3 = torch.float8_e4m3fn
+
+
+def pin_e4m3_decode_table(lib=None):
+    """Every code's value equals torch's float8_e4m3fn value (a library special case)."""
+    codes = np.arange(256, dtype=np.uint8)
+    mine = oracle.e4m3_to_double(codes, lib=lib)
+    ref = torch.from_numpy(codes).view(_E4M3).double().numpy()
+    assert np.array_equal(np.isnan(mine), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(mine[ok], ref[ok])
+
+
+def _e4m3_samples():
+    rng = np.random.default_rng(7)
+    x = rng.standard_normal(4000) * np.exp(rng.uniform(-14, 6.2, 4000))
+    finite = torch.arange(256, dtype=torch.uint8).view(_E4M3).double().numpy()
+    finite = np.unique(finite[np.isfinite(finite)])
+    mids = (finite[1:] + finite[:-1]) / 2       # exact ties between neighbouring codes
+    x = np.concatenate([x, mids, -mids, finite, [0.0, -0.0]]).astype(np.float32)
+    return x[np.abs(x) <= 448]
+
+
+def pin_e4m3_encode_matches_torch(lib=None):
+    """In range, the encode is torch's round-to-nearest-even cast, ties included."""
+    x = _e4m3_samples()
+    mine = oracle.e4m3_from_float(x, lib=lib)
+    ref = torch.from_numpy(x).to(_E4M3).view(torch.uint8).numpy()
+    assert np.array_equal(mine, ref)
+
+
+def pin_e4m3_encode_is_nearest(lib=None):
+    """Brute force over all finite codes: the chosen code is a nearest one, and of two
+    nearest ones the one with an even mantissa field."""
+    x = _e4m3_samples()[::7]
+    codes = np.array([c for c in range(256) if (c & 0x7f) != 0x7f], dtype=np.uint8)
+    vals = torch.from_numpy(codes).view(_E4M3).double().numpy()
+    mine = oracle.e4m3_from_float(x, lib=lib)
+    for xi, ci in zip(x.astype(np.float64), mine):
+        d = np.abs(vals - xi)
+        best = codes[d == d.min()]
+        best_vals = set(torch.from_numpy(best).view(_E4M3).double().numpy().tolist())
+        got = float(torch.tensor([ci], dtype=torch.uint8).view(_E4M3).double())
+        assert got in best_vals, (xi, ci)
+        if len(best_vals) > 1:
+            assert ci & 1 == 0, (xi, ci)
+
+
+def pin_e4m3_saturates(lib=None):
+    big = np.array([448.0, 449.0, 463.9, 464.0, 470.0, 479.0, 500.0, 1e6, np.inf], dtype=np.float32)
+    assert (oracle.e4m3_from_float(big, lib=lib) == 0x7E).all()
+    assert (oracle.e4m3_from_float(-big, lib=lib) == 0xFE).all()
+    assert (oracle.e4m3_from_float(np.array([np.nan], np.float32), lib=lib) & 0x7F == 0x7F).all()
+
+
+def _fp8_batch(i, **kw):
+    Hq, Hkv, D, bs, lens = SMALL_GEOMETRIES[i]
+    return workloads.make_custom(400 + i, lens, Hq, Hkv, D, bs, kv_dtype="fp8", **kw)
+
+
+def _dequantized(b, kc, vc):
+    k = torch.from_numpy(np.asarray(kc)).view(_E4M3).double() * b.k_scale.double()[None, None, :, None]
+    v = torch.from_numpy(np.asarray(vc)).view(_E4M3).double() * b.v_scale.double()[None, None, :, None]
+    return k, v
+
+
+def pin_fp8_decode_equals_dequantized_sdpa(lib=None):
+    """Attention over the dequantized cache, by torch SDPA in fp64 on gathered rows."""
+    for i in range(len(SMALL_GEOMETRIES)):
+        b = _fp8_batch(i, with_append=False)
+        got = oracle.paged_decode_fp8(b.q, b.k_cache, b.v_cache, b.k_scale, b.v_scale, b.block_tables.numpy(),
+                                      b.context_lens.numpy(), b.num_kv_heads, b.block_size, b.scale, lib=lib)
+        k, v = _dequantized(b, b.k_cache.numpy(), b.v_cache.numpy())
+        _close(got, sdpa_reference(b, k, v), what=f"fp8 geometry {i}")
+
+
+def pin_fp8_append_matches_torch_quantization(lib=None):
+    """The append's codes are torch's cast of the fp32 quotient x / scale[h]."""
+    for i in (1, 4, 5):  # 2, 8 and 1 kv heads (K and V scales differ past head 0)
+        b = _fp8_batch(i, poison=False)
+        kc, vc = oracle.kv_append_fp8(b.k_cache, b.v_cache, b.k_new, b.v_new, b.k_scale, b.v_scale,
+                                      b.slot_mapping.numpy(), b.block_size, lib=lib)
+        bs = b.block_size
+        for t, slot in enumerate(b.slot_mapping.tolist()):
+            if slot < 0:
+                continue
+            kq = (b.k_new[t].float() / b.k_scale[:, None]).to(_E4M3).view(torch.uint8).numpy()
+            vq = (b.v_new[t].float() / b.v_scale[:, None]).to(_E4M3).view(torch.uint8).numpy()
+            assert np.array_equal(kc[slot // bs, slot % bs], kq) and np.array_equal(vc[slot // bs, slot % bs], vq)
+
+
+def pin_fp8_scales_act_as_the_pages_define(lib=None):
+    """A K scale factor c is a softmax scale factor c; a V scale factor c scales the output."""
+    b = _fp8_batch(1, with_append=False)
+    args = (b.block_tables.numpy(), b.context_lens.numpy(), b.num_kv_heads, b.block_size)
+    base = oracle.paged_decode_fp8(b.q, b.k_cache, b.v_cache, b.k_scale, b.v_scale, *args, b.scale, lib=lib)
+    twice_k = oracle.paged_decode_fp8(b.q, b.k_cache, b.v_cache, b.k_scale * 2, b.v_scale, *args, b.scale, lib=lib)
+    twice_s = oracle.paged_decode_fp8(b.q, b.k_cache, b.v_cache, b.k_scale, b.v_scale, *args, 2 * b.scale, lib=lib)
+    _close(twice_k, twice_s, what="K scale vs softmax scale")
+    half_v = oracle.paged_decode_fp8(b.q, b.k_cache, b.v_cache, b.k_scale, b.v_scale / 2, *args, b.scale, lib=lib)
+    _close(half_v, base / 2, what="V scale")
+
+
+def pin_fp8_poisoned_slots_are_never_read(lib=None):
+    b = _fp8_batch(3, with_append=False)   # NaN codes in every slot no table reaches
+    got = oracle.paged_decode_fp8(b.q, b.k_cache, b.v_cache, b.k_scale, b.v_scale, b.block_tables.numpy(),
+                                  b.context_lens.numpy(), b.num_kv_heads, b.block_size, b.scale, lib=lib)
+    assert np.isfinite(got).all()
+
+
 ALL_PINS = [
     pin_sdpa_random,
     pin_golden,
@@ -305,4 +417,12 @@ ALL_PINS = [
     pin_append_then_attend_one_token,
     pin_append_builds_the_sequence,
     pin_append_duplicate_slot_last_wins,
+    pin_e4m3_decode_table,
+    pin_e4m3_encode_matches_torch,
+    pin_e4m3_encode_is_nearest,
+    pin_e4m3_saturates,
+    pin_fp8_decode_equals_dequantized_sdpa,
+    pin_fp8_append_matches_torch_quantization,
+    pin_fp8_scales_act_as_the_pages_define,
+    pin_fp8_poisoned_slots_are_never_read,
 ]

@@ -18,7 +18,7 @@ MUTANTS = [
     ("scale dropped", "x[t] = scale * dot;", "x[t] = dot;"),
     ("head grouping j mod Hkv", "const int h = j / group;", "const int h = j % num_kv_heads;"),
     ("q row of the kv head", "((int64_t)s * num_q_heads + j) * head_dim", "((int64_t)s * num_q_heads + h) * head_dim"),
-    ("values read from K", "v_cache + pool_row", "k_cache + pool_row"),
+    ("values read from K", "pool_value(V, vrow + d, h)", "pool_value(K, vrow + d, h)"),
     ("block table ignored", "table[t / block_size]", "(t / block_size)"),
     ("offset off by one", "pool_row(p, t % block_size", "pool_row(p, (t + 1) % block_size"),
     ("last token dropped from PV", "for (int t = 0; t < context_len; ++t) {\n        double w",
@@ -28,6 +28,13 @@ MUTANTS = [
      "int64_t src = (i * num_kv_heads) * (int64_t)head_dim;"),
     ("append crosses k and v", "k_cache[dst + d] = k[src + d];", "k_cache[dst + d] = v[src + d];"),
     ("append offset 0", "int off = (int)(slot % block_size);", "int off = 0;"),
+    ("e4m3 exponent bias", "ldexp((double)(8 + m), e - 10)", "ldexp((double)(8 + m), e - 9)"),
+    ("e4m3 subnormal step", "ldexp((double)m, -9)", "ldexp((double)m, -8)"),
+    ("e4m3 encode truncates", "double m = nearbyint((a / ldexp(1.0, E) - 1.0) * 8.0);",
+     "double m = floor((a / ldexp(1.0, E) - 1.0) * 8.0);"),
+    ("e4m3 no saturation", "if (a >= 448.0)", "if (a >= 480.0)"),
+    ("fp8 scale of head 0", "* (double)P->scale[h];", "* (double)P->scale[0];"),
+    ("fp8 append uses the K scale for V", "/ v_scale[h];", "/ k_scale[h];"),
 ]
 
 

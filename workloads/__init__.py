@@ -15,4 +15,7 @@ from .decode_batches import (  # noqa: F401
     kv_bytes,
     unique_kv_bytes,
     BF16_NAN_BITS,
+    E4M3_NAN_CODE,
+    fp8_scales,
+    kv_element_bytes,
 )

@@ -23,7 +23,14 @@ Recipe (the same for every consumer: oracle tests, CUDA tests, benchmark):
    sequence's last block and every unused block hold NaN when ``poison`` is on,
    so that a stray read or a missed append shows up as NaN.
 
-This module holds no attention arithmetic.
+FP8 cache (``kv_dtype="fp8"``): the pools hold e4m3 codes drawn directly,
+not quantized from anything -- sign uniform, exponent field uniform in
+[4, 11], mantissa field uniform in [0, 7] (values 2^-3 .. 30 in magnitude) --
+and one fp32 scale per kv head for K, 2^-4 (1 + h / Hkv), and for V,
+2^-4 (1 + h / (2 Hkv)). The step's new k / v stay bf16 (the append quantizes
+them). Poisoned slots hold the NaN code 0x7f.
+
+This module holds no attention arithmetic and no quantization.
 """
 from __future__ import annotations
 
@@ -135,6 +142,9 @@ class DecodeBatch:
     v_cache: torch.Tensor           # bf16 [NB][bs][Hkv][D]
     k_new: torch.Tensor             # bf16 [S][Hkv][D]
     v_new: torch.Tensor             # bf16 [S][Hkv][D]
+    kv_dtype: str = "bf16"          # "bf16", or "fp8": pools of e4m3 codes (uint8) with per-head scales
+    k_scale: Optional[torch.Tensor] = None   # fp32 [Hkv] (fp8 only)
+    v_scale: Optional[torch.Tensor] = None
 
     @property
     def device(self) -> torch.device:
@@ -165,6 +175,30 @@ def _randn_bf16(shape, gen: torch.Generator, device) -> torch.Tensor:
         hi = min(n, lo + _CHUNK)
         out[lo:hi] = torch.randn(hi - lo, generator=gen, device=device, dtype=torch.float32).to(torch.bfloat16)
     return out.view(*shape)
+
+
+def _random_e4m3(shape, gen: torch.Generator, device) -> torch.Tensor:
+    """e4m3 codes drawn field by field (see the module docstring)."""
+    n = int(np.prod(shape))
+    out = torch.empty(n, dtype=torch.uint8, device=device)
+    for lo in range(0, n, _CHUNK):
+        hi = min(n, lo + _CHUNK)
+        sign = torch.randint(0, 2, (hi - lo,), generator=gen, device=device, dtype=torch.int32)
+        expo = torch.randint(4, 12, (hi - lo,), generator=gen, device=device, dtype=torch.int32)
+        mant = torch.randint(0, 8, (hi - lo,), generator=gen, device=device, dtype=torch.int32)
+        out[lo:hi] = (sign * 128 + expo * 8 + mant).to(torch.uint8)
+    return out.view(*shape)
+
+
+E4M3_NAN_CODE = 0x7F
+
+
+def fp8_scales(num_kv_heads: int):
+    """The recipe's per-head scales (fp32 [Hkv]) for K and V."""
+    h = torch.arange(num_kv_heads, dtype=torch.float64)
+    k = (2.0 ** -4) * (1 + h / num_kv_heads)
+    v = (2.0 ** -4) * (1 + h / (2 * num_kv_heads))
+    return k.to(torch.float32), v.to(torch.float32)
 
 
 def _assign_tables(cfg: Config, lens: np.ndarray, rng: np.random.Generator):
@@ -226,13 +260,17 @@ def _valid_slot_mask(tables: np.ndarray, present: np.ndarray, bs: int, num_block
 
 def _poison(cache: torch.Tensor, mask: np.ndarray) -> None:
     nb, bs, hkv, d = cache.shape
-    flat = cache.view(nb * bs, hkv * d).view(torch.int16)
     bad = torch.from_numpy(~mask).to(cache.device)
+    if cache.dtype == torch.uint8:
+        cache.view(nb * bs, hkv * d)[bad] = E4M3_NAN_CODE
+        return
+    flat = cache.view(nb * bs, hkv * d).view(torch.int16)
     flat[bad] = np.int16(BF16_NAN_BITS)
 
 
 def _build(cfg: Config, lens: np.ndarray, rng: np.random.Generator, seed: int, device,
-           poison: bool, with_append: bool) -> DecodeBatch:
+           poison: bool, with_append: bool, kv_dtype: str = "bf16") -> DecodeBatch:
+    assert kv_dtype in ("bf16", "fp8")
     tables, num_blocks, mb = _assign_tables(cfg, lens, rng)
     bs = cfg.block_size
     if with_append:
@@ -245,8 +283,15 @@ def _build(cfg: Config, lens: np.ndarray, rng: np.random.Generator, seed: int, d
     Hq, Hkv, D = cfg.num_q_heads, cfg.num_kv_heads, cfg.head_dim
     S = len(lens)
     q = _randn_bf16((S, Hq, D), gen, device)
-    k_cache = _randn_bf16((num_blocks, bs, Hkv, D), gen, device)
-    v_cache = _randn_bf16((num_blocks, bs, Hkv, D), gen, device)
+    if kv_dtype == "fp8":
+        k_cache = _random_e4m3((num_blocks, bs, Hkv, D), gen, device)
+        v_cache = _random_e4m3((num_blocks, bs, Hkv, D), gen, device)
+        k_scale, v_scale = fp8_scales(Hkv)
+        k_scale, v_scale = k_scale.to(device), v_scale.to(device)
+    else:
+        k_cache = _randn_bf16((num_blocks, bs, Hkv, D), gen, device)
+        v_cache = _randn_bf16((num_blocks, bs, Hkv, D), gen, device)
+        k_scale = v_scale = None
     k_new = _randn_bf16((S, Hkv, D), gen, device)
     v_new = _randn_bf16((S, Hkv, D), gen, device)
     if poison:
@@ -262,11 +307,12 @@ def _build(cfg: Config, lens: np.ndarray, rng: np.random.Generator, seed: int, d
         block_tables=torch.from_numpy(tables),
         slot_mapping=torch.from_numpy(slots),
         q=q, k_cache=k_cache, v_cache=v_cache, k_new=k_new, v_new=v_new,
+        kv_dtype=kv_dtype, k_scale=k_scale, v_scale=v_scale,
     )
 
 
 def make_batch(name: str, seed: Optional[int] = None, device="cpu", poison: bool = True,
-               lens_override: Optional[List[int]] = None) -> DecodeBatch:
+               lens_override: Optional[List[int]] = None, kv_dtype: str = "bf16") -> DecodeBatch:
     """Build the decode batch ``name`` with its values on ``device``."""
     cfg = CONFIGS[name]
     seed = cfg.seed if seed is None else seed
@@ -275,13 +321,13 @@ def make_batch(name: str, seed: Optional[int] = None, device="cpu", poison: bool
     if lens_override is not None:
         lens = np.asarray(lens_override, dtype=np.int64)
         cfg = dataclasses.replace(cfg, max_context=max(cfg.max_context, int(lens.max(initial=1))))
-    return _build(cfg, lens, rng, seed, device, poison, with_append=True)
+    return _build(cfg, lens, rng, seed, device, poison, with_append=True, kv_dtype=kv_dtype)
 
 
 def make_custom(seed: int, lens: Sequence[int], num_q_heads: int, num_kv_heads: int, head_dim: int,
                 block_size: int, scale: Optional[float] = None, pool_factor: float = 1.5,
                 max_context: Optional[int] = None, device="cpu", poison: bool = True,
-                with_append: bool = True, shared_prefix_tokens: int = 0) -> DecodeBatch:
+                with_append: bool = True, shared_prefix_tokens: int = 0, kv_dtype: str = "bf16") -> DecodeBatch:
     """A batch of any geometry, built by the same recipe as the named configs.
 
     ``with_append=False`` gives a pool that already holds all L tokens of every
@@ -298,7 +344,7 @@ def make_custom(seed: int, lens: Sequence[int], num_q_heads: int, num_kv_heads: 
         pool_factor=pool_factor, prefix_tokens=shared_prefix_tokens,
     )
     rng = np.random.default_rng(seed)
-    return _build(cfg, lens, rng, seed, device, poison, with_append)
+    return _build(cfg, lens, rng, seed, device, poison, with_append, kv_dtype=kv_dtype)
 
 
 def permute_pool(batch: DecodeBatch, seed: int) -> DecodeBatch:
@@ -359,10 +405,14 @@ def unshare_prefix(batch: DecodeBatch) -> DecodeBatch:
     )
 
 
+def kv_element_bytes(batch: DecodeBatch) -> int:
+    return 1 if batch.kv_dtype == "fp8" else 2
+
+
 def kv_bytes(batch: DecodeBatch) -> int:
     """Algorithmic K+V bytes one decode step reads: every attended token once per kv head."""
     total_tokens = int(batch.context_lens.to(torch.int64).sum())
-    return total_tokens * 2 * batch.num_kv_heads * batch.head_dim * 2
+    return total_tokens * 2 * batch.num_kv_heads * batch.head_dim * kv_element_bytes(batch)
 
 
 def unique_kv_bytes(batch: DecodeBatch) -> int:
@@ -376,4 +426,4 @@ def unique_kv_bytes(batch: DecodeBatch) -> int:
         for b in range((L + bs - 1) // bs):
             p = int(tables[s, b])
             used[p] = max(used.get(p, 0), min(bs, L - b * bs))
-    return sum(used.values()) * 2 * batch.num_kv_heads * batch.head_dim * 2
+    return sum(used.values()) * 2 * batch.num_kv_heads * batch.head_dim * kv_element_bytes(batch)
