@@ -155,6 +155,47 @@ int paged_attn_decode_ex(void *out, const void *q, const void *k_cache, const vo
                          void *stream);
 
 /*
+ * FP8 KV cache. The pools hold e4m3 codes (1 sign, 4 exponent bits with bias
+ * 7, 3 mantissa bits; 0x7f / 0xff are NaN), laid out like the bf16 pools,
+ * [num_blocks][block_size][num_kv_heads][head_dim] bytes, with one fp32 scale
+ * per kv head for K (k_scale, device [num_kv_heads]) and one for V: element d
+ * of head h stands for e4m3(code) * scale[h]. This halves the bytes a decode
+ * reads (runbyai post 449, section 5, names quantization among the means for
+ * long contexts; the format and the per-head scales are this library's).
+ *
+ * kv_cache_append_fp8: like kv_cache_append, storing for each element x of
+ * token i, head h the e4m3 code nearest to the fp32 quotient x / scale[h]
+ * (ties to an even mantissa), saturated to +-448. head_dim must be a
+ * multiple of 16.
+ *
+ * paged_attn_decode_fp8 / paged_attn_decode_append_fp8: paged_attn_decode_ex /
+ * paged_attn_decode_append over e4m3 pools (same arguments plus the scales).
+ * The codes are widened exactly to f16 and multiplied on tensor cores
+ * (mma.sync f16, fp32 accumulation); q is rounded to f16 after scaling each
+ * query row by a power of two that puts its largest magnitude in [2^14,
+ * 2^15); probabilities are rounded to f16. Supported: head_dim 128, or 64
+ * with head packing (an even num_kv_heads and num_q_heads / num_kv_heads <=
+ * 4, so that every row read is 128 bytes); block_size 16 or 32; opts->math 0
+ * or 2 (1 returns PKV_ERR_UNSUPPORTED). Default: 2 ring stages per warp.
+ */
+int kv_cache_append_fp8(const void *k, const void *v, void *k_cache, void *v_cache, const int64_t *slot_mapping,
+                        const float *k_scale, const float *v_scale, int num_tokens, int num_kv_heads, int head_dim,
+                        int block_size, int num_blocks, int32_t *d_status, void *stream);
+
+int paged_attn_decode_fp8(void *out, const void *q, const void *k_cache, const void *v_cache, const float *k_scale,
+                          const float *v_scale, const int32_t *block_tables, const int32_t *context_lens,
+                          int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size, float scale,
+                          int max_blocks_per_seq, int num_blocks, void *workspace, size_t workspace_bytes,
+                          const pkv_decode_options *opts, void *stream);
+
+int paged_attn_decode_append_fp8(void *out, const void *q, const void *k_new, const void *v_new,
+                                 const int64_t *slot_mapping, void *k_cache, void *v_cache, const float *k_scale,
+                                 const float *v_scale, const int32_t *block_tables, const int32_t *context_lens,
+                                 int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                                 float scale, int max_blocks_per_seq, int num_blocks, void *workspace,
+                                 size_t workspace_bytes, const pkv_decode_options *opts, void *stream);
+
+/*
  * One whole decode step in one launch: kv_cache_append of the step's token of
  * every sequence, then paged_attn_decode over contexts that include it (the
  * decode step of "Deep Dive into vLLM", section 2: each generated token's key
@@ -270,7 +311,8 @@ int pkv_selftest_bounded_wait(int32_t *d_status, void *stream);
 /*
  * Copy-on-write block copies: for c < num_copies, physical block dst[c] of
  * both pools becomes a copy of block src[c] (block_size rows of num_kv_heads *
- * head_dim bf16). src, dst: device int32 [num_copies] (from
+ * head_dim elements of elem_bytes bytes: 2 for bf16 pools, 1 for e4m3 pools;
+ * a row must be a multiple of 16 bytes). src, dst: device int32 [num_copies] (from
  * pkv_bm_take_copies). The copies must not chain (no dst is another copy's
  * src); the block manager never produces such a list. An id outside
  * [0, num_blocks) skips that copy and ORs PKV_STATUS_BAD_BLOCK_ID into
@@ -278,7 +320,8 @@ int pkv_selftest_bounded_wait(int32_t *d_status, void *stream);
  * other write of the pools in the same step.
  */
 int kv_block_copy(void *k_cache, void *v_cache, const int32_t *src, const int32_t *dst, int num_copies,
-                  int num_kv_heads, int head_dim, int block_size, int num_blocks, int32_t *d_status, void *stream);
+                  int num_kv_heads, int head_dim, int elem_bytes, int block_size, int num_blocks, int32_t *d_status,
+                  void *stream);
 
 /*
  * Host-side block manager of one KV pool (no CUDA calls; thread-safe).

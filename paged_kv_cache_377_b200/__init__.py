@@ -16,10 +16,13 @@ from ._binding import (  # noqa: F401
     PagedKVError,
     allocate_workspace,
     kv_cache_append,
+    kv_cache_append_fp8,
     library,
     library_path,
     paged_attn_decode,
     paged_attn_decode_append,
+    paged_attn_decode_append_fp8,
+    paged_attn_decode_fp8,
     read_status,
     selftest_bounded_wait,
     validate,
@@ -38,6 +41,9 @@ __all__ = [
     "library_path",
     "paged_attn_decode",
     "paged_attn_decode_append",
+    "paged_attn_decode_append_fp8",
+    "paged_attn_decode_fp8",
+    "kv_cache_append_fp8",
     "read_status",
     "validate",
     "workspace_bytes",

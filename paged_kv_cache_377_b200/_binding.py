@@ -73,6 +73,14 @@ def library() -> ctypes.CDLL:
             lib.paged_attn_decode_append.restype = I
             lib.paged_attn_decode_append.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, F, I, I, P, Z,
                                                      ctypes.POINTER(_Options), P]
+            lib.paged_attn_decode_fp8.restype = I
+            lib.paged_attn_decode_fp8.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, F, I, I, P, Z,
+                                                  ctypes.POINTER(_Options), P]
+            lib.paged_attn_decode_append_fp8.restype = I
+            lib.paged_attn_decode_append_fp8.argtypes = [P, P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, F, I, I, P,
+                                                         Z, ctypes.POINTER(_Options), P]
+            lib.kv_cache_append_fp8.restype = I
+            lib.kv_cache_append_fp8.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, P, P]
             lib.kv_cache_append.restype = I
             lib.kv_cache_append.argtypes = [P, P, P, P, P, I, I, I, I, I, P, P]
             lib.pkv_validate.restype = I
@@ -282,3 +290,91 @@ def paged_attn_decode_noalloc(out: torch.Tensor, q: torch.Tensor, k_cache: torch
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
         S, Hq, Hkv, D, bs, float(scale), block_tables.shape[1], NB, _ptr(status), _stream(stream)))
     return out
+
+
+def _need_scales(k_scale, v_scale, hkv):
+    _need(k_scale, "k_scale", torch.float32, 1)
+    _need(v_scale, "v_scale", torch.float32, 1)
+    if k_scale.shape[0] != hkv or v_scale.shape[0] != hkv:
+        raise ValueError("k_scale and v_scale must have num_kv_heads entries")
+
+
+def paged_attn_decode_fp8(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                          k_scale: torch.Tensor, v_scale: torch.Tensor, block_tables: torch.Tensor,
+                          context_lens: torch.Tensor, scale: float, workspace: torch.Tensor, stream=None,
+                          **options) -> torch.Tensor:
+    """paged_attn_decode over e4m3 pools (uint8 [NB, bs, Hkv, D]) with fp32 per-head scales [Hkv]."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need(out, "out", torch.bfloat16, 3)
+    _need(k_cache, "k_cache", torch.uint8, 4)
+    _need(v_cache, "v_cache", torch.uint8, 4)
+    _need(block_tables, "block_tables", torch.int32, 2)
+    _need(context_lens, "context_lens", torch.int32, 1)
+    _need(workspace, "workspace", torch.uint8, 1)
+    S, Hq, D = q.shape
+    NB, bs, Hkv, D2 = k_cache.shape
+    if out.shape != q.shape or v_cache.shape != k_cache.shape or D2 != D:
+        raise ValueError("shape mismatch between q/out or k_cache/v_cache")
+    if block_tables.shape[0] != S or context_lens.shape[0] != S:
+        raise ValueError("block_tables and context_lens must have num_seqs rows")
+    _need_scales(k_scale, v_scale, Hkv)
+    opts = _Options(**{k: int(options.get(k, 0)) for k, _ in _Options._fields_})
+    _check("paged_attn_decode_fp8", library().paged_attn_decode_fp8(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), _ptr(block_tables),
+        _ptr(context_lens), S, Hq, Hkv, D, bs, float(scale), block_tables.shape[1], NB, _ptr(workspace),
+        workspace.numel(), ctypes.byref(opts), _stream(stream)))
+    return out
+
+
+def paged_attn_decode_append_fp8(out: torch.Tensor, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                                 slot_mapping: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                                 k_scale: torch.Tensor, v_scale: torch.Tensor, block_tables: torch.Tensor,
+                                 context_lens: torch.Tensor, scale: float, workspace: torch.Tensor, stream=None,
+                                 **options) -> torch.Tensor:
+    """The one-launch decode step over e4m3 pools (the new bf16 rows are quantized)."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need(out, "out", torch.bfloat16, 3)
+    _need(k_new, "k_new", torch.bfloat16, 3)
+    _need(v_new, "v_new", torch.bfloat16, 3)
+    _need(slot_mapping, "slot_mapping", torch.int64, 1)
+    _need(k_cache, "k_cache", torch.uint8, 4)
+    _need(v_cache, "v_cache", torch.uint8, 4)
+    _need(block_tables, "block_tables", torch.int32, 2)
+    _need(context_lens, "context_lens", torch.int32, 1)
+    _need(workspace, "workspace", torch.uint8, 1)
+    S, Hq, D = q.shape
+    NB, bs, Hkv, D2 = k_cache.shape
+    if out.shape != q.shape or v_cache.shape != k_cache.shape or D2 != D:
+        raise ValueError("shape mismatch between q/out or k_cache/v_cache")
+    if k_new.shape != (S, Hkv, D) or v_new.shape != k_new.shape or slot_mapping.shape[0] != S:
+        raise ValueError("k_new / v_new must be [num_seqs, num_kv_heads, head_dim] and slot_mapping [num_seqs]")
+    if block_tables.shape[0] != S or context_lens.shape[0] != S:
+        raise ValueError("block_tables and context_lens must have num_seqs rows")
+    _need_scales(k_scale, v_scale, Hkv)
+    opts = _Options(**{k: int(options.get(k, 0)) for k, _ in _Options._fields_})
+    _check("paged_attn_decode_append_fp8", library().paged_attn_decode_append_fp8(
+        _ptr(out), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(slot_mapping), _ptr(k_cache), _ptr(v_cache),
+        _ptr(k_scale), _ptr(v_scale), _ptr(block_tables), _ptr(context_lens), S, Hq, Hkv, D, bs, float(scale),
+        block_tables.shape[1], NB, _ptr(workspace), workspace.numel(), ctypes.byref(opts), _stream(stream)))
+    return out
+
+
+def kv_cache_append_fp8(k: torch.Tensor, v: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                        slot_mapping: torch.Tensor, k_scale: torch.Tensor, v_scale: torch.Tensor,
+                        status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Quantizing append into e4m3 pools: code = e4m3(x / scale[h]), rounded to nearest, saturated."""
+    _need(k, "k", torch.bfloat16, 3)
+    _need(v, "v", torch.bfloat16, 3)
+    _need(k_cache, "k_cache", torch.uint8, 4)
+    _need(v_cache, "v_cache", torch.uint8, 4)
+    _need(slot_mapping, "slot_mapping", torch.int64, 1)
+    if status is not None:
+        _need(status, "status", torch.int32, 1)
+    T, Hkv, D = k.shape
+    NB, bs, Hkv2, D2 = k_cache.shape
+    if v.shape != k.shape or v_cache.shape != k_cache.shape or (Hkv2, D2) != (Hkv, D) or slot_mapping.shape[0] != T:
+        raise ValueError("shape mismatch between k/v, caches and slot_mapping")
+    _need_scales(k_scale, v_scale, Hkv)
+    _check("kv_cache_append_fp8", library().kv_cache_append_fp8(
+        _ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache), _ptr(slot_mapping), _ptr(k_scale), _ptr(v_scale), T, Hkv,
+        D, bs, NB, _ptr(status), _stream(stream)))

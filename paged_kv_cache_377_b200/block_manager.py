@@ -53,7 +53,7 @@ def _lib():
             lib.pkv_bm_last_error.restype = ctypes.c_char_p
             lib.pkv_bm_last_error.argtypes = []
             lib.kv_block_copy.restype = I
-            lib.kv_block_copy.argtypes = [P, P, P, P, I, I, I, I, I, P, P]
+            lib.kv_block_copy.argtypes = [P, P, P, P, I, I, I, I, I, I, P, P]
             _ready = True
     return lib
 
@@ -150,9 +150,11 @@ class BlockManager:
 
 def kv_block_copy(k_cache: torch.Tensor, v_cache: torch.Tensor, src: torch.Tensor, dst: torch.Tensor,
                   status: Optional[torch.Tensor] = None, stream=None) -> None:
-    """Block dst[c] of both pools becomes a copy of block src[c] (device int32 tensors)."""
-    _need(k_cache, "k_cache", torch.bfloat16, 4)
-    _need(v_cache, "v_cache", torch.bfloat16, 4)
+    """Block dst[c] of both pools (bf16, or uint8 e4m3 codes) becomes a copy of block src[c]
+    (device int32 tensors)."""
+    dtype = k_cache.dtype if k_cache.dtype in (torch.bfloat16, torch.uint8) else torch.bfloat16
+    _need(k_cache, "k_cache", dtype, 4)
+    _need(v_cache, "v_cache", dtype, 4)
     _need(src, "src", torch.int32, 1)
     _need(dst, "dst", torch.int32, 1)
     if status is not None:
@@ -161,4 +163,5 @@ def kv_block_copy(k_cache: torch.Tensor, v_cache: torch.Tensor, src: torch.Tenso
         raise ValueError("k_cache / v_cache or src / dst shapes differ")
     NB, bs, Hkv, D = k_cache.shape
     _check("kv_block_copy", _lib().kv_block_copy(_ptr(k_cache), _ptr(v_cache), _ptr(src), _ptr(dst), src.numel(),
-                                                 Hkv, D, bs, NB, _ptr(status), _stream(stream)))
+                                                 Hkv, D, k_cache.element_size(), bs, NB, _ptr(status),
+                                                 _stream(stream)))

@@ -59,19 +59,22 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// Tensor map over a pool [num_blocks][bs][Hkv][D] bf16 seen as 4D
-// (64, D/64, Hkv, num_blocks*bs), innermost first; one box = one 64-column half
-// of all bs rows of one kv head of one block: (64, 1, 1, bs), 128-byte
-// swizzled in shared memory (a tile is D/64 such [bs][128 B] halves).
-int make_pool_map(CUtensorMap *map, const void *pool, int num_blocks, int bs, int hkv, int d) {
+// Tensor map over a pool [num_blocks][bs][Hkv][D] of `es`-byte elements (bf16:
+// 2, e4m3 codes: 1) seen as 4D (128/es, D*es/128, Hkv, num_blocks*bs),
+// innermost first; one box = one 128-byte column slice of all bs rows of one
+// kv head of one block: (128/es, 1, 1, bs), 128-byte swizzled in shared memory
+// (a tile is D*es/128 such [bs][128 B] slices).
+int make_pool_map(CUtensorMap *map, const void *pool, int num_blocks, int bs, int hkv, int d, int es = 2) {
     auto fn = encode_fn();
     if (!fn) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
-    cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(d / 64), static_cast<cuuint64_t>(hkv),
+    const cuuint64_t inner = 128 / es;
+    cuuint64_t dims[4] = {inner, static_cast<cuuint64_t>(d) * es / 128, static_cast<cuuint64_t>(hkv),
                           static_cast<cuuint64_t>(num_blocks) * bs};
-    cuuint64_t strides[3] = {64 * 2, static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(hkv) * d * 2};
-    cuuint32_t box[4] = {64, 1, 1, static_cast<cuuint32_t>(bs)};
+    cuuint64_t strides[3] = {128, static_cast<cuuint64_t>(d) * es, static_cast<cuuint64_t>(hkv) * d * es};
+    cuuint32_t box[4] = {static_cast<cuuint32_t>(inner), 1, 1, static_cast<cuuint32_t>(bs)};
     cuuint32_t estr[4] = {1, 1, 1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(pool), dims, strides, box, estr,
+    CUresult r = fn(map, es == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+                    const_cast<void *>(pool), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
@@ -126,6 +129,7 @@ constexpr int kDefaultPieceCost = 4;
 
 int default_stages(int head_dim, int block_size, int math) {
     if (math == pkv::kMathTensorCore) return 1;
+    if (math == pkv::kMathFp8) return 2;  // half the bytes per block: two blocks in flight per warp
     const int stage_bytes = 2 * block_size * head_dim * 2;
     int r = (64 * 1024) / (pkv::kConsumerWarps * stage_bytes);
     return r < 1 ? 1 : r > pkv::kMaxStagesPerWarp ? pkv::kMaxStagesPerWarp : r;
@@ -151,13 +155,19 @@ int pkv_decode_workspace_bytes(int num_seqs, int num_q_heads, int head_dim, size
 
 namespace {
 
-// Decode, optionally with the fused append (k_new, v_new, slots all non-NULL).
+// Decode, optionally with the fused append (k_new, v_new, slots all non-NULL),
+// over bf16 pools or, with k_scale / v_scale non-NULL, e4m3 pools.
 int decode_impl(void *out, const void *q, const void *k_new, const void *v_new, const int64_t *slots,
-                const void *k_cache, const void *v_cache, const int32_t *block_tables, const int32_t *context_lens,
+                const void *k_cache, const void *v_cache, const float *k_scale, const float *v_scale,
+                const int32_t *block_tables, const int32_t *context_lens,
                 int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size, float scale,
                 int max_blocks_per_seq, int num_blocks, void *workspace, size_t workspace_bytes,
                 const pkv_decode_options *opts, void *stream) {
     if (num_seqs < 0) return fail(PKV_ERR_INVALID_ARGUMENT, "num_seqs < 0");
+    const bool fp8 = k_scale != nullptr || v_scale != nullptr;
+    if (fp8 && (!k_scale || !v_scale)) return fail(PKV_ERR_INVALID_ARGUMENT, "k_scale and v_scale must not be NULL");
+    if (fp8 && (!aligned(k_scale, 4) || !aligned(v_scale, 4)))
+        return fail(PKV_ERR_INVALID_ARGUMENT, "k_scale and v_scale must be 4-byte aligned");
     const bool fused = slots != nullptr;
     if (fused && (!k_new || !v_new)) return fail(PKV_ERR_INVALID_ARGUMENT, "k_new and v_new must not be NULL");
     if (fused && (!aligned(k_new, 16) || !aligned(v_new, 16)))
@@ -196,16 +206,22 @@ int decode_impl(void *out, const void *q, const void *k_new, const void *v_new, 
         return fail(PKV_ERR_INVALID_ARGUMENT, "num_ctas %d exceeds %d", o.num_ctas, pkv::kMaxCtas);
     if (static_cast<int64_t>(num_kv_heads) * (max_blocks_per_seq + 64) * pkv::kMaxSeqsPerLaunch > 0x7fffffff)
         return fail(PKV_ERR_INVALID_ARGUMENT, "num_kv_heads * max_blocks_per_seq too large");
-    const int math = o.math ? o.math : pkv::kMathTensorCore;
+    if (fp8 && o.math == pkv::kMathCudaCore)
+        return fail(PKV_ERR_UNSUPPORTED, "e4m3 pools are decoded on tensor cores only (math 0 or 2)");
+    const int math = fp8 ? pkv::kMathFp8 : o.math ? o.math : pkv::kMathTensorCore;
     // Head packing: kv heads 2h, 2h + 1 of head_dim 64 read as one head of 128
-    // (256-byte rows instead of 128-byte ones); the kernel then sees half the
-    // kv heads, twice the head_dim and twice the group.
-    const bool can_pack = math == pkv::kMathTensorCore && head_dim == 64 && num_kv_heads % 2 == 0 &&
+    // (256-byte rows instead of 128-byte ones; for e4m3 pools, 128-byte rows
+    // instead of 64-byte ones); the kernel then sees half the kv heads, twice
+    // the head_dim and twice the group.
+    const bool can_pack = math != pkv::kMathCudaCore && head_dim == 64 && num_kv_heads % 2 == 0 &&
                           2 * group <= PKV_MAX_GROUP;
     if (o.head_pack == 2 && !can_pack)
         return fail(PKV_ERR_UNSUPPORTED, "head_pack 2 needs tensor-core math, head_dim 64, an even num_kv_heads "
                                          "and num_q_heads / num_kv_heads <= %d", PKV_MAX_GROUP / 2);
     const int pack = o.head_pack == 1 ? 1 : can_pack ? 2 : 1;
+    if (fp8 && head_dim * pack != 128)
+        return fail(PKV_ERR_UNSUPPORTED, "e4m3 pools need head_dim 128, or head_dim 64 with head packing (an even "
+                                         "num_kv_heads and num_q_heads / num_kv_heads <= %d)", PKV_MAX_GROUP / 2);
     const int kd = head_dim * pack, khkv = num_kv_heads / pack, kgroup = group * pack;  // as the kernel sees them
     const int ns = o.num_stages ? o.num_stages : default_stages(kd, block_size, math);
     if (ns < 1 || ns > pkv::kMaxStagesPerWarp)
@@ -222,8 +238,9 @@ int decode_impl(void *out, const void *q, const void *k_new, const void *v_new, 
     if (num_seqs == 0) return ok();
 
     CUtensorMap tm_k, tm_v;
-    if ((rc = make_pool_map(&tm_k, k_cache, num_blocks, block_size, khkv, kd)) != PKV_OK) return rc;
-    if ((rc = make_pool_map(&tm_v, v_cache, num_blocks, block_size, khkv, kd)) != PKV_OK) return rc;
+    const int es = fp8 ? 1 : 2;
+    if ((rc = make_pool_map(&tm_k, k_cache, num_blocks, block_size, khkv, kd, es)) != PKV_OK) return rc;
+    if ((rc = make_pool_map(&tm_v, v_cache, num_blocks, block_size, khkv, kd, es)) != PKV_OK) return rc;
 
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -271,6 +288,8 @@ int decode_impl(void *out, const void *q, const void *k_new, const void *v_new, 
             a.k_cache = const_cast<void *>(k_cache);
             a.v_cache = const_cast<void *>(v_cache);
         }
+        a.k_scale = k_scale;
+        a.v_scale = v_scale;
         e = pkv::decode_launch(kd, block_size, gp, math, tm_k, tm_v, a, grid, smem, st);
         if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
     }
@@ -286,9 +305,33 @@ int paged_attn_decode_ex(void *out, const void *q, const void *k_cache, const vo
                          int num_kv_heads, int head_dim, int block_size, float scale, int max_blocks_per_seq,
                          int num_blocks, void *workspace, size_t workspace_bytes, const pkv_decode_options *opts,
                          void *stream) {
-    return decode_impl(out, q, nullptr, nullptr, nullptr, k_cache, v_cache, block_tables, context_lens, num_seqs,
-                       num_q_heads, num_kv_heads, head_dim, block_size, scale, max_blocks_per_seq, num_blocks,
-                       workspace, workspace_bytes, opts, stream);
+    return decode_impl(out, q, nullptr, nullptr, nullptr, k_cache, v_cache, nullptr, nullptr, block_tables,
+                       context_lens, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, scale,
+                       max_blocks_per_seq, num_blocks, workspace, workspace_bytes, opts, stream);
+}
+
+int paged_attn_decode_fp8(void *out, const void *q, const void *k_cache, const void *v_cache, const float *k_scale,
+                          const float *v_scale, const int32_t *block_tables, const int32_t *context_lens,
+                          int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size, float scale,
+                          int max_blocks_per_seq, int num_blocks, void *workspace, size_t workspace_bytes,
+                          const pkv_decode_options *opts, void *stream) {
+    if (!k_scale || !v_scale) return fail(PKV_ERR_INVALID_ARGUMENT, "k_scale and v_scale must not be NULL");
+    return decode_impl(out, q, nullptr, nullptr, nullptr, k_cache, v_cache, k_scale, v_scale, block_tables,
+                       context_lens, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, scale,
+                       max_blocks_per_seq, num_blocks, workspace, workspace_bytes, opts, stream);
+}
+
+int paged_attn_decode_append_fp8(void *out, const void *q, const void *k_new, const void *v_new,
+                                 const int64_t *slot_mapping, void *k_cache, void *v_cache, const float *k_scale,
+                                 const float *v_scale, const int32_t *block_tables, const int32_t *context_lens,
+                                 int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                                 float scale, int max_blocks_per_seq, int num_blocks, void *workspace,
+                                 size_t workspace_bytes, const pkv_decode_options *opts, void *stream) {
+    if (!slot_mapping) return fail(PKV_ERR_INVALID_ARGUMENT, "slot_mapping must not be NULL");
+    if (!k_scale || !v_scale) return fail(PKV_ERR_INVALID_ARGUMENT, "k_scale and v_scale must not be NULL");
+    return decode_impl(out, q, k_new, v_new, slot_mapping, k_cache, v_cache, k_scale, v_scale, block_tables,
+                       context_lens, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, scale,
+                       max_blocks_per_seq, num_blocks, workspace, workspace_bytes, opts, stream);
 }
 
 int paged_attn_decode_append(void *out, const void *q, const void *k_new, const void *v_new,
@@ -298,9 +341,9 @@ int paged_attn_decode_append(void *out, const void *q, const void *k_new, const 
                              int num_blocks, void *workspace, size_t workspace_bytes,
                              const pkv_decode_options *opts, void *stream) {
     if (!slot_mapping) return fail(PKV_ERR_INVALID_ARGUMENT, "slot_mapping must not be NULL");
-    return decode_impl(out, q, k_new, v_new, slot_mapping, k_cache, v_cache, block_tables, context_lens, num_seqs,
-                       num_q_heads, num_kv_heads, head_dim, block_size, scale, max_blocks_per_seq, num_blocks,
-                       workspace, workspace_bytes, opts, stream);
+    return decode_impl(out, q, k_new, v_new, slot_mapping, k_cache, v_cache, nullptr, nullptr, block_tables,
+                       context_lens, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, scale,
+                       max_blocks_per_seq, num_blocks, workspace, workspace_bytes, opts, stream);
 }
 
 int paged_attn_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
@@ -331,20 +374,45 @@ int kv_cache_append(const void *k, const void *v, void *k_cache, void *v_cache, 
     return ok();
 }
 
+int kv_cache_append_fp8(const void *k, const void *v, void *k_cache, void *v_cache, const int64_t *slot_mapping,
+                        const float *k_scale, const float *v_scale, int num_tokens, int num_kv_heads, int head_dim,
+                        int block_size, int num_blocks, int32_t *d_status, void *stream) {
+    if (num_tokens < 0) return fail(PKV_ERR_INVALID_ARGUMENT, "num_tokens < 0");
+    if (!k || !v || !k_cache || !v_cache || !slot_mapping || !k_scale || !v_scale)
+        return fail(PKV_ERR_INVALID_ARGUMENT, "a required pointer is NULL");
+    if (num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0)
+        return fail(PKV_ERR_INVALID_ARGUMENT, "num_kv_heads, head_dim, block_size and num_blocks must be positive");
+    if (head_dim % 16 != 0) return fail(PKV_ERR_UNSUPPORTED, "head_dim %d is not a multiple of 16", head_dim);
+    if (!aligned(k, 16) || !aligned(v, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(k_scale, 4) || !aligned(v_scale, 4))
+        return fail(PKV_ERR_INVALID_ARGUMENT, "k, v, k_cache and v_cache must be 16-byte aligned, scales 4-byte");
+    if (d_status && !aligned(d_status, 4)) return fail(PKV_ERR_INVALID_ARGUMENT, "d_status misaligned");
+    if (num_tokens == 0) return ok();
+    cudaError_t e = pkv::append_fp8_launch(k, v, k_cache, v_cache, slot_mapping, k_scale, v_scale, num_tokens,
+                                           num_kv_heads, head_dim, block_size, num_blocks, d_status,
+                                           static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "append launch");
+    return ok();
+}
+
 int kv_block_copy(void *k_cache, void *v_cache, const int32_t *src, const int32_t *dst, int num_copies,
-                  int num_kv_heads, int head_dim, int block_size, int num_blocks, int32_t *d_status, void *stream) {
+                  int num_kv_heads, int head_dim, int elem_bytes, int block_size, int num_blocks, int32_t *d_status,
+                  void *stream) {
     if (num_copies < 0) return fail(PKV_ERR_INVALID_ARGUMENT, "num_copies < 0");
     if (!k_cache || !v_cache || (num_copies > 0 && (!src || !dst)))
         return fail(PKV_ERR_INVALID_ARGUMENT, "a required pointer is NULL");
     if (num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks <= 0)
         return fail(PKV_ERR_INVALID_ARGUMENT, "num_kv_heads, head_dim, block_size and num_blocks must be positive");
-    if (head_dim % 8 != 0) return fail(PKV_ERR_UNSUPPORTED, "head_dim %d is not a multiple of 8", head_dim);
+    if (elem_bytes != 1 && elem_bytes != 2) return fail(PKV_ERR_INVALID_ARGUMENT, "elem_bytes must be 1 or 2");
+    if ((head_dim * elem_bytes) % 16 != 0)
+        return fail(PKV_ERR_UNSUPPORTED, "a row of head_dim %d is not a multiple of 16 bytes", head_dim);
     if (!aligned(k_cache, 16) || !aligned(v_cache, 16))
         return fail(PKV_ERR_INVALID_ARGUMENT, "k_cache and v_cache must be 16-byte aligned");
     if (d_status && !aligned(d_status, 4)) return fail(PKV_ERR_INVALID_ARGUMENT, "d_status misaligned");
     if (num_copies == 0) return ok();
     cudaError_t e = pkv::block_copy_launch(k_cache, v_cache, src, dst, num_copies, block_size, num_kv_heads,
-                                           head_dim, num_blocks, d_status, static_cast<cudaStream_t>(stream));
+                                           head_dim * elem_bytes, num_blocks, d_status,
+                                           static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "block copy launch");
     return ok();
 }

@@ -40,6 +40,33 @@ __global__ void __launch_bounds__(256)
     v_cache[dst] = __ldg(v + src);
 }
 
+// The append into e4m3 pools: one thread per 16 codes of one (token, kv head)
+// row, K and V; each code is e4m3(rn, satfinite)(x / scale[h]) of its bf16
+// source x, the division in fp32.
+__global__ void __launch_bounds__(256)
+    kv_append_fp8_kernel(const uint4 *__restrict__ k, const uint4 *__restrict__ v, uint4 *__restrict__ k_cache,
+                         uint4 *__restrict__ v_cache, const int64_t *__restrict__ slot_mapping,
+                         const float *__restrict__ k_scale, const float *__restrict__ v_scale, int num_tokens,
+                         int num_kv_heads, int chunks_per_row, int block_size, int num_blocks, int32_t *status) {
+    const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int64_t rows = static_cast<int64_t>(num_tokens) * num_kv_heads;
+    if (idx >= rows * chunks_per_row) return;
+    const int64_t row = idx / chunks_per_row;  // token * num_kv_heads + head
+    const int c = static_cast<int>(idx - row * chunks_per_row);
+    const int64_t i = row / num_kv_heads;
+    const int h = static_cast<int>(row - i * num_kv_heads);
+    const int64_t slot = __ldg(slot_mapping + i);
+    if (slot < 0) return;
+    if (slot >= static_cast<int64_t>(num_blocks) * block_size) {
+        if (status && h == 0 && c == 0) atomicOr(status, PKV_STATUS_BAD_SLOT);
+        return;
+    }
+    const int64_t dst = (slot * num_kv_heads + h) * chunks_per_row + c;  // 16 codes per chunk
+    const int64_t src = (row * chunks_per_row + c) * 2;                  // 16 bf16 = two uint4
+    k_cache[dst] = quantize16_e4m3(__ldg(k + src), __ldg(k + src + 1), __ldg(k_scale + h));
+    v_cache[dst] = quantize16_e4m3(__ldg(v + src), __ldg(v + src + 1), __ldg(v_scale + h));
+}
+
 // One thread per (sequence, logical block) entry the sequence needs.
 __global__ void __launch_bounds__(256)
     validate_kernel(const int32_t *__restrict__ block_tables, const int32_t *__restrict__ context_lens, int num_seqs,
@@ -84,9 +111,9 @@ __global__ void block_copy_kernel(uint4 *__restrict__ k_cache, uint4 *__restrict
 }  // namespace
 
 cudaError_t block_copy_launch(void *k_cache, void *v_cache, const int32_t *src, const int32_t *dst,
-                              int num_copies, int block_size, int num_kv_heads, int head_dim, int num_blocks,
+                              int num_copies, int block_size, int num_kv_heads, int row_bytes, int num_blocks,
                               int32_t *status, cudaStream_t stream) {
-    const int64_t per_block = static_cast<int64_t>(block_size) * num_kv_heads * head_dim / 8;  // 16-byte elements
+    const int64_t per_block = static_cast<int64_t>(block_size) * num_kv_heads * row_bytes / 16;  // 16-byte elements
     const int64_t total = static_cast<int64_t>(num_copies) * 2 * per_block;
     if (total == 0) return cudaSuccess;
     int64_t grid = (total + 255) / 256;
@@ -94,6 +121,21 @@ cudaError_t block_copy_launch(void *k_cache, void *v_cache, const int32_t *src, 
     block_copy_kernel<<<static_cast<unsigned>(grid), 256, 0, stream>>>(
         static_cast<uint4 *>(k_cache), static_cast<uint4 *>(v_cache), src, dst, num_copies, per_block, num_blocks,
         status);
+    return cudaGetLastError();
+}
+
+cudaError_t append_fp8_launch(const void *k, const void *v, void *k_cache, void *v_cache, const int64_t *slot_mapping,
+                              const float *k_scale, const float *v_scale, int num_tokens, int num_kv_heads,
+                              int head_dim, int block_size, int num_blocks, int32_t *status, cudaStream_t stream) {
+    const int chunks = head_dim / 16;
+    const int64_t total = static_cast<int64_t>(num_tokens) * num_kv_heads * chunks;
+    if (total == 0) return cudaSuccess;
+    const int64_t grid = (total + 255) / 256;
+    if (grid > 0x7fffffff) return cudaErrorInvalidValue;
+    kv_append_fp8_kernel<<<static_cast<unsigned>(grid), 256, 0, stream>>>(
+        static_cast<const uint4 *>(k), static_cast<const uint4 *>(v), static_cast<uint4 *>(k_cache),
+        static_cast<uint4 *>(v_cache), slot_mapping, k_scale, v_scale, num_tokens, num_kv_heads, chunks, block_size,
+        num_blocks, status);
     return cudaGetLastError();
 }
 

@@ -44,6 +44,9 @@
 #include <set>
 #include <tuple>
 
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
 #include "device_utils.cuh"
 #include "launch.h"
 
@@ -185,7 +188,8 @@ struct CoreMath {
     }
 
     // query rows of the GQA group, pre-scaled into base-2 logits
-    __device__ __forceinline__ void load_q(uint32_t qslot, int group, float scale_log2, int /*pack: always 1 here*/) {
+    __device__ __forceinline__ void load_q(uint32_t qslot, int group, float scale_log2, int /*pack: always 1 here*/,
+                                           const DecodeArgs & /*a*/, int /*h*/) {
         const uint32_t qa = qslot + ch * 16;
         const float2 sc = make_float2(scale_log2, scale_log2);
 #pragma unroll
@@ -390,7 +394,8 @@ struct MmaMath {
     // B fragment (k = dim, n = head): two consecutive dims of q[l/4]; heads past the group are 0.
     // With pack = 2 the slot holds rows of D / 2 dims and query row g is
     // placed in half g / (group / 2) of the virtual head, zeros in the other.
-    __device__ __forceinline__ void load_q(uint32_t qslot, int group, float sl2, int pack) {
+    __device__ __forceinline__ void load_q(uint32_t qslot, int group, float sl2, int pack, const DecodeArgs & /*a*/,
+                                           int /*h*/) {
         scale_log2 = sl2;
         const int g = lane >> 2, k2 = (lane & 3) * 2;
         const int half = pack == 2 ? g / (group >> 1) : 0;
@@ -543,6 +548,254 @@ struct MmaMath {
     }
 };
 
+// ------------------------------------------------------------------ e4m3 tensor-core math
+
+// d += a (16x16 f16, row) * b (16x8 f16, col), fp32 accumulate.
+__device__ __forceinline__ void mma_16816_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Two e4m3 codes (low byte first) -> two f16 in one register, exactly
+// (every e4m3 value is an f16 value).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two_codes & 0xffffu), __NV_E4M3);
+    return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+}
+
+__device__ __forceinline__ uint32_t f16x2_bits(float lo, float hi) {
+    const __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+// Tensor-core math over e4m3 pools (tiles of BS rows x 128 one-byte codes,
+// 128-byte swizzled), f16 products with fp32 accumulation:
+//   S^T[t][g] = K[t][:] . q[g][:]   as in MmaMath, but ldmatrix gives a lane
+//     four consecutive codes of a row, so inside each 16-dim chunk the k index
+//     runs over dims in the order (4l, 4l+1 | 4l+2, 4l+3) and q's B fragments
+//     are built in the same order;
+//   O^T[d][g] += V[t][d] . P[g][t]  ldmatrix .trans gives a lane two 2-code
+//     columns of two token rows; one byte permute splits them into (dim 2r,
+//     tokens) and (dim 2r+1, tokens), so fragment rows r and r + 8 of a dim
+//     tile are dims 2r and 2r+1.
+// q is converted to f16 after scaling its row by a power of two that puts
+// the row's largest magnitude in [2^14, 2^15) (no overflow, bf16's 8
+// significant bits kept); the power of two, the head's K scale and the
+// softmax scale fold into one per-column logit multiplier. P is rounded to
+// f16. The head's V scale multiplies the accumulators at export.
+template <int BS>
+struct Fp8Math {
+    static constexpr int D = 128;  // bytes (codes) per tile row
+    static constexpr int GP = 8;
+    static constexpr int KC = D / 16;  // 16-dim chunks of q.K
+    static constexpr int TT = BS / 16;
+    static constexpr int DT = D / 16;  // dim tiles of P.V
+
+    int lane;
+    uint32_t pscr;        // this warp's f16 P[GP][BS] (shared address)
+    uint32_t qb[KC][2];   // f16 B fragments of q (row-scaled, chunk-permuted)
+    float mult0, mult1;   // base-2 logit multiplier of this lane's two columns
+    const float *vsc0, *vsc1;  // V scale of this lane's two columns (read at export)
+    float acc[DT][4];     // O^T fragments (rows: dims 2r, 2r+1 of each tile)
+    float m0, m1, l0, l1;
+
+    __device__ __forceinline__ void init(int warp, int lane_, uint8_t *base, const DecodeLayout &ly) {
+        lane = lane_;
+        pscr = smem_u32(base + ly.pscr) + warp * (GP * BS * 2);
+    }
+
+    // q rows are bf16 of D / pack dims; with pack = 2 row g lies in half g / (group / 2).
+    __device__ __forceinline__ void load_q(uint32_t qslot, int group, float sl2, int pack, const DecodeArgs &a,
+                                           int h) {
+        const int g = lane >> 2, t = lane & 3;
+        const int half = pack == 2 ? g / (group >> 1) : 0;
+        const int dr = D / pack;
+        float v[KC][4];
+        float mx = 0.f;
+#pragma unroll
+        for (int kc = 0; kc < KC; ++kc) {
+            const bool mine = g < group && (pack == 1 || kc / (KC / 2) == half);
+            const uint32_t lo = mine ? lds32(qslot + (g * dr + 16 * kc - half * dr + 4 * t) * 2) : 0u;
+            const uint32_t hi = mine ? lds32(qslot + (g * dr + 16 * kc - half * dr + 4 * t + 2) * 2) : 0u;
+            const float2 f0 = bf16x2_to_float2(lo), f1 = bf16x2_to_float2(hi);
+            v[kc][0] = f0.x;
+            v[kc][1] = f0.y;
+            v[kc][2] = f1.x;
+            v[kc][3] = f1.y;
+            mx = fmaxf(mx, fmaxf(fmaxf(fabsf(f0.x), fabsf(f0.y)), fmaxf(fabsf(f1.x), fabsf(f1.y))));
+        }
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        // power of two 2^(eb - 127) with the row max in [2^14, 2^15); its inverse is exact too
+        const int e = static_cast<int>((__float_as_uint(mx) >> 23) & 0xffu);  // biased exponent of the max
+        const int eb = mx > 0.f ? min(max(127 + 14 - (e - 127), 1), 253) : 127;
+        const float ps = __uint_as_float(static_cast<uint32_t>(eb) << 23);
+        const float inv_ps = __uint_as_float(static_cast<uint32_t>(254 - eb) << 23);
+#pragma unroll
+        for (int kc = 0; kc < KC; ++kc) {
+            qb[kc][0] = f16x2_bits(v[kc][0] * ps, v[kc][1] * ps);
+            qb[kc][1] = f16x2_bits(v[kc][2] * ps, v[kc][3] * ps);
+        }
+        const int n0 = 2 * t, n1 = n0 + 1;
+        const float ip0 = __shfl_sync(0xffffffffu, inv_ps, 4 * n0), ip1 = __shfl_sync(0xffffffffu, inv_ps, 4 * n1);
+        const int hg = pack == 2 ? (group >> 1) : group;  // query rows per real head
+        const int h0 = pack * h + (n0 < group ? n0 / hg : 0), h1 = pack * h + (n1 < group ? n1 / hg : 0);
+        mult0 = n0 < group ? sl2 * __ldg(a.k_scale + h0) * ip0 : 0.f;
+        mult1 = n1 < group ? sl2 * __ldg(a.k_scale + h1) * ip1 : 0.f;
+        vsc0 = a.v_scale + h0;
+        vsc1 = a.v_scale + h1;
+    }
+
+    __device__ __forceinline__ void reset() {
+        m0 = m1 = -INFINITY;
+        l0 = l1 = 0.f;
+#pragma unroll
+        for (int dt = 0; dt < DT; ++dt)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) acc[dt][k] = 0.f;
+    }
+
+    __device__ __forceinline__ void block(uint32_t ktile, uint32_t vtile, int valid) {
+        const int mi = lane >> 3, r = lane & 7;
+        const int tr = lane >> 2;
+        // S^T = K . Q^T; one ldmatrix x4 covers tokens 0-15 of two 16-dim chunks
+        float s[TT][4], s2[TT][4];
+#pragma unroll
+        for (int mt = 0; mt < TT; ++mt) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) s[mt][k] = s2[mt][k] = 0.f;
+#pragma unroll
+            for (int kp = 0; kp < KC / 2; ++kp) {
+                uint32_t x[4];
+                ldsm_x4(x, tile_addr<BS>(ktile, 16 * mt + r + 8 * (mi & 1), 2 * kp + (mi >> 1)));
+                const uint32_t a0[4] = {e4m3x2_to_f16x2(x[0]), e4m3x2_to_f16x2(x[1]), e4m3x2_to_f16x2(x[0] >> 16),
+                                        e4m3x2_to_f16x2(x[1] >> 16)};
+                mma_16816_f16(s[mt], a0, qb[2 * kp][0], qb[2 * kp][1]);
+                const uint32_t a1[4] = {e4m3x2_to_f16x2(x[2]), e4m3x2_to_f16x2(x[3]), e4m3x2_to_f16x2(x[2] >> 16),
+                                        e4m3x2_to_f16x2(x[3] >> 16)};
+                mma_16816_f16(s2[mt], a1, qb[2 * kp + 1][0], qb[2 * kp + 1][1]);
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) s[mt][k] += s2[mt][k];
+        }
+        // base-2 logits; tokens past the context are selected away (their rows may hold NaN codes)
+        float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+        for (int mt = 0; mt < TT; ++mt) {
+            const int t0 = 16 * mt + tr, t1 = t0 + 8;
+            s[mt][0] = t0 < valid ? s[mt][0] * mult0 : -INFINITY;
+            s[mt][1] = t0 < valid ? s[mt][1] * mult1 : -INFINITY;
+            s[mt][2] = t1 < valid ? s[mt][2] * mult0 : -INFINITY;
+            s[mt][3] = t1 < valid ? s[mt][3] * mult1 : -INFINITY;
+            mx0 = fmaxf(mx0, fmaxf(s[mt][0], s[mt][2]));
+            mx1 = fmaxf(mx1, fmaxf(s[mt][1], s[mt][3]));
+        }
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+        }
+        const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+        const float a0 = fast_exp2(m0 - n0), a1 = fast_exp2(m1 - n1);
+        // probabilities rounded to f16 for the P.V product; the sums take the rounded values
+        const int g0 = 2 * (lane & 3);
+        float ps0 = 0.f, ps1 = 0.f;
+#pragma unroll
+        for (int mt = 0; mt < TT; ++mt) {
+            const int t0 = 16 * mt + tr;
+            const __half p0 = __float2half_rn(fast_exp2(s[mt][0] - n0));
+            const __half p1 = __float2half_rn(fast_exp2(s[mt][1] - n1));
+            const __half p2 = __float2half_rn(fast_exp2(s[mt][2] - n0));
+            const __half p3 = __float2half_rn(fast_exp2(s[mt][3] - n1));
+            ps0 += __half2float(p0) + __half2float(p2);
+            ps1 += __half2float(p1) + __half2float(p3);
+            sts16(pscr + (g0 * BS + t0) * 2, __half_as_ushort(p0));
+            sts16(pscr + ((g0 + 1) * BS + t0) * 2, __half_as_ushort(p1));
+            sts16(pscr + (g0 * BS + t0 + 8) * 2, __half_as_ushort(p2));
+            sts16(pscr + ((g0 + 1) * BS + t0 + 8) * 2, __half_as_ushort(p3));
+        }
+        l0 = l0 * a0 + ps0;
+        l1 = l1 * a1 + ps1;
+        if (__any_sync(0xffffffffu, n0 != m0 || n1 != m1)) {
+#pragma unroll
+            for (int dt = 0; dt < DT; ++dt) {
+                acc[dt][0] *= a0;
+                acc[dt][1] *= a1;
+                acc[dt][2] *= a0;
+                acc[dt][3] *= a1;
+            }
+        }
+        m0 = n0;
+        m1 = n1;
+        __syncwarp();
+
+        // O^T += V^T . P^T; one ldmatrix x4 .trans covers tokens 0-15 of two dim tiles
+#pragma unroll
+        for (int ks = 0; ks < TT; ++ks) {
+            const uint32_t pb = pscr + ((lane >> 2) * BS + 16 * ks + 2 * (lane & 3)) * 2;
+            const uint32_t b0 = lds32(pb), b1 = lds32(pb + 16);
+            // V rows past the context may hold NaN codes: zero them in the fragments
+            uint32_t keep_lo = 0xffffffffu, keep_hi = 0xffffffffu;
+            if (valid < BS) {
+                const int t = 16 * ks + 2 * (lane & 3);
+                keep_lo = (t < valid ? 0x0000ffffu : 0u) | (t + 1 < valid ? 0xffff0000u : 0u);
+                keep_hi = (t + 8 < valid ? 0x0000ffffu : 0u) | (t + 9 < valid ? 0xffff0000u : 0u);
+            }
+#pragma unroll
+            for (int dp = 0; dp < DT / 2; ++dp) {
+                uint32_t x[4];
+                ldsm_x4_trans(x, tile_addr<BS>(vtile, 16 * ks + r + 8 * (mi & 1), 2 * dp + (mi >> 1)));
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    // x[2j]: tokens 0-7 of tile 2dp + j, x[2j + 1]: tokens 8-15; bytes
+                    // (t, 2r) (t, 2r+1) (t+1, 2r) (t+1, 2r+1) -> (t, 2r) (t+1, 2r) | (t, 2r+1) (t+1, 2r+1)
+                    const uint32_t lo = __byte_perm(x[2 * j], 0u, 0x3120), hi = __byte_perm(x[2 * j + 1], 0u, 0x3120);
+                    const uint32_t av[4] = {e4m3x2_to_f16x2(lo) & keep_lo, e4m3x2_to_f16x2(lo >> 16) & keep_lo,
+                                            e4m3x2_to_f16x2(hi) & keep_hi, e4m3x2_to_f16x2(hi >> 16) & keep_hi};
+                    mma_16816_f16(acc[2 * dp + j], av, b0, b1);
+                }
+            }
+        }
+        __syncwarp();  // P scratch is rewritten by the next block
+    }
+
+    __device__ __forceinline__ void export_state(float *merge_acc, float *merge_m, float *merge_l, int warp, int G) {
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+            l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+            l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+        }
+        const int g0 = 2 * (lane & 3), dr = lane >> 2;
+        if (lane < 4) {
+            if (g0 < G) {
+                merge_m[warp * G + g0] = m0;
+                merge_l[warp * G + g0] = l0;
+            }
+            if (g0 + 1 < G) {
+                merge_m[warp * G + g0 + 1] = m1;
+                merge_l[warp * G + g0 + 1] = l1;
+            }
+        }
+        float *r0 = merge_acc + (warp * G + g0) * D;
+        float *r1 = r0 + D;
+        const float vs0 = g0 < G ? __ldg(vsc0) : 0.f, vs1 = g0 + 1 < G ? __ldg(vsc1) : 0.f;
+#pragma unroll
+        for (int dt = 0; dt < DT; ++dt) {
+            if (g0 < G) {
+                r0[16 * dt + 2 * dr] = acc[dt][0] * vs0;
+                r0[16 * dt + 2 * dr + 1] = acc[dt][2] * vs0;
+            }
+            if (g0 + 1 < G) {
+                r1[16 * dt + 2 * dr] = acc[dt][1] * vs1;
+                r1[16 * dt + 2 * dr + 1] = acc[dt][3] * vs1;
+            }
+        }
+    }
+};
+
 // ------------------------------------------------------------------ pipeline
 
 struct Smem {
@@ -647,12 +900,14 @@ __device__ __forceinline__ void merge_pieces(const DecodeArgs &a, const int *pie
 // in flight than the ring can hold. Block-table entries of its next 32 blocks
 // are looked up one batch ahead. Warp 0 also bulk-copies the query rows of the piece after
 // next. All four warps meet at the end of every piece to merge their states.
-template <int D, int BS, class Math>
+template <int D, int BS, class Math, int ES>
 __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUtensorMap *tm_v, const DecodeArgs &a,
                                             const Smem &sm, const DecodeLayout &ly, PieceIter pieces, long long x0,
                                             long long x1, long long W, int C, int pcost, int warp, int lane) {
-    constexpr uint32_t kTile = BS * D * 2;
-    constexpr uint32_t kHalf = BS * 128;
+    static_assert(ES == 1 || ES == 2, "pool element bytes");
+    constexpr uint32_t kTile = BS * D * ES;   // bytes of one K (or V) tile
+    constexpr uint32_t kHalf = BS * 128;      // one TMA copy: BS rows of 128 bytes
+    constexpr int kCopies = D * ES / 128;     // copies per tile
     const int R = a.num_stages;
     const int G = a.group;
     const int DR = D / a.pack;  // dims per row of q, out and the partials
@@ -707,7 +962,7 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
             const int pp = jp < 32 ? pp_a : pp_b, hp = jp < 32 ? hp_a : hp_b;
             if (lane == 0 && kp < nk && pp >= 0 && pp < a.num_blocks && !*sm.abort_flag) {
 #pragma unroll
-                for (int half = 0; half < D / 64; ++half) {
+                for (int half = 0; half < kCopies; ++half) {
                     tma_prefetch_l2_4d(tm_k, 0, half, hp, pp * BS);
                     tma_prefetch_l2_4d(tm_v, 0, half, hp, pp * BS);
                 }
@@ -726,7 +981,7 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
                 uint8_t *dst = sm.base + ly.stages + static_cast<uint32_t>(stage) * 2u * kTile;
                 mbar_arrive_expect_tx(&sm.full[stage], 2u * kTile);
 #pragma unroll
-                for (int half = 0; half < D / 64; ++half) {
+                for (int half = 0; half < kCopies; ++half) {
                     tma_load_4d(dst + half * kHalf, tm_k, &sm.full[stage], 0, half, h, p * BS);
                     tma_load_4d(dst + kTile + half * kHalf, tm_v, &sm.full[stage], 0, half, h, p * BS);
                 }
@@ -766,7 +1021,7 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
         const int slot = npiece & 1;
         if (npiece >= 1 && ahead.next(pa)) issue_q(n_ahead++);  // every warp has read slot (npiece + 1) % 2
         mbar_wait_bounded(&sm.qfull[slot], static_cast<uint32_t>(npiece >> 1) & 1u, sm.abort_flag, a.status);
-        math.load_q(sbase + ly.qbuf + slot * qbytes, G, a.scale_log2, a.pack);
+        math.load_q(sbase + ly.qbuf + slot * qbytes, G, a.scale_log2, a.pack, a, pc.h);
         math.reset();
         ++npiece;
 
@@ -780,18 +1035,22 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
                 rphase ^= 1u;
             }
             // Fused append: the block holding position L - 1 takes the step's new
-            // row (fetched while the block's copy is in flight).
-            constexpr int kChunks = D / 8;  // 16-byte chunks of a row
-            const int bi = pc.b0 + i;      // block within the segment
+            // row (fetched while the block's copy is in flight; lanes < kChunks
+            // the K row, the next kChunks lanes the V row, 16 stored bytes each).
+            constexpr int kChunks = D * ES / 16;  // 16-byte chunks of a stored row
+            constexpr int kElems = 16 / ES;       // elements per chunk
+            const int bi = pc.b0 + i;             // block within the segment
             const bool tail = a.slots != nullptr && (bi + 1) * BS >= pc.L;
             long long slot = -1;
-            uint4 patch = make_uint4(0u, 0u, 0u, 0u);
+            auto patch_src = [&]() {  // this lane's chunk of the new row (bf16 source)
+                return reinterpret_cast<const uint4 *>(
+                    static_cast<const __nv_bfloat16 *>(lane < kChunks ? a.k_new : a.v_new) +
+                    (static_cast<size_t>(pc.s) * a.num_kv_heads + pc.h) * D + (lane % kChunks) * kElems);
+            };
+            uint4 patch = make_uint4(0u, 0u, 0u, 0u);  // bf16 pools: loaded while the copy is in flight
             if (tail) {
                 slot = __ldg(a.slots + pc.s);
-                if (slot >= 0 && lane < 2 * kChunks)
-                    patch = __ldg(reinterpret_cast<const uint4 *>(
-                        static_cast<const __nv_bfloat16 *>(lane < kChunks ? a.k_new : a.v_new) +
-                        (static_cast<size_t>(pc.s) * a.num_kv_heads + pc.h) * D + (lane % kChunks) * 8));
+                if (ES == 2 && slot >= 0 && lane < 2 * kChunks) patch = __ldg(patch_src());
             }
             if (mbar_wait_bounded(&sm.full[stage], par, sm.abort_flag, a.status)) inflight &= ~(1u << stage);
             if (!sm.stage_bad[stage] && !*sm.abort_flag) {
@@ -803,9 +1062,19 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
                     if (slot == want) {
                         if (lane < 2 * kChunks) {
                             const int c = lane % kChunks;
-                            sts128(tile_addr<BS>(lane < kChunks ? ktile : ktile + kTile, t, c), patch);
-                            *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(lane < kChunks ? a.k_cache : a.v_cache) +
-                                                       (static_cast<size_t>(want) * a.num_kv_heads + pc.h) * D + c * 8) = patch;
+                            uint4 row;
+                            if constexpr (ES == 2) {
+                                row = patch;
+                            } else {  // quantize: element d of real head r -> e4m3(x / scale[r])
+                                const int real = pc.h * a.pack + (c * kElems) / (D / a.pack);
+                                const float sc = __ldg((lane < kChunks ? a.k_scale : a.v_scale) + real);
+                                const uint4 *src = patch_src();
+                                row = quantize16_e4m3(__ldg(src), __ldg(src + 1), sc);
+                            }
+                            sts128(tile_addr<BS>(lane < kChunks ? ktile : ktile + kTile, t, c), row);
+                            *reinterpret_cast<uint4 *>(static_cast<uint8_t *>(lane < kChunks ? a.k_cache : a.v_cache) +
+                                                       ((static_cast<size_t>(want) * a.num_kv_heads + pc.h) * D) * ES +
+                                                       c * 16) = row;
                             fence_proxy_async_shared();  // before a later copy overwrites the stage
                         }
                         __syncwarp();
@@ -919,7 +1188,7 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
 // The tensor-core path fits 128 registers per thread, so 4 CTAs (16 warps)
 // share an SM; the CUDA-core path keeps its larger per-thread state.
 template <int D, int BS, int GP, int MATH>
-__global__ void __launch_bounds__(kDecodeThreads, MATH == kMathTensorCore ? 4 : 1)
+__global__ void __launch_bounds__(kDecodeThreads, MATH == kMathCudaCore ? 1 : 4)
     paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                         const DecodeArgs a) {
     static_assert(D == 64 || D == 128, "head_dim");
@@ -927,8 +1196,9 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathTensorCore ? 4 : 
     static_assert(GP == 1 || GP == 2 || GP == 4 || GP == 8, "group");
     static_assert(MATH == kMathCudaCore || GP == 8, "the tensor-core path pads the group to 8");
     extern __shared__ uint8_t smem_raw[];
-    const DecodeLayout ly = decode_layout(D, BS, GP, a.group, MATH == kMathTensorCore, kConsumerWarps * a.num_stages,
-                                          a.num_seqs);
+    constexpr int ES = MATH == kMathFp8 ? 1 : 2;  // bytes per pool element
+    const DecodeLayout ly = decode_layout(D, BS, GP, a.group, MATH != kMathCudaCore, kConsumerWarps * a.num_stages,
+                                          a.num_seqs, ES);
     Smem sm;
     sm.base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     sm.full = reinterpret_cast<uint64_t *>(sm.base + ly.bars);
@@ -1028,12 +1298,21 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathTensorCore ? 4 : 
                     if (tid == 0) atomicOr(a.status, PKV_STATUS_BAD_SLOT);
                 } else if (slot >= 0) {
                     const size_t row = static_cast<size_t>(a.num_kv_heads) * D;  // elements of one token's row
-                    for (int e = tid; e < 2 * static_cast<int>(row / 8); e += kDecodeThreads) {
-                        const int kv = e / static_cast<int>(row / 8), c = e % static_cast<int>(row / 8);
-                        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(
-                            static_cast<const __nv_bfloat16 *>(kv ? a.v_new : a.k_new) + s * row + c * 8));
-                        *reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(kv ? a.v_cache : a.k_cache) +
-                                                   static_cast<size_t>(slot) * row + c * 8) = v;
+                    constexpr int kElems = 16 / ES;                              // elements per stored 16 bytes
+                    const int chunks = static_cast<int>(row / kElems);
+                    for (int e = tid; e < 2 * chunks; e += kDecodeThreads) {
+                        const int kv = e / chunks, c = e % chunks;
+                        const uint4 *src = reinterpret_cast<const uint4 *>(
+                            static_cast<const __nv_bfloat16 *>(kv ? a.v_new : a.k_new) + s * row + c * kElems);
+                        uint4 v;
+                        if constexpr (ES == 2) {
+                            v = __ldg(src);
+                        } else {
+                            const int real = (c * kElems) / (D / a.pack);  // real kv head of the chunk
+                            v = quantize16_e4m3(__ldg(src), __ldg(src + 1), __ldg((kv ? a.v_scale : a.k_scale) + real));
+                        }
+                        *reinterpret_cast<uint4 *>(static_cast<uint8_t *>(kv ? a.v_cache : a.k_cache) +
+                                                   (static_cast<size_t>(slot) * row) * ES + c * 16) = v;
                     }
                 }
             }
@@ -1052,17 +1331,22 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathTensorCore ? 4 : 
     pieces.Hkv = a.num_kv_heads;
 
     if constexpr (MATH == kMathCudaCore) {
-        decode_warp<D, BS, CoreMath<D, BS, GP>>(&tm_k, &tm_v, a, sm, ly, pieces, x0, x1, W, gridDim.x, pcost, warp,
-                                                lane);
+        decode_warp<D, BS, CoreMath<D, BS, GP>, 2>(&tm_k, &tm_v, a, sm, ly, pieces, x0, x1, W, gridDim.x, pcost,
+                                                   warp, lane);
+    } else if constexpr (MATH == kMathTensorCore) {
+        decode_warp<D, BS, MmaMath<D, BS>, 2>(&tm_k, &tm_v, a, sm, ly, pieces, x0, x1, W, gridDim.x, pcost, warp,
+                                              lane);
     } else {
-        decode_warp<D, BS, MmaMath<D, BS>>(&tm_k, &tm_v, a, sm, ly, pieces, x0, x1, W, gridDim.x, pcost, warp, lane);
+        static_assert(D == 128, "the e4m3 path reads 128-byte rows (head_dim 64 packs head pairs)");
+        decode_warp<D, BS, Fp8Math<BS>, 1>(&tm_k, &tm_v, a, sm, ly, pieces, x0, x1, W, gridDim.x, pcost, warp,
+                                           lane);
     }
 }
 
 using KernelFn = void (*)(const CUtensorMap, const CUtensorMap, const DecodeArgs);
 
 // The tensor-core path always pads the group to 8 (one n8 tile).
-int effective_group_pad(int group_pad, int math) { return math == kMathTensorCore ? 8 : group_pad; }
+int effective_group_pad(int group_pad, int math) { return math == kMathCudaCore ? group_pad : 8; }
 
 KernelFn pick(int D, int BS, int GP, int math) {
 #define PKV_CASE(d, bs, gp, m) \
@@ -1071,6 +1355,7 @@ KernelFn pick(int D, int BS, int GP, int math) {
     PKV_CASE(d, bs, 1, kMathCudaCore) PKV_CASE(d, bs, 2, kMathCudaCore) PKV_CASE(d, bs, 4, kMathCudaCore) \
     PKV_CASE(d, bs, 8, kMathCudaCore) PKV_CASE(d, bs, 8, kMathTensorCore)
     PKV_GP(64, 16) PKV_GP(64, 32) PKV_GP(128, 16) PKV_GP(128, 32)
+    PKV_CASE(128, 16, 8, kMathFp8) PKV_CASE(128, 32, 8, kMathFp8)
 #undef PKV_GP
 #undef PKV_CASE
     return nullptr;
@@ -1084,8 +1369,8 @@ bool decode_variant_exists(int head_dim, int block_size, int group_pad, int math
 
 size_t decode_smem_bytes(int head_dim, int block_size, int group_pad, int group, int math, int num_stages,
                          int num_seqs) {
-    return decode_layout(head_dim, block_size, effective_group_pad(group_pad, math), group, math == kMathTensorCore,
-                         kConsumerWarps * num_stages, num_seqs)
+    return decode_layout(head_dim, block_size, effective_group_pad(group_pad, math), group, math != kMathCudaCore,
+                         kConsumerWarps * num_stages, num_seqs, math == kMathFp8 ? 1 : 2)
         .total;
 }
 

@@ -48,8 +48,12 @@ struct DecodeArgs {
     const void *k_new;
     const void *v_new;
     const int64_t *slots;
-    void *k_cache;               // bf16 pool [NB][BS][Hkv][D], written by the fused append
+    void *k_cache;               // pool [NB][BS][Hkv][D] (bf16, or e4m3 codes), written by the fused append
     void *v_cache;
+    // e4m3 pools: fp32 scale per REAL kv head (element = e4m3(code) * scale); the
+    // fused append stores e4m3(rn, satfinite)(x / scale) computed in fp32.
+    const float *k_scale;
+    const float *v_scale;
     float scale_log2;            // scale * log2(e): logits are kept in base 2
 };
 
@@ -64,17 +68,17 @@ __host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) { return (x
 // group, G = the actual group (query heads per kv head), tensor_core = the
 // mma.sync math path (its probability scratch is bf16 [8][BS] per warp).
 __host__ __device__ inline DecodeLayout decode_layout(int D, int BS, int GP, int G, bool tensor_core, int num_stages,
-                                                      int num_seqs) {
+                                                      int num_seqs, int kv_elem_bytes = 2) {
     DecodeLayout L;
     uint32_t off = 0;
-    const uint32_t tile = static_cast<uint32_t>(BS * D * 2);
+    const uint32_t tile = static_cast<uint32_t>(BS * D * kv_elem_bytes);
     L.stages = off;
     off += static_cast<uint32_t>(num_stages) * 2u * tile;          // [stage][K tile, V tile]
     L.qbuf = off;
     off += 2u * G * D * 2;                                          // two query slots [G][D] bf16
     off = align_up(off, 16);
     L.pscr = off;
-    off += kConsumerWarps * (tensor_core ? BS * 16 : BS * GP * 8);  // per warp probabilities
+    off += kConsumerWarps * (tensor_core ? BS * 16 : BS * GP * 8);  // per warp probabilities (16-bit [8][BS] on tensor cores)
     L.merge_acc = off;
     off += kConsumerWarps * G * D * 4;                              // per warp fp32 [G][D]
     L.merge_m = off;

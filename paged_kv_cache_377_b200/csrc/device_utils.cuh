@@ -4,6 +4,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <stdint.h>
 
 #include "pagedkv.h"
@@ -175,6 +176,24 @@ __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
         : "=f"(d.x), "=f"(d.y)
         : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
     return d;
+}
+
+// 16 bf16 values (two 16-byte loads) -> 16 e4m3 codes of x / scale: fp32
+// division rounded to nearest, then conversion to nearest e4m3 with
+// saturation at +-448.
+__device__ __forceinline__ uint4 quantize16_e4m3(uint4 a, uint4 b, float scale) {
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    uint32_t out[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 p = bf16x2_to_float2(w[2 * i]), q = bf16x2_to_float2(w[2 * i + 1]);
+        const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(p.x, scale), __fdiv_rn(p.y, scale)),
+                                                     __NV_SATFINITE, __NV_E4M3);
+        const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(__fdiv_rn(q.x, scale), __fdiv_rn(q.y, scale)),
+                                                     __NV_SATFINITE, __NV_E4M3);
+        out[i] = (lo & 0xffffu) | (hi << 16);
+    }
+    return make_uint4(out[0], out[1], out[2], out[3]);
 }
 
 // 2^x through the SFU (PTX ex2.approx.ftz.f32; 2^-inf = +0).

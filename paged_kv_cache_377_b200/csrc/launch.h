@@ -10,7 +10,9 @@
 
 namespace pkv {
 
-enum DecodeMath { kMathCudaCore = 1, kMathTensorCore = 2 };
+// kMathFp8: tensor-core (f16 mma.sync) math over e4m3 pools with per-head
+// scales; chosen by the fp8 entry points, not by the math option.
+enum DecodeMath { kMathCudaCore = 1, kMathTensorCore = 2, kMathFp8 = 3 };
 
 // True when the (head_dim, block_size, padded group, math) combination is compiled in.
 bool decode_variant_exists(int head_dim, int block_size, int group_pad, int math);
@@ -33,8 +35,12 @@ cudaError_t append_launch(const void *k, const void *v, void *k_cache, void *v_c
                           int num_tokens, int num_kv_heads, int head_dim, int block_size, int num_blocks,
                           int32_t *status, cudaStream_t stream);
 
+cudaError_t append_fp8_launch(const void *k, const void *v, void *k_cache, void *v_cache, const int64_t *slot_mapping,
+                              const float *k_scale, const float *v_scale, int num_tokens, int num_kv_heads,
+                              int head_dim, int block_size, int num_blocks, int32_t *status, cudaStream_t stream);
+
 cudaError_t block_copy_launch(void *k_cache, void *v_cache, const int32_t *src, const int32_t *dst,
-                              int num_copies, int block_size, int num_kv_heads, int head_dim, int num_blocks,
+                              int num_copies, int block_size, int num_kv_heads, int row_bytes, int num_blocks,
                               int32_t *status, cudaStream_t stream);
 
 cudaError_t validate_launch(const int32_t *block_tables, const int32_t *context_lens, int num_seqs,

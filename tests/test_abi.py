@@ -129,11 +129,13 @@ def test_fused_step_checks_its_extra_arguments():
 def test_block_copy_checks_arguments():
     lib = pkv.library()
     pkv.block_manager._lib()  # sets the argument types
-    assert lib.kv_block_copy(P, P, None, P, 2, 2, 64, 16, 8, None, None) == -1
+    assert lib.kv_block_copy(P, P, None, P, 2, 2, 64, 2, 16, 8, None, None) == -1
     assert "NULL" in lib.pkv_last_error().decode()
-    assert lib.kv_block_copy(P, P, P, P, 2, 2, 60, 16, 8, None, None) == -2
-    assert lib.kv_block_copy(P, P, P, P, -1, 2, 64, 16, 8, None, None) == -1
-    assert lib.kv_block_copy(P, P, None, None, 0, 2, 64, 16, 8, None, None) == 0  # nothing to copy
+    assert lib.kv_block_copy(P, P, P, P, 2, 2, 60, 2, 16, 8, None, None) == -2
+    assert lib.kv_block_copy(P, P, P, P, 2, 2, 24, 1, 16, 8, None, None) == -2   # 24-byte rows
+    assert lib.kv_block_copy(P, P, P, P, 2, 2, 64, 4, 16, 8, None, None) == -1   # elem_bytes
+    assert lib.kv_block_copy(P, P, P, P, -1, 2, 64, 2, 16, 8, None, None) == -1
+    assert lib.kv_block_copy(P, P, None, None, 0, 2, 64, 2, 16, 8, None, None) == 0  # nothing to copy
 
 
 def test_binding_refuses_cpu_tensors():
