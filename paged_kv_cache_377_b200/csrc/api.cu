@@ -129,7 +129,7 @@ constexpr int kDefaultPieceCost = 4;
 
 int default_stages(int head_dim, int block_size, int math) {
     if (math == pkv::kMathTensorCore) return 1;
-    if (math == pkv::kMathFp8) return 2;  // half the bytes per block: two blocks in flight per warp
+    if (math == pkv::kMathFp8) return head_dim == 256 ? 1 : 2;  // about 8 KB of blocks in flight per warp
     const int stage_bytes = 2 * block_size * head_dim * 2;
     int r = (64 * 1024) / (pkv::kConsumerWarps * stage_bytes);
     return r < 1 ? 1 : r > pkv::kMaxStagesPerWarp ? pkv::kMaxStagesPerWarp : r;
@@ -213,13 +213,14 @@ int decode_impl(void *out, const void *q, const void *k_new, const void *v_new, 
     // (256-byte rows instead of 128-byte ones; for e4m3 pools, 128-byte rows
     // instead of 64-byte ones); the kernel then sees half the kv heads, twice
     // the head_dim and twice the group.
-    const bool can_pack = math != pkv::kMathCudaCore && head_dim == 64 && num_kv_heads % 2 == 0 &&
-                          2 * group <= PKV_MAX_GROUP;
+    // For e4m3 pools head_dim 128 packs too: rows of 256 codes.
+    const bool can_pack = math != pkv::kMathCudaCore && (head_dim == 64 || (fp8 && head_dim == 128)) &&
+                          num_kv_heads % 2 == 0 && 2 * group <= PKV_MAX_GROUP;
     if (o.head_pack == 2 && !can_pack)
-        return fail(PKV_ERR_UNSUPPORTED, "head_pack 2 needs tensor-core math, head_dim 64, an even num_kv_heads "
-                                         "and num_q_heads / num_kv_heads <= %d", PKV_MAX_GROUP / 2);
+        return fail(PKV_ERR_UNSUPPORTED, "head_pack 2 needs tensor-core math, head_dim 64 (or 128 for e4m3 pools), an "
+                                         "even num_kv_heads and num_q_heads / num_kv_heads <= %d", PKV_MAX_GROUP / 2);
     const int pack = o.head_pack == 1 ? 1 : can_pack ? 2 : 1;
-    if (fp8 && head_dim * pack != 128)
+    if (fp8 && head_dim == 64 && pack != 2)
         return fail(PKV_ERR_UNSUPPORTED, "e4m3 pools need head_dim 128, or head_dim 64 with head packing (an even "
                                          "num_kv_heads and num_q_heads / num_kv_heads <= %d)", PKV_MAX_GROUP / 2);
     const int kd = head_dim * pack, khkv = num_kv_heads / pack, kgroup = group * pack;  // as the kernel sees them
@@ -251,7 +252,7 @@ int decode_impl(void *out, const void *q, const void *k_new, const void *v_new, 
     // in shared memory); launches run in stream order and reuse the workspace.
     for (int s0 = 0; s0 < num_seqs; s0 += pkv::kMaxSeqsPerLaunch) {
         const int sc = num_seqs - s0 < pkv::kMaxSeqsPerLaunch ? num_seqs - s0 : pkv::kMaxSeqsPerLaunch;
-        const size_t smem = pkv::decode_smem_bytes(kd, block_size, gp, kgroup, math, ns, sc);
+        const size_t smem = pkv::decode_smem_bytes(kd, block_size, gp, kgroup, math, ns, sc, pack);
         int per_sm = 0;
         cudaError_t e = pkv::decode_prepare(kd, block_size, gp, math, smem, &per_sm);
         if (e != cudaSuccess) return cuda_fail(e, "decode kernel setup");

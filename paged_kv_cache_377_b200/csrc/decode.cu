@@ -303,7 +303,8 @@ struct CoreMath {
     }
 
     // This warp's (m, l, acc) into the merge area ([warp][G][D], [warp][G]).
-    __device__ __forceinline__ void export_state(float *merge_acc, float *merge_m, float *merge_l, int warp, int G) {
+    __device__ __forceinline__ void export_state(float *merge_acc, float *merge_m, float *merge_l, int warp, int G,
+                                                 int /*pack: always 1 here*/) {
         // token groups of a warp share m_run: their accumulators just add
 #pragma unroll
         for (int o = LPT; o < 32; o <<= 1)
@@ -515,7 +516,8 @@ struct MmaMath {
         __syncwarp();  // P scratch is rewritten by the next block
     }
 
-    __device__ __forceinline__ void export_state(float *merge_acc, float *merge_m, float *merge_l, int warp, int G) {
+    __device__ __forceinline__ void export_state(float *merge_acc, float *merge_m, float *merge_l, int warp, int G,
+                                                 int pack) {
 #pragma unroll
         for (int o = 4; o < 32; o <<= 1) {
             l0 += __shfl_xor_sync(0xffffffffu, l0, o);
@@ -532,15 +534,19 @@ struct MmaMath {
                 merge_l[warp * G + g0 + 1] = l1;
             }
         }
-        float *r0 = merge_acc + (warp * G + g0) * D;
-        float *r1 = r0 + D;
+        // rows of D / pack floats: with pack = 2 a column keeps only its own half
+        const int DR = D / pack;
+        const int h0 = pack == 2 ? g0 / (G >> 1) : 0, h1 = pack == 2 ? (g0 + 1) / (G >> 1) : 0;
+        float *r0 = merge_acc + (warp * G + g0) * DR - h0 * DR;
+        float *r1 = merge_acc + (warp * G + g0 + 1) * DR - h1 * DR;
 #pragma unroll
         for (int dt = 0; dt < DT; ++dt) {
-            if (g0 < G) {
+            const int half = (16 * dt) / DR;  // all 16 dims of a tile lie in one half
+            if (g0 < G && half == h0) {
                 r0[16 * dt + dr] = acc[dt][0];
                 r0[16 * dt + dr + 8] = acc[dt][2];
             }
-            if (g0 + 1 < G) {
+            if (g0 + 1 < G && half == h1) {
                 r1[16 * dt + dr] = acc[dt][1];
                 r1[16 * dt + dr + 8] = acc[dt][3];
             }
@@ -571,32 +577,39 @@ __device__ __forceinline__ uint32_t f16x2_bits(float lo, float hi) {
     return *reinterpret_cast<const uint32_t *>(&h);
 }
 
-// Tensor-core math over e4m3 pools (tiles of BS rows x 128 one-byte codes,
-// 128-byte swizzled), f16 products with fp32 accumulation:
+// Tensor-core math over e4m3 pools, f16 products with fp32 accumulation. A
+// tile holds BS rows of 128 * HP one-byte codes (128-byte swizzled slices):
+// HP = 1 -- one virtual head of 128 dims (head_dim 128, or two heads of 64
+// packed as in MmaMath); HP = 2 -- two real heads of 128 side by side
+// (256-byte rows read from the pool), each query column using only its own
+// head's slice.
 //   S^T[t][g] = K[t][:] . q[g][:]   as in MmaMath, but ldmatrix gives a lane
 //     four consecutive codes of a row, so inside each 16-dim chunk the k index
 //     runs over dims in the order (4l, 4l+1 | 4l+2, 4l+3) and q's B fragments
-//     are built in the same order;
+//     are built in the same order; with HP = 2 a column's B fragment is zero
+//     on the other head's chunks;
 //   O^T[d][g] += V[t][d] . P[g][t]  ldmatrix .trans gives a lane two 2-code
 //     columns of two token rows; one byte permute splits them into (dim 2r,
 //     tokens) and (dim 2r+1, tokens), so fragment rows r and r + 8 of a dim
-//     tile are dims 2r and 2r+1.
+//     tile are dims 2r and 2r+1. With HP = 2 each dim tile is multiplied
+//     twice, by each head's slice with P zeroed outside that head's columns,
+//     so the accumulators hold every column's own 128 dims.
 // q is converted to f16 after scaling its row by a power of two that puts
 // the row's largest magnitude in [2^14, 2^15) (no overflow, bf16's 8
 // significant bits kept); the power of two, the head's K scale and the
 // softmax scale fold into one per-column logit multiplier. P is rounded to
 // f16. The head's V scale multiplies the accumulators at export.
-template <int BS>
+template <int BS, int HP>
 struct Fp8Math {
-    static constexpr int D = 128;  // bytes (codes) per tile row
+    static constexpr int D = 128 * HP;  // codes per tile row (the kernel's head_dim)
     static constexpr int GP = 8;
-    static constexpr int KC = D / 16;  // 16-dim chunks of q.K
     static constexpr int TT = BS / 16;
-    static constexpr int DT = D / 16;  // dim tiles of P.V
+    static constexpr int DT = 8;        // dim tiles of the accumulators (128 dims)
 
     int lane;
+    int my_half;          // HP = 2: the head (0/1) of this lane's B-fragment column lane / 4
     uint32_t pscr;        // this warp's f16 P[GP][BS] (shared address)
-    uint32_t qb[KC][2];   // f16 B fragments of q (row-scaled, chunk-permuted)
+    uint32_t qb[8][2];    // f16 B fragments of q (row-scaled, chunk-permuted), 8 chunks of 16 dims
     float mult0, mult1;   // base-2 logit multiplier of this lane's two columns
     const float *vsc0, *vsc1;  // V scale of this lane's two columns (read at export)
     float acc[DT][4];     // O^T fragments (rows: dims 2r, 2r+1 of each tile)
@@ -607,19 +620,30 @@ struct Fp8Math {
         pscr = smem_u32(base + ly.pscr) + warp * (GP * BS * 2);
     }
 
-    // q rows are bf16 of D / pack dims; with pack = 2 row g lies in half g / (group / 2).
+    // q rows are bf16 of D / pack dims. HP = 1, pack = 2: row g lies in half
+    // g / (group / 2) of the 128 dims. HP = 2 (pack = 2): row g is 128 dims of
+    // head g / (group / 2).
     __device__ __forceinline__ void load_q(uint32_t qslot, int group, float sl2, int pack, const DecodeArgs &a,
                                            int h) {
         const int g = lane >> 2, t = lane & 3;
         const int half = pack == 2 ? g / (group >> 1) : 0;
         const int dr = D / pack;
-        float v[KC][4];
+        my_half = HP == 2 ? half : 0;
+        float v[8][4];
         float mx = 0.f;
 #pragma unroll
-        for (int kc = 0; kc < KC; ++kc) {
-            const bool mine = g < group && (pack == 1 || kc / (KC / 2) == half);
-            const uint32_t lo = mine ? lds32(qslot + (g * dr + 16 * kc - half * dr + 4 * t) * 2) : 0u;
-            const uint32_t hi = mine ? lds32(qslot + (g * dr + 16 * kc - half * dr + 4 * t + 2) * 2) : 0u;
+        for (int kc = 0; kc < 8; ++kc) {
+            bool mine;
+            int col;
+            if constexpr (HP == 2) {
+                mine = g < group;
+                col = 16 * kc;
+            } else {
+                mine = g < group && (pack == 1 || kc / 4 == half);
+                col = 16 * kc - half * dr;
+            }
+            const uint32_t lo = mine ? lds32(qslot + (g * dr + col + 4 * t) * 2) : 0u;
+            const uint32_t hi = mine ? lds32(qslot + (g * dr + col + 4 * t + 2) * 2) : 0u;
             const float2 f0 = bf16x2_to_float2(lo), f1 = bf16x2_to_float2(hi);
             v[kc][0] = f0.x;
             v[kc][1] = f0.y;
@@ -635,7 +659,7 @@ struct Fp8Math {
         const float ps = __uint_as_float(static_cast<uint32_t>(eb) << 23);
         const float inv_ps = __uint_as_float(static_cast<uint32_t>(254 - eb) << 23);
 #pragma unroll
-        for (int kc = 0; kc < KC; ++kc) {
+        for (int kc = 0; kc < 8; ++kc) {
             qb[kc][0] = f16x2_bits(v[kc][0] * ps, v[kc][1] * ps);
             qb[kc][1] = f16x2_bits(v[kc][2] * ps, v[kc][3] * ps);
         }
@@ -668,15 +692,20 @@ struct Fp8Math {
 #pragma unroll
             for (int k = 0; k < 4; ++k) s[mt][k] = s2[mt][k] = 0.f;
 #pragma unroll
-            for (int kp = 0; kp < KC / 2; ++kp) {
+            for (int kp = 0; kp < 4 * HP; ++kp) {
+                // chunks 2kp, 2kp + 1 of the row; with HP = 2 they belong to head kp / 4
+                const bool on = HP == 1 || my_half == kp / 4;
+                const int qc = (2 * kp) % 8;
+                const uint32_t b00 = on ? qb[qc][0] : 0u, b01 = on ? qb[qc][1] : 0u;
+                const uint32_t b10 = on ? qb[qc + 1][0] : 0u, b11 = on ? qb[qc + 1][1] : 0u;
                 uint32_t x[4];
                 ldsm_x4(x, tile_addr<BS>(ktile, 16 * mt + r + 8 * (mi & 1), 2 * kp + (mi >> 1)));
                 const uint32_t a0[4] = {e4m3x2_to_f16x2(x[0]), e4m3x2_to_f16x2(x[1]), e4m3x2_to_f16x2(x[0] >> 16),
                                         e4m3x2_to_f16x2(x[1] >> 16)};
-                mma_16816_f16(s[mt], a0, qb[2 * kp][0], qb[2 * kp][1]);
+                mma_16816_f16(s[mt], a0, b00, b01);
                 const uint32_t a1[4] = {e4m3x2_to_f16x2(x[2]), e4m3x2_to_f16x2(x[3]), e4m3x2_to_f16x2(x[2] >> 16),
                                         e4m3x2_to_f16x2(x[3] >> 16)};
-                mma_16816_f16(s2[mt], a1, qb[2 * kp + 1][0], qb[2 * kp + 1][1]);
+                mma_16816_f16(s2[mt], a1, b10, b11);
             }
 #pragma unroll
             for (int k = 0; k < 4; ++k) s[mt][k] += s2[mt][k];
@@ -745,24 +774,33 @@ struct Fp8Math {
                 keep_hi = (t + 8 < valid ? 0x0000ffffu : 0u) | (t + 9 < valid ? 0xffff0000u : 0u);
             }
 #pragma unroll
-            for (int dp = 0; dp < DT / 2; ++dp) {
-                uint32_t x[4];
-                ldsm_x4_trans(x, tile_addr<BS>(vtile, 16 * ks + r + 8 * (mi & 1), 2 * dp + (mi >> 1)));
+            for (int hs = 0; hs < HP; ++hs) {
+                // head slice hs; with HP = 2 only the columns of head hs take it
+                const bool on = HP == 1 || my_half == hs;
+                const uint32_t c0 = on ? b0 : 0u, c1 = on ? b1 : 0u;
 #pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    // x[2j]: tokens 0-7 of tile 2dp + j, x[2j + 1]: tokens 8-15; bytes
-                    // (t, 2r) (t, 2r+1) (t+1, 2r) (t+1, 2r+1) -> (t, 2r) (t+1, 2r) | (t, 2r+1) (t+1, 2r+1)
-                    const uint32_t lo = __byte_perm(x[2 * j], 0u, 0x3120), hi = __byte_perm(x[2 * j + 1], 0u, 0x3120);
-                    const uint32_t av[4] = {e4m3x2_to_f16x2(lo) & keep_lo, e4m3x2_to_f16x2(lo >> 16) & keep_lo,
-                                            e4m3x2_to_f16x2(hi) & keep_hi, e4m3x2_to_f16x2(hi >> 16) & keep_hi};
-                    mma_16816_f16(acc[2 * dp + j], av, b0, b1);
+                for (int dp = 0; dp < DT / 2; ++dp) {
+                    uint32_t x[4];
+                    ldsm_x4_trans(x, tile_addr<BS>(vtile, 16 * ks + r + 8 * (mi & 1), 8 * hs + 2 * dp + (mi >> 1)));
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        // x[2j]: tokens 0-7 of tile 2dp + j, x[2j + 1]: tokens 8-15; bytes
+                        // (t, 2r) (t, 2r+1) (t+1, 2r) (t+1, 2r+1) -> (t, 2r) (t+1, 2r) | (t, 2r+1) (t+1, 2r+1)
+                        const uint32_t lo = __byte_perm(x[2 * j], 0u, 0x3120), hi = __byte_perm(x[2 * j + 1], 0u, 0x3120);
+                        const uint32_t av[4] = {e4m3x2_to_f16x2(lo) & keep_lo, e4m3x2_to_f16x2(lo >> 16) & keep_lo,
+                                                e4m3x2_to_f16x2(hi) & keep_hi, e4m3x2_to_f16x2(hi >> 16) & keep_hi};
+                        mma_16816_f16(acc[2 * dp + j], av, c0, c1);
+                    }
                 }
             }
         }
         __syncwarp();  // P scratch is rewritten by the next block
     }
 
-    __device__ __forceinline__ void export_state(float *merge_acc, float *merge_m, float *merge_l, int warp, int G) {
+    // Rows of D / pack floats: HP = 2 -- the column's own 128 dims; HP = 1 with
+    // pack = 2 -- the column's own half of the 128.
+    __device__ __forceinline__ void export_state(float *merge_acc, float *merge_m, float *merge_l, int warp, int G,
+                                                 int pack) {
 #pragma unroll
         for (int o = 4; o < 32; o <<= 1) {
             l0 += __shfl_xor_sync(0xffffffffu, l0, o);
@@ -779,16 +817,19 @@ struct Fp8Math {
                 merge_l[warp * G + g0 + 1] = l1;
             }
         }
-        float *r0 = merge_acc + (warp * G + g0) * D;
-        float *r1 = r0 + D;
+        const int DR = D / pack;
+        const int h0 = HP == 1 && pack == 2 ? g0 / (G >> 1) : 0, h1 = HP == 1 && pack == 2 ? (g0 + 1) / (G >> 1) : 0;
+        float *r0 = merge_acc + (warp * G + g0) * DR - h0 * DR;
+        float *r1 = merge_acc + (warp * G + g0 + 1) * DR - h1 * DR;
         const float vs0 = g0 < G ? __ldg(vsc0) : 0.f, vs1 = g0 + 1 < G ? __ldg(vsc1) : 0.f;
 #pragma unroll
         for (int dt = 0; dt < DT; ++dt) {
-            if (g0 < G) {
+            const int half = HP == 1 ? (16 * dt) / DR : 0;
+            if (g0 < G && half == h0) {
                 r0[16 * dt + 2 * dr] = acc[dt][0] * vs0;
                 r0[16 * dt + 2 * dr + 1] = acc[dt][2] * vs0;
             }
-            if (g0 + 1 < G) {
+            if (g0 + 1 < G && half == h1) {
                 r1[16 * dt + 2 * dr] = acc[dt][1] * vs1;
                 r1[16 * dt + 2 * dr + 1] = acc[dt][3] * vs1;
             }
@@ -1089,7 +1130,7 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
         }
         gb_base += nblk;
 
-        math.export_state(merge_acc, merge_m, merge_l, warp, G);
+        math.export_state(merge_acc, merge_m, merge_l, warp, G, a.pack);
         named_barrier_sync(1, kConsumerWarps * 32);
 
         // merge the warps' states (log-sum-exp identity) and store
@@ -1106,7 +1147,7 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
 #pragma unroll
                 for (int w = 0; w < kConsumerWarps; ++w) {
                     const float f = fast_exp2(merge_m[w * G + g] - M);
-                    const float2 av = *reinterpret_cast<const float2 *>(merge_acc + (w * G + g) * D + d);
+                    const float2 av = *reinterpret_cast<const float2 *>(merge_acc + (w * G + g) * DR + col);
                     ls += merge_l[w * G + g] * f;
                     a0 += av.x * f;
                     a1 += av.y * f;
@@ -1188,17 +1229,19 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
 // The tensor-core path fits 128 registers per thread, so 4 CTAs (16 warps)
 // share an SM; the CUDA-core path keeps its larger per-thread state.
 template <int D, int BS, int GP, int MATH>
-__global__ void __launch_bounds__(kDecodeThreads, MATH == kMathCudaCore ? 1 : 4)
+// Two-head e4m3 tiles (D = 256) take ~58 KB of shared memory: 3 CTAs per SM,
+// which leaves them ~170 registers per thread.
+__global__ void __launch_bounds__(kDecodeThreads, MATH == kMathCudaCore ? 1 : (MATH == kMathFp8 && D == 256) ? 3 : 4)
     paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                         const DecodeArgs a) {
-    static_assert(D == 64 || D == 128, "head_dim");
+    static_assert(D == 64 || D == 128 || (D == 256 && MATH == kMathFp8), "head_dim");
     static_assert(BS == 16 || BS == 32, "block_size");
     static_assert(GP == 1 || GP == 2 || GP == 4 || GP == 8, "group");
     static_assert(MATH == kMathCudaCore || GP == 8, "the tensor-core path pads the group to 8");
     extern __shared__ uint8_t smem_raw[];
     constexpr int ES = MATH == kMathFp8 ? 1 : 2;  // bytes per pool element
     const DecodeLayout ly = decode_layout(D, BS, GP, a.group, MATH != kMathCudaCore, kConsumerWarps * a.num_stages,
-                                          a.num_seqs, ES);
+                                          a.num_seqs, ES, D / a.pack);
     Smem sm;
     sm.base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     sm.full = reinterpret_cast<uint64_t *>(sm.base + ly.bars);
@@ -1337,9 +1380,9 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathCudaCore ? 1 : 4)
         decode_warp<D, BS, MmaMath<D, BS>, 2>(&tm_k, &tm_v, a, sm, ly, pieces, x0, x1, W, gridDim.x, pcost, warp,
                                               lane);
     } else {
-        static_assert(D == 128, "the e4m3 path reads 128-byte rows (head_dim 64 packs head pairs)");
-        decode_warp<D, BS, Fp8Math<BS>, 1>(&tm_k, &tm_v, a, sm, ly, pieces, x0, x1, W, gridDim.x, pcost, warp,
-                                           lane);
+        static_assert(D == 128 || D == 256, "the e4m3 path reads rows of 128 or 256 codes");
+        decode_warp<D, BS, Fp8Math<BS, D / 128>, 1>(&tm_k, &tm_v, a, sm, ly, pieces, x0, x1, W, gridDim.x, pcost,
+                                                    warp, lane);
     }
 }
 
@@ -1356,6 +1399,7 @@ KernelFn pick(int D, int BS, int GP, int math) {
     PKV_CASE(d, bs, 8, kMathCudaCore) PKV_CASE(d, bs, 8, kMathTensorCore)
     PKV_GP(64, 16) PKV_GP(64, 32) PKV_GP(128, 16) PKV_GP(128, 32)
     PKV_CASE(128, 16, 8, kMathFp8) PKV_CASE(128, 32, 8, kMathFp8)
+    PKV_CASE(256, 16, 8, kMathFp8) PKV_CASE(256, 32, 8, kMathFp8)
 #undef PKV_GP
 #undef PKV_CASE
     return nullptr;
@@ -1368,9 +1412,9 @@ bool decode_variant_exists(int head_dim, int block_size, int group_pad, int math
 }
 
 size_t decode_smem_bytes(int head_dim, int block_size, int group_pad, int group, int math, int num_stages,
-                         int num_seqs) {
+                         int num_seqs, int pack) {
     return decode_layout(head_dim, block_size, effective_group_pad(group_pad, math), group, math != kMathCudaCore,
-                         kConsumerWarps * num_stages, num_seqs, math == kMathFp8 ? 1 : 2)
+                         kConsumerWarps * num_stages, num_seqs, math == kMathFp8 ? 1 : 2, head_dim / pack)
         .total;
 }
 

@@ -67,20 +67,22 @@ __host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) { return (x
 // slack for aligning the dynamic shared-memory base. GP = compile-time padded
 // group, G = the actual group (query heads per kv head), tensor_core = the
 // mma.sync math path (its probability scratch is bf16 [8][BS] per warp).
+// kv_elem_bytes = bytes per pool element; dr = dims per stored q / out row
+// (D / pack).
 __host__ __device__ inline DecodeLayout decode_layout(int D, int BS, int GP, int G, bool tensor_core, int num_stages,
-                                                      int num_seqs, int kv_elem_bytes = 2) {
+                                                      int num_seqs, int kv_elem_bytes, int dr) {
     DecodeLayout L;
     uint32_t off = 0;
     const uint32_t tile = static_cast<uint32_t>(BS * D * kv_elem_bytes);
     L.stages = off;
     off += static_cast<uint32_t>(num_stages) * 2u * tile;          // [stage][K tile, V tile]
     L.qbuf = off;
-    off += 2u * G * D * 2;                                          // two query slots [G][D] bf16
+    off += 2u * G * dr * 2;                                         // two query slots [G][dr] bf16
     off = align_up(off, 16);
     L.pscr = off;
     off += kConsumerWarps * (tensor_core ? BS * 16 : BS * GP * 8);  // per warp probabilities (16-bit [8][BS] on tensor cores)
     L.merge_acc = off;
-    off += kConsumerWarps * G * D * 4;                              // per warp fp32 [G][D]
+    off += kConsumerWarps * G * dr * 4;                             // per warp fp32 [G][dr]
     L.merge_m = off;
     off += kConsumerWarps * G * 4;
     L.merge_l = off;

@@ -19,7 +19,7 @@ bool decode_variant_exists(int head_dim, int block_size, int group_pad, int math
 
 // Shared-memory bytes per CTA of a decode variant (num_stages = stages per consumer warp).
 size_t decode_smem_bytes(int head_dim, int block_size, int group_pad, int group, int math, int num_stages,
-                         int num_seqs);
+                         int num_seqs, int pack);
 
 // Sets the variant's dynamic shared-memory limit (once per device) and returns
 // how many CTAs of it fit on one SM.

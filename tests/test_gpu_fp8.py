@@ -75,7 +75,7 @@ def test_fp8_step_matches_oracle(name):
 
 @pytest.mark.parametrize("name", ["opt125m", "qwen25_7b_prefix", "skewed_long"])
 @pytest.mark.parametrize("opts", [dict(num_ctas=1), dict(num_ctas=7), dict(num_ctas=300), dict(num_ctas=1024),
-                                  dict(num_stages=1), dict(num_stages=4, ctas_per_sm=2)])
+                                  dict(num_stages=1), dict(num_stages=3, ctas_per_sm=1)])
 def test_fp8_grid_splits_and_rings(name, opts):
     b, (ref, _, _) = case(name)
     out, _, _, st = one_launch(b, **opts)
@@ -100,6 +100,18 @@ def test_fp8_every_supported_group_and_shape(G, D, bs):
         assert st == 0
         assert np.array_equal(kc.numpy(), kc_ref) and np.array_equal(vc.numpy(), vc_ref)
         assert_close_to_oracle(out.double().numpy(), ref, what=f"fp8 G={G} D={D} bs={bs} C={num_ctas}")
+
+
+@pytest.mark.parametrize("name", ["llama3_8b", "skewed_long"])
+@pytest.mark.parametrize("opts", [dict(head_pack=1), dict(head_pack=2), dict(head_pack=2, num_ctas=1000),
+                                  dict(head_pack=2, num_stages=2)])
+def test_fp8_one_and_two_head_rows(name, opts):
+    """head_dim 128 reads kv-head pairs as 256-code rows by default; head_pack 1 reads 128-code rows."""
+    b, (ref, kc_ref, vc_ref) = case(name)
+    out, kc, vc, st = one_launch(b, **opts)
+    assert st == 0
+    assert np.array_equal(kc.numpy(), kc_ref) and np.array_equal(vc.numpy(), vc_ref)
+    assert_close_to_oracle(out.double().numpy(), ref, what=f"fp8 {name} {opts}")
 
 
 def test_fp8_refuses_what_it_cannot_read():
