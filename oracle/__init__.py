@@ -77,6 +77,12 @@ def _bind(path: str):
         ctypes.c_int, ctypes.c_int64, ctypes.c_double,
         P, ctypes.c_int64, ctypes.c_int,
     ]
+    lib.oracle_paged_prefill.restype = ctypes.c_int
+    lib.oracle_paged_prefill.argtypes = [
+        P, P, P, P, P, P, P,
+        ctypes.c_int, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+        ctypes.c_int, ctypes.c_int64, ctypes.c_double, ctypes.c_int,
+    ]
     lib.oracle_kv_append_fp8.restype = ctypes.c_int
     lib.oracle_kv_append_fp8.argtypes = [
         P, P, P, P, P, P, P, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64,
@@ -271,3 +277,25 @@ def decode_step_fp8(batch, pairs: Optional[Sequence[int]] = None, num_threads: i
                            batch.context_lens.numpy(), batch.num_kv_heads, batch.block_size, batch.scale,
                            pairs=pairs, num_threads=num_threads, lib=lib)
     return out, kc, vc
+
+
+def paged_prefill(q, k_cache, v_cache, block_tables, context_lens, query_start, num_kv_heads: int,
+                  block_size: int, scale: float, num_threads: int = 0, lib=None) -> np.ndarray:
+    """fp64 multi-query paged attention: q bf16 [T][Hq][D] packed by query_start [S+1];
+    query i of sequence s attends causally to positions 0 .. L_s - n_s + i. Returns [T][Hq][D]."""
+    qb, kb, vb = _bits(q), _bits(k_cache), _bits(v_cache)
+    T, Hq, D = qb.shape
+    NB = kb.shape[0]
+    assert kb.shape == (NB, block_size, num_kv_heads, D) and vb.shape == kb.shape
+    bt = _i32(block_tables)
+    cl = _i32(context_lens)
+    qs = _i32(query_start)
+    S = cl.shape[0]
+    assert qs.shape == (S + 1,) and bt.shape[0] == S
+    out = np.zeros((T, Hq, D), dtype=np.float64)
+    rc = (lib or _load()).oracle_paged_prefill(
+        _ptr(out), _ptr(qb), _ptr(kb), _ptr(vb), _ptr(bt), _ptr(cl), _ptr(qs), S, T, Hq, num_kv_heads, D,
+        block_size, bt.shape[1], NB, float(scale), int(num_threads))
+    if rc != 0:
+        raise OracleError(f"oracle_paged_prefill returned {rc}")
+    return out

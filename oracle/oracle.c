@@ -36,6 +36,14 @@
  * Token i goes to slot slot_mapping[i] = physical_block * bs + offset; a
  * negative slot means "no write".
  *
+ * Chunked prefill / mixed batches ("vLLM Fundamentals", section "Continuous
+ * Batching": long prefills are cut into chunks under a per-step token budget
+ * and mixed with decodes; each request processes some number of tokens per
+ * step): sequence s brings n_s query tokens, the last n_s of its L_s cached
+ * tokens. Query i (position p = L_s - n_s + i) attends, causally, to the
+ * cache positions 0 .. p -- the same plain definition over a shorter
+ * context. n_s = 1 is the decode step.
+ *
  * FP8 cache (runbyai post 449, section 5, names quantization among the means
  * for long contexts; the format is the task's reading): pools of e4m3 codes
  * (1 sign, 4 exponent bits with bias 7, 3 mantissa bits; exponent 15 with
@@ -123,14 +131,13 @@ static int64_t pool_row(int64_t p, int off, int h, int block_size, int num_kv_he
  * Returns 0, or -2 when a table entry it needs is outside [0, num_blocks).
  */
 static int decode_one(double *out, double *x,
-                      const uint16_t *q, const Pool *K, const Pool *V,
+                      const uint16_t *qrow, const Pool *K, const Pool *V,
                       const int32_t *block_tables, int context_len,
                       int s, int j, int num_q_heads, int num_kv_heads, int head_dim,
                       int block_size, int max_blocks_per_seq, int64_t num_blocks, double scale)
 {
     const int group = num_q_heads / num_kv_heads;
     const int h = j / group;
-    const uint16_t *qrow = q + ((int64_t)s * num_q_heads + j) * head_dim;
     const int32_t *table = block_tables + (int64_t)s * max_blocks_per_seq;
 
     for (int d = 0; d < head_dim; ++d)
@@ -226,7 +233,8 @@ static int decode_pool(double *out, const uint16_t *q, const Pool *K, const Pool
             int s = (int)(flat / num_q_heads);
             int j = (int)(flat % num_q_heads);
             if (mine == 0)
-                mine = decode_one(out + k * head_dim, x, q, K, V, block_tables,
+                mine = decode_one(out + k * head_dim, x, q + ((int64_t)s * num_q_heads + j) * head_dim, K, V,
+                                  block_tables,
                                   context_lens[s], s, j, num_q_heads, num_kv_heads, head_dim,
                                   block_size, max_blocks_per_seq, num_blocks, scale);
         }
@@ -348,4 +356,80 @@ int oracle_kv_append_fp8(uint8_t *k_cache, uint8_t *v_cache, const uint16_t *k, 
         }
     }
     return 0;
+}
+
+/*
+ * Multi-query paged attention (chunked prefill, mixed batches), fp64.
+ *
+ * out           [num_tokens][num_q_heads][head_dim] doubles
+ * q             bf16 bits [num_tokens][num_q_heads][head_dim]; the queries of
+ *               sequence s are rows query_start[s] .. query_start[s + 1] - 1
+ * query_start   [num_seqs + 1], non-decreasing, query_start[0] = 0,
+ *               query_start[num_seqs] = num_tokens; n_s = query_start[s+1] -
+ *               query_start[s] <= context_lens[s]
+ * the rest as oracle_paged_decode.  Query i of sequence s sits at position
+ * p = context_lens[s] - n_s + i and attends to positions 0 .. p.
+ *
+ * Returns 0; -1 for a bad argument; -2 for a table entry outside the pool;
+ * -3 for a context length outside [0, max_blocks_per_seq * block_size].
+ */
+int oracle_paged_prefill(double *out, const uint16_t *q, const uint16_t *k_cache, const uint16_t *v_cache,
+                         const int32_t *block_tables, const int32_t *context_lens, const int32_t *query_start,
+                         int num_seqs, int64_t num_tokens, int num_q_heads, int num_kv_heads, int head_dim,
+                         int block_size, int max_blocks_per_seq, int64_t num_blocks, double scale, int num_threads)
+{
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !query_start)
+        return -1;
+    if (num_seqs < 0 || num_tokens < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+        block_size <= 0 || max_blocks_per_seq < 0 || num_blocks < 0 || num_q_heads % num_kv_heads != 0)
+        return -1;
+    if (query_start[0] != 0 || query_start[num_seqs] != num_tokens)
+        return -1;
+    int max_len = 0;
+    for (int s = 0; s < num_seqs; ++s) {
+        int64_t n = (int64_t)query_start[s + 1] - query_start[s];
+        if (n < 0)
+            return -1;
+        if (context_lens[s] < 0 || (int64_t)context_lens[s] > (int64_t)max_blocks_per_seq * block_size)
+            return -3;
+        if (n > context_lens[s])
+            return -1;
+        if (context_lens[s] > max_len)
+            max_len = context_lens[s];
+    }
+    Pool K = {k_cache, NULL, NULL}, V = {v_cache, NULL, NULL};
+    int status = 0;
+#ifdef _OPENMP
+    if (num_threads <= 0)
+        num_threads = omp_get_max_threads();
+#pragma omp parallel num_threads(num_threads)
+#endif
+    {
+        double *x = (double *)malloc(sizeof(double) * (size_t)(max_len > 0 ? max_len : 1));
+        int mine = x ? 0 : -1;
+#ifdef _OPENMP
+#pragma omp for schedule(dynamic, 1) collapse(2)
+#endif
+        for (int s = 0; s < num_seqs; ++s) {
+            for (int j = 0; j < num_q_heads; ++j) {
+                int n = query_start[s + 1] - query_start[s];
+                for (int i = 0; i < n && mine == 0; ++i) {
+                    int64_t row = (int64_t)query_start[s] + i;
+                    int p = context_lens[s] - n + i;           /* this query's position */
+                    /* decode of this one query over the context 0 .. p of sequence s */
+                    mine = decode_one(out + (row * num_q_heads + j) * head_dim, x,
+                                      q + (row * num_q_heads + j) * (int64_t)head_dim, &K, &V, block_tables,
+                                      p + 1, s, j, num_q_heads, num_kv_heads, head_dim, block_size,
+                                      max_blocks_per_seq, num_blocks, scale);
+                }
+            }
+        }
+        free(x);
+#ifdef _OPENMP
+#pragma omp critical
+#endif
+        if (mine != 0 && status == 0)
+            status = mine;
+    }
+    return status;
 }

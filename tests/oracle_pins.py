@@ -399,6 +399,77 @@ def pin_fp8_poisoned_slots_are_never_read(lib=None):
     assert np.isfinite(got).all()
 
 
+# ---------------------------------------------------------------- multi-query (chunked prefill)
+
+PREFILL_CASES = [
+    # (chunk_lens, context_lens, Hq, Hkv, D, bs)
+    ([3, 1, 0, 20], [10, 5, 7, 40], 4, 2, 16, 4),
+    ([8, 8], [8, 33], 2, 1, 32, 8),
+    ([5, 2, 9], [5, 17, 60], 6, 3, 8, 16),
+]
+
+
+def _prefill(b, lib, **kw):
+    return oracle.paged_prefill(b.q, b.k_cache, b.v_cache, b.block_tables.numpy(), b.context_lens.numpy(),
+                                b.query_start.numpy(), b.num_kv_heads, b.block_size, kw.get("scale", b.scale),
+                                lib=lib)
+
+
+def pin_prefill_causal_sdpa(lib=None):
+    """torch SDPA in fp64 on gathered rows with the causal mask of a chunk at the end of its context."""
+    for i, (n, L, Hq, Hkv, D, bs) in enumerate(PREFILL_CASES):
+        b = workloads.make_prefill(500 + i, n, L, Hq, Hkv, D, bs)
+        got = _prefill(b, lib)
+        G = Hq // Hkv
+        qs = b.query_start.numpy()
+        for s, (k, v) in enumerate(gather_contiguous(b)):
+            ns = int(qs[s + 1] - qs[s])
+            if ns == 0:
+                continue
+            Ls = k.shape[0]
+            kt = torch.from_numpy(k).permute(1, 0, 2).repeat_interleave(G, dim=0)[None]
+            vt = torch.from_numpy(v).permute(1, 0, 2).repeat_interleave(G, dim=0)[None]
+            qt = b.q[qs[s]:qs[s + 1]].double().permute(1, 0, 2)[None]                  # [1][Hq][n][D]
+            allowed = torch.arange(Ls)[None, :] <= (Ls - ns + torch.arange(ns))[:, None]
+            ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=allowed, scale=b.scale)
+            _close(got[qs[s]:qs[s + 1]], ref[0].permute(1, 0, 2).numpy(), what=f"prefill case {i} seq {s}")
+
+
+def pin_prefill_single_queries_are_decodes(lib=None):
+    """Chunks of one token are decode steps over the whole context."""
+    L = [9, 1, 30, 17]
+    b = workloads.make_prefill(510, [1] * len(L), L, 4, 2, 16, 4)
+    got = _prefill(b, lib)
+    dec = oracle.paged_decode(b.q, b.k_cache, b.v_cache, b.block_tables.numpy(), b.context_lens.numpy(),
+                              b.num_kv_heads, b.block_size, b.scale, lib=lib)
+    _close(got, dec, what="n = 1")
+
+
+def pin_prefill_equal_keys_give_prefix_means(lib=None):
+    """All keys equal: query i of a chunk gets the mean of V over positions 0 .. p_i."""
+    b = workloads.make_prefill(520, [6, 3], [6, 12], 2, 1, 8, 4, poison=False)
+    kc = b.k_cache.clone()
+    kc[:] = kc[0, 0, 0]
+    b = dataclasses.replace(b, k_cache=kc)
+    got = _prefill(b, lib)
+    qs = b.query_start.numpy()
+    for s, (_, v) in enumerate(gather_contiguous(b)):
+        ns = int(qs[s + 1] - qs[s])
+        Ls = v.shape[0]
+        for i in range(ns):
+            p = Ls - ns + i
+            _close(got[qs[s] + i], np.repeat(v[:p + 1].mean(axis=0), b.num_q_heads // b.num_kv_heads, axis=0),
+                   what=f"equal keys seq {s} query {i}")
+
+
+def pin_prefill_block_permutation_invariance(lib=None):
+    n, L, Hq, Hkv, D, bs = PREFILL_CASES[0]
+    b = workloads.make_prefill(530, n, L, Hq, Hkv, D, bs)
+    pb = workloads.permute_pool(b, seed=5)
+    pb = dataclasses.replace(b, k_cache=pb.k_cache, v_cache=pb.v_cache, block_tables=pb.block_tables)
+    _close(_prefill(pb, lib), _prefill(b, lib), what="prefill permutation")
+
+
 ALL_PINS = [
     pin_sdpa_random,
     pin_golden,
@@ -425,4 +496,8 @@ ALL_PINS = [
     pin_fp8_append_matches_torch_quantization,
     pin_fp8_scales_act_as_the_pages_define,
     pin_fp8_poisoned_slots_are_never_read,
+    pin_prefill_causal_sdpa,
+    pin_prefill_single_queries_are_decodes,
+    pin_prefill_equal_keys_give_prefix_means,
+    pin_prefill_block_permutation_invariance,
 ]

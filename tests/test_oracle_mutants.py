@@ -17,7 +17,8 @@ MUTANTS = [
     ("normalise by count", "z += w;", "z += 1.0;"),
     ("scale dropped", "x[t] = scale * dot;", "x[t] = dot;"),
     ("head grouping j mod Hkv", "const int h = j / group;", "const int h = j % num_kv_heads;"),
-    ("q row of the kv head", "((int64_t)s * num_q_heads + j) * head_dim", "((int64_t)s * num_q_heads + h) * head_dim"),
+    ("q row of the kv head", "q + ((int64_t)s * num_q_heads + j) * head_dim",
+     "q + ((int64_t)s * num_q_heads + j / (num_q_heads / num_kv_heads)) * head_dim"),
     ("values read from K", "pool_value(V, vrow + d, h)", "pool_value(K, vrow + d, h)"),
     ("block table ignored", "table[t / block_size]", "(t / block_size)"),
     ("offset off by one", "pool_row(p, t % block_size", "pool_row(p, (t + 1) % block_size"),
@@ -35,6 +36,10 @@ MUTANTS = [
     ("e4m3 no saturation", "if (a >= 448.0)", "if (a >= 480.0)"),
     ("fp8 scale of head 0", "* (double)P->scale[h];", "* (double)P->scale[0];"),
     ("fp8 append uses the K scale for V", "/ v_scale[h];", "/ k_scale[h];"),
+    ("prefill sees one token too few", "int p = context_lens[s] - n + i;", "int p = context_lens[s] - n + i - 1;"),
+    ("prefill sees the whole context", "int p = context_lens[s] - n + i;", "int p = context_lens[s] - 1;"),
+    ("prefill reads the chunk's first query", "q + (row * num_q_heads + j) * (int64_t)head_dim",
+     "q + ((int64_t)query_start[s] * num_q_heads + j) * (int64_t)head_dim"),
 ]
 
 

@@ -18,4 +18,7 @@ from .decode_batches import (  # noqa: F401
     E4M3_NAN_CODE,
     fp8_scales,
     kv_element_bytes,
+    PrefillBatch,
+    make_prefill,
+    prefill_flops,
 )

@@ -427,3 +427,47 @@ def unique_kv_bytes(batch: DecodeBatch) -> int:
             p = int(tables[s, b])
             used[p] = max(used.get(p, 0), min(bs, L - b * bs))
     return sum(used.values()) * 2 * batch.num_kv_heads * batch.head_dim * kv_element_bytes(batch)
+
+
+@dataclasses.dataclass
+class PrefillBatch(DecodeBatch):
+    """A mixed batch of query chunks: q is [T][Hq][D], the queries of sequence s
+    are rows query_start[s] .. query_start[s + 1] - 1, the last n_s of its L_s
+    tokens (already in the pool). k_new / v_new / slot_mapping are unused."""
+
+    query_start: Optional[torch.Tensor] = None   # int32 [S + 1] (host)
+
+
+def make_prefill(seed: int, chunk_lens: Sequence[int], context_lens: Sequence[int], num_q_heads: int,
+                 num_kv_heads: int, head_dim: int, block_size: int, scale: Optional[float] = None,
+                 pool_factor: float = 1.25, device="cpu", poison: bool = True) -> PrefillBatch:
+    """A chunked-prefill / mixed batch by the decode recipe (pool of all L tokens,
+    poisoned elsewhere), then the T = sum(chunk_lens) query rows, N(0, 1) in bf16
+    from the same generator stream, drawn after the pool."""
+    n = np.asarray(chunk_lens, dtype=np.int64)
+    lens = np.asarray(context_lens, dtype=np.int64)
+    assert len(n) == len(lens) and (n <= lens).all() and (n >= 0).all()
+    b = make_custom(seed, lens, num_q_heads, num_kv_heads, head_dim, block_size, scale=scale,
+                    pool_factor=pool_factor, device=device, poison=poison, with_append=False)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed + 1_000_003)
+    T = int(n.sum())
+    q = _randn_bf16((max(T, 0), num_q_heads, head_dim), gen, device) if T else torch.empty(
+        0, num_q_heads, head_dim, dtype=torch.bfloat16, device=device)
+    qs = np.zeros(len(n) + 1, dtype=np.int32)
+    qs[1:] = np.cumsum(n)
+    fields = {f.name: getattr(b, f.name) for f in dataclasses.fields(DecodeBatch)}
+    fields["q"] = q
+    return PrefillBatch(**fields, query_start=torch.from_numpy(qs))
+
+
+def prefill_flops(batch: PrefillBatch) -> int:
+    """Multiply-adds x 2 of q.K and P.V: every query token attends to p + 1 positions."""
+    qs = batch.query_start.numpy()
+    lens = batch.context_lens.numpy()
+    total = 0
+    for s in range(len(lens)):
+        n = int(qs[s + 1] - qs[s])
+        L = int(lens[s])
+        total += n * (L - n) + n * (n + 1) // 2  # sum over queries of (p + 1)
+    return total * batch.num_q_heads * batch.head_dim * 4
