@@ -155,6 +155,39 @@ int paged_attn_decode_ex(void *out, const void *q, const void *k_cache, const vo
                          void *stream);
 
 /*
+ * Multi-query paged attention: chunked prefill and mixed batches ("vLLM
+ * Fundamentals", section "Continuous Batching": long prefills are cut into
+ * chunks under a token budget and batched with decodes). Sequence s brings
+ * n_s = query_start[s + 1] - query_start[s] query tokens, the LAST n_s of its
+ * context_lens[s] tokens, whose keys and values are already in the pool
+ * (kv_cache_append). Query i of sequence s sits at position
+ * p = context_lens[s] - n_s + i and attends causally to positions 0 .. p:
+ *   out[query_start[s] + i][j] = softmax_t<=p(scale q.K_t) . V_t, kv head j / G.
+ * A decode step is the case n_s = 1.
+ *
+ * out, q        device bf16 [num_tokens][num_q_heads][head_dim]
+ * query_start   device int32 [num_seqs + 1]: 0, then non-decreasing, ending at
+ *               num_tokens; every n_s <= context_lens[s] and <= max_query_len
+ *               (host int: the largest n_s, which sizes the grid)
+ * d_status      device int32 status word (required): a sequence whose
+ *               query_start / context length is inconsistent is skipped and sets
+ *               PKV_STATUS_BAD_CONTEXT_LEN; a bad table entry sets
+ *               PKV_STATUS_BAD_BLOCK_ID (that block is skipped).
+ * The rest as paged_attn_decode. Supported: head_dim 64 / 128, block_size
+ * 16 / 32, group <= 8, num_seqs and num_kv_heads <= 65535, max_blocks_per_seq *
+ * 4 bytes + 2 K/V blocks of shared memory per CTA. One launch; no workspace.
+ * Kernel: a CTA per (64 rows of (query token, group head), sequence, kv head)
+ * streams the K/V blocks its rows need (TMA tile copies, 2-stage ring) and
+ * computes S = Q K^T, a causal online softmax and O += P V on tensor cores
+ * (mma.sync m16n8k16 bf16, fp32 accumulate; P rounded to bf16).
+ */
+int paged_attn_prefill(void *out, const void *q, const void *k_cache, const void *v_cache,
+                       const int32_t *block_tables, const int32_t *context_lens, const int32_t *query_start,
+                       int num_seqs, int num_tokens, int max_query_len, int num_q_heads, int num_kv_heads,
+                       int head_dim, int block_size, float scale, int max_blocks_per_seq, int num_blocks,
+                       int32_t *d_status, void *stream);
+
+/*
  * FP8 KV cache. The pools hold e4m3 codes (1 sign, 4 exponent bits with bias
  * 7, 3 mantissa bits; 0x7f / 0xff are NaN), laid out like the bf16 pools,
  * [num_blocks][block_size][num_kv_heads][head_dim] bytes, with one fp32 scale

@@ -81,6 +81,8 @@ def library() -> ctypes.CDLL:
                                                          Z, ctypes.POINTER(_Options), P]
             lib.kv_cache_append_fp8.restype = I
             lib.kv_cache_append_fp8.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, P, P]
+            lib.paged_attn_prefill.restype = I
+            lib.paged_attn_prefill.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, I, I, P, P]
             lib.kv_cache_append.restype = I
             lib.kv_cache_append.argtypes = [P, P, P, P, P, I, I, I, I, I, P, P]
             lib.pkv_validate.restype = I
@@ -378,3 +380,30 @@ def kv_cache_append_fp8(k: torch.Tensor, v: torch.Tensor, k_cache: torch.Tensor,
     _check("kv_cache_append_fp8", library().kv_cache_append_fp8(
         _ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache), _ptr(slot_mapping), _ptr(k_scale), _ptr(v_scale), T, Hkv,
         D, bs, NB, _ptr(status), _stream(stream)))
+
+
+def paged_attn_prefill(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                       block_tables: torch.Tensor, context_lens: torch.Tensor, query_start: torch.Tensor,
+                       max_query_len: int, scale: float, status: torch.Tensor, stream=None) -> torch.Tensor:
+    """Multi-query paged attention: q bf16 [T, Hq, D]; the queries of sequence s are rows
+    query_start[s] .. query_start[s+1]-1, the last tokens of its context, attending causally."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need(out, "out", torch.bfloat16, 3)
+    _need(k_cache, "k_cache", torch.bfloat16, 4)
+    _need(v_cache, "v_cache", torch.bfloat16, 4)
+    _need(block_tables, "block_tables", torch.int32, 2)
+    _need(context_lens, "context_lens", torch.int32, 1)
+    _need(query_start, "query_start", torch.int32, 1)
+    _need(status, "status", torch.int32, 1)
+    T, Hq, D = q.shape
+    NB, bs, Hkv, D2 = k_cache.shape
+    S = context_lens.shape[0]
+    if out.shape != q.shape or v_cache.shape != k_cache.shape or D2 != D:
+        raise ValueError("shape mismatch between q/out or k_cache/v_cache")
+    if block_tables.shape[0] != S or query_start.shape[0] != S + 1:
+        raise ValueError("block_tables needs num_seqs rows and query_start num_seqs + 1 entries")
+    _check("paged_attn_prefill", library().paged_attn_prefill(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens), _ptr(query_start),
+        S, T, int(max_query_len), Hq, Hkv, D, bs, float(scale), block_tables.shape[1], NB, _ptr(status),
+        _stream(stream)))
+    return out

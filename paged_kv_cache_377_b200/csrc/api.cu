@@ -375,6 +375,73 @@ int kv_cache_append(const void *k, const void *v, void *k_cache, void *v_cache, 
     return ok();
 }
 
+int paged_attn_prefill(void *out, const void *q, const void *k_cache, const void *v_cache,
+                       const int32_t *block_tables, const int32_t *context_lens, const int32_t *query_start,
+                       int num_seqs, int num_tokens, int max_query_len, int num_q_heads, int num_kv_heads,
+                       int head_dim, int block_size, float scale, int max_blocks_per_seq, int num_blocks,
+                       int32_t *d_status, void *stream) {
+    if (num_seqs < 0 || num_tokens < 0 || max_query_len < 0)
+        return fail(PKV_ERR_INVALID_ARGUMENT, "num_seqs, num_tokens and max_query_len must be >= 0");
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !query_start || !d_status)
+        return fail(PKV_ERR_INVALID_ARGUMENT, "a required pointer is NULL");
+    if (num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0 || max_blocks_per_seq <= 0 ||
+        num_blocks <= 0)
+        return fail(PKV_ERR_INVALID_ARGUMENT, "head counts, head_dim, block_size, max_blocks_per_seq and "
+                                              "num_blocks must be positive");
+    if (num_q_heads % num_kv_heads != 0)
+        return fail(PKV_ERR_INVALID_ARGUMENT, "num_q_heads %d is not a multiple of num_kv_heads %d", num_q_heads,
+                    num_kv_heads);
+    if (!std::isfinite(scale)) return fail(PKV_ERR_INVALID_ARGUMENT, "scale is not finite");
+    const int group = num_q_heads / num_kv_heads;
+    if (head_dim != 64 && head_dim != 128)
+        return fail(PKV_ERR_UNSUPPORTED, "head_dim %d not supported (64 or 128)", head_dim);
+    if (block_size != 16 && block_size != 32)
+        return fail(PKV_ERR_UNSUPPORTED, "block_size %d not supported (16 or 32)", block_size);
+    if (group > PKV_MAX_GROUP)
+        return fail(PKV_ERR_UNSUPPORTED, "num_q_heads / num_kv_heads = %d exceeds %d", group, PKV_MAX_GROUP);
+    if (static_cast<int64_t>(num_blocks) * block_size > 0x7fffffff ||
+        static_cast<int64_t>(max_blocks_per_seq) * block_size > 0x7fffffff)
+        return fail(PKV_ERR_INVALID_ARGUMENT, "pool or table too large: blocks * block_size must be < 2^31");
+    if (num_seqs > 65535 || num_kv_heads > 65535)
+        return fail(PKV_ERR_UNSUPPORTED, "at most 65535 sequences and kv heads per call");
+    if (static_cast<int64_t>(num_tokens) * num_q_heads * head_dim > (int64_t(1) << 40))
+        return fail(PKV_ERR_INVALID_ARGUMENT, "num_tokens too large");
+    if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(d_status, 4))
+        return fail(PKV_ERR_INVALID_ARGUMENT, "out, q, k_cache and v_cache must be 16-byte aligned");
+    const size_t smem = pkv::prefill_smem_bytes(head_dim, block_size, max_blocks_per_seq);
+    if (smem > 227 * 1024)
+        return fail(PKV_ERR_UNSUPPORTED, "max_blocks_per_seq %d needs %zu bytes of shared memory", max_blocks_per_seq,
+                    smem);
+    if (num_seqs == 0 || num_tokens == 0 || max_query_len == 0) return ok();
+    const int64_t tiles = (static_cast<int64_t>(max_query_len) * group + pkv::prefill_rows_per_cta() - 1) /
+                          pkv::prefill_rows_per_cta();
+    if (tiles > 0x7fffffff) return fail(PKV_ERR_INVALID_ARGUMENT, "max_query_len too large");
+    CUtensorMap tm_k, tm_v;
+    int rc;
+    if ((rc = make_pool_map(&tm_k, k_cache, num_blocks, block_size, num_kv_heads, head_dim)) != PKV_OK) return rc;
+    if ((rc = make_pool_map(&tm_v, v_cache, num_blocks, block_size, num_kv_heads, head_dim)) != PKV_OK) return rc;
+    pkv::PrefillArgs a{};
+    a.out = out;
+    a.q = q;
+    a.block_tables = block_tables;
+    a.context_lens = context_lens;
+    a.query_start = query_start;
+    a.status = d_status;
+    a.num_seqs = num_seqs;
+    a.num_tokens = num_tokens;
+    a.num_q_heads = num_q_heads;
+    a.num_kv_heads = num_kv_heads;
+    a.group = group;
+    a.max_blocks_per_seq = max_blocks_per_seq;
+    a.num_blocks = num_blocks;
+    a.max_query_len = max_query_len;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    cudaError_t e = pkv::prefill_launch(head_dim, block_size, tm_k, tm_v, a, static_cast<int>(tiles), smem,
+                                        static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
+    return ok();
+}
+
 int kv_cache_append_fp8(const void *k, const void *v, void *k_cache, void *v_cache, const int64_t *slot_mapping,
                         const float *k_scale, const float *v_scale, int num_tokens, int num_kv_heads, int head_dim,
                         int block_size, int num_blocks, int32_t *d_status, void *stream) {

@@ -35,6 +35,23 @@ cudaError_t append_launch(const void *k, const void *v, void *k_cache, void *v_c
                           int num_tokens, int num_kv_heads, int head_dim, int block_size, int num_blocks,
                           int32_t *status, cudaStream_t stream);
 
+// Multi-query paged attention (prefill.cu).
+struct PrefillArgs {
+    void *out;                    // bf16 [T][Hq][D]
+    const void *q;                // bf16 [T][Hq][D]
+    const int32_t *block_tables;  // [S][MB]
+    const int32_t *context_lens;  // [S]
+    const int32_t *query_start;   // [S + 1]
+    int32_t *status;
+    int num_seqs, num_tokens, num_q_heads, num_kv_heads, group, max_blocks_per_seq, num_blocks, max_query_len;
+    float scale_log2;
+};
+
+size_t prefill_smem_bytes(int head_dim, int block_size, int max_blocks_per_seq);
+cudaError_t prefill_launch(int head_dim, int block_size, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
+                           const PrefillArgs &args, int tiles, size_t smem_bytes, cudaStream_t stream);
+int prefill_rows_per_cta();
+
 cudaError_t append_fp8_launch(const void *k, const void *v, void *k_cache, void *v_cache, const int64_t *slot_mapping,
                               const float *k_scale, const float *v_scale, int num_tokens, int num_kv_heads,
                               int head_dim, int block_size, int num_blocks, int32_t *status, cudaStream_t stream);

@@ -1,0 +1,100 @@
+"""Multi-query paged attention (chunked prefill, mixed batches) through the C
+ABI, against the fp64 oracle: query i of a sequence's n-token chunk attends
+causally to positions 0 .. L - n + i. Tolerance |err| <= 8e-3 + 8e-3 |ref|."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_kv_cache_377_b200 as pkv
+import workloads
+from helpers import assert_close_to_oracle
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def run(b, max_query_len=None):
+    qs = b.query_start
+    mq = int((qs[1:] - qs[:-1]).max()) if max_query_len is None else max_query_len
+    out = torch.full(b.q.shape, float("nan"), dtype=torch.bfloat16, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    pkv.paged_attn_prefill(out, b.q.to(DEV), b.k_cache.to(DEV), b.v_cache.to(DEV), b.block_tables.to(DEV),
+                           b.context_lens.to(DEV), qs.to(DEV), mq, b.scale, status)
+    torch.cuda.synchronize()
+    return out.cpu(), pkv.read_status(status)
+
+
+def ref_of(b):
+    return oracle.paged_prefill(b.q, b.k_cache, b.v_cache, b.block_tables.numpy(), b.context_lens.numpy(),
+                                b.query_start.numpy(), b.num_kv_heads, b.block_size, b.scale)
+
+
+@pytest.mark.parametrize("G", [1, 2, 4, 7, 8])
+@pytest.mark.parametrize("D,bs", [(64, 16), (64, 32), (128, 16), (128, 32)])
+def test_mixed_batch_matches_oracle(G, D, bs):
+    chunks = [1, 7, 16, 64, 130, 0, 1, 33]
+    ctx = [1, 40, 16, 64, 700, 9, 1029, 33]
+    b = workloads.make_prefill(3000 + 11 * G + D + bs, chunks, ctx, 2 * G, 2, D, bs)
+    out, st = run(b)
+    assert st == 0
+    assert_close_to_oracle(out.double().numpy(), ref_of(b), what=f"prefill G={G} D={D} bs={bs}")
+
+
+def test_single_token_chunks_match_the_decode_kernel():
+    lens = [1, 5, 300, 1024, 77]
+    b = workloads.make_prefill(3100, [1] * len(lens), lens, 32, 8, 128, 16)
+    out, st = run(b)
+    assert st == 0
+    ref = ref_of(b)
+    assert_close_to_oracle(out.double().numpy(), ref, what="n = 1")
+    dec = torch.empty_like(b.q, device=DEV)
+    ws = pkv.allocate_workspace(b.num_seqs, b.num_q_heads, b.head_dim, device=DEV)
+    pkv.paged_attn_decode(dec, b.q.to(DEV), b.k_cache.to(DEV), b.v_cache.to(DEV), b.block_tables.to(DEV),
+                          b.context_lens.to(DEV), b.scale, ws)
+    assert_close_to_oracle(dec.double().cpu().numpy(), ref, what="decode kernel on the same rows")
+
+
+def test_llama_shaped_chunked_prefill_sampled_rows():
+    rng = np.random.default_rng(31)
+    chunks = [512, 256, 384, 128, 1, 1, 1, 1]
+    ctx = [int(c + rng.integers(0, 3000)) for c in chunks]
+    b = workloads.make_prefill(3200, chunks, ctx, 32, 8, 128, 16, device="cuda").to("cpu")
+    out, st = run(b)
+    assert st == 0
+    T, Hq = b.q.shape[0], b.num_q_heads
+    rows = np.random.default_rng(2).choice(T, size=48, replace=False)
+    sub_qs = []
+    # the oracle on the sampled query tokens only: one one-token chunk per sampled row
+    qs = b.query_start.numpy()
+    seq_of = np.searchsorted(qs, rows, side="right") - 1
+    for r, s in zip(rows, seq_of):
+        n = int(qs[s + 1] - qs[s])
+        p = int(b.context_lens[s]) - n + int(r - qs[s])
+        sub_qs.append((s, p + 1, r))
+    lens = np.array([x[1] for x in sub_qs], dtype=np.int32)
+    tables = b.block_tables.numpy()[[x[0] for x in sub_qs]]
+    q = b.q[[x[2] for x in sub_qs]]
+    ref = oracle.paged_decode(q, b.k_cache, b.v_cache, tables, lens, b.num_kv_heads, b.block_size, b.scale)
+    assert_close_to_oracle(out[rows].double().numpy(), ref, what="llama-shaped chunked prefill (sampled)")
+
+
+def test_inconsistent_chunks_are_flagged_and_skipped():
+    b = workloads.make_prefill(3300, [3, 4], [10, 12], 4, 2, 64, 16)
+    bad_lens = b.context_lens.clone()
+    bad_lens[1] = 2                                   # a chunk of 4 cannot end a context of 2
+    b2 = workloads.PrefillBatch(**{**b.__dict__, "context_lens": bad_lens})
+    out, st = run(b2)
+    assert st & pkv.PKV_STATUS_BAD_CONTEXT_LEN
+    ref = ref_of(b)
+    assert_close_to_oracle(out[:3].double().numpy(), ref[:3], what="the consistent sequence")
+
+
+def test_bad_block_id_is_flagged_not_faulted():
+    b = workloads.make_prefill(3400, [5, 2], [40, 20], 4, 2, 128, 16)
+    tables = b.block_tables.clone()
+    tables[0, 1] = b.num_blocks + 7
+    b2 = workloads.PrefillBatch(**{**b.__dict__, "block_tables": tables})
+    _, st = run(b2)
+    assert st & pkv.PKV_STATUS_BAD_BLOCK_ID
