@@ -40,6 +40,16 @@ sys.path.insert(0, ROOT)
 import workloads  # noqa: E402
 
 METRIC = "paged decode KV GB/s & % of B200 HBM peak; seq·tokens/s per decode step"
+PREFILL_METRIC = "multi-query paged attention TFLOP/s (chunked prefill)"
+
+# Multi-query (chunked prefill) workloads: chunk lengths and a context draw per sequence.
+PREFILL_WORKLOADS = {
+    "prefill_llama_chunks": dict(
+        description="Llama-3-8B GQA heads: 16 seqs x 512-token chunks at the end of contexts 512 + U[0, 3584], "
+                    "32/8 heads, D128, bs16",
+        chunks=[512] * 16, ctx=lambda rng: [512 + int(x) for x in rng.integers(0, 3585, 16)],
+        heads=(32, 8), head_dim=128, block_size=16),
+}
 FALLBACK_HBM_GBS = 6650.0
 PROFILES = os.path.join(ROOT, "profiles")
 
@@ -52,7 +62,9 @@ def parse_args(argv=None):
     p.add_argument("--steps", type=int, default=200)
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--workload", default="llama3_8b", choices=workloads.CONFIG_ORDER)
+    p.add_argument("--workload", default="llama3_8b", choices=list(workloads.CONFIG_ORDER) + list(PREFILL_WORKLOADS))
+    p.add_argument("--kv-dtype", default="bf16", choices=["bf16", "fp8"],
+                   help="decode workloads: bf16 pools, or e4m3 codes with per-head scales")
     p.add_argument("--num-ctas", type=int, default=0)
     p.add_argument("--num-stages", type=int, default=0)
     p.add_argument("--ctas-per-sm", type=int, default=0)
@@ -234,15 +246,32 @@ class Step:
                          ctas_per_sm=args.ctas_per_sm, math=args.math, l2_prefetch=args.l2_prefetch,
                          piece_cost=args.piece_cost, head_pack=args.head_pack)
         self.ws = pkv.allocate_workspace(b.num_seqs, b.num_q_heads, b.head_dim, device=device)
+        self.fp8 = b.kv_dtype == "fp8"
+        if self.fp8:
+            self.ks = b.k_scale.to(device)
+            self.vs = b.v_scale.to(device)
 
     def append(self, stream=None):
+        if self.fp8:
+            self.pkv.kv_cache_append_fp8(self.k_new, self.v_new, self.kc, self.vc, self.slots, self.ks, self.vs,
+                                         self.status, stream=stream)
+            return
         self.pkv.kv_cache_append(self.k_new, self.v_new, self.kc, self.vc, self.slots, self.status, stream=stream)
 
     def decode(self, stream=None):
+        if self.fp8:
+            self.pkv.paged_attn_decode_fp8(self.out, self.q, self.kc, self.vc, self.ks, self.vs, self.bt, self.cl,
+                                           self.b.scale, self.ws, stream=stream, **self.opts)
+            return
         self.pkv.paged_attn_decode(self.out, self.q, self.kc, self.vc, self.bt, self.cl, self.b.scale, self.ws,
                                    stream=stream, **self.opts)
 
     def fused_step(self, stream=None):
+        if self.fp8:
+            self.pkv.paged_attn_decode_append_fp8(self.out, self.q, self.k_new, self.v_new, self.slots, self.kc,
+                                                  self.vc, self.ks, self.vs, self.bt, self.cl, self.b.scale, self.ws,
+                                                  stream=stream, **self.opts)
+            return
         self.pkv.paged_attn_decode_append(self.out, self.q, self.k_new, self.v_new, self.slots, self.kc, self.vc,
                                           self.bt, self.cl, self.b.scale, self.ws, stream=stream, **self.opts)
 
@@ -277,7 +306,7 @@ def run_ours(args, rank, world, local_rank):
     if args.seqs:  # the workload's recipe cut to its first N lengths (pool sized for those)
         lens = cfg.lengths(np.random.default_rng(rank_seed(cfg.seed, rank)))[:args.seqs].tolist()
     batch = workloads.make_batch(args.workload, seed=rank_seed(cfg.seed, rank), device=device, poison=False,
-                                 lens_override=lens)
+                                 lens_override=lens, kv_dtype=args.kv_dtype)
     step = Step(batch, args, device)
     kv = workloads.kv_bytes(batch)
     ctx_tokens = int(batch.context_lens.sum())
@@ -342,7 +371,7 @@ def run_ours(args, rank, world, local_rank):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "f32",
+        "dtype": "f32" if args.kv_dtype == "bf16" else "f32 (e4m3 KV, f16 products)",
         "data": "synthetic",
         "config": config_block(args, batch, world),
         "pct_of_hbm_peak": round(100.0 * value / (hbm * world), 2),
@@ -417,7 +446,7 @@ def config_block(args, batch, world):
         "context_tokens": int(batch.context_lens.sum()),
         "kv_bytes_per_step": workloads.kv_bytes(batch),
         "unique_kv_bytes_per_step": workloads.unique_kv_bytes(batch),
-        "kv_dtype": "bf16",
+        "kv_dtype": batch.kv_dtype,
         "l2": "inputs larger than L2, and L2 flushed (memset 2x L2) between timed steps",
         "parallelism": "replicas: one independent batch per GPU" if world > 1 else "single GPU",
         "step": ("kv_cache_append + paged_attn_decode (two launches)" if args.two_launch else
@@ -450,8 +479,13 @@ def cpu_baseline(batch, kv, S, ctx_tokens, min_seconds=10.0, max_runs=5):
     n1 = int(max(1, min(S, int((per_seq.cumsum(0) < 2.0).sum()) or 1)))
     pairs = np.arange(n1 * host.num_q_heads, dtype=np.int64)
     t0 = time.perf_counter()
-    oracle.paged_decode(host.q, host.k_cache, host.v_cache, host.block_tables.numpy(), host.context_lens.numpy(),
-                        host.num_kv_heads, host.block_size, host.scale, pairs=pairs, num_threads=1)
+    if host.kv_dtype == "fp8":
+        oracle.paged_decode_fp8(host.q, host.k_cache, host.v_cache, host.k_scale, host.v_scale,
+                                host.block_tables.numpy(), host.context_lens.numpy(), host.num_kv_heads,
+                                host.block_size, host.scale, pairs=pairs, num_threads=1)
+    else:
+        oracle.paged_decode(host.q, host.k_cache, host.v_cache, host.block_tables.numpy(), host.context_lens.numpy(),
+                            host.num_kv_heads, host.block_size, host.scale, pairs=pairs, num_threads=1)
     t1 = time.perf_counter() - t0
     kv1 = int(host.context_lens[:n1].sum()) * host.num_kv_heads * host.head_dim * 2 * 2
     return {
@@ -464,6 +498,23 @@ def cpu_baseline(batch, kv, S, ctx_tokens, min_seconds=10.0, max_runs=5):
         "seq_per_s": round(S / t, 2),
         "single_thread": {"value": round(kv1 / t1 / 1e9, 4), "unit": "GB/s", "cores": 1,
                           "sample": f"decode of the first {n1} sequences (all heads), {t1:.2f} s"},
+    }
+
+
+def run_reference_prefill(args):
+    """The oracle's multi-query attention on a bounded sample of the workload."""
+    b = make_prefill_batch(args.workload, 0, "cpu")
+    sb = prefill_sample(b)
+    rate, sec = oracle_prefill_rate(sb, seconds_min=10.0)
+    return {
+        "metric": PREFILL_METRIC, "value": round(rate, 6), "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * sec, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "description": PREFILL_WORKLOADS[args.workload]["description"]},
+        "impl": "reference",
+        "cpu_baseline": {"value": round(rate, 6), "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+                         "sample": f"the last 16 queries of the first 2 sequences, median run {sec:.2f} s"},
+        "e2e": {"value": round(rate, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
 
@@ -528,6 +579,152 @@ def run_reference(args):
     }
 
 
+# ----------------------------------------------------------------------------- multi-query (prefill)
+
+def make_prefill_batch(name, rank, device):
+    w = PREFILL_WORKLOADS[name]
+    seed = rank_seed(11, rank)
+    ctx = w["ctx"](np.random.default_rng(seed))
+    Hq, Hkv = w["heads"]
+    return workloads.make_prefill(seed, w["chunks"], ctx, Hq, Hkv, w["head_dim"], w["block_size"], device=device,
+                                  poison=False)
+
+
+def prefill_sample(b, n_seqs=2, n_queries=16):
+    """The last n_queries queries of the first n_seqs sequences, as a smaller prefill batch."""
+    qs = b.query_start.numpy()
+    rows, chunks = [], []
+    for s in range(n_seqs):
+        n = min(n_queries, int(qs[s + 1] - qs[s]))
+        rows += list(range(int(qs[s + 1]) - n, int(qs[s + 1])))
+        chunks.append(n)
+    sub_qs = np.concatenate([[0], np.cumsum(chunks)]).astype(np.int32)
+    return workloads.PrefillBatch(**{**b.__dict__, "num_seqs": n_seqs, "q": b.q[rows].cpu(),
+                                     "context_lens": b.context_lens[:n_seqs], "block_tables": b.block_tables[:n_seqs],
+                                     "query_start": torch.from_numpy(sub_qs), "k_cache": b.k_cache.cpu(),
+                                     "v_cache": b.v_cache.cpu()})
+
+
+def oracle_prefill_rate(b, seconds_min=3.0):
+    import oracle
+    runs, t_all = [], time.perf_counter()
+    while len(runs) < 5 and time.perf_counter() - t_all < seconds_min:
+        t0 = time.perf_counter()
+        oracle.paged_prefill(b.q, b.k_cache, b.v_cache, b.block_tables.numpy(), b.context_lens.numpy(),
+                             b.query_start.numpy(), b.num_kv_heads, b.block_size, b.scale)
+        runs.append(time.perf_counter() - t0)
+    return workloads.prefill_flops(b) / statistics.median(runs) / 1e12, statistics.median(runs)
+
+
+def run_prefill(args, rank, world, local_rank):
+    import paged_kv_cache_377_b200 as pkv
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    b = make_prefill_batch(args.workload, rank, device)
+    flops = workloads.prefill_flops(b)
+    T = b.q.shape[0]
+    bt, cl, qs = b.block_tables.to(device), b.context_lens.to(device), b.query_start.to(device)
+    mq = int((b.query_start[1:] - b.query_start[:-1]).max())
+    out = torch.empty_like(b.q)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    stream = torch.cuda.current_stream(device)
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    flush = torch.empty(2 * l2, dtype=torch.uint8, device=device)
+
+    def step(q=b.q):
+        pkv.paged_attn_prefill(out, q, b.k_cache, b.v_cache, bt, cl, qs, mq, b.scale, status)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    sampler = ClockSampler(local_rank)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    with sampler:
+        for i in range(K):
+            flush.zero_()
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    ms = [x.elapsed_time(y) for x, y in ev]
+    if pkv.read_status(status):
+        raise RuntimeError("device status set after the timed steps")
+    (sum_flops,), (max_ms,) = aggregate([flops * K], [sum(ms)])
+    value = sum_flops / (max_ms / 1e3) / 1e12
+    mean_ms = statistics.fmean(ms)
+    peak = measured_tflops()
+
+    e2e = None
+    if not args.no_e2e:  # q copied in from pinned host memory and out read back, every step
+        q_host = b.q.cpu().pin_memory()
+        out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        q_dev = torch.empty_like(b.q)
+        for _ in range(max(args.warmup, 3)):
+            q_dev.copy_(q_host, non_blocking=True); step(q_dev); out_host.copy_(out, non_blocking=True)
+        torch.cuda.synchronize()
+        ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        for i in range(K):
+            flush.zero_()
+            ev2[i][0].record(stream)
+            q_dev.copy_(q_host, non_blocking=True)
+            step(q_dev)
+            out_host.copy_(out, non_blocking=True)
+            ev2[i][1].record(stream)
+        torch.cuda.synchronize()
+        (sf,), (mx,) = aggregate([flops * K], [sum(x.elapsed_time(y) for x, y in ev2)])
+        e2e = {"value": round(sf / (mx / 1e3) / 1e12, 2), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": q_host.numel() * 2 + 0, "d2h_bytes_per_step": out_host.numel() * 2,
+               "ms_per_step": round(mx / K, 4)}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        sb = prefill_sample(b)
+        rate, sec = oracle_prefill_rate(sb)
+        cpu = {"value": round(rate, 6), "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+               "sample": f"the last 16 queries of the first 2 sequences ({sb.q.shape[0]} query tokens), "
+                         f"median run {sec:.2f} s"}
+    w = PREFILL_WORKLOADS[args.workload]
+    return {
+        "metric": PREFILL_METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(max_ms / K, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16 (fp32 accumulate)",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "description": w["description"], "num_seqs": b.num_seqs,
+                   "query_tokens": T, "context_tokens": int(b.context_lens.sum()), "flops_per_step": flops,
+                   "l2": "L2 flushed (memset 2x L2) between timed steps",
+                   "parallelism": "replicas: one independent batch per GPU" if world > 1 else "single GPU"},
+        "roofline": {"kernel": "paged_prefill_kernel (one launch per step)", "bound": "tensor",
+                     "achieved": round(flops / (mean_ms / 1e3) / 1e12, 2), "peak": peak[0],
+                     "peak_kind": f"{peak[1]} bf16_tflops (cuBLAS burst)", "unit": "TFLOP/s",
+                     "frac": round(flops / (mean_ms / 1e3) / 1e12 / peak[0], 4),
+                     "algorithmic_flops_per_launch": flops, "traffic": None},
+        "clocks": sampler.summary(),
+        "gpu_launches": K,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+    }
+
+
+def measured_tflops():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    return 1590.0, "fallback"
+
+
 # ----------------------------------------------------------------------------- main
 
 def main(argv=None):
@@ -538,7 +735,10 @@ def main(argv=None):
     if args.impl == "reference":
         if rank != 0:
             return 0
-        print(json.dumps(run_reference(args)), flush=True)
+        if args.workload in PREFILL_WORKLOADS:
+            print(json.dumps(run_reference_prefill(args)), flush=True)
+        else:
+            print(json.dumps(run_reference(args)), flush=True)
         return 0
     if world > 1:
         import torch.distributed as dist
@@ -546,7 +746,10 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        result = run_ours(args, rank, world, local_rank)
+        if args.workload in PREFILL_WORKLOADS:
+            result = run_prefill(args, rank, world, local_rank)
+        else:
+            result = run_ours(args, rank, world, local_rank)
         if rank == 0:
             print(json.dumps(result), flush=True)
     finally:
