@@ -461,15 +461,24 @@ struct MmaMath {
                 keep_lo = (t < valid ? 0x0000ffffu : 0u) | (t + 1 < valid ? 0xffff0000u : 0u);
                 keep_hi = (t + 8 < valid ? 0x0000ffffu : 0u) | (t + 9 < valid ? 0xffff0000u : 0u);
             }
+            if (valid < BS) {  // the segment's last block only
 #pragma unroll
-            for (int dt = 0; dt < DT; ++dt) {
-                uint32_t a[4];
-                ldsm_x4_trans(a, tile_addr<BS>(vtile, 16 * ks + r + 8 * (mi >> 1), 2 * dt + (mi & 1)));
-                a[0] &= keep_lo;
-                a[1] &= keep_lo;
-                a[2] &= keep_hi;
-                a[3] &= keep_hi;
-                mma_16816(acc[dt], a, b0, b1);
+                for (int dt = 0; dt < DT; ++dt) {
+                    uint32_t a[4];
+                    ldsm_x4_trans(a, tile_addr<BS>(vtile, 16 * ks + r + 8 * (mi >> 1), 2 * dt + (mi & 1)));
+                    a[0] &= keep_lo;
+                    a[1] &= keep_lo;
+                    a[2] &= keep_hi;
+                    a[3] &= keep_hi;
+                    mma_16816(acc[dt], a, b0, b1);
+                }
+            } else {
+#pragma unroll
+                for (int dt = 0; dt < DT; ++dt) {
+                    uint32_t a[4];
+                    ldsm_x4_trans(a, tile_addr<BS>(vtile, 16 * ks + r + 8 * (mi >> 1), 2 * dt + (mi & 1)));
+                    mma_16816(acc[dt], a, b0, b1);
+                }
             }
         }
         __syncwarp();  // P scratch is rewritten by the next block
@@ -737,6 +746,8 @@ struct Fp8Math {
                 // head slice hs; with HP = 2 only the columns of head hs take it
                 const bool on = HP == 1 || my_half == hs;
                 const uint32_t c0 = on ? b0 : 0u, c1 = on ? b1 : 0u;
+                // the masks matter in the segment's last block only
+                const uint32_t klo = valid < BS ? keep_lo : 0xffffffffu, khi = valid < BS ? keep_hi : 0xffffffffu;
 #pragma unroll
                 for (int dp = 0; dp < DT / 2; ++dp) {
                     uint32_t x[4];
@@ -746,8 +757,14 @@ struct Fp8Math {
                         // x[2j]: tokens 0-7 of tile 2dp + j, x[2j + 1]: tokens 8-15; bytes
                         // (t, 2r) (t, 2r+1) (t+1, 2r) (t+1, 2r+1) -> (t, 2r) (t+1, 2r) | (t, 2r+1) (t+1, 2r+1)
                         const uint32_t lo = __byte_perm(x[2 * j], 0u, 0x3120), hi = __byte_perm(x[2 * j + 1], 0u, 0x3120);
-                        const uint32_t av[4] = {e4m3x2_to_f16x2(lo) & keep_lo, e4m3x2_to_f16x2(lo >> 16) & keep_lo,
-                                                e4m3x2_to_f16x2(hi) & keep_hi, e4m3x2_to_f16x2(hi >> 16) & keep_hi};
+                        uint32_t av[4] = {e4m3x2_to_f16x2(lo), e4m3x2_to_f16x2(lo >> 16), e4m3x2_to_f16x2(hi),
+                                          e4m3x2_to_f16x2(hi >> 16)};
+                        if (valid < BS) {
+                            av[0] &= klo;
+                            av[1] &= klo;
+                            av[2] &= khi;
+                            av[3] &= khi;
+                        }
                         mma_16816_f16(acc[2 * dp + j], av, c0, c1);
                     }
                 }
