@@ -188,6 +188,21 @@ int paged_attn_prefill(void *out, const void *q, const void *k_cache, const void
                        int32_t *d_status, void *stream);
 
 /*
+ * paged_attn_prefill with a choice of kernel: 0 = default (tcgen05 where it
+ * applies, else mma.sync), 1 = the mma.sync kernel, 2 = the tcgen05 kernel
+ * (PKV_ERR_UNSUPPORTED unless num_q_heads / num_kv_heads is 1, 2, 4 or 8).
+ * The tcgen05 kernel: a CTA per 128 rows of (query token, group head) of a
+ * sequence and kv head; S = Q K^T and O += P V on tcgen05.mma with fp32
+ * accumulators in tensor memory (P rounded to bf16), Q and the K/V blocks
+ * staged by TMA, one thread per query row for the causal online softmax.
+ */
+int paged_attn_prefill_ex(void *out, const void *q, const void *k_cache, const void *v_cache,
+                          const int32_t *block_tables, const int32_t *context_lens, const int32_t *query_start,
+                          int num_seqs, int num_tokens, int max_query_len, int num_q_heads, int num_kv_heads,
+                          int head_dim, int block_size, float scale, int max_blocks_per_seq, int num_blocks,
+                          int32_t *d_status, int kernel, void *stream);
+
+/*
  * FP8 KV cache. The pools hold e4m3 codes (1 sign, 4 exponent bits with bias
  * 7, 3 mantissa bits; 0x7f / 0xff are NaN), laid out like the bf16 pools,
  * [num_blocks][block_size][num_kv_heads][head_dim] bytes, with one fp32 scale

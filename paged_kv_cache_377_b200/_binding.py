@@ -83,6 +83,8 @@ def library() -> ctypes.CDLL:
             lib.kv_cache_append_fp8.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, P, P]
             lib.paged_attn_prefill.restype = I
             lib.paged_attn_prefill.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, I, I, P, P]
+            lib.paged_attn_prefill_ex.restype = I
+            lib.paged_attn_prefill_ex.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, I, I, P, I, P]
             lib.kv_cache_append.restype = I
             lib.kv_cache_append.argtypes = [P, P, P, P, P, I, I, I, I, I, P, P]
             lib.pkv_validate.restype = I
@@ -384,9 +386,11 @@ def kv_cache_append_fp8(k: torch.Tensor, v: torch.Tensor, k_cache: torch.Tensor,
 
 def paged_attn_prefill(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
                        block_tables: torch.Tensor, context_lens: torch.Tensor, query_start: torch.Tensor,
-                       max_query_len: int, scale: float, status: torch.Tensor, stream=None) -> torch.Tensor:
+                       max_query_len: int, scale: float, status: torch.Tensor, kernel: int = 0,
+                       stream=None) -> torch.Tensor:
     """Multi-query paged attention: q bf16 [T, Hq, D]; the queries of sequence s are rows
-    query_start[s] .. query_start[s+1]-1, the last tokens of its context, attending causally."""
+    query_start[s] .. query_start[s+1]-1, the last tokens of its context, attending causally.
+    kernel: 0 = default (tcgen05 where it applies), 1 = mma.sync, 2 = tcgen05."""
     _need(q, "q", torch.bfloat16, 3)
     _need(out, "out", torch.bfloat16, 3)
     _need(k_cache, "k_cache", torch.bfloat16, 4)
@@ -402,8 +406,8 @@ def paged_attn_prefill(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor
         raise ValueError("shape mismatch between q/out or k_cache/v_cache")
     if block_tables.shape[0] != S or query_start.shape[0] != S + 1:
         raise ValueError("block_tables needs num_seqs rows and query_start num_seqs + 1 entries")
-    _check("paged_attn_prefill", library().paged_attn_prefill(
+    _check("paged_attn_prefill", library().paged_attn_prefill_ex(
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens), _ptr(query_start),
         S, T, int(max_query_len), Hq, Hkv, D, bs, float(scale), block_tables.shape[1], NB, _ptr(status),
-        _stream(stream)))
+        int(kernel), _stream(stream)))
     return out

@@ -19,7 +19,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libpagedkv.so")
-SOURCES = ["api.cu", "decode.cu", "append.cu", "selftest.cu", "block_manager.cu", "prefill.cu"]
+SOURCES = ["api.cu", "decode.cu", "append.cu", "selftest.cu", "block_manager.cu", "prefill.cu", "prefill_tc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
                 "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]

@@ -81,6 +81,25 @@ int make_pool_map(CUtensorMap *map, const void *pool, int num_blocks, int bs, in
     return PKV_OK;
 }
 
+// Tensor map over the queries q [T][Hkv][G][D] bf16 seen as 5D (64, D/64, G,
+// Hkv, T): one box = one 64-column slice of 128 / G query tokens x G heads,
+// i.e. 128 rows (token, head) of 128 bytes, 128-byte swizzled.
+int make_query_map(CUtensorMap *map, const void *q, int num_tokens, int hkv, int group, int d) {
+    auto fn = encode_fn();
+    if (!fn) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    cuuint64_t dims[5] = {64, static_cast<cuuint64_t>(d / 64), static_cast<cuuint64_t>(group),
+                          static_cast<cuuint64_t>(hkv), static_cast<cuuint64_t>(num_tokens)};
+    cuuint64_t strides[4] = {128, static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(group) * d * 2,
+                             static_cast<cuuint64_t>(hkv) * group * d * 2};
+    cuuint32_t box[5] = {64, 1, static_cast<cuuint32_t>(group), 1, static_cast<cuuint32_t>(128 / group)};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(q), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled (queries) failed (%d)", static_cast<int>(r));
+    return PKV_OK;
+}
+
 // Launch epochs tag the per-segment piece counters, so a workspace never needs
 // clearing between calls (a counter from an older launch restarts at 1).
 unsigned long long next_epoch() {
@@ -380,6 +399,17 @@ int paged_attn_prefill(void *out, const void *q, const void *k_cache, const void
                        int num_seqs, int num_tokens, int max_query_len, int num_q_heads, int num_kv_heads,
                        int head_dim, int block_size, float scale, int max_blocks_per_seq, int num_blocks,
                        int32_t *d_status, void *stream) {
+    return paged_attn_prefill_ex(out, q, k_cache, v_cache, block_tables, context_lens, query_start, num_seqs,
+                                 num_tokens, max_query_len, num_q_heads, num_kv_heads, head_dim, block_size, scale,
+                                 max_blocks_per_seq, num_blocks, d_status, 0, stream);
+}
+
+int paged_attn_prefill_ex(void *out, const void *q, const void *k_cache, const void *v_cache,
+                          const int32_t *block_tables, const int32_t *context_lens, const int32_t *query_start,
+                          int num_seqs, int num_tokens, int max_query_len, int num_q_heads, int num_kv_heads,
+                          int head_dim, int block_size, float scale, int max_blocks_per_seq, int num_blocks,
+                          int32_t *d_status, int kernel, void *stream) {
+    if (kernel < 0 || kernel > 2) return fail(PKV_ERR_INVALID_ARGUMENT, "kernel must be 0, 1 or 2");
     if (num_seqs < 0 || num_tokens < 0 || max_query_len < 0)
         return fail(PKV_ERR_INVALID_ARGUMENT, "num_seqs, num_tokens and max_query_len must be >= 0");
     if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !query_start || !d_status)
@@ -408,13 +438,19 @@ int paged_attn_prefill(void *out, const void *q, const void *k_cache, const void
         return fail(PKV_ERR_INVALID_ARGUMENT, "num_tokens too large");
     if (!aligned(out, 16) || !aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(d_status, 4))
         return fail(PKV_ERR_INVALID_ARGUMENT, "out, q, k_cache and v_cache must be 16-byte aligned");
-    const size_t smem = pkv::prefill_smem_bytes(head_dim, block_size, max_blocks_per_seq);
+    // tcgen05 kernel: 128 rows must be whole query tokens (group 1, 2, 4, 8)
+    const size_t smem_tc = pkv::prefill_tc_smem_bytes(head_dim, max_blocks_per_seq);
+    const bool tc_ok = (group == 1 || group == 2 || group == 4 || group == 8) && smem_tc <= 227 * 1024;
+    if (kernel == 2 && !tc_ok)
+        return fail(PKV_ERR_UNSUPPORTED, "the tcgen05 kernel needs num_q_heads / num_kv_heads in {1, 2, 4, 8}");
+    const bool use_tc = kernel == 2 || (kernel == 0 && tc_ok);
+    const size_t smem = use_tc ? smem_tc : pkv::prefill_smem_bytes(head_dim, block_size, max_blocks_per_seq);
     if (smem > 227 * 1024)
         return fail(PKV_ERR_UNSUPPORTED, "max_blocks_per_seq %d needs %zu bytes of shared memory", max_blocks_per_seq,
                     smem);
     if (num_seqs == 0 || num_tokens == 0 || max_query_len == 0) return ok();
-    const int64_t tiles = (static_cast<int64_t>(max_query_len) * group + pkv::prefill_rows_per_cta() - 1) /
-                          pkv::prefill_rows_per_cta();
+    const int rows_per_cta = use_tc ? pkv::prefill_tc_rows_per_cta() : pkv::prefill_rows_per_cta();
+    const int64_t tiles = (static_cast<int64_t>(max_query_len) * group + rows_per_cta - 1) / rows_per_cta;
     if (tiles > 0x7fffffff) return fail(PKV_ERR_INVALID_ARGUMENT, "max_query_len too large");
     CUtensorMap tm_k, tm_v;
     int rc;
@@ -436,8 +472,16 @@ int paged_attn_prefill(void *out, const void *q, const void *k_cache, const void
     a.num_blocks = num_blocks;
     a.max_query_len = max_query_len;
     a.scale_log2 = scale * 1.4426950408889634f;
-    cudaError_t e = pkv::prefill_launch(head_dim, block_size, tm_k, tm_v, a, static_cast<int>(tiles), smem,
-                                        static_cast<cudaStream_t>(stream));
+    cudaError_t e;
+    if (use_tc) {
+        CUtensorMap tm_q;
+        if ((rc = make_query_map(&tm_q, q, num_tokens, num_kv_heads, group, head_dim)) != PKV_OK) return rc;
+        e = pkv::prefill_tc_launch(head_dim, block_size, tm_q, tm_k, tm_v, a, static_cast<int>(tiles), smem,
+                                   static_cast<cudaStream_t>(stream));
+    } else {
+        e = pkv::prefill_launch(head_dim, block_size, tm_k, tm_v, a, static_cast<int>(tiles), smem,
+                                static_cast<cudaStream_t>(stream));
+    }
     if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
     return ok();
 }

@@ -52,6 +52,12 @@ cudaError_t prefill_launch(int head_dim, int block_size, const CUtensorMap &tm_k
                            const PrefillArgs &args, int tiles, size_t smem_bytes, cudaStream_t stream);
 int prefill_rows_per_cta();
 
+size_t prefill_tc_smem_bytes(int head_dim, int max_blocks_per_seq);
+cudaError_t prefill_tc_launch(int head_dim, int block_size, const CUtensorMap &tm_q, const CUtensorMap &tm_k,
+                              const CUtensorMap &tm_v, const PrefillArgs &args, int tiles, size_t smem_bytes,
+                              cudaStream_t stream);
+int prefill_tc_rows_per_cta();
+
 cudaError_t append_fp8_launch(const void *k, const void *v, void *k_cache, void *v_cache, const int64_t *slot_mapping,
                               const float *k_scale, const float *v_scale, int num_tokens, int num_kv_heads,
                               int head_dim, int block_size, int num_blocks, int32_t *status, cudaStream_t stream);

@@ -15,13 +15,13 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def run(b, max_query_len=None):
+def run(b, max_query_len=None, kernel=0):
     qs = b.query_start
     mq = int((qs[1:] - qs[:-1]).max()) if max_query_len is None else max_query_len
     out = torch.full(b.q.shape, float("nan"), dtype=torch.bfloat16, device=DEV)
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
     pkv.paged_attn_prefill(out, b.q.to(DEV), b.k_cache.to(DEV), b.v_cache.to(DEV), b.block_tables.to(DEV),
-                           b.context_lens.to(DEV), qs.to(DEV), mq, b.scale, status)
+                           b.context_lens.to(DEV), qs.to(DEV), mq, b.scale, status, kernel=kernel)
     torch.cuda.synchronize()
     return out.cpu(), pkv.read_status(status)
 
@@ -31,15 +31,20 @@ def ref_of(b):
                                 b.query_start.numpy(), b.num_kv_heads, b.block_size, b.scale)
 
 
+@pytest.mark.parametrize("kernel", [1, 2])
 @pytest.mark.parametrize("G", [1, 2, 4, 7, 8])
 @pytest.mark.parametrize("D,bs", [(64, 16), (64, 32), (128, 16), (128, 32)])
-def test_mixed_batch_matches_oracle(G, D, bs):
+def test_mixed_batch_matches_oracle(G, D, bs, kernel):
     chunks = [1, 7, 16, 64, 130, 0, 1, 33]
     ctx = [1, 40, 16, 64, 700, 9, 1029, 33]
     b = workloads.make_prefill(3000 + 11 * G + D + bs, chunks, ctx, 2 * G, 2, D, bs)
-    out, st = run(b)
+    if kernel == 2 and G not in (1, 2, 4, 8):
+        with pytest.raises(pkv.PagedKVError, match="tcgen05"):
+            run(b, kernel=2)
+        return
+    out, st = run(b, kernel=kernel)
     assert st == 0
-    assert_close_to_oracle(out.double().numpy(), ref_of(b), what=f"prefill G={G} D={D} bs={bs}")
+    assert_close_to_oracle(out.double().numpy(), ref_of(b), what=f"prefill G={G} D={D} bs={bs} kernel={kernel}")
 
 
 def test_single_token_chunks_match_the_decode_kernel():
@@ -54,6 +59,15 @@ def test_single_token_chunks_match_the_decode_kernel():
     pkv.paged_attn_decode(dec, b.q.to(DEV), b.k_cache.to(DEV), b.v_cache.to(DEV), b.block_tables.to(DEV),
                           b.context_lens.to(DEV), b.scale, ws)
     assert_close_to_oracle(dec.double().cpu().numpy(), ref, what="decode kernel on the same rows")
+
+
+@pytest.mark.parametrize("kernel", [1, 2])
+def test_long_chunk_of_one_sequence(kernel):
+    """One 300-token chunk at the end of a 2000-token context: several 128-row tiles, many iterations."""
+    b = workloads.make_prefill(3150, [300, 4], [2000, 70], 16, 4, 128, 16)
+    out, st = run(b, kernel=kernel)
+    assert st == 0
+    assert_close_to_oracle(out.double().numpy(), ref_of(b), what=f"long chunk kernel={kernel}")
 
 
 def test_llama_shaped_chunked_prefill_sampled_rows():
