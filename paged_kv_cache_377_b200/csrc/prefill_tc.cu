@@ -3,21 +3,24 @@
 //
 // Same operation as prefill.cu (chunked prefill / mixed batches: query i of a
 // sequence's n-token chunk attends causally to positions 0 .. L - n + i).
-// One CTA per (128 rows of (query token, group head), sequence, kv head):
-//   - TMA loads the CTA's 128 query rows once (a 5D box over q viewed as
-//     [T][Hkv][G][D]) and streams the context through a 2-stage ring of 64
-//     tokens (64 / BS paged blocks) of K and V, 128-byte swizzled tiles;
-//   - one thread issues S = Q K^T (M 128, N 64, K = head_dim in steps of 16)
-//     into tensor memory and commits it to an mbarrier;
-//   - each of the 128 threads owns one query row (one tensor-memory lane):
-//     it loads its 64 logits, masks the positions its query may not see,
-//     updates its running maximum and sum, writes its row of P in bf16 to
-//     shared memory (the operand layout), and rescales its row of O in tensor
-//     memory when its maximum has grown by more than 2^8 since the last
-//     rescale (otherwise the stale maximum stays the reference: every P is
-//     then < 2^8 and the result is the same);
-//   - the thread issues O += P V (M 128, N = head_dim, K 64 tokens; V read as
-//     an N-major operand straight from its TMA tile) and commits it.
+// One CTA per (128 rows of (query token, group head), sequence, kv head), two
+// CTAs per SM, five warps:
+//   - warp 4 (one lane issues) loads the CTA's 128 query rows once by TMA (a
+//     5D box over q viewed as [T][Hkv][G][D]) and streams the context in
+//     iterations of 64 tokens (64 / BS paged blocks) through separate 2-stage
+//     rings of K and V (128-byte swizzled tiles); it issues S = Q K^T (M 128,
+//     N 64, K = head_dim in steps of 16) into one of two tensor-memory
+//     buffers, and O += P V (M 128, N = head_dim, K 64; P read from tensor
+//     memory, V as an N-major operand straight from its TMA tile). S of the
+//     next iteration runs on the tensor cores while the softmax of this one
+//     runs; a K stage is refilled as soon as its S is done, a V stage as soon
+//     as its P V is done;
+//   - warps 0-3: thread r owns query row r (tensor-memory lane r): it loads its
+//     64 logits, masks the positions its query may not see, updates its
+//     running maximum and sum, writes its row of P in bf16 over the S buffer,
+//     and rescales its row of O in tensor memory when its maximum has grown by
+//     more than 2^8 since the last rescale (otherwise the stale maximum stays
+//     the reference: every P is then < 2^8 and the result is the same).
 // All waits are bounded (1 s); a wait that gives up flags the status word,
 // the CTA drains what it issued and frees its tensor memory.
 #include <cuda_bf16.h>
@@ -28,11 +31,13 @@
 namespace pkv {
 namespace {
 
-constexpr int kTcThreads = 128;
-constexpr int kTcRows = 128;    // query rows per CTA (= tensor-memory lanes)
+constexpr int kSoftmaxThreads = 128;  // warps 0-3: one query row (tensor-memory lane) each
+constexpr int kTcThreads = 160;       // + warp 4: copies and MMAs
+constexpr int kTcRows = 128;          // query rows per CTA (= tensor-memory lanes)
 constexpr int kTcTokens = 64;   // context tokens per iteration
-// Tensor-memory columns: S takes 64, O head_dim; allocations are powers of two.
-__host__ __device__ constexpr uint32_t tmem_cols(int D) { return D == 64 ? 128u : 256u; }
+// Tensor-memory columns: two S / P buffers of 64 and O (head_dim); allocations
+// are powers of two, so both head sizes take 256 (two CTAs fill an SM's 512).
+__host__ __device__ constexpr uint32_t tmem_cols(int) { return 256u; }
 
 __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
     // UMMA shared-memory matrix descriptor: start, leading / stride byte offsets
@@ -110,8 +115,36 @@ __device__ __forceinline__ void tma_load_5d(void *dst, const CUtensorMap *map, u
         : "memory");
 }
 
+// 16 consecutive 32-bit columns of this thread's lane (warp-collective).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+    __syncwarp();
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+        "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+        : "memory");
+}
+
+// O += P V with P (A, M x K, K-major) in tensor memory.
+__device__ __forceinline__ void umma_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t db, uint32_t idesc,
+                                        uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %5, %5, %5}, p;\n\t}" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(db), "r"(idesc), "r"(accumulate), "r"(0u)
+        : "memory");
+}
+
+// A bounded wait whose outcome is the same for the whole warp (tensor-memory
+// loads and stores that follow are warp-collective).
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort, int32_t *status) {
+    const bool got = mbar_wait_bounded(bar, parity, abort, status);
+    return __all_sync(0xffffffffu, got);
+}
+
 template <int D, int BS>
-__global__ void __launch_bounds__(kTcThreads, 1)
+__global__ void __launch_bounds__(kTcThreads, 2)
     paged_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v, const PrefillArgs a) {
     static_assert(D == 64 || D == 128, "head_dim");
@@ -123,7 +156,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     constexpr int BPI = kTcTokens / BS;                   // paged blocks per iteration
 
     const int tile = blockIdx.x, s = blockIdx.y, h = blockIdx.z;
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     const int q0 = __ldg(a.query_start + s), q1 = __ldg(a.query_start + s + 1);
     const int n = q1 - q0;
@@ -140,258 +173,290 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int i0 = row0 / G;  // first query token of the tile
     const int last_query = (min(row0 + kTcRows, rows) - 1) / G;
     const int ntok = L - n + last_query + 1;              // positions 0 .. p of the last row
-    const int nit = (ntok + kTcTokens - 1) / kTcTokens;   // iterations of 64 tokens
+    const int nit = (ntok + kTcTokens - 1) / kTcTokens;   // iterations of 64 tokens (>= 1)
 
-    // ---- shared memory: Q | stage 0 K, V | stage 1 K, V | P | table | barriers
+    // ---- shared memory: Q | K stages 0, 1 | V stages 0, 1 | barriers | table
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sq = base;
-    uint8_t *skv = sq + HALVES * kQHalf;
-    uint8_t *sp = skv + 2 * 2 * kTileKV;
-    int *table = reinterpret_cast<int *>(sp + kTcRows * 128);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(table + ((a.max_blocks_per_seq + 3) & ~3));
-    uint64_t *q_full = bars, *kv_full = bars + 1, *s_full = bars + 3, *pv_done = bars + 4;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 6);
+    uint8_t *sk = sq + HALVES * kQHalf;   // [2][kTileKV]
+    uint8_t *sv = sk + 2 * kTileKV;       // [2][kTileKV]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sv + 2 * kTileKV);
+    uint64_t *q_full = bars, *k_full = bars + 1, *v_full = bars + 3, *s_full = bars + 5, *pv_done = bars + 7,
+             *p_ready = bars + 8;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 9);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    volatile int *stage_bad = abort_flag + 1;  // [2]
+    int *table = reinterpret_cast<int *>(bars + 10);
 
-    if (warp == 0) {
+    if (warp == 4) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                      "r"(tmem_cols(D)));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::);
         tc_fence_before();
-    }
-    if (tid == 32) {
-        mbar_init(q_full, 1);
-        mbar_init(&kv_full[0], 1);
-        mbar_init(&kv_full[1], 1);
-        mbar_init(s_full, 1);
-        mbar_init(pv_done, 1);
-        *abort_flag = 0;
-        stage_bad[0] = stage_bad[1] = 0;
-        fence_mbar_init();
-        tma_prefetch_desc(&tm_q);
-        tma_prefetch_desc(&tm_k);
-        tma_prefetch_desc(&tm_v);
+        if (lane == 0) {
+            mbar_init(q_full, 1);
+            for (int i = 0; i < 2; ++i) {
+                mbar_init(&k_full[i], 1);
+                mbar_init(&v_full[i], 1);
+                mbar_init(&s_full[i], 1);
+            }
+            mbar_init(pv_done, 1);
+            mbar_init(p_ready, kSoftmaxThreads);
+            *abort_flag = 0;
+            fence_mbar_init();
+            tma_prefetch_desc(&tm_q);
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+        }
     }
     for (int b = tid; b < nit * BPI && b < a.max_blocks_per_seq; b += kTcThreads)
         table[b] = __ldg(a.block_tables + static_cast<size_t>(s) * a.max_blocks_per_seq + b);
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *tmem_slot;
-    const uint32_t t_s = tbase, t_o = tbase + 64;  // S: columns 0-63, O: 64 .. 64 + D
+    // tensor memory: S / P buffers at columns 0 and 64, O at 128 .. 128 + D
+    const uint32_t t_o = tbase + 128;
 
-    // ---- producer: thread 0 issues every copy and MMA
-    uint32_t kv_issued = 0, kv_par = 0;  // stages with a K/V copy in flight, and its phase
-    int s_commits = 0, pv_commits = 0;    // MMA batches committed to s_full / pv_done
-    auto issue_kv = [&](int it) {
-        const int st = it & 1;
-        uint8_t *kdst = skv + st * 2 * kTileKV, *vdst = kdst + kTileKV;
-        int bad = 0;
-        uint32_t bytes = 0;
-        for (int j = 0; j < BPI; ++j) {
-            const int b = it * BPI + j;
-            if (b * BS >= ntok) break;
-            const int p = table[b];
-            if (p < 0 || p >= a.num_blocks) {
-                bad = 1;
-                continue;
-            }
-            bytes += 2u * HALVES * BS * 128;
-        }
-        stage_bad[st] = bad;
-        if (bad) atomicOr(a.status, PKV_STATUS_BAD_BLOCK_ID);
-        mbar_arrive_expect_tx(&kv_full[st], bytes);
-        for (int j = 0; j < BPI; ++j) {
-            const int b = it * BPI + j;
-            if (b * BS >= ntok) break;
-            const int p = table[b];
-            if (p < 0 || p >= a.num_blocks) continue;
+    if (warp == 4) {
+        // ---------------- producer: TMA copies and MMAs (lane 0 issues)
+        const bool leader = lane == 0;
+        int k_use0 = -1, k_use1 = -1, v_use0 = -1, v_use1 = -1;  // last use of each stage issued
+        uint64_t *last_commit = nullptr;
+        uint32_t last_commit_par = 0;
+        bool q_pending = false;
+        // copies of iteration it into stage it & 1 (K or V); a bad block id is
+        // flagged and its tile skipped
+        auto issue = [&](int it, bool is_v) {
+            const int st = it & 1;
+            uint64_t *bar = is_v ? &v_full[st] : &k_full[st];
+            uint8_t *dst = (is_v ? sv : sk) + st * kTileKV;
+            const CUtensorMap *map = is_v ? &tm_v : &tm_k;
+            if (leader) {
+                uint32_t bytes = 0;
+                for (int j = 0; j < BPI; ++j) {
+                    const int b = it * BPI + j;
+                    if (b * BS >= ntok) break;
+                    const int p = table[b];
+                    if (p < 0 || p >= a.num_blocks) {
+                        if (!is_v) atomicOr(a.status, PKV_STATUS_BAD_BLOCK_ID);
+                        continue;
+                    }
+                    bytes += HALVES * BS * 128;
+                }
+                mbar_arrive_expect_tx(bar, bytes);
+                for (int j = 0; j < BPI; ++j) {
+                    const int b = it * BPI + j;
+                    if (b * BS >= ntok) break;
+                    const int p = table[b];
+                    if (p < 0 || p >= a.num_blocks) continue;
 #pragma unroll
-            for (int hf = 0; hf < HALVES; ++hf) {
-                tma_load_4d(kdst + hf * kHalfKV + j * BS * 128, &tm_k, &kv_full[st], 0, hf, h, p * BS);
-                tma_load_4d(vdst + hf * kHalfKV + j * BS * 128, &tm_v, &kv_full[st], 0, hf, h, p * BS);
+                    for (int hf = 0; hf < HALVES; ++hf)
+                        tma_load_4d(dst + hf * kHalfKV + j * BS * 128, map, bar, 0, hf, h, p * BS);
+                }
             }
-        }
-        kv_issued |= 1u << st;
-        kv_par = (kv_par & ~(1u << st)) | ((static_cast<uint32_t>(it >> 1) & 1u) << st);
-    };
-    if (tid == 0) {
-        mbar_arrive_expect_tx(q_full, HALVES * kQHalf);
-#pragma unroll
-        for (int hf = 0; hf < HALVES; ++hf)
-            tma_load_5d(sq + hf * kQHalf, &tm_q, q_full, 0, hf, 0, h, q0 + i0);
-        issue_kv(0);
-        if (nit > 1) issue_kv(1);
-    }
-
-    // ---- this thread's query row
-    const int r = tid;                                  // tensor-memory lane / row of the tile
-    const int row = row0 + r;
-    const bool live = row < rows;
-    const int qi = min(row, rows - 1) / G;              // query token of the row
-    const int p_row = L - n + qi;                       // last position it may see
-    const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
-    float m_ref = -INFINITY, l_run = 0.f;
-    bool ok = mbar_wait_bounded(q_full, 0, abort_flag, a.status);
-    uint32_t s_par = 0, pv_par = 0;
-
-    for (int it = 0; it < nit; ++it) {
-        const int st = it & 1;
-        const uint32_t kbase = smem_u32(skv + st * 2 * kTileKV), vbase = kbase + kTileKV;
-        // S = Q K^T (thread 0), once this stage has landed
-        if (tid == 0 && ok && !*abort_flag) {
-            if (mbar_wait_bounded(&kv_full[st], (kv_par >> st) & 1u, abort_flag, a.status)) {
-                kv_issued &= ~(1u << st);
-                tc_fence_after();
+            int &use = is_v ? (st ? v_use1 : v_use0) : (st ? k_use1 : k_use0);
+            use = it >> 1;
+        };
+        auto issue_s = [&](int it) {  // S(it) = Q K(it)^T into buffer it & 1
+            const int b = it & 1;
+            if (leader) {
+                const uint32_t kb = smem_u32(sk + b * kTileKV);
 #pragma unroll
                 for (int hf = 0; hf < HALVES; ++hf)
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        umma(t_s, smem_desc(smem_u32(sq) + hf * kQHalf + kk * 32, 16, 1024),
-                             smem_desc(kbase + hf * kHalfKV + kk * 32, 16, 1024), instr_desc(128, 64, false),
+                        umma(tbase + 64 * b, smem_desc(smem_u32(sq) + hf * kQHalf + kk * 32, 16, 1024),
+                             smem_desc(kb + hf * kHalfKV + kk * 32, 16, 1024), instr_desc(128, 64, false),
                              (hf | kk) != 0);
-                umma_commit(s_full);
-                ++s_commits;
+                umma_commit(&s_full[b]);
             }
-        }
-        ok = ok && mbar_wait_bounded(s_full, s_par, abort_flag, a.status);
-        s_par ^= 1u;
-        tc_fence_after();
-        // softmax over this row's 64 logits
-        float x[64];
-        {
-            float t0[32], t1[32];
-            tmem_ld32(t_s + lane_addr, t0);
-            tmem_ld32(t_s + lane_addr + 32, t1);
+            last_commit = &s_full[b];
+            last_commit_par = static_cast<uint32_t>(it >> 1) & 1u;
+        };
+        if (leader) {
+            mbar_arrive_expect_tx(q_full, HALVES * kQHalf);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                x[i] = t0[i];
-                x[32 + i] = t1[i];
-            }
+            for (int hf = 0; hf < HALVES; ++hf)
+                tma_load_5d(sq + hf * kQHalf, &tm_q, q_full, 0, hf, 0, h, q0 + i0);
         }
-        float mx = -INFINITY;
-#pragma unroll
-        for (int t = 0; t < 64; ++t) {
-            const int pos = it * kTcTokens + t;
-            x[t] = pos <= p_row ? x[t] * a.scale_log2 : -INFINITY;
-            mx = fmaxf(mx, x[t]);
+        q_pending = true;
+        issue(0, false);
+        issue(0, true);
+        if (nit > 1) {
+            issue(1, false);
+            issue(1, true);
         }
-        // the reference maximum moves only when it would be exceeded by more than 2^8
-        float m_new = m_ref;
-        if (mx > m_ref + 8.f) m_new = mx;
-        const float alpha = fast_exp2(m_ref - m_new);  // 0 on the first update
-        // O += P V of the previous iteration must be done before O is rescaled or P rewritten
-        if (it > 0) {
-            ok = ok && mbar_wait_bounded(pv_done, pv_par, abort_flag, a.status);
-            pv_par ^= 1u;
+        bool ok = warp_wait(q_full, 0, abort_flag, a.status);
+        if (ok) q_pending = false;
+        ok = ok && warp_wait(&k_full[0], 0, abort_flag, a.status);
+        if (ok) {
             tc_fence_after();
-            // this row's O in tensor memory times alpha; tcgen05.ld / st are
-            // warp-collective, so the whole warp takes the branch together
-            if (__any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll
-                for (int cb = 0; cb < D / 32; ++cb) {
-                    float o[32];
-                    tmem_ld32(t_o + lane_addr + cb * 32, o);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) o[i] *= alpha;
-                    tmem_st32(t_o + lane_addr + cb * 32, o);
+            issue_s(0);
+        }
+        for (int it = 0; ok && it < nit; ++it) {
+            const int b = it & 1, nb = b ^ 1;
+            if (it + 1 < nit) {
+                // S(it + 1) into the other buffer, which held P(it - 1)
+                if (!(ok = warp_wait(&k_full[nb], static_cast<uint32_t>((it + 1) >> 1) & 1u, abort_flag, a.status)))
+                    break;
+                if (it >= 1 && !(ok = warp_wait(pv_done, static_cast<uint32_t>(it - 1) & 1u, abort_flag, a.status)))
+                    break;
+                tc_fence_after();
+                issue_s(it + 1);
+                // V stage nb is free once O += P(it - 1) V(it - 1) is done
+                if (it >= 1) issue(it + 1, true);
+                // K stage b is free once S(it) is done
+                if (it + 2 < nit) {
+                    if (!(ok = warp_wait(&s_full[b], static_cast<uint32_t>(it >> 1) & 1u, abort_flag, a.status)))
+                        break;
+                    issue(it + 2, false);
                 }
             }
-        }
-        // P in bf16, written in the 128-byte swizzled operand layout (row r, 8 chunks)
-        float ps = 0.f;
-        uint8_t *prow = sp + r * 128;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            uint32_t w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const __nv_bfloat162 v2 =
-                    __floats2bfloat162_rn(fast_exp2(x[8 * c + 2 * e] - m_new), fast_exp2(x[8 * c + 2 * e + 1] - m_new));
-                ps += __low2float(v2) + __high2float(v2);
-                w[e] = *reinterpret_cast<const uint32_t *>(&v2);
-            }
-            *reinterpret_cast<uint4 *>(prow + ((c ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-        l_run = l_run * alpha + ps;
-        m_ref = m_new;
-        // V rows past the tile's last position (past the context, or in blocks
-        // not loaded) may hold anything: zero them so that P = 0 there
-        // multiplies zeros
-        if (it == nit - 1 && ok) {
-            const int valid = ntok - it * kTcTokens;  // tokens of this iteration the tile may see
-            for (int e = tid; e < HALVES * kTcTokens * 8; e += kTcThreads) {
-                const int hf = e / (kTcTokens * 8), t = (e / 8) % kTcTokens, c = e % 8;
-                if (t >= valid)
-                    *reinterpret_cast<uint4 *>(skv + st * 2 * kTileKV + kTileKV + hf * kHalfKV + t * 128 +
-                                               ((c ^ (t & 7)) << 4)) = make_uint4(0u, 0u, 0u, 0u);
-            }
-        }
-        fence_proxy_async_shared();  // P and the zeroed V rows, before the MMA reads them
-        tc_fence_before();
-        __syncthreads();
-        // O += P V (thread 0), then refill this stage two iterations ahead
-        if (tid == 0 && ok && !*abort_flag) {
+            // O += P(it) V(it), once the softmax warps have written P(it)
+            if (!(ok = warp_wait(&v_full[b], static_cast<uint32_t>(it >> 1) & 1u, abort_flag, a.status))) break;
+            if (!(ok = warp_wait(p_ready, static_cast<uint32_t>(it) & 1u, abort_flag, a.status))) break;
             tc_fence_after();
-            if (!stage_bad[st]) {
+            if (leader) {
+                const uint32_t vb = smem_u32(sv + b * kTileKV);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    umma(t_o, smem_desc(smem_u32(sp) + kk * 32, 16, 1024),
-                         smem_desc(vbase + kk * 16 * 128, kHalfKV, 1024), instr_desc(128, D, true),
-                         (it | kk) != 0);
+                    umma_ts(t_o, tbase + 64 * b + kk * 8, smem_desc(vb + kk * 16 * 128, kHalfKV, 1024),
+                            instr_desc(128, D, true), (it | kk) != 0);
+                umma_commit(pv_done);
             }
-            umma_commit(pv_done);
-            ++pv_commits;
-            if (it + 2 < nit) {
-                // the stage is free once this MMA has read it
-                if (mbar_wait_bounded(pv_done, pv_par, abort_flag, a.status)) issue_kv(it + 2);
-            }
+            last_commit = pv_done;
+            last_commit_par = static_cast<uint32_t>(it) & 1u;
+            __syncwarp();
         }
-    }
-    // the last O += P V
-    if (nit > 0) {
-        ok = ok && mbar_wait_bounded(pv_done, pv_par, abort_flag, a.status);
-        tc_fence_after();
-    }
-    // drain copies and MMAs still in flight (only after a wait gave up): a
-    // commit's arrival covers every MMA the thread issued before it
-    if (tid == 0) {
-        for (int st = 0; st < 2; ++st)
-            if ((kv_issued >> st) & 1u) mbar_wait_drain(&kv_full[st], (kv_par >> st) & 1u, a.status);
-        if (s_commits > 0) mbar_wait_drain(s_full, static_cast<uint32_t>(s_commits - 1) & 1u, a.status);
-        if (pv_commits > 0) mbar_wait_drain(pv_done, static_cast<uint32_t>(pv_commits - 1) & 1u, a.status);
-    }
-
-    // ---- normalise and store this row (every lane reads its lane of O: the
-    // tensor-memory load is warp-collective; only real rows are stored)
-    const bool store = ok && !*abort_flag && live;
-    const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-    __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(a.out) +
-                         (static_cast<size_t>(q0 + qi) * a.num_q_heads + h * G + min(row, rows - 1) % G) * D;
+        // drain what is still in flight (only after a wait gave up): copies, and
+        // the MMAs (a commit's arrival covers every MMA issued before it)
+        if (q_pending) mbar_wait_drain(q_full, 0, a.status);
+        if (k_use0 >= 0) mbar_wait_drain(&k_full[0], static_cast<uint32_t>(k_use0) & 1u, a.status);
+        if (k_use1 >= 0) mbar_wait_drain(&k_full[1], static_cast<uint32_t>(k_use1) & 1u, a.status);
+        if (v_use0 >= 0) mbar_wait_drain(&v_full[0], static_cast<uint32_t>(v_use0) & 1u, a.status);
+        if (v_use1 >= 0) mbar_wait_drain(&v_full[1], static_cast<uint32_t>(v_use1) & 1u, a.status);
+        if (last_commit) mbar_wait_drain(last_commit, last_commit_par, a.status);
+        __syncwarp();
+    } else {
+        // ---------------- softmax warps: thread r owns query row r (tensor-memory lane r)
+        const int r = tid;
+        const int row = row0 + r;
+        const bool live = row < rows;
+        const int qi = min(row, rows - 1) / G;              // query token of the row
+        const int p_row = L - n + qi;                       // last position it may see
+        const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+        float m_ref = -INFINITY, l_run = 0.f;
+        bool ok = true;
+        for (int it = 0; it < nit; ++it) {
+            const int b = it & 1;
+            const uint32_t t_s = tbase + 64 * b + lane_addr;
+            if (!(ok = warp_wait(&s_full[b], static_cast<uint32_t>(it >> 1) & 1u, abort_flag, a.status))) break;
+            tc_fence_after();
+            float x[64];
+            {
+                float t0[32];
+                tmem_ld32(t_s, t0);
 #pragma unroll
-    for (int cb = 0; cb < D / 32; ++cb) {
-        float o[32];
-        tmem_ld32(t_o + lane_addr + cb * 32, o);
-        if (store) {
+                for (int i = 0; i < 32; ++i) x[i] = t0[i];
+                tmem_ld32(t_s + 32, t0);
 #pragma unroll
-            for (int i = 0; i < 32; i += 8) {
-                uint4 v;
-                const __nv_bfloat162 a0 = __floats2bfloat162_rn(o[i] * inv, o[i + 1] * inv);
-                const __nv_bfloat162 a1 = __floats2bfloat162_rn(o[i + 2] * inv, o[i + 3] * inv);
-                const __nv_bfloat162 a2 = __floats2bfloat162_rn(o[i + 4] * inv, o[i + 5] * inv);
-                const __nv_bfloat162 a3 = __floats2bfloat162_rn(o[i + 6] * inv, o[i + 7] * inv);
-                v.x = *reinterpret_cast<const uint32_t *>(&a0);
-                v.y = *reinterpret_cast<const uint32_t *>(&a1);
-                v.z = *reinterpret_cast<const uint32_t *>(&a2);
-                v.w = *reinterpret_cast<const uint32_t *>(&a3);
-                *reinterpret_cast<uint4 *>(dst + cb * 32 + i) = v;
+                for (int i = 0; i < 32; ++i) x[32 + i] = t0[i];
+            }
+            float mx = -INFINITY;
+#pragma unroll
+            for (int t = 0; t < 64; ++t) {
+                const int pos = it * kTcTokens + t;
+                x[t] = pos <= p_row ? x[t] * a.scale_log2 : -INFINITY;
+                mx = fmaxf(mx, x[t]);
+            }
+            // the reference maximum moves only when it would be exceeded by more than 2^8
+            float m_new = m_ref;
+            if (mx > m_ref + 8.f) m_new = mx;
+            const float alpha = fast_exp2(m_ref - m_new);  // 0 on the first update
+            // P in bf16 over this buffer's first 32 columns (two values per column)
+            float ps = 0.f;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t w[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const int t = 32 * half + 2 * e;
+                    const __nv_bfloat162 v2 = __floats2bfloat162_rn(fast_exp2(x[t] - m_new), fast_exp2(x[t + 1] - m_new));
+                    ps += __low2float(v2) + __high2float(v2);
+                    w[e] = *reinterpret_cast<const uint32_t *>(&v2);
+                }
+                tmem_st16(t_s + 16 * half, w);
+            }
+            asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+            l_run = l_run * alpha + ps;
+            m_ref = m_new;
+            // O += P(it - 1) V(it - 1) must be done before O is rescaled
+            if (it > 0) {
+                if (!(ok = warp_wait(pv_done, static_cast<uint32_t>(it - 1) & 1u, abort_flag, a.status))) break;
+                tc_fence_after();
+                if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+                    for (int cb = 0; cb < D / 32; ++cb) {
+                        float o[32];
+                        tmem_ld32(t_o + lane_addr + cb * 32, o);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) o[i] *= alpha;
+                        tmem_st32(t_o + lane_addr + cb * 32, o);
+                    }
+                }
+            }
+            // V rows past the tile's last position (past the context, or in
+            // blocks not loaded) may hold anything: zero them so that P = 0
+            // there multiplies zeros
+            if (it == nit - 1) {
+                if (!(ok = warp_wait(&v_full[b], static_cast<uint32_t>(it >> 1) & 1u, abort_flag, a.status))) break;
+                const int valid = ntok - it * kTcTokens;
+                uint8_t *vt = sv + b * kTileKV;
+                for (int e = tid; e < HALVES * kTcTokens * 8; e += kSoftmaxThreads) {
+                    const int hf = e / (kTcTokens * 8), t = (e / 8) % kTcTokens, c = e % 8;
+                    if (t >= valid)
+                        *reinterpret_cast<uint4 *>(vt + hf * kHalfKV + t * 128 + ((c ^ (t & 7)) << 4)) =
+                            make_uint4(0u, 0u, 0u, 0u);
+                }
+                fence_proxy_async_shared();
+            }
+            tc_fence_before();
+            mbar_arrive(p_ready);
+        }
+        if (ok) {
+            ok = warp_wait(pv_done, static_cast<uint32_t>(nit - 1) & 1u, abort_flag, a.status);
+            tc_fence_after();
+        }
+        // normalise and store this row (every lane reads its lane of O: the
+        // tensor-memory load is warp-collective; only real rows are stored)
+        const bool store = ok && !*abort_flag && live;
+        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+        __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(a.out) +
+                             (static_cast<size_t>(q0 + qi) * a.num_q_heads + h * G + min(row, rows - 1) % G) * D;
+#pragma unroll
+        for (int cb = 0; cb < D / 32; ++cb) {
+            float o[32];
+            tmem_ld32(t_o + lane_addr + cb * 32, o);
+            if (store) {
+#pragma unroll
+                for (int i = 0; i < 32; i += 8) {
+                    uint4 v;
+                    const __nv_bfloat162 a0 = __floats2bfloat162_rn(o[i] * inv, o[i + 1] * inv);
+                    const __nv_bfloat162 a1 = __floats2bfloat162_rn(o[i + 2] * inv, o[i + 3] * inv);
+                    const __nv_bfloat162 a2 = __floats2bfloat162_rn(o[i + 4] * inv, o[i + 5] * inv);
+                    const __nv_bfloat162 a3 = __floats2bfloat162_rn(o[i + 6] * inv, o[i + 7] * inv);
+                    v.x = *reinterpret_cast<const uint32_t *>(&a0);
+                    v.y = *reinterpret_cast<const uint32_t *>(&a1);
+                    v.z = *reinterpret_cast<const uint32_t *>(&a2);
+                    v.w = *reinterpret_cast<const uint32_t *>(&a3);
+                    *reinterpret_cast<uint4 *>(dst + cb * 32 + i) = v;
+                }
             }
         }
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) {
+    if (warp == 4) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tbase), "r"(tmem_cols(D)));
     }
@@ -411,8 +476,10 @@ PrefillTcFn pick_tc(int D, int BS) {
 
 size_t prefill_tc_smem_bytes(int head_dim, int max_blocks_per_seq) {
     const size_t halves = head_dim / 64;
-    return halves * kTcRows * 128 + 2 * 2 * halves * kTcTokens * 128 + kTcRows * 128 +
-           static_cast<size_t>((max_blocks_per_seq + 3) & ~3) * 4 + 6 * 8 + 32 + 1024;
+    const size_t bytes = halves * kTcRows * 128 + 2 * 2 * halves * kTcTokens * 128 + 10 * 8 +
+                         static_cast<size_t>(max_blocks_per_seq) * 4 + 1024;
+    // at most two CTAs per SM: their tensor memory (256 columns each) fills the SM's 512
+    return bytes < 80 * 1024 ? 80 * 1024 : bytes;
 }
 
 cudaError_t prefill_tc_launch(int head_dim, int block_size, const CUtensorMap &tm_q, const CUtensorMap &tm_k,
