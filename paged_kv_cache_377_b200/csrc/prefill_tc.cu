@@ -32,7 +32,8 @@ namespace pkv {
 namespace {
 
 constexpr int kSoftmaxThreads = 128;  // warps 0-3: one query row (tensor-memory lane) each
-constexpr int kTcThreads = 160;       // + warp 4: copies and MMAs
+constexpr int kTcThreads = 192;       // + warp 4: TMA copies, warp 5: MMAs
+constexpr int kTcBarriers = 15;
 constexpr int kTcRows = 128;          // query rows per CTA (= tensor-memory lanes)
 constexpr int kTcTokens = 64;   // context tokens per iteration
 // Tensor-memory columns: two S / P buffers of 64 and O (head_dim); allocations
@@ -182,32 +183,41 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     uint8_t *sk = sq + HALVES * kQHalf;   // [2][kTileKV]
     uint8_t *sv = sk + 2 * kTileKV;       // [2][kTileKV]
     uint64_t *bars = reinterpret_cast<uint64_t *>(sv + 2 * kTileKV);
-    uint64_t *q_full = bars, *k_full = bars + 1, *v_full = bars + 3, *s_full = bars + 5, *pv_done = bars + 7,
-             *p_ready = bars + 8;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 9);
+    // p_ready has one barrier per S / P buffer: a softmax warp that needs no
+    // rescale may run one iteration ahead of the others, never two (S(it + 2)
+    // waits for P(it) V(it)). For the same reason pv_done may be two phases
+    // behind a warp that has finished its loop: the final O is signalled on a
+    // barrier of its own, o_full. k_free / v_free tell the load warp that the
+    // MMA reading a stage is done (one commit per use, so the load warp, which
+    // waits for every use in turn, is never two phases behind).
+    uint64_t *q_full = bars, *k_full = bars + 1, *v_full = bars + 3, *k_free = bars + 5, *v_free = bars + 7,
+             *s_full = bars + 9, *p_ready = bars + 11, *pv_done = bars + 13, *o_full = bars + 14;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kTcBarriers);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    int *table = reinterpret_cast<int *>(bars + 10);
+    int *table = reinterpret_cast<int *>(bars + kTcBarriers + 1);
 
-    if (warp == 4) {
+    if (warp == 5) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                      "r"(tmem_cols(D)));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::);
         tc_fence_before();
-        if (lane == 0) {
-            mbar_init(q_full, 1);
-            for (int i = 0; i < 2; ++i) {
-                mbar_init(&k_full[i], 1);
-                mbar_init(&v_full[i], 1);
-                mbar_init(&s_full[i], 1);
-            }
-            mbar_init(pv_done, 1);
-            mbar_init(p_ready, kSoftmaxThreads);
-            *abort_flag = 0;
-            fence_mbar_init();
-            tma_prefetch_desc(&tm_q);
-            tma_prefetch_desc(&tm_k);
-            tma_prefetch_desc(&tm_v);
+    } else if (warp == 4 && lane == 0) {
+        mbar_init(q_full, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&k_full[i], 1);
+            mbar_init(&v_full[i], 1);
+            mbar_init(&k_free[i], 1);
+            mbar_init(&v_free[i], 1);
+            mbar_init(&s_full[i], 1);
+            mbar_init(&p_ready[i], kSoftmaxThreads);
         }
+        mbar_init(pv_done, 1);
+        mbar_init(o_full, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
     }
     for (int b = tid; b < nit * BPI && b < a.max_blocks_per_seq; b += kTcThreads)
         table[b] = __ldg(a.block_tables + static_cast<size_t>(s) * a.max_blocks_per_seq + b);
@@ -218,45 +228,63 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     const uint32_t t_o = tbase + 128;
 
     if (warp == 4) {
-        // ---------------- producer: TMA copies and MMAs (lane 0 issues)
-        const bool leader = lane == 0;
+        // ---------------- load warp: every TMA copy; lane j copies one
+        // 128-byte column slice of one paged block
         int k_use0 = -1, k_use1 = -1, v_use0 = -1, v_use1 = -1;  // last use of each stage issued
-        uint64_t *last_commit = nullptr;
-        uint32_t last_commit_par = 0;
-        bool q_pending = false;
-        // copies of iteration it into stage it & 1 (K or V); a bad block id is
-        // flagged and its tile skipped
+        const int jb = lane / HALVES, hf = lane % HALVES;
         auto issue = [&](int it, bool is_v) {
             const int st = it & 1;
             uint64_t *bar = is_v ? &v_full[st] : &k_full[st];
-            uint8_t *dst = (is_v ? sv : sk) + st * kTileKV;
-            const CUtensorMap *map = is_v ? &tm_v : &tm_k;
-            if (leader) {
-                uint32_t bytes = 0;
-                for (int j = 0; j < BPI; ++j) {
-                    const int b = it * BPI + j;
-                    if (b * BS >= ntok) break;
-                    const int p = table[b];
-                    if (p < 0 || p >= a.num_blocks) {
-                        if (!is_v) atomicOr(a.status, PKV_STATUS_BAD_BLOCK_ID);
-                        continue;
-                    }
-                    bytes += HALVES * BS * 128;
-                }
-                mbar_arrive_expect_tx(bar, bytes);
-                for (int j = 0; j < BPI; ++j) {
-                    const int b = it * BPI + j;
-                    if (b * BS >= ntok) break;
-                    const int p = table[b];
-                    if (p < 0 || p >= a.num_blocks) continue;
-#pragma unroll
-                    for (int hf = 0; hf < HALVES; ++hf)
-                        tma_load_4d(dst + hf * kHalfKV + j * BS * 128, map, bar, 0, hf, h, p * BS);
+            const int b = it * BPI + jb;
+            bool mine = lane < BPI * HALVES && b * BS < ntok;
+            int p = 0;
+            if (mine) {
+                p = table[b];
+                if (p < 0 || p >= a.num_blocks) {
+                    if (!is_v && hf == 0) atomicOr(a.status, PKV_STATUS_BAD_BLOCK_ID);
+                    mine = false;
                 }
             }
+            const unsigned m = __ballot_sync(0xffffffffu, mine);
+            if (lane == 0) mbar_arrive_expect_tx(bar, static_cast<uint32_t>(__popc(m)) * BS * 128u);
+            __syncwarp();
+            if (mine)
+                tma_load_4d((is_v ? sv : sk) + st * kTileKV + hf * kHalfKV + jb * BS * 128, is_v ? &tm_v : &tm_k, bar,
+                            0, hf, h, p * BS);
             int &use = is_v ? (st ? v_use1 : v_use0) : (st ? k_use1 : k_use0);
             use = it >> 1;
         };
+        if (lane == 0) {
+            mbar_arrive_expect_tx(q_full, HALVES * kQHalf);
+#pragma unroll
+            for (int q = 0; q < HALVES; ++q) tma_load_5d(sq + q * kQHalf, &tm_q, q_full, 0, q, 0, h, q0 + i0);
+        }
+        issue(0, false);
+        if (nit > 1) issue(1, false);
+        issue(0, true);
+        if (nit > 1) issue(1, true);
+        bool ok = true;
+        for (int it = 0; it + 2 < nit; ++it) {
+            // stage it & 1 is free once S(it) (K) or P(it) V(it) (V) is done
+            const uint32_t par = static_cast<uint32_t>(it >> 1) & 1u;
+            if (!(ok = warp_wait(&k_free[it & 1], par, abort_flag, a.status))) break;
+            issue(it + 2, false);
+            if (!(ok = warp_wait(&v_free[it & 1], par, abort_flag, a.status))) break;
+            issue(it + 2, true);
+        }
+        // copies still in flight (only after a wait gave up) land before exit
+        if (!ok || *abort_flag) {
+            mbar_wait_drain(q_full, 0, a.status);
+            if (k_use0 >= 0) mbar_wait_drain(&k_full[0], static_cast<uint32_t>(k_use0) & 1u, a.status);
+            if (k_use1 >= 0) mbar_wait_drain(&k_full[1], static_cast<uint32_t>(k_use1) & 1u, a.status);
+            if (v_use0 >= 0) mbar_wait_drain(&v_full[0], static_cast<uint32_t>(v_use0) & 1u, a.status);
+            if (v_use1 >= 0) mbar_wait_drain(&v_full[1], static_cast<uint32_t>(v_use1) & 1u, a.status);
+        }
+        __syncwarp();
+    } else if (warp == 5) {
+        // ---------------- MMA warp (lane 0 issues)
+        const bool leader = lane == 0;
+        bool o_committed = false;  // o_full committed (after the last P V, or by the drain)
         auto issue_s = [&](int it) {  // S(it) = Q K(it)^T into buffer it & 1
             const int b = it & 1;
             if (leader) {
@@ -269,25 +297,10 @@ __global__ void __launch_bounds__(kTcThreads, 2)
                              smem_desc(kb + hf * kHalfKV + kk * 32, 16, 1024), instr_desc(128, 64, false),
                              (hf | kk) != 0);
                 umma_commit(&s_full[b]);
+                umma_commit(&k_free[b]);
             }
-            last_commit = &s_full[b];
-            last_commit_par = static_cast<uint32_t>(it >> 1) & 1u;
         };
-        if (leader) {
-            mbar_arrive_expect_tx(q_full, HALVES * kQHalf);
-#pragma unroll
-            for (int hf = 0; hf < HALVES; ++hf)
-                tma_load_5d(sq + hf * kQHalf, &tm_q, q_full, 0, hf, 0, h, q0 + i0);
-        }
-        q_pending = true;
-        issue(0, false);
-        issue(0, true);
-        if (nit > 1) {
-            issue(1, false);
-            issue(1, true);
-        }
         bool ok = warp_wait(q_full, 0, abort_flag, a.status);
-        if (ok) q_pending = false;
         ok = ok && warp_wait(&k_full[0], 0, abort_flag, a.status);
         if (ok) {
             tc_fence_after();
@@ -303,18 +316,10 @@ __global__ void __launch_bounds__(kTcThreads, 2)
                     break;
                 tc_fence_after();
                 issue_s(it + 1);
-                // V stage nb is free once O += P(it - 1) V(it - 1) is done
-                if (it >= 1) issue(it + 1, true);
-                // K stage b is free once S(it) is done
-                if (it + 2 < nit) {
-                    if (!(ok = warp_wait(&s_full[b], static_cast<uint32_t>(it >> 1) & 1u, abort_flag, a.status)))
-                        break;
-                    issue(it + 2, false);
-                }
             }
             // O += P(it) V(it), once the softmax warps have written P(it)
             if (!(ok = warp_wait(&v_full[b], static_cast<uint32_t>(it >> 1) & 1u, abort_flag, a.status))) break;
-            if (!(ok = warp_wait(p_ready, static_cast<uint32_t>(it) & 1u, abort_flag, a.status))) break;
+            if (!(ok = warp_wait(&p_ready[b], static_cast<uint32_t>(it >> 1) & 1u, abort_flag, a.status))) break;
             tc_fence_after();
             if (leader) {
                 const uint32_t vb = smem_u32(sv + b * kTileKV);
@@ -323,19 +328,18 @@ __global__ void __launch_bounds__(kTcThreads, 2)
                     umma_ts(t_o, tbase + 64 * b + kk * 8, smem_desc(vb + kk * 16 * 128, kHalfKV, 1024),
                             instr_desc(128, D, true), (it | kk) != 0);
                 umma_commit(pv_done);
+                umma_commit(&v_free[b]);
+                if (it == nit - 1) umma_commit(o_full);
             }
-            last_commit = pv_done;
-            last_commit_par = static_cast<uint32_t>(it) & 1u;
+            if (it == nit - 1) o_committed = true;
             __syncwarp();
         }
-        // drain what is still in flight (only after a wait gave up): copies, and
-        // the MMAs (a commit's arrival covers every MMA issued before it)
-        if (q_pending) mbar_wait_drain(q_full, 0, a.status);
-        if (k_use0 >= 0) mbar_wait_drain(&k_full[0], static_cast<uint32_t>(k_use0) & 1u, a.status);
-        if (k_use1 >= 0) mbar_wait_drain(&k_full[1], static_cast<uint32_t>(k_use1) & 1u, a.status);
-        if (v_use0 >= 0) mbar_wait_drain(&v_full[0], static_cast<uint32_t>(v_use0) & 1u, a.status);
-        if (v_use1 >= 0) mbar_wait_drain(&v_full[1], static_cast<uint32_t>(v_use1) & 1u, a.status);
-        if (last_commit) mbar_wait_drain(last_commit, last_commit_par, a.status);
+        // MMAs still in flight (only after a wait gave up) finish before the
+        // tensor memory is freed: a commit's arrival covers every MMA issued
+        // before it, and o_full has a single phase, so its wait cannot alias
+        if (!o_committed && leader) umma_commit(o_full);
+        __syncwarp();
+        mbar_wait_drain(o_full, 0, a.status);
         __syncwarp();
     } else {
         // ---------------- softmax warps: thread r owns query row r (tensor-memory lane r)
@@ -390,19 +394,20 @@ __global__ void __launch_bounds__(kTcThreads, 2)
             asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
             l_run = l_run * alpha + ps;
             m_ref = m_new;
-            // O += P(it - 1) V(it - 1) must be done before O is rescaled
-            if (it > 0) {
+            // a warp whose maximum moved rescales its rows of O, once
+            // O += P(it - 1) V(it - 1) is done; otherwise it does not wait: the
+            // MMAs issued by one thread run in order, so P(it) V(it) may be
+            // issued behind P(it - 1) V(it - 1) straight away
+            if (it > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
                 if (!(ok = warp_wait(pv_done, static_cast<uint32_t>(it - 1) & 1u, abort_flag, a.status))) break;
                 tc_fence_after();
-                if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-                    for (int cb = 0; cb < D / 32; ++cb) {
-                        float o[32];
-                        tmem_ld32(t_o + lane_addr + cb * 32, o);
+                for (int cb = 0; cb < D / 32; ++cb) {
+                    float o[32];
+                    tmem_ld32(t_o + lane_addr + cb * 32, o);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) o[i] *= alpha;
-                        tmem_st32(t_o + lane_addr + cb * 32, o);
-                    }
+                    for (int i = 0; i < 32; ++i) o[i] *= alpha;
+                    tmem_st32(t_o + lane_addr + cb * 32, o);
                 }
             }
             // V rows past the tile's last position (past the context, or in
@@ -421,10 +426,10 @@ __global__ void __launch_bounds__(kTcThreads, 2)
                 fence_proxy_async_shared();
             }
             tc_fence_before();
-            mbar_arrive(p_ready);
+            mbar_arrive(&p_ready[b]);
         }
         if (ok) {
-            ok = warp_wait(pv_done, static_cast<uint32_t>(nit - 1) & 1u, abort_flag, a.status);
+            ok = warp_wait(o_full, 0, abort_flag, a.status);
             tc_fence_after();
         }
         // normalise and store this row (every lane reads its lane of O: the
@@ -456,7 +461,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 4) {
+    if (warp == 5) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tbase), "r"(tmem_cols(D)));
     }
@@ -476,7 +481,7 @@ PrefillTcFn pick_tc(int D, int BS) {
 
 size_t prefill_tc_smem_bytes(int head_dim, int max_blocks_per_seq) {
     const size_t halves = head_dim / 64;
-    const size_t bytes = halves * kTcRows * 128 + 2 * 2 * halves * kTcTokens * 128 + 10 * 8 +
+    const size_t bytes = halves * kTcRows * 128 + 2 * 2 * halves * kTcTokens * 128 + (kTcBarriers + 1) * 8 +
                          static_cast<size_t>(max_blocks_per_seq) * 4 + 1024;
     // at most two CTAs per SM: their tensor memory (256 columns each) fills the SM's 512
     return bytes < 80 * 1024 ? 80 * 1024 : bytes;
