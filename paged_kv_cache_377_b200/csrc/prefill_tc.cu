@@ -33,7 +33,7 @@ namespace {
 
 constexpr int kSoftmaxThreads = 128;  // warps 0-3: one query row (tensor-memory lane) each
 constexpr int kTcThreads = 192;       // + warp 4: TMA copies, warp 5: MMAs
-constexpr int kTcBarriers = 15;
+constexpr int kTcBarriers = 12;
 constexpr int kTcRows = 128;          // query rows per CTA (= tensor-memory lanes)
 constexpr int kTcTokens = 64;   // context tokens per iteration
 // Tensor-memory columns: two S / P buffers of 64 and O (head_dim); allocations
@@ -183,15 +183,17 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     uint8_t *sk = sq + HALVES * kQHalf;   // [2][kTileKV]
     uint8_t *sv = sk + 2 * kTileKV;       // [2][kTileKV]
     uint64_t *bars = reinterpret_cast<uint64_t *>(sv + 2 * kTileKV);
-    // p_ready has one barrier per S / P buffer: a softmax warp that needs no
-    // rescale may run one iteration ahead of the others, never two (S(it + 2)
-    // waits for P(it) V(it)). For the same reason pv_done may be two phases
-    // behind a warp that has finished its loop: the final O is signalled on a
-    // barrier of its own, o_full. k_free / v_free tell the load warp that the
-    // MMA reading a stage is done (one commit per use, so the load warp, which
-    // waits for every use in turn, is never two phases behind).
-    uint64_t *q_full = bars, *k_full = bars + 1, *v_full = bars + 3, *k_free = bars + 5, *v_free = bars + 7,
-             *s_full = bars + 9, *p_ready = bars + 11, *pv_done = bars + 13, *o_full = bars + 14;
+    // Barriers, each with one phase per use of its stage or buffer b = it & 1:
+    //   s_full[b]  S(it) is in tensor memory (and K stage b may be refilled);
+    //   p_ready[b] the 128 softmax threads wrote P(it) over it;
+    //   pv_free[b] O += P(it) V(it) is done (V stage b may be refilled, S / P
+    //              buffer b may take S(it + 2), O may be rescaled).
+    // A softmax warp that needs no rescale may run one iteration ahead of the
+    // others, never two (S(it + 2) waits for P(it) V(it)), so no wait on these
+    // is two phases behind or ahead of its barrier. A warp that has finished
+    // its loop may be: the final O is signalled on a barrier of its own, o_full.
+    uint64_t *q_full = bars, *k_full = bars + 1, *v_full = bars + 3, *s_full = bars + 5, *p_ready = bars + 7,
+             *pv_free = bars + 9, *o_full = bars + 11;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kTcBarriers);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     int *table = reinterpret_cast<int *>(bars + kTcBarriers + 1);
@@ -206,12 +208,10 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         for (int i = 0; i < 2; ++i) {
             mbar_init(&k_full[i], 1);
             mbar_init(&v_full[i], 1);
-            mbar_init(&k_free[i], 1);
-            mbar_init(&v_free[i], 1);
+            mbar_init(&pv_free[i], 1);
             mbar_init(&s_full[i], 1);
             mbar_init(&p_ready[i], kSoftmaxThreads);
         }
-        mbar_init(pv_done, 1);
         mbar_init(o_full, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -267,9 +267,9 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         for (int it = 0; it + 2 < nit; ++it) {
             // stage it & 1 is free once S(it) (K) or P(it) V(it) (V) is done
             const uint32_t par = static_cast<uint32_t>(it >> 1) & 1u;
-            if (!(ok = warp_wait(&k_free[it & 1], par, abort_flag, a.status))) break;
+            if (!(ok = warp_wait(&s_full[it & 1], par, abort_flag, a.status))) break;
             issue(it + 2, false);
-            if (!(ok = warp_wait(&v_free[it & 1], par, abort_flag, a.status))) break;
+            if (!(ok = warp_wait(&pv_free[it & 1], par, abort_flag, a.status))) break;
             issue(it + 2, true);
         }
         // copies still in flight (only after a wait gave up) land before exit
@@ -285,19 +285,22 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         // ---------------- MMA warp (lane 0 issues)
         const bool leader = lane == 0;
         bool o_committed = false;  // o_full committed (after the last P V, or by the drain)
+        // descriptors of stage / buffer 0; the start address (16-byte units)
+        // is the low field, so an offset is added to the descriptor itself
+        const uint64_t dq = smem_desc(smem_u32(sq), 16, 1024);
+        const uint64_t dk = smem_desc(smem_u32(sk), 16, 1024);
+        const uint64_t dv = smem_desc(smem_u32(sv), kHalfKV, 1024);
         auto issue_s = [&](int it) {  // S(it) = Q K(it)^T into buffer it & 1
             const int b = it & 1;
             if (leader) {
-                const uint32_t kb = smem_u32(sk + b * kTileKV);
+                const uint64_t dkb = dk + ((b * kTileKV) >> 4);
 #pragma unroll
                 for (int hf = 0; hf < HALVES; ++hf)
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        umma(tbase + 64 * b, smem_desc(smem_u32(sq) + hf * kQHalf + kk * 32, 16, 1024),
-                             smem_desc(kb + hf * kHalfKV + kk * 32, 16, 1024), instr_desc(128, 64, false),
-                             (hf | kk) != 0);
+                        umma(tbase + 64 * b, dq + ((hf * kQHalf + kk * 32) >> 4), dkb + ((hf * kHalfKV + kk * 32) >> 4),
+                             instr_desc(128, 64, false), (hf | kk) != 0);
                 umma_commit(&s_full[b]);
-                umma_commit(&k_free[b]);
             }
         };
         bool ok = warp_wait(q_full, 0, abort_flag, a.status);
@@ -312,7 +315,8 @@ __global__ void __launch_bounds__(kTcThreads, 2)
                 // S(it + 1) into the other buffer, which held P(it - 1)
                 if (!(ok = warp_wait(&k_full[nb], static_cast<uint32_t>((it + 1) >> 1) & 1u, abort_flag, a.status)))
                     break;
-                if (it >= 1 && !(ok = warp_wait(pv_done, static_cast<uint32_t>(it - 1) & 1u, abort_flag, a.status)))
+                if (it >= 1 &&
+                    !(ok = warp_wait(&pv_free[nb], static_cast<uint32_t>((it - 1) >> 1) & 1u, abort_flag, a.status)))
                     break;
                 tc_fence_after();
                 issue_s(it + 1);
@@ -322,17 +326,15 @@ __global__ void __launch_bounds__(kTcThreads, 2)
             if (!(ok = warp_wait(&p_ready[b], static_cast<uint32_t>(it >> 1) & 1u, abort_flag, a.status))) break;
             tc_fence_after();
             if (leader) {
-                const uint32_t vb = smem_u32(sv + b * kTileKV);
+                const uint64_t dvb = dv + ((b * kTileKV) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    umma_ts(t_o, tbase + 64 * b + kk * 8, smem_desc(vb + kk * 16 * 128, kHalfKV, 1024),
-                            instr_desc(128, D, true), (it | kk) != 0);
-                umma_commit(pv_done);
-                umma_commit(&v_free[b]);
+                    umma_ts(t_o, tbase + 64 * b + kk * 8, dvb + ((kk * 16 * 128) >> 4), instr_desc(128, D, true),
+                            (it | kk) != 0);
+                umma_commit(&pv_free[b]);
                 if (it == nit - 1) umma_commit(o_full);
             }
             if (it == nit - 1) o_committed = true;
-            __syncwarp();
         }
         // MMAs still in flight (only after a wait gave up) finish before the
         // tensor memory is freed: a commit's arrival covers every MMA issued
@@ -366,31 +368,53 @@ __global__ void __launch_bounds__(kTcThreads, 2)
 #pragma unroll
                 for (int i = 0; i < 32; ++i) x[32 + i] = t0[i];
             }
-            float mx = -INFINITY;
+            // x c with c < 0 is (-x)(-c): work with a positive factor
+            if (a.scale_log2 < 0.f) {
 #pragma unroll
-            for (int t = 0; t < 64; ++t) {
-                const int pos = it * kTcTokens + t;
-                x[t] = pos <= p_row ? x[t] * a.scale_log2 : -INFINITY;
-                mx = fmaxf(mx, x[t]);
+                for (int t = 0; t < 64; ++t) x[t] = -x[t];
             }
-            // the reference maximum moves only when it would be exceeded by more than 2^8
+            // positions past this row's last one exist only near the end
+            if (it * kTcTokens + kTcTokens - 1 > p_row) {
+#pragma unroll
+                for (int t = 0; t < 64; ++t)
+                    if (it * kTcTokens + t > p_row) x[t] = -INFINITY;
+            }
+            // maximum of the logits (before the positive factor), as a tree
+            float mx;
+            {
+                float m4[4] = {x[0], x[1], x[2], x[3]};
+#pragma unroll
+                for (int t = 4; t < 64; t += 4) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) m4[e] = fmaxf(m4[e], x[t + e]);
+                }
+                mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+            }
+            // log2-domain maximum; the reference moves only when it would be
+            // exceeded by more than 2^8
+            const float c = fabsf(a.scale_log2);
             float m_new = m_ref;
-            if (mx > m_ref + 8.f) m_new = mx;
+            if (mx * c > m_ref + 8.f) m_new = mx * c;
             const float alpha = fast_exp2(m_ref - m_new);  // 0 on the first update
-            // P in bf16 over this buffer's first 32 columns (two values per column)
-            float ps = 0.f;
+            const float neg_m = -m_new;
+            // P = 2^(x c - m) in bf16 over this buffer's first 32 columns (two
+            // values per column); the row sum takes the fp32 values
+            float ps0 = 0.f, ps1 = 0.f;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t w[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
                     const int t = 32 * half + 2 * e;
-                    const __nv_bfloat162 v2 = __floats2bfloat162_rn(fast_exp2(x[t] - m_new), fast_exp2(x[t + 1] - m_new));
-                    ps += __low2float(v2) + __high2float(v2);
+                    const float p0 = fast_exp2(fmaf(x[t], c, neg_m)), p1 = fast_exp2(fmaf(x[t + 1], c, neg_m));
+                    ps0 += p0;
+                    ps1 += p1;
+                    const __nv_bfloat162 v2 = __floats2bfloat162_rn(p0, p1);
                     w[e] = *reinterpret_cast<const uint32_t *>(&v2);
                 }
                 tmem_st16(t_s + 16 * half, w);
             }
+            const float ps = ps0 + ps1;
             asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
             l_run = l_run * alpha + ps;
             m_ref = m_new;
@@ -399,7 +423,8 @@ __global__ void __launch_bounds__(kTcThreads, 2)
             // MMAs issued by one thread run in order, so P(it) V(it) may be
             // issued behind P(it - 1) V(it - 1) straight away
             if (it > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-                if (!(ok = warp_wait(pv_done, static_cast<uint32_t>(it - 1) & 1u, abort_flag, a.status))) break;
+                if (!(ok = warp_wait(&pv_free[b ^ 1], static_cast<uint32_t>((it - 1) >> 1) & 1u, abort_flag, a.status)))
+                    break;
                 tc_fence_after();
 #pragma unroll
                 for (int cb = 0; cb < D / 32; ++cb) {

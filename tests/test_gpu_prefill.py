@@ -70,6 +70,17 @@ def test_long_chunk_of_one_sequence(kernel):
     assert_close_to_oracle(out.double().numpy(), ref_of(b), what=f"long chunk kernel={kernel}")
 
 
+@pytest.mark.parametrize("kernel", [1, 2])
+@pytest.mark.parametrize("scale", [-0.2, 0.01, 1.5])
+def test_scales_of_either_sign_and_size(kernel, scale):
+    """A negative scale flips which logit is largest; a large one makes the running
+    maximum move often (rescales of O in tensor memory)."""
+    b = workloads.make_prefill(3160, [200, 9], [900, 300], 8, 2, 128, 16, scale=scale)
+    out, st = run(b, kernel=kernel)
+    assert st == 0
+    assert_close_to_oracle(out.double().numpy(), ref_of(b), what=f"scale {scale} kernel={kernel}")
+
+
 def test_llama_shaped_chunked_prefill_sampled_rows():
     rng = np.random.default_rng(31)
     chunks = [512, 256, 384, 128, 1, 1, 1, 1]
