@@ -87,6 +87,30 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// 64 consecutive fp32 columns of this thread's lane in one load and one wait
+// (warp-collective).
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
+    __syncwarp();
+    uint32_t r[64];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// One lane of the warp (the same one every time), chosen by elect.sync.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
     __syncwarp();
     asm volatile(
@@ -282,8 +306,9 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         }
         __syncwarp();
     } else if (warp == 5) {
-        // ---------------- MMA warp (lane 0 issues)
-        const bool leader = lane == 0;
+        // ---------------- MMA warp (one elected lane issues; the operands are
+        // computed by the whole warp, outside the branch)
+        const bool leader = elect_one();
         bool o_committed = false;  // o_full committed (after the last P V, or by the drain)
         // descriptors of stage / buffer 0; the start address (16-byte units)
         // is the low field, so an offset is added to the descriptor itself
@@ -292,13 +317,14 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         const uint64_t dv = smem_desc(smem_u32(sv), kHalfKV, 1024);
         auto issue_s = [&](int it) {  // S(it) = Q K(it)^T into buffer it & 1
             const int b = it & 1;
+            const uint64_t dkb = dk + ((b * kTileKV) >> 4);
+            const uint32_t ts = tbase + 64 * b;
             if (leader) {
-                const uint64_t dkb = dk + ((b * kTileKV) >> 4);
 #pragma unroll
                 for (int hf = 0; hf < HALVES; ++hf)
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        umma(tbase + 64 * b, dq + ((hf * kQHalf + kk * 32) >> 4), dkb + ((hf * kHalfKV + kk * 32) >> 4),
+                        umma(ts, dq + ((hf * kQHalf + kk * 32) >> 4), dkb + ((hf * kHalfKV + kk * 32) >> 4),
                              instr_desc(128, 64, false), (hf | kk) != 0);
                 umma_commit(&s_full[b]);
             }
@@ -325,12 +351,12 @@ __global__ void __launch_bounds__(kTcThreads, 2)
             if (!(ok = warp_wait(&v_full[b], static_cast<uint32_t>(it >> 1) & 1u, abort_flag, a.status))) break;
             if (!(ok = warp_wait(&p_ready[b], static_cast<uint32_t>(it >> 1) & 1u, abort_flag, a.status))) break;
             tc_fence_after();
+            const uint64_t dvb = dv + ((b * kTileKV) >> 4);
+            const uint32_t tp = tbase + 64 * b;
             if (leader) {
-                const uint64_t dvb = dv + ((b * kTileKV) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    umma_ts(t_o, tbase + 64 * b + kk * 8, dvb + ((kk * 16 * 128) >> 4), instr_desc(128, D, true),
-                            (it | kk) != 0);
+                    umma_ts(t_o, tp + kk * 8, dvb + ((kk * 16 * 128) >> 4), instr_desc(128, D, true), (it | kk) != 0);
                 umma_commit(&pv_free[b]);
                 if (it == nit - 1) umma_commit(o_full);
             }
@@ -359,15 +385,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
             if (!(ok = warp_wait(&s_full[b], static_cast<uint32_t>(it >> 1) & 1u, abort_flag, a.status))) break;
             tc_fence_after();
             float x[64];
-            {
-                float t0[32];
-                tmem_ld32(t_s, t0);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) x[i] = t0[i];
-                tmem_ld32(t_s + 32, t0);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) x[32 + i] = t0[i];
-            }
+            tmem_ld64(t_s, x);
             // x c with c < 0 is (-x)(-c): work with a positive factor
             if (a.scale_log2 < 0.f) {
 #pragma unroll
