@@ -102,6 +102,18 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
     for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// Non-blocking test of an mbarrier phase (mbarrier.try_wait may suspend the
+// thread for a while; this does not).
+__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // One lane of the warp (the same one every time), chosen by elect.sync.
 __device__ __forceinline__ bool elect_one() {
     uint32_t pred;
@@ -287,14 +299,45 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         if (nit > 1) issue(1, false);
         issue(0, true);
         if (nit > 1) issue(1, true);
+        // K(it) once S(it - 2) is done (its stage is free), V(it) once
+        // P(it - 2) V(it - 2) is done, each as soon as it may: both are polled,
+        // so that neither waits behind the other; bounded like every wait
         bool ok = true;
-        for (int it = 0; it + 2 < nit; ++it) {
-            // stage it & 1 is free once S(it) (K) or P(it) V(it) (V) is done
-            const uint32_t par = static_cast<uint32_t>(it >> 1) & 1u;
-            if (!(ok = warp_wait(&s_full[it & 1], par, abort_flag, a.status))) break;
-            issue(it + 2, false);
-            if (!(ok = warp_wait(&pv_free[it & 1], par, abort_flag, a.status))) break;
-            issue(it + 2, true);
+        int nk = 2, nv = 2;
+        uint64_t t_prog = 0;  // start of the current stretch without progress
+        for (uint32_t spin = 1; nk < nit || nv < nit; ++spin) {
+            bool moved = false;
+            if (nk < nit &&
+                __all_sync(0xffffffffu, mbar_test(&s_full[nk & 1], static_cast<uint32_t>((nk - 2) >> 1) & 1u))) {
+                issue(nk++, false);
+                moved = true;
+            }
+            if (nv < nit &&
+                __all_sync(0xffffffffu, mbar_test(&pv_free[nv & 1], static_cast<uint32_t>((nv - 2) >> 1) & 1u))) {
+                issue(nv++, true);
+                moved = true;
+            }
+            if (moved) {
+                t_prog = 0;
+                continue;
+            }
+            if (__any_sync(0xffffffffu, *abort_flag != 0)) {
+                ok = false;
+                break;
+            }
+            __nanosleep(32);  // leave the issue slots to the softmax warps
+            if ((spin & 15u) == 0) {
+                const uint64_t now = globaltimer_ns();
+                if (t_prog == 0) t_prog = now;
+                if (now - t_prog > kWaitLimitNs) {
+                    if (lane == 0) {
+                        *abort_flag = 1;
+                        atomicOr(a.status, PKV_STATUS_WAIT_TIMEOUT);
+                    }
+                    ok = false;
+                    break;
+                }
+            }
         }
         // copies still in flight (only after a wait gave up) land before exit
         if (!ok || *abort_flag) {
