@@ -81,6 +81,8 @@ def parse_args(argv=None):
                    help="L2 flush (memset of 2x L2) between timed steps: auto = only when the step's K/V "
                         "is under 4x L2 (larger inputs leave nothing in L2 for the next step)")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--prefill-kernel", type=int, default=0, choices=[0, 1, 2],
+                   help="multi-query kernel: 0 default (tcgen05 where it applies), 1 mma.sync, 2 tcgen05")
     return p.parse_args(argv)
 
 
@@ -129,6 +131,28 @@ def decode_sources_sha():
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
+
+
+def prefill_sources_sha():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "paged_kv_cache_377_b200", "csrc")
+    for name in ("prefill_tc.cu", "device_utils.cuh"):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_prefill_traffic(workload: str):
+    """DRAM bytes per tcgen05 prefill launch from a committed ncu capture, if it was
+    taken on the current kernel sources (else None)."""
+    path = os.path.join(PROFILES, "prefill_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        e = json.load(f).get(workload)
+    if not e or e.get("prefill_sources_sha") != prefill_sources_sha():
+        return None
+    return e.get("dram_bytes_per_launch")
 
 
 def profiled_traffic(workload: str):
@@ -669,7 +693,8 @@ def run_prefill(args, rank, world, local_rank):
     flush = torch.empty(2 * l2, dtype=torch.uint8, device=device)
 
     def step(q=b.q):
-        pkv.paged_attn_prefill(out, q, b.k_cache, b.v_cache, bt, cl, qs, mq, b.scale, status)
+        pkv.paged_attn_prefill(out, q, b.k_cache, b.v_cache, bt, cl, qs, mq, b.scale, status,
+                               kernel=args.prefill_kernel)
 
     for _ in range(args.warmup):
         step()
@@ -742,11 +767,14 @@ def run_prefill(args, rank, world, local_rank):
                    "query_tokens": T, "context_tokens": int(b.context_lens.sum()), "flops_per_step": flops,
                    "l2": "L2 flushed (memset 2x L2) between timed steps",
                    "parallelism": "replicas: one independent batch per GPU" if world > 1 else "single GPU"},
-        "roofline": {"kernel": "paged_prefill_kernel (one launch per step)", "bound": "tensor",
+        "roofline": {"kernel": ("paged_prefill_kernel (mma.sync" if args.prefill_kernel == 1 else
+                               "paged_prefill_tc_kernel (tcgen05") + "; one launch per step)", "bound": "tensor",
                      "achieved": round(flops / (mean_ms / 1e3) / 1e12, 2), "peak": peak[0],
                      "peak_kind": f"{peak[1]} bf16_tflops (cuBLAS burst)", "unit": "TFLOP/s",
                      "frac": round(flops / (mean_ms / 1e3) / 1e12 / peak[0], 4),
-                     "algorithmic_flops_per_launch": flops, "traffic": None},
+                     "algorithmic_flops_per_launch": flops,
+                     "traffic": profiled_prefill_traffic(args.workload) if args.prefill_kernel != 1 else None,
+                     "traffic_unit": "DRAM bytes per launch (ncu)"},
         "clocks": sampler.summary(),
         "gpu_launches": K,
         "e2e": e2e,
