@@ -114,6 +114,26 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Largest of three (sm_100 three-input max.f32).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// Packed fp32 add of both halves (sm_100 f32x2).
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\t"
+        "mov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
 // One lane of the warp (the same one every time), chosen by elect.sync.
 __device__ __forceinline__ bool elect_one() {
     uint32_t pred;
@@ -440,16 +460,19 @@ __global__ void __launch_bounds__(kTcThreads, 2)
                 for (int t = 0; t < 64; ++t)
                     if (it * kTcTokens + t > p_row) x[t] = -INFINITY;
             }
-            // maximum of the logits (before the positive factor), as a tree
+            // maximum of the logits (before the positive factor): three-input
+            // max, four independent chains
             float mx;
             {
                 float m4[4] = {x[0], x[1], x[2], x[3]};
 #pragma unroll
-                for (int t = 4; t < 64; t += 4) {
+                for (int t = 4; t < 60; t += 8) {  // x[4 .. 59]
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) m4[e] = fmaxf(m4[e], x[t + e]);
+                    for (int e = 0; e < 4; ++e) m4[e] = fmax3(m4[e], x[t + e], x[t + 4 + e]);
                 }
-                mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+#pragma unroll
+                for (int e = 0; e < 4; ++e) m4[e] = fmaxf(m4[e], x[60 + e]);  // x[60 .. 63]
+                mx = fmax3(fmaxf(m4[0], m4[1]), m4[2], m4[3]);
             }
             // log2-domain maximum; the reference moves only when it would be
             // exceeded by more than 2^8
@@ -457,24 +480,28 @@ __global__ void __launch_bounds__(kTcThreads, 2)
             float m_new = m_ref;
             if (mx * c > m_ref + 8.f) m_new = mx * c;
             const float alpha = fast_exp2(m_ref - m_new);  // 0 on the first update
-            const float neg_m = -m_new;
             // P = 2^(x c - m) in bf16 over this buffer's first 32 columns (two
-            // values per column); the row sum takes the fp32 values
-            float ps0 = 0.f, ps1 = 0.f;
+            // values per column); x c - m and the fp32 row sum on packed pairs
+            const float2 cc = make_float2(c, c), nm = make_float2(-m_new, -m_new);
+            float2 ps2a = make_float2(0.f, 0.f), ps2b = make_float2(0.f, 0.f);
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t w[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
                     const int t = 32 * half + 2 * e;
-                    const float p0 = fast_exp2(fmaf(x[t], c, neg_m)), p1 = fast_exp2(fmaf(x[t + 1], c, neg_m));
-                    ps0 += p0;
-                    ps1 += p1;
-                    const __nv_bfloat162 v2 = __floats2bfloat162_rn(p0, p1);
+                    const float2 arg = ffma2(make_float2(x[t], x[t + 1]), cc, nm);
+                    const float2 pr = make_float2(fast_exp2(arg.x), fast_exp2(arg.y));
+                    if (e & 1)
+                        ps2b = fadd2(ps2b, pr);
+                    else
+                        ps2a = fadd2(ps2a, pr);
+                    const __nv_bfloat162 v2 = __floats2bfloat162_rn(pr.x, pr.y);
                     w[e] = *reinterpret_cast<const uint32_t *>(&v2);
                 }
                 tmem_st16(t_s + 16 * half, w);
             }
+            const float ps0 = ps2a.x + ps2b.x, ps1 = ps2a.y + ps2b.y;
             const float ps = ps0 + ps1;
             asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
             l_run = l_run * alpha + ps;
