@@ -174,12 +174,16 @@ int paged_attn_decode_ex(void *out, const void *q, const void *k_cache, const vo
  *               PKV_STATUS_BAD_CONTEXT_LEN; a bad table entry sets
  *               PKV_STATUS_BAD_BLOCK_ID (that block is skipped).
  * The rest as paged_attn_decode. Supported: head_dim 64 / 128, block_size
- * 16 / 32, group <= 8, num_seqs and num_kv_heads <= 65535, max_blocks_per_seq *
- * 4 bytes + 2 K/V blocks of shared memory per CTA. One launch; no workspace.
- * Kernel: a CTA per (64 rows of (query token, group head), sequence, kv head)
+ * 16 / 32, group <= 8, num_seqs and num_kv_heads <= 65535, and a block table
+ * row (max_blocks_per_seq * 4 bytes) that fits shared memory next to the
+ * kernel's tiles. One launch; no workspace.
+ * Kernel: paged_attn_prefill_ex with kernel 0 -- the tcgen05 kernel when the
+ * group num_q_heads / num_kv_heads is 1, 2, 4 or 8 and its shared memory
+ * (about 100 KB + max_blocks_per_seq * 4 bytes) fits, else the mma.sync
+ * kernel: a CTA per (64 rows of (query token, group head), sequence, kv head)
  * streams the K/V blocks its rows need (TMA tile copies, 2-stage ring) and
- * computes S = Q K^T, a causal online softmax and O += P V on tensor cores
- * (mma.sync m16n8k16 bf16, fp32 accumulate; P rounded to bf16).
+ * computes S = Q K^T, a causal online softmax and O += P V (mma.sync
+ * m16n8k16 bf16, fp32 accumulate; P rounded to bf16).
  */
 int paged_attn_prefill(void *out, const void *q, const void *k_cache, const void *v_cache,
                        const int32_t *block_tables, const int32_t *context_lens, const int32_t *query_start,
@@ -190,11 +194,16 @@ int paged_attn_prefill(void *out, const void *q, const void *k_cache, const void
 /*
  * paged_attn_prefill with a choice of kernel: 0 = default (tcgen05 where it
  * applies, else mma.sync), 1 = the mma.sync kernel, 2 = the tcgen05 kernel
- * (PKV_ERR_UNSUPPORTED unless num_q_heads / num_kv_heads is 1, 2, 4 or 8).
+ * (PKV_ERR_UNSUPPORTED unless num_q_heads / num_kv_heads is 1, 2, 4 or 8 and
+ * its shared memory fits); another value returns PKV_ERR_INVALID_ARGUMENT.
  * The tcgen05 kernel: a CTA per 128 rows of (query token, group head) of a
- * sequence and kv head; S = Q K^T and O += P V on tcgen05.mma with fp32
- * accumulators in tensor memory (P rounded to bf16), Q and the K/V blocks
- * staged by TMA, one thread per query row for the causal online softmax.
+ * sequence and kv head, two CTAs per SM (about 100 KB of shared memory and
+ * 256 tensor-memory columns each); S = Q K^T and O += P V on tcgen05.mma with
+ * fp32 accumulators in tensor memory (P rounded to bf16, the softmax sums in
+ * fp32), Q and the K/V blocks staged by TMA, one thread per query row for
+ * the causal online softmax. Every wait inside it is bounded (1 s): one that
+ * gives up sets PKV_STATUS_WAIT_TIMEOUT in d_status and the CTA drains its
+ * copies and MMAs and frees its tensor memory before it exits.
  */
 int paged_attn_prefill_ex(void *out, const void *q, const void *k_cache, const void *v_cache,
                           const int32_t *block_tables, const int32_t *context_lens, const int32_t *query_start,
