@@ -440,9 +440,13 @@ int paged_attn_prefill_ex(void *out, const void *q, const void *k_cache, const v
         return fail(PKV_ERR_INVALID_ARGUMENT, "out, q, k_cache and v_cache must be 16-byte aligned");
     // tcgen05 kernel: 128 rows must be whole query tokens (group 1, 2, 4, 8)
     const size_t smem_tc = pkv::prefill_tc_smem_bytes(head_dim, max_blocks_per_seq);
-    const bool tc_ok = (group == 1 || group == 2 || group == 4 || group == 8) && smem_tc <= 227 * 1024;
-    if (kernel == 2 && !tc_ok)
+    const bool tc_group = group == 1 || group == 2 || group == 4 || group == 8;
+    const bool tc_ok = tc_group && smem_tc <= 227 * 1024;
+    if (kernel == 2 && !tc_group)
         return fail(PKV_ERR_UNSUPPORTED, "the tcgen05 kernel needs num_q_heads / num_kv_heads in {1, 2, 4, 8}");
+    if (kernel == 2 && !tc_ok)
+        return fail(PKV_ERR_UNSUPPORTED, "the tcgen05 kernel needs %zu bytes of shared memory for max_blocks_per_seq %d",
+                    smem_tc, max_blocks_per_seq);
     const bool use_tc = kernel == 2 || (kernel == 0 && tc_ok);
     const size_t smem = use_tc ? smem_tc : pkv::prefill_smem_bytes(head_dim, block_size, max_blocks_per_seq);
     if (smem > 227 * 1024)

@@ -81,6 +81,19 @@ def test_scales_of_either_sign_and_size(kernel, scale):
     assert_close_to_oracle(out.double().numpy(), ref_of(b), what=f"scale {scale} kernel={kernel}")
 
 
+def test_long_tables_fall_back_to_the_mma_sync_kernel():
+    """A block-table row too long for the tcgen05 kernel's shared memory: kernel 2
+    refuses it, the default runs the mma.sync kernel."""
+    b = workloads.make_prefill(3170, [20, 5], [90, 40], 8, 2, 128, 16)
+    pad = torch.full((b.num_seqs, 40000 - b.block_tables.shape[1]), -1, dtype=torch.int32)
+    b2 = workloads.PrefillBatch(**{**b.__dict__, "block_tables": torch.cat([b.block_tables, pad], dim=1)})
+    with pytest.raises(pkv.PagedKVError, match="shared memory"):
+        run(b2, kernel=2)
+    out, st = run(b2)
+    assert st == 0
+    assert_close_to_oracle(out.double().numpy(), ref_of(b), what="long table, default kernel")
+
+
 def test_llama_shaped_chunked_prefill_sampled_rows():
     rng = np.random.default_rng(31)
     chunks = [512, 256, 384, 128, 1, 1, 1, 1]
