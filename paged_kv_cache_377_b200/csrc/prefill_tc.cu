@@ -212,7 +212,8 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     constexpr uint32_t kQHalf = kTcRows * 128;
     constexpr int BPI = kTcTokens / BS;                   // paged blocks per iteration
 
-    const int tile = blockIdx.x, s = blockIdx.y, h = blockIdx.z;
+    // later row tiles see more context (more iterations): they go first
+    const int tile = gridDim.x - 1 - blockIdx.x, s = blockIdx.y, h = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     const int q0 = __ldg(a.query_start + s), q1 = __ldg(a.query_start + s + 1);
