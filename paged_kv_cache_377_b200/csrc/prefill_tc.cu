@@ -4,23 +4,26 @@
 // Same operation as prefill.cu (chunked prefill / mixed batches: query i of a
 // sequence's n-token chunk attends causally to positions 0 .. L - n + i).
 // One CTA per (128 rows of (query token, group head), sequence, kv head), two
-// CTAs per SM, five warps:
-//   - warp 4 (one lane issues) loads the CTA's 128 query rows once by TMA (a
-//     5D box over q viewed as [T][Hkv][G][D]) and streams the context in
-//     iterations of 64 tokens (64 / BS paged blocks) through separate 2-stage
-//     rings of K and V (128-byte swizzled tiles); it issues S = Q K^T (M 128,
-//     N 64, K = head_dim in steps of 16) into one of two tensor-memory
-//     buffers, and O += P V (M 128, N = head_dim, K 64; P read from tensor
-//     memory, V as an N-major operand straight from its TMA tile). S of the
-//     next iteration runs on the tensor cores while the softmax of this one
-//     runs; a K stage is refilled as soon as its S is done, a V stage as soon
-//     as its P V is done;
+// CTAs per SM (256 tensor-memory columns each), six warps; launched with the
+// row tiles that see the most context first:
+//   - warp 4 issues every TMA copy: the CTA's 128 query rows once (a 5D box
+//     over q viewed as [T][Hkv][G][D]) and the context in iterations of 64
+//     tokens (64 / BS paged blocks) through separate 2-stage rings of K and V
+//     (128-byte swizzled tiles; one lane per block slice). It polls for the
+//     MMA that frees each stage, so K and V refills never queue behind each
+//     other;
+//   - warp 5 (an elected lane) issues the MMAs: S = Q K^T (M 128, N 64, K =
+//     head_dim in steps of 16) into one of two tensor-memory buffers, and
+//     O += P V (M 128, N = head_dim, K 64; P read from tensor memory, V as an
+//     N-major operand straight from its TMA tile). S of the next iteration
+//     runs on the tensor cores while the softmax of this one runs;
 //   - warps 0-3: thread r owns query row r (tensor-memory lane r): it loads its
-//     64 logits, masks the positions its query may not see, updates its
-//     running maximum and sum, writes its row of P in bf16 over the S buffer,
-//     and rescales its row of O in tensor memory when its maximum has grown by
-//     more than 2^8 since the last rescale (otherwise the stale maximum stays
-//     the reference: every P is then < 2^8 and the result is the same).
+//     64 logits in one tensor-memory load, masks the positions its query may
+//     not see, updates its running maximum and sum, writes its row of P in
+//     bf16 over the S buffer, and rescales its row of O in tensor memory when
+//     its maximum has grown by more than 2^8 since the last rescale
+//     (otherwise the stale maximum stays the reference: every P is then < 2^8
+//     and the result is the same).
 // All waits are bounded (1 s); a wait that gives up flags the status word,
 // the CTA drains what it issued and frees its tensor memory.
 #include <cuda_bf16.h>
