@@ -158,3 +158,39 @@ def test_missing_library_fails_loudly(monkeypatch):
     monkeypatch.setattr(_binding._build, "build", no_build)
     with pytest.raises(RuntimeError, match="nvcc"):
         pkv.workspace_bytes(1, 1, 64)
+
+
+def _prefill(**kw):
+    args = dict(out=P, q=P, k=P, v=P, bt=P, cl=P, qs=P, S=2, T=9, MQ=5, Hq=8, Hkv=2, D=128, bs=16, scale=0.125,
+                MB=8, NB=32, st=P, kernel=0)
+    args.update(kw)
+    lib = pkv.library()
+    rc = lib.paged_attn_prefill_ex(args["out"], args["q"], args["k"], args["v"], args["bt"], args["cl"], args["qs"],
+                                   args["S"], args["T"], args["MQ"], args["Hq"], args["Hkv"], args["D"], args["bs"],
+                                   args["scale"], args["MB"], args["NB"], args["st"], args["kernel"], None)
+    return rc, lib.pkv_last_error().decode()
+
+
+@pytest.mark.parametrize("kw,code,msg", [
+    (dict(kernel=3), -1, "kernel must be"),
+    (dict(st=None), -1, "NULL"),
+    (dict(qs=None), -1, "NULL"),
+    (dict(MQ=-1), -1, "max_query_len"),
+    (dict(Hq=6, Hkv=4), -1, "multiple"),
+    (dict(D=96), -2, "head_dim"),
+    (dict(bs=8), -2, "block_size"),
+    (dict(Hq=32, Hkv=2), -2, "exceeds"),
+    (dict(scale=float("nan")), -1, "scale"),
+    (dict(out=ctypes.c_void_p(4096 + 8)), -1, "aligned"),
+    (dict(kernel=2, Hq=6, Hkv=2), -2, "tcgen05"),                       # group 3: 128 rows are not whole tokens
+    (dict(kernel=2, MB=40000), -2, "shared memory"),                   # the table row does not fit beside the tiles
+])
+def test_prefill_rejects_bad_arguments_without_touching_the_gpu(kw, code, msg):
+    rc, err = _prefill(**kw)
+    assert rc == code and msg in err, (rc, err)
+
+
+@pytest.mark.parametrize("kw", [dict(S=0), dict(T=0), dict(MQ=0), dict(T=0, kernel=2), dict(T=0, kernel=1)])
+def test_prefill_of_empty_batch_is_a_no_op(kw):
+    rc, err = _prefill(**kw)
+    assert rc == 0, err
