@@ -40,6 +40,11 @@ MUTANTS = [
     ("prefill sees the whole context", "int p = context_lens[s] - n + i;", "int p = context_lens[s] - 1;"),
     ("prefill reads the chunk's first query", "q + (row * num_q_heads + j) * (int64_t)head_dim",
      "q + ((int64_t)query_start[s] * num_q_heads + j) * (int64_t)head_dim"),
+    ("prefill output rows transposed", "mine = decode_one(out + (row * num_q_heads + j) * head_dim, x,",
+     "mine = decode_one(out + ((int64_t)j * num_tokens + row) * head_dim, x,"),
+    ("prefill chunk rows reversed", "int64_t row = (int64_t)query_start[s] + i;",
+     "int64_t row = (int64_t)query_start[s + 1] - 1 - i;"),
+    ("prefill reads sequence 0's table", "p + 1, s, j, num_q_heads", "p + 1, 0, j, num_q_heads"),
 ]
 
 
