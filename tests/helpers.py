@@ -76,6 +76,53 @@ def load_golden(name: str):
     return batch, expected
 
 
+def prefill_golden_names() -> List[str]:
+    return sorted(os.path.basename(p)[:-5] for p in glob.glob(os.path.join(GOLDEN_DIR, "prefill", "*.json")))
+
+
+def load_golden_prefill(name: str):
+    """A multi-query golden fixture as a PrefillBatch, plus its exact expected rows
+    keyed by (query token row, q head). Query rows are keyed by token row; pool
+    slots the fixture does not name hold NaN; vectors are padded with zeros."""
+    with open(os.path.join(GOLDEN_DIR, "prefill", name + ".json")) as f:
+        fx = json.load(f)
+    Hq, Hkv, D, bs, NB = fx["num_q_heads"], fx["num_kv_heads"], fx["head_dim"], fx["block_size"], fx["num_blocks"]
+    tables = np.asarray(fx["block_tables"], dtype=np.int32)
+    lens = np.asarray(fx["context_lens"], dtype=np.int32)
+    qs = np.asarray(fx["query_start"], dtype=np.int32)
+    S, T = len(lens), int(qs[-1])
+    sc = fx["scale"]
+    scale = math.log(sc["ln"]) if "ln" in sc else float(sc["value"])
+    q = torch.zeros(T, Hq, D, dtype=torch.float32)
+    for k, vals in fx["q"].items():
+        r, j = _key(k)
+        q[r, j, :len(vals)] = torch.tensor(vals, dtype=torch.float32)
+    kc = torch.full((NB, bs, Hkv, D), float("nan"), dtype=torch.float32)
+    vc = torch.full((NB, bs, Hkv, D), float("nan"), dtype=torch.float32)
+    for name_, cache in (("k", kc), ("v", vc)):
+        for k, vals in fx[name_].items():
+            p, off, h = _key(k)
+            cache[p, off, h, :] = 0.0
+            cache[p, off, h, :len(vals)] = torch.tensor(vals, dtype=torch.float32)
+    for t in (q, kc, vc):
+        assert torch.equal(t.to(torch.bfloat16).float().nan_to_num(7.0), t.nan_to_num(7.0)), "fixture values must be bf16-exact"
+    batch = workloads.PrefillBatch(
+        name=name, seed=0, num_seqs=S, num_q_heads=Hq, num_kv_heads=Hkv, head_dim=D, block_size=bs,
+        scale=scale, max_blocks_per_seq=tables.shape[1], num_blocks=NB,
+        context_lens=torch.from_numpy(lens), block_tables=torch.from_numpy(tables),
+        slot_mapping=torch.full((T,), -1, dtype=torch.int64),
+        q=q.to(torch.bfloat16), k_cache=kc.to(torch.bfloat16), v_cache=vc.to(torch.bfloat16),
+        k_new=torch.zeros(T, Hkv, D, dtype=torch.bfloat16), v_new=torch.zeros(T, Hkv, D, dtype=torch.bfloat16),
+        query_start=torch.from_numpy(qs),
+    )
+    expected: Dict[tuple, np.ndarray] = {}
+    for k, vals in fx["expected"].items():
+        row = np.zeros(D, dtype=np.float64)
+        row[:len(vals)] = [float(Fraction(v)) for v in vals]
+        expected[_key(k)] = row
+    return batch, expected
+
+
 def gather_contiguous(batch, k_cache=None, v_cache=None):
     """Per sequence, the K and V rows in logical order, as fp64 [L][Hkv][D] arrays.
 

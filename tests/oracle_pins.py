@@ -25,7 +25,8 @@ import torch
 
 import oracle
 import workloads
-from helpers import bf16_bits, gather_contiguous, golden_names, load_golden, sdpa_reference
+from helpers import (bf16_bits, gather_contiguous, golden_names, load_golden, load_golden_prefill,
+                     prefill_golden_names, sdpa_reference)
 
 TIGHT = 1e-12
 
@@ -435,6 +436,17 @@ def pin_prefill_causal_sdpa(lib=None):
             _close(got[qs[s]:qs[s + 1]], ref[0].permute(1, 0, 2).numpy(), what=f"prefill case {i} seq {s}")
 
 
+def pin_prefill_golden(lib=None):
+    """Worked multi-query examples with exact expected rows (tests/golden/prefill)."""
+    names = prefill_golden_names()
+    assert names, "no multi-query golden fixtures"
+    for name in names:
+        b, expected = load_golden_prefill(name)
+        got = _prefill(b, lib)
+        for (r, j), row in expected.items():
+            _close(got[r, j], row, tol=1e-14, what=f"prefill golden {name} ({r},{j})")
+
+
 def pin_prefill_single_queries_are_decodes(lib=None):
     """Chunks of one token are decode steps over the whole context."""
     L = [9, 1, 30, 17]
@@ -497,6 +509,7 @@ ALL_PINS = [
     pin_fp8_scales_act_as_the_pages_define,
     pin_fp8_poisoned_slots_are_never_read,
     pin_prefill_causal_sdpa,
+    pin_prefill_golden,
     pin_prefill_single_queries_are_decodes,
     pin_prefill_equal_keys_give_prefix_means,
     pin_prefill_block_permutation_invariance,
