@@ -8,7 +8,7 @@ import torch
 import oracle
 import paged_kv_cache_377_b200 as pkv
 import workloads
-from helpers import assert_close_to_oracle
+from helpers import assert_close_to_oracle, gather_contiguous, load_golden_prefill, prefill_golden_names
 
 pytestmark = pytest.mark.gpu
 
@@ -92,6 +92,44 @@ def test_long_tables_fall_back_to_the_mma_sync_kernel():
     out, st = run(b2)
     assert st == 0
     assert_close_to_oracle(out.double().numpy(), ref_of(b), what="long table, default kernel")
+
+
+def _relayout(b, block_size, seed):
+    """The same sequences in a fresh pool of block_size-token blocks, in a shuffled
+    physical order; slots past each context hold NaN."""
+    rows = gather_contiguous(b)
+    nblk = [(int(L) + block_size - 1) // block_size for L in b.context_lens]
+    NB = max(sum(nblk), 1)
+    perm = np.random.default_rng(seed).permutation(NB)
+    kc = torch.full((NB, block_size, b.num_kv_heads, b.head_dim), float("nan"), dtype=torch.float64)
+    vc = kc.clone()
+    tables = np.zeros((b.num_seqs, max(max(nblk), 1)), dtype=np.int32)
+    nxt = 0
+    for s_, (k, v) in enumerate(rows):
+        for lb in range(nblk[s_]):
+            p = int(perm[nxt])
+            nxt += 1
+            tables[s_, lb] = p
+            t = np.arange(lb * block_size, min((lb + 1) * block_size, k.shape[0]))
+            kc[p, :len(t)] = torch.from_numpy(k[t])
+            vc[p, :len(t)] = torch.from_numpy(v[t])
+    return workloads.PrefillBatch(**{**b.__dict__, "block_size": block_size, "num_blocks": NB,
+                                     "max_blocks_per_seq": tables.shape[1], "block_tables": torch.from_numpy(tables),
+                                     "k_cache": kc.to(torch.bfloat16), "v_cache": vc.to(torch.bfloat16)})
+
+
+@pytest.mark.parametrize("kernel", [1, 2])
+@pytest.mark.parametrize("bs", [16, 32])
+@pytest.mark.parametrize("name", prefill_golden_names())
+def test_worked_examples_give_their_exact_values(name, bs, kernel):
+    """The multi-query golden fixtures (values derived by hand), re-laid in the
+    kernels' block sizes: every output within the bf16 tolerance of its exact value."""
+    b, expected = load_golden_prefill(name)
+    out, st = run(_relayout(b, bs, seed=bs), kernel=kernel)
+    assert st == 0
+    got = out.double().numpy()
+    for (r, j), row in expected.items():
+        assert np.all(np.abs(got[r, j] - row) <= 8e-3 + 8e-3 * np.abs(row)), (name, r, j, got[r, j][:2], row[:2])
 
 
 def test_llama_shaped_chunked_prefill_sampled_rows():
