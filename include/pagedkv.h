@@ -233,7 +233,9 @@ int paged_attn_prefill_ex(void *out, const void *q, const void *k_cache, const v
  * 2^15); probabilities are rounded to f16. Supported: head_dim 128, or 64
  * with head packing (an even num_kv_heads and num_q_heads / num_kv_heads <=
  * 4, so that every row read is 128 bytes); block_size 16 or 32; opts->math 0
- * or 2 (1 returns PKV_ERR_UNSUPPORTED). Default: 2 ring stages per warp.
+ * or 2 (1 returns PKV_ERR_UNSUPPORTED). Default ring: about 8 KB of blocks
+ * in flight per warp -- 1 stage when kv heads are read in pairs (rows of 256
+ * codes, the default for head_dim 128), else 2.
  */
 int kv_cache_append_fp8(const void *k, const void *v, void *k_cache, void *v_cache, const int64_t *slot_mapping,
                         const float *k_scale, const float *v_scale, int num_tokens, int num_kv_heads, int head_dim,
