@@ -90,7 +90,8 @@ extern "C" {
  *                     [bs][Hkv/2][2D]), so that each token row of a read is
  *                     256 contiguous bytes instead of 128. Possible on tensor
  *                     cores with head_dim 64, an even num_kv_heads and a group
- *                     of at most 4; asking for 2 elsewhere returns
+ *                     of at most 4 (on e4m3 pools also with head_dim 128, see
+ *                     paged_attn_decode_fp8); asking for 2 elsewhere returns
  *                     PKV_ERR_UNSUPPORTED.
  */
 typedef struct pkv_decode_options {
