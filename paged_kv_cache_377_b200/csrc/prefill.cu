@@ -7,6 +7,11 @@
 // (already appended to the paged pool); query i sits at position
 // p = L_s - n_s + i and attends causally to positions 0 .. p. Decode is n_s = 1.
 //
+// This is the mma.sync kernel: the fallback of paged_attn_prefill for groups
+// the tcgen05 kernel (prefill_tc.cu) cannot tile (other than 1, 2, 4, 8) and
+// for block tables too long for its shared memory, and kernel 1 of
+// paged_attn_prefill_ex.
+//
 // Structure: one CTA per (64-row tile, sequence, kv head); a row is a (query
 // token, group head) pair, row = i * G + g, so the GQA group shares every K/V
 // tile. 4 warps x 16 rows. The CTA streams the blocks its last row needs
