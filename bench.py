@@ -405,7 +405,8 @@ def run_ours(args, rank, world, local_rank):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "f32" if args.kv_dtype == "bf16" else "f32 (e4m3 KV, f16 products)",
+        "dtype": ("bf16 products, f32 accumulate" if args.kv_dtype == "bf16" else
+                  "f16 products of e4m3 KV, f32 accumulate"),
         "data": "synthetic",
         "config": config_block(args, batch, world),
         "pct_of_hbm_peak": round(100.0 * value / (hbm * world), 2),
@@ -741,7 +742,7 @@ def run_prefill(args, rank, world, local_rank):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16 (fp32 accumulate)",
+        "dtype": "bf16 products, f32 accumulate",
         "data": "synthetic",
         "config": {"workload": args.workload, "description": w["description"], "num_seqs": b.num_seqs,
                    "query_tokens": T, "context_tokens": int(b.context_lens.sum()), "flops_per_step": flops,

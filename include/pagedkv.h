@@ -308,7 +308,10 @@ int paged_attn_decode_append(void *out, const void *q, const void *k_new, const 
  *     PKV_ERR_INVALID_ARGUMENT and a message giving both sizes.
  *   - The first call on a device looks up the scratch's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture begins.
+ *     before any stream capture begins. The address is kept for the life of
+ *     the process: after cudaDeviceReset, or anything else that destroys the
+ *     device's primary context, do not call this entry point again in that
+ *     process (it would hand the kernels the old context's address).
  *   - All calls share the one scratch, which keeps the last call's contents.
  *     Calls that overlap on the GPU (different streams, no ordering between
  *     them) race on it and give wrong results: order them.

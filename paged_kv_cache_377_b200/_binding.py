@@ -140,6 +140,20 @@ def allocate_workspace(num_seqs: int, num_q_heads: int, head_dim: int, device=No
     return torch.zeros(n, dtype=torch.uint8, device=device if device is not None else "cuda")
 
 
+def _decode_shapes(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                   block_tables: torch.Tensor, context_lens: torch.Tensor):
+    """(S, Hq, D, NB, bs, Hkv) of a decode call, after checking that the tensors
+    agree: the C ABI sees only pointers and the sizes passed with them, so a
+    short table or a head_dim mismatch would become out-of-bounds device accesses."""
+    S, Hq, D = q.shape
+    NB, bs, Hkv, D2 = k_cache.shape
+    if out.shape != q.shape or v_cache.shape != k_cache.shape or D2 != D:
+        raise ValueError("shape mismatch between q/out or k_cache/v_cache")
+    if block_tables.shape[0] != S or context_lens.shape[0] != S:
+        raise ValueError("block_tables and context_lens must have num_seqs rows")
+    return S, Hq, D, NB, bs, Hkv
+
+
 def paged_attn_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
                       block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float,
                       workspace: torch.Tensor, num_ctas: int = 0, num_stages: int = 0,
@@ -159,12 +173,7 @@ def paged_attn_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
     _need(block_tables, "block_tables", torch.int32, 2)
     _need(context_lens, "context_lens", torch.int32, 1)
     _need(workspace, "workspace", torch.uint8, 1)
-    S, Hq, D = q.shape
-    NB, bs, Hkv, D2 = k_cache.shape
-    if out.shape != q.shape or v_cache.shape != k_cache.shape or D2 != D:
-        raise ValueError("shape mismatch between q/out or k_cache/v_cache")
-    if block_tables.shape[0] != S or context_lens.shape[0] != S:
-        raise ValueError("block_tables and context_lens must have num_seqs rows")
+    S, Hq, D, NB, bs, Hkv = _decode_shapes(out, q, k_cache, v_cache, block_tables, context_lens)
     opts = _Options(num_ctas, num_stages, ctas_per_sm, math, l2_prefetch, piece_cost, head_pack)
     _check("paged_attn_decode", library().paged_attn_decode_ex(
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
@@ -274,12 +283,6 @@ def paged_attn_decode_noalloc(out: torch.Tensor, q: torch.Tensor, k_cache: torch
     int32 device tensor overwritten with the call's status bits.
     """
     global _noalloc_ready
-    lib = library()
-    if not _noalloc_ready:
-        P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
-        lib.paged_attn_decode_noalloc.restype = I
-        lib.paged_attn_decode_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, I, I, P, P]
-        _noalloc_ready = True
     _need(q, "q", torch.bfloat16, 3)
     _need(out, "out", torch.bfloat16, 3)
     _need(k_cache, "k_cache", torch.bfloat16, 4)
@@ -288,8 +291,13 @@ def paged_attn_decode_noalloc(out: torch.Tensor, q: torch.Tensor, k_cache: torch
     _need(context_lens, "context_lens", torch.int32, 1)
     if status is not None:
         _need(status, "status", torch.int32, 1)
-    S, Hq, D = q.shape
-    NB, bs, Hkv, _ = k_cache.shape
+    S, Hq, D, NB, bs, Hkv = _decode_shapes(out, q, k_cache, v_cache, block_tables, context_lens)
+    lib = library()
+    if not _noalloc_ready:
+        P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+        lib.paged_attn_decode_noalloc.restype = I
+        lib.paged_attn_decode_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, I, I, P, P]
+        _noalloc_ready = True
     _check("paged_attn_decode_noalloc", lib.paged_attn_decode_noalloc(
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
         S, Hq, Hkv, D, bs, float(scale), block_tables.shape[1], NB, _ptr(status), _stream(stream)))

@@ -579,7 +579,8 @@ std::vector<void *> g_noalloc_ptr;  // device address of g_noalloc_scratch, per 
 
 // In host code g_noalloc_scratch names a host-side stand-in, not device memory:
 // the kernels get the address cudaGetSymbolAddress returns for the current
-// device, looked up on the first call on that device and cached.
+// device, looked up on the first call on that device and cached for the life
+// of the process (a device reset, which would move the array, is not followed).
 int noalloc_scratch(void **ptr) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);

@@ -22,3 +22,16 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_sessionfinish(session, exitstatus):
+    """With PKV_PARITY_LOG=<file>, write the largest normalised errors each parity check saw."""
+    path = os.environ.get("PKV_PARITY_LOG")
+    if not path:
+        return
+    import json
+
+    from helpers import PARITY_LOG
+    with open(path, "w") as f:
+        for rec in PARITY_LOG:
+            f.write(json.dumps(rec) + "\n")

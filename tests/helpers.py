@@ -175,8 +175,45 @@ def bf16_bits(t: torch.Tensor) -> np.ndarray:
     return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
 
 
-def assert_close_to_oracle(got: np.ndarray, ref: np.ndarray, atol: float = ATOL, rtol: float = RTOL, what: str = ""):
-    """Elementwise |got - ref| <= atol + rtol*|ref|; NaN anywhere fails."""
+# Normalised per-row bounds, applied next to the elementwise one. A row is one
+# output vector (the last axis: one query token and q head). On long contexts
+# |ref| shrinks like 1/sqrt(L) (about 4e-3 at 64K tokens), so the elementwise
+# bound's absolute term is wider than the values themselves and a lost or
+# mis-weighted context piece would hide inside it; these two do not scale with
+# |ref|. Paging changes where K/V live, not what attention computes ("vLLM
+# Fundamentals: Paged Attention and Batching", section "Paged Attention"), so the
+# paged result must be the plain one up to the arithmetic's rounding: bf16
+# output rounding alone gives a relative error up to 2^-9 per element, the
+# probabilities' bf16 (or f16) rounding about as much again.
+REL_L2 = 1e-2        # ||got - ref||_2 / ||ref||_2 per row
+MAX_OVER_RMS = 4e-2  # max|got - ref| / rms(ref) per row
+
+# Largest normalised errors seen, per call (written out when PKV_PARITY_LOG names a file).
+PARITY_LOG: List[dict] = []
+
+
+def row_errors(got: np.ndarray, ref: np.ndarray):
+    """Per row (last axis): relative L2 error and max|err| / rms(ref); rows with
+    ref == 0 everywhere give 0 (the elementwise bound covers them)."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    n = ref.shape[-1] if ref.ndim else 1
+    g2 = got.reshape(-1, n)
+    r2 = ref.reshape(-1, n)
+    err = g2 - r2
+    rnorm = np.sqrt((r2 * r2).sum(axis=1))
+    live = rnorm > 0
+    rel = np.zeros(len(r2))
+    mor = np.zeros(len(r2))
+    rel[live] = np.sqrt((err[live] ** 2).sum(axis=1)) / rnorm[live]
+    mor[live] = np.abs(err[live]).max(axis=1) / (rnorm[live] / np.sqrt(n))
+    return rel, mor
+
+
+def assert_close_to_oracle(got: np.ndarray, ref: np.ndarray, atol: float = ATOL, rtol: float = RTOL, what: str = "",
+                           normalised: bool = True):
+    """Elementwise |got - ref| <= atol + rtol*|ref|; NaN anywhere fails. With
+    ``normalised`` (the default), every row must also meet REL_L2 and MAX_OVER_RMS."""
     got = np.asarray(got, dtype=np.float64)
     assert got.shape == ref.shape, (got.shape, ref.shape)
     assert not np.isnan(got).any(), f"{what}: NaN in output"
@@ -188,3 +225,14 @@ def assert_close_to_oracle(got: np.ndarray, ref: np.ndarray, atol: float = ATOL,
         raise AssertionError(
             f"{what}: {int(bad.sum())} of {bad.size} elements out of tolerance; max err {err.max():.3e}; "
             f"first {idx.tolist()} got {got[tuple(idx[0])]} ref {ref[tuple(idx[0])]}")
+    if not normalised or got.size == 0:
+        return
+    rel, mor = row_errors(got, ref)
+    PARITY_LOG.append({"what": what, "rows": int(len(rel)), "rel_l2_max": float(rel.max()),
+                       "max_over_rms_max": float(mor.max())})
+    if (rel > REL_L2).any() or (mor > MAX_OVER_RMS).any():
+        r = int(np.argmax(np.maximum(rel / REL_L2, mor / MAX_OVER_RMS)))
+        raise AssertionError(
+            f"{what}: {int((rel > REL_L2).sum())} rows above relative L2 {REL_L2} and {int((mor > MAX_OVER_RMS).sum())} "
+            f"above max|err|/rms {MAX_OVER_RMS} (of {len(rel)}); worst row {r}: relative L2 {rel[r]:.3e}, "
+            f"max|err|/rms {mor[r]:.3e}")

@@ -194,3 +194,35 @@ def test_prefill_rejects_bad_arguments_without_touching_the_gpu(kw, code, msg):
 def test_prefill_of_empty_batch_is_a_no_op(kw):
     rc, err = _prefill(**kw)
     assert rc == 0, err
+
+
+@pytest.mark.parametrize("bad", ["out", "v_cache", "head_dim", "block_tables", "context_lens"])
+def test_noalloc_binding_checks_shapes_before_calling_the_library(monkeypatch, bad):
+    """paged_attn_decode_noalloc's binding checks that the tensors agree, like
+    paged_attn_decode's: the C ABI cannot see tensor lengths, so a short table or
+    a head_dim mismatch would reach the kernel as out-of-bounds accesses."""
+    import torch
+    from paged_kv_cache_377_b200 import _binding
+
+    calls = []
+    monkeypatch.setattr(_binding, "_need", lambda *a, **k: None)      # CPU tensors stand in for device ones
+    monkeypatch.setattr(_binding, "library", lambda: calls.append(1))
+    S, Hq, Hkv, D, NB, bs, MB = 3, 8, 2, 64, 10, 16, 4
+    t = dict(out=torch.zeros(S, Hq, D, dtype=torch.bfloat16), q=torch.zeros(S, Hq, D, dtype=torch.bfloat16),
+             k_cache=torch.zeros(NB, bs, Hkv, D, dtype=torch.bfloat16),
+             v_cache=torch.zeros(NB, bs, Hkv, D, dtype=torch.bfloat16),
+             block_tables=torch.zeros(S, MB, dtype=torch.int32), context_lens=torch.zeros(S, dtype=torch.int32))
+    if bad == "out":
+        t["out"] = torch.zeros(S + 1, Hq, D, dtype=torch.bfloat16)
+    elif bad == "v_cache":
+        t["v_cache"] = torch.zeros(NB - 1, bs, Hkv, D, dtype=torch.bfloat16)
+    elif bad == "head_dim":
+        t["k_cache"] = t["v_cache"] = torch.zeros(NB, bs, Hkv, 2 * D, dtype=torch.bfloat16)
+    elif bad == "block_tables":
+        t["block_tables"] = torch.zeros(S - 1, MB, dtype=torch.int32)
+    else:
+        t["context_lens"] = torch.zeros(S - 1, dtype=torch.int32)
+    with pytest.raises(ValueError):
+        _binding.paged_attn_decode_noalloc(t["out"], t["q"], t["k_cache"], t["v_cache"], t["block_tables"],
+                                           t["context_lens"], 0.125)
+    assert calls == [], "the library was reached with inconsistent shapes"

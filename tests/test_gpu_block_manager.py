@@ -3,14 +3,15 @@
 Prompts are written with kv_cache_append at the slots the manager hands out,
 copy-on-write copies run in kv_block_copy, and every decode step is one
 paged_attn_decode_append over the tables the manager packs. Each step's output
-must match brute-force attention over the sequences' own token lists (bf16
-tolerance), and the device pools must equal, bit for bit, a host pool that
-took the same writes and copies.
+must match the fp64 oracle over a host pool that took the same writes and
+copies, and brute-force attention over the sequences' own token lists (bf16
+tolerance); the device pools must equal that host pool bit for bit.
 """
 import numpy as np
 import pytest
 import torch
 
+import oracle
 import paged_kv_cache_377_b200 as pkv
 from bm_stream import HostPool, Stream, random_stream
 from helpers import assert_close_to_oracle
@@ -46,8 +47,12 @@ def test_stream_on_the_gpu(seed, Hq, Hkv, D, bs):
                                      torch.from_numpy(x["slots"]).to(dev), kc, vc, torch.from_numpy(x["bt"]).to(dev),
                                      torch.from_numpy(x["cl"]).to(dev), scale, ws)
         assert pkv.read_status(ws) == 0 and pkv.read_status(status) == 0
-        ref = st.reference(ids, x["q"], scale)
-        assert_close_to_oracle(out.double().cpu().numpy(), ref, what=f"step {steps[0]}")
+        got = out.double().cpu().numpy()
+        # the fp64 oracle over the host pool and the tables the manager packed ...
+        ref = oracle.paged_decode(x["q"], host.k, host.v, x["bt"], x["cl"], Hkv, bs, scale)
+        assert_close_to_oracle(got, ref, what=f"step {steps[0]} (oracle)")
+        # ... and brute force over each sequence's own token list, with no table at all
+        assert_close_to_oracle(got, st.reference(ids, x["q"], scale), what=f"step {steps[0]} (token lists)")
         steps[0] += 1
 
     copies = random_stream(st, write_prompt, step, steps=40, max_blocks=MB, seed=seed)

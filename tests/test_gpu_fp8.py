@@ -153,3 +153,29 @@ def test_fp8_block_permutation_is_bitwise_invariant():
     out1, _, _, _ = one_launch(b)
     out2, _, _, _ = one_launch(workloads.permute_pool(b, seed=9))
     assert same_bits(out1, out2)
+
+
+@pytest.mark.parametrize("Hq,Hkv,D,bs", [(32, 8, 128, 16), (8, 2, 64, 32), (4, 2, 128, 32), (4, 4, 128, 16)])
+def test_fp8_decode_reads_every_finite_code(Hq, Hkv, D, bs):
+    """The pools hold every finite e4m3 code -- subnormals, both zeros and +-448
+    included -- in a scrambled order (the recipe's random codes stop at 30 in
+    magnitude). Scales of 2^-8 .. 2^-7 keep the logits moderate."""
+    lens = [1, bs - 1, bs + 1, 300, 777, 0, 2000]
+    b = workloads.make_custom(4242 + D + bs + Hq, lens, Hq, Hkv, D, bs, kv_dtype="fp8")
+    finite = torch.tensor([c for c in range(256) if c not in (0x7F, 0xFF)], dtype=torch.uint8)
+    for pool, shift in ((b.k_cache, 0), (b.v_cache, 101)):
+        flat = pool.view(-1)
+        live = flat != workloads.E4M3_NAN_CODE      # poisoned slots keep their NaN code
+        idx = torch.arange(int(live.sum()))
+        flat[live] = finite[(idx * 97 + shift) % len(finite)]   # 97 and 254 are coprime: every code recurs
+    h = torch.arange(Hkv, dtype=torch.float32)
+    b.k_scale = (2.0 ** -8) * (1 + h / Hkv)
+    b.v_scale = (2.0 ** -8) * (1 + h / (2 * Hkv))
+    ref, kc_ref, vc_ref = oracle.decode_step(b)
+    for run in (one_launch, two_launch):
+        for num_ctas in (0, 9):
+            out, kc, vc, st = run(b, num_ctas=num_ctas)
+            assert st == 0
+            assert np.array_equal(kc.numpy(), kc_ref) and np.array_equal(vc.numpy(), vc_ref)
+            assert_close_to_oracle(out.double().numpy(), ref,
+                                   what=f"fp8 every code Hq={Hq} Hkv={Hkv} D={D} bs={bs} {run.__name__} C={num_ctas}")

@@ -46,7 +46,36 @@ def test_noalloc_matches_the_workspace_entry_point_on_two_calls_in_a_row():
         b = workloads.make_batch(name, device=dev)
         with_ws, no_ws, status, ws_status = _decode_both(b, dev)
         assert status == 0 and ws_status == 0, (name, status, ws_status)
+        # same kernel, options and grid: bit for bit (a stale partial left in the
+        # scratch by the previous call could otherwise hide inside a tolerance)
+        assert torch.equal(no_ws.view(torch.int16), with_ws.view(torch.int16)), f"noalloc vs workspace, {name}"
         assert_close_to_oracle(no_ws.double().numpy(), with_ws.double().numpy(), what=f"noalloc vs workspace, {name}")
+
+
+@pytest.mark.gpu
+def test_noalloc_status_reports_only_its_own_call():
+    """d_status is overwritten per call: a call that meets a bad block id reports
+    it, and the clean call after it, on the same scratch, reports 0."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    b = workloads.make_custom(81, [40, 40], 4, 2, 64, 16, with_append=False, poison=False, device=dev)
+    q, kc, vc, cl = b.q, b.k_cache, b.v_cache, b.context_lens.to(dev)
+    good = b.block_tables.to(dev)
+    bad = good.clone()
+    bad[1, 1] = b.num_blocks + 5
+    from paged_kv_cache_377_b200._binding import paged_attn_decode_noalloc
+    status = torch.full((1,), -1, dtype=torch.int32, device=dev)
+    out = torch.empty_like(q)
+    paged_attn_decode_noalloc(out, q, kc, vc, bad, cl, b.scale, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == pkv.PKV_STATUS_BAD_BLOCK_ID
+    paged_attn_decode_noalloc(out, q, kc, vc, good, cl, b.scale, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ws = pkv.allocate_workspace(b.num_seqs, b.num_q_heads, b.head_dim, device=dev)
+    ref = torch.empty_like(q)
+    pkv.paged_attn_decode(ref, q, kc, vc, good, cl, b.scale, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
 
 
 def test_noalloc_rejects_batches_beyond_its_scratch():
