@@ -72,6 +72,7 @@ def parse_args(argv=None):
     p.add_argument("--l2-prefetch", type=int, default=0)
     p.add_argument("--piece-cost", type=int, default=0)
     p.add_argument("--head-pack", type=int, default=0)
+    p.add_argument("--tile-tokens", type=int, default=0)
     p.add_argument("--two-launch", action="store_true",
                    help="run the step as kv_cache_append + paged_attn_decode instead of the one-launch call")
     p.add_argument("--seqs", type=int, default=0,
@@ -271,7 +272,7 @@ class Step:
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
         self.opts = dict(num_ctas=args.num_ctas, num_stages=args.num_stages,
                          ctas_per_sm=args.ctas_per_sm, math=args.math, l2_prefetch=args.l2_prefetch,
-                         piece_cost=args.piece_cost, head_pack=args.head_pack)
+                         piece_cost=args.piece_cost, head_pack=args.head_pack, tile_tokens=args.tile_tokens)
         self.ws = pkv.allocate_workspace(b.num_seqs, b.num_q_heads, b.head_dim, device=device)
         self.fp8 = b.kv_dtype == "fp8"
         if self.fp8:
@@ -393,7 +394,7 @@ def run_ours(args, rank, world, local_rank):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(batch, kv, S, ctx_tokens)
 
-    traffic = profiled_traffic(args.workload)
+    traffic = profiled_traffic(args.workload + ("_fp8" if args.kv_dtype == "fp8" else ""))
     result = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -516,7 +517,7 @@ def config_block(args, batch, world):
     }
     if args.seqs:
         c["seqs_kept"] = args.seqs
-    for k in ("num_ctas", "num_stages", "ctas_per_sm", "math", "l2_prefetch", "piece_cost", "head_pack"):
+    for k in ("num_ctas", "num_stages", "ctas_per_sm", "math", "l2_prefetch", "piece_cost", "head_pack", "tile_tokens"):
         if getattr(args, k):
             c[k] = getattr(args, k)
     return c

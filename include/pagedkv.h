@@ -68,7 +68,7 @@ extern "C" {
  *                     every CTA that fits on the device at once. The KV blocks
  *                     of a launch are split evenly over the CTAs, so this also
  *                     sets how finely long contexts are split.
- *   num_stages        shared-memory stages (one KV block each) per warp (1..4; a
+ *   num_stages        shared-memory stages (one KV tile each) per warp (1..4; a
  *                     CTA has 4 warps); default: 1 on tensor cores, about 64 KB
  *                     of KV blocks per CTA on CUDA cores.
  *   ctas_per_sm       resident CTAs per SM of the default grid; default: the
@@ -93,6 +93,12 @@ extern "C" {
  *                     of at most 4 (on e4m3 pools also with head_dim 128, see
  *                     paged_attn_decode_fp8); asking for 2 elsewhere returns
  *                     PKV_ERR_UNSUPPORTED.
+ *   tile_tokens       token rows per shared-memory tile: 0 = default (16), 16, or
+ *                     32 (block_size 32 only). With 16, a 32-token block is read
+ *                     as two tiles of 16 rows, so that the stages of a CTA are as
+ *                     small as for 16-token blocks and twice as many CTAs fit on
+ *                     an SM; more than block_size returns PKV_ERR_INVALID_ARGUMENT.
+ *                     The result does not depend on it beyond rounding order.
  */
 typedef struct pkv_decode_options {
     int num_ctas;
@@ -102,6 +108,7 @@ typedef struct pkv_decode_options {
     int l2_prefetch;
     int piece_cost;
     int head_pack;
+    int tile_tokens;
 } pkv_decode_options;
 
 /*

@@ -32,7 +32,7 @@ class PagedKVError(RuntimeError):
 class _Options(ctypes.Structure):
     _fields_ = [("num_ctas", ctypes.c_int), ("num_stages", ctypes.c_int),
                 ("ctas_per_sm", ctypes.c_int), ("math", ctypes.c_int), ("l2_prefetch", ctypes.c_int),
-                ("piece_cost", ctypes.c_int), ("head_pack", ctypes.c_int)]
+                ("piece_cost", ctypes.c_int), ("head_pack", ctypes.c_int), ("tile_tokens", ctypes.c_int)]
 
 
 def library_path() -> str:
@@ -158,7 +158,7 @@ def paged_attn_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
                       block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float,
                       workspace: torch.Tensor, num_ctas: int = 0, num_stages: int = 0,
                       ctas_per_sm: int = 0, math: int = 0, l2_prefetch: int = 0, piece_cost: int = 0,
-                      head_pack: int = 0,
+                      head_pack: int = 0, tile_tokens: int = 0,
                       stream=None) -> torch.Tensor:
     """out[s, j] = softmax_t(scale * q[s, j] . K_t) . V_t over the sequence's paged tokens.
 
@@ -174,7 +174,7 @@ def paged_attn_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
     _need(context_lens, "context_lens", torch.int32, 1)
     _need(workspace, "workspace", torch.uint8, 1)
     S, Hq, D, NB, bs, Hkv = _decode_shapes(out, q, k_cache, v_cache, block_tables, context_lens)
-    opts = _Options(num_ctas, num_stages, ctas_per_sm, math, l2_prefetch, piece_cost, head_pack)
+    opts = _Options(num_ctas, num_stages, ctas_per_sm, math, l2_prefetch, piece_cost, head_pack, tile_tokens)
     _check("paged_attn_decode", library().paged_attn_decode_ex(
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
         S, Hq, Hkv, D, bs, float(scale), block_tables.shape[1], NB, _ptr(workspace), workspace.numel(),
@@ -187,7 +187,7 @@ def paged_attn_decode_append(out: torch.Tensor, q: torch.Tensor, k_new: torch.Te
                              block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float,
                              workspace: torch.Tensor, num_ctas: int = 0, num_stages: int = 0,
                              ctas_per_sm: int = 0, math: int = 0, l2_prefetch: int = 0, piece_cost: int = 0,
-                             head_pack: int = 0, stream=None) -> torch.Tensor:
+                             head_pack: int = 0, tile_tokens: int = 0, stream=None) -> torch.Tensor:
     """One decode step in one launch: append k_new / v_new (bf16 [S, Hkv, D]) at
     slot_mapping (int64 [S], the slot of each sequence's last position, < 0 =
     none), then the same attention as paged_attn_decode over contexts that
@@ -211,7 +211,7 @@ def paged_attn_decode_append(out: torch.Tensor, q: torch.Tensor, k_new: torch.Te
         raise ValueError("k_new / v_new must be [num_seqs, num_kv_heads, head_dim] and slot_mapping [num_seqs]")
     if block_tables.shape[0] != S or context_lens.shape[0] != S:
         raise ValueError("block_tables and context_lens must have num_seqs rows")
-    opts = _Options(num_ctas, num_stages, ctas_per_sm, math, l2_prefetch, piece_cost, head_pack)
+    opts = _Options(num_ctas, num_stages, ctas_per_sm, math, l2_prefetch, piece_cost, head_pack, tile_tokens)
     _check("paged_attn_decode_append", library().paged_attn_decode_append(
         _ptr(out), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(slot_mapping), _ptr(k_cache), _ptr(v_cache),
         _ptr(block_tables), _ptr(context_lens), S, Hq, Hkv, D, bs, float(scale), block_tables.shape[1], NB,

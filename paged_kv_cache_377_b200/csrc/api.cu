@@ -61,17 +61,20 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // Tensor map over a pool [num_blocks][bs][Hkv][D] of `es`-byte elements (bf16:
 // 2, e4m3 codes: 1) seen as 4D (128/es, D*es/128, Hkv, num_blocks*bs),
-// innermost first; one box = one 128-byte column slice of all bs rows of one
-// kv head of one block: (128/es, 1, 1, bs), 128-byte swizzled in shared memory
-// (a tile is D*es/128 such [bs][128 B] slices).
-int make_pool_map(CUtensorMap *map, const void *pool, int num_blocks, int bs, int hkv, int d, int es = 2) {
+// innermost first; one box = one 128-byte column slice of `rows` consecutive
+// token rows (a whole block, or a 16-row half of a 32-token block) of one kv
+// head: (128/es, 1, 1, rows), 128-byte swizzled in shared memory (a tile is
+// D*es/128 such [rows][128 B] slices).
+int make_pool_map(CUtensorMap *map, const void *pool, int num_blocks, int bs, int hkv, int d, int es = 2,
+                  int rows = 0) {
+    if (rows == 0) rows = bs;
     auto fn = encode_fn();
     if (!fn) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
     const cuuint64_t inner = 128 / es;
     cuuint64_t dims[4] = {inner, static_cast<cuuint64_t>(d) * es / 128, static_cast<cuuint64_t>(hkv),
                           static_cast<cuuint64_t>(num_blocks) * bs};
     cuuint64_t strides[3] = {128, static_cast<cuuint64_t>(d) * es, static_cast<cuuint64_t>(hkv) * d * es};
-    cuuint32_t box[4] = {static_cast<cuuint32_t>(inner), 1, 1, static_cast<cuuint32_t>(bs)};
+    cuuint32_t box[4] = {static_cast<cuuint32_t>(inner), 1, 1, static_cast<cuuint32_t>(rows)};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = fn(map, es == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
                     const_cast<void *>(pool), dims, strides, box, estr,
@@ -215,12 +218,14 @@ int decode_impl(void *out, const void *q, const void *k_new, const void *v_new, 
         !aligned(workspace, 256))
         return fail(PKV_ERR_INVALID_ARGUMENT,
                     "out, q, k_cache and v_cache must be 16-byte aligned and workspace 256-byte aligned");
-    pkv_decode_options o = {0, 0, 0, 0, 0, 0, 0};
+    pkv_decode_options o = {0, 0, 0, 0, 0, 0, 0, 0};
     if (opts) o = *opts;
     if (o.num_ctas < 0 || o.num_stages < 0 || o.ctas_per_sm < 0 || o.math < 0 || o.math > 2 ||
         o.l2_prefetch < -1 || o.l2_prefetch > 32 || o.piece_cost < -1 || o.piece_cost > 64 || o.head_pack < 0 ||
-        o.head_pack > 2)
+        o.head_pack > 2 || (o.tile_tokens != 0 && o.tile_tokens != 16 && o.tile_tokens != 32))
         return fail(PKV_ERR_INVALID_ARGUMENT, "negative or unknown option");
+    if (o.tile_tokens > block_size)
+        return fail(PKV_ERR_INVALID_ARGUMENT, "tile_tokens %d exceeds block_size %d", o.tile_tokens, block_size);
     if (o.num_ctas > pkv::kMaxCtas)
         return fail(PKV_ERR_INVALID_ARGUMENT, "num_ctas %d exceeds %d", o.num_ctas, pkv::kMaxCtas);
     if (static_cast<int64_t>(num_kv_heads) * (max_blocks_per_seq + 64) * pkv::kMaxSeqsPerLaunch > 0x7fffffff)
@@ -243,11 +248,15 @@ int decode_impl(void *out, const void *q, const void *k_new, const void *v_new, 
         return fail(PKV_ERR_UNSUPPORTED, "e4m3 pools need head_dim 128, or head_dim 64 with head packing (an even "
                                          "num_kv_heads and num_q_heads / num_kv_heads <= %d)", PKV_MAX_GROUP / 2);
     const int kd = head_dim * pack, khkv = num_kv_heads / pack, kgroup = group * pack;  // as the kernel sees them
-    const int ns = o.num_stages ? o.num_stages : default_stages(kd, block_size, math);
+    // Tiles of 16 token rows by default: a 32-token block is read as two tiles,
+    // so that a CTA's stages are as small as for 16-token blocks and as many
+    // CTAs fit on an SM.
+    const int tile = o.tile_tokens ? o.tile_tokens : 16;
+    const int ns = o.num_stages ? o.num_stages : default_stages(kd, tile, math);
     if (ns < 1 || ns > pkv::kMaxStagesPerWarp)
         return fail(PKV_ERR_INVALID_ARGUMENT, "num_stages %d outside [1, %d]", ns, pkv::kMaxStagesPerWarp);
     const int gp = group_pad(kgroup);
-    if (!pkv::decode_variant_exists(kd, block_size, gp, math))
+    if (!pkv::decode_variant_exists(kd, tile, gp, math))
         return fail(PKV_ERR_UNSUPPORTED, "no kernel for head_dim %d, block_size %d, group %d, math %d", head_dim,
                     block_size, group, math);
     const WorkspaceLayout wl = workspace_layout(num_seqs, num_q_heads, head_dim);
@@ -259,8 +268,8 @@ int decode_impl(void *out, const void *q, const void *k_new, const void *v_new, 
 
     CUtensorMap tm_k, tm_v;
     const int es = fp8 ? 1 : 2;
-    if ((rc = make_pool_map(&tm_k, k_cache, num_blocks, block_size, khkv, kd, es)) != PKV_OK) return rc;
-    if ((rc = make_pool_map(&tm_v, v_cache, num_blocks, block_size, khkv, kd, es)) != PKV_OK) return rc;
+    if ((rc = make_pool_map(&tm_k, k_cache, num_blocks, block_size, khkv, kd, es, tile)) != PKV_OK) return rc;
+    if ((rc = make_pool_map(&tm_v, v_cache, num_blocks, block_size, khkv, kd, es, tile)) != PKV_OK) return rc;
 
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -271,9 +280,9 @@ int decode_impl(void *out, const void *q, const void *k_new, const void *v_new, 
     // in shared memory); launches run in stream order and reuse the workspace.
     for (int s0 = 0; s0 < num_seqs; s0 += pkv::kMaxSeqsPerLaunch) {
         const int sc = num_seqs - s0 < pkv::kMaxSeqsPerLaunch ? num_seqs - s0 : pkv::kMaxSeqsPerLaunch;
-        const size_t smem = pkv::decode_smem_bytes(kd, block_size, gp, kgroup, math, ns, sc, pack);
+        const size_t smem = pkv::decode_smem_bytes(kd, tile, gp, kgroup, math, ns, sc, pack);
         int per_sm = 0;
-        cudaError_t e = pkv::decode_prepare(kd, block_size, gp, math, smem, &per_sm);
+        cudaError_t e = pkv::decode_prepare(kd, tile, gp, math, smem, &per_sm);
         if (e != cudaSuccess) return cuda_fail(e, "decode kernel setup");
         if (per_sm <= 0) return fail(PKV_ERR_INVALID_ARGUMENT, "shared memory %zu bytes per CTA does not fit", smem);
         if (o.ctas_per_sm > 0 && o.ctas_per_sm < per_sm) per_sm = o.ctas_per_sm;
@@ -294,6 +303,7 @@ int decode_impl(void *out, const void *q, const void *k_new, const void *v_new, 
         a.num_kv_heads = khkv;
         a.group = kgroup;
         a.pack = pack;
+        a.sub = block_size / tile;
         a.max_blocks_per_seq = max_blocks_per_seq;
         a.num_blocks = num_blocks;
         a.num_stages = ns;
@@ -310,7 +320,7 @@ int decode_impl(void *out, const void *q, const void *k_new, const void *v_new, 
         }
         a.k_scale = k_scale;
         a.v_scale = v_scale;
-        e = pkv::decode_launch(kd, block_size, gp, math, tm_k, tm_v, a, grid, smem, st);
+        e = pkv::decode_launch(kd, tile, gp, math, tm_k, tm_v, a, grid, smem, st);
         if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
     }
     return ok();

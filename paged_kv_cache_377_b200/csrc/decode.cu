@@ -207,8 +207,10 @@ struct CoreMath {
         }
     }
 
-    // One KV block: logits, block-wise online-softmax update, P.V.
-    __device__ __forceinline__ void block(uint32_t ktile, uint32_t vtile, int valid) {
+    // One KV tile in two steps: qk() -- logits and the block-wise online-softmax
+    // update, leaving the probabilities in the warp's scratch -- reads only the
+    // K tile; pv() -- P.V -- only the V tile.
+    __device__ __forceinline__ void qk(uint32_t ktile, int valid) {
 #pragma unroll
         for (int pass = 0; pass < NPASS; ++pass) {
             const int t = pass * TPP + tg;
@@ -270,7 +272,9 @@ struct CoreMath {
             }
         }
         __syncwarp();
+    }
 
+    __device__ __forceinline__ void pv(uint32_t vtile, int valid) {
         // P.V: tokens past the context are skipped, never multiplied by p = 0
 #pragma unroll
         for (int pass = 0; pass < NPASS; ++pass) {
@@ -378,7 +382,9 @@ struct MmaMath {
             for (int k = 0; k < 4; ++k) acc[dt][k] = 0.f;
     }
 
-    __device__ __forceinline__ void block(uint32_t ktile, uint32_t vtile, int valid) {
+    // One KV tile in two steps: qk() reads only the K tile (logits, online-softmax
+    // update, P into the warp's scratch), pv() only the V tile.
+    __device__ __forceinline__ void qk(uint32_t ktile, int valid) {
         const int mi = lane >> 3, r = lane & 7;
         const int tr = lane >> 2;  // fragment row of this lane
         // S^T = K . Q^T; ldmatrix x4 gives the A fragment (rows t, cols d) of one k-step
@@ -448,7 +454,10 @@ struct MmaMath {
         m0 = n0;
         m1 = n1;
         __syncwarp();
+    }
 
+    __device__ __forceinline__ void pv(uint32_t vtile, int valid) {
+        const int mi = lane >> 3, r = lane & 7;
         // O^T += V^T . P^T; ldmatrix x4 .trans gives the A fragment (rows d, cols t)
 #pragma unroll
         for (int ks = 0; ks < TT; ++ks) {
@@ -650,7 +659,8 @@ struct Fp8Math {
             for (int k = 0; k < 4; ++k) acc[dt][k] = 0.f;
     }
 
-    __device__ __forceinline__ void block(uint32_t ktile, uint32_t vtile, int valid) {
+    // One KV tile in two steps, as in MmaMath: qk() reads only the K tile, pv() only the V tile.
+    __device__ __forceinline__ void qk(uint32_t ktile, int valid) {
         const int mi = lane >> 3, r = lane & 7;
         const int tr = lane >> 2;
         // S^T = K . Q^T; one ldmatrix x4 covers tokens 0-15 of two 16-dim chunks
@@ -728,7 +738,10 @@ struct Fp8Math {
         m0 = n0;
         m1 = n1;
         __syncwarp();
+    }
 
+    __device__ __forceinline__ void pv(uint32_t vtile, int valid) {
+        const int mi = lane >> 3, r = lane & 7;
         // O^T += V^T . P^T; one ldmatrix x4 .trans covers tokens 0-15 of two dim tiles
 #pragma unroll
         for (int ks = 0; ks < TT; ++ks) {
@@ -817,9 +830,9 @@ struct Fp8Math {
 
 struct Smem {
     uint8_t *base;
-    uint64_t *full, *qfull;
+    uint64_t *full, *full_v, *qfull;  // per stage: K tile landed, V tile landed; query slots
     volatile int *stage_bad;
-    int *stage_blk;  // [kMaxStages] physical block whose copy the stage holds
+    int *stage_blk;  // [kMaxStages] first pool row of the tile whose copy the stage holds
     volatile int *abort_flag;
     volatile int *merge_flag;  // [1 + 2 * 2]: how many segments this CTA completed (<= 2), then
                                // (s, h) of each
@@ -938,7 +951,11 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
     // ---- issue side: this warp's blocks k = 0 .. nk-1 are global blocks x0 + warp + 4k
     const long long span = x1 - x0;
     const int nk = span > warp ? static_cast<int>((span - warp + kConsumerWarps - 1) / kConsumerWarps) : 0;
-    auto lookup = [&](int kb, int &p, int &h) {  // lane j: block kb + j -> (physical block, kv head)
+    // Tile j of a segment is rows [j % sub * BS, +BS) of the pool block in table
+    // entry j / sub; a tile is addressed by its first pool row, -1 if the table
+    // entry is not a block of the pool.
+    const int sub_shift = a.sub == 2 ? 1 : 0;
+    auto lookup = [&](int kb, int &p, int &h) {  // lane j: tile kb + j -> (first pool row or -1, kv head)
         p = 0;
         h = 0;
         const int k = kb + lane;
@@ -953,16 +970,23 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
             const int n = sm.prefix[lo + 1] - sm.prefix[lo];
             const int r = static_cast<int>(x - static_cast<long long>(a.num_kv_heads) * sm.prefix[lo]);
             h = r / n;
-            p = __ldg(a.block_tables + static_cast<size_t>(lo) * a.max_blocks_per_seq + (r - h * n));
+            const int j = r - h * n;
+            const int pb = __ldg(a.block_tables + static_cast<size_t>(lo) * a.max_blocks_per_seq + (j >> sub_shift));
+            p = (pb < 0 || pb >= a.num_blocks) ? -1 : ((pb << sub_shift) + (j & (a.sub - 1))) * BS;
         }
     };
     int bat_k = 0, bat_p, bat_h, nxt_p, nxt_h;
     lookup(0, bat_p, bat_h);
     lookup(32, nxt_p, nxt_h);
-    uint32_t inflight = 0, inflight_par = 0;  // stages whose copy this warp issued and has not yet seen land
+    // Copies this warp issued and has not yet seen land: bit `stage` of the K
+    // (low 16 bits) and V (high 16 bits) halves, with the phase parity each waits for.
+    uint32_t inflight = 0, inflight_par = 0;
     // Block k goes to stage warp + 4 (k % R) with phase parity (k / R) & 1, so
-    // block k + R reuses block k's stage with the other parity.
-    auto issue = [&](int k, int stage, uint32_t par) {  // warp-uniform; k increases call after call
+    // block k + R reuses block k's stage with the other parity. The K and V
+    // tiles of a stage complete on their own barriers (full, full_v): the K tile
+    // is refilled as soon as q.K is done, while P.V still reads the V tile.
+    int iss_p = 0, iss_h = 0;  // the last K copy's block, for the V copy that follows it
+    auto issue_k = [&](int k, int stage, uint32_t par) {  // warp-uniform; k increases call after call
         if (k >= nk) return;
         if (k - bat_k >= 32) {
             bat_k += 32;
@@ -972,42 +996,61 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
         }
         const int p = __shfl_sync(0xffffffffu, bat_p, k - bat_k);
         const int h = __shfl_sync(0xffffffffu, bat_h, k - bat_k);
+        iss_p = p;
+        iss_h = h;
         if (a.prefetch > 0) {  // this warp's block k + prefetch, from the current or the next batch (<= 32 ahead)
             const int kp = k + a.prefetch, jp = kp - bat_k;
             const int pp_a = __shfl_sync(0xffffffffu, bat_p, jp & 31), pp_b = __shfl_sync(0xffffffffu, nxt_p, jp & 31);
             const int hp_a = __shfl_sync(0xffffffffu, bat_h, jp & 31), hp_b = __shfl_sync(0xffffffffu, nxt_h, jp & 31);
             const int pp = jp < 32 ? pp_a : pp_b, hp = jp < 32 ? hp_a : hp_b;
-            if (lane == 0 && kp < nk && pp >= 0 && pp < a.num_blocks && !*sm.abort_flag) {
+            if (lane == 0 && kp < nk && pp >= 0 && !*sm.abort_flag) {
 #pragma unroll
                 for (int half = 0; half < kCopies; ++half) {
-                    tma_prefetch_l2_4d(tm_k, 0, half, hp, pp * BS);
-                    tma_prefetch_l2_4d(tm_v, 0, half, hp, pp * BS);
+                    tma_prefetch_l2_4d(tm_k, 0, half, hp, pp);
+                    tma_prefetch_l2_4d(tm_v, 0, half, hp, pp);
                 }
             }
         }
         if (lane == 0 && !*sm.abort_flag) {
-            const bool bad = p < 0 || p >= a.num_blocks;
+            const bool bad = p < 0;
             sm.stage_bad[stage] = bad ? 1 : 0;
             sm.stage_blk[stage] = p;
             if (bad) {
                 atomicOr(a.status, PKV_STATUS_BAD_BLOCK_ID);
                 mbar_arrive(&sm.full[stage]);
             } else {
-                // The stage's previous contents were read with ldmatrix / ld.shared whose
+                // The tile's previous contents were read with ldmatrix / ld.shared whose
                 // results this warp has already consumed, so the copy cannot overtake them.
                 uint8_t *dst = sm.base + ly.stages + static_cast<uint32_t>(stage) * 2u * kTile;
-                mbar_arrive_expect_tx(&sm.full[stage], 2u * kTile);
+                mbar_arrive_expect_tx(&sm.full[stage], kTile);
 #pragma unroll
-                for (int half = 0; half < kCopies; ++half) {
-                    tma_load_4d(dst + half * kHalf, tm_k, &sm.full[stage], 0, half, h, p * BS);
-                    tma_load_4d(dst + kTile + half * kHalf, tm_v, &sm.full[stage], 0, half, h, p * BS);
-                }
+                for (int half = 0; half < kCopies; ++half)
+                    tma_load_4d(dst + half * kHalf, tm_k, &sm.full[stage], 0, half, h, p);
                 inflight |= 1u << stage;
                 inflight_par = (inflight_par & ~(1u << stage)) | (par << stage);
             }
         }
     };
-    for (int k = 0; k < R; ++k) issue(k, warp + kConsumerWarps * k, 0u);
+    auto issue_v = [&](int k, int stage, uint32_t par) {  // the V tile of the block issue_k(k) fetched
+        if (k >= nk) return;
+        if (lane == 0 && !*sm.abort_flag) {
+            if (iss_p < 0) {
+                mbar_arrive(&sm.full_v[stage]);
+            } else {
+                uint8_t *dst = sm.base + ly.stages + static_cast<uint32_t>(stage) * 2u * kTile + kTile;
+                mbar_arrive_expect_tx(&sm.full_v[stage], kTile);
+#pragma unroll
+                for (int half = 0; half < kCopies; ++half)
+                    tma_load_4d(dst + half * kHalf, tm_v, &sm.full_v[stage], 0, half, iss_h, iss_p);
+                inflight |= 1u << (16 + stage);
+                inflight_par = (inflight_par & ~(1u << (16 + stage))) | (par << (16 + stage));
+            }
+        }
+    };
+    for (int k = 0; k < R; ++k) {
+        issue_k(k, warp + kConsumerWarps * k, 0u);
+        issue_v(k, warp + kConsumerWarps * k, 0u);
+    }
 
     // ---- query rows: warp 0 copies piece n + 1's rows while piece n is computed
     uint32_t q_issued = 0, q_issued_par = 0;
@@ -1069,40 +1112,55 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
                 slot = __ldg(a.slots + pc.s);
                 if (ES == 2 && slot >= 0 && lane < 2 * kChunks) patch = __ldg(patch_src());
             }
+            const int valid = min(BS, pc.L - bi * BS);
+            const uint32_t ktile = sbase + ly.stages + static_cast<uint32_t>(stage) * 2u * kTile;
+            // this lane's chunk of the new row goes into the staged tile and the pool
+            auto put_row = [&](long long want, int t) {
+                const int c = lane % kChunks;
+                uint4 row;
+                if constexpr (ES == 2) {
+                    row = patch;
+                } else {  // quantize: element d of real head r -> e4m3(x / scale[r])
+                    const int real = pc.h * a.pack + (c * kElems) / (D / a.pack);
+                    const float sc = __ldg((lane < kChunks ? a.k_scale : a.v_scale) + real);
+                    const uint4 *src = patch_src();
+                    row = quantize16_e4m3(__ldg(src), __ldg(src + 1), sc);
+                }
+                sts128(tile_addr<BS>(lane < kChunks ? ktile : ktile + kTile, t, c), row);
+                *reinterpret_cast<uint4 *>(static_cast<uint8_t *>(lane < kChunks ? a.k_cache : a.v_cache) +
+                                           ((static_cast<size_t>(want) * a.num_kv_heads + pc.h) * D) * ES + c * 16) =
+                    row;
+                fence_proxy_async_shared();  // before a later copy overwrites the tile
+            };
             if (mbar_wait_bounded(&sm.full[stage], par, sm.abort_flag, a.status)) inflight &= ~(1u << stage);
-            if (!sm.stage_bad[stage] && !*sm.abort_flag) {
-                const int valid = min(BS, pc.L - bi * BS);
-                const uint32_t ktile = sbase + ly.stages + static_cast<uint32_t>(stage) * 2u * kTile;
+            const bool live = !sm.stage_bad[stage] && !*sm.abort_flag;
+            long long want = -1;  // the slot this block's new row goes to, if it takes one
+            if (live) {
                 if (tail && slot >= 0) {
-                    const int t = valid - 1;  // row of position L - 1 in this block
-                    const long long want = static_cast<long long>(sm.stage_blk[stage]) * BS + t;
-                    if (slot == want) {
-                        if (lane < 2 * kChunks) {
-                            const int c = lane % kChunks;
-                            uint4 row;
-                            if constexpr (ES == 2) {
-                                row = patch;
-                            } else {  // quantize: element d of real head r -> e4m3(x / scale[r])
-                                const int real = pc.h * a.pack + (c * kElems) / (D / a.pack);
-                                const float sc = __ldg((lane < kChunks ? a.k_scale : a.v_scale) + real);
-                                const uint4 *src = patch_src();
-                                row = quantize16_e4m3(__ldg(src), __ldg(src + 1), sc);
-                            }
-                            sts128(tile_addr<BS>(lane < kChunks ? ktile : ktile + kTile, t, c), row);
-                            *reinterpret_cast<uint4 *>(static_cast<uint8_t *>(lane < kChunks ? a.k_cache : a.v_cache) +
-                                                       ((static_cast<size_t>(want) * a.num_kv_heads + pc.h) * D) * ES +
-                                                       c * 16) = row;
-                            fence_proxy_async_shared();  // before a later copy overwrites the stage
-                        }
-                        __syncwarp();
-                    } else if (lane == 0) {
-                        atomicOr(a.status, PKV_STATUS_BAD_SLOT);  // not the last position: not appended
+                    want = static_cast<long long>(sm.stage_blk[stage]) + (valid - 1);  // row of position L - 1
+                    if (slot != want) {
+                        want = -1;
+                        if (lane == 0) atomicOr(a.status, PKV_STATUS_BAD_SLOT);  // not the last position: not appended
                     }
                 }
-                math.block(ktile, ktile + kTile, valid);
+                if (want >= 0) {
+                    if (lane < kChunks) put_row(want, valid - 1);
+                    __syncwarp();
+                }
+                math.qk(ktile, valid);
             }
             __syncwarp();
-            issue(k + R, stage, par ^ 1u);  // the stage just freed takes this warp's block k + R
+            issue_k(k + R, stage, par ^ 1u);  // the K tile just read takes this warp's block k + R
+            if (mbar_wait_bounded(&sm.full_v[stage], par, sm.abort_flag, a.status)) inflight &= ~(1u << (16 + stage));
+            if (live && !*sm.abort_flag) {
+                if (want >= 0) {
+                    if (lane >= kChunks && lane < 2 * kChunks) put_row(want, valid - 1);
+                    __syncwarp();
+                }
+                math.pv(ktile + kTile, valid);
+            }
+            __syncwarp();
+            issue_v(k + R, stage, par ^ 1u);  // and its V tile
         }
         gb_base += nblk;
 
@@ -1170,8 +1228,11 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
     // Leave no copy in flight into shared memory when the CTA exits (only
     // possible after a wait gave up).
     if (lane == 0) {
-        for (int st = 0; st < kMaxStages; ++st)
+        for (int st = 0; st < kMaxStages; ++st) {
             if ((inflight >> st) & 1u) mbar_wait_drain(&sm.full[st], (inflight_par >> st) & 1u, a.status);
+            if ((inflight >> (16 + st)) & 1u)
+                mbar_wait_drain(&sm.full_v[st], (inflight_par >> (16 + st)) & 1u, a.status);
+        }
         // the last copy into each query slot: landed already unless a wait gave up
         if (warp == 0)
             for (int slot = 0; slot < 2; ++slot)
@@ -1221,7 +1282,8 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathCudaCore ? 1 : (M
     Smem sm;
     sm.base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     sm.full = reinterpret_cast<uint64_t *>(sm.base + ly.bars);
-    sm.qfull = sm.full + kMaxStages;
+    sm.full_v = sm.full + kMaxStages;
+    sm.qfull = sm.full_v + kMaxStages;
     sm.stage_bad = reinterpret_cast<volatile int *>(sm.base + ly.flags);
     sm.abort_flag = sm.stage_bad + kMaxStages;
     sm.scan = reinterpret_cast<int *>(sm.base + ly.flags) + kMaxStages + 1;
@@ -1235,6 +1297,7 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathCudaCore ? 1 : (M
     if (tid == 0) {
         for (int i = 0; i < kConsumerWarps * a.num_stages; ++i) {
             mbar_init(&sm.full[i], 1);
+            mbar_init(&sm.full_v[i], 1);
             sm.stage_bad[i] = 0;
         }
         for (int i = 0; i < 2; ++i) mbar_init(&sm.qfull[i], 1);
@@ -1250,7 +1313,7 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathCudaCore ? 1 : (M
     // prefix[s] = blocks of sequences < s (clamped lengths), wprefix[s] = their
     // weight (blocks + piece_cost per non-empty sequence); lens[s] = clamped length
     const int S = a.num_seqs;
-    const int cap = a.max_blocks_per_seq * BS;
+    const int cap = a.max_blocks_per_seq * BS * a.sub;
     const int pcost = min(max(a.piece_cost, 0), 64);  // validated on the host; a bad value moves no index
     const int per = (S + kDecodeThreads - 1) / kDecodeThreads;
     const int lo = min(S, tid * per), hi = min(S, lo + per);
@@ -1303,8 +1366,9 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathCudaCore ? 1 : (M
         sm.wprefix[S] = total_w;
     }
     __syncthreads();
-    if (blockIdx.x == 0)  // sequences with no context get all-zero rows (no piece covers them)
-        for (int s = 0; s < S; ++s)
+    // Sequences with no context get all-zero rows (no piece covers them); CTA c
+    // takes sequences c, c + C, ... so that no CTA walks the whole batch.
+    for (int s = blockIdx.x; s < S; s += gridDim.x)
             if (sm.lens[s] == 0) {
                 for (int e = tid; e < a.num_q_heads * (D / a.pack) / 2; e += kDecodeThreads)
                     reinterpret_cast<__nv_bfloat162 *>(static_cast<__nv_bfloat16 *>(a.out) +
@@ -1313,7 +1377,7 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathCudaCore ? 1 : (M
                 // fused append of a sequence with no context: no block computes it,
                 // so its rows go straight to the pool (if the slot is in it)
                 const long long slot = a.slots ? __ldg(a.slots + s) : -1;
-                if (slot >= static_cast<long long>(a.num_blocks) * BS) {
+                if (slot >= static_cast<long long>(a.num_blocks) * BS * a.sub) {
                     if (tid == 0) atomicOr(a.status, PKV_STATUS_BAD_SLOT);
                 } else if (slot >= 0) {
                     const size_t row = static_cast<size_t>(a.num_kv_heads) * D;  // elements of one token's row

@@ -40,6 +40,7 @@ struct DecodeArgs {
     int prefetch;                // blocks a warp prefetches into L2 beyond the one it loads (0 = none)
     int piece_cost;              // extra weight, in blocks, of every non-empty segment when splitting work
     int pack;                    // 1, or 2: two real kv heads per virtual head (see above)
+    int sub;                     // tiles per pool block: 1, or 2 (a 32-token block read as two 16-token tiles)
     // Fused append (slots != nullptr): the step's new token of sequence s, rows
     // k_new[s][h] / v_new[s][h] ([S][Hkv][D] like a pool row), belongs at
     // slots[s], which must be the slot of position L_s - 1. The warp that
@@ -89,7 +90,7 @@ __host__ __device__ inline DecodeLayout decode_layout(int D, int BS, int GP, int
     off += kConsumerWarps * G * 4;
     off = align_up(off, 8);
     L.bars = off;
-    off += (kMaxStages + 2) * 8;                                    // full[stage], qfull[2]
+    off += (2 * kMaxStages + 2) * 8;                                // full[stage], full_v[stage], qfull[2]
     L.flags = off;
     off += (2 * kMaxStages + 1 + 2 * kConsumerWarps + 1 + 4 * 2) * 4;  // stage_bad, abort, scan, merges, stage_blk
     L.prefix = off;

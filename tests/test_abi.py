@@ -110,6 +110,15 @@ def test_options_are_checked():
     rc = lib.paged_attn_decode_ex(P, P, P, P, P, P, 4, 8, 2, 128, 16, 0.125, 3, 16, P, 1 << 20,
                                   ctypes.byref(opts), None)
     assert rc == -2 and "head_pack" in lib.pkv_last_error().decode()
+    # tiles of 16 or 32 token rows, never more than a block
+    opts = pkv._binding._Options(0, 0, 0, 0, 0, 0, 0, 24)
+    rc = lib.paged_attn_decode_ex(P, P, P, P, P, P, 4, 2, 1, 64, 32, 0.125, 3, 16, P, 1 << 20,
+                                  ctypes.byref(opts), None)
+    assert rc == -1 and "unknown option" in lib.pkv_last_error().decode()
+    opts = pkv._binding._Options(0, 0, 0, 0, 0, 0, 0, 32)
+    rc = lib.paged_attn_decode_ex(P, P, P, P, P, P, 4, 2, 1, 64, 16, 0.125, 3, 16, P, 1 << 20,
+                                  ctypes.byref(opts), None)
+    assert rc == -1 and "tile_tokens" in lib.pkv_last_error().decode()
 
 
 def test_fused_step_checks_its_extra_arguments():

@@ -73,6 +73,18 @@ def test_grid_sizes_split_contexts_differently(name, num_ctas, math):
     assert_close_to_oracle(out.double().numpy(), ref, what=f"{name} num_ctas={num_ctas}")
 
 
+@pytest.mark.parametrize("math", MATHS)
+@pytest.mark.parametrize("tile", [16, 32])
+@pytest.mark.parametrize("num_ctas", [0, 1, 1024])
+def test_block_size_32_read_as_whole_or_half_tiles(math, tile, num_ctas):
+    """32-token blocks are read as two 16-row tiles by default, or whole (tile_tokens 32)."""
+    b, ref, kc_ref, vc_ref = config_case("skewed_long")
+    out, kc, vc, st = run_step(b, math=math, tile_tokens=tile, num_ctas=num_ctas)
+    assert st == 0
+    assert np.array_equal(bf16_bits(kc), kc_ref) and np.array_equal(bf16_bits(vc), vc_ref)
+    assert_close_to_oracle(out.double().numpy(), ref, what=f"skewed_long tile={tile} C={num_ctas} math={math}")
+
+
 @pytest.mark.parametrize("opts", [dict(num_stages=1), dict(num_stages=2), dict(num_stages=4), dict(ctas_per_sm=1),
                                   dict(num_stages=3, ctas_per_sm=2, num_ctas=100),
                                   dict(math=2, num_stages=1), dict(math=2, num_stages=4, ctas_per_sm=1),
@@ -104,12 +116,14 @@ def test_every_group_size_and_shape(G, D, bs):
     b = workloads.make_custom(1000 + G * 7 + D + bs, lens, 2 * G, 2, D, bs)
     ref, _, _ = oracle.decode_step(b)
     # head_pack 0 packs kv-head pairs where it can (tensor cores, D 64, G <= 4); 1 never does
+    tiles = (16, 32) if bs == 32 else (16,)
     for math, pack in [(1, 0), (2, 0), (2, 1)]:
         for num_ctas in (0, 37):
-            out, _, _, st = run_step(b, num_ctas=num_ctas, math=math, head_pack=pack)
-            assert st == 0
-            assert_close_to_oracle(out.double().numpy(), ref,
-                                   what=f"G={G} D={D} bs={bs} C={num_ctas} math={math} pack={pack}")
+            for tile in tiles:
+                out, _, _, st = run_step(b, num_ctas=num_ctas, math=math, head_pack=pack, tile_tokens=tile)
+                assert st == 0
+                assert_close_to_oracle(out.double().numpy(), ref,
+                                       what=f"G={G} D={D} bs={bs} C={num_ctas} math={math} pack={pack} tile={tile}")
 
 
 @pytest.mark.parametrize("math", MATHS)

@@ -96,10 +96,11 @@ def test_fp8_every_supported_group_and_shape(G, D, bs):
         return
     ref, kc_ref, vc_ref = oracle.decode_step(b)
     for num_ctas in (0, 37):
-        out, kc, vc, st = one_launch(b, num_ctas=num_ctas)
-        assert st == 0
-        assert np.array_equal(kc.numpy(), kc_ref) and np.array_equal(vc.numpy(), vc_ref)
-        assert_close_to_oracle(out.double().numpy(), ref, what=f"fp8 G={G} D={D} bs={bs} C={num_ctas}")
+        for tile in ((16, 32) if bs == 32 else (16,)):
+            out, kc, vc, st = one_launch(b, num_ctas=num_ctas, tile_tokens=tile)
+            assert st == 0
+            assert np.array_equal(kc.numpy(), kc_ref) and np.array_equal(vc.numpy(), vc_ref)
+            assert_close_to_oracle(out.double().numpy(), ref, what=f"fp8 G={G} D={D} bs={bs} C={num_ctas} tile={tile}")
 
 
 @pytest.mark.parametrize("name", ["llama3_8b", "skewed_long"])

@@ -76,12 +76,14 @@ def test_fused_step_matches_oracle_and_the_two_launch_step(name, math):
 
 @pytest.mark.parametrize("opts", [dict(num_ctas=1), dict(num_ctas=7), dict(num_ctas=300), dict(num_ctas=1024),
                                   dict(head_pack=1), dict(head_pack=2, num_ctas=999), dict(num_stages=2),
-                                  dict(math=1, num_ctas=1024)])
+                                  dict(math=1, num_ctas=1024), dict(tile_tokens=32), dict(tile_tokens=32, num_ctas=1)])
 @pytest.mark.parametrize("name", ["opt125m", "skewed_long", "qwen25_7b_prefix"])
 def test_fused_step_is_bitwise_the_two_launch_step_under_every_split(name, opts):
     b, _ = case(name)
     if "head_pack" in opts and b.head_dim != 64:
         pytest.skip("head packing needs head_dim 64")
+    if opts.get("tile_tokens", 0) > b.block_size:
+        pytest.skip("tiles of 32 rows need 32-token blocks")
     out, kc, vc, st = fused(b, **opts)
     out2, kc2, vc2, st2 = unfused(b, **opts)
     assert st == 0 and st2 == 0
