@@ -73,6 +73,9 @@ def parse_args(argv=None):
     p.add_argument("--piece-cost", type=int, default=0)
     p.add_argument("--head-pack", type=int, default=0)
     p.add_argument("--tile-tokens", type=int, default=0)
+    p.add_argument("--prefix-groups", choices=["auto", "off"], default="auto",
+                   help="auto: pass the runs of sequences that share leading blocks (found on the host tables, "
+                        "as an engine's block manager knows them) so that shared blocks are read once per group")
     p.add_argument("--two-launch", action="store_true",
                    help="run the step as kv_cache_append + paged_attn_decode instead of the one-launch call")
     p.add_argument("--seqs", type=int, default=0,
@@ -273,6 +276,12 @@ class Step:
         self.opts = dict(num_ctas=args.num_ctas, num_stages=args.num_stages,
                          ctas_per_sm=args.ctas_per_sm, math=args.math, l2_prefetch=args.l2_prefetch,
                          piece_cost=args.piece_cost, head_pack=args.head_pack, tile_tokens=args.tile_tokens)
+        self.groups = None
+        if getattr(args, "prefix_groups", "off") == "auto" and b.kv_dtype == "bf16":
+            g = pkv.find_prefix_groups(b.block_tables, b.context_lens, b.block_size)
+            if len(g):
+                self.groups = g
+                self.opts["prefix_groups"] = g
         self.ws = pkv.allocate_workspace(b.num_seqs, b.num_q_heads, b.head_dim, device=device)
         self.fp8 = b.kv_dtype == "fp8"
         if self.fp8:
@@ -336,6 +345,9 @@ def run_ours(args, rank, world, local_rank):
     batch = workloads.make_batch(args.workload, seed=rank_seed(cfg.seed, rank), device=device, poison=False,
                                  lens_override=lens, kv_dtype=args.kv_dtype)
     step = Step(batch, args, device)
+    args.groups_desc = (None if step.groups is None else
+                        {"begin": step.groups.begin.tolist(), "end": step.groups.end.tolist(),
+                         "blocks": step.groups.blocks.tolist()})
     kv = workloads.kv_bytes(batch)
     ctx_tokens = int(batch.context_lens.sum())
     S = batch.num_seqs
@@ -511,6 +523,7 @@ def config_block(args, batch, world):
         "unique_kv_bytes_per_step": workloads.unique_kv_bytes(batch),
         "kv_dtype": batch.kv_dtype,
         "l2": getattr(args, "l2_policy", "L2 flushed (memset 2x L2) between timed steps"),
+        "prefix_groups": getattr(args, "groups_desc", None),
         "parallelism": "replicas: one independent batch per GPU" if world > 1 else "single GPU",
         "step": ("kv_cache_append + paged_attn_decode (two launches)" if args.two_launch else
                  "paged_attn_decode_append (append + attention, one launch)"),

@@ -58,6 +58,7 @@ extern "C" {
 #define PKV_STATUS_BAD_CONTEXT_LEN 2  /* context_lens[s] < 0 or > max_blocks_per_seq * block_size; clamped */
 #define PKV_STATUS_WAIT_TIMEOUT 4     /* a bounded wait inside a kernel gave up; outputs are not valid */
 #define PKV_STATUS_BAD_SLOT 8         /* an append slot is >= num_blocks * block_size; that token is skipped */
+#define PKV_STATUS_BAD_PREFIX_GROUP 16 /* a prefix-group member's table differs from the group's shared blocks */
 
 /* Supported shapes of the decode kernels. */
 #define PKV_MAX_GROUP 8               /* num_q_heads / num_kv_heads <= 8 */
@@ -100,6 +101,36 @@ extern "C" {
  *                     an SM; more than block_size returns PKV_ERR_INVALID_ARGUMENT.
  *                     The result does not depend on it beyond rounding order.
  */
+/*
+ * Prefix groups: runs of consecutive sequences of a batch whose block tables
+ * start with the same physical blocks -- a shared system prompt, or the
+ * parallel samples and beam candidates of one prompt, which share the blocks
+ * of their common tokens ("Deep Dive into vLLM", section 2.2, Flexible
+ * Sharing; runbyai.xyz post 449, section 3). Group g is sequences begin[g] ..
+ * end[g] - 1 (at least two), whose tables agree on entries 0 .. blocks[g] - 1;
+ * groups are disjoint and in increasing order (begin[g + 1] >= end[g]). Given as pkv_decode_options.prefix_groups, the decode reads
+ * those shared blocks once per group and kv head for all the group's query
+ * rows (up to 64 rows per CTA) instead of once per sequence, and merges them
+ * with each sequence's own blocks by the log-sum-exp identity; the result is
+ * the same attention (up to rounding order). A member whose context ends
+ * inside the shared blocks attends only to its own tokens.
+ * The kernel checks that each member's table entries equal the group's first
+ * sequence's (for the tokens the member attends) and sets
+ * PKV_STATUS_BAD_PREFIX_GROUP otherwise (that member's output is then wrong).
+ * Used with bf16 pools on tensor cores (math 0 or 2) with 16-row tiles; head
+ * packing is not applied to a batch with groups. At most PKV_MAX_PREFIX_GROUPS
+ * groups per 2048 sequences; groups beyond that, groups a 2048-sequence launch
+ * boundary leaves with one member, and batches whose workspace has no room
+ * for the group partials are decoded without the grouping (same results).
+ */
+#define PKV_MAX_PREFIX_GROUPS 16
+typedef struct pkv_prefix_groups {
+    int num_groups;
+    const int32_t *begin;   /* host [num_groups]: first sequence of each group */
+    const int32_t *end;     /* host [num_groups]: one past its last; begin + 2 <= end <= next begin, <= num_seqs */
+    const int32_t *blocks;  /* host [num_groups]: shared leading table entries, 1 .. max_blocks_per_seq */
+} pkv_prefix_groups;
+
 typedef struct pkv_decode_options {
     int num_ctas;
     int num_stages;
@@ -109,7 +140,21 @@ typedef struct pkv_decode_options {
     int piece_cost;
     int head_pack;
     int tile_tokens;
+    const pkv_prefix_groups *prefix_groups;  /* NULL: none */
 } pkv_decode_options;
+
+/*
+ * Finds prefix groups in host copies of a batch's tables (for example the
+ * rows pkv_bm_pack produced): maximal runs, scanned from the first sequence,
+ * of at least two consecutive sequences whose tables agree on at least
+ * min_blocks leading entries that every member's context covers; blocks[g] is
+ * the run's longest such agreement. Writes at most max_groups groups into
+ * begin[], end[], blocks[] and sets *num_groups. Host only; returns PKV_OK or
+ * PKV_ERR_INVALID_ARGUMENT.
+ */
+int pkv_find_prefix_groups(const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
+                           int max_blocks_per_seq, int block_size, int min_blocks, int32_t *begin, int32_t *end,
+                           int32_t *blocks, int max_groups, int *num_groups);
 
 /*
  * Bytes of device workspace paged_attn_decode needs for this shape

@@ -9,12 +9,16 @@ nvcc), every call raises: there is no CPU fallback.
 from __future__ import annotations
 
 from ._binding import (  # noqa: F401
+    PKV_MAX_PREFIX_GROUPS,
     PKV_STATUS_BAD_BLOCK_ID,
     PKV_STATUS_BAD_CONTEXT_LEN,
+    PKV_STATUS_BAD_PREFIX_GROUP,
     PKV_STATUS_BAD_SLOT,
     PKV_STATUS_WAIT_TIMEOUT,
     PagedKVError,
+    PrefixGroups,
     allocate_workspace,
+    find_prefix_groups,
     kv_cache_append,
     kv_cache_append_fp8,
     library,
@@ -35,7 +39,9 @@ __all__ = [
     "BlockManager",
     "OutOfBlocks",
     "PagedKVError",
+    "PrefixGroups",
     "allocate_workspace",
+    "find_prefix_groups",
     "kv_block_copy",
     "kv_cache_append",
     "library",

@@ -7,6 +7,7 @@ import os
 import threading
 from typing import Optional
 
+import numpy as np
 import torch
 
 from . import build as _build
@@ -16,6 +17,8 @@ PKV_STATUS_BAD_BLOCK_ID = 1
 PKV_STATUS_BAD_CONTEXT_LEN = 2
 PKV_STATUS_WAIT_TIMEOUT = 4
 PKV_STATUS_BAD_SLOT = 8
+PKV_STATUS_BAD_PREFIX_GROUP = 16
+PKV_MAX_PREFIX_GROUPS = 16
 
 _lock = threading.Lock()
 _lib: Optional[ctypes.CDLL] = None
@@ -29,10 +32,68 @@ class PagedKVError(RuntimeError):
         self.code = code
 
 
+class _PrefixGroups(ctypes.Structure):
+    _fields_ = [("num_groups", ctypes.c_int), ("begin", ctypes.c_void_p), ("end", ctypes.c_void_p),
+                ("blocks", ctypes.c_void_p)]
+
+
 class _Options(ctypes.Structure):
     _fields_ = [("num_ctas", ctypes.c_int), ("num_stages", ctypes.c_int),
                 ("ctas_per_sm", ctypes.c_int), ("math", ctypes.c_int), ("l2_prefetch", ctypes.c_int),
-                ("piece_cost", ctypes.c_int), ("head_pack", ctypes.c_int), ("tile_tokens", ctypes.c_int)]
+                ("piece_cost", ctypes.c_int), ("head_pack", ctypes.c_int), ("tile_tokens", ctypes.c_int),
+                ("prefix_groups", ctypes.c_void_p)]
+
+
+class PrefixGroups:
+    """Runs of consecutive sequences sharing their leading blocks (pkv_prefix_groups):
+    group g is sequences begin[g] .. end[g] - 1, sharing table entries 0 .. blocks[g] - 1."""
+
+    def __init__(self, begin, end, blocks):
+        self.begin = np.ascontiguousarray(begin, dtype=np.int32)
+        self.end = np.ascontiguousarray(end, dtype=np.int32)
+        self.blocks = np.ascontiguousarray(blocks, dtype=np.int32)
+        if not (len(self.begin) == len(self.end) == len(self.blocks)):
+            raise ValueError("begin, end and blocks must have one entry per group")
+        self._c = _PrefixGroups(len(self.begin), self.begin.ctypes.data, self.end.ctypes.data,
+                                self.blocks.ctypes.data)
+
+    def __len__(self):
+        return len(self.begin)
+
+    def __repr__(self):
+        return f"PrefixGroups(begin={self.begin.tolist()}, end={self.end.tolist()}, blocks={self.blocks.tolist()})"
+
+    def c_ptr(self):
+        return ctypes.addressof(self._c) if len(self) else None
+
+
+def find_prefix_groups(block_tables, context_lens, block_size: int, min_blocks: int = 1,
+                       max_groups: int = PKV_MAX_PREFIX_GROUPS) -> PrefixGroups:
+    """pkv_find_prefix_groups on HOST copies of a batch's tables (int32 [S][MB]) and lengths (int32 [S])."""
+    bt = np.ascontiguousarray(block_tables.cpu().numpy() if isinstance(block_tables, torch.Tensor) else block_tables,
+                              dtype=np.int32)
+    cl = np.ascontiguousarray(context_lens.cpu().numpy() if isinstance(context_lens, torch.Tensor) else context_lens,
+                              dtype=np.int32)
+    if bt.ndim != 2 or cl.shape != (bt.shape[0],):
+        raise ValueError("block_tables must be [S][MB] and context_lens [S]")
+    begin = np.zeros(max(max_groups, 1), dtype=np.int32)
+    end = np.zeros_like(begin)
+    blocks = np.zeros_like(begin)
+    n = ctypes.c_int(0)
+    lib = library()
+    rc = lib.pkv_find_prefix_groups(bt.ctypes.data, cl.ctypes.data, bt.shape[0], max(bt.shape[1], 1), block_size,
+                                    min_blocks, begin.ctypes.data, end.ctypes.data, blocks.ctypes.data, max_groups,
+                                    ctypes.byref(n))
+    if rc != PKV_OK:
+        raise PagedKVError("pkv_find_prefix_groups", rc, lib.pkv_bm_last_error().decode())
+    k = n.value
+    return PrefixGroups(begin[:k], end[:k], blocks[:k])
+
+
+def _options(num_ctas=0, num_stages=0, ctas_per_sm=0, math=0, l2_prefetch=0, piece_cost=0, head_pack=0,
+             tile_tokens=0, prefix_groups: Optional[PrefixGroups] = None) -> _Options:
+    return _Options(num_ctas, num_stages, ctas_per_sm, math, l2_prefetch, piece_cost, head_pack, tile_tokens,
+                    prefix_groups.c_ptr() if prefix_groups is not None else None)
 
 
 def library_path() -> str:
@@ -93,6 +154,10 @@ def library() -> ctypes.CDLL:
             lib.pkv_selftest_bounded_wait.argtypes = [P, P]
             lib.pkv_read_status.restype = I
             lib.pkv_read_status.argtypes = [P, ctypes.POINTER(ctypes.c_int32), I, P]
+            lib.pkv_find_prefix_groups.restype = I
+            lib.pkv_find_prefix_groups.argtypes = [P, P, I, I, I, I, P, P, P, I, ctypes.POINTER(I)]
+            lib.pkv_bm_last_error.restype = ctypes.c_char_p
+            lib.pkv_bm_last_error.argtypes = []
             _lib = lib
         return _lib
 
@@ -158,13 +223,15 @@ def paged_attn_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
                       block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float,
                       workspace: torch.Tensor, num_ctas: int = 0, num_stages: int = 0,
                       ctas_per_sm: int = 0, math: int = 0, l2_prefetch: int = 0, piece_cost: int = 0,
-                      head_pack: int = 0, tile_tokens: int = 0,
+                      head_pack: int = 0, tile_tokens: int = 0, prefix_groups: Optional[PrefixGroups] = None,
                       stream=None) -> torch.Tensor:
     """out[s, j] = softmax_t(scale * q[s, j] . K_t) . V_t over the sequence's paged tokens.
 
     q, out: bf16 [S, Hq, D]; k_cache, v_cache: bf16 [NB, bs, Hkv, D];
     block_tables: int32 [S, MB]; context_lens: int32 [S]; workspace: uint8 from
     allocate_workspace(). Enqueued on ``stream`` (default: torch's current stream).
+    prefix_groups: runs of sequences sharing their leading blocks (find_prefix_groups),
+    whose shared blocks are then read once per group.
     """
     _need(q, "q", torch.bfloat16, 3)
     _need(out, "out", torch.bfloat16, 3)
@@ -174,7 +241,8 @@ def paged_attn_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
     _need(context_lens, "context_lens", torch.int32, 1)
     _need(workspace, "workspace", torch.uint8, 1)
     S, Hq, D, NB, bs, Hkv = _decode_shapes(out, q, k_cache, v_cache, block_tables, context_lens)
-    opts = _Options(num_ctas, num_stages, ctas_per_sm, math, l2_prefetch, piece_cost, head_pack, tile_tokens)
+    opts = _options(num_ctas, num_stages, ctas_per_sm, math, l2_prefetch, piece_cost, head_pack, tile_tokens,
+                    prefix_groups)
     _check("paged_attn_decode", library().paged_attn_decode_ex(
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
         S, Hq, Hkv, D, bs, float(scale), block_tables.shape[1], NB, _ptr(workspace), workspace.numel(),
@@ -187,7 +255,8 @@ def paged_attn_decode_append(out: torch.Tensor, q: torch.Tensor, k_new: torch.Te
                              block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float,
                              workspace: torch.Tensor, num_ctas: int = 0, num_stages: int = 0,
                              ctas_per_sm: int = 0, math: int = 0, l2_prefetch: int = 0, piece_cost: int = 0,
-                             head_pack: int = 0, tile_tokens: int = 0, stream=None) -> torch.Tensor:
+                             head_pack: int = 0, tile_tokens: int = 0, prefix_groups: Optional[PrefixGroups] = None,
+                             stream=None) -> torch.Tensor:
     """One decode step in one launch: append k_new / v_new (bf16 [S, Hkv, D]) at
     slot_mapping (int64 [S], the slot of each sequence's last position, < 0 =
     none), then the same attention as paged_attn_decode over contexts that
@@ -211,7 +280,8 @@ def paged_attn_decode_append(out: torch.Tensor, q: torch.Tensor, k_new: torch.Te
         raise ValueError("k_new / v_new must be [num_seqs, num_kv_heads, head_dim] and slot_mapping [num_seqs]")
     if block_tables.shape[0] != S or context_lens.shape[0] != S:
         raise ValueError("block_tables and context_lens must have num_seqs rows")
-    opts = _Options(num_ctas, num_stages, ctas_per_sm, math, l2_prefetch, piece_cost, head_pack, tile_tokens)
+    opts = _options(num_ctas, num_stages, ctas_per_sm, math, l2_prefetch, piece_cost, head_pack, tile_tokens,
+                    prefix_groups)
     _check("paged_attn_decode_append", library().paged_attn_decode_append(
         _ptr(out), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(slot_mapping), _ptr(k_cache), _ptr(v_cache),
         _ptr(block_tables), _ptr(context_lens), S, Hq, Hkv, D, bs, float(scale), block_tables.shape[1], NB,
@@ -330,7 +400,7 @@ def paged_attn_decode_fp8(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Ten
     if block_tables.shape[0] != S or context_lens.shape[0] != S:
         raise ValueError("block_tables and context_lens must have num_seqs rows")
     _need_scales(k_scale, v_scale, Hkv)
-    opts = _Options(**{k: int(options.get(k, 0)) for k, _ in _Options._fields_})
+    opts = _options(**options)
     _check("paged_attn_decode_fp8", library().paged_attn_decode_fp8(
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), _ptr(block_tables),
         _ptr(context_lens), S, Hq, Hkv, D, bs, float(scale), block_tables.shape[1], NB, _ptr(workspace),
@@ -363,7 +433,7 @@ def paged_attn_decode_append_fp8(out: torch.Tensor, q: torch.Tensor, k_new: torc
     if block_tables.shape[0] != S or context_lens.shape[0] != S:
         raise ValueError("block_tables and context_lens must have num_seqs rows")
     _need_scales(k_scale, v_scale, Hkv)
-    opts = _Options(**{k: int(options.get(k, 0)) for k, _ in _Options._fields_})
+    opts = _options(**options)
     _check("paged_attn_decode_append_fp8", library().paged_attn_decode_append_fp8(
         _ptr(out), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(slot_mapping), _ptr(k_cache), _ptr(v_cache),
         _ptr(k_scale), _ptr(v_scale), _ptr(block_tables), _ptr(context_lens), S, Hq, Hkv, D, bs, float(scale),

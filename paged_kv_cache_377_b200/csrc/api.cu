@@ -149,6 +149,70 @@ constexpr int kDefaultL2Prefetch = 0;  // measured on the Llama-shaped batch: an
 // Qwen- and OPT-shaped and skewed batches: 4 is within 1% of the best for each.
 constexpr int kDefaultPieceCost = 4;
 
+// Prefix tiles one prefix unit streams before it stores its partials: long
+// enough to amortise the unit's start (q fragments, first copies), short enough
+// that a group's shared blocks are spread over many CTAs.
+constexpr int kPrefixTilesPerPiece = 16;
+
+// The prefix units of one launch (sequences s0 .. s0 + sc - 1): the groups of
+// the caller's descriptor that have at least two members in the launch, as
+// kernel parameters. Leaves a.num_groups = 0 when grouping does not apply.
+void plan_prefix_groups(const pkv_prefix_groups *pg, int s0, int sc, int hkv, int group, int sub, int ctas,
+                        pkv::DecodeArgs &a) {
+    a.num_groups = 0;
+    a.prefix_ctas = 0;
+    a.tiles_per_piece = 1;
+    a.prefix_np = 0;
+    a.pre_base = 0;
+    if (!pg || pg->num_groups <= 0) return;
+    int n = 0, max_tiles = 0;
+    for (int g = 0; g < pg->num_groups && n < pkv::kMaxPrefixGroups; ++g) {
+        const int lo = pg->begin[g] > s0 ? pg->begin[g] : s0;
+        const int hi = pg->end[g] < s0 + sc ? pg->end[g] : s0 + sc;
+        if (hi - lo < 2) continue;
+        a.grp_begin[n] = lo - s0;
+        a.grp_end[n] = hi - s0;
+        a.grp_tiles[n] = pg->blocks[g] * sub;
+        if (a.grp_tiles[n] > max_tiles) max_tiles = a.grp_tiles[n];
+        const int per = pkv::kPrefixRows / group;  // members whose rows fit one unit
+        const int row_tiles = (hi - lo + per - 1) / per;
+        a.grp_row_tiles[n] = row_tiles;
+        a.grp_members[n] = (hi - lo + row_tiles - 1) / row_tiles;  // spread evenly over the row tiles
+        ++n;
+    }
+    if (n == 0) return;
+    // Partial rows: the workspace holds (S + 1024) * Hq rows; the suffix pieces
+    // take bases below sc * Hkv + ctas, the prefix pieces sc * Hkv * np after them.
+    const long long room = 1024LL * hkv - ctas;
+    const long long np_max = room / (static_cast<long long>(sc) * hkv);
+    if (np_max < 1) return;
+    int tpp = kPrefixTilesPerPiece;
+    if ((max_tiles + tpp - 1) / tpp > np_max) tpp = static_cast<int>((max_tiles + np_max - 1) / np_max);
+    long long units = 0;
+    for (;;) {
+        units = 0;
+        for (int g = 0; g < n; ++g)
+            units += static_cast<long long>(hkv) * a.grp_row_tiles[g] * ((a.grp_tiles[g] + tpp - 1) / tpp);
+        if (units <= ctas / 2 || tpp >= max_tiles) break;
+        tpp *= 2;  // fewer, longer pieces until the units leave most CTAs to the suffixes
+    }
+    if (units > ctas - 1) return;  // no CTA would be left for the suffixes
+    a.num_groups = n;
+    a.tiles_per_piece = tpp;
+    int np = 0;
+    long long u = 0;
+    for (int g = 0; g < n; ++g) {
+        a.grp_unit0[g] = static_cast<int>(u);
+        const int pieces = (a.grp_tiles[g] + tpp - 1) / tpp;
+        if (pieces > np) np = pieces;
+        u += static_cast<long long>(hkv) * a.grp_row_tiles[g] * pieces;
+    }
+    a.grp_unit0[n] = static_cast<int>(u);
+    a.prefix_ctas = static_cast<int>(u);
+    a.prefix_np = np;
+    a.pre_base = sc * hkv + ctas;
+}
+
 int default_stages(int head_dim, int block_size, int math) {
     if (math == pkv::kMathTensorCore) return 1;
     if (math == pkv::kMathFp8) return head_dim == 256 ? 1 : 2;  // about 8 KB of blocks in flight per warp
@@ -218,7 +282,7 @@ int decode_impl(void *out, const void *q, const void *k_new, const void *v_new, 
         !aligned(workspace, 256))
         return fail(PKV_ERR_INVALID_ARGUMENT,
                     "out, q, k_cache and v_cache must be 16-byte aligned and workspace 256-byte aligned");
-    pkv_decode_options o = {0, 0, 0, 0, 0, 0, 0, 0};
+    pkv_decode_options o = {0, 0, 0, 0, 0, 0, 0, 0, nullptr};
     if (opts) o = *opts;
     if (o.num_ctas < 0 || o.num_stages < 0 || o.ctas_per_sm < 0 || o.math < 0 || o.math > 2 ||
         o.l2_prefetch < -1 || o.l2_prefetch > 32 || o.piece_cost < -1 || o.piece_cost > 64 || o.head_pack < 0 ||
@@ -233,6 +297,27 @@ int decode_impl(void *out, const void *q, const void *k_new, const void *v_new, 
     if (fp8 && o.math == pkv::kMathCudaCore)
         return fail(PKV_ERR_UNSUPPORTED, "e4m3 pools are decoded on tensor cores only (math 0 or 2)");
     const int math = fp8 ? pkv::kMathFp8 : o.math ? o.math : pkv::kMathTensorCore;
+    const pkv_prefix_groups *pg = o.prefix_groups;
+    if (pg && pg->num_groups < 0) return fail(PKV_ERR_INVALID_ARGUMENT, "prefix_groups.num_groups < 0");
+    if (pg && pg->num_groups > 0) {
+        if (!pg->begin || !pg->end || !pg->blocks)
+            return fail(PKV_ERR_INVALID_ARGUMENT, "prefix_groups arrays are NULL");
+        for (int g = 0; g < pg->num_groups; ++g) {
+            if (pg->begin[g] < (g ? pg->end[g - 1] : 0) || pg->end[g] < pg->begin[g] + 2 || pg->end[g] > num_seqs)
+                return fail(PKV_ERR_INVALID_ARGUMENT,
+                            "prefix group %d [%d, %d): groups need two or more members, in order, within num_seqs", g,
+                            pg->begin[g], pg->end[g]);
+            if (pg->blocks[g] < 1 || pg->blocks[g] > max_blocks_per_seq)
+                return fail(PKV_ERR_INVALID_ARGUMENT, "prefix_groups.blocks[%d] = %d outside [1, %d]", g,
+                            pg->blocks[g], max_blocks_per_seq);
+        }
+        if (math != pkv::kMathTensorCore)
+            return fail(PKV_ERR_UNSUPPORTED, "prefix groups need bf16 pools on tensor cores (math 0 or 2)");
+        if (o.head_pack == 2) return fail(PKV_ERR_UNSUPPORTED, "prefix groups are decoded without head packing");
+        if (o.tile_tokens == 32) return fail(PKV_ERR_UNSUPPORTED, "prefix groups are read in 16-row tiles");
+    } else {
+        pg = nullptr;
+    }
     // Head packing: kv heads 2h, 2h + 1 of head_dim 64 read as one head of 128
     // (256-byte rows instead of 128-byte ones; for e4m3 pools, 128-byte rows
     // instead of 64-byte ones); the kernel then sees half the kv heads, twice
@@ -243,7 +328,7 @@ int decode_impl(void *out, const void *q, const void *k_new, const void *v_new, 
     if (o.head_pack == 2 && !can_pack)
         return fail(PKV_ERR_UNSUPPORTED, "head_pack 2 needs tensor-core math, head_dim 64 (or 128 for e4m3 pools), an "
                                          "even num_kv_heads and num_q_heads / num_kv_heads <= %d", PKV_MAX_GROUP / 2);
-    const int pack = o.head_pack == 1 ? 1 : can_pack ? 2 : 1;
+    const int pack = o.head_pack == 1 || pg ? 1 : can_pack ? 2 : 1;
     if (fp8 && head_dim == 64 && pack != 2)
         return fail(PKV_ERR_UNSUPPORTED, "e4m3 pools need head_dim 128, or head_dim 64 with head packing (an even "
                                          "num_kv_heads and num_q_heads / num_kv_heads <= %d)", PKV_MAX_GROUP / 2);
@@ -310,6 +395,7 @@ int decode_impl(void *out, const void *q, const void *k_new, const void *v_new, 
         a.prefetch = o.l2_prefetch > 0 ? o.l2_prefetch : o.l2_prefetch == 0 ? kDefaultL2Prefetch : 0;
         a.piece_cost = o.piece_cost > 0 ? o.piece_cost : o.piece_cost == 0 ? kDefaultPieceCost : 0;
         a.scale_log2 = scale * 1.4426950408889634f;
+        plan_prefix_groups(pg, s0, sc, khkv, kgroup, a.sub, grid, a);
         if (fused) {
             const size_t row = static_cast<size_t>(num_kv_heads) * head_dim;  // elements per token
             a.k_new = static_cast<const __nv_bfloat16 *>(k_new) + static_cast<size_t>(s0) * row;

@@ -229,3 +229,45 @@ int pkv_bm_pack(const pkv_block_manager *bm, const int64_t *seq_ids, int num_seq
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Prefix groups of a packed batch (see pkv_find_prefix_groups in pagedkv.h):
+// runs of consecutive sequences whose tables start with the same physical
+// blocks, which the decode then reads once per group.
+extern "C" int pkv_find_prefix_groups(const int32_t *block_tables, const int32_t *context_lens, int num_seqs,
+                                      int max_blocks_per_seq, int block_size, int min_blocks, int32_t *begin,
+                                      int32_t *end, int32_t *blocks, int max_groups, int *num_groups) {
+    if (!num_groups || num_seqs < 0 || max_blocks_per_seq <= 0 || block_size <= 0 || min_blocks < 1 ||
+        max_groups < 0 || (num_seqs > 0 && (!block_tables || !context_lens)) ||
+        (max_groups > 0 && (!begin || !end || !blocks)))
+        return bm_fail(PKV_ERR_INVALID_ARGUMENT, "bad argument");
+    auto covered = [&](int s) {  // table entries the context of s uses
+        const int64_t L = context_lens[s] < 0 ? 0 : context_lens[s];
+        const int64_t n = (L + block_size - 1) / block_size;
+        return static_cast<int>(n < max_blocks_per_seq ? n : max_blocks_per_seq);
+    };
+    auto row = [&](int s) { return block_tables + static_cast<int64_t>(s) * max_blocks_per_seq; };
+    int n = 0, s = 0;
+    while (s < num_seqs && n < max_groups) {
+        int shared = covered(s), e = s + 1;
+        while (e < num_seqs) {
+            const int lim = shared < covered(e) ? shared : covered(e);
+            int c = 0;
+            while (c < lim && row(s)[c] == row(e)[c]) ++c;
+            if (c < min_blocks) break;
+            shared = c;
+            ++e;
+        }
+        if (e - s >= 2) {
+            begin[n] = s;
+            end[n] = e;
+            blocks[n] = shared;
+            ++n;
+            s = e;
+        } else {
+            ++s;
+        }
+    }
+    *num_groups = n;
+    return PKV_OK;
+}

@@ -54,7 +54,9 @@
 namespace pkv {
 namespace {
 
-// A piece: blocks [b0, b1) of segment (s, h), processed by one CTA.
+// A piece: blocks [b0, b1) of segment (s, h), processed by one CTA. L is the
+// context length past the sequence's shared prefix (read by prefix units), so
+// that block b of the segment holds positions b BS .. b BS + BS - 1 of those.
 struct Piece {
     int s, h, b0, b1, L;
     bool whole;  // the piece is the entire segment (no merge needed)
@@ -67,7 +69,8 @@ struct PieceIter {
     long long x, x1;
     const int *pre;
     const int *lens;
-    int S, Hkv;
+    const int *ptiles;
+    int S, Hkv, BS;
 
     __device__ __forceinline__ bool next(Piece &pc) {
         if (x >= x1) return false;
@@ -87,8 +90,9 @@ struct PieceIter {
         pc.h = h;
         pc.b0 = r - h * n;
         pc.b1 = pc.b0 + static_cast<int>(end - x);
-        pc.L = lens[lo];
-        pc.whole = pc.b0 == 0 && end == seg_end;
+        const int t0 = ptiles[lo];
+        pc.L = lens[lo] - t0 * BS;
+        pc.whole = pc.b0 == 0 && end == seg_end && t0 == 0;  // no prefix pieces to merge with
         x = end;
         return true;
     }
@@ -840,6 +844,8 @@ struct Smem {
     int *prefix;
     int *wprefix;
     int *lens;
+    int *ptiles;     // [S] shared-prefix tiles of each sequence (0: not in a prefix group)
+    uint64_t *empty;  // prefix units: all four warps are done with a stage
 };
 
 // The CTAs holding pieces of segment (s, h). CTA c covers weight positions
@@ -868,15 +874,48 @@ __device__ __forceinline__ int piece_cta(const SegmentSpan &sp, int i, long long
     return W >= C ? sp.c0 + i : static_cast<int>(((sp.v_first + i + 1) * C - 1) / W);
 }
 
-// Merge of the pieces of segment (s, h), held by CTAs piece_ctas[0 ..
-// npieces) (log-sum-exp identity, pieces in CTA order): out = sum_c 2^(lse_c - M) o_c / sum_c 2^(lse_c - M), taken in one
-// pass with a running maximum. A thread merges 4-dim elements of the G x D
+// Prefix pieces of sequence s that hold some of its tokens: the prefix units
+// of its group whose tiles start below its length.
+__device__ __forceinline__ int live_prefix_pieces(int s, const Smem &sm, int BS, int tiles_per_piece) {
+    const int pt = sm.ptiles[s], L = sm.lens[s];
+    if (pt == 0 || L == 0) return 0;
+    const int t = min((L + BS - 1) / BS, pt);
+    return (t + tiles_per_piece - 1) / tiles_per_piece;
+}
+
+// Pieces segment (s, h) is merged from: its live prefix pieces, then the
+// suffix pieces the CTA split gives it (none when the suffix is empty).
+__device__ __forceinline__ int segment_pieces(int s, int h, const Smem &sm, int Hkv, long long W, int C, int pcost,
+                                              int BS, int tiles_per_piece, SegmentSpan *sp_out) {
+    SegmentSpan sp{0, 0, 0};
+    if (sm.prefix[s + 1] > sm.prefix[s]) sp = segment_span(s, h, sm, Hkv, W, C, pcost);
+    if (sp_out) *sp_out = sp;
+    return live_prefix_pieces(s, sm, BS, tiles_per_piece) + sp.npieces;
+}
+
+// Lists the partial-row bases of segment (s, h)'s pieces (prefix pieces first)
+// into `list`; threads of the CTA share the work. Returns the count.
+__device__ __forceinline__ int list_pieces(const DecodeArgs &a, int s, int h, const Smem &sm, long long W, int C,
+                                           int pcost, int BS, int *list, int ctid) {
+    SegmentSpan sp;
+    const int n = segment_pieces(s, h, sm, a.num_kv_heads, W, C, pcost, BS, a.tiles_per_piece, &sp);
+    const int npre = n - sp.npieces;
+    const int seg = s * a.num_kv_heads + h;
+    for (int j = ctid; j < n; j += kConsumerWarps * 32)
+        list[j] = j < npre ? a.pre_base + seg * a.prefix_np + j : seg + piece_cta(sp, j - npre, W, C);
+    return n;
+}
+
+// Merge of the pieces of segment (s, h) whose partials sit at rows
+// piece_base[i] * G + g, i < npieces (log-sum-exp identity, in list order: the
+// prefix pieces, then the suffix pieces in CTA order): out = sum_c 2^(lse_c - M)
+// o_c / sum_c 2^(lse_c - M), taken in one pass with a running maximum. A thread merges 4-dim elements of the G x D
 // output (at most two) and loads four pieces ahead, so that the merge costs a
 // few L2 round trips rather than one per piece. Partials written by other SMs
 // are read past L1.
 template <int D>
-__device__ __forceinline__ void merge_pieces(const DecodeArgs &a, const int *piece_ctas, int npieces, size_t seg,
-                                             int s, int h, int ctid) {
+__device__ __forceinline__ void merge_pieces(const DecodeArgs &a, const int *piece_base, int npieces, int s, int h,
+                                             int ctid) {
     constexpr int kAhead = 4;
     const int G = a.group;
     const int DR = D / a.pack;
@@ -894,7 +933,7 @@ __device__ __forceinline__ void merge_pieces(const DecodeArgs &a, const int *pie
             for (int i = 0; i < kAhead; ++i) {
                 lse[i] = -INFINITY;
                 if (ib + i < npieces) {
-                    const size_t pr = (seg + piece_ctas[ib + i]) * G + g;
+                    const size_t pr = static_cast<size_t>(piece_base[ib + i]) * G + g;
                     lse[i] = __ldcg(a.lse_part + pr);
                     o[i] = __ldcg(reinterpret_cast<const float4 *>(a.o_part + pr * DR + col));
                 }
@@ -933,7 +972,7 @@ __device__ __forceinline__ void merge_pieces(const DecodeArgs &a, const int *pie
 template <int D, int BS, class Math, int ES>
 __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUtensorMap *tm_v, const DecodeArgs &a,
                                             const Smem &sm, const DecodeLayout &ly, PieceIter pieces, long long x0,
-                                            long long x1, long long W, int C, int pcost, int warp, int lane) {
+                                            long long x1, long long W, int pcost, int warp, int lane) {
     static_assert(ES == 1 || ES == 2, "pool element bytes");
     constexpr uint32_t kTile = BS * D * ES;   // bytes of one K (or V) tile
     constexpr uint32_t kHalf = BS * 128;      // one TMA copy: BS rows of 128 bytes
@@ -970,7 +1009,7 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
             const int n = sm.prefix[lo + 1] - sm.prefix[lo];
             const int r = static_cast<int>(x - static_cast<long long>(a.num_kv_heads) * sm.prefix[lo]);
             h = r / n;
-            const int j = r - h * n;
+            const int j = r - h * n + sm.ptiles[lo];  // logical tile of the context
             const int pb = __ldg(a.block_tables + static_cast<size_t>(lo) * a.max_blocks_per_seq + (j >> sub_shift));
             p = (pb < 0 || pb >= a.num_blocks) ? -1 : ((pb << sub_shift) + (j & (a.sub - 1))) * BS;
         }
@@ -1099,7 +1138,7 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
             // the K row, the next kChunks lanes the V row, 16 stored bytes each).
             constexpr int kChunks = D * ES / 16;  // 16-byte chunks of a stored row
             constexpr int kElems = 16 / ES;       // elements per chunk
-            const int bi = pc.b0 + i;             // block within the segment
+            const int bi = pc.b0 + i;             // block of the segment
             const bool tail = a.slots != nullptr && (bi + 1) * BS >= pc.L;
             long long slot = -1;
             auto patch_src = [&]() {  // this lane's chunk of the new row (bf16 source)
@@ -1194,7 +1233,8 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
                 *reinterpret_cast<__nv_bfloat162 *>(static_cast<__nv_bfloat16 *>(a.out) + row * DR + col) =
                     __floats2bfloat162_rn(o0, o1);
             } else {
-                const size_t pr = (seg + blockIdx.x) * G + g;  // piece (segment + CTA), row g
+                // piece (segment + CTA), row g; CTAs are numbered after the prefix units
+                const size_t pr = (seg + blockIdx.x - a.prefix_ctas) * G + g;
                 *reinterpret_cast<float2 *>(a.o_part + pr * DR + col) = make_float2(o0, o1);
                 if (col == 0) a.lse_part[pr] = ls > 0.f ? M + __log2f(ls) : -INFINITY;
             }
@@ -1205,7 +1245,8 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
             __threadfence();
             named_barrier_sync(1, kConsumerWarps * 32);
             if (ctid == 0) {
-                const SegmentSpan sp = segment_span(pc.s, pc.h, sm, a.num_kv_heads, W, C, pcost);
+                const int total = segment_pieces(pc.s, pc.h, sm, a.num_kv_heads, W, gridDim.x - a.prefix_ctas, pcost,
+                                                 BS, a.tiles_per_piece, nullptr);
                 unsigned long long *cnt = a.seg_count + seg;
                 unsigned long long old = atomicAdd(cnt, 0ull), now;
                 for (;;) {  // count = 1 for the first piece of this launch (stale epochs restart)
@@ -1215,7 +1256,7 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
                     old = prev;
                 }
                 const int pending = sm.merge_flag[0];
-                if (static_cast<int>(now & 0xffffull) == sp.npieces && pending < 2) {  // never more than two (below)
+                if (static_cast<int>(now & 0xffffull) == total && pending < 2) {  // never more than two (below)
                     volatile int *m = sm.merge_flag + 1 + 2 * pending;
                     m[0] = pc.s;
                     m[1] = pc.h;
@@ -1252,14 +1293,288 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
         __threadfence();
         // the grid's total weight, reloaded rather than kept live across the loop
         const long long Wt = static_cast<long long>(a.num_kv_heads) * sm.wprefix[a.num_seqs];
-        const SegmentSpan sp = segment_span(s, h, sm, a.num_kv_heads, Wt, gridDim.x, pcost);
-        // the CTA of each piece, listed in the (now idle) stage buffers: at least
-        // 16 KB, and a segment has at most kMaxCtas pieces
-        int *piece_ctas = reinterpret_cast<int *>(sm.base + ly.stages);
+        // the partial of each piece, listed in the (now idle) stage buffers: at
+        // least 16 KB, and a segment has at most kMaxCtas + 1024 pieces
+        int *list = reinterpret_cast<int *>(sm.base + ly.stages);
         if (i > 0) named_barrier_sync(1, kConsumerWarps * 32);  // the previous merge is done with the list
-        for (int j = ctid; j < sp.npieces; j += kConsumerWarps * 32) piece_ctas[j] = piece_cta(sp, j, Wt, gridDim.x);
+        const int n = list_pieces(a, s, h, sm, Wt, gridDim.x - a.prefix_ctas, pcost, BS, list, ctid);
         named_barrier_sync(1, kConsumerWarps * 32);
-        merge_pieces<D>(a, piece_ctas, sp.npieces, static_cast<size_t>(s) * a.num_kv_heads + h, s, h, ctid);
+        merge_pieces<D>(a, list, n, s, h, ctid);
+    }
+}
+
+
+// ------------------------------------------------------------------ shared prefixes
+
+// One prefix unit: the query rows of up to kPrefixRows (sequence, q head)
+// pairs -- the G rows of each member of one row tile of a prefix group, for
+// kv head h -- against tiles [t0, t1) of the group's shared prefix, which are
+// read once for all of them. Sharing a physical block is the same as owning
+// a copy of it ("Deep Dive into vLLM", section 2.2; runbyai post 449, section
+// 3), so a block read here serves every member. Flash-attention style on
+// mma.sync: warp w takes rows 16 w .. 16 w + 15 as M, a tile's 16 tokens as N
+// (S = Q K^T), then P as the A operand of O += P V; the four warps consume one
+// CTA-wide ring of K/V tiles that warp 0 refills. Each row leaves an fp32
+// partial and its log2-sum-exp; the last piece of a segment to be stored merges
+// the segment (prefix pieces first, then the suffix pieces).
+template <int D>
+__device__ __forceinline__ void prefix_unit(const CUtensorMap *tm_k, const CUtensorMap *tm_v, const DecodeArgs &a,
+                                         const Smem &sm, const DecodeLayout &ly, long long W, int C, int pcost,
+                                         int warp, int lane) {
+    constexpr int BS = 16;
+    constexpr int KST = D / 16;             // k-steps of q.K
+    constexpr int NT = D / 8;               // 8-dim n-tiles of P.V
+    constexpr uint32_t kTile = BS * D * 2;  // bytes of one K (or V) tile
+    constexpr uint32_t kHalf = BS * 128;    // one TMA copy: 16 rows of 128 bytes
+    constexpr int kCopies = D * 2 / 128;
+    const int G = a.group, Hkv = a.num_kv_heads;
+    const int ctid = warp * 32 + lane;
+    const int NST = kConsumerWarps * a.num_stages;  // the CTA's stages, one ring
+
+    // ---- which unit: group g, kv head h, row tile rt, prefix piece tp
+    const int u = blockIdx.x;
+    int g = 0;
+    while (g + 1 < a.num_groups && a.grp_unit0[g + 1] <= u) ++g;
+    const int T = a.grp_tiles[g];
+    const int np = (T + a.tiles_per_piece - 1) / a.tiles_per_piece;
+    const int v = u - a.grp_unit0[g];
+    const int tp = v % np, rt = (v / np) % a.grp_row_tiles[g], h = v / np / a.grp_row_tiles[g];
+    const int m0 = a.grp_begin[g] + rt * a.grp_members[g];
+    const int m1 = min(a.grp_end[g], m0 + a.grp_members[g]);
+    const int rows = (m1 - m0) * G;
+    const int t0 = tp * a.tiles_per_piece;
+    int lim_max = 0;  // prefix tokens any member attends to
+    for (int m = m0; m < m1; ++m) lim_max = max(lim_max, min(sm.lens[m], T * BS));
+    const int t1 = min(min(T, t0 + a.tiles_per_piece), (lim_max + BS - 1) / BS);
+    const int ntiles = max(0, t1 - t0);
+
+    // ---- this lane's two rows: fragment rows lane/4 and lane/4 + 8 of the warp,
+    // i.e. unit rows R = 16 warp + lane/4 + 8 k: member R / G, q head h G + R % G
+    const int tq = lane & 3;
+    int row_lim[2];  // prefix tokens the row attends (0: none, or a padding row)
+    // q rows r and r + 8 (a padding row reads row 0 of the batch: its logits are
+    // selected away). Their A fragments (dims 2 tq, 2 tq + 1 and + 8 of each
+    // k-step) are re-read from L1 at every tile rather than held in 32 registers
+    // beside the 64 of the accumulators.
+    const uint32_t *qr[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        const int R = 16 * warp + (lane >> 2) + 8 * k;
+        const int sq = m0 + R / G;
+        row_lim[k] = R < rows ? min(sm.lens[sq], T * BS) : 0;
+        qr[k] = reinterpret_cast<const uint32_t *>(static_cast<const __nv_bfloat16 *>(a.q)) +
+                (R < rows ? (static_cast<size_t>(sq) * a.num_q_heads + h * G + R % G) * (D / 2) : 0);
+    }
+
+    // ---- the ring: tile j of the piece goes to stage j % NST (K on full, V on full_v)
+    const int *ltab = a.block_tables + static_cast<size_t>(a.grp_begin[g]) * a.max_blocks_per_seq;
+    const int sub_shift = a.sub == 2 ? 1 : 0;
+    // each member's table must hold the group's blocks wherever this piece
+    // covers tokens the member attends (a caller's wrong grouping is reported)
+    if (ntiles > 0) {
+        const int b0 = t0 >> sub_shift, nb = ((t1 - 1) >> sub_shift) - b0 + 1;
+        for (int e = ctid; e < (m1 - m0) * nb; e += kConsumerWarps * 32) {
+            const int m = m0 + e / nb, b = b0 + e % nb;
+            const int att = (min(sm.lens[m], T * BS) + BS - 1) / BS;  // tiles the member attends
+            if ((b << sub_shift) < att &&
+                __ldg(a.block_tables + static_cast<size_t>(m) * a.max_blocks_per_seq + b) != __ldg(ltab + b))
+                atomicOr(a.status, PKV_STATUS_BAD_PREFIX_GROUP);
+        }
+    }
+    uint32_t inflight = 0, inflight_par = 0;  // producer (warp 0, lane 0): copies not yet seen landing
+    auto issue_tile = [&](int j) {
+        const int st = j % NST;
+        const uint32_t par = static_cast<uint32_t>(j / NST) & 1u;
+        const int tile = t0 + j;
+        const int pb = __ldg(ltab + (tile >> sub_shift));
+        if (*sm.abort_flag) return;
+        if (pb < 0 || pb >= a.num_blocks) {
+            atomicOr(a.status, PKV_STATUS_BAD_BLOCK_ID);
+            sm.stage_bad[st] = 1;
+            mbar_arrive(&sm.full[st]);
+            mbar_arrive(&sm.full_v[st]);
+            return;
+        }
+        sm.stage_bad[st] = 0;
+        const int prow = ((pb << sub_shift) + (tile & (a.sub - 1))) * BS;  // first pool row of the tile
+        uint8_t *dst = sm.base + ly.stages + static_cast<uint32_t>(st) * 2u * kTile;
+        mbar_arrive_expect_tx(&sm.full[st], kTile);
+#pragma unroll
+        for (int c = 0; c < kCopies; ++c) tma_load_4d(dst + c * kHalf, tm_k, &sm.full[st], 0, c, h, prow);
+        mbar_arrive_expect_tx(&sm.full_v[st], kTile);
+#pragma unroll
+        for (int c = 0; c < kCopies; ++c) tma_load_4d(dst + kTile + c * kHalf, tm_v, &sm.full_v[st], 0, c, h, prow);
+        inflight |= (1u << st) | (1u << (16 + st));
+        inflight_par = (inflight_par & ~((1u << st) | (1u << (16 + st)))) | (par << st) | (par << (16 + st));
+    };
+    if (warp == 0 && lane == 0)
+        for (int j = 0; j < min(NST, ntiles); ++j) issue_tile(j);
+
+    float acc[NT][4];
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) acc[n][k] = 0.f;
+    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+    const int mi = lane >> 3, r8 = lane & 7;
+    const uint32_t sbase = smem_u32(sm.base) + ly.stages;
+
+    for (int j = 0; j < ntiles; ++j) {
+        const int st = j % NST;
+        const uint32_t par = static_cast<uint32_t>(j / NST) & 1u;
+        const uint32_t ktile = sbase + static_cast<uint32_t>(st) * 2u * kTile, vtile = ktile + kTile;
+        const int tok0 = (t0 + j) * BS;  // context position of the tile's first row
+        if (mbar_wait_bounded(&sm.full[st], par, sm.abort_flag, a.status) && warp == 0 && lane == 0)
+            inflight &= ~(1u << st);
+        const bool live = !sm.stage_bad[st] && !*sm.abort_flag;
+        float sc[2][4];  // S for tokens 0-7 and 8-15: (row r: 2 tq, 2 tq + 1), (row r + 8: same)
+#pragma unroll
+        for (int n = 0; n < 2; ++n)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) sc[n][k] = 0.f;
+        if (live) {
+#pragma unroll
+            for (int kk = 0; kk < KST; ++kk) {
+                const uint32_t qa[4] = {__ldg(qr[0] + 8 * kk + tq), __ldg(qr[1] + 8 * kk + tq),
+                                        __ldg(qr[0] + 8 * kk + 4 + tq), __ldg(qr[1] + 8 * kk + 4 + tq)};
+                uint32_t b[4];  // B fragments (k = dims, n = tokens) of tokens 0-7 and 8-15
+                ldsm_x4(b, tile_addr<BS>(ktile, 8 * (mi >> 1) + r8, 2 * kk + (mi & 1)));
+                mma_16816(sc[0], qa, b[0], b[1]);
+                mma_16816(sc[1], qa, b[2], b[3]);
+            }
+        }
+        // base-2 logits; tokens a row does not attend are selected away
+        float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+        for (int n = 0; n < 2; ++n)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int rr = k >> 1, t = tok0 + 8 * n + 2 * tq + (k & 1);
+                sc[n][k] = (live && t < row_lim[rr]) ? sc[n][k] * a.scale_log2 : -INFINITY;
+                mx[rr] = fmaxf(mx[rr], sc[n][k]);
+            }
+        float alpha[2], mref[2];
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {
+            mx[rr] = fmaxf(mx[rr], __shfl_xor_sync(0xffffffffu, mx[rr], 1));
+            mx[rr] = fmaxf(mx[rr], __shfl_xor_sync(0xffffffffu, mx[rr], 2));
+            const float mn = fmaxf(m_run[rr], mx[rr]);
+            mref[rr] = mn == -INFINITY ? 0.f : mn;  // a row with nothing attended yet: every p is 0
+            alpha[rr] = fast_exp2(m_run[rr] - mref[rr]);
+            m_run[rr] = mn;
+        }
+        // probabilities in bf16 (the sums take the rounded values), as the A operand of P.V
+        uint32_t pa[4];
+#pragma unroll
+        for (int n = 0; n < 2; ++n)
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {
+                const __nv_bfloat162 p2 = __floats2bfloat162_rn(fast_exp2(sc[n][2 * rr] - mref[rr]),
+                                                               fast_exp2(sc[n][2 * rr + 1] - mref[rr]));
+                const float2 pf = __bfloat1622float2(p2);
+                l_run[rr] = l_run[rr] * (n == 0 ? alpha[rr] : 1.f) + pf.x + pf.y;
+                pa[2 * n + rr] = *reinterpret_cast<const uint32_t *>(&p2);
+            }
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+            acc[n][0] *= alpha[0];
+            acc[n][1] *= alpha[0];
+            acc[n][2] *= alpha[1];
+            acc[n][3] *= alpha[1];
+        }
+        if (mbar_wait_bounded(&sm.full_v[st], par, sm.abort_flag, a.status) && warp == 0 && lane == 0)
+            inflight &= ~(1u << (16 + st));
+        if (live && !*sm.abort_flag) {
+            // V rows no row of the unit attends may hold anything: zero them in the fragments
+            const int vmax = lim_max - tok0;
+            uint32_t keep_lo = 0xffffffffu, keep_hi = 0xffffffffu;  // tokens 2 tq, 2 tq + 1 and + 8
+            if (vmax < BS) {
+                keep_lo = (2 * tq < vmax ? 0x0000ffffu : 0u) | (2 * tq + 1 < vmax ? 0xffff0000u : 0u);
+                keep_hi = (2 * tq + 8 < vmax ? 0x0000ffffu : 0u) | (2 * tq + 9 < vmax ? 0xffff0000u : 0u);
+            }
+#pragma unroll
+            for (int dp = 0; dp < NT / 2; ++dp) {
+                uint32_t b[4];  // B fragments (k = tokens, n = dims) of dims 16 dp .. +7 and +8 .. +15
+                ldsm_x4_trans(b, tile_addr<BS>(vtile, 8 * (mi & 1) + r8, 2 * dp + (mi >> 1)));
+                b[0] &= keep_lo;
+                b[1] &= keep_hi;
+                b[2] &= keep_lo;
+                b[3] &= keep_hi;
+                mma_16816(acc[2 * dp], pa, b[0], b[1]);
+                mma_16816(acc[2 * dp + 1], pa, b[2], b[3]);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.empty[st]);
+        // warp 0 refills the stage of the previous tile once every warp is done with it
+        if (warp == 0 && lane == 0 && j >= 1 && j - 1 + NST < ntiles) {
+            const int jp = j - 1;
+            if (mbar_wait_bounded(&sm.empty[jp % NST], static_cast<uint32_t>(jp / NST) & 1u, sm.abort_flag, a.status))
+                issue_tile(jp + NST);
+        }
+        __syncwarp();
+    }
+    // with no copy in flight (possible only after a wait gave up) the stages are free
+    if (warp == 0 && lane == 0)
+        for (int st = 0; st < kMaxStages; ++st) {
+            if ((inflight >> st) & 1u) mbar_wait_drain(&sm.full[st], (inflight_par >> st) & 1u, a.status);
+            if ((inflight >> (16 + st)) & 1u)
+                mbar_wait_drain(&sm.full_v[st], (inflight_par >> (16 + st)) & 1u, a.status);
+        }
+    named_barrier_sync(1, kConsumerWarps * 32);
+    if (*sm.abort_flag || ntiles == 0) return;
+
+    // ---- this piece's partial of every row that attends some of its tokens
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+        l_run[rr] += __shfl_xor_sync(0xffffffffu, l_run[rr], 1);
+        l_run[rr] += __shfl_xor_sync(0xffffffffu, l_run[rr], 2);
+    }
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+        if (row_lim[rr] <= t0 * BS) continue;  // attends none of this piece (or a padding row)
+        const int R = 16 * warp + (lane >> 2) + 8 * rr;
+        const int sq = m0 + R / G, gq = R % G;
+        const size_t pr = static_cast<size_t>(a.pre_base + (sq * Hkv + h) * a.prefix_np + tp) * G + gq;
+        const float inv = 1.f / l_run[rr];
+        float *dst = a.o_part + pr * D + 2 * tq;
+#pragma unroll
+        for (int n = 0; n < NT; ++n)
+            *reinterpret_cast<float2 *>(dst + 8 * n) = make_float2(acc[n][2 * rr] * inv, acc[n][2 * rr + 1] * inv);
+        if (tq == 0) a.lse_part[pr] = m_run[rr] + __log2f(l_run[rr]);
+    }
+
+    // ---- count the piece in on each member's segment; merge the segments it completes
+    __threadfence();
+    named_barrier_sync(1, kConsumerWarps * 32);
+    int *mlist = reinterpret_cast<int *>(sm.base + ly.stages);  // [0] count, [1 ..] members to merge
+    int *plist = mlist + 2 * kPrefixRows;                        // partial rows of one segment
+    if (ctid == 0) mlist[0] = 0;
+    named_barrier_sync(1, kConsumerWarps * 32);
+    if (ctid < m1 - m0) {
+        const int s = m0 + ctid;
+        if (min(sm.lens[s], T * BS) > t0 * BS) {
+            const int total = segment_pieces(s, h, sm, Hkv, W, C, pcost, BS, a.tiles_per_piece, nullptr);
+            unsigned long long *cnt = a.seg_count + static_cast<size_t>(s) * Hkv + h;
+            unsigned long long old = atomicAdd(cnt, 0ull), now;
+            for (;;) {  // count = 1 for the first piece of this launch (stale epochs restart)
+                now = (old >> 16) == a.epoch ? old + 1 : (a.epoch << 16) | 1ull;
+                const unsigned long long prev = atomicCAS(cnt, old, now);
+                if (prev == old) break;
+                old = prev;
+            }
+            if (static_cast<int>(now & 0xffffull) == total) mlist[1 + atomicAdd(mlist, 1)] = s;
+        }
+    }
+    named_barrier_sync(1, kConsumerWarps * 32);
+    const int nmerge = mlist[0];
+    for (int i = 0; i < nmerge; ++i) {
+        const int s = mlist[1 + i];
+        __threadfence();
+        const int n = list_pieces(a, s, h, sm, W, C, pcost, BS, plist, ctid);
+        named_barrier_sync(1, kConsumerWarps * 32);
+        merge_pieces<D>(a, plist, n, s, h, ctid);
+        named_barrier_sync(1, kConsumerWarps * 32);  // the list is rewritten by the next merge
     }
 }
 
@@ -1292,12 +1607,15 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathCudaCore ? 1 : (M
     sm.prefix = reinterpret_cast<int *>(sm.base + ly.prefix);
     sm.wprefix = reinterpret_cast<int *>(sm.base + ly.wprefix);
     sm.lens = reinterpret_cast<int *>(sm.base + ly.lens);
+    sm.ptiles = reinterpret_cast<int *>(sm.base + ly.ptiles);
+    sm.empty = sm.qfull + 2;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     if (tid == 0) {
         for (int i = 0; i < kConsumerWarps * a.num_stages; ++i) {
             mbar_init(&sm.full[i], 1);
             mbar_init(&sm.full_v[i], 1);
+            mbar_init(&sm.empty[i], kConsumerWarps);
             sm.stage_bad[i] = 0;
         }
         for (int i = 0; i < 2; ++i) mbar_init(&sm.qfull[i], 1);
@@ -1311,7 +1629,9 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathCudaCore ? 1 : (M
     }
 
     // prefix[s] = blocks of sequences < s (clamped lengths), wprefix[s] = their
-    // weight (blocks + piece_cost per non-empty sequence); lens[s] = clamped length
+    // weight (blocks + piece_cost per non-empty sequence); lens[s] = clamped
+    // length; ptiles[s] = tiles of its group's shared prefix, which prefix units
+    // read (its blocks here are those of the rest, the suffix)
     const int S = a.num_seqs;
     const int cap = a.max_blocks_per_seq * BS * a.sub;
     const int pcost = min(max(a.piece_cost, 0), 64);  // validated on the host; a bad value moves no index
@@ -1325,7 +1645,14 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathCudaCore ? 1 : (M
             L = min(max(L, 0), cap);
         }
         sm.lens[s] = L;
-        const int n = (L + BS - 1) / BS;
+        int pt = 0;
+        for (int gi = 0; gi < a.num_groups; ++gi)
+            if (s >= a.grp_begin[gi] && s < a.grp_end[gi]) pt = a.grp_tiles[gi];
+        sm.ptiles[s] = pt;
+        // the fused append writes position L - 1 from the suffix: none inside a shared prefix
+        if (pt > 0 && a.slots != nullptr && L > 0 && L <= pt * BS && blockIdx.x == 0 && __ldg(a.slots + s) >= 0)
+            atomicOr(a.status, PKV_STATUS_BAD_SLOT);
+        const int n = max(0, (L + BS - 1) / BS - pt);
         mine += n;
         mine_w += n > 0 ? n + pcost : 0;
     }
@@ -1352,7 +1679,7 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathCudaCore ? 1 : (M
     for (int s = lo; s < hi; ++s) {
         sm.prefix[s] = run;
         sm.wprefix[s] = run_w;
-        const int n = (sm.lens[s] + BS - 1) / BS;
+        const int n = max(0, (sm.lens[s] + BS - 1) / BS - sm.ptiles[s]);
         run += n;
         run_w += n > 0 ? n + pcost : 0;
     }
@@ -1400,28 +1727,37 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathCudaCore ? 1 : (M
                 }
             }
 
+    // CTAs [0, prefix_ctas) run the prefix units; the others split the suffix
+    // blocks by weight, numbered from 0
     const long long W = static_cast<long long>(a.num_kv_heads) * sm.wprefix[S];
-    const long long x0 = blocks_below(weight_begin(blockIdx.x, W, gridDim.x), sm.prefix, sm.wprefix, S,
-                                      a.num_kv_heads, pcost);
-    const long long x1 = blocks_below(weight_begin(blockIdx.x + 1, W, gridDim.x), sm.prefix, sm.wprefix, S,
-                                      a.num_kv_heads, pcost);
+    const int cta = static_cast<int>(blockIdx.x) - a.prefix_ctas, C = static_cast<int>(gridDim.x) - a.prefix_ctas;
+    if constexpr (MATH == kMathTensorCore) {
+        if (cta < 0) {
+            prefix_unit<D>(&tm_k, &tm_v, a, sm, ly, W, C, pcost, warp, lane);
+            return;
+        }
+    }
+    const long long x0 = blocks_below(weight_begin(cta, W, C), sm.prefix, sm.wprefix, S, a.num_kv_heads, pcost);
+    const long long x1 = blocks_below(weight_begin(cta + 1, W, C), sm.prefix, sm.wprefix, S, a.num_kv_heads, pcost);
     PieceIter pieces;
     pieces.x = x0;
     pieces.x1 = x1;
     pieces.pre = sm.prefix;
     pieces.lens = sm.lens;
+    pieces.ptiles = sm.ptiles;
+    pieces.BS = BS;
     pieces.S = S;
     pieces.Hkv = a.num_kv_heads;
 
     if constexpr (MATH == kMathCudaCore) {
-        decode_warp<D, BS, CoreMath<D, BS, GP>, 2>(&tm_k, &tm_v, a, sm, ly, pieces, x0, x1, W, gridDim.x, pcost,
+        decode_warp<D, BS, CoreMath<D, BS, GP>, 2>(&tm_k, &tm_v, a, sm, ly, pieces, x0, x1, W, pcost,
                                                    warp, lane);
     } else if constexpr (MATH == kMathTensorCore) {
-        decode_warp<D, BS, MmaMath<D, BS>, 2>(&tm_k, &tm_v, a, sm, ly, pieces, x0, x1, W, gridDim.x, pcost, warp,
+        decode_warp<D, BS, MmaMath<D, BS>, 2>(&tm_k, &tm_v, a, sm, ly, pieces, x0, x1, W, pcost, warp,
                                               lane);
     } else {
         static_assert(D == 128 || D == 256, "the e4m3 path reads rows of 128 or 256 codes");
-        decode_warp<D, BS, Fp8Math<BS, D / 128>, 1>(&tm_k, &tm_v, a, sm, ly, pieces, x0, x1, W, gridDim.x, pcost,
+        decode_warp<D, BS, Fp8Math<BS, D / 128>, 1>(&tm_k, &tm_v, a, sm, ly, pieces, x0, x1, W, pcost,
                                                     warp, lane);
     }
 }

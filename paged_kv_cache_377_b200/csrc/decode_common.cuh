@@ -13,6 +13,8 @@ constexpr int kMaxStagesPerWarp = kMaxStages / kConsumerWarps;
 constexpr int kMaxSeqsPerLaunch = 2048;               // per-sequence tables kept in shared memory
 constexpr int kMaxCtas = 1024;                        // grid limit; bounds the pieces of a launch
 constexpr int kWorkspaceHeaderBytes = 256;
+constexpr int kMaxPrefixGroups = 16;                  // prefix groups per launch (kernel parameters)
+constexpr int kPrefixRows = 64;                       // query rows of one prefix unit: 16 per warp
 
 // With pack = 2 the kernel runs on a view of the pool with half the kv heads
 // and twice the head_dim: kv heads 2h', 2h' + 1 of head_dim D / 2 are the two
@@ -56,10 +58,30 @@ struct DecodeArgs {
     const float *k_scale;
     const float *v_scale;
     float scale_log2;            // scale * log2(e): logits are kept in base 2
+    // Prefix groups (bf16 pools, pack 1, tensor cores). Group g is the
+    // sequences grp_begin[g] .. grp_end[g] - 1 of the launch, whose
+    // tables agree on the blocks of their first grp_tiles[g] tiles; those tiles
+    // are read once per group by prefix units, the rest of each context (its
+    // suffix) as usual. CTAs [0, prefix_ctas) run one prefix unit each: the
+    // members of row tile rt (grp_members[g] per row tile) and kv head h against
+    // prefix piece tp (tiles_per_piece tiles), unit index grp_unit0[g] + (h *
+    // grp_row_tiles[g] + rt) * pieces + tp. Their partials take rows (pre_base +
+    // (s * Hkv + h) * prefix_np + tp) * G + g of o_part / lse_part.
+    int num_groups;
+    int prefix_ctas;
+    int tiles_per_piece;
+    int prefix_np;
+    int pre_base;
+    int grp_begin[kMaxPrefixGroups];
+    int grp_end[kMaxPrefixGroups];
+    int grp_tiles[kMaxPrefixGroups];
+    int grp_unit0[kMaxPrefixGroups + 1];
+    int grp_members[kMaxPrefixGroups];
+    int grp_row_tiles[kMaxPrefixGroups];
 };
 
 struct DecodeLayout {
-    uint32_t stages, qbuf, pscr, merge_acc, merge_m, merge_l, bars, flags, prefix, wprefix, lens, total;
+    uint32_t stages, qbuf, pscr, merge_acc, merge_m, merge_l, bars, flags, prefix, wprefix, lens, ptiles, total;
 };
 
 __host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
@@ -90,7 +112,7 @@ __host__ __device__ inline DecodeLayout decode_layout(int D, int BS, int GP, int
     off += kConsumerWarps * G * 4;
     off = align_up(off, 8);
     L.bars = off;
-    off += (2 * kMaxStages + 2) * 8;                                // full[stage], full_v[stage], qfull[2]
+    off += (3 * kMaxStages + 2) * 8;                                // full[stage], full_v[stage], qfull[2], empty[stage]
     L.flags = off;
     off += (2 * kMaxStages + 1 + 2 * kConsumerWarps + 1 + 4 * 2) * 4;  // stage_bad, abort, scan, merges, stage_blk
     L.prefix = off;
@@ -99,6 +121,8 @@ __host__ __device__ inline DecodeLayout decode_layout(int D, int BS, int GP, int
     off += static_cast<uint32_t>(num_seqs + 1) * 4;                 // weighted blocks before each sequence
     L.lens = off;
     off += static_cast<uint32_t>(num_seqs) * 4;                     // clamped context lengths
+    L.ptiles = off;
+    off += static_cast<uint32_t>(num_seqs) * 4;                     // shared-prefix tiles of each sequence (0: none)
     L.total = align_up(off, 16) + 1024;
     return L;
 }

@@ -4,6 +4,7 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
 
 import paged_kv_cache_377_b200 as pkv
@@ -235,3 +236,50 @@ def test_noalloc_binding_checks_shapes_before_calling_the_library(monkeypatch, b
         _binding.paged_attn_decode_noalloc(t["out"], t["q"], t["k_cache"], t["v_cache"], t["block_tables"],
                                            t["context_lens"], 0.125)
     assert calls == [], "the library was reached with inconsistent shapes"
+
+
+def test_find_prefix_groups_on_host_tables():
+    bt = np.array([[5, 6, 7, -1], [5, 6, 9, -1], [5, 6, 7, 8], [1, 2, 3, -1], [1, 2, 4, -1], [0, -1, -1, -1],
+                   [3, 4, -1, -1], [3, 4, -1, -1]], dtype=np.int32)
+    cl = np.array([40, 35, 60, 33, 33, 10, 20, 32], dtype=np.int32)
+    g = pkv.find_prefix_groups(bt, cl, 16)
+    assert g.begin.tolist() == [0, 3, 6] and g.end.tolist() == [3, 5, 8] and g.blocks.tolist() == [2, 2, 2]
+    # a context that covers fewer entries bounds what the run shares (seq 6 covers 2 blocks)
+    g = pkv.find_prefix_groups(bt[6:], cl[6:], 16)
+    assert g.blocks.tolist() == [2]
+    assert len(pkv.find_prefix_groups(bt, cl, 16, min_blocks=3)) == 0
+    assert len(pkv.find_prefix_groups(bt, cl, 16, max_groups=2)) == 2
+    lib = pkv.library()
+    n = ctypes.c_int(0)
+    assert lib.pkv_find_prefix_groups(None, None, 3, 4, 16, 1, None, None, None, 0, ctypes.byref(n)) == -1
+    assert lib.pkv_find_prefix_groups(None, None, 0, 4, 16, 1, None, None, None, 0, ctypes.byref(n)) == 0 and n.value == 0
+
+
+@pytest.mark.parametrize("begin,end,blocks,code,msg", [
+    ([0], [1], [2], -1, "two or more"),
+    ([2, 3], [4, 5], [2, 2], -1, "two or more"),       # overlapping groups
+    ([0], [5], [2], -1, "two or more"),                # past num_seqs (4)
+    ([0], [3], [0], -1, "blocks"),
+    ([0], [3], [4], -1, "blocks"),                     # more than max_blocks_per_seq (3)
+])
+def test_decode_checks_prefix_groups_without_touching_the_gpu(begin, end, blocks, code, msg):
+    lib = pkv.library()
+    groups = pkv.PrefixGroups(begin, end, blocks)
+    opts = pkv._binding._options(prefix_groups=groups)
+    rc = lib.paged_attn_decode_ex(P, P, P, P, P, P, 4, 2, 1, 64, 16, 0.125, 3, 16, P, 1 << 20,
+                                  ctypes.byref(opts), None)
+    assert rc == code and msg in lib.pkv_last_error().decode(), (rc, lib.pkv_last_error())
+
+
+def test_prefix_groups_need_bf16_pools_on_tensor_cores():
+    lib = pkv.library()
+    groups = pkv.PrefixGroups([0], [3], [2])
+    for kw, msg in [(dict(math=1), "tensor cores"), (dict(head_pack=2), "head packing"), (dict(tile_tokens=32), "16-row")]:
+        opts = pkv._binding._options(prefix_groups=groups, **kw)
+        rc = lib.paged_attn_decode_ex(P, P, P, P, P, P, 4, 4, 2, 64, 32, 0.125, 3, 16, P, 1 << 20,
+                                      ctypes.byref(opts), None)
+        assert rc == -2 and msg in lib.pkv_last_error().decode(), (kw, rc, lib.pkv_last_error())
+    opts = pkv._binding._options(prefix_groups=groups)
+    rc = lib.paged_attn_decode_fp8(P, P, P, P, P, P, P, P, 4, 4, 2, 128, 16, 0.125, 3, 16, P, 1 << 20,
+                                   ctypes.byref(opts), None)
+    assert rc == -2 and "tensor cores" in lib.pkv_last_error().decode()
