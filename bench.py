@@ -73,6 +73,7 @@ def parse_args(argv=None):
     p.add_argument("--piece-cost", type=int, default=0)
     p.add_argument("--head-pack", type=int, default=0)
     p.add_argument("--tile-tokens", type=int, default=0)
+    p.add_argument("--prefix-tiles", type=int, default=0)
     p.add_argument("--prefix-groups", choices=["auto", "off"], default="auto",
                    help="auto: pass the runs of sequences that share leading blocks (found on the host tables, "
                         "as an engine's block manager knows them) so that shared blocks are read once per group")
@@ -275,7 +276,8 @@ class Step:
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
         self.opts = dict(num_ctas=args.num_ctas, num_stages=args.num_stages,
                          ctas_per_sm=args.ctas_per_sm, math=args.math, l2_prefetch=args.l2_prefetch,
-                         piece_cost=args.piece_cost, head_pack=args.head_pack, tile_tokens=args.tile_tokens)
+                         piece_cost=args.piece_cost, head_pack=args.head_pack, tile_tokens=args.tile_tokens,
+                         prefix_tiles=args.prefix_tiles)
         self.groups = None
         if getattr(args, "prefix_groups", "off") == "auto" and b.kv_dtype == "bf16":
             g = pkv.find_prefix_groups(b.block_tables, b.context_lens, b.block_size)
@@ -530,7 +532,8 @@ def config_block(args, batch, world):
     }
     if args.seqs:
         c["seqs_kept"] = args.seqs
-    for k in ("num_ctas", "num_stages", "ctas_per_sm", "math", "l2_prefetch", "piece_cost", "head_pack", "tile_tokens"):
+    for k in ("num_ctas", "num_stages", "ctas_per_sm", "math", "l2_prefetch", "piece_cost", "head_pack", "tile_tokens",
+              "prefix_tiles"):
         if getattr(args, k):
             c[k] = getattr(args, k)
     return c

@@ -100,6 +100,11 @@ extern "C" {
  *                     small as for 16-token blocks and twice as many CTAs fit on
  *                     an SM; more than block_size returns PKV_ERR_INVALID_ARGUMENT.
  *                     The result does not depend on it beyond rounding order.
+ *   prefix_groups     see pkv_prefix_groups above (NULL: none).
+ *   prefix_tiles      16-row tiles of a shared prefix that one CTA streams before
+ *                     storing its partials (1..4096); default 16. Fewer spread a
+ *                     group's shared blocks over more CTAs; more partials to
+ *                     merge. Raised as needed to leave most CTAs to the rest.
  */
 /*
  * Prefix groups: runs of consecutive sequences of a batch whose block tables
@@ -141,6 +146,7 @@ typedef struct pkv_decode_options {
     int head_pack;
     int tile_tokens;
     const pkv_prefix_groups *prefix_groups;  /* NULL: none */
+    int prefix_tiles;
 } pkv_decode_options;
 
 /*

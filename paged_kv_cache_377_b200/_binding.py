@@ -41,7 +41,7 @@ class _Options(ctypes.Structure):
     _fields_ = [("num_ctas", ctypes.c_int), ("num_stages", ctypes.c_int),
                 ("ctas_per_sm", ctypes.c_int), ("math", ctypes.c_int), ("l2_prefetch", ctypes.c_int),
                 ("piece_cost", ctypes.c_int), ("head_pack", ctypes.c_int), ("tile_tokens", ctypes.c_int),
-                ("prefix_groups", ctypes.c_void_p)]
+                ("prefix_groups", ctypes.c_void_p), ("prefix_tiles", ctypes.c_int)]
 
 
 class PrefixGroups:
@@ -91,9 +91,9 @@ def find_prefix_groups(block_tables, context_lens, block_size: int, min_blocks: 
 
 
 def _options(num_ctas=0, num_stages=0, ctas_per_sm=0, math=0, l2_prefetch=0, piece_cost=0, head_pack=0,
-             tile_tokens=0, prefix_groups: Optional[PrefixGroups] = None) -> _Options:
+             tile_tokens=0, prefix_groups: Optional[PrefixGroups] = None, prefix_tiles=0) -> _Options:
     return _Options(num_ctas, num_stages, ctas_per_sm, math, l2_prefetch, piece_cost, head_pack, tile_tokens,
-                    prefix_groups.c_ptr() if prefix_groups is not None else None)
+                    prefix_groups.c_ptr() if prefix_groups is not None else None, prefix_tiles)
 
 
 def library_path() -> str:
@@ -224,7 +224,7 @@ def paged_attn_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
                       workspace: torch.Tensor, num_ctas: int = 0, num_stages: int = 0,
                       ctas_per_sm: int = 0, math: int = 0, l2_prefetch: int = 0, piece_cost: int = 0,
                       head_pack: int = 0, tile_tokens: int = 0, prefix_groups: Optional[PrefixGroups] = None,
-                      stream=None) -> torch.Tensor:
+                      prefix_tiles: int = 0, stream=None) -> torch.Tensor:
     """out[s, j] = softmax_t(scale * q[s, j] . K_t) . V_t over the sequence's paged tokens.
 
     q, out: bf16 [S, Hq, D]; k_cache, v_cache: bf16 [NB, bs, Hkv, D];
@@ -242,7 +242,7 @@ def paged_attn_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
     _need(workspace, "workspace", torch.uint8, 1)
     S, Hq, D, NB, bs, Hkv = _decode_shapes(out, q, k_cache, v_cache, block_tables, context_lens)
     opts = _options(num_ctas, num_stages, ctas_per_sm, math, l2_prefetch, piece_cost, head_pack, tile_tokens,
-                    prefix_groups)
+                    prefix_groups, prefix_tiles)
     _check("paged_attn_decode", library().paged_attn_decode_ex(
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(context_lens),
         S, Hq, Hkv, D, bs, float(scale), block_tables.shape[1], NB, _ptr(workspace), workspace.numel(),
@@ -256,7 +256,7 @@ def paged_attn_decode_append(out: torch.Tensor, q: torch.Tensor, k_new: torch.Te
                              workspace: torch.Tensor, num_ctas: int = 0, num_stages: int = 0,
                              ctas_per_sm: int = 0, math: int = 0, l2_prefetch: int = 0, piece_cost: int = 0,
                              head_pack: int = 0, tile_tokens: int = 0, prefix_groups: Optional[PrefixGroups] = None,
-                             stream=None) -> torch.Tensor:
+                             prefix_tiles: int = 0, stream=None) -> torch.Tensor:
     """One decode step in one launch: append k_new / v_new (bf16 [S, Hkv, D]) at
     slot_mapping (int64 [S], the slot of each sequence's last position, < 0 =
     none), then the same attention as paged_attn_decode over contexts that
@@ -281,7 +281,7 @@ def paged_attn_decode_append(out: torch.Tensor, q: torch.Tensor, k_new: torch.Te
     if block_tables.shape[0] != S or context_lens.shape[0] != S:
         raise ValueError("block_tables and context_lens must have num_seqs rows")
     opts = _options(num_ctas, num_stages, ctas_per_sm, math, l2_prefetch, piece_cost, head_pack, tile_tokens,
-                    prefix_groups)
+                    prefix_groups, prefix_tiles)
     _check("paged_attn_decode_append", library().paged_attn_decode_append(
         _ptr(out), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(slot_mapping), _ptr(k_cache), _ptr(v_cache),
         _ptr(block_tables), _ptr(context_lens), S, Hq, Hkv, D, bs, float(scale), block_tables.shape[1], NB,

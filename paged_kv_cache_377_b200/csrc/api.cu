@@ -158,7 +158,7 @@ constexpr int kPrefixTilesPerPiece = 16;
 // the caller's descriptor that have at least two members in the launch, as
 // kernel parameters. Leaves a.num_groups = 0 when grouping does not apply.
 void plan_prefix_groups(const pkv_prefix_groups *pg, int s0, int sc, int hkv, int group, int sub, int ctas,
-                        pkv::DecodeArgs &a) {
+                        int tiles_per_piece, pkv::DecodeArgs &a) {
     a.num_groups = 0;
     a.prefix_ctas = 0;
     a.tiles_per_piece = 1;
@@ -186,7 +186,7 @@ void plan_prefix_groups(const pkv_prefix_groups *pg, int s0, int sc, int hkv, in
     const long long room = 1024LL * hkv - ctas;
     const long long np_max = room / (static_cast<long long>(sc) * hkv);
     if (np_max < 1) return;
-    int tpp = kPrefixTilesPerPiece;
+    int tpp = tiles_per_piece > 0 ? tiles_per_piece : kPrefixTilesPerPiece;
     if ((max_tiles + tpp - 1) / tpp > np_max) tpp = static_cast<int>((max_tiles + np_max - 1) / np_max);
     long long units = 0;
     for (;;) {
@@ -282,11 +282,12 @@ int decode_impl(void *out, const void *q, const void *k_new, const void *v_new, 
         !aligned(workspace, 256))
         return fail(PKV_ERR_INVALID_ARGUMENT,
                     "out, q, k_cache and v_cache must be 16-byte aligned and workspace 256-byte aligned");
-    pkv_decode_options o = {0, 0, 0, 0, 0, 0, 0, 0, nullptr};
+    pkv_decode_options o = {0, 0, 0, 0, 0, 0, 0, 0, nullptr, 0};
     if (opts) o = *opts;
     if (o.num_ctas < 0 || o.num_stages < 0 || o.ctas_per_sm < 0 || o.math < 0 || o.math > 2 ||
         o.l2_prefetch < -1 || o.l2_prefetch > 32 || o.piece_cost < -1 || o.piece_cost > 64 || o.head_pack < 0 ||
-        o.head_pack > 2 || (o.tile_tokens != 0 && o.tile_tokens != 16 && o.tile_tokens != 32))
+        o.head_pack > 2 || (o.tile_tokens != 0 && o.tile_tokens != 16 && o.tile_tokens != 32) || o.prefix_tiles < 0 ||
+        o.prefix_tiles > 4096)
         return fail(PKV_ERR_INVALID_ARGUMENT, "negative or unknown option");
     if (o.tile_tokens > block_size)
         return fail(PKV_ERR_INVALID_ARGUMENT, "tile_tokens %d exceeds block_size %d", o.tile_tokens, block_size);
@@ -395,7 +396,7 @@ int decode_impl(void *out, const void *q, const void *k_new, const void *v_new, 
         a.prefetch = o.l2_prefetch > 0 ? o.l2_prefetch : o.l2_prefetch == 0 ? kDefaultL2Prefetch : 0;
         a.piece_cost = o.piece_cost > 0 ? o.piece_cost : o.piece_cost == 0 ? kDefaultPieceCost : 0;
         a.scale_log2 = scale * 1.4426950408889634f;
-        plan_prefix_groups(pg, s0, sc, khkv, kgroup, a.sub, grid, a);
+        plan_prefix_groups(pg, s0, sc, khkv, kgroup, a.sub, grid, o.prefix_tiles, a);
         if (fused) {
             const size_t row = static_cast<size_t>(num_kv_heads) * head_dim;  // elements per token
             a.k_new = static_cast<const __nv_bfloat16 *>(k_new) + static_cast<size_t>(s0) * row;
