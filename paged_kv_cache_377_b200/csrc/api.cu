@@ -397,6 +397,15 @@ int decode_impl(void *out, const void *q, const void *k_new, const void *v_new, 
         a.piece_cost = o.piece_cost > 0 ? o.piece_cost : o.piece_cost == 0 ? kDefaultPieceCost : 0;
         a.scale_log2 = scale * 1.4426950408889634f;
         plan_prefix_groups(pg, s0, sc, khkv, kgroup, a.sub, grid, o.prefix_tiles, a);
+        // a launch with prefix groups runs the kernel that has the prefix units
+        // (same shared memory and CTAs per SM)
+        const int kmath = a.num_groups > 0 ? pkv::kMathTensorCoreGroups : math;
+        if (kmath != math) {
+            int per_sm_g = 0;
+            e = pkv::decode_prepare(kd, tile, gp, kmath, smem, &per_sm_g);
+            if (e != cudaSuccess) return cuda_fail(e, "decode kernel setup");
+            if (per_sm_g < per_sm) return fail(PKV_ERR_CUDA, "the prefix-group kernel fits fewer CTAs per SM");
+        }
         if (fused) {
             const size_t row = static_cast<size_t>(num_kv_heads) * head_dim;  // elements per token
             a.k_new = static_cast<const __nv_bfloat16 *>(k_new) + static_cast<size_t>(s0) * row;
@@ -407,7 +416,7 @@ int decode_impl(void *out, const void *q, const void *k_new, const void *v_new, 
         }
         a.k_scale = k_scale;
         a.v_scale = v_scale;
-        e = pkv::decode_launch(kd, tile, gp, math, tm_k, tm_v, a, grid, smem, st);
+        e = pkv::decode_launch(kd, tile, gp, kmath, tm_k, tm_v, a, grid, smem, st);
         if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
     }
     return ok();

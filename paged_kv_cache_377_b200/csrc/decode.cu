@@ -893,30 +893,39 @@ __device__ __forceinline__ int segment_pieces(int s, int h, const Smem &sm, int 
     return live_prefix_pieces(s, sm, BS, tiles_per_piece) + sp.npieces;
 }
 
-// Lists the partial-row bases of segment (s, h)'s pieces (prefix pieces first)
-// into `list`; threads of the CTA share the work. Returns the count.
-__device__ __forceinline__ int list_pieces(const DecodeArgs &a, int s, int h, const Smem &sm, long long W, int C,
-                                           int pcost, int BS, int *list, int ctid) {
+// The partial-row bases of segment (s, h)'s pieces, prefix pieces first:
+// operator()(i) is piece i's base (its partial rows are base * G + g).
+struct PieceBases {
     SegmentSpan sp;
-    const int n = segment_pieces(s, h, sm, a.num_kv_heads, W, C, pcost, BS, a.tiles_per_piece, &sp);
-    const int npre = n - sp.npieces;
-    const int seg = s * a.num_kv_heads + h;
-    for (int j = ctid; j < n; j += kConsumerWarps * 32)
-        list[j] = j < npre ? a.pre_base + seg * a.prefix_np + j : seg + piece_cta(sp, j - npre, W, C);
+    long long W;
+    int C, npre, seg, pre;  // pre: base of the segment's first prefix piece
+    __device__ __forceinline__ int operator()(int i) const {
+        return i < npre ? pre + i : seg + piece_cta(sp, i - npre, W, C);
+    }
+};
+
+// Pieces of segment (s, h) and where their partials are (returns the count).
+__device__ __forceinline__ int piece_bases(const DecodeArgs &a, int s, int h, const Smem &sm, long long W, int C,
+                                           int pcost, int BS, PieceBases &pb) {
+    const int n = segment_pieces(s, h, sm, a.num_kv_heads, W, C, pcost, BS, a.tiles_per_piece, &pb.sp);
+    pb.W = W;
+    pb.C = C;
+    pb.npre = n - pb.sp.npieces;
+    pb.seg = s * a.num_kv_heads + h;
+    pb.pre = a.pre_base + pb.seg * a.prefix_np;
     return n;
 }
 
 // Merge of the pieces of segment (s, h) whose partials sit at rows
-// piece_base[i] * G + g, i < npieces (log-sum-exp identity, in list order: the
+// base(i) * G + g, i < npieces (log-sum-exp identity, in that order: the
 // prefix pieces, then the suffix pieces in CTA order): out = sum_c 2^(lse_c - M)
 // o_c / sum_c 2^(lse_c - M), taken in one pass with a running maximum. A thread merges 4-dim elements of the G x D
 // output (at most two) and loads four pieces ahead, so that the merge costs a
 // few L2 round trips rather than one per piece. Partials written by other SMs
 // are read past L1.
-template <int D>
-__device__ __forceinline__ void merge_pieces(const DecodeArgs &a, const int *piece_base, int npieces, int s, int h,
+template <int D, int kAhead = 4, class Base>
+__device__ __forceinline__ void merge_pieces(const DecodeArgs &a, const Base &base, int npieces, int s, int h,
                                              int ctid) {
-    constexpr int kAhead = 4;
     const int G = a.group;
     const int DR = D / a.pack;
 #pragma unroll 1
@@ -933,7 +942,7 @@ __device__ __forceinline__ void merge_pieces(const DecodeArgs &a, const int *pie
             for (int i = 0; i < kAhead; ++i) {
                 lse[i] = -INFINITY;
                 if (ib + i < npieces) {
-                    const size_t pr = static_cast<size_t>(piece_base[ib + i]) * G + g;
+                    const size_t pr = static_cast<size_t>(base(ib + i)) * G + g;
                     lse[i] = __ldcg(a.lse_part + pr);
                     o[i] = __ldcg(reinterpret_cast<const float4 *>(a.o_part + pr * DR + col));
                 }
@@ -969,7 +978,7 @@ __device__ __forceinline__ void merge_pieces(const DecodeArgs &a, const int *pie
 // in flight than the ring can hold. Block-table entries of its next 32 blocks
 // are looked up one batch ahead. Warp 0 also bulk-copies the query rows of the piece after
 // next. All four warps meet at the end of every piece to merge their states.
-template <int D, int BS, class Math, int ES>
+template <int D, int BS, class Math, int ES, bool GROUPS>
 __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUtensorMap *tm_v, const DecodeArgs &a,
                                             const Smem &sm, const DecodeLayout &ly, PieceIter pieces, long long x0,
                                             long long x1, long long W, int pcost, int warp, int lane) {
@@ -1009,7 +1018,7 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
             const int n = sm.prefix[lo + 1] - sm.prefix[lo];
             const int r = static_cast<int>(x - static_cast<long long>(a.num_kv_heads) * sm.prefix[lo]);
             h = r / n;
-            const int j = r - h * n + sm.ptiles[lo];  // logical tile of the context
+            const int j = r - h * n + (GROUPS ? sm.ptiles[lo] : 0);  // logical tile of the context
             const int pb = __ldg(a.block_tables + static_cast<size_t>(lo) * a.max_blocks_per_seq + (j >> sub_shift));
             p = (pb < 0 || pb >= a.num_blocks) ? -1 : ((pb << sub_shift) + (j & (a.sub - 1))) * BS;
         }
@@ -1256,11 +1265,27 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
                     old = prev;
                 }
                 const int pending = sm.merge_flag[0];
-                if (static_cast<int>(now & 0xffffull) == total && pending < 2) {  // never more than two (below)
-                    volatile int *m = sm.merge_flag + 1 + 2 * pending;
-                    m[0] = pc.s;
-                    m[1] = pc.h;
-                    sm.merge_flag[0] = pending + 1;
+                sm.merge_flag[5] = 0;
+                if (static_cast<int>(now & 0xffffull) == total) {
+                    if (GROUPS && sm.ptiles[pc.s] > 0) {
+                        // a shared-prefix segment: all its suffix pieces can be
+                        // cut ones, so this CTA may complete many; merged now
+                        sm.merge_flag[5] = 1;
+                    } else if (pending < 2) {  // never more than two (below)
+                        volatile int *m = sm.merge_flag + 1 + 2 * pending;
+                        m[0] = pc.s;
+                        m[1] = pc.h;
+                        sm.merge_flag[0] = pending + 1;
+                    }
+                }
+            }
+            named_barrier_sync(1, kConsumerWarps * 32);
+            if constexpr (GROUPS) {
+                if (sm.merge_flag[5] && !*sm.abort_flag) {
+                    __threadfence();
+                    PieceBases pb;
+                    const int n = piece_bases(a, pc.s, pc.h, sm, W, gridDim.x - a.prefix_ctas, pcost, BS, pb);
+                    merge_pieces<D, 1>(a, pb, n, pc.s, pc.h, ctid);  // one piece at a time: the loop's state is live
                 }
             }
         }
@@ -1293,13 +1318,9 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
         __threadfence();
         // the grid's total weight, reloaded rather than kept live across the loop
         const long long Wt = static_cast<long long>(a.num_kv_heads) * sm.wprefix[a.num_seqs];
-        // the partial of each piece, listed in the (now idle) stage buffers: at
-        // least 16 KB, and a segment has at most kMaxCtas + 1024 pieces
-        int *list = reinterpret_cast<int *>(sm.base + ly.stages);
-        if (i > 0) named_barrier_sync(1, kConsumerWarps * 32);  // the previous merge is done with the list
-        const int n = list_pieces(a, s, h, sm, Wt, gridDim.x - a.prefix_ctas, pcost, BS, list, ctid);
-        named_barrier_sync(1, kConsumerWarps * 32);
-        merge_pieces<D>(a, list, n, s, h, ctid);
+        PieceBases pb;
+        const int n = piece_bases(a, s, h, sm, Wt, gridDim.x - a.prefix_ctas, pcost, BS, pb);
+        merge_pieces<D>(a, pb, n, s, h, ctid);
     }
 }
 
@@ -1548,7 +1569,6 @@ __device__ __forceinline__ void prefix_unit(const CUtensorMap *tm_k, const CUten
     __threadfence();
     named_barrier_sync(1, kConsumerWarps * 32);
     int *mlist = reinterpret_cast<int *>(sm.base + ly.stages);  // [0] count, [1 ..] members to merge
-    int *plist = mlist + 2 * kPrefixRows;                        // partial rows of one segment
     if (ctid == 0) mlist[0] = 0;
     named_barrier_sync(1, kConsumerWarps * 32);
     if (ctid < m1 - m0) {
@@ -1571,10 +1591,9 @@ __device__ __forceinline__ void prefix_unit(const CUtensorMap *tm_k, const CUten
     for (int i = 0; i < nmerge; ++i) {
         const int s = mlist[1 + i];
         __threadfence();
-        const int n = list_pieces(a, s, h, sm, W, C, pcost, BS, plist, ctid);
-        named_barrier_sync(1, kConsumerWarps * 32);
-        merge_pieces<D>(a, plist, n, s, h, ctid);
-        named_barrier_sync(1, kConsumerWarps * 32);  // the list is rewritten by the next merge
+        PieceBases pb;
+        const int n = piece_bases(a, s, h, sm, W, C, pcost, BS, pb);
+        merge_pieces<D>(a, pb, n, s, h, ctid);
     }
 }
 
@@ -1590,6 +1609,7 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathCudaCore ? 1 : (M
     static_assert(BS == 16 || BS == 32, "block_size");
     static_assert(GP == 1 || GP == 2 || GP == 4 || GP == 8, "group");
     static_assert(MATH == kMathCudaCore || GP == 8, "the tensor-core path pads the group to 8");
+    constexpr bool GROUPS = MATH == kMathTensorCoreGroups;
     extern __shared__ uint8_t smem_raw[];
     constexpr int ES = MATH == kMathFp8 ? 1 : 2;  // bytes per pool element
     const DecodeLayout ly = decode_layout(D, BS, GP, a.group, MATH != kMathCudaCore, kConsumerWarps * a.num_stages,
@@ -1731,7 +1751,7 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathCudaCore ? 1 : (M
     // blocks by weight, numbered from 0
     const long long W = static_cast<long long>(a.num_kv_heads) * sm.wprefix[S];
     const int cta = static_cast<int>(blockIdx.x) - a.prefix_ctas, C = static_cast<int>(gridDim.x) - a.prefix_ctas;
-    if constexpr (MATH == kMathTensorCore) {
+    if constexpr (GROUPS) {
         if (cta < 0) {
             prefix_unit<D>(&tm_k, &tm_v, a, sm, ly, W, C, pcost, warp, lane);
             return;
@@ -1750,14 +1770,14 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathCudaCore ? 1 : (M
     pieces.Hkv = a.num_kv_heads;
 
     if constexpr (MATH == kMathCudaCore) {
-        decode_warp<D, BS, CoreMath<D, BS, GP>, 2>(&tm_k, &tm_v, a, sm, ly, pieces, x0, x1, W, pcost,
+        decode_warp<D, BS, CoreMath<D, BS, GP>, 2, false>(&tm_k, &tm_v, a, sm, ly, pieces, x0, x1, W, pcost,
                                                    warp, lane);
-    } else if constexpr (MATH == kMathTensorCore) {
-        decode_warp<D, BS, MmaMath<D, BS>, 2>(&tm_k, &tm_v, a, sm, ly, pieces, x0, x1, W, pcost, warp,
+    } else if constexpr (MATH == kMathTensorCore || GROUPS) {
+        decode_warp<D, BS, MmaMath<D, BS>, 2, GROUPS>(&tm_k, &tm_v, a, sm, ly, pieces, x0, x1, W, pcost, warp,
                                               lane);
     } else {
         static_assert(D == 128 || D == 256, "the e4m3 path reads rows of 128 or 256 codes");
-        decode_warp<D, BS, Fp8Math<BS, D / 128>, 1>(&tm_k, &tm_v, a, sm, ly, pieces, x0, x1, W, pcost,
+        decode_warp<D, BS, Fp8Math<BS, D / 128>, 1, false>(&tm_k, &tm_v, a, sm, ly, pieces, x0, x1, W, pcost,
                                                     warp, lane);
     }
 }
@@ -1776,6 +1796,7 @@ KernelFn pick(int D, int BS, int GP, int math) {
     PKV_GP(64, 16) PKV_GP(64, 32) PKV_GP(128, 16) PKV_GP(128, 32)
     PKV_CASE(128, 16, 8, kMathFp8) PKV_CASE(128, 32, 8, kMathFp8)
     PKV_CASE(256, 16, 8, kMathFp8) PKV_CASE(256, 32, 8, kMathFp8)
+    PKV_CASE(64, 16, 8, kMathTensorCoreGroups) PKV_CASE(128, 16, 8, kMathTensorCoreGroups)
 #undef PKV_GP
 #undef PKV_CASE
     return nullptr;

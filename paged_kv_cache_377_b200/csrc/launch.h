@@ -12,7 +12,10 @@ namespace pkv {
 
 // kMathFp8: tensor-core (f16 mma.sync) math over e4m3 pools with per-head
 // scales; chosen by the fp8 entry points, not by the math option.
-enum DecodeMath { kMathCudaCore = 1, kMathTensorCore = 2, kMathFp8 = 3 };
+// kMathTensorCoreGroups: kMathTensorCore plus the prefix units of prefix
+// groups; chosen for a launch that has groups (a kernel of its own, so that
+// launches without groups keep the leaner register allocation).
+enum DecodeMath { kMathCudaCore = 1, kMathTensorCore = 2, kMathFp8 = 3, kMathTensorCoreGroups = 4 };
 
 // True when the (head_dim, block_size, padded group, math) combination is compiled in.
 bool decode_variant_exists(int head_dim, int block_size, int group_pad, int math);
