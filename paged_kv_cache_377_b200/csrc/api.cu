@@ -366,9 +366,18 @@ int decode_impl(void *out, const void *q, const void *k_new, const void *v_new, 
     // in shared memory); launches run in stream order and reuse the workspace.
     for (int s0 = 0; s0 < num_seqs; s0 += pkv::kMaxSeqsPerLaunch) {
         const int sc = num_seqs - s0 < pkv::kMaxSeqsPerLaunch ? num_seqs - s0 : pkv::kMaxSeqsPerLaunch;
-        const size_t smem = pkv::decode_smem_bytes(kd, tile, gp, kgroup, math, ns, sc, pack);
+        // a launch that may have prefix groups is sized for the kernel with the
+        // prefix units (its shared memory can be larger)
+        bool may_group = false;
+        for (int g = 0; pg && g < pg->num_groups; ++g) {
+            const int lo = pg->begin[g] > s0 ? pg->begin[g] : s0;
+            const int hi = pg->end[g] < s0 + sc ? pg->end[g] : s0 + sc;
+            may_group |= hi - lo >= 2;
+        }
+        const int gmath = may_group ? pkv::kMathTensorCoreGroups : math;
+        const size_t smem = pkv::decode_smem_bytes(kd, tile, gp, kgroup, gmath, ns, sc, pack);
         int per_sm = 0;
-        cudaError_t e = pkv::decode_prepare(kd, tile, gp, math, smem, &per_sm);
+        cudaError_t e = pkv::decode_prepare(kd, tile, gp, gmath, smem, &per_sm);
         if (e != cudaSuccess) return cuda_fail(e, "decode kernel setup");
         if (per_sm <= 0) return fail(PKV_ERR_INVALID_ARGUMENT, "shared memory %zu bytes per CTA does not fit", smem);
         if (o.ctas_per_sm > 0 && o.ctas_per_sm < per_sm) per_sm = o.ctas_per_sm;
@@ -396,15 +405,16 @@ int decode_impl(void *out, const void *q, const void *k_new, const void *v_new, 
         a.prefetch = o.l2_prefetch > 0 ? o.l2_prefetch : o.l2_prefetch == 0 ? kDefaultL2Prefetch : 0;
         a.piece_cost = o.piece_cost > 0 ? o.piece_cost : o.piece_cost == 0 ? kDefaultPieceCost : 0;
         a.scale_log2 = scale * 1.4426950408889634f;
-        plan_prefix_groups(pg, s0, sc, khkv, kgroup, a.sub, grid, o.prefix_tiles, a);
-        // a launch with prefix groups runs the kernel that has the prefix units
-        // (same shared memory and CTAs per SM)
+        plan_prefix_groups(may_group ? pg : nullptr, s0, sc, khkv, kgroup, a.sub, grid, o.prefix_tiles, a);
+        // a launch whose groups were planned runs the kernel with the prefix
+        // units; one whose groups were dropped runs the plain kernel in the
+        // same shared memory and grid
         const int kmath = a.num_groups > 0 ? pkv::kMathTensorCoreGroups : math;
-        if (kmath != math) {
-            int per_sm_g = 0;
-            e = pkv::decode_prepare(kd, tile, gp, kmath, smem, &per_sm_g);
+        if (kmath != gmath) {
+            int per_sm_b = 0;
+            e = pkv::decode_prepare(kd, tile, gp, kmath, smem, &per_sm_b);
             if (e != cudaSuccess) return cuda_fail(e, "decode kernel setup");
-            if (per_sm_g < per_sm) return fail(PKV_ERR_CUDA, "the prefix-group kernel fits fewer CTAs per SM");
+            if (per_sm_b < per_sm) return fail(PKV_ERR_CUDA, "the decode kernel fits fewer CTAs per SM");
         }
         if (fused) {
             const size_t row = static_cast<size_t>(num_kv_heads) * head_dim;  // elements per token

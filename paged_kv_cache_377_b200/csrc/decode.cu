@@ -278,6 +278,11 @@ struct CoreMath {
         __syncwarp();
     }
 
+    __device__ __forceinline__ void block(uint32_t ktile, uint32_t vtile, int valid) {
+        qk(ktile, valid);
+        pv(vtile, valid);
+    }
+
     __device__ __forceinline__ void pv(uint32_t vtile, int valid) {
         // P.V: tokens past the context are skipped, never multiplied by p = 0
 #pragma unroll
@@ -458,6 +463,11 @@ struct MmaMath {
         m0 = n0;
         m1 = n1;
         __syncwarp();
+    }
+
+    __device__ __forceinline__ void block(uint32_t ktile, uint32_t vtile, int valid) {
+        qk(ktile, valid);
+        pv(vtile, valid);
     }
 
     __device__ __forceinline__ void pv(uint32_t vtile, int valid) {
@@ -744,6 +754,11 @@ struct Fp8Math {
         __syncwarp();
     }
 
+    __device__ __forceinline__ void block(uint32_t ktile, uint32_t vtile, int valid) {
+        qk(ktile, valid);
+        pv(vtile, valid);
+    }
+
     __device__ __forceinline__ void pv(uint32_t vtile, int valid) {
         const int mi = lane >> 3, r = lane & 7;
         // O^T += V^T . P^T; one ldmatrix x4 .trans covers tokens 0-15 of two dim tiles
@@ -834,7 +849,7 @@ struct Fp8Math {
 
 struct Smem {
     uint8_t *base;
-    uint64_t *full, *full_v, *qfull;  // per stage: K tile landed, V tile landed; query slots
+    uint64_t *full, *qfull;  // per stage: its K and V tiles landed; query slots
     volatile int *stage_bad;
     int *stage_blk;  // [kMaxStages] first pool row of the tile whose copy the stage holds
     volatile int *abort_flag;
@@ -919,53 +934,75 @@ __device__ __forceinline__ int piece_bases(const DecodeArgs &a, int s, int h, co
 // Merge of the pieces of segment (s, h) whose partials sit at rows
 // base(i) * G + g, i < npieces (log-sum-exp identity, in that order: the
 // prefix pieces, then the suffix pieces in CTA order): out = sum_c 2^(lse_c - M)
-// o_c / sum_c 2^(lse_c - M), taken in one pass with a running maximum. A thread merges 4-dim elements of the G x D
-// output (at most two) and loads four pieces ahead, so that the merge costs a
-// few L2 round trips rather than one per piece. Partials written by other SMs
-// are read past L1.
-template <int D, int kAhead = 4, class Base>
+// o_c / sum_c 2^(lse_c - M), taken in one pass with a running maximum. A
+// thread merges 4-dim elements of the G x D output (at most two) with the
+// loads of kAhead pieces of both in flight, so that the merge costs a few L2
+// round trips rather than one per piece. Partials written by other SMs are
+// read past L1.
+// Elements a thread merges: the G x D / 4 float4 columns over the CTA's threads (G <= 8).
+template <int D>
+constexpr int merge_elems() { return (8 * (D / 4) + kConsumerWarps * 32 - 1) / (kConsumerWarps * 32); }
+
+template <int D, int kAhead = (8 / merge_elems<D>() > 0 ? 8 / merge_elems<D>() : 1), class Base>
 __device__ __forceinline__ void merge_pieces(const DecodeArgs &a, const Base &base, int npieces, int s, int h,
                                              int ctid) {
+    constexpr int kE = merge_elems<D>();
     const int G = a.group;
     const int DR = D / a.pack;
-#pragma unroll 1
-    for (int e = ctid; e < G * (D / 4); e += kConsumerWarps * 32) {
-        const int g = e / (D / 4);
-        const int col = (e % (D / 4)) * 4 - (a.pack == 2 ? g / (G >> 1) : 0) * DR;
-        if (col < 0 || col >= DR) continue;  // the other half of a packed virtual head
-        float M = -INFINITY, den = 0.f;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int ib = 0; ib < npieces; ib += kAhead) {
-            float lse[kAhead];
-            float4 o[kAhead];
+    int eg[kE], ecol[kE];
+    float M[kE], den[kE];
+    float4 acc[kE];
 #pragma unroll
-            for (int i = 0; i < kAhead; ++i) {
-                lse[i] = -INFINITY;
-                if (ib + i < npieces) {
-                    const size_t pr = static_cast<size_t>(base(ib + i)) * G + g;
-                    lse[i] = __ldcg(a.lse_part + pr);
-                    o[i] = __ldcg(reinterpret_cast<const float4 *>(a.o_part + pr * DR + col));
+    for (int k = 0; k < kE; ++k) {
+        const int e = ctid + k * kConsumerWarps * 32;
+        eg[k] = e / (D / 4);
+        ecol[k] = (e % (D / 4)) * 4 - (a.pack == 2 ? eg[k] / (G >> 1) : 0) * DR;
+        if (e >= G * (D / 4) || ecol[k] < 0 || ecol[k] >= DR) ecol[k] = -1;  // none, or the other half of a packed head
+        M[k] = -INFINITY;
+        den[k] = 0.f;
+        acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    // every element's loads of kAhead pieces are in flight together
+    for (int ib = 0; ib < npieces; ib += kAhead) {
+        float lse[kAhead][kE];
+        float4 o[kAhead][kE];
+#pragma unroll
+        for (int i = 0; i < kAhead; ++i) {
+            const size_t pb = ib + i < npieces ? static_cast<size_t>(base(ib + i)) : 0;
+#pragma unroll
+            for (int k = 0; k < kE; ++k) {
+                lse[i][k] = -INFINITY;
+                if (ib + i < npieces && ecol[k] >= 0) {
+                    const size_t pr = pb * G + eg[k];
+                    lse[i][k] = __ldcg(a.lse_part + pr);
+                    o[i][k] = __ldcg(reinterpret_cast<const float4 *>(a.o_part + pr * DR + ecol[k]));
                 }
             }
-#pragma unroll
-            for (int i = 0; i < kAhead; ++i) {
-                if (!(lse[i] > -INFINITY)) continue;  // no piece here
-                const float Mn = fmaxf(M, lse[i]);
-                const float r = fast_exp2(M - Mn), w = fast_exp2(lse[i] - Mn);
-                den = den * r + w;
-                acc.x = acc.x * r + w * o[i].x;
-                acc.y = acc.y * r + w * o[i].y;
-                acc.z = acc.z * r + w * o[i].z;
-                acc.w = acc.w * r + w * o[i].w;
-                M = Mn;
-            }
         }
-        const size_t row = static_cast<size_t>(s) * a.num_q_heads + static_cast<size_t>(h) * G + g;
-        const float inv = 1.f / den;
+#pragma unroll
+        for (int i = 0; i < kAhead; ++i)
+#pragma unroll
+            for (int k = 0; k < kE; ++k) {
+                if (!(lse[i][k] > -INFINITY)) continue;  // no piece here
+                const float Mn = fmaxf(M[k], lse[i][k]);
+                const float r = fast_exp2(M[k] - Mn), w = fast_exp2(lse[i][k] - Mn);
+                den[k] = den[k] * r + w;
+                acc[k].x = acc[k].x * r + w * o[i][k].x;
+                acc[k].y = acc[k].y * r + w * o[i][k].y;
+                acc[k].z = acc[k].z * r + w * o[i][k].z;
+                acc[k].w = acc[k].w * r + w * o[i][k].w;
+                M[k] = Mn;
+            }
+    }
+#pragma unroll
+    for (int k = 0; k < kE; ++k) {
+        if (ecol[k] < 0) continue;
+        const size_t row = static_cast<size_t>(s) * a.num_q_heads + static_cast<size_t>(h) * G + eg[k];
+        const float inv = 1.f / den[k];
         __nv_bfloat162 *dst =
-            reinterpret_cast<__nv_bfloat162 *>(static_cast<__nv_bfloat16 *>(a.out) + row * DR + col);
-        dst[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-        dst[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+            reinterpret_cast<__nv_bfloat162 *>(static_cast<__nv_bfloat16 *>(a.out) + row * DR + ecol[k]);
+        dst[0] = __floats2bfloat162_rn(acc[k].x * inv, acc[k].y * inv);
+        dst[1] = __floats2bfloat162_rn(acc[k].z * inv, acc[k].w * inv);
     }
 }
 
@@ -1026,15 +1063,12 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
     int bat_k = 0, bat_p, bat_h, nxt_p, nxt_h;
     lookup(0, bat_p, bat_h);
     lookup(32, nxt_p, nxt_h);
-    // Copies this warp issued and has not yet seen land: bit `stage` of the K
-    // (low 16 bits) and V (high 16 bits) halves, with the phase parity each waits for.
-    uint32_t inflight = 0, inflight_par = 0;
+    uint32_t inflight = 0, inflight_par = 0;  // stages whose copy this warp issued and has not yet seen land
     // Block k goes to stage warp + 4 (k % R) with phase parity (k / R) & 1, so
-    // block k + R reuses block k's stage with the other parity. The K and V
-    // tiles of a stage complete on their own barriers (full, full_v): the K tile
-    // is refilled as soon as q.K is done, while P.V still reads the V tile.
-    int iss_p = 0, iss_h = 0;  // the last K copy's block, for the V copy that follows it
-    auto issue_k = [&](int k, int stage, uint32_t par) {  // warp-uniform; k increases call after call
+    // block k + R reuses block k's stage with the other parity. (Refilling the
+    // K tile as soon as q.K is done, on a barrier of its own, measured slower:
+    // the wait between q.K and P.V keeps the compiler from overlapping them.)
+    auto issue = [&](int k, int stage, uint32_t par) {  // warp-uniform; k increases call after call
         if (k >= nk) return;
         if (k - bat_k >= 32) {
             bat_k += 32;
@@ -1044,8 +1078,6 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
         }
         const int p = __shfl_sync(0xffffffffu, bat_p, k - bat_k);
         const int h = __shfl_sync(0xffffffffu, bat_h, k - bat_k);
-        iss_p = p;
-        iss_h = h;
         if (a.prefetch > 0) {  // this warp's block k + prefetch, from the current or the next batch (<= 32 ahead)
             const int kp = k + a.prefetch, jp = kp - bat_k;
             const int pp_a = __shfl_sync(0xffffffffu, bat_p, jp & 31), pp_b = __shfl_sync(0xffffffffu, nxt_p, jp & 31);
@@ -1067,38 +1099,21 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
                 atomicOr(a.status, PKV_STATUS_BAD_BLOCK_ID);
                 mbar_arrive(&sm.full[stage]);
             } else {
-                // The tile's previous contents were read with ldmatrix / ld.shared whose
+                // The stage's previous contents were read with ldmatrix / ld.shared whose
                 // results this warp has already consumed, so the copy cannot overtake them.
                 uint8_t *dst = sm.base + ly.stages + static_cast<uint32_t>(stage) * 2u * kTile;
-                mbar_arrive_expect_tx(&sm.full[stage], kTile);
+                mbar_arrive_expect_tx(&sm.full[stage], 2u * kTile);
 #pragma unroll
-                for (int half = 0; half < kCopies; ++half)
+                for (int half = 0; half < kCopies; ++half) {
                     tma_load_4d(dst + half * kHalf, tm_k, &sm.full[stage], 0, half, h, p);
+                    tma_load_4d(dst + kTile + half * kHalf, tm_v, &sm.full[stage], 0, half, h, p);
+                }
                 inflight |= 1u << stage;
                 inflight_par = (inflight_par & ~(1u << stage)) | (par << stage);
             }
         }
     };
-    auto issue_v = [&](int k, int stage, uint32_t par) {  // the V tile of the block issue_k(k) fetched
-        if (k >= nk) return;
-        if (lane == 0 && !*sm.abort_flag) {
-            if (iss_p < 0) {
-                mbar_arrive(&sm.full_v[stage]);
-            } else {
-                uint8_t *dst = sm.base + ly.stages + static_cast<uint32_t>(stage) * 2u * kTile + kTile;
-                mbar_arrive_expect_tx(&sm.full_v[stage], kTile);
-#pragma unroll
-                for (int half = 0; half < kCopies; ++half)
-                    tma_load_4d(dst + half * kHalf, tm_v, &sm.full_v[stage], 0, half, iss_h, iss_p);
-                inflight |= 1u << (16 + stage);
-                inflight_par = (inflight_par & ~(1u << (16 + stage))) | (par << (16 + stage));
-            }
-        }
-    };
-    for (int k = 0; k < R; ++k) {
-        issue_k(k, warp + kConsumerWarps * k, 0u);
-        issue_v(k, warp + kConsumerWarps * k, 0u);
-    }
+    for (int k = 0; k < R; ++k) issue(k, warp + kConsumerWarps * k, 0u);
 
     // ---- query rows: warp 0 copies piece n + 1's rows while piece n is computed
     uint32_t q_issued = 0, q_issued_par = 0;
@@ -1181,34 +1196,20 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
                 fence_proxy_async_shared();  // before a later copy overwrites the tile
             };
             if (mbar_wait_bounded(&sm.full[stage], par, sm.abort_flag, a.status)) inflight &= ~(1u << stage);
-            const bool live = !sm.stage_bad[stage] && !*sm.abort_flag;
-            long long want = -1;  // the slot this block's new row goes to, if it takes one
-            if (live) {
+            if (!sm.stage_bad[stage] && !*sm.abort_flag) {
                 if (tail && slot >= 0) {
-                    want = static_cast<long long>(sm.stage_blk[stage]) + (valid - 1);  // row of position L - 1
-                    if (slot != want) {
-                        want = -1;
-                        if (lane == 0) atomicOr(a.status, PKV_STATUS_BAD_SLOT);  // not the last position: not appended
+                    const long long want = static_cast<long long>(sm.stage_blk[stage]) + (valid - 1);  // row of L - 1
+                    if (slot == want) {
+                        if (lane < 2 * kChunks) put_row(want, valid - 1);
+                        __syncwarp();
+                    } else if (lane == 0) {
+                        atomicOr(a.status, PKV_STATUS_BAD_SLOT);  // not the last position: not appended
                     }
                 }
-                if (want >= 0) {
-                    if (lane < kChunks) put_row(want, valid - 1);
-                    __syncwarp();
-                }
-                math.qk(ktile, valid);
+                math.block(ktile, ktile + kTile, valid);
             }
             __syncwarp();
-            issue_k(k + R, stage, par ^ 1u);  // the K tile just read takes this warp's block k + R
-            if (mbar_wait_bounded(&sm.full_v[stage], par, sm.abort_flag, a.status)) inflight &= ~(1u << (16 + stage));
-            if (live && !*sm.abort_flag) {
-                if (want >= 0) {
-                    if (lane >= kChunks && lane < 2 * kChunks) put_row(want, valid - 1);
-                    __syncwarp();
-                }
-                math.pv(ktile + kTile, valid);
-            }
-            __syncwarp();
-            issue_v(k + R, stage, par ^ 1u);  // and its V tile
+            issue(k + R, stage, par ^ 1u);  // the stage just freed takes this warp's block k + R
         }
         gb_base += nblk;
 
@@ -1294,11 +1295,8 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
     // Leave no copy in flight into shared memory when the CTA exits (only
     // possible after a wait gave up).
     if (lane == 0) {
-        for (int st = 0; st < kMaxStages; ++st) {
+        for (int st = 0; st < kMaxStages; ++st)
             if ((inflight >> st) & 1u) mbar_wait_drain(&sm.full[st], (inflight_par >> st) & 1u, a.status);
-            if ((inflight >> (16 + st)) & 1u)
-                mbar_wait_drain(&sm.full_v[st], (inflight_par >> (16 + st)) & 1u, a.status);
-        }
         // the last copy into each query slot: landed already unless a wait gave up
         if (warp == 0)
             for (int slot = 0; slot < 2; ++slot)
@@ -1333,18 +1331,20 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
 // read once for all of them. Sharing a physical block is the same as owning
 // a copy of it ("Deep Dive into vLLM", section 2.2; runbyai post 449, section
 // 3), so a block read here serves every member. Flash-attention style on
-// mma.sync: warp w takes rows 16 w .. 16 w + 15 as M, a tile's 16 tokens as N
-// (S = Q K^T), then P as the A operand of O += P V; the four warps consume one
-// CTA-wide ring of K/V tiles that warp 0 refills. Each row leaves an fp32
-// partial and its log2-sum-exp; the last piece of a segment to be stored merges
-// the segment (prefix pieces first, then the suffix pieces).
+// mma.sync: warp w takes rows 16 w .. 16 w + 15 as M (q staged once in shared
+// memory, read by ldmatrix), a tile's 16 tokens as N (S = Q K^T), then P as
+// the A operand of O += P V; the four warps consume one CTA-wide ring of K/V
+// tiles that warp 0 refills. Each row leaves an fp32 partial and its
+// log2-sum-exp; the last piece of a segment to be stored merges the segment
+// (prefix pieces first, then the suffix pieces).
 template <int D>
 __device__ __forceinline__ void prefix_unit(const CUtensorMap *tm_k, const CUtensorMap *tm_v, const DecodeArgs &a,
-                                         const Smem &sm, const DecodeLayout &ly, long long W, int C, int pcost,
-                                         int warp, int lane) {
+                                            const Smem &sm, const DecodeLayout &ly, long long W, int C, int pcost,
+                                            int warp, int lane) {
     constexpr int BS = 16;
     constexpr int KST = D / 16;             // k-steps of q.K
     constexpr int NT = D / 8;               // 8-dim n-tiles of P.V
+    constexpr int QC = D / 8;               // 16-byte chunks of a q row
     constexpr uint32_t kTile = BS * D * 2;  // bytes of one K (or V) tile
     constexpr uint32_t kHalf = BS * 128;    // one TMA copy: 16 rows of 128 bytes
     constexpr int kCopies = D * 2 / 128;
@@ -1369,27 +1369,51 @@ __device__ __forceinline__ void prefix_unit(const CUtensorMap *tm_k, const CUten
     const int t1 = min(min(T, t0 + a.tiles_per_piece), (lim_max + BS - 1) / BS);
     const int ntiles = max(0, t1 - t0);
 
-    // ---- this lane's two rows: fragment rows lane/4 and lane/4 + 8 of the warp,
-    // i.e. unit rows R = 16 warp + lane/4 + 8 k: member R / G, q head h G + R % G
-    const int tq = lane & 3;
-    int row_lim[2];  // prefix tokens the row attends (0: none, or a padding row)
-    // q rows r and r + 8 (a padding row reads row 0 of the batch: its logits are
-    // selected away). Their A fragments (dims 2 tq, 2 tq + 1 and + 8 of each
-    // k-step) are re-read from L1 at every tile rather than held in 32 registers
-    // beside the 64 of the accumulators.
-    const uint32_t *qr[2];
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-        const int R = 16 * warp + (lane >> 2) + 8 * k;
-        const int sq = m0 + R / G;
-        row_lim[k] = R < rows ? min(sm.lens[sq], T * BS) : 0;
-        qr[k] = reinterpret_cast<const uint32_t *>(static_cast<const __nv_bfloat16 *>(a.q)) +
-                (R < rows ? (static_cast<size_t>(sq) * a.num_q_heads + h * G + R % G) * (D / 2) : 0);
-    }
-
-    // ---- the ring: tile j of the piece goes to stage j % NST (K on full, V on full_v)
+    // ---- the ring: tile j of the piece goes to stage j % NST, K and V on one barrier
     const int *ltab = a.block_tables + static_cast<size_t>(a.grp_begin[g]) * a.max_blocks_per_seq;
     const int sub_shift = a.sub == 2 ? 1 : 0;
+    uint32_t inflight = 0, inflight_par = 0;  // producer (warp 0, lane 0): copies not yet seen landing
+    auto issue_tile = [&](int j) {
+        const int st = j % NST;
+        const uint32_t par = static_cast<uint32_t>(j / NST) & 1u;
+        const int tile = t0 + j;
+        const int pb = __ldg(ltab + (tile >> sub_shift));
+        if (*sm.abort_flag) return;
+        if (pb < 0 || pb >= a.num_blocks) {
+            atomicOr(a.status, PKV_STATUS_BAD_BLOCK_ID);
+            sm.stage_bad[st] = 1;
+            mbar_arrive(&sm.full[st]);
+            return;
+        }
+        sm.stage_bad[st] = 0;
+        const int prow = ((pb << sub_shift) + (tile & (a.sub - 1))) * BS;  // first pool row of the tile
+        uint8_t *dst = sm.base + ly.stages + static_cast<uint32_t>(st) * 2u * kTile;
+        mbar_arrive_expect_tx(&sm.full[st], 2u * kTile);
+#pragma unroll
+        for (int c = 0; c < kCopies; ++c) {
+            tma_load_4d(dst + c * kHalf, tm_k, &sm.full[st], 0, c, h, prow);
+            tma_load_4d(dst + kTile + c * kHalf, tm_v, &sm.full[st], 0, c, h, prow);
+        }
+        inflight |= 1u << st;
+        inflight_par = (inflight_par & ~(1u << st)) | (par << st);
+    };
+    if (warp == 0 && lane == 0)
+        for (int j = 0; j < min(NST, ntiles); ++j) issue_tile(j);
+
+    // ---- q rows of the unit into shared memory, bf16 [kPrefixRows][D]; chunk c
+    // of row R at chunk (c & ~7) | ((c ^ R) & 7), so that ldmatrix's 8 rows of one
+    // chunk hit 8 distinct bank groups (padding rows are zeros)
+    uint8_t *qs = sm.base + ly.prefix_q;
+    const uint32_t qs_addr = smem_u32(qs);
+    for (int e = ctid; e < kPrefixRows * QC; e += kConsumerWarps * 32) {
+        const int R = e / QC, c = e % QC;
+        uint4 val = make_uint4(0u, 0u, 0u, 0u);
+        if (R < rows)
+            val = __ldg(reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(a.q) +
+                                                        (static_cast<size_t>(m0 + R / G) * a.num_q_heads + h * G +
+                                                         R % G) * D) + c);
+        *reinterpret_cast<uint4 *>(qs + R * (D * 2) + (((c & ~7) | ((c ^ R) & 7)) << 4)) = val;
+    }
     // each member's table must hold the group's blocks wherever this piece
     // covers tokens the member attends (a caller's wrong grouping is reported)
     if (ntiles > 0) {
@@ -1402,34 +1426,19 @@ __device__ __forceinline__ void prefix_unit(const CUtensorMap *tm_k, const CUten
                 atomicOr(a.status, PKV_STATUS_BAD_PREFIX_GROUP);
         }
     }
-    uint32_t inflight = 0, inflight_par = 0;  // producer (warp 0, lane 0): copies not yet seen landing
-    auto issue_tile = [&](int j) {
-        const int st = j % NST;
-        const uint32_t par = static_cast<uint32_t>(j / NST) & 1u;
-        const int tile = t0 + j;
-        const int pb = __ldg(ltab + (tile >> sub_shift));
-        if (*sm.abort_flag) return;
-        if (pb < 0 || pb >= a.num_blocks) {
-            atomicOr(a.status, PKV_STATUS_BAD_BLOCK_ID);
-            sm.stage_bad[st] = 1;
-            mbar_arrive(&sm.full[st]);
-            mbar_arrive(&sm.full_v[st]);
-            return;
-        }
-        sm.stage_bad[st] = 0;
-        const int prow = ((pb << sub_shift) + (tile & (a.sub - 1))) * BS;  // first pool row of the tile
-        uint8_t *dst = sm.base + ly.stages + static_cast<uint32_t>(st) * 2u * kTile;
-        mbar_arrive_expect_tx(&sm.full[st], kTile);
+    named_barrier_sync(1, kConsumerWarps * 32);  // q staged
+
+    // ---- this lane's two rows: fragment rows lane/4 and lane/4 + 8 of the warp,
+    // i.e. unit rows R = 16 warp + lane/4 + 8 k: member R / G, q head h G + R % G
+    const int tq = lane & 3;
+    int row_lim[2];  // prefix tokens the row attends (0: none, or a padding row)
 #pragma unroll
-        for (int c = 0; c < kCopies; ++c) tma_load_4d(dst + c * kHalf, tm_k, &sm.full[st], 0, c, h, prow);
-        mbar_arrive_expect_tx(&sm.full_v[st], kTile);
-#pragma unroll
-        for (int c = 0; c < kCopies; ++c) tma_load_4d(dst + kTile + c * kHalf, tm_v, &sm.full_v[st], 0, c, h, prow);
-        inflight |= (1u << st) | (1u << (16 + st));
-        inflight_par = (inflight_par & ~((1u << st) | (1u << (16 + st)))) | (par << st) | (par << (16 + st));
-    };
-    if (warp == 0 && lane == 0)
-        for (int j = 0; j < min(NST, ntiles); ++j) issue_tile(j);
+    for (int k = 0; k < 2; ++k) {
+        const int R = 16 * warp + (lane >> 2) + 8 * k;
+        row_lim[k] = R < rows ? min(sm.lens[m0 + R / G], T * BS) : 0;
+    }
+    // ldmatrix rows of the q A fragments: matrix lane / 8 = (rows +0 / +8, chunk +0 / +1)
+    const int qrow = 16 * warp + (lane & 7) + 8 * ((lane >> 3) & 1), qch = lane >> 4;
 
     float acc[NT][4];
 #pragma unroll
@@ -1456,9 +1465,10 @@ __device__ __forceinline__ void prefix_unit(const CUtensorMap *tm_k, const CUten
         if (live) {
 #pragma unroll
             for (int kk = 0; kk < KST; ++kk) {
-                const uint32_t qa[4] = {__ldg(qr[0] + 8 * kk + tq), __ldg(qr[1] + 8 * kk + tq),
-                                        __ldg(qr[0] + 8 * kk + 4 + tq), __ldg(qr[1] + 8 * kk + 4 + tq)};
-                uint32_t b[4];  // B fragments (k = dims, n = tokens) of tokens 0-7 and 8-15
+                uint32_t qa[4], b[4];
+                const int c = 2 * kk + qch;
+                ldsm_x4(qa, qs_addr + qrow * (D * 2) + (((c & ~7) | ((c ^ qrow) & 7)) << 4));
+                // B fragments (k = dims, n = tokens) of tokens 0-7 and 8-15
                 ldsm_x4(b, tile_addr<BS>(ktile, 8 * (mi >> 1) + r8, 2 * kk + (mi & 1)));
                 mma_16816(sc[0], qa, b[0], b[1]);
                 mma_16816(sc[1], qa, b[2], b[3]);
@@ -1503,9 +1513,7 @@ __device__ __forceinline__ void prefix_unit(const CUtensorMap *tm_k, const CUten
             acc[n][2] *= alpha[1];
             acc[n][3] *= alpha[1];
         }
-        if (mbar_wait_bounded(&sm.full_v[st], par, sm.abort_flag, a.status) && warp == 0 && lane == 0)
-            inflight &= ~(1u << (16 + st));
-        if (live && !*sm.abort_flag) {
+        if (live) {
             // V rows no row of the unit attends may hold anything: zero them in the fragments
             const int vmax = lim_max - tok0;
             uint32_t keep_lo = 0xffffffffu, keep_hi = 0xffffffffu;  // tokens 2 tq, 2 tq + 1 and + 8
@@ -1537,11 +1545,8 @@ __device__ __forceinline__ void prefix_unit(const CUtensorMap *tm_k, const CUten
     }
     // with no copy in flight (possible only after a wait gave up) the stages are free
     if (warp == 0 && lane == 0)
-        for (int st = 0; st < kMaxStages; ++st) {
+        for (int st = 0; st < kMaxStages; ++st)
             if ((inflight >> st) & 1u) mbar_wait_drain(&sm.full[st], (inflight_par >> st) & 1u, a.status);
-            if ((inflight >> (16 + st)) & 1u)
-                mbar_wait_drain(&sm.full_v[st], (inflight_par >> (16 + st)) & 1u, a.status);
-        }
     named_barrier_sync(1, kConsumerWarps * 32);
     if (*sm.abort_flag || ntiles == 0) return;
 
@@ -1588,9 +1593,9 @@ __device__ __forceinline__ void prefix_unit(const CUtensorMap *tm_k, const CUten
     }
     named_barrier_sync(1, kConsumerWarps * 32);
     const int nmerge = mlist[0];
+    if (nmerge > 0) __threadfence();
     for (int i = 0; i < nmerge; ++i) {
         const int s = mlist[1 + i];
-        __threadfence();
         PieceBases pb;
         const int n = piece_bases(a, s, h, sm, W, C, pcost, BS, pb);
         merge_pieces<D>(a, pb, n, s, h, ctid);
@@ -1613,12 +1618,11 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathCudaCore ? 1 : (M
     extern __shared__ uint8_t smem_raw[];
     constexpr int ES = MATH == kMathFp8 ? 1 : 2;  // bytes per pool element
     const DecodeLayout ly = decode_layout(D, BS, GP, a.group, MATH != kMathCudaCore, kConsumerWarps * a.num_stages,
-                                          a.num_seqs, ES, D / a.pack);
+                                          a.num_seqs, ES, D / a.pack, MATH == kMathTensorCoreGroups);
     Smem sm;
     sm.base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     sm.full = reinterpret_cast<uint64_t *>(sm.base + ly.bars);
-    sm.full_v = sm.full + kMaxStages;
-    sm.qfull = sm.full_v + kMaxStages;
+    sm.qfull = sm.full + kMaxStages;
     sm.stage_bad = reinterpret_cast<volatile int *>(sm.base + ly.flags);
     sm.abort_flag = sm.stage_bad + kMaxStages;
     sm.scan = reinterpret_cast<int *>(sm.base + ly.flags) + kMaxStages + 1;
@@ -1634,7 +1638,6 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathCudaCore ? 1 : (M
     if (tid == 0) {
         for (int i = 0; i < kConsumerWarps * a.num_stages; ++i) {
             mbar_init(&sm.full[i], 1);
-            mbar_init(&sm.full_v[i], 1);
             mbar_init(&sm.empty[i], kConsumerWarps);
             sm.stage_bad[i] = 0;
         }
@@ -1811,7 +1814,8 @@ bool decode_variant_exists(int head_dim, int block_size, int group_pad, int math
 size_t decode_smem_bytes(int head_dim, int block_size, int group_pad, int group, int math, int num_stages,
                          int num_seqs, int pack) {
     return decode_layout(head_dim, block_size, effective_group_pad(group_pad, math), group, math != kMathCudaCore,
-                         kConsumerWarps * num_stages, num_seqs, math == kMathFp8 ? 1 : 2, head_dim / pack)
+                         kConsumerWarps * num_stages, num_seqs, math == kMathFp8 ? 1 : 2, head_dim / pack,
+                         math == kMathTensorCoreGroups)
         .total;
 }
 

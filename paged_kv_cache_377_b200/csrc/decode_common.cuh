@@ -81,7 +81,8 @@ struct DecodeArgs {
 };
 
 struct DecodeLayout {
-    uint32_t stages, qbuf, pscr, merge_acc, merge_m, merge_l, bars, flags, prefix, wprefix, lens, ptiles, total;
+    uint32_t stages, qbuf, pscr, merge_acc, merge_m, merge_l, bars, flags, prefix, wprefix, lens, ptiles, prefix_q,
+        total;
 };
 
 __host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
@@ -91,9 +92,12 @@ __host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) { return (x
 // group, G = the actual group (query heads per kv head), tensor_core = the
 // mma.sync math path (its probability scratch is bf16 [8][BS] per warp).
 // kv_elem_bytes = bytes per pool element; dr = dims per stored q / out row
-// (D / pack).
+// (D / pack). groups: the launch has prefix units, whose kPrefixRows query rows
+// (bf16 [rows][D], 16-byte chunks XOR-swizzled by row) take the area of the
+// query slots, probability scratch and merge area (unused by a prefix unit)
+// when it is large enough, else an area of their own at the end.
 __host__ __device__ inline DecodeLayout decode_layout(int D, int BS, int GP, int G, bool tensor_core, int num_stages,
-                                                      int num_seqs, int kv_elem_bytes, int dr) {
+                                                      int num_seqs, int kv_elem_bytes, int dr, bool groups = false) {
     DecodeLayout L;
     uint32_t off = 0;
     const uint32_t tile = static_cast<uint32_t>(BS * D * kv_elem_bytes);
@@ -112,7 +116,7 @@ __host__ __device__ inline DecodeLayout decode_layout(int D, int BS, int GP, int
     off += kConsumerWarps * G * 4;
     off = align_up(off, 8);
     L.bars = off;
-    off += (3 * kMaxStages + 2) * 8;                                // full[stage], full_v[stage], qfull[2], empty[stage]
+    off += (2 * kMaxStages + 2) * 8;                                // full[stage], qfull[2], empty[stage]
     L.flags = off;
     off += (2 * kMaxStages + 1 + 2 * kConsumerWarps + 1 + 4 * 2) * 4;  // stage_bad, abort, scan, merges, stage_blk
     L.prefix = off;
@@ -123,6 +127,12 @@ __host__ __device__ inline DecodeLayout decode_layout(int D, int BS, int GP, int
     off += static_cast<uint32_t>(num_seqs) * 4;                     // clamped context lengths
     L.ptiles = off;
     off += static_cast<uint32_t>(num_seqs) * 4;                     // shared-prefix tiles of each sequence (0: none)
+    L.prefix_q = L.qbuf;
+    if (groups && L.merge_l + kConsumerWarps * G * 4 - L.qbuf < static_cast<uint32_t>(kPrefixRows * D * 2)) {
+        off = align_up(off, 128);
+        L.prefix_q = off;
+        off += kPrefixRows * D * 2;
+    }
     L.total = align_up(off, 16) + 1024;
     return L;
 }
