@@ -145,9 +145,10 @@ WorkspaceLayout workspace_layout(int num_seqs, int num_q_heads, int head_dim) {
 // deeper ring: 4 CTAs of 4 warps per SM with 8 KB blocks); about 64 KB of
 // blocks in flight per CTA for the CUDA-core path, which fits fewer CTAs.
 constexpr int kDefaultL2Prefetch = 0;  // measured on the Llama-shaped batch: any prefetch distance was slower
-// Weight of a piece's fixed cost, in KV blocks. Swept 1..10 on the Llama-,
-// Qwen- and OPT-shaped and skewed batches: 4 is within 1% of the best for each.
-constexpr int kDefaultPieceCost = 4;
+// Weight of a piece's fixed cost, in 16-row tiles. With 16-row tiles and one
+// barrier per stage, 8 beat 4 on every batch (same box: Llama-shaped 364.8 ->
+// 355.0 us, OPT-shaped 43.9 -> 42.5, skewed 139.6 -> 132.2, e4m3 308.7 -> 296.0).
+constexpr int kDefaultPieceCost = 8;
 
 // Prefix tiles one prefix unit streams before it stores its partials: long
 // enough to amortise the unit's start (q fragments, first copies), short enough
