@@ -853,6 +853,7 @@ struct Smem {
     volatile int *stage_bad;
     int *stage_blk;  // [kMaxStages] first pool row of the tile whose copy the stage holds
     volatile int *abort_flag;
+    unsigned *defer;           // [kDeferBits / 32]: piece i of this CTA completes a shared-prefix segment
     volatile int *merge_flag;  // [1 + 2 * 2]: how many segments this CTA completed (<= 2), then
                                // (s, h) of each
     int *scan;
@@ -1269,9 +1270,11 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
                 sm.merge_flag[5] = 0;
                 if (static_cast<int>(now & 0xffffull) == total) {
                     if (GROUPS && sm.ptiles[pc.s] > 0) {
-                        // a shared-prefix segment: all its suffix pieces can be
-                        // cut ones, so this CTA may complete many; merged now
-                        sm.merge_flag[5] = 1;
+                        // a shared-prefix segment: all its suffix pieces can be cut
+                        // ones, so this CTA may complete many; merged after the
+                        // loop (piece npiece - 1 of the CTA), or now past kDeferBits
+                        if (npiece - 1 < kDeferBits) sm.defer[(npiece - 1) >> 5] |= 1u << ((npiece - 1) & 31);
+                        else sm.merge_flag[5] = 1;
                     } else if (pending < 2) {  // never more than two (below)
                         volatile int *m = sm.merge_flag + 1 + 2 * pending;
                         m[0] = pc.s;
@@ -1309,6 +1312,24 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
     // The barrier makes every warp's drain complete and the flags final and
     // the same for all threads.
     named_barrier_sync(1, kConsumerWarps * 32);
+    if constexpr (GROUPS) {
+        if (!*sm.abort_flag) {
+            // the shared-prefix segments this CTA completed, in the order of its pieces
+            const long long Wt = static_cast<long long>(a.num_kv_heads) * sm.wprefix[a.num_seqs];
+            PieceIter walk = pieces;  // from the CTA's first block again
+            walk.x = x0;
+            Piece wp;
+            bool fenced = false;
+            for (int i = 0; i < kDeferBits && walk.next(wp); ++i) {
+                if (!((sm.defer[i >> 5] >> (i & 31)) & 1u)) continue;
+                if (!fenced) __threadfence();
+                fenced = true;
+                PieceBases pb;
+                const int n = piece_bases(a, wp.s, wp.h, sm, Wt, gridDim.x - a.prefix_ctas, pcost, BS, pb);
+                merge_pieces<D>(a, pb, n, wp.s, wp.h, ctid);
+            }
+        }
+    }
     const int pending = *sm.abort_flag ? 0 : sm.merge_flag[0];
     for (int i = 0; i < pending; ++i) {
         const volatile int *m = sm.merge_flag + 1 + 2 * i;
@@ -1628,6 +1649,7 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathCudaCore ? 1 : (M
     sm.scan = reinterpret_cast<int *>(sm.base + ly.flags) + kMaxStages + 1;
     sm.merge_flag = reinterpret_cast<volatile int *>(sm.scan + 2 * kConsumerWarps);
     sm.stage_blk = const_cast<int *>(sm.merge_flag) + 1 + 4 * 2;
+    sm.defer = reinterpret_cast<unsigned *>(sm.stage_blk + kMaxStages);
     sm.prefix = reinterpret_cast<int *>(sm.base + ly.prefix);
     sm.wprefix = reinterpret_cast<int *>(sm.base + ly.wprefix);
     sm.lens = reinterpret_cast<int *>(sm.base + ly.lens);
@@ -1644,6 +1666,7 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathCudaCore ? 1 : (M
         for (int i = 0; i < 2; ++i) mbar_init(&sm.qfull[i], 1);
         *sm.abort_flag = 0;
         sm.merge_flag[0] = 0;
+        for (int i = 0; i < kDeferBits / 32; ++i) sm.defer[i] = 0u;
         fence_mbar_init();
     }
     if (tid == 32) {
