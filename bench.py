@@ -62,7 +62,7 @@ def parse_args(argv=None):
     p.add_argument("--steps", type=int, default=200)
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--workload", default="llama3_8b", choices=list(workloads.CONFIG_ORDER) + list(PREFILL_WORKLOADS))
+    p.add_argument("--workload", default="llama3_8b", choices=list(workloads.CONFIGS) + list(PREFILL_WORKLOADS))
     p.add_argument("--kv-dtype", default="bf16", choices=["bf16", "fp8"],
                    help="decode workloads: bf16 pools, or e4m3 codes with per-head scales")
     p.add_argument("--num-ctas", type=int, default=0)
@@ -74,8 +74,8 @@ def parse_args(argv=None):
     p.add_argument("--head-pack", type=int, default=0)
     p.add_argument("--tile-tokens", type=int, default=0)
     p.add_argument("--prefix-tiles", type=int, default=0)
-    p.add_argument("--prefix-groups", choices=["auto", "off"], default="auto",
-                   help="auto: pass the runs of sequences that share leading blocks (found on the host tables, "
+    p.add_argument("--prefix-groups", choices=["on", "off"], default="off",
+                   help="on: pass the runs of sequences that share leading blocks (found on the host tables, "
                         "as an engine's block manager knows them) so that shared blocks are read once per group")
     p.add_argument("--two-launch", action="store_true",
                    help="run the step as kv_cache_append + paged_attn_decode instead of the one-launch call")
@@ -279,7 +279,7 @@ class Step:
                          piece_cost=args.piece_cost, head_pack=args.head_pack, tile_tokens=args.tile_tokens,
                          prefix_tiles=args.prefix_tiles)
         self.groups = None
-        if getattr(args, "prefix_groups", "off") == "auto" and b.kv_dtype == "bf16":
+        if getattr(args, "prefix_groups", "off") == "on" and b.kv_dtype == "bf16":
             g = pkv.find_prefix_groups(b.block_tables, b.context_lens, b.block_size)
             if len(g):
                 self.groups = g

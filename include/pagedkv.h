@@ -102,9 +102,12 @@ extern "C" {
  *                     The result does not depend on it beyond rounding order.
  *   prefix_groups     see pkv_prefix_groups above (NULL: none).
  *   prefix_tiles      16-row tiles of a shared prefix that one CTA streams before
- *                     storing its partials (1..4096); default 16. Fewer spread a
- *                     group's shared blocks over more CTAs; more partials to
- *                     merge. Raised as needed to leave most CTAs to the rest.
+ *                     storing its partials (1..4096); default: the CTAs are
+ *                     split between the shared prefixes and the rest in
+ *                     proportion to their work (the rest bounded by
+ *                     max_blocks_per_seq, the lengths being on the device).
+ *                     Raised as needed to fit the workspace and leave a CTA
+ *                     to the rest.
  */
 /*
  * Prefix groups: runs of consecutive sequences of a batch whose block tables

@@ -150,23 +150,29 @@ constexpr int kDefaultL2Prefetch = 0;  // measured on the Llama-shaped batch: an
 // 355.0 us, OPT-shaped 43.9 -> 42.5, skewed 139.6 -> 132.2, e4m3 308.7 -> 296.0).
 constexpr int kDefaultPieceCost = 8;
 
-// Prefix tiles one prefix unit streams before it stores its partials: long
-// enough to amortise the unit's start (q fragments, first copies), short enough
-// that a group's shared blocks are spread over many CTAs.
-constexpr int kPrefixTilesPerPiece = 16;
+// Work of one shared-prefix tile (64 query rows) against one suffix tile (the G
+// rows of one sequence), for splitting the CTAs between the two: the prefix
+// tile does about 64 / G times the math but reads the same bytes, mostly from L2.
+constexpr int kPrefixTileCost = 3;
 
 // The prefix units of one launch (sequences s0 .. s0 + sc - 1): the groups of
 // the caller's descriptor that have at least two members in the launch, as
 // kernel parameters. Leaves a.num_groups = 0 when grouping does not apply.
+// The CTAs are split between prefix units and suffixes in proportion to their
+// work: the prefix tiles, and at most max_blocks_per_seq * sub tiles per
+// sequence (less each group's shared ones) for the suffixes -- the host knows
+// the table width, not the context lengths. tiles_per_piece > 0 sets the
+// tiles of one unit instead.
 void plan_prefix_groups(const pkv_prefix_groups *pg, int s0, int sc, int hkv, int group, int sub, int ctas,
-                        int tiles_per_piece, pkv::DecodeArgs &a) {
+                        int max_blocks_per_seq, int tiles_per_piece, pkv::DecodeArgs &a) {
     a.num_groups = 0;
     a.prefix_ctas = 0;
     a.tiles_per_piece = 1;
     a.prefix_np = 0;
     a.pre_base = 0;
-    if (!pg || pg->num_groups <= 0) return;
+    if (!pg || pg->num_groups <= 0 || ctas < 2) return;
     int n = 0, max_tiles = 0;
+    long long prefix_work = 0, suffix_bound = static_cast<long long>(sc) * max_blocks_per_seq * sub;
     for (int g = 0; g < pg->num_groups && n < pkv::kMaxPrefixGroups; ++g) {
         const int lo = pg->begin[g] > s0 ? pg->begin[g] : s0;
         const int hi = pg->end[g] < s0 + sc ? pg->end[g] : s0 + sc;
@@ -179,6 +185,8 @@ void plan_prefix_groups(const pkv_prefix_groups *pg, int s0, int sc, int hkv, in
         const int row_tiles = (hi - lo + per - 1) / per;
         a.grp_row_tiles[n] = row_tiles;
         a.grp_members[n] = (hi - lo + row_tiles - 1) / row_tiles;  // spread evenly over the row tiles
+        prefix_work += static_cast<long long>(row_tiles) * a.grp_tiles[n];
+        suffix_bound -= static_cast<long long>(hi - lo) * a.grp_tiles[n];
         ++n;
     }
     if (n == 0) return;
@@ -187,15 +195,26 @@ void plan_prefix_groups(const pkv_prefix_groups *pg, int s0, int sc, int hkv, in
     const long long room = 1024LL * hkv - ctas;
     const long long np_max = room / (static_cast<long long>(sc) * hkv);
     if (np_max < 1) return;
-    int tpp = tiles_per_piece > 0 ? tiles_per_piece : kPrefixTilesPerPiece;
+    int tpp = tiles_per_piece;
+    if (tpp <= 0) {
+        // units in proportion to the prefix's share of the work (at least one CTA each way)
+        const double share = static_cast<double>(kPrefixTileCost * prefix_work) /
+                             static_cast<double>(kPrefixTileCost * prefix_work + (suffix_bound > 0 ? suffix_bound : 0));
+        long long target = static_cast<long long>(share * ctas);
+        if (target < 1) target = 1;
+        if (target > ctas - 1) target = ctas - 1;
+        const long long unit_tiles = static_cast<long long>(hkv) * prefix_work;  // (head, row tile, tile) triples
+        tpp = static_cast<int>((unit_tiles + target - 1) / target);
+        if (tpp < 1) tpp = 1;
+    }
     if ((max_tiles + tpp - 1) / tpp > np_max) tpp = static_cast<int>((max_tiles + np_max - 1) / np_max);
     long long units = 0;
     for (;;) {
         units = 0;
         for (int g = 0; g < n; ++g)
             units += static_cast<long long>(hkv) * a.grp_row_tiles[g] * ((a.grp_tiles[g] + tpp - 1) / tpp);
-        if (units <= ctas / 2 || tpp >= max_tiles) break;
-        tpp *= 2;  // fewer, longer pieces until the units leave most CTAs to the suffixes
+        if (units <= ctas - 1 || tpp >= max_tiles) break;
+        ++tpp;  // rounding up the pieces made too many units
     }
     if (units > ctas - 1) return;  // no CTA would be left for the suffixes
     a.num_groups = n;
@@ -406,7 +425,8 @@ int decode_impl(void *out, const void *q, const void *k_new, const void *v_new, 
         a.prefetch = o.l2_prefetch > 0 ? o.l2_prefetch : o.l2_prefetch == 0 ? kDefaultL2Prefetch : 0;
         a.piece_cost = o.piece_cost > 0 ? o.piece_cost : o.piece_cost == 0 ? kDefaultPieceCost : 0;
         a.scale_log2 = scale * 1.4426950408889634f;
-        plan_prefix_groups(may_group ? pg : nullptr, s0, sc, khkv, kgroup, a.sub, grid, o.prefix_tiles, a);
+        plan_prefix_groups(may_group ? pg : nullptr, s0, sc, khkv, kgroup, a.sub, grid, max_blocks_per_seq,
+                           o.prefix_tiles, a);
         // a launch whose groups were planned runs the kernel with the prefix
         // units; one whose groups were dropped runs the plain kernel in the
         // same shared memory and grid

@@ -156,3 +156,20 @@ def test_groups_are_refused_where_they_cannot_apply():
         fused(b, groups, math=1)
     with pytest.raises(pkv.PagedKVError, match="two or more members"):
         fused(b, pkv.PrefixGroups([0], [1], [3]))
+
+
+@pytest.mark.parametrize("grouped", [True, False])
+def test_long_shared_prefix_sampled_rows(grouped):
+    """32 sequences sharing a 32768-token prompt (its K/V larger than L2), checked
+    on sampled rows against the oracle, with and without the grouping."""
+    b = workloads.make_batch("shared_long_prefix", device=DEV).to("cpu")
+    groups = pkv.find_prefix_groups(b.block_tables, b.context_lens, b.block_size) if grouped else None
+    if grouped:
+        assert len(groups) == 1 and groups.blocks[0] == 2048
+    pairs = list(range(0, b.num_seqs * b.num_q_heads, 13))
+    ref, kc_ref, vc_ref = oracle.decode_step(b, pairs=pairs)
+    out, kc, vc, st = fused(b, groups)
+    assert st == 0, st
+    assert np.array_equal(kc, kc_ref) and np.array_equal(vc, vc_ref)
+    got = out.double().numpy().reshape(-1, b.head_dim)[pairs]
+    assert_close_to_oracle(got, ref, what=f"shared long prefix, grouped={grouped}")

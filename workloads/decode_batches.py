@@ -119,6 +119,16 @@ CONFIGS: Dict[str, Config] = {
 }
 CONFIG_ORDER = ["tiny", "opt125m", "llama3_8b", "qwen25_7b_prefix", "skewed_long"]
 
+# An extra bench workload (not one of the five parity configs above): a long
+# shared prompt whose K/V does not fit in L2, the case prefix groups are for.
+CONFIGS["shared_long_prefix"] = Config(
+    "shared_long_prefix", 5, 32, 32, 8, 128, 16, 1.0 / math.sqrt(128),
+    _prefix_plus_suffix(32, 32768, 1, 512), 32768 + 512,
+    pool="shared_prefix", prefix_tokens=32768,
+    description="Llama-3-8B GQA heads: 32 seqs sharing a 32768-token prompt (2048 blocks, 134 MB of K/V) "
+                "+ private suffix U[1,512], D128, bs16",
+)
+
 
 @dataclasses.dataclass
 class DecodeBatch:
