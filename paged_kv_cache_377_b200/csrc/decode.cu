@@ -1435,18 +1435,6 @@ __device__ __forceinline__ void prefix_unit(const CUtensorMap *tm_k, const CUten
                                                          R % G) * D) + c);
         *reinterpret_cast<uint4 *>(qs + R * (D * 2) + (((c & ~7) | ((c ^ R) & 7)) << 4)) = val;
     }
-    // each member's table must hold the group's blocks wherever this piece
-    // covers tokens the member attends (a caller's wrong grouping is reported)
-    if (ntiles > 0) {
-        const int b0 = t0 >> sub_shift, nb = ((t1 - 1) >> sub_shift) - b0 + 1;
-        for (int e = ctid; e < (m1 - m0) * nb; e += kConsumerWarps * 32) {
-            const int m = m0 + e / nb, b = b0 + e % nb;
-            const int att = (min(sm.lens[m], T * BS) + BS - 1) / BS;  // tiles the member attends
-            if ((b << sub_shift) < att &&
-                __ldg(a.block_tables + static_cast<size_t>(m) * a.max_blocks_per_seq + b) != __ldg(ltab + b))
-                atomicOr(a.status, PKV_STATUS_BAD_PREFIX_GROUP);
-        }
-    }
     named_barrier_sync(1, kConsumerWarps * 32);  // q staged
 
     // ---- this lane's two rows: fragment rows lane/4 and lane/4 + 8 of the warp,
@@ -1478,11 +1466,11 @@ __device__ __forceinline__ void prefix_unit(const CUtensorMap *tm_k, const CUten
         if (mbar_wait_bounded(&sm.full[st], par, sm.abort_flag, a.status) && warp == 0 && lane == 0)
             inflight &= ~(1u << st);
         const bool live = !sm.stage_bad[st] && !*sm.abort_flag;
-        float sc[2][4];  // S for tokens 0-7 and 8-15: (row r: 2 tq, 2 tq + 1), (row r + 8: same)
+        float sc[2][4], sc2[2][4];  // S for tokens 0-7 and 8-15: (row r: 2 tq, 2 tq + 1), (row r + 8: same)
 #pragma unroll
         for (int n = 0; n < 2; ++n)
 #pragma unroll
-            for (int k = 0; k < 4; ++k) sc[n][k] = 0.f;
+            for (int k = 0; k < 4; ++k) sc[n][k] = sc2[n][k] = 0.f;
         if (live) {
 #pragma unroll
             for (int kk = 0; kk < KST; ++kk) {
@@ -1491,9 +1479,14 @@ __device__ __forceinline__ void prefix_unit(const CUtensorMap *tm_k, const CUten
                 ldsm_x4(qa, qs_addr + qrow * (D * 2) + (((c & ~7) | ((c ^ qrow) & 7)) << 4));
                 // B fragments (k = dims, n = tokens) of tokens 0-7 and 8-15
                 ldsm_x4(b, tile_addr<BS>(ktile, 8 * (mi >> 1) + r8, 2 * kk + (mi & 1)));
-                mma_16816(sc[0], qa, b[0], b[1]);
-                mma_16816(sc[1], qa, b[2], b[3]);
+                // even and odd k-steps accumulate apart: four independent chains
+                mma_16816((kk & 1) ? sc2[0] : sc[0], qa, b[0], b[1]);
+                mma_16816((kk & 1) ? sc2[1] : sc[1], qa, b[2], b[3]);
             }
+#pragma unroll
+            for (int n = 0; n < 2; ++n)
+#pragma unroll
+                for (int k = 0; k < 4; ++k) sc[n][k] += sc2[n][k];
         }
         // base-2 logits; tokens a row does not attend are selected away
         float mx[2] = {-INFINITY, -INFINITY};
@@ -1527,12 +1520,14 @@ __device__ __forceinline__ void prefix_unit(const CUtensorMap *tm_k, const CUten
                 l_run[rr] = l_run[rr] * (n == 0 ? alpha[rr] : 1.f) + pf.x + pf.y;
                 pa[2 * n + rr] = *reinterpret_cast<const uint32_t *>(&p2);
             }
+        if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {  // some row's maximum grew
 #pragma unroll
-        for (int n = 0; n < NT; ++n) {
-            acc[n][0] *= alpha[0];
-            acc[n][1] *= alpha[0];
-            acc[n][2] *= alpha[1];
-            acc[n][3] *= alpha[1];
+            for (int n = 0; n < NT; ++n) {
+                acc[n][0] *= alpha[0];
+                acc[n][1] *= alpha[0];
+                acc[n][2] *= alpha[1];
+                acc[n][3] *= alpha[1];
+            }
         }
         if (live) {
             // V rows no row of the unit attends may hold anything: zero them in the fragments
@@ -1570,6 +1565,22 @@ __device__ __forceinline__ void prefix_unit(const CUtensorMap *tm_k, const CUten
             if ((inflight >> st) & 1u) mbar_wait_drain(&sm.full[st], (inflight_par >> st) & 1u, a.status);
     named_barrier_sync(1, kConsumerWarps * 32);
     if (*sm.abort_flag || ntiles == 0) return;
+
+    // ---- each member's table must hold the group's blocks wherever this piece
+    // covers tokens the member attends (a caller's wrong grouping is reported);
+    // checked after the tiles, with independent loads and one flag per thread
+    {
+        const int b0 = t0 >> sub_shift, nb = ((t1 - 1) >> sub_shift) - b0 + 1;
+        bool bad = false;
+#pragma unroll 4
+        for (int e = ctid; e < (m1 - m0) * nb; e += kConsumerWarps * 32) {
+            const int m = m0 + e / nb, b = b0 + e % nb;
+            const int att = (min(sm.lens[m], T * BS) + BS - 1) / BS;  // tiles the member attends
+            const int mine = __ldg(a.block_tables + static_cast<size_t>(m) * a.max_blocks_per_seq + b);
+            bad |= (b << sub_shift) < att && mine != __ldg(ltab + b);
+        }
+        if (bad) atomicOr(a.status, PKV_STATUS_BAD_PREFIX_GROUP);
+    }
 
     // ---- this piece's partial of every row that attends some of its tokens
 #pragma unroll
