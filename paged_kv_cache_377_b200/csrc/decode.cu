@@ -556,11 +556,20 @@ __device__ __forceinline__ void mma_16816_f16(float (&d)[4], const uint32_t (&a)
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// Two e4m3 codes (low byte first) -> two f16 in one register, exactly
-// (every e4m3 value is an f16 value).
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
-    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two_codes & 0xffffu), __NV_E4M3);
-    return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+// Two e4m3 codes of w -- the bytes SEL places in bytes 0 and 2 (SEL's other
+// nibbles are 4: zero bytes) -- as an f16x2 of each code's value times 2^-8,
+// exactly: the code's magnitude bits (exponent, then mantissa) move to bits
+// 7..13 of the f16 and its sign to bit 15; an f16 with exponent field e and
+// mantissa m is then 2^(e-15) (1 + m/8), the code's 2^(e-7) (1 + m/8) times
+// 2^-8, and the subnormal codes land on the f16 subnormals the same way. The
+// sign moves one place up by adding the sign bit to itself. Exact for every
+// finite code; the two NaN codes become +-480 x 2^-8 (the kernel only meets
+// them in rows it masks). Integer adds and a shift, instead of a conversion
+// instruction that occupies the ALU pipe four times as long.
+template <uint32_t SEL>
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2_lo8(uint32_t w) {
+    const uint32_t t = __byte_perm(w, 0u, SEL);
+    return (t + (t & 0x00800080u)) << 7;
 }
 
 __device__ __forceinline__ uint32_t f16x2_bits(float lo, float hi) {
@@ -658,8 +667,9 @@ struct Fp8Math {
         const float ip0 = __shfl_sync(0xffffffffu, inv_ps, 4 * n0), ip1 = __shfl_sync(0xffffffffu, inv_ps, 4 * n1);
         const int hg = pack == 2 ? (group >> 1) : group;  // query rows per real head
         const int h0 = pack * h + (n0 < group ? n0 / hg : 0), h1 = pack * h + (n1 < group ? n1 / hg : 0);
-        mult0 = n0 < group ? sl2 * __ldg(a.k_scale + h0) * ip0 : 0.f;
-        mult1 = n1 < group ? sl2 * __ldg(a.k_scale + h1) * ip1 : 0.f;
+        // x 2^8: the K codes enter the products as f16 of value code x 2^-8
+        mult0 = n0 < group ? sl2 * __ldg(a.k_scale + h0) * ip0 * 256.f : 0.f;
+        mult1 = n1 < group ? sl2 * __ldg(a.k_scale + h1) * ip1 * 256.f : 0.f;
         vsc0 = a.v_scale + h0;
         vsc1 = a.v_scale + h1;
     }
@@ -692,11 +702,12 @@ struct Fp8Math {
                 const uint32_t b10 = on ? qb[qc + 1][0] : 0u, b11 = on ? qb[qc + 1][1] : 0u;
                 uint32_t x[4];
                 ldsm_x4(x, tile_addr<BS>(ktile, 16 * mt + r + 8 * (mi & 1), 2 * kp + (mi >> 1)));
-                const uint32_t a0[4] = {e4m3x2_to_f16x2(x[0]), e4m3x2_to_f16x2(x[1]), e4m3x2_to_f16x2(x[0] >> 16),
-                                        e4m3x2_to_f16x2(x[1] >> 16)};
+                // codes as f16 x 2^-8 (the logit multiplier holds the 2^8)
+                const uint32_t a0[4] = {e4m3x2_to_f16x2_lo8<0x4140>(x[0]), e4m3x2_to_f16x2_lo8<0x4140>(x[1]),
+                                        e4m3x2_to_f16x2_lo8<0x4342>(x[0]), e4m3x2_to_f16x2_lo8<0x4342>(x[1])};
                 mma_16816_f16(s[mt], a0, b00, b01);
-                const uint32_t a1[4] = {e4m3x2_to_f16x2(x[2]), e4m3x2_to_f16x2(x[3]), e4m3x2_to_f16x2(x[2] >> 16),
-                                        e4m3x2_to_f16x2(x[3] >> 16)};
+                const uint32_t a1[4] = {e4m3x2_to_f16x2_lo8<0x4140>(x[2]), e4m3x2_to_f16x2_lo8<0x4140>(x[3]),
+                                        e4m3x2_to_f16x2_lo8<0x4342>(x[2]), e4m3x2_to_f16x2_lo8<0x4342>(x[3])};
                 mma_16816_f16(s2[mt], a1, b10, b11);
             }
 #pragma unroll
@@ -787,10 +798,11 @@ struct Fp8Math {
 #pragma unroll
                     for (int j = 0; j < 2; ++j) {
                         // x[2j]: tokens 0-7 of tile 2dp + j, x[2j + 1]: tokens 8-15; bytes
-                        // (t, 2r) (t, 2r+1) (t+1, 2r) (t+1, 2r+1) -> (t, 2r) (t+1, 2r) | (t, 2r+1) (t+1, 2r+1)
-                        const uint32_t lo = __byte_perm(x[2 * j], 0u, 0x3120), hi = __byte_perm(x[2 * j + 1], 0u, 0x3120);
-                        uint32_t av[4] = {e4m3x2_to_f16x2(lo), e4m3x2_to_f16x2(lo >> 16), e4m3x2_to_f16x2(hi),
-                                          e4m3x2_to_f16x2(hi >> 16)};
+                        // (t, 2r) (t, 2r+1) (t+1, 2r) (t+1, 2r+1) -> (t, 2r) (t+1, 2r) | (t, 2r+1) (t+1, 2r+1),
+                        // as f16 x 2^-8 (the V scale holds the 2^8)
+                        uint32_t av[4] = {e4m3x2_to_f16x2_lo8<0x4240>(x[2 * j]), e4m3x2_to_f16x2_lo8<0x4341>(x[2 * j]),
+                                          e4m3x2_to_f16x2_lo8<0x4240>(x[2 * j + 1]),
+                                          e4m3x2_to_f16x2_lo8<0x4341>(x[2 * j + 1])};
                         if (valid < BS) {
                             av[0] &= klo;
                             av[1] &= klo;
@@ -829,7 +841,8 @@ struct Fp8Math {
         const int h0 = HP == 1 && pack == 2 ? g0 / (G >> 1) : 0, h1 = HP == 1 && pack == 2 ? (g0 + 1) / (G >> 1) : 0;
         float *r0 = merge_acc + (warp * G + g0) * DR - h0 * DR;
         float *r1 = merge_acc + (warp * G + g0 + 1) * DR - h1 * DR;
-        const float vs0 = g0 < G ? __ldg(vsc0) : 0.f, vs1 = g0 + 1 < G ? __ldg(vsc1) : 0.f;
+        // x 2^8: the V codes enter the products as f16 of value code x 2^-8
+        const float vs0 = g0 < G ? __ldg(vsc0) * 256.f : 0.f, vs1 = g0 + 1 < G ? __ldg(vsc1) * 256.f : 0.f;
 #pragma unroll
         for (int dt = 0; dt < DT; ++dt) {
             const int half = HP == 1 ? (16 * dt) / DR : 0;
