@@ -148,7 +148,14 @@ constexpr int kDefaultL2Prefetch = 0;  // measured on the Llama-shaped batch: an
 // Weight of a piece's fixed cost, in 16-row tiles. With 16-row tiles and one
 // barrier per stage, 8 beat 4 on every batch (same box: Llama-shaped 364.8 ->
 // 355.0 us, OPT-shaped 43.9 -> 42.5, skewed 139.6 -> 132.2, e4m3 308.7 -> 296.0).
+// A piece's merge grows with the query heads per kv head: with more than 4,
+// 16 (Qwen-shaped, 7 per kv head: 42.6 -> 40.8 us; 8 -> 16 on the Llama-shaped
+// batch, 4 per kv head: 354.9 -> 357.5). e4m3 pools: 12 (after the bit-placement
+// conversion: Llama-shaped 265.5 -> 260.6 us, OPT-shaped 40.6 -> 38.3, skewed
+// 119.0 -> 119.8).
 constexpr int kDefaultPieceCost = 8;
+constexpr int kDefaultPieceCostWideGroup = 16;
+constexpr int kDefaultPieceCostFp8 = 12;
 
 // Work of one shared-prefix tile (64 query rows) against one suffix tile (the G
 // rows of one sequence), for splitting the CTAs between the two: the prefix
@@ -423,7 +430,8 @@ int decode_impl(void *out, const void *q, const void *k_new, const void *v_new, 
         a.num_blocks = num_blocks;
         a.num_stages = ns;
         a.prefetch = o.l2_prefetch > 0 ? o.l2_prefetch : o.l2_prefetch == 0 ? kDefaultL2Prefetch : 0;
-        a.piece_cost = o.piece_cost > 0 ? o.piece_cost : o.piece_cost == 0 ? kDefaultPieceCost : 0;
+        const int pcost_default = fp8 ? kDefaultPieceCostFp8 : group > 4 ? kDefaultPieceCostWideGroup : kDefaultPieceCost;
+        a.piece_cost = o.piece_cost > 0 ? o.piece_cost : o.piece_cost == 0 ? pcost_default : 0;
         a.scale_log2 = scale * 1.4426950408889634f;
         plan_prefix_groups(may_group ? pg : nullptr, s0, sc, khkv, kgroup, a.sub, grid, max_blocks_per_seq,
                            o.prefix_tiles, a);
