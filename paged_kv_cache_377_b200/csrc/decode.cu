@@ -608,6 +608,7 @@ struct Fp8Math {
 
     int lane;
     int my_half;          // HP = 2: the head (0/1) of this lane's B-fragment column lane / 4
+    bool c1_head0, c1_head1;  // HP = 2: the heads of this lane's two accumulator columns are 1
     uint32_t pscr;        // this warp's f16 P[GP][BS] (shared address)
     uint32_t qb[8][2];    // f16 B fragments of q (row-scaled, chunk-permuted), 8 chunks of 16 dims
     float mult0, mult1;   // base-2 logit multiplier of this lane's two columns
@@ -668,6 +669,8 @@ struct Fp8Math {
         const int hg = pack == 2 ? (group >> 1) : group;  // query rows per real head
         const int h0 = pack * h + (n0 < group ? n0 / hg : 0), h1 = pack * h + (n1 < group ? n1 / hg : 0);
         // x 2^8: the K codes enter the products as f16 of value code x 2^-8
+        c1_head0 = HP == 2 && n0 < group && n0 / hg == 1;
+        c1_head1 = HP == 2 && n1 < group && n1 / hg == 1;
         mult0 = n0 < group ? sl2 * __ldg(a.k_scale + h0) * ip0 * 256.f : 0.f;
         mult1 = n1 < group ? sl2 * __ldg(a.k_scale + h1) * ip1 * 256.f : 0.f;
         vsc0 = a.v_scale + h0;
@@ -693,25 +696,51 @@ struct Fp8Math {
         for (int mt = 0; mt < TT; ++mt) {
 #pragma unroll
             for (int k = 0; k < 4; ++k) s[mt][k] = s2[mt][k] = 0.f;
+            if constexpr (HP == 1) {
+                // chunks 2kp, 2kp + 1 into two independent chains
 #pragma unroll
-            for (int kp = 0; kp < 4 * HP; ++kp) {
-                // chunks 2kp, 2kp + 1 of the row; with HP = 2 they belong to head kp / 4
-                const bool on = HP == 1 || my_half == kp / 4;
-                const int qc = (2 * kp) % 8;
-                const uint32_t b00 = on ? qb[qc][0] : 0u, b01 = on ? qb[qc][1] : 0u;
-                const uint32_t b10 = on ? qb[qc + 1][0] : 0u, b11 = on ? qb[qc + 1][1] : 0u;
-                uint32_t x[4];
-                ldsm_x4(x, tile_addr<BS>(ktile, 16 * mt + r + 8 * (mi & 1), 2 * kp + (mi >> 1)));
-                // codes as f16 x 2^-8 (the logit multiplier holds the 2^8)
-                const uint32_t a0[4] = {e4m3x2_to_f16x2_lo8<0x4140>(x[0]), e4m3x2_to_f16x2_lo8<0x4140>(x[1]),
-                                        e4m3x2_to_f16x2_lo8<0x4342>(x[0]), e4m3x2_to_f16x2_lo8<0x4342>(x[1])};
-                mma_16816_f16(s[mt], a0, b00, b01);
-                const uint32_t a1[4] = {e4m3x2_to_f16x2_lo8<0x4140>(x[2]), e4m3x2_to_f16x2_lo8<0x4140>(x[3]),
-                                        e4m3x2_to_f16x2_lo8<0x4342>(x[2]), e4m3x2_to_f16x2_lo8<0x4342>(x[3])};
-                mma_16816_f16(s2[mt], a1, b10, b11);
+                for (int kp = 0; kp < 4; ++kp) {
+                    uint32_t x[4];
+                    ldsm_x4(x, tile_addr<BS>(ktile, 16 * mt + r + 8 * (mi & 1), 2 * kp + (mi >> 1)));
+                    // codes as f16 x 2^-8 (the logit multiplier holds the 2^8)
+                    const uint32_t a0[4] = {e4m3x2_to_f16x2_lo8<0x4140>(x[0]), e4m3x2_to_f16x2_lo8<0x4140>(x[1]),
+                                            e4m3x2_to_f16x2_lo8<0x4342>(x[0]), e4m3x2_to_f16x2_lo8<0x4342>(x[1])};
+                    mma_16816_f16(s[mt], a0, qb[2 * kp][0], qb[2 * kp][1]);
+                    const uint32_t a1[4] = {e4m3x2_to_f16x2_lo8<0x4140>(x[2]), e4m3x2_to_f16x2_lo8<0x4140>(x[3]),
+                                            e4m3x2_to_f16x2_lo8<0x4342>(x[2]), e4m3x2_to_f16x2_lo8<0x4342>(x[3])};
+                    mma_16816_f16(s2[mt], a1, qb[2 * kp + 1][0], qb[2 * kp + 1][1]);
+                }
+#pragma unroll
+                for (int k = 0; k < 4; ++k) s[mt][k] += s2[mt][k];
+            } else {
+                // Two heads per row: head 0's 128 dims accumulate in s, head 1's in
+                // s2, every column against both (each lane's q fragment holds its
+                // own head's q), and each column keeps its own head's chain -- no
+                // per-lane masking of the q fragments. The heads alternate: two
+                // independent chains.
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int kp = (j >> 1) + 4 * (j & 1);  // 0, 4, 1, 5, ...: head j & 1
+                    const int qc = (2 * kp) % 8;
+                    uint32_t x[4];
+                    ldsm_x4(x, tile_addr<BS>(ktile, 16 * mt + r + 8 * (mi & 1), 2 * kp + (mi >> 1)));
+                    // codes as f16 x 2^-8 (the logit multiplier holds the 2^8)
+                    const uint32_t a0[4] = {e4m3x2_to_f16x2_lo8<0x4140>(x[0]), e4m3x2_to_f16x2_lo8<0x4140>(x[1]),
+                                            e4m3x2_to_f16x2_lo8<0x4342>(x[0]), e4m3x2_to_f16x2_lo8<0x4342>(x[1])};
+                    const uint32_t a1[4] = {e4m3x2_to_f16x2_lo8<0x4140>(x[2]), e4m3x2_to_f16x2_lo8<0x4140>(x[3]),
+                                            e4m3x2_to_f16x2_lo8<0x4342>(x[2]), e4m3x2_to_f16x2_lo8<0x4342>(x[3])};
+                    auto step = [&](float (&acc_h)[4]) {
+                        mma_16816_f16(acc_h, a0, qb[qc][0], qb[qc][1]);
+                        mma_16816_f16(acc_h, a1, qb[qc + 1][0], qb[qc + 1][1]);
+                    };
+                    if (j & 1) step(s2[mt]);
+                    else step(s[mt]);
+                }
+                s[mt][0] = c1_head0 ? s2[mt][0] : s[mt][0];
+                s[mt][1] = c1_head1 ? s2[mt][1] : s[mt][1];
+                s[mt][2] = c1_head0 ? s2[mt][2] : s[mt][2];
+                s[mt][3] = c1_head1 ? s2[mt][3] : s[mt][3];
             }
-#pragma unroll
-            for (int k = 0; k < 4; ++k) s[mt][k] += s2[mt][k];
         }
         // base-2 logits; tokens past the context are selected away (their rows may hold NaN codes)
         float mx0 = -INFINITY, mx1 = -INFINITY;
