@@ -4,14 +4,16 @@
 // Same operation as prefill.cu (chunked prefill / mixed batches: query i of a
 // sequence's n-token chunk attends causally to positions 0 .. L - n + i).
 // One CTA per (128 rows of (query token, group head), sequence, kv head), two
-// CTAs per SM (256 tensor-memory columns each), six warps; launched with the
+// CTAs per SM (256 tensor-memory columns each), seven warps; launched with the
 // row tiles that see the most context first:
-//   - warp 4 issues every TMA copy: the CTA's 128 query rows once (a 5D box
-//     over q viewed as [T][Hkv][G][D]) and the context in iterations of 64
-//     tokens (64 / BS paged blocks) through separate 2-stage rings of K and V
-//     (128-byte swizzled tiles; one lane per block slice). It polls for the
-//     MMA that frees each stage, so K and V refills never queue behind each
-//     other;
+//   - warps 4 and 6 issue the TMA copies: warp 4 the CTA's 128 query rows once
+//     (a 5D box over q viewed as [T][Hkv][G][D]) and the K tiles, warp 6 the V
+//     tiles, of the context in iterations of 64 tokens (64 / BS paged blocks)
+//     through separate 2-stage rings (128-byte swizzled tiles; one lane per
+//     block slice). Each blocks on the MMA that frees its next stage and is
+//     woken when it completes, so K and V refills never queue behind each
+//     other and start as soon as a stage is free (one warp polling both
+//     rings issued them ~1.5 us late: a %globaltimer trace);
 //   - warp 5 (an elected lane) issues the MMAs: S = Q K^T (M 128, N 64, K =
 //     head_dim in steps of 16) into one of two tensor-memory buffers, and
 //     O += P V (M 128, N = head_dim, K 64; P read from tensor memory, V as an
@@ -35,7 +37,7 @@ namespace pkv {
 namespace {
 
 constexpr int kSoftmaxThreads = 128;  // warps 0-3: one query row (tensor-memory lane) each
-constexpr int kTcThreads = 192;       // + warp 4: TMA copies, warp 5: MMAs
+constexpr int kTcThreads = 224;       // + warp 4: Q and K copies, warp 5: MMAs, warp 6: V copies
 constexpr int kTcBarriers = 12;
 constexpr int kTcRows = 128;          // query rows per CTA (= tensor-memory lanes)
 constexpr int kTcTokens = 64;   // context tokens per iteration
@@ -287,12 +289,13 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     // tensor memory: S / P buffers at columns 0 and 64, O at 128 .. 128 + D
     const uint32_t t_o = tbase + 128;
 
-    if (warp == 4) {
-        // ---------------- load warp: every TMA copy; lane j copies one
+    if (warp == 4 || warp == 6) {
+        // ---------------- load warps (4: Q and K, 6: V); lane j copies one
         // 128-byte column slice of one paged block
-        int k_use0 = -1, k_use1 = -1, v_use0 = -1, v_use1 = -1;  // last use of each stage issued
+        const bool is_v = warp == 6;
+        int use0 = -1, use1 = -1;  // last use of each stage issued
         const int jb = lane / HALVES, hf = lane % HALVES;
-        auto issue = [&](int it, bool is_v) {
+        auto issue = [&](int it) {
             const int st = it & 1;
             uint64_t *bar = is_v ? &v_full[st] : &k_full[st];
             const int b = it * BPI + jb;
@@ -311,65 +314,30 @@ __global__ void __launch_bounds__(kTcThreads, 2)
             if (mine)
                 tma_load_4d((is_v ? sv : sk) + st * kTileKV + hf * kHalfKV + jb * BS * 128, is_v ? &tm_v : &tm_k, bar,
                             0, hf, h, p * BS);
-            int &use = is_v ? (st ? v_use1 : v_use0) : (st ? k_use1 : k_use0);
-            use = it >> 1;
+            (st ? use1 : use0) = it >> 1;
         };
-        if (lane == 0) {
+        if (!is_v && lane == 0) {
             mbar_arrive_expect_tx(q_full, HALVES * kQHalf);
 #pragma unroll
             for (int q = 0; q < HALVES; ++q) tma_load_5d(sq + q * kQHalf, &tm_q, q_full, 0, q, 0, h, q0 + i0);
         }
-        issue(0, false);
-        if (nit > 1) issue(1, false);
-        issue(0, true);
-        if (nit > 1) issue(1, true);
+        issue(0);
+        if (nit > 1) issue(1);
         // K(it) once S(it - 2) is done (its stage is free), V(it) once
-        // P(it - 2) V(it - 2) is done, each as soon as it may: both are polled,
-        // so that neither waits behind the other; bounded like every wait
+        // P(it - 2) V(it - 2) is done; bounded like every wait. Neither barrier
+        // can run two phases ahead: S(it) needs K(it), P(it) V(it) needs V(it).
         bool ok = true;
-        int nk = 2, nv = 2;
-        uint64_t t_prog = 0;  // start of the current stretch without progress
-        for (uint32_t spin = 1; nk < nit || nv < nit; ++spin) {
-            bool moved = false;
-            if (nk < nit &&
-                __all_sync(0xffffffffu, mbar_test(&s_full[nk & 1], static_cast<uint32_t>((nk - 2) >> 1) & 1u))) {
-                issue(nk++, false);
-                moved = true;
-            }
-            if (nv < nit &&
-                __all_sync(0xffffffffu, mbar_test(&pv_free[nv & 1], static_cast<uint32_t>((nv - 2) >> 1) & 1u))) {
-                issue(nv++, true);
-                moved = true;
-            }
-            if (moved) {
-                t_prog = 0;
-                continue;
-            }
-            if (__any_sync(0xffffffffu, *abort_flag != 0)) {
-                ok = false;
-                break;
-            }
-            __nanosleep(32);  // leave the issue slots to the softmax warps
-            if ((spin & 15u) == 0) {
-                const uint64_t now = globaltimer_ns();
-                if (t_prog == 0) t_prog = now;
-                if (now - t_prog > kWaitLimitNs) {
-                    if (lane == 0) {
-                        *abort_flag = 1;
-                        atomicOr(a.status, PKV_STATUS_WAIT_TIMEOUT);
-                    }
-                    ok = false;
-                    break;
-                }
-            }
+        for (int nx = 2; nx < nit; ++nx) {
+            uint64_t *freed = is_v ? &pv_free[nx & 1] : &s_full[nx & 1];
+            if (!(ok = warp_wait(freed, static_cast<uint32_t>((nx - 2) >> 1) & 1u, abort_flag, a.status))) break;
+            issue(nx);
         }
         // copies still in flight (only after a wait gave up) land before exit
         if (!ok || *abort_flag) {
-            mbar_wait_drain(q_full, 0, a.status);
-            if (k_use0 >= 0) mbar_wait_drain(&k_full[0], static_cast<uint32_t>(k_use0) & 1u, a.status);
-            if (k_use1 >= 0) mbar_wait_drain(&k_full[1], static_cast<uint32_t>(k_use1) & 1u, a.status);
-            if (v_use0 >= 0) mbar_wait_drain(&v_full[0], static_cast<uint32_t>(v_use0) & 1u, a.status);
-            if (v_use1 >= 0) mbar_wait_drain(&v_full[1], static_cast<uint32_t>(v_use1) & 1u, a.status);
+            if (!is_v) mbar_wait_drain(q_full, 0, a.status);
+            uint64_t *full = is_v ? v_full : k_full;
+            if (use0 >= 0) mbar_wait_drain(&full[0], static_cast<uint32_t>(use0) & 1u, a.status);
+            if (use1 >= 0) mbar_wait_drain(&full[1], static_cast<uint32_t>(use1) & 1u, a.status);
         }
         __syncwarp();
     } else if (warp == 5) {
