@@ -1726,6 +1726,18 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathCudaCore ? 1 : (M
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
     }
+    // The table entries of the first copies are read once the prologue has
+    // split the work; meanwhile warp 2 brings this CTA's share of the launch's
+    // block tables into L2 (a hint: line by line, inside the array), so those
+    // reads hit L2 rather than HBM.
+    if (warp == 2) {
+        const size_t bytes = static_cast<size_t>(a.num_seqs) * a.max_blocks_per_seq * sizeof(int32_t);
+        const size_t per = (bytes + gridDim.x - 1) / gridDim.x;
+        const size_t end = min(bytes, (blockIdx.x + 1) * per);
+        const char *tables = reinterpret_cast<const char *>(a.block_tables);
+        for (size_t off = blockIdx.x * per + lane * 128; off < end; off += 32 * 128)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(tables + off));
+    }
 
     // prefix[s] = blocks of sequences < s (clamped lengths), wprefix[s] = their
     // weight (blocks + piece_cost per non-empty sequence); lens[s] = clamped
