@@ -407,9 +407,13 @@ int decode_impl(void *out, const void *q, const void *k_new, const void *v_new, 
         cudaError_t e = pkv::decode_prepare(kd, tile, gp, gmath, smem, &per_sm);
         if (e != cudaSuccess) return cuda_fail(e, "decode kernel setup");
         if (per_sm <= 0) return fail(PKV_ERR_INVALID_ARGUMENT, "shared memory %zu bytes per CTA does not fit", smem);
+        const int resident = sms * per_sm;  // CTAs that fit on the device at once
         if (o.ctas_per_sm > 0 && o.ctas_per_sm < per_sm) per_sm = o.ctas_per_sm;
         int grid = o.num_ctas > 0 ? o.num_ctas : sms * per_sm;
         if (grid > pkv::kMaxCtas) grid = pkv::kMaxCtas;
+        // the kernel with prefix units is launched cooperatively (its CTAs wait
+        // for one another's pieces): no more CTAs than fit at once
+        if (may_group && grid > resident) grid = resident;
         pkv::DecodeArgs a{};
         a.out = static_cast<__nv_bfloat16 *>(out) + static_cast<size_t>(s0) * num_q_heads * head_dim;
         a.q = static_cast<const __nv_bfloat16 *>(q) + static_cast<size_t>(s0) * num_q_heads * head_dim;

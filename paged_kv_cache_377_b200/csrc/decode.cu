@@ -1309,29 +1309,16 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
                     old = prev;
                 }
                 const int pending = sm.merge_flag[0];
-                sm.merge_flag[5] = 0;
                 if (static_cast<int>(now & 0xffffull) == total) {
+                    // a shared-prefix segment is merged by its designated CTA
+                    // (merge_grouped_segments), whoever completes it
                     if (GROUPS && sm.ptiles[pc.s] > 0) {
-                        // a shared-prefix segment: all its suffix pieces can be cut
-                        // ones, so this CTA may complete many; merged after the
-                        // loop (piece npiece - 1 of the CTA), or now past kDeferBits
-                        if (npiece - 1 < kDeferBits) sm.defer[(npiece - 1) >> 5] |= 1u << ((npiece - 1) & 31);
-                        else sm.merge_flag[5] = 1;
                     } else if (pending < 2) {  // never more than two (below)
                         volatile int *m = sm.merge_flag + 1 + 2 * pending;
                         m[0] = pc.s;
                         m[1] = pc.h;
                         sm.merge_flag[0] = pending + 1;
                     }
-                }
-            }
-            named_barrier_sync(1, kConsumerWarps * 32);
-            if constexpr (GROUPS) {
-                if (sm.merge_flag[5] && !*sm.abort_flag) {
-                    __threadfence();
-                    PieceBases pb;
-                    const int n = piece_bases(a, pc.s, pc.h, sm, W, gridDim.x - a.prefix_ctas, pcost, BS, pb);
-                    merge_pieces<D, 1>(a, pb, n, pc.s, pc.h, ctid);  // one piece at a time: the loop's state is live
                 }
             }
         }
@@ -1354,24 +1341,6 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
     // The barrier makes every warp's drain complete and the flags final and
     // the same for all threads.
     named_barrier_sync(1, kConsumerWarps * 32);
-    if constexpr (GROUPS) {
-        if (!*sm.abort_flag) {
-            // the shared-prefix segments this CTA completed, in the order of its pieces
-            const long long Wt = static_cast<long long>(a.num_kv_heads) * sm.wprefix[a.num_seqs];
-            PieceIter walk = pieces;  // from the CTA's first block again
-            walk.x = x0;
-            Piece wp;
-            bool fenced = false;
-            for (int i = 0; i < kDeferBits && walk.next(wp); ++i) {
-                if (!((sm.defer[i >> 5] >> (i & 31)) & 1u)) continue;
-                if (!fenced) __threadfence();
-                fenced = true;
-                PieceBases pb;
-                const int n = piece_bases(a, wp.s, wp.h, sm, Wt, gridDim.x - a.prefix_ctas, pcost, BS, pb);
-                merge_pieces<D>(a, pb, n, wp.s, wp.h, ctid);
-            }
-        }
-    }
     const int pending = *sm.abort_flag ? 0 : sm.merge_flag[0];
     for (int i = 0; i < pending; ++i) {
         const volatile int *m = sm.merge_flag + 1 + 2 * i;
@@ -1644,16 +1613,13 @@ __device__ __forceinline__ void prefix_unit(const CUtensorMap *tm_k, const CUten
         if (tq == 0) a.lse_part[pr] = m_run[rr] + __log2f(l_run[rr]);
     }
 
-    // ---- count the piece in on each member's segment; merge the segments it completes
+    // ---- count the piece in on each member's segment (its designated CTA
+    // merges the segment once every piece is in: merge_grouped_segments)
     __threadfence();
-    named_barrier_sync(1, kConsumerWarps * 32);
-    int *mlist = reinterpret_cast<int *>(sm.base + ly.stages);  // [0] count, [1 ..] members to merge
-    if (ctid == 0) mlist[0] = 0;
     named_barrier_sync(1, kConsumerWarps * 32);
     if (ctid < m1 - m0) {
         const int s = m0 + ctid;
         if (min(sm.lens[s], T * BS) > t0 * BS) {
-            const int total = segment_pieces(s, h, sm, Hkv, W, C, pcost, BS, a.tiles_per_piece, nullptr);
             unsigned long long *cnt = a.seg_count + static_cast<size_t>(s) * Hkv + h;
             unsigned long long old = atomicAdd(cnt, 0ull), now;
             for (;;) {  // count = 1 for the first piece of this launch (stale epochs restart)
@@ -1662,16 +1628,54 @@ __device__ __forceinline__ void prefix_unit(const CUtensorMap *tm_k, const CUten
                 if (prev == old) break;
                 old = prev;
             }
-            if (static_cast<int>(now & 0xffffull) == total) mlist[1 + atomicAdd(mlist, 1)] = s;
         }
     }
-    named_barrier_sync(1, kConsumerWarps * 32);
-    const int nmerge = mlist[0];
-    if (nmerge > 0) __threadfence();
-    for (int i = 0; i < nmerge; ++i) {
-        const int s = mlist[1 + i];
+}
+
+// The merges of the shared-prefix segments, spread over the grid: segment k
+// of the launch's grouped segments (members in order, kv heads inner) is
+// merged by CTA k mod gridDim.x once all its pieces are in. The last piece
+// to arrive would otherwise merge them, and a prefix unit is the last for
+// up to all the members of its row tile (a per-warp trace: one unit spent
+// 119 us merging 16 segments while most CTAs were done). Every CTA runs this
+// after its own work; the launch is cooperative, so all CTAs are resident
+// and a CTA waiting for a segment never holds a slot the segment's pieces
+// need. The wait is bounded: past it the status word and the abort flag are
+// set and the segment is left unmerged.
+template <int D>
+__device__ __forceinline__ void merge_grouped_segments(const DecodeArgs &a, const Smem &sm, int C, int pcost, int BS,
+                                                       int ctid) {
+    const int Hkv = a.num_kv_heads;
+    int ng = 0;
+    for (int g = 0; g < a.num_groups; ++g) ng += (a.grp_end[g] - a.grp_begin[g]) * Hkv;
+    const long long W = static_cast<long long>(Hkv) * sm.wprefix[a.num_seqs];
+    for (int k = blockIdx.x; k < ng; k += gridDim.x) {
+        int g = 0, r = k;  // member r / Hkv of group g, kv head r % Hkv
+        while (r >= (a.grp_end[g] - a.grp_begin[g]) * Hkv) {
+            r -= (a.grp_end[g] - a.grp_begin[g]) * Hkv;
+            ++g;
+        }
+        const int s = a.grp_begin[g] + r / Hkv, h = r % Hkv;
         PieceBases pb;
         const int n = piece_bases(a, s, h, sm, W, C, pcost, BS, pb);
+        if (n == 0) continue;  // no context: a zero row, written by the prologue
+        // wait (bounded) until every piece is counted in; one thread polls
+        if (ctid == 0) {
+            const volatile unsigned long long *cnt = a.seg_count + static_cast<size_t>(s) * Hkv + h;
+            const unsigned long long want = (a.epoch << 16) | static_cast<unsigned long long>(n);
+            const uint64_t t_start = globaltimer_ns();
+            while (*cnt != want) {
+                if (*sm.abort_flag || globaltimer_ns() - t_start > kWaitLimitNs) {
+                    *sm.abort_flag = 1;
+                    atomicOr(a.status, PKV_STATUS_WAIT_TIMEOUT);
+                    break;
+                }
+                __nanosleep(200);
+            }
+        }
+        named_barrier_sync(1, kConsumerWarps * 32);
+        if (*sm.abort_flag) return;
+        __threadfence();
         merge_pieces<D>(a, pb, n, s, h, ctid);
     }
 }
@@ -1845,6 +1849,8 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathCudaCore ? 1 : (M
     if constexpr (GROUPS) {
         if (cta < 0) {
             prefix_unit<D>(&tm_k, &tm_v, a, sm, ly, W, C, pcost, warp, lane);
+            named_barrier_sync(1, kConsumerWarps * 32);
+            merge_grouped_segments<D>(a, sm, C, pcost, BS, tid);
             return;
         }
     }
@@ -1866,6 +1872,10 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathCudaCore ? 1 : (M
     } else if constexpr (MATH == kMathTensorCore || GROUPS) {
         decode_warp<D, BS, MmaMath<D, BS>, 2, GROUPS>(&tm_k, &tm_v, a, sm, ly, pieces, x0, x1, W, pcost, warp,
                                               lane);
+        if constexpr (GROUPS) {
+            named_barrier_sync(1, kConsumerWarps * 32);
+            merge_grouped_segments<D>(a, sm, C, pcost, BS, tid);
+        }
     } else {
         static_assert(D == 128 || D == 256, "the e4m3 path reads rows of 128 or 256 codes");
         decode_warp<D, BS, Fp8Math<BS, D / 128>, 1, false>(&tm_k, &tm_v, a, sm, ly, pieces, x0, x1, W, pcost,
@@ -1932,6 +1942,15 @@ cudaError_t decode_launch(int head_dim, int block_size, int group_pad, int math,
                           cudaStream_t stream) {
     KernelFn fn = pick(head_dim, block_size, effective_group_pad(group_pad, math), math);
     if (!fn) return cudaErrorInvalidValue;
+    if (math == kMathTensorCoreGroups) {
+        // CTAs of this kernel wait for one another's pieces (shared-prefix
+        // merges): a cooperative launch keeps them all resident at once
+        CUtensorMap k = tm_k, v = tm_v;
+        DecodeArgs d = args;
+        void *params[] = {&k, &v, &d};
+        return cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(fn), dim3(grid), dim3(kDecodeThreads), params,
+                                           smem_bytes, stream);
+    }
     fn<<<grid, kDecodeThreads, smem_bytes, stream>>>(tm_k, tm_v, args);
     return cudaGetLastError();
 }
