@@ -895,7 +895,6 @@ struct Smem {
     volatile int *stage_bad;
     int *stage_blk;  // [kMaxStages] first pool row of the tile whose copy the stage holds
     volatile int *abort_flag;
-    unsigned *defer;           // [kDeferBits / 32]: piece i of this CTA completes a shared-prefix segment
     volatile int *merge_flag;  // [1 + 2 * 2]: how many segments this CTA completed (<= 2), then
                                // (s, h) of each
     int *scan;
@@ -1309,11 +1308,11 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
                     old = prev;
                 }
                 const int pending = sm.merge_flag[0];
-                if (static_cast<int>(now & 0xffffull) == total) {
-                    // a shared-prefix segment is merged by its designated CTA
-                    // (merge_grouped_segments), whoever completes it
-                    if (GROUPS && sm.ptiles[pc.s] > 0) {
-                    } else if (pending < 2) {  // never more than two (below)
+                // (a shared-prefix segment is merged by its designated CTA,
+                // merge_grouped_segments, whoever completes it)
+                const bool designated = GROUPS && sm.ptiles[pc.s] > 0;
+                if (static_cast<int>(now & 0xffffull) == total && !designated) {
+                    if (pending < 2) {  // never more than two (below)
                         volatile int *m = sm.merge_flag + 1 + 2 * pending;
                         m[0] = pc.s;
                         m[1] = pc.h;
@@ -1706,7 +1705,6 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathCudaCore ? 1 : (M
     sm.scan = reinterpret_cast<int *>(sm.base + ly.flags) + kMaxStages + 1;
     sm.merge_flag = reinterpret_cast<volatile int *>(sm.scan + 2 * kConsumerWarps);
     sm.stage_blk = const_cast<int *>(sm.merge_flag) + 1 + 4 * 2;
-    sm.defer = reinterpret_cast<unsigned *>(sm.stage_blk + kMaxStages);
     sm.prefix = reinterpret_cast<int *>(sm.base + ly.prefix);
     sm.wprefix = reinterpret_cast<int *>(sm.base + ly.wprefix);
     sm.lens = reinterpret_cast<int *>(sm.base + ly.lens);
@@ -1723,7 +1721,6 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathCudaCore ? 1 : (M
         for (int i = 0; i < 2; ++i) mbar_init(&sm.qfull[i], 1);
         *sm.abort_flag = 0;
         sm.merge_flag[0] = 0;
-        for (int i = 0; i < kDeferBits / 32; ++i) sm.defer[i] = 0u;
         fence_mbar_init();
     }
     if (tid == 32) {

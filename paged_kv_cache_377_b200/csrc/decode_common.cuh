@@ -15,7 +15,6 @@ constexpr int kMaxCtas = 1024;                        // grid limit; bounds the 
 constexpr int kWorkspaceHeaderBytes = 256;
 constexpr int kMaxPrefixGroups = 16;                  // prefix groups per launch (kernel parameters)
 constexpr int kPrefixRows = 64;                       // query rows of one prefix unit: 16 per warp
-constexpr int kDeferBits = 256;                       // pieces of a CTA whose shared-prefix merges wait for its end
 
 // With pack = 2 the kernel runs on a view of the pool with half the kv heads
 // and twice the head_dim: kv heads 2h', 2h' + 1 of head_dim D / 2 are the two
@@ -120,7 +119,6 @@ __host__ __device__ inline DecodeLayout decode_layout(int D, int BS, int GP, int
     off += (2 * kMaxStages + 2) * 8;                                // full[stage], qfull[2], empty[stage]
     L.flags = off;
     off += (2 * kMaxStages + 1 + 2 * kConsumerWarps + 1 + 4 * 2) * 4;  // stage_bad, abort, scan, merges, stage_blk
-    off += kDeferBits / 8;                                          // deferred merges (bits)
     L.prefix = off;
     off += static_cast<uint32_t>(num_seqs + 1) * 4;                 // blocks before each sequence
     L.wprefix = off;
