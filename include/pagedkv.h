@@ -131,6 +131,9 @@ extern "C" {
  * groups per 2048 sequences; groups beyond that, groups a 2048-sequence launch
  * boundary leaves with one member, and batches whose workspace has no room
  * for the group partials are decoded without the grouping (same results).
+ * A launch with groups is cooperative (cudaLaunchCooperativeKernel: its CTAs
+ * wait, bounded, for one another's pieces of the shared-prefix segments they
+ * merge), so num_ctas is reduced to the CTAs that fit on the device at once.
  */
 #define PKV_MAX_PREFIX_GROUPS 16
 typedef struct pkv_prefix_groups {
