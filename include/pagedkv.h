@@ -172,9 +172,13 @@ int pkv_find_prefix_groups(const int32_t *block_tables, const int32_t *context_l
 /*
  * Bytes of device workspace paged_attn_decode needs for this shape
  * (host-only; returns PKV_OK and sets *bytes).
- * Layout: [0, 256) header whose first int32 is the device status word; one
- * counter per (sequence, kv head) of a launch, tagged with the launch's epoch
- * so the workspace never needs clearing; fp32 partial outputs and
+ * Layout: [0, 256) header whose first int32 is the device status word, and
+ * whose bytes [8, 20) count the decode launches made with the workspace (each
+ * launch advances the count at its end, so every launch -- each replay of a
+ * captured CUDA graph too -- has an epoch of its own); one counter per
+ * (sequence, kv head) of a launch, tagged with that epoch, so the workspace
+ * never needs clearing (zero it whole or not at all: zeroing the launch count
+ * alone would let old counters be read as new); fp32 partial outputs and
  * log2-sum-exp values of the context pieces that CTA boundaries cut. At most
  * 2048 sequences go in one launch; longer batches reuse the workspace launch
  * after launch.

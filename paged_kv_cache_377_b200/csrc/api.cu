@@ -9,7 +9,6 @@
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 
-#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -103,13 +102,6 @@ int make_query_map(CUtensorMap *map, const void *q, int num_tokens, int hkv, int
     return PKV_OK;
 }
 
-// Launch epochs tag the per-segment piece counters, so a workspace never needs
-// clearing between calls (a counter from an older launch restarts at 1).
-unsigned long long next_epoch() {
-    static std::atomic<unsigned long long> epoch{0};
-    return (epoch.fetch_add(1, std::memory_order_relaxed) + 1) & ((1ull << 48) - 1);
-}
-
 int sm_count() {
     int dev = 0, n = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 0;
@@ -122,7 +114,8 @@ int sm_count() {
     return cache[dev];
 }
 
-// Workspace layout: [0, 256) header (status word) | per-segment piece
+// Workspace layout: [0, 256) header (status word at 0; the launch epoch at 8
+// and the CTAs started at 16, advanced by the kernels) | per-segment piece
 // counters [S_chunk * Hkv <= S_chunk * Hq] uint64 | fp32 partial outputs [rows][D] | fp32 log2-sum-exp [rows],
 // rows = (S_chunk + kMaxCtas) * Hq bounds the pieces' rows of one launch
 // (pieces <= S_chunk * Hkv + C, each with G <= Hq rows).
@@ -422,7 +415,8 @@ int decode_impl(void *out, const void *q, const void *k_new, const void *v_new, 
         a.o_part = reinterpret_cast<float *>(ws + wl.o_part);
         a.lse_part = reinterpret_cast<float *>(ws + wl.lse_part);
         a.seg_count = reinterpret_cast<unsigned long long *>(ws + wl.seg_count);
-        a.epoch = next_epoch();
+        a.launch_epoch = reinterpret_cast<unsigned long long *>(ws + pkv::kLaunchCounterOffset);
+        a.ctas_started = reinterpret_cast<unsigned int *>(ws + pkv::kLaunchCounterOffset + 8);
         a.status = reinterpret_cast<int32_t *>(ws);
         a.num_seqs = sc;
         a.num_q_heads = num_q_heads;
@@ -767,9 +761,10 @@ extern "C" int paged_attn_decode_noalloc(void *out, const void *q, const void *k
     if ((rc = noalloc_scratch(&scratch)) != PKV_OK) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     // The scratch keeps the previous call's contents: zero its status word so
-    // this call reports only its own problems. The partials need no clearing
-    // (every one that is read was written earlier in the same call).
-    cudaError_t e = cudaMemsetAsync(scratch, 0, pkv::kWorkspaceHeaderBytes, st);
+    // this call reports only its own problems. The launch counter after it
+    // and the partials need no clearing (every partial that is read was
+    // written earlier in the same call).
+    cudaError_t e = cudaMemsetAsync(scratch, 0, sizeof(int32_t), st);
     if (e != cudaSuccess) return cuda_fail(e, "clearing the static scratch's status word");
     rc = paged_attn_decode_ex(out, q, k_cache, v_cache, block_tables, context_lens, num_seqs, num_q_heads,
                               num_kv_heads, head_dim, block_size, scale, max_blocks_per_seq, num_blocks, scratch,

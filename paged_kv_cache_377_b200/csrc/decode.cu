@@ -903,6 +903,7 @@ struct Smem {
     int *lens;
     int *ptiles;     // [S] shared-prefix tiles of each sequence (0: not in a prefix group)
     uint64_t *empty;  // prefix units: all four warps are done with a stage
+    volatile unsigned long long *epoch;  // this launch's epoch (read from the workspace header)
 };
 
 // The CTAs holding pieces of segment (s, h). CTA c covers weight positions
@@ -1300,9 +1301,10 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
                 const int total = segment_pieces(pc.s, pc.h, sm, a.num_kv_heads, W, gridDim.x - a.prefix_ctas, pcost,
                                                  BS, a.tiles_per_piece, nullptr);
                 unsigned long long *cnt = a.seg_count + seg;
+                const unsigned long long ep = *sm.epoch;
                 unsigned long long old = atomicAdd(cnt, 0ull), now;
                 for (;;) {  // count = 1 for the first piece of this launch (stale epochs restart)
-                    now = (old >> 16) == a.epoch ? old + 1 : (a.epoch << 16) | 1ull;
+                    now = (old >> 16) == ep ? old + 1 : (ep << 16) | 1ull;
                     const unsigned long long prev = atomicCAS(cnt, old, now);
                     if (prev == old) break;
                     old = prev;
@@ -1620,9 +1622,10 @@ __device__ __forceinline__ void prefix_unit(const CUtensorMap *tm_k, const CUten
         const int s = m0 + ctid;
         if (min(sm.lens[s], T * BS) > t0 * BS) {
             unsigned long long *cnt = a.seg_count + static_cast<size_t>(s) * Hkv + h;
+            const unsigned long long ep = *sm.epoch;
             unsigned long long old = atomicAdd(cnt, 0ull), now;
             for (;;) {  // count = 1 for the first piece of this launch (stale epochs restart)
-                now = (old >> 16) == a.epoch ? old + 1 : (a.epoch << 16) | 1ull;
+                now = (old >> 16) == ep ? old + 1 : (ep << 16) | 1ull;
                 const unsigned long long prev = atomicCAS(cnt, old, now);
                 if (prev == old) break;
                 old = prev;
@@ -1661,7 +1664,7 @@ __device__ __forceinline__ void merge_grouped_segments(const DecodeArgs &a, cons
         // wait (bounded) until every piece is counted in; one thread polls
         if (ctid == 0) {
             const volatile unsigned long long *cnt = a.seg_count + static_cast<size_t>(s) * Hkv + h;
-            const unsigned long long want = (a.epoch << 16) | static_cast<unsigned long long>(n);
+            const unsigned long long want = (*sm.epoch << 16) | static_cast<unsigned long long>(n);
             const uint64_t t_start = globaltimer_ns();
             while (*cnt != want) {
                 if (*sm.abort_flag || globaltimer_ns() - t_start > kWaitLimitNs) {
@@ -1677,6 +1680,26 @@ __device__ __forceinline__ void merge_grouped_segments(const DecodeArgs &a, cons
         __threadfence();
         merge_pieces<D>(a, pb, n, s, h, ctid);
     }
+}
+
+// The end of this CTA's part of the launch. CTA 0 advances the workspace's
+// epoch for the next launch once every CTA of this one has started (each
+// counted itself after reading the epoch; by CTA 0's end they all have, so
+// the bounded wait is a formality) and resets the count. The next launch
+// starts after this one has ended, so it needs no fence.
+__device__ __forceinline__ void finish_launch(const DecodeArgs &a, const Smem &sm, int tid) {
+    if (blockIdx.x != 0 || tid != 0) return;
+    const volatile unsigned int *started = a.ctas_started;
+    const uint64_t t0 = globaltimer_ns();
+    while (*started < gridDim.x) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {  // left for the next launch's counters to restart
+            atomicOr(a.status, PKV_STATUS_WAIT_TIMEOUT);
+            return;
+        }
+        __nanosleep(100);
+    }
+    *reinterpret_cast<volatile unsigned int *>(a.ctas_started) = 0u;
+    *reinterpret_cast<volatile unsigned long long *>(a.launch_epoch) = (*sm.epoch + 1) & ((1ull << 48) - 1);
 }
 
 // The tensor-core path fits 128 registers per thread, so 4 CTAs (16 warps)
@@ -1710,6 +1733,7 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathCudaCore ? 1 : (M
     sm.lens = reinterpret_cast<int *>(sm.base + ly.lens);
     sm.ptiles = reinterpret_cast<int *>(sm.base + ly.ptiles);
     sm.empty = sm.qfull + 2;
+    sm.epoch = reinterpret_cast<volatile unsigned long long *>(sm.empty + kMaxStages);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     if (tid == 0) {
@@ -1723,6 +1747,10 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathCudaCore ? 1 : (M
         sm.merge_flag[0] = 0;
         fence_mbar_init();
     }
+    // The workspace's launch count (the previous launch advanced it): loaded
+    // now, stored for the CTA's threads after the prologue's own loads.
+    unsigned long long launch_epoch = 0;
+    if (tid == 0) launch_epoch = *reinterpret_cast<volatile unsigned long long *>(a.launch_epoch);
     if (tid == 32) {
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
@@ -1803,6 +1831,11 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathCudaCore ? 1 : (M
         }
         sm.prefix[S] = total;
         sm.wprefix[S] = total_w;
+        *sm.epoch = launch_epoch & ((1ull << 48) - 1);
+        // this CTA has read the epoch: counted as started (the added value
+        // depends on the loaded one -- always 0 + 1 -- so the count cannot be
+        // seen before the read is done; nobody waits for it here)
+        atomicAdd(a.ctas_started, 1u + static_cast<unsigned>(launch_epoch >> 63));
     }
     __syncthreads();
     // Sequences with no context get all-zero rows (no piece covers them); CTA c
@@ -1848,6 +1881,7 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathCudaCore ? 1 : (M
             prefix_unit<D>(&tm_k, &tm_v, a, sm, ly, W, C, pcost, warp, lane);
             named_barrier_sync(1, kConsumerWarps * 32);
             merge_grouped_segments<D>(a, sm, C, pcost, BS, tid);
+            finish_launch(a, sm, tid);
             return;
         }
     }
@@ -1878,6 +1912,7 @@ __global__ void __launch_bounds__(kDecodeThreads, MATH == kMathCudaCore ? 1 : (M
         decode_warp<D, BS, Fp8Math<BS, D / 128>, 1, false>(&tm_k, &tm_v, a, sm, ly, pieces, x0, x1, W, pcost,
                                                     warp, lane);
     }
+    finish_launch(a, sm, tid);
 }
 
 using KernelFn = void (*)(const CUtensorMap, const CUtensorMap, const DecodeArgs);

@@ -13,6 +13,7 @@ constexpr int kMaxStagesPerWarp = kMaxStages / kConsumerWarps;
 constexpr int kMaxSeqsPerLaunch = 2048;               // per-sequence tables kept in shared memory
 constexpr int kMaxCtas = 1024;                        // grid limit; bounds the pieces of a launch
 constexpr int kWorkspaceHeaderBytes = 256;
+constexpr int kLaunchCounterOffset = 8;               // header bytes [8, 16): launches so far; [16, 20): CTAs started
 constexpr int kMaxPrefixGroups = 16;                  // prefix groups per launch (kernel parameters)
 constexpr int kPrefixRows = 64;                       // query rows of one prefix unit: 16 per warp
 
@@ -29,8 +30,14 @@ struct DecodeArgs {
     const int32_t *context_lens; // [S]
     float *o_part;               // fp32 [piece][G][D / pack], piece = s * Hkv + h + cta
     float *lse_part;             // fp32 [piece][G], log2 domain
-    unsigned long long *seg_count;  // [S * Hkv] (call epoch << 16 | pieces stored), per segment
-    unsigned long long epoch;    // this launch's epoch (< 2^48), unique in the process
+    unsigned long long *seg_count;  // [S * Hkv] (launch epoch << 16 | pieces stored), per segment
+    // Workspace header words: the launches of this workspace so far (the
+    // epoch that tags the counters) and the CTAs of the current launch that
+    // have read it. CTA 0 advances the epoch at its end, once all have, so
+    // each launch -- a CUDA graph's replays included -- has its own and the
+    // counters never need clearing.
+    unsigned long long *launch_epoch;
+    unsigned int *ctas_started;
     int32_t *status;             // device status word
     int num_seqs;
     int num_q_heads;
@@ -116,7 +123,7 @@ __host__ __device__ inline DecodeLayout decode_layout(int D, int BS, int GP, int
     off += kConsumerWarps * G * 4;
     off = align_up(off, 8);
     L.bars = off;
-    off += (2 * kMaxStages + 2) * 8;                                // full[stage], qfull[2], empty[stage]
+    off += (2 * kMaxStages + 3) * 8;                                // full[stage], qfull[2], empty[stage], epoch
     L.flags = off;
     off += (2 * kMaxStages + 1 + 2 * kConsumerWarps + 1 + 4 * 2) * 4;  // stage_bad, abort, scan, merges, stage_blk
     L.prefix = off;
