@@ -462,20 +462,41 @@ def run_e2e(step, args, flush, stream, kv, world):
     inputs (q, new k/v, tables, lengths, slots) from pinned memory and reads `out`
     back; the KV pool stays resident on the device (it is the cache).
 
-    As a serving loop would, the copies run on their own streams and overlap the
-    neighbouring steps' kernels: step i's inputs go to one of two device buffer
-    sets while step i - 1 computes, and its output is read back while step i + 1
-    computes. The timed region runs from the first input copy to the last
+    As a serving loop would, the inputs sit packed in one pinned buffer and go
+    over in one copy per step; the copies run on their own streams and overlap
+    the neighbouring steps' kernels: step i's inputs go to one of two device
+    buffer sets while step i - 1 computes, and its output is read back while
+    step i + 1 computes. The bf16 one-launch step is launched through
+    ``DecodeAppendCall`` (its buffers checked once, as a serving loop's static
+    buffers are). The timed region runs from the first input copy to the last
     read-back. No L2 flush: the pool (far larger than L2) is read once per step."""
     names = ("q", "k_new", "v_new", "bt", "cl", "slots")
-    host = {n: getattr(step, n).cpu().pin_memory() for n in names}
-    bufs = [{n: torch.empty_like(getattr(step, n)) for n in names} for _ in range(2)]
+    srcs = {n: getattr(step, n) for n in names}
+    offs, off = {}, 0
+    for n in names:  # each input at a 256-byte boundary of the packed buffers
+        offs[n] = off
+        off += (srcs[n].numel() * srcs[n].element_size() + 255) // 256 * 256
+    packed_host = torch.empty(off, dtype=torch.uint8, pin_memory=True)
+
+    def views(buf):
+        return {n: buf[offs[n]:offs[n] + srcs[n].numel() * srcs[n].element_size()].view(srcs[n].dtype)
+                .view(srcs[n].shape) for n in names}
+
+    for n, v in views(packed_host).items():
+        v.copy_(srcs[n].cpu())
+    packed_dev = [torch.empty(off, dtype=torch.uint8, device=step.q.device) for _ in range(2)]
+    bufs = [views(d) for d in packed_dev]
     outs = [torch.empty_like(step.out) for _ in range(2)]
     out_host = [torch.empty(step.out.shape, dtype=step.out.dtype, pin_memory=True) for _ in range(2)]
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    h2d = sum(t.numel() * t.element_size() for t in srcs.values())
     d2h = out_host[0].numel() * out_host[0].element_size()
     K = args.steps
     h2d_stream, d2h_stream = torch.cuda.Stream(), torch.cuda.Stream()
+    prepared = None
+    if step.fused and not step.fp8:
+        prepared = [step.pkv.DecodeAppendCall(outs[b], bufs[b]["q"], bufs[b]["k_new"], bufs[b]["v_new"],
+                                              bufs[b]["slots"], step.kc, step.vc, bufs[b]["bt"], bufs[b]["cl"],
+                                              step.b.scale, step.ws, stream=stream, **step.opts) for b in range(2)]
 
     def run(n_steps, timed):
         copied = [torch.cuda.Event() for _ in range(n_steps)]
@@ -488,16 +509,18 @@ def run_e2e(step, args, flush, stream, kv, world):
             with torch.cuda.stream(h2d_stream):
                 if i >= 2:
                     h2d_stream.wait_event(computed[i - 2])  # buffer set b is free again
-                for n in names:
-                    bufs[b][n].copy_(host[n], non_blocking=True)
+                packed_dev[b].copy_(packed_host, non_blocking=True)
                 copied[i].record(h2d_stream)
             stream.wait_event(copied[i])
             if i >= 2:
                 stream.wait_event(read[i - 2])  # out[b] has been read back
-            for n in names:
-                setattr(step, n, bufs[b][n])
-            step.out = outs[b]
-            step.run()
+            if prepared is not None:
+                prepared[b]()
+            else:
+                for n in names:
+                    setattr(step, n, bufs[b][n])
+                step.out = outs[b]
+                step.run()
             computed[i].record(stream)
             with torch.cuda.stream(d2h_stream):
                 d2h_stream.wait_event(computed[i])
@@ -513,7 +536,8 @@ def run_e2e(step, args, flush, stream, kv, world):
     (sum_kv,), (max_ms,) = aggregate([kv * K], [total_ms])
     return {"value": round(sum_kv / (max_ms / 1e3) / 1e9, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": round(max_ms / K, 5),
-            "how": "H2D / D2H on their own streams, overlapping the neighbouring steps; no L2 flush (pool > L2)"}
+            "how": "inputs packed in one pinned buffer, one H2D copy per step; H2D / D2H on their own streams, "
+                   "overlapping the neighbouring steps; no L2 flush (pool > L2)"}
 
 
 def config_block(args, batch, world):

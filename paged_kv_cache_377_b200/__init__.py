@@ -9,6 +9,7 @@ nvcc), every call raises: there is no CPU fallback.
 from __future__ import annotations
 
 from ._binding import (  # noqa: F401
+    DecodeAppendCall,
     PKV_MAX_PREFIX_GROUPS,
     PKV_STATUS_BAD_BLOCK_ID,
     PKV_STATUS_BAD_CONTEXT_LEN,
@@ -37,6 +38,7 @@ from .block_manager import BlockManager, OutOfBlocks, kv_block_copy  # noqa: F40
 
 __all__ = [
     "BlockManager",
+    "DecodeAppendCall",
     "OutOfBlocks",
     "PagedKVError",
     "PrefixGroups",

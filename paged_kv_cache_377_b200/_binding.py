@@ -250,18 +250,9 @@ def paged_attn_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
     return out
 
 
-def paged_attn_decode_append(out: torch.Tensor, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
-                             slot_mapping: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
-                             block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float,
-                             workspace: torch.Tensor, num_ctas: int = 0, num_stages: int = 0,
-                             ctas_per_sm: int = 0, math: int = 0, l2_prefetch: int = 0, piece_cost: int = 0,
-                             head_pack: int = 0, tile_tokens: int = 0, prefix_groups: Optional[PrefixGroups] = None,
-                             prefix_tiles: int = 0, stream=None) -> torch.Tensor:
-    """One decode step in one launch: append k_new / v_new (bf16 [S, Hkv, D]) at
-    slot_mapping (int64 [S], the slot of each sequence's last position, < 0 =
-    none), then the same attention as paged_attn_decode over contexts that
-    include the new token. Bit-identical to kv_cache_append + paged_attn_decode.
-    """
+def _decode_append_args(out, q, k_new, v_new, slot_mapping, k_cache, v_cache, block_tables, context_lens, scale,
+                        workspace, stream, options):
+    """Checks the fused step's tensors and returns (argument tuple, objects it points into)."""
     _need(q, "q", torch.bfloat16, 3)
     _need(out, "out", torch.bfloat16, 3)
     _need(k_new, "k_new", torch.bfloat16, 3)
@@ -280,13 +271,60 @@ def paged_attn_decode_append(out: torch.Tensor, q: torch.Tensor, k_new: torch.Te
         raise ValueError("k_new / v_new must be [num_seqs, num_kv_heads, head_dim] and slot_mapping [num_seqs]")
     if block_tables.shape[0] != S or context_lens.shape[0] != S:
         raise ValueError("block_tables and context_lens must have num_seqs rows")
-    opts = _options(num_ctas, num_stages, ctas_per_sm, math, l2_prefetch, piece_cost, head_pack, tile_tokens,
-                    prefix_groups, prefix_tiles)
-    _check("paged_attn_decode_append", library().paged_attn_decode_append(
-        _ptr(out), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(slot_mapping), _ptr(k_cache), _ptr(v_cache),
-        _ptr(block_tables), _ptr(context_lens), S, Hq, Hkv, D, bs, float(scale), block_tables.shape[1], NB,
-        _ptr(workspace), workspace.numel(), ctypes.byref(opts), _stream(stream)))
+    opts = _options(**options)
+    args = (_ptr(out), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(slot_mapping), _ptr(k_cache), _ptr(v_cache),
+            _ptr(block_tables), _ptr(context_lens), S, Hq, Hkv, D, bs, float(scale), block_tables.shape[1], NB,
+            _ptr(workspace), workspace.numel(), ctypes.byref(opts), _stream(stream))
+    return args, (opts, options.get("prefix_groups"))
+
+
+def paged_attn_decode_append(out: torch.Tensor, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                             slot_mapping: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                             block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float,
+                             workspace: torch.Tensor, num_ctas: int = 0, num_stages: int = 0,
+                             ctas_per_sm: int = 0, math: int = 0, l2_prefetch: int = 0, piece_cost: int = 0,
+                             head_pack: int = 0, tile_tokens: int = 0, prefix_groups: Optional[PrefixGroups] = None,
+                             prefix_tiles: int = 0, stream=None) -> torch.Tensor:
+    """One decode step in one launch: append k_new / v_new (bf16 [S, Hkv, D]) at
+    slot_mapping (int64 [S], the slot of each sequence's last position, < 0 =
+    none), then the same attention as paged_attn_decode over contexts that
+    include the new token. Bit-identical to kv_cache_append + paged_attn_decode.
+    """
+    args, _keep = _decode_append_args(out, q, k_new, v_new, slot_mapping, k_cache, v_cache, block_tables,
+                                      context_lens, scale, workspace, stream,
+                                      dict(num_ctas=num_ctas, num_stages=num_stages, ctas_per_sm=ctas_per_sm,
+                                           math=math, l2_prefetch=l2_prefetch, piece_cost=piece_cost,
+                                           head_pack=head_pack, tile_tokens=tile_tokens,
+                                           prefix_groups=prefix_groups, prefix_tiles=prefix_tiles))
+    _check("paged_attn_decode_append", library().paged_attn_decode_append(*args))
     return out
+
+
+class DecodeAppendCall:
+    """paged_attn_decode_append over fixed device buffers, checked and
+    marshalled once: ``call()`` then costs the C entry alone.
+
+    For a serving loop that keeps a step's inputs in static buffers and refills
+    them between steps (as a captured CUDA graph also needs). The buffers must
+    stay allocated with the same shapes while the object is used; the stream is
+    the one given (default: torch's current stream at construction). The
+    keyword options are those of paged_attn_decode_append.
+    """
+
+    def __init__(self, out, q, k_new, v_new, slot_mapping, k_cache, v_cache, block_tables, context_lens, scale,
+                 workspace, stream=None, **options):
+        self._args, self._keep = _decode_append_args(out, q, k_new, v_new, slot_mapping, k_cache, v_cache,
+                                                     block_tables, context_lens, scale, workspace, stream, options)
+        self._tensors = (out, q, k_new, v_new, slot_mapping, k_cache, v_cache, block_tables, context_lens,
+                         workspace)
+        self._fn = library().paged_attn_decode_append
+        self.out = out
+
+    def __call__(self) -> torch.Tensor:
+        rc = self._fn(*self._args)
+        if rc != PKV_OK:
+            _check("paged_attn_decode_append", rc)
+        return self.out
 
 
 def kv_cache_append(k: torch.Tensor, v: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,

@@ -283,3 +283,17 @@ def test_prefix_groups_need_bf16_pools_on_tensor_cores():
     rc = lib.paged_attn_decode_fp8(P, P, P, P, P, P, P, P, 4, 4, 2, 128, 16, 0.125, 3, 16, P, 1 << 20,
                                    ctypes.byref(opts), None)
     assert rc == -2 and "tensor cores" in lib.pkv_last_error().decode()
+
+
+def test_prepared_decode_call_checks_its_tensors_once_at_construction():
+    """DecodeAppendCall runs the fused step's argument checks when built (here:
+    host tensors are refused before anything is enqueued)."""
+    import torch
+    S, Hq, Hkv, D, NB, bs = 2, 4, 2, 64, 8, 16
+    bf = torch.bfloat16
+    args = (torch.empty(S, Hq, D, dtype=bf), torch.empty(S, Hq, D, dtype=bf), torch.empty(S, Hkv, D, dtype=bf),
+            torch.empty(S, Hkv, D, dtype=bf), torch.zeros(S, dtype=torch.int64), torch.empty(NB, bs, Hkv, D, dtype=bf),
+            torch.empty(NB, bs, Hkv, D, dtype=bf), torch.zeros(S, 4, dtype=torch.int32),
+            torch.ones(S, dtype=torch.int32), 0.125, torch.zeros(1 << 16, dtype=torch.uint8))
+    with pytest.raises(ValueError, match="CUDA device"):
+        pkv.DecodeAppendCall(*args)

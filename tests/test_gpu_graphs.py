@@ -127,3 +127,21 @@ def test_a_workspace_reused_by_many_calls_keeps_every_result():
         torch.cuda.synchronize()
         assert torch.equal(st.out.cpu().view(torch.int16), want.view(torch.int16)), f"call {i}"
     assert pkv.read_status(ws) == 0
+
+
+def test_a_prepared_call_matches_the_plain_call_bitwise():
+    """DecodeAppendCall launches the same step as paged_attn_decode_append; with
+    its buffers refilled between calls it gives each new step's result."""
+    b = workloads.make_batch("skewed_long", device="cuda").to("cpu")
+    st = Step(b)
+    call = pkv.DecodeAppendCall(st.out, st.q, st.kn, st.vn, st.slots, st.kc, st.vc, st.bt, st.cl, b.scale, st.ws)
+    gen = torch.Generator().manual_seed(3)
+    for _ in range(2):
+        q = torch.randn(b.q.shape, generator=gen).to(torch.bfloat16)
+        st.q.copy_(q)
+        st.out.fill_(float("nan"))
+        call()
+        torch.cuda.synchronize()
+        assert torch.equal(st.out.cpu().view(torch.int16), eager(b, q=q).view(torch.int16))
+    assert pkv.read_status(st.ws) == 0
+
