@@ -466,9 +466,9 @@ def run_e2e(step, args, flush, stream, kv, world):
     over in one copy per step; the copies run on their own streams and overlap
     the neighbouring steps' kernels: step i's inputs go to one of two device
     buffer sets while step i - 1 computes, and its output is read back while
-    step i + 1 computes. The bf16 one-launch step is launched through
-    ``DecodeAppendCall`` (its buffers checked once, as a serving loop's static
-    buffers are). The timed region runs from the first input copy to the last
+    step i + 1 computes. The one-launch step is launched through
+    ``DecodeAppendCall`` / ``DecodeAppendFp8Call`` (its buffers checked once, as
+    a serving loop's static buffers are). The timed region runs from the first input copy to the last
     read-back. No L2 flush: the pool (far larger than L2) is read once per step."""
     names = ("q", "k_new", "v_new", "bt", "cl", "slots")
     srcs = {n: getattr(step, n) for n in names}
@@ -493,7 +493,12 @@ def run_e2e(step, args, flush, stream, kv, world):
     K = args.steps
     h2d_stream, d2h_stream = torch.cuda.Stream(), torch.cuda.Stream()
     prepared = None
-    if step.fused and not step.fp8:
+    if step.fused and step.fp8:
+        prepared = [step.pkv.DecodeAppendFp8Call(outs[b], bufs[b]["q"], bufs[b]["k_new"], bufs[b]["v_new"],
+                                                 bufs[b]["slots"], step.kc, step.vc, step.ks, step.vs, bufs[b]["bt"],
+                                                 bufs[b]["cl"], step.b.scale, step.ws, stream=stream, **step.opts)
+                    for b in range(2)]
+    elif step.fused:
         prepared = [step.pkv.DecodeAppendCall(outs[b], bufs[b]["q"], bufs[b]["k_new"], bufs[b]["v_new"],
                                               bufs[b]["slots"], step.kc, step.vc, bufs[b]["bt"], bufs[b]["cl"],
                                               step.b.scale, step.ws, stream=stream, **step.opts) for b in range(2)]

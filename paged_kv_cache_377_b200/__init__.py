@@ -10,6 +10,7 @@ from __future__ import annotations
 
 from ._binding import (  # noqa: F401
     DecodeAppendCall,
+    DecodeAppendFp8Call,
     PKV_MAX_PREFIX_GROUPS,
     PKV_STATUS_BAD_BLOCK_ID,
     PKV_STATUS_BAD_CONTEXT_LEN,
@@ -39,6 +40,7 @@ from .block_manager import BlockManager, OutOfBlocks, kv_block_copy  # noqa: F40
 __all__ = [
     "BlockManager",
     "DecodeAppendCall",
+    "DecodeAppendFp8Call",
     "OutOfBlocks",
     "PagedKVError",
     "PrefixGroups",

@@ -446,12 +446,9 @@ def paged_attn_decode_fp8(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Ten
     return out
 
 
-def paged_attn_decode_append_fp8(out: torch.Tensor, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
-                                 slot_mapping: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
-                                 k_scale: torch.Tensor, v_scale: torch.Tensor, block_tables: torch.Tensor,
-                                 context_lens: torch.Tensor, scale: float, workspace: torch.Tensor, stream=None,
-                                 **options) -> torch.Tensor:
-    """The one-launch decode step over e4m3 pools (the new bf16 rows are quantized)."""
+def _decode_append_fp8_args(out, q, k_new, v_new, slot_mapping, k_cache, v_cache, k_scale, v_scale, block_tables,
+                            context_lens, scale, workspace, stream, options):
+    """Checks the e4m3 fused step's tensors and returns (argument tuple, objects it points into)."""
     _need(q, "q", torch.bfloat16, 3)
     _need(out, "out", torch.bfloat16, 3)
     _need(k_new, "k_new", torch.bfloat16, 3)
@@ -472,11 +469,46 @@ def paged_attn_decode_append_fp8(out: torch.Tensor, q: torch.Tensor, k_new: torc
         raise ValueError("block_tables and context_lens must have num_seqs rows")
     _need_scales(k_scale, v_scale, Hkv)
     opts = _options(**options)
-    _check("paged_attn_decode_append_fp8", library().paged_attn_decode_append_fp8(
-        _ptr(out), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(slot_mapping), _ptr(k_cache), _ptr(v_cache),
-        _ptr(k_scale), _ptr(v_scale), _ptr(block_tables), _ptr(context_lens), S, Hq, Hkv, D, bs, float(scale),
-        block_tables.shape[1], NB, _ptr(workspace), workspace.numel(), ctypes.byref(opts), _stream(stream)))
+    args = (_ptr(out), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(slot_mapping), _ptr(k_cache), _ptr(v_cache),
+            _ptr(k_scale), _ptr(v_scale), _ptr(block_tables), _ptr(context_lens), S, Hq, Hkv, D, bs, float(scale),
+            block_tables.shape[1], NB, _ptr(workspace), workspace.numel(), ctypes.byref(opts), _stream(stream))
+    return args, (opts, options.get("prefix_groups"))
+
+
+def paged_attn_decode_append_fp8(out: torch.Tensor, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                                 slot_mapping: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                                 k_scale: torch.Tensor, v_scale: torch.Tensor, block_tables: torch.Tensor,
+                                 context_lens: torch.Tensor, scale: float, workspace: torch.Tensor, stream=None,
+                                 **options) -> torch.Tensor:
+    """The one-launch decode step over e4m3 pools (the new bf16 rows are quantized)."""
+    args, _keep = _decode_append_fp8_args(out, q, k_new, v_new, slot_mapping, k_cache, v_cache, k_scale, v_scale,
+                                          block_tables, context_lens, scale, workspace, stream, options)
+    _check("paged_attn_decode_append_fp8", library().paged_attn_decode_append_fp8(*args))
     return out
+
+
+class DecodeAppendFp8Call:
+    """paged_attn_decode_append_fp8 over fixed device buffers, checked and
+    marshalled once (the e4m3 counterpart of DecodeAppendCall): ``call()``
+    then costs the C entry alone. The buffers, scales included, must stay
+    allocated with the same shapes while the object is used.
+    """
+
+    def __init__(self, out, q, k_new, v_new, slot_mapping, k_cache, v_cache, k_scale, v_scale, block_tables,
+                 context_lens, scale, workspace, stream=None, **options):
+        self._args, self._keep = _decode_append_fp8_args(out, q, k_new, v_new, slot_mapping, k_cache, v_cache,
+                                                         k_scale, v_scale, block_tables, context_lens, scale,
+                                                         workspace, stream, options)
+        self._tensors = (out, q, k_new, v_new, slot_mapping, k_cache, v_cache, k_scale, v_scale, block_tables,
+                         context_lens, workspace)
+        self._fn = library().paged_attn_decode_append_fp8
+        self.out = out
+
+    def __call__(self) -> torch.Tensor:
+        rc = self._fn(*self._args)
+        if rc != PKV_OK:
+            _check("paged_attn_decode_append_fp8", rc)
+        return self.out
 
 
 def kv_cache_append_fp8(k: torch.Tensor, v: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,

@@ -297,3 +297,17 @@ def test_prepared_decode_call_checks_its_tensors_once_at_construction():
             torch.ones(S, dtype=torch.int32), 0.125, torch.zeros(1 << 16, dtype=torch.uint8))
     with pytest.raises(ValueError, match="CUDA device"):
         pkv.DecodeAppendCall(*args)
+
+
+def test_prepared_fp8_call_checks_its_tensors_once_at_construction():
+    """DecodeAppendFp8Call runs the e4m3 fused step's argument checks when built
+    (host tensors are refused before anything is enqueued)."""
+    import torch
+    S, Hq, Hkv, D, NB, bs = 2, 4, 2, 128, 8, 16
+    bf, u8 = torch.bfloat16, torch.uint8
+    good = [torch.empty(S, Hq, D, dtype=bf), torch.empty(S, Hq, D, dtype=bf), torch.empty(S, Hkv, D, dtype=bf),
+            torch.empty(S, Hkv, D, dtype=bf), torch.zeros(S, dtype=torch.int64), torch.empty(NB, bs, Hkv, D, dtype=u8),
+            torch.empty(NB, bs, Hkv, D, dtype=u8), torch.ones(Hkv), torch.ones(Hkv), torch.zeros(S, 4, dtype=torch.int32),
+            torch.ones(S, dtype=torch.int32), 0.125, torch.zeros(1 << 16, dtype=u8)]
+    with pytest.raises(ValueError, match="CUDA device"):
+        pkv.DecodeAppendFp8Call(*good)

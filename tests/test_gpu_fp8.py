@@ -6,6 +6,7 @@ and round it to the nearest e4m3, ties to even, saturating), and the decode
 must match the oracle's attention over the exactly dequantized cache within
 the bf16 output tolerance |err| <= 8e-3 + 8e-3 |ref|.
 """
+import dataclasses
 import functools
 
 import numpy as np
@@ -180,3 +181,27 @@ def test_fp8_decode_reads_every_finite_code(Hq, Hkv, D, bs):
             assert np.array_equal(kc.numpy(), kc_ref) and np.array_equal(vc.numpy(), vc_ref)
             assert_close_to_oracle(out.double().numpy(), ref,
                                    what=f"fp8 every code Hq={Hq} Hkv={Hkv} D={D} bs={bs} {run.__name__} C={num_ctas}")
+
+
+def test_fp8_prepared_call_matches_the_plain_call_bitwise():
+    """DecodeAppendFp8Call launches the same e4m3 step as
+    paged_attn_decode_append_fp8; with q refilled between calls each call gives
+    that step's result (the appended row is the same each time)."""
+    b, _ = case("opt125m")
+    x = _dev(b)
+    ws = pkv.allocate_workspace(b.num_seqs, b.num_q_heads, b.head_dim)
+    out = torch.empty_like(x["q"])
+    call = pkv.DecodeAppendFp8Call(out, x["q"], x["kn"], x["vn"], x["slots"], x["kc"], x["vc"], x["ks"], x["vs"],
+                                   x["bt"], x["cl"], b.scale, ws)
+    gen = torch.Generator().manual_seed(11)
+    for i in range(2):
+        q = torch.randn(b.q.shape, generator=gen).to(torch.bfloat16)
+        x["q"].copy_(q)
+        out.fill_(float("nan"))
+        call()
+        torch.cuda.synchronize()
+        want, kc, vc, st = one_launch(dataclasses.replace(b, q=q))
+        assert st == 0
+        assert same_bits(out.cpu(), want), f"call {i}"
+        assert torch.equal(x["kc"].cpu(), kc) and torch.equal(x["vc"].cpu(), vc)
+    assert pkv.read_status(ws) == 0
