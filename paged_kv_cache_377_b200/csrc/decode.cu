@@ -1295,14 +1295,22 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
         if (!pc.whole) {
             // A segment cut between CTAs: count this CTA's piece in; the CTA that
             // stores the segment's last piece merges them all.
+            // Thread 0 reads the counter while the partials drain, the first
+            // guess of the CAS below (a stale guess costs one retry), and counts
+            // the segment's pieces meanwhile.
+            unsigned long long guess = 0;
+            int total = 0;
+            if (ctid == 0) {
+                guess = *reinterpret_cast<volatile unsigned long long *>(a.seg_count + seg);
+                total = segment_pieces(pc.s, pc.h, sm, a.num_kv_heads, W, gridDim.x - a.prefix_ctas, pcost, BS,
+                                       a.tiles_per_piece, nullptr);
+            }
             __threadfence();
             named_barrier_sync(1, kConsumerWarps * 32);
             if (ctid == 0) {
-                const int total = segment_pieces(pc.s, pc.h, sm, a.num_kv_heads, W, gridDim.x - a.prefix_ctas, pcost,
-                                                 BS, a.tiles_per_piece, nullptr);
                 unsigned long long *cnt = a.seg_count + seg;
                 const unsigned long long ep = *sm.epoch;
-                unsigned long long old = atomicAdd(cnt, 0ull), now;
+                unsigned long long old = guess, now;
                 for (;;) {  // count = 1 for the first piece of this launch (stale epochs restart)
                     now = (old >> 16) == ep ? old + 1 : (ep << 16) | 1ull;
                     const unsigned long long prev = atomicCAS(cnt, old, now);
@@ -1615,7 +1623,11 @@ __device__ __forceinline__ void prefix_unit(const CUtensorMap *tm_k, const CUten
     }
 
     // ---- count the piece in on each member's segment (its designated CTA
-    // merges the segment once every piece is in: merge_grouped_segments)
+    // merges the segment once every piece is in: merge_grouped_segments); the
+    // counters are read while the partials drain, the CAS's first guesses
+    unsigned long long guess = 0;
+    if (ctid < m1 - m0)
+        guess = *reinterpret_cast<volatile unsigned long long *>(a.seg_count + static_cast<size_t>(m0 + ctid) * Hkv + h);
     __threadfence();
     named_barrier_sync(1, kConsumerWarps * 32);
     if (ctid < m1 - m0) {
@@ -1623,7 +1635,7 @@ __device__ __forceinline__ void prefix_unit(const CUtensorMap *tm_k, const CUten
         if (min(sm.lens[s], T * BS) > t0 * BS) {
             unsigned long long *cnt = a.seg_count + static_cast<size_t>(s) * Hkv + h;
             const unsigned long long ep = *sm.epoch;
-            unsigned long long old = atomicAdd(cnt, 0ull), now;
+            unsigned long long old = guess, now;
             for (;;) {  // count = 1 for the first piece of this launch (stale epochs restart)
                 now = (old >> 16) == ep ? old + 1 : (ep << 16) | 1ull;
                 const unsigned long long prev = atomicCAS(cnt, old, now);
