@@ -66,9 +66,12 @@ extern "C" {
 /*
  * Tuning knobs of paged_attn_decode_ex. Zero in any field means "default".
  *   num_ctas          CTAs of the persistent decode grid (1..1024); default:
- *                     every CTA that fits on the device at once. The KV blocks
- *                     of a launch are split evenly over the CTAs, so this also
- *                     sets how finely long contexts are split.
+ *                     every CTA that fits on the device at once, or fewer for
+ *                     a batch whose weight -- bounded by num_seqs x kv heads x
+ *                     (max_blocks_per_seq tiles + piece cost), the lengths
+ *                     being on the device -- gives a CTA under 16 tiles. The
+ *                     KV blocks of a launch are split evenly over the CTAs, so
+ *                     this also sets how finely long contexts are split.
  *   num_stages        shared-memory stages (one KV tile each) per warp (1..4; a
  *                     CTA has 4 warps); default: 1 on tensor cores, about 64 KB
  *                     of KV blocks per CTA on CUDA cores.
@@ -206,9 +209,10 @@ int pkv_decode_workspace_bytes(int num_seqs, int num_q_heads, int head_dim, size
  * Per call (and per 2048 sequences): one persistent decode kernel whose CTAs
  * each take an equal share of the batch's KV blocks (weighted per context
  * piece); a context split between CTAs is merged (log-sum-exp) by the CTA that
- * stores its last piece. For a given device and options, results are bitwise
- * reproducible and depend only on the logical order of tokens, not on where
- * their blocks sit in the pool.
+ * stores its last piece. For a given device, options and batch shape (the
+ * default grid depends on num_seqs and max_blocks_per_seq), results are
+ * bitwise reproducible and depend only on the logical order of tokens, not on
+ * where their blocks sit in the pool.
  */
 int paged_attn_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
                       const int32_t *block_tables, const int32_t *context_lens,

@@ -149,6 +149,9 @@ constexpr int kDefaultL2Prefetch = 0;  // measured on the Llama-shaped batch: an
 constexpr int kDefaultPieceCost = 8;
 constexpr int kDefaultPieceCostWideGroup = 16;
 constexpr int kDefaultPieceCostFp8 = 12;
+// Least weight (tiles, piece cost included) per CTA of a default grid: the 4
+// warps of a CTA hold 4 to 8 tiles in flight.
+constexpr int kMinCtaWeight = 16;
 
 // Work of one shared-prefix tile (64 query rows) against one suffix tile (the G
 // rows of one sequence), for splitting the CTAs between the two: the prefix
@@ -404,6 +407,18 @@ int decode_impl(void *out, const void *q, const void *k_new, const void *v_new, 
         if (o.ctas_per_sm > 0 && o.ctas_per_sm < per_sm) per_sm = o.ctas_per_sm;
         int grid = o.num_ctas > 0 ? o.num_ctas : sms * per_sm;
         if (grid > pkv::kMaxCtas) grid = pkv::kMaxCtas;
+        const int pcost_default = fp8 ? kDefaultPieceCostFp8 : group > 4 ? kDefaultPieceCostWideGroup : kDefaultPieceCost;
+        const int pcost = o.piece_cost > 0 ? o.piece_cost : o.piece_cost == 0 ? pcost_default : 0;
+        // A batch too small to give every CTA kMinCtaWeight tiles of weight runs
+        // on fewer CTAs (the weight is bounded from above by the table width:
+        // the lengths stay on the device). A CTA's warps take several tiles at
+        // once, so smaller pieces finish no sooner, and every cut costs a merge.
+        if (o.num_ctas <= 0 && !may_group) {
+            const long long wmax = static_cast<long long>(khkv) * sc *
+                                   (static_cast<long long>(max_blocks_per_seq) * (block_size / tile) + pcost);
+            const long long want = (wmax + kMinCtaWeight - 1) / kMinCtaWeight;
+            if (want < grid) grid = want < 1 ? 1 : static_cast<int>(want);
+        }
         // the kernel with prefix units is launched cooperatively (its CTAs wait
         // for one another's pieces): no more CTAs than fit at once
         if (may_group && grid > resident) grid = resident;
@@ -428,8 +443,7 @@ int decode_impl(void *out, const void *q, const void *k_new, const void *v_new, 
         a.num_blocks = num_blocks;
         a.num_stages = ns;
         a.prefetch = o.l2_prefetch > 0 ? o.l2_prefetch : o.l2_prefetch == 0 ? kDefaultL2Prefetch : 0;
-        const int pcost_default = fp8 ? kDefaultPieceCostFp8 : group > 4 ? kDefaultPieceCostWideGroup : kDefaultPieceCost;
-        a.piece_cost = o.piece_cost > 0 ? o.piece_cost : o.piece_cost == 0 ? pcost_default : 0;
+        a.piece_cost = pcost;
         a.scale_log2 = scale * 1.4426950408889634f;
         plan_prefix_groups(may_group ? pg : nullptr, s0, sc, khkv, kgroup, a.sub, grid, max_blocks_per_seq,
                            o.prefix_tiles, a);

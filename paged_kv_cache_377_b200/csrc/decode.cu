@@ -975,47 +975,69 @@ __device__ __forceinline__ int piece_bases(const DecodeArgs &a, int s, int h, co
 }
 
 // Merge of the pieces of segment (s, h) whose partials sit at rows
-// base(i) * G + g, i < npieces (log-sum-exp identity, in that order: the
-// prefix pieces, then the suffix pieces in CTA order): out = sum_c 2^(lse_c - M)
-// o_c / sum_c 2^(lse_c - M), taken in one pass with a running maximum. A
-// thread merges 4-dim elements of the G x D output (at most two) with the
-// loads of kAhead pieces of both in flight, so that the merge costs a few L2
-// round trips rather than one per piece. Partials written by other SMs are
-// read past L1.
+// base(i) * G + g, i < npieces (log-sum-exp identity): out = sum_c 2^(lse_c - M)
+// o_c / sum_c 2^(lse_c - M), with a running maximum. The pieces are dealt to J
+// interleaved subsets (i = j, j + J, j + 2J, ...): J, a power of two up to 32,
+// spreads a long merge over the threads that a small output leaves idle. Thread
+// ctid merges subset ctid mod J of the 4-dim elements ctid / J + k * (threads /
+// J), k < kE, with the loads of kAhead pieces of each in flight; the J threads
+// of an element (consecutive lanes) then combine in a butterfly and the
+// element's subset-0 thread stores it, so the result depends on npieces and G
+// only. Partials written by other SMs are read past L1.
 // Elements a thread merges: the G x D / 4 float4 columns over the CTA's threads (G <= 8).
 template <int D>
 constexpr int merge_elems() { return (8 * (D / 4) + kConsumerWarps * 32 - 1) / (kConsumerWarps * 32); }
+
+// a (running state) absorbs b: both log2-sum-exp states of the same element
+__device__ __forceinline__ void lse_absorb(float &Ma, float &da, float4 &aa, float Mb, float db, const float4 &ab) {
+    if (!(Mb > -INFINITY)) return;  // b holds no piece
+    const float Mn = fmaxf(Ma, Mb);
+    const float r = fast_exp2(Ma - Mn), w = fast_exp2(Mb - Mn);
+    da = da * r + db * w;
+    aa.x = aa.x * r + ab.x * w;
+    aa.y = aa.y * r + ab.y * w;
+    aa.z = aa.z * r + ab.z * w;
+    aa.w = aa.w * r + ab.w * w;
+    Ma = Mn;
+}
 
 template <int D, int kAhead = (8 / merge_elems<D>() > 0 ? 8 / merge_elems<D>() : 1), class Base>
 __device__ __forceinline__ void merge_pieces(const DecodeArgs &a, const Base &base, int npieces, int s, int h,
                                              int ctid) {
     constexpr int kE = merge_elems<D>();
+    constexpr int kThreads = kConsumerWarps * 32;
     const int G = a.group;
     const int DR = D / a.pack;
+    const int E = G * (D / 4);  // float4 elements of the segment's output rows
+    int J = 1;
+    while (2 * J * E <= kE * kThreads && 2 * J <= npieces && 2 * J <= 32) J *= 2;
+    const int j = ctid & (J - 1);  // this thread's subset of the pieces
+    const int per = kThreads / J;  // threads per subset
     int eg[kE], ecol[kE];
     float M[kE], den[kE];
     float4 acc[kE];
 #pragma unroll
     for (int k = 0; k < kE; ++k) {
-        const int e = ctid + k * kConsumerWarps * 32;
+        const int e = ctid / J + k * per;
         eg[k] = e / (D / 4);
         ecol[k] = (e % (D / 4)) * 4 - (a.pack == 2 ? eg[k] / (G >> 1) : 0) * DR;
-        if (e >= G * (D / 4) || ecol[k] < 0 || ecol[k] >= DR) ecol[k] = -1;  // none, or the other half of a packed head
+        if (e >= E || ecol[k] < 0 || ecol[k] >= DR) ecol[k] = -1;  // none, or the other half of a packed head
         M[k] = -INFINITY;
         den[k] = 0.f;
         acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     // every element's loads of kAhead pieces are in flight together
-    for (int ib = 0; ib < npieces; ib += kAhead) {
+    for (int ib = j; ib < npieces; ib += kAhead * J) {
         float lse[kAhead][kE];
         float4 o[kAhead][kE];
 #pragma unroll
         for (int i = 0; i < kAhead; ++i) {
-            const size_t pb = ib + i < npieces ? static_cast<size_t>(base(ib + i)) : 0;
+            const int pi = ib + i * J;
+            const size_t pb = pi < npieces ? static_cast<size_t>(base(pi)) : 0;
 #pragma unroll
             for (int k = 0; k < kE; ++k) {
                 lse[i][k] = -INFINITY;
-                if (ib + i < npieces && ecol[k] >= 0) {
+                if (pi < npieces && ecol[k] >= 0) {
                     const size_t pr = pb * G + eg[k];
                     lse[i][k] = __ldcg(a.lse_part + pr);
                     o[i][k] = __ldcg(reinterpret_cast<const float4 *>(a.o_part + pr * DR + ecol[k]));
@@ -1025,18 +1047,22 @@ __device__ __forceinline__ void merge_pieces(const DecodeArgs &a, const Base &ba
 #pragma unroll
         for (int i = 0; i < kAhead; ++i)
 #pragma unroll
-            for (int k = 0; k < kE; ++k) {
-                if (!(lse[i][k] > -INFINITY)) continue;  // no piece here
-                const float Mn = fmaxf(M[k], lse[i][k]);
-                const float r = fast_exp2(M[k] - Mn), w = fast_exp2(lse[i][k] - Mn);
-                den[k] = den[k] * r + w;
-                acc[k].x = acc[k].x * r + w * o[i][k].x;
-                acc[k].y = acc[k].y * r + w * o[i][k].y;
-                acc[k].z = acc[k].z * r + w * o[i][k].z;
-                acc[k].w = acc[k].w * r + w * o[i][k].w;
-                M[k] = Mn;
-            }
+            for (int k = 0; k < kE; ++k) lse_absorb(M[k], den[k], acc[k], lse[i][k], 1.f, o[i][k]);
     }
+    // the J subsets of each element: a butterfly over the J consecutive lanes
+    for (int off = 1; off < J; off <<= 1) {
+#pragma unroll
+        for (int k = 0; k < kE; ++k) {
+            const float Mb = __shfl_xor_sync(0xffffffffu, M[k], off), db = __shfl_xor_sync(0xffffffffu, den[k], off);
+            float4 ab;
+            ab.x = __shfl_xor_sync(0xffffffffu, acc[k].x, off);
+            ab.y = __shfl_xor_sync(0xffffffffu, acc[k].y, off);
+            ab.z = __shfl_xor_sync(0xffffffffu, acc[k].z, off);
+            ab.w = __shfl_xor_sync(0xffffffffu, acc[k].w, off);
+            lse_absorb(M[k], den[k], acc[k], Mb, db, ab);
+        }
+    }
+    if (j != 0) return;
 #pragma unroll
     for (int k = 0; k < kE; ++k) {
         if (ecol[k] < 0) continue;
