@@ -974,6 +974,23 @@ __device__ __forceinline__ int piece_bases(const DecodeArgs &a, int s, int h, co
     return n;
 }
 
+// Counts a piece in on its segment's counter (launch epoch << 16 | pieces
+// counted) and returns the counter after it. A counter an older launch left
+// restarts at 1 through a CAS; once it carries this launch's epoch it keeps it
+// for the rest of the launch, so later pieces take a plain add -- no retries
+// when the many pieces of a long context arrive together. guess: a recent read
+// of the counter.
+__device__ __forceinline__ unsigned long long count_piece_in(unsigned long long *cnt, unsigned long long ep,
+                                                              unsigned long long guess) {
+    unsigned long long old = guess;
+    for (;;) {
+        if ((old >> 16) == ep) return atomicAdd(cnt, 1ull) + 1ull;
+        const unsigned long long prev = atomicCAS(cnt, old, (ep << 16) | 1ull);
+        if (prev == old) return (ep << 16) | 1ull;
+        old = prev;
+    }
+}
+
 // Merge of the pieces of segment (s, h) whose partials sit at rows
 // base(i) * G + g, i < npieces (log-sum-exp identity): out = sum_c 2^(lse_c - M)
 // o_c / sum_c 2^(lse_c - M), with a running maximum. The pieces are dealt to J
@@ -1321,9 +1338,9 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
         if (!pc.whole) {
             // A segment cut between CTAs: count this CTA's piece in; the CTA that
             // stores the segment's last piece merges them all.
-            // Thread 0 reads the counter while the partials drain, the first
-            // guess of the CAS below (a stale guess costs one retry), and counts
-            // the segment's pieces meanwhile.
+            // Thread 0 reads the counter while the partials drain (the count-in's
+            // first guess; a stale one costs a retry) and counts the segment's
+            // pieces meanwhile.
             unsigned long long guess = 0;
             int total = 0;
             if (ctid == 0) {
@@ -1336,13 +1353,7 @@ __device__ __forceinline__ void decode_warp(const CUtensorMap *tm_k, const CUten
             if (ctid == 0) {
                 unsigned long long *cnt = a.seg_count + seg;
                 const unsigned long long ep = *sm.epoch;
-                unsigned long long old = guess, now;
-                for (;;) {  // count = 1 for the first piece of this launch (stale epochs restart)
-                    now = (old >> 16) == ep ? old + 1 : (ep << 16) | 1ull;
-                    const unsigned long long prev = atomicCAS(cnt, old, now);
-                    if (prev == old) break;
-                    old = prev;
-                }
+                const unsigned long long now = count_piece_in(cnt, ep, guess);
                 const int pending = sm.merge_flag[0];
                 // (a shared-prefix segment is merged by its designated CTA,
                 // merge_grouped_segments, whoever completes it)
@@ -1661,13 +1672,7 @@ __device__ __forceinline__ void prefix_unit(const CUtensorMap *tm_k, const CUten
         if (min(sm.lens[s], T * BS) > t0 * BS) {
             unsigned long long *cnt = a.seg_count + static_cast<size_t>(s) * Hkv + h;
             const unsigned long long ep = *sm.epoch;
-            unsigned long long old = guess, now;
-            for (;;) {  // count = 1 for the first piece of this launch (stale epochs restart)
-                now = (old >> 16) == ep ? old + 1 : (ep << 16) | 1ull;
-                const unsigned long long prev = atomicCAS(cnt, old, now);
-                if (prev == old) break;
-                old = prev;
-            }
+            count_piece_in(cnt, ep, guess);
         }
     }
 }
