@@ -146,9 +146,13 @@ constexpr int kDefaultL2Prefetch = 0;  // measured on the Llama-shaped batch: an
 // batch, 4 per kv head: 354.9 -> 357.5). e4m3 pools: 12 (after the bit-placement
 // conversion: Llama-shaped 265.5 -> 260.6 us, OPT-shaped 40.6 -> 38.3, skewed
 // 119.0 -> 119.8).
+// Head-packed bf16 pools (head_dim 64 in pairs): 12 (after the plain-add
+// count-in, OPT-shaped 41.0 -> 39.0 us at 12, 40.3 at 16; 12 instead of 8 cost
+// the Llama-shaped batch 2 us and the skewed one 1 us).
 constexpr int kDefaultPieceCost = 8;
 constexpr int kDefaultPieceCostWideGroup = 16;
 constexpr int kDefaultPieceCostFp8 = 12;
+constexpr int kDefaultPieceCostPacked = 12;
 // Least weight (tiles, piece cost included) per CTA of a default grid: the 4
 // warps of a CTA hold 4 to 8 tiles in flight.
 constexpr int kMinCtaWeight = 16;
@@ -407,7 +411,10 @@ int decode_impl(void *out, const void *q, const void *k_new, const void *v_new, 
         if (o.ctas_per_sm > 0 && o.ctas_per_sm < per_sm) per_sm = o.ctas_per_sm;
         int grid = o.num_ctas > 0 ? o.num_ctas : sms * per_sm;
         if (grid > pkv::kMaxCtas) grid = pkv::kMaxCtas;
-        const int pcost_default = fp8 ? kDefaultPieceCostFp8 : group > 4 ? kDefaultPieceCostWideGroup : kDefaultPieceCost;
+        const int pcost_default = fp8 ? kDefaultPieceCostFp8
+                                  : group > 4 ? kDefaultPieceCostWideGroup
+                                  : pack == 2 ? kDefaultPieceCostPacked
+                                              : kDefaultPieceCost;
         const int pcost = o.piece_cost > 0 ? o.piece_cost : o.piece_cost == 0 ? pcost_default : 0;
         // A batch too small to give every CTA kMinCtaWeight tiles of weight runs
         // on fewer CTAs (the weight is bounded from above by the table width:
