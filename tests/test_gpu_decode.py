@@ -273,3 +273,21 @@ def test_bounded_wait_gives_up_and_reports():
     out, _, _, st = run_step(b)
     assert st == 0
     assert_close_to_oracle(out.double().numpy(), ref, what="after the timeout self-test")
+
+
+@pytest.mark.parametrize("L", [4096, 32768])
+def test_single_long_context_at_default_options(L):
+    """One sequence (Llama heads) at the default launch: a 4,096-token context
+    runs on the smaller grid a batch this size gets (one CTA per 16 tiles of
+    its weight), a 32,768-token one on the full grid, cut into ~74 pieces per
+    kv head that count themselves in together and are merged over spread
+    merge slots. Both against the oracle, with the pools bit-exact."""
+    b = workloads.make_custom(4100 + L // 1024, [L], 32, 8, 128, 16, device="cuda").to("cpu")
+    ref, kc_ref, vc_ref = oracle.decode_step(b)
+    out, kc, vc, st = run_step(b)
+    assert st == 0, f"status {st}"
+    assert np.array_equal(bf16_bits(kc), kc_ref) and np.array_equal(bf16_bits(vc), vc_ref)
+    assert_close_to_oracle(out.double().numpy(), ref, what=f"one context of {L} tokens")
+    # a second launch on a fresh workspace: bitwise the same
+    out2, _, _, st2 = run_step(b)
+    assert st2 == 0 and torch.equal(out.view(torch.int16), out2.view(torch.int16))
