@@ -87,8 +87,9 @@ extern "C" {
  *                     kv head) segment adds when the batch is split between CTAs,
  *                     standing for a piece's fixed cost (1..64); -1 = none;
  *                     default 8, 16 where a kv head serves more than 4 query
- *                     heads, 12 on e4m3 pools and with head packing. Keeps
- *                     CTAs that get many short contexts from finishing last.
+ *                     heads (24 on e4m3 pools), 12 on e4m3 pools and with head
+ *                     packing. Keeps CTAs that get many short contexts from
+ *                     finishing last.
  *   head_pack         0 = default (2 where possible), 1 = off, 2 = read kv heads
  *                     2h and 2h + 1 together as one head of twice the head_dim
  *                     (the pool's [bs][Hkv][D] rows are the same bytes as
