@@ -69,7 +69,7 @@ extern "C" {
  *                     every CTA that fits on the device at once, or fewer for
  *                     a batch whose weight -- bounded by num_seqs x kv heads x
  *                     (max_blocks_per_seq tiles + piece cost), the lengths
- *                     being on the device -- gives a CTA under 16 tiles. The
+ *                     being on the device -- gives a CTA under 8 tiles. The
  *                     KV blocks of a launch are split evenly over the CTAs, so
  *                     this also sets how finely long contexts are split.
  *   num_stages        shared-memory stages (one KV tile each) per warp (1..4; a

@@ -156,9 +156,12 @@ constexpr int kDefaultPieceCostPacked = 12;
 // e4m3 pools with more than 4 query heads per kv head: 24 (Qwen-shaped, 7 per
 // kv head: 47.2 us at 12, 46.5 at 16, 45.1 at 24).
 constexpr int kDefaultPieceCostFp8WideGroup = 24;
-// Least weight (tiles, piece cost included) per CTA of a default grid: the 4
-// warps of a CTA hold 4 to 8 tiles in flight.
-constexpr int kMinCtaWeight = 16;
+// Least weight (tiles, piece cost included) per CTA of a default grid. With
+// many pieces of one context counted in by a plain add, 8 beat 16 on every
+// small batch (same box: tiny 16.4 -> 12.3 us, one 2,048-token context 24.6
+// -> 22.5, 4 x 512 24.6 -> 20.5, 8 x 1,024 Qwen-shaped 26.6 -> 24.6); 4 and 2
+// were slower on the Qwen- and OPT-shaped ones.
+constexpr int kMinCtaWeight = 8;
 
 // Work of one shared-prefix tile (64 query rows) against one suffix tile (the G
 // rows of one sequence), for splitting the CTAs between the two: the prefix
