@@ -29,6 +29,7 @@ from ._binding import (  # noqa: F401
     paged_attn_decode_append,
     paged_attn_decode_append_fp8,
     paged_attn_decode_fp8,
+    paged_attn_decode_noalloc,
     paged_attn_prefill,
     read_status,
     selftest_bounded_wait,
@@ -54,6 +55,7 @@ __all__ = [
     "paged_attn_decode_append",
     "paged_attn_decode_append_fp8",
     "paged_attn_decode_fp8",
+    "paged_attn_decode_noalloc",
     "paged_attn_prefill",
     "kv_cache_append_fp8",
     "read_status",
